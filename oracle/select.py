@@ -1,0 +1,70 @@
+"""Exactly-read index set I of one unit: sink + local window + top blocks.
+
+Follows vAttention, Method, overall framework: the deterministic set I_f is
+the attention sink (first tokens), the local window (latest tokens) and the
+top-scoring tokens of an approximate top-k.  The top-k here ranks 16-token
+blocks by their mean key (the block-level selection of Quest / ArkVale that
+the RESA page wraps), one index set per KV head because the group's query
+heads share the K/V reads.
+
+Readings where the pages are silent:
+  * candidate blocks are those that do not overlap the sink or the window;
+  * score_c = sum_{h in group} q_h . kbar_c (the 1/sqrt(d) factor is positive
+    and common, so it does not change the ranking and is left out);
+  * ties go to the lower block index: rank by (score desc, index asc);
+  * the decision is taken in fp64.
+
+Parity pins (tests/test_oracle_select.py): brute force over all subsets on
+tiny inputs, sorting with Python's own sort, all-equal scores, planted blocks
+whose rank is known.
+"""
+import numpy as np
+
+BLOCK = 16
+
+
+def candidate_blocks(L, sink, local):
+    """Blocks c with [16c, 16c+16) disjoint from [0, sink) and [L-local, L)."""
+    lo = -(-sink // BLOCK)
+    hi = max(L - local, 0) // BLOCK
+    return np.arange(lo, max(hi, lo), dtype=np.int64)
+
+
+def block_scores(q, blk_mean, cand):
+    """q [G, d], blk_mean [nb, d] -> score of each candidate block (fp64)."""
+    per_head = q @ blk_mean[cand].T            # [G, n_cand]
+    return per_head.sum(axis=0)
+
+
+def top_blocks(scores, cand, k):
+    """The k best candidates by (score desc, block index asc), returned in
+    ascending block order."""
+    k = min(int(k), len(cand))
+    order = np.lexsort((cand, -scores))        # last key is the primary key
+    return np.sort(cand[order[:k]])
+
+
+def index_set(L, sink, local, blocks):
+    """Sorted token positions read exactly: [0,sink) u [L-local,L) u blocks."""
+    mask = np.zeros(L, dtype=bool)
+    mask[: min(sink, L)] = True
+    mask[max(L - local, 0):] = True
+    for c in blocks:
+        mask[BLOCK * c: BLOCK * c + BLOCK] = True
+    return np.flatnonzero(mask)
+
+
+def tail_set(L, idx):
+    """Sorted positions not read exactly (the residual / tail T)."""
+    mask = np.ones(L, dtype=bool)
+    mask[idx] = False
+    return np.flatnonzero(mask)
+
+
+def select_unit(q, blk_mean, L, sink, local, k_blocks):
+    """Full selection of one unit: (chosen blocks ascending, I, T)."""
+    cand = candidate_blocks(L, sink, local)
+    sc = block_scores(q, blk_mean, cand)
+    blocks = top_blocks(sc, cand, k_blocks)
+    idx = index_set(L, sink, local, blocks)
+    return blocks, idx, tail_set(L, idx)

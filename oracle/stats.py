@@ -1,0 +1,62 @@
+"""Prefill-end statistics of one unit (sequence b, KV head g).
+
+Follows RESA, Method, key design 1 ("Prior Estimator"):
+  * the typical query mu_Q and typical key mu_K are means of the historical
+    queries / keys; here mu_Q[h] is the mean over the L context queries of
+    query head h, and mu_K the mean of the L cached keys of the KV head;
+  * the prior logit row mu_Q K^T / sqrt(d) does not depend on the decode
+    query, so it is computed once at prefill end: its softmax-weighted sum of
+    V is O_Est and its exponential sum is the normaliser (stored as
+    log_z0 = ln sum_j exp(s * mu_Q . K_j), without the query-dependent bias);
+    this is the "one extra query appended at prefill end, L -> L+1".
+
+Also the totals the count-aware proxy needs (OpenAttention, stage 04: tail
+sums are totals minus the selected part), and the 16-token block means the
+block selector ranks (Quest/ArkVale-style page summaries named on the RESA
+page's related work), rounded once to the cache dtype.
+
+Parity pins (tests/test_oracle_stats.py): closed forms for constant keys /
+queries (log_z0 = ln L + s mu_Q.kappa, O_Est = mean V), O_Est against torch's
+scaled_dot_product_attention with query mu_Q, block means against torch's
+bf16 cast where the mean is an fp32 value.
+"""
+import numpy as np
+
+from .numerics import round_to
+
+BLOCK = 16
+
+
+def block_means(k, kv_dtype):
+    """k [L, d] float64 -> [L/16, d]: mean of each 16-token block, computed in
+    fp64 and rounded once to the cache dtype (nearest, ties to even)."""
+    L, d = k.shape
+    assert L % BLOCK == 0
+    return round_to(k.reshape(L // BLOCK, BLOCK, d).mean(axis=1), kv_dtype)
+
+
+def prefill_stats(q_ctx, k, v, scale, kv_dtype):
+    """q_ctx [G, L, d], k [L, d], v [L, d] (float64 holding the cache values).
+
+    Returns a dict with
+      mu_q [G, d], o_est [G, d], log_z0 [G],            (per query head)
+      mu_k [d], sum_k [d], sum_v [d],                    (per KV head)
+      blk_mean [L/16, d] (cache dtype values), kbar_absmax (max |blk_mean|).
+    """
+    G, L, d = q_ctx.shape
+    mu_q = q_ctx.mean(axis=1)
+    sum_k = k.sum(axis=0)
+    sum_v = v.sum(axis=0)
+    mu_k = sum_k / L
+    p0 = scale * (mu_q @ k.T)                  # prior logits of the typical query [G, L]
+    m = p0.max(axis=1, keepdims=True)
+    w = np.exp(p0 - m)
+    a = w.sum(axis=1)
+    log_z0 = np.log(a) + m[:, 0]
+    o_est = (w @ v) / a[:, None]
+    bm = block_means(k, kv_dtype)
+    return {
+        "mu_q": mu_q, "o_est": o_est, "log_z0": log_z0,
+        "mu_k": mu_k, "sum_k": sum_k, "sum_v": sum_v,
+        "blk_mean": bm, "kbar_absmax": float(np.abs(bm).max()),
+    }

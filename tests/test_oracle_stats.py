@@ -1,0 +1,61 @@
+"""Pins for oracle.stats: closed forms and an independent attention routine."""
+import math
+
+import numpy as np
+import torch
+
+from oracle.numerics import round_to_bf16
+from oracle.stats import block_means, prefill_stats
+
+
+def _sdpa(q, k, v, scale):
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a))[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(
+        t(q), t(k), t(v), scale=scale)[0, 0].numpy()
+
+
+def test_constant_keys_closed_form():
+    rng = np.random.default_rng(0)
+    G, L, d = 3, 96, 8
+    kappa = round_to_bf16(rng.standard_normal(d))
+    k = np.tile(kappa, (L, 1))
+    v = rng.standard_normal((L, d))
+    mu = rng.standard_normal((G, d))
+    noise = rng.standard_normal((G, L // 2, d))
+    q_ctx = mu[:, None, :] + np.concatenate([noise, -noise], axis=1)  # mean exactly mu
+    s = 1 / math.sqrt(d)
+    st = prefill_stats(q_ctx, k, v, s, "bf16")
+    np.testing.assert_allclose(st["mu_q"], mu, rtol=0, atol=1e-13)
+    np.testing.assert_array_equal(st["mu_k"], kappa)
+    np.testing.assert_allclose(st["sum_k"], L * kappa, rtol=1e-15)
+    np.testing.assert_allclose(st["log_z0"], math.log(L) + s * (mu @ kappa), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(st["o_est"], np.tile(v.mean(0), (G, 1)), atol=1e-13)
+    np.testing.assert_array_equal(st["blk_mean"], np.tile(kappa, (L // 16, 1)))
+    assert st["kbar_absmax"] == np.abs(kappa).max()
+
+
+def test_o_est_is_attention_of_the_typical_query():
+    rng = np.random.default_rng(1)
+    G, L, d = 4, 256, 16
+    q_ctx = rng.standard_normal((G, L, d)) + rng.standard_normal((G, 1, d))
+    k = rng.standard_normal((L, d)) * 2
+    v = rng.standard_normal((L, d))
+    s = 0.3
+    st = prefill_stats(q_ctx, k, v, s, "f32")
+    mu = q_ctx.mean(axis=1)
+    np.testing.assert_allclose(st["o_est"], _sdpa(mu, k, v, s), rtol=1e-12, atol=1e-12)
+    lse = torch.logsumexp(torch.from_numpy(s * mu @ k.T), dim=1).numpy()
+    np.testing.assert_allclose(st["log_z0"], lse, rtol=1e-14)
+
+
+def test_block_means_against_torch_cast():
+    # blocks of 16 small integers times 2^-6: the fp64 mean is exactly an
+    # fp32 value, so torch's fp32 -> bf16 cast is an independent reference
+    rng = np.random.default_rng(2)
+    L, d = 16 * 50, 32
+    k = rng.integers(-3000, 3000, size=(L, d)).astype(np.float64) * 2.0 ** -6
+    means32 = (k.reshape(-1, 16, d).sum(1) / 16).astype(np.float32)
+    assert np.array_equal(means32.astype(np.float64), k.reshape(-1, 16, d).mean(1))
+    want = torch.from_numpy(means32).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(block_means(k, "bf16"), want)
+    np.testing.assert_array_equal(block_means(k, "f32"), means32.astype(np.float64))
