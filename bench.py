@@ -1,0 +1,446 @@
+#!/usr/bin/env python
+"""Decode-attention benchmark: sparse decode with residual tail estimation over
+a 32K bf16 GQA KV cache at a 1% read, against the in-build dense flash-decode.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
+
+One step = one decode step of the whole batch through the hot path: block
+scoring + exact top-k (sa_select, one kernel) then gather + online softmax +
+residual fold + split combine (sa_decode, one kernel).  Inputs (KV cache,
+prefill statistics, queries) are resident in HBM before timing; L2 is flushed
+(256 MB write) before every timed step and the flush is outside the timed
+events.  Prints ONE JSON line on rank 0.
+
+--impl reference times the fp64 CPU oracle (the reference arm of this build)
+on a bounded sample of the same workload, on the host cores.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn tokens/sec & HBM GB/s (% of roofline) at 32K, 1% read, vs dense"
+UNIT = "tokens/s"
+FLUSH_BYTES = 256 << 20
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="batched")
+    ap.add_argument("--read", type=float, default=0.01, help="read budget (fraction of L)")
+    ap.add_argument("--mode", default="resa", choices=["drop", "resa", "proxy", "sample"])
+    ap.add_argument("--sample-b", type=int, default=64)
+    ap.add_argument("--queries", type=int, default=64, help="distinct decode queries cycled through")
+    ap.add_argument("--dense-steps", type=int, default=50)
+    ap.add_argument("--mode-steps", type=int, default=200)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--small", action="store_true", help="profiling case: B=4 (same kernels, smaller batch)")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# bytes the method must move (algorithmic), per unit = (sequence, KV head)
+
+def select_bytes_per_unit(w, sg, esz, b_draws):
+    """Block summaries of every candidate + the group's queries + outputs."""
+    return sg["n_cand"] * w.d * esz + w.G * w.d * esz + 4 * sg["kk"] + 4 * b_draws + 4
+
+
+def decode_bytes_per_unit(w, sg, esz, mode, b_draws):
+    rows = sg["n_i"] + (b_draws if mode == "sample" else 0)
+    byts = rows * 2 * w.d * esz + w.G * w.d * esz + 4 * sg["kk"] + w.G * w.d * 4
+    if mode == "sample":
+        byts += 4 * b_draws
+    if mode == "resa":
+        byts += w.G * (2 * w.d + 1) * 4 + w.d * 4       # mu_q, o_est, log_z0 per head; mu_k
+    if mode == "proxy":
+        byts += 2 * w.d * 4                              # sum_k, sum_v
+    return byts
+
+
+def set_geom(L, sink, local, k_blocks):
+    s_eff = min(sink, L)
+    w_eff = min(min(local, L), L - s_eff)
+    c_lo = -(-sink // 16)
+    c_hi = max((L - local) // 16 if L - local > 0 else 0, c_lo)
+    n_cand = c_hi - c_lo
+    kk = min(k_blocks, n_cand)
+    n_i = s_eff + w_eff + 16 * kk
+    return {"n_cand": n_cand, "kk": kk, "n_i": n_i, "n_t": L - n_i}
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (nvidia-smi, read-only)
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY, "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 9:
+                rows.append(f)
+        os.unlink(self.path)
+        return summarize_clocks(rows)
+
+
+def summarize_clocks(rows):
+    if not rows:
+        return None
+    sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+    mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+            "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; only timings cross ranks)
+
+def dist_setup(n_gpus):
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return ws, rank, local
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def reduce_max(x, device=None):
+    """Max of a float over ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle arm
+
+def cpu_oracle_sample(w, sp_kw, mode, seconds, max_units=None, seq=0):
+    """Times the fp64 oracle (select + decode of one unit = one KV head of one
+    sequence) on the host, over units of one sequence, until `seconds` pass.
+    Returns (units_per_s, units, threads)."""
+    import numpy as np
+    import torch
+    from threadpoolctl import threadpool_info
+
+    import synth
+    from oracle import modes, rng, select, stats
+
+    s = synth.make_sequence(w, seq, device="cpu")
+    qs = synth.make_queries(w, seq, 4, s["mu_q"], device="cpu")
+    scale = 1.0 / math.sqrt(w.d)
+    units = []
+    for g in range(w.Hkv):
+        K = s["k"][g].double().numpy()
+        V = s["v"][g].double().numpy()
+        st = stats.prefill_stats(s["q_ctx"][g * w.G:(g + 1) * w.G].double().numpy(), K, V, scale, w.dtype)
+        units.append((g, K, V, st))
+    done = 0
+    t0 = time.perf_counter()
+    while True:
+        for g, K, V, st in units:
+            step = done % qs.shape[0]
+            q = qs[step, g * w.G:(g + 1) * w.G].double().numpy()
+            blocks, idx, tail = select.select_unit(q, st["blk_mean"], w.L, sp_kw["sink"], sp_kw["local"],
+                                                   sp_kw["k_blocks"])
+            pos = rng.sample_positions(sp_kw["seed"], seq, g, step, tail, sp_kw["sample_b"]) if mode == "sample" else None
+            modes.run_mode(mode, q, K, V, idx, st, scale, pos=pos)
+            done += 1
+            if max_units is not None and done >= max_units:
+                break
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_units is not None and done >= max_units):
+            break
+    threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+    return done / el, done, threads
+
+
+def run_reference(args, w, sg, sp_kw, rank):
+    if rank != 0:
+        return 0
+    per_step = max(1, w.Hkv)              # one step = one sequence's decode step (all KV heads)
+    total = (args.warmup + args.steps) * per_step
+    # bounded: the whole run stays within a few minutes
+    rate, units, threads = cpu_oracle_sample(w, sp_kw, args.mode, seconds=min(120.0, 1e9), max_units=total)
+    value = rate / w.Hkv
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, sg, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": "%d units (KV head x decode step) of sequence 0, mode %s, fp64 numpy" % (units, args.mode)},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def workload_config(w, sg, args):
+    return {"workload": "%s decode: B%d, %dq/%dkv heads, d%d, L%d, %s, %g%% read (sink %d + window %d + %d blocks of 16 = %d tokens)"
+            % (w.name, w.B, w.Hq, w.Hkv, w.d, w.L, w.dtype, 100 * args.read, w.sink, w.local, sg["kk"], sg["n_i"]),
+            "global_batch": w.B * args.gpus, "seq_len": w.L, "mode": args.mode, "k_blocks": sg["kk"],
+            "read_tokens": sg["n_i"], "l2": "flushed before every timed step (256 MB write, untimed)",
+            "parallelism": "replicas (dp%d, no collective on the data path)" % args.gpus}
+
+
+# ---------------------------------------------------------------------------
+
+def main(argv=None):
+    args = parse_args(argv)
+    import synth
+    w = synth.WORKLOADS[args.workload]
+    if args.small:
+        w = synth.scaled(w, B=4)
+    kb = w.k_blocks_for(args.read) if w.k_blocks is None else w.k_blocks
+    sg = set_geom(w.L, w.sink, w.local, kb)
+    sp_kw = dict(sink=w.sink, local=w.local, k_blocks=kb, sample_b=args.sample_b, seed=2024)
+    ws, rank, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        rc = run_reference(args, w, sg, sp_kw, rank)
+        barrier()
+        return rc
+
+    import numpy as np
+    import torch
+
+    import kv_cache_residual_b200 as sa
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    esz = 2 if w.dtype == "bf16" else 4
+    nq = max(1, min(args.queries, args.steps + args.warmup))
+    # weak scaling: every rank holds its own batch (sequence seeds offset by rank)
+    wr = synth.scaled(w, seed=w.seed + 100_000 * rank)
+    data = synth.make_batch(wr, device=dev, steps=nq)
+    stats = sa.prefill_stats(data["q_ctx"], data["k"], data["v"])
+    del data["q_ctx"]
+    torch.cuda.empty_cache()
+    K, V, Q = data["k"], data["v"], data["q"]
+    bdraw = args.sample_b if args.mode == "sample" else 0
+    sps = [sa.SelectParams(sink=w.sink, local=w.local, k_blocks=kb, sample_b=bdraw, sample_cap=max(bdraw, 1),
+                           seed=2024, step=t) for t in range(nq)]
+    sel = sa.select(Q[0], stats, sps[0])
+    out = torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(t, mode):
+        sp = sps[t % nq]
+        sa.select(Q[t % nq], stats, sp, selection=sel)
+        sa.decode(Q[t % nq], K, V, stats, sel, sp, mode=mode, out=out)
+
+    def timed(n, fn, n_events=3):
+        """Runs fn(t, ev) n times with an L2 flush before each; returns per-step
+        lists of event-pair durations (ms)."""
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_events)] for _ in range(n)]
+        for t in range(n):
+            flush.zero_()
+            fn(t, evs[t])
+        torch.cuda.synchronize()
+        return [[evs[t][i].elapsed_time(evs[t][i + 1]) for i in range(n_events - 1)] for t in range(n)]
+
+    def sparse_step(mode):
+        def fn(t, ev):
+            sp = sps[t % nq]
+            ev[0].record(stream)
+            sa.select(Q[t % nq], stats, sp, selection=sel)
+            ev[1].record(stream)
+            sa.decode(Q[t % nq], K, V, stats, sel, sp, mode=mode, out=out)
+            ev[2].record(stream)
+        return fn
+
+    # warm-up (untimed)
+    for t in range(args.warmup):
+        flush.zero_()
+        step(t, args.mode)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    per = timed(args.steps, sparse_step(args.mode))
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    sel_ms = [p[0] for p in per]
+    dec_ms = [p[1] for p in per]
+    total_ms = sum(a + b for a, b in per)
+    total_ms = reduce_max(total_ms, dev)
+    ms_per_step = total_ms / args.steps
+    value = ws * w.B * args.steps / (total_ms / 1e3)
+
+    sel_b = select_bytes_per_unit(w, sg, esz, bdraw) * w.B * w.Hkv
+    dec_b = decode_bytes_per_unit(w, sg, esz, args.mode, bdraw) * w.B * w.Hkv
+    peaks = {}
+    pk_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pk_path):
+        peaks = json.load(open(pk_path))
+    peak = peaks.get("hbm_gbs")
+    peak_src = "measured (MEASURED_PEAKS.json hbm_gbs)" if peak else "fallback 6650 GB/s"
+    peak = peak or 6650.0
+    sel_avg = statistics.mean(sel_ms)
+    dec_avg = statistics.mean(dec_ms)
+    sel_gbs = sel_b / (sel_avg * 1e-3) / 1e9
+    dec_gbs = dec_b / (dec_avg * 1e-3) / 1e9
+    step_gbs = (sel_b + dec_b) / (ms_per_step * 1e-3) / 1e9
+
+    # other modes (same selection kernel)
+    mode_vals = {}
+    for m in ("drop", "resa", "proxy", "sample"):
+        if m == "sample" and bdraw == 0:
+            sps_m = [sa.SelectParams(sink=w.sink, local=w.local, k_blocks=kb, sample_b=args.sample_b,
+                                     sample_cap=args.sample_b, seed=2024, step=t) for t in range(nq)]
+            sel_m = sa.select(Q[0], stats, sps_m[0])
+
+            def fn(t, ev, sps_m=sps_m, sel_m=sel_m):
+                sp = sps_m[t % nq]
+                ev[0].record(stream)
+                sa.select(Q[t % nq], stats, sp, selection=sel_m)
+                ev[1].record(stream)
+                sa.decode(Q[t % nq], K, V, stats, sel_m, sp, mode="sample", out=out)
+                ev[2].record(stream)
+        else:
+            fn = sparse_step(m)
+        timed(3, fn)
+        pm = timed(args.mode_steps, fn)
+        ms = sum(a + b for a, b in pm) / len(pm)
+        mode_vals[m] = {"tokens_per_s": w.B / (ms * 1e-3), "ms_per_step": ms,
+                        "decode_us": 1e3 * statistics.mean(p[1] for p in pm)}
+
+    # dense flash-decode reference (in-build)
+    def dense_fn(t, ev):
+        ev[0].record(stream)
+        sa.dense_decode(Q[t % nq], K, V, out=out)
+        ev[1].record(stream)
+    timed(3, dense_fn, 2)
+    pd = timed(args.dense_steps, dense_fn, 2)
+    dense_ms = statistics.mean(p[0] for p in pd)
+    dense_bytes = 2 * w.B * w.Hkv * w.L * w.d * esz + w.B * w.Hq * w.d * (esz + 4)
+    dense = {"tokens_per_s": w.B / (dense_ms * 1e-3), "ms_per_step": dense_ms,
+             "hbm_gbs": dense_bytes / (dense_ms * 1e-3) / 1e9,
+             "frac": dense_bytes / (dense_ms * 1e-3) / 1e9 / peak}
+
+    # end to end through the public API: pinned host q in, host output back
+    e2e = None
+    if not args.no_e2e:
+        q_host = Q.cpu().pin_memory()
+        q_dev = torch.empty_like(Q[0])
+        o_host = torch.empty(w.B, w.Hq, w.d, dtype=torch.float32).pin_memory()
+
+        def e2e_fn(t, ev):
+            sp = sps[t % nq]
+            ev[0].record(stream)
+            q_dev.copy_(q_host[t % nq], non_blocking=True)
+            sa.select(q_dev, stats, sp, selection=sel)
+            sa.decode(q_dev, K, V, stats, sel, sp, mode=args.mode, out=out)
+            o_host.copy_(out, non_blocking=True)
+            ev[1].record(stream)
+        timed(3, e2e_fn, 2)
+        pe = timed(min(args.steps, 500), e2e_fn, 2)
+        e2e_ms = reduce_max(sum(p[0] for p in pe), dev) / len(pe)
+        e2e = {"value": ws * w.B / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": int(Q[0].numel() * Q.element_size()),
+               "d2h_bytes_per_step": int(out.numel() * 4)}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu:
+        rate, units, threads = cpu_oracle_sample(w, sp_kw, args.mode, args.cpu_seconds)
+        cpu = {"value": rate / w.Hkv, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": "%d units (one KV head of sequence 0 at one decode step each), %.0f s, mode %s, fp64 numpy"
+                         % (units, args.cpu_seconds, args.mode)}
+
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tp):
+        tr = json.load(open(tp))
+        key = "%s:%s:%s" % (args.workload, args.read, "k_select")
+        if key in tr:
+            traffic = tr[key]
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded generator, Llama-3.1-8B layer shapes)",
+            "config": workload_config(w, sg, args),
+            "roofline": {"bound": "hbm", "kernel": "k_select (block scoring + top-k)", "achieved": sel_gbs,
+                         "peak": peak, "unit": "GB/s", "frac": sel_gbs / peak, "traffic": traffic,
+                         "bytes_per_launch": sel_b, "us_per_launch": 1e3 * sel_avg, "peak_source": peak_src},
+            "step_roofline": {"achieved": step_gbs, "frac": step_gbs / peak, "bytes_per_step": sel_b + dec_b,
+                              "decode_gbs": dec_gbs, "decode_us": 1e3 * dec_avg, "decode_bytes": dec_b},
+            "dense": dense, "speedup_vs_dense": dense_ms / ms_per_step, "modes": mode_vals,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps, "clocks": clk,
+        }
+        print(json.dumps(line))
+    barrier()
+    try:
+        import torch.distributed as dist
+        if dist.is_initialized():
+            dist.destroy_process_group()
+    except Exception:
+        pass
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

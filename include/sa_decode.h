@@ -1,0 +1,208 @@
+/*
+ * sa_decode.h -- C ABI of libsa_b200.so: sparse single-token decode attention
+ * over a long GQA KV cache, with the unread tail added back by a residual
+ * estimator.  Built for NVIDIA B200 (sm_100a).
+ *
+ * One decode step of one unit u = (sequence b, KV head g) reads exactly
+ *   I = attention sink [0, sink) + local window [L-local, L) + the k_blocks
+ *       best 16-token blocks, ranked by sum_{h in group} q_h . kbar_c
+ *       (kbar_c = mean key of block c),
+ * and estimates the rest T (|T| = n_T) with one of
+ *   SA_DROP    no estimate (plain sparse attention);
+ *   SA_RESA    the RESA rank-1 prior: O_Est and the normaliser Z computed once
+ *              at prefill end, bias (q - mu_Q) . mu_K / sqrt(d), merged in
+ *              O(|I|) by removing the prior terms at I and adding the exact ones
+ *              ("RESA: Bringing Back What Sparse Attention Ignores with Residual
+ *              Estimation", Method, key designs 1 and 2);
+ *   SA_PROXY   one virtual token: key = tail-mean K, value = tail-mean V,
+ *              logit + ln n_T, tail sums = prefill totals minus the selected
+ *              rows ("OpenAttention: One Percent Is Enough with Tail Proxies",
+ *              abstract and method stage 04);
+ *   SA_SAMPLE  b tail positions drawn uniformly with replacement, weighted
+ *              n_T / b ("vAttention: Verified Sparse Attention via Sampling",
+ *              Method, key design 1, paper eq. 3), b fixed or from the CLT
+ *              budget of key designs 2-3.
+ * With n_T = 0 every mode is exact dense attention.
+ *
+ * Conventions for every entry point
+ *   - Pointers are DEVICE pointers to caller-owned memory (PyTorch tensors),
+ *     16-byte aligned, dense row-major in the layouts stated below.  The
+ *     library never allocates or frees device memory; scratch comes in `ws`.
+ *   - `stream` is a cudaStream_t passed as void*; NULL = the legacy default
+ *     stream.  Every call only enqueues work: no host synchronisation.
+ *   - Argument errors return SA_ERR_INVALID_ARG / SA_ERR_UNSUPPORTED /
+ *     SA_ERR_WORKSPACE before anything is launched; a failed launch returns
+ *     SA_ERR_CUDA.  Nothing aborts or traps.
+ *   - Workspace: size it with sa_workspace_size(); it must be ZERO-FILLED
+ *     once when first allocated.  Each call leaves its completion counters at
+ *     zero again, so the same buffer can be reused by later calls on the same
+ *     stream.  Calls that share a workspace must not overlap on the GPU.
+ *   - Outputs are fp32.  Results are deterministic: no floating-point
+ *     atomics; partial results are combined in a fixed order.
+ *
+ * Layouts (dtype = shape.dtype for the cache and all queries)
+ *   k, v        [B, Hkv, L, d]       KV cache
+ *   q_ctx       [B, Hq, L, d]        context queries (prefill only)
+ *   q           [B, Hq, d]           decode queries of this step
+ *   query head h belongs to KV head h / (Hq / Hkv).
+ */
+#ifndef SA_DECODE_H
+#define SA_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SA_API __attribute__((visibility("default")))
+#else
+#define SA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SA_OK = 0,
+    SA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer   */
+    SA_ERR_UNSUPPORTED = 2,  /* a valid request this build does not handle   */
+    SA_ERR_WORKSPACE = 3,    /* ws NULL or smaller than sa_workspace_size()  */
+    SA_ERR_CUDA = 4          /* a kernel launch failed                      */
+} sa_status;
+
+typedef enum { SA_F32 = 0, SA_BF16 = 1 } sa_dtype;
+
+typedef enum { SA_DROP = 0, SA_RESA = 1, SA_PROXY = 2, SA_SAMPLE = 3 } sa_mode;
+
+typedef enum {
+    SA_OP_PREFILL = 0,   /* sa_prefill_stats */
+    SA_OP_SELECT = 1,    /* sa_select        */
+    SA_OP_DECODE = 2,    /* sa_decode        */
+    SA_OP_DENSE = 3      /* sa_dense_decode  */
+} sa_op;
+
+/* Supported: d in {64, 128}; Hq % Hkv == 0 with G = Hq/Hkv in {1,2,4,8};
+ * L a positive multiple of 16, L < 2^31 / d; B, Hkv >= 1. */
+typedef struct {
+    int B, Hq, Hkv, d, L;
+    sa_dtype dtype;
+} sa_shape;
+
+/* Prefill-end statistics, written by sa_prefill_stats, read by sa_select and
+ * sa_decode.  All caller-allocated (RESA page, key design 1: "computed once at
+ * prefill end").
+ *   mu_q        [B, Hq, d]   f32  typical query: mean of the L context queries
+ *   o_est       [B, Hq, d]   f32  sum_j softmax_j(s mu_q . K_j) V_j
+ *   log_z0      [B, Hq]      f32  ln sum_j exp(s mu_q . K_j)  (no bias)
+ *   mu_k        [B, Hkv, d]  f32  typical key: mean of the L cached keys
+ *   sum_k       [B, Hkv, d]  f32  sum of the L cached keys
+ *   sum_v       [B, Hkv, d]  f32  sum of the L cached values
+ *   blk_mean    [B, Hkv, L/16, d] in dtype: 16-token block means, summed in
+ *               fp64 and rounded once (nearest, ties to even)
+ *   kbar_absmax [B, Hkv]     f32  max |blk_mean| (bounds the fp32 scoring
+ *               error in sa_select)                                          */
+typedef struct {
+    float* mu_q;
+    float* o_est;
+    float* log_z0;
+    float* mu_k;
+    float* sum_k;
+    float* sum_v;
+    void* blk_mean;
+    float* kbar_absmax;
+} sa_stats;
+
+/* Which tokens one step reads exactly, and how the tail is sampled.
+ *   sink, local   >= 0: first / last tokens always read (vAttention page,
+ *                 overall framework: sink + local window + top-k)
+ *   k_blocks      >= 0: blocks chosen per unit among those disjoint from the
+ *                 sink and the window (fewer if fewer candidates exist)
+ *   sample_b      draws per unit for SA_SAMPLE when clt_base == 0
+ *   clt_base      > 0: choose b per unit by the CLT budget (vAttention, key
+ *                 designs 2-3) from the first clt_base draws, target (eps,
+ *                 delta) on the output, b clamped to [clt_base, min(n_T,
+ *                 sample_cap)]; 0: fixed sample_b
+ *   sample_cap    capacity per unit of sa_selection.samp_idx (>= sample_b)
+ *   seed, step    SplitMix64 stream of unit (b, g) at this step:
+ *                 key = out(out(out(out(seed)^b)^g)^step), draw i =
+ *                 out(key + i*0x9E3779B97F4A7C15), out(x) = SplitMix64 mixer
+ *                 of x + 0x9E3779B97F4A7C15; rank = ((draw>>32)*n_T)>>32     */
+typedef struct {
+    int sink, local, k_blocks;
+    int sample_b, clt_base, sample_cap;
+    float eps, delta;
+    uint64_t seed;
+    int step;
+} sa_select_params;
+
+/* Output of sa_select, input of sa_decode (caller-allocated).
+ *   blk_idx     [B, Hkv, k_blocks] int32: chosen block indices, ascending;
+ *               min(k_blocks, n_cand) valid entries per unit, rest = -1
+ *   samp_idx    [B, Hkv, sample_cap] int32: drawn token positions (draw order)
+ *   samp_count  [B, Hkv] int32: draws per unit (0 unless sampling)
+ *   n_rescored  [B, Hkv] int32 or NULL: candidates whose fp32 score fell
+ *               within the rounding bound of the k-th and were rescored in
+ *               fp64 (diagnostic)                                            */
+typedef struct {
+    int32_t* blk_idx;
+    int32_t* samp_idx;
+    int32_t* samp_count;
+    int32_t* n_rescored;
+} sa_selection;
+
+/* mode; lambda = prior weight of SA_RESA in [0,1] (1 = the RESA page's
+ * merge, 0 = plain sparse attention); scale = softmax scale (0 = 1/sqrt(d)). */
+typedef struct {
+    sa_mode mode;
+    float lambda;
+    float scale;
+} sa_decode_params;
+
+/* Bytes of zero-initialised scratch the op needs for this shape (params may
+ * be NULL for SA_OP_PREFILL and SA_OP_DENSE).  0 on invalid arguments. */
+SA_API size_t sa_workspace_size(const sa_shape* shape, const sa_select_params* params, int op);
+
+/* Prefill-end statistics (RESA page, key design 1: mu_Q, mu_K, O_Est and Z
+ * as one extra query at prefill end; OpenAttention stage 04: totals for the
+ * tail means; block means for the selector).  Reads q_ctx once and k, v once.
+ * scale = softmax scale (0 = 1/sqrt(d)). */
+SA_API sa_status sa_prefill_stats(const sa_shape* shape, const void* q_ctx, const void* k,
+                           const void* v, const sa_stats* out, float scale,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* Block means of blocks [blk_begin, blk_end) of every unit into blk_mean
+ * ([B, Hkv, L/16, d], dtype) and raises kbar_absmax [B, Hkv] to cover them
+ * (for a cache that grew by whole blocks).  No workspace. */
+SA_API sa_status sa_block_summaries(const sa_shape* shape, const void* k, int blk_begin, int blk_end,
+                             void* blk_mean, float* kbar_absmax, void* stream);
+
+/* Selection of one decode step for every unit: block scores, exact top-k by
+ * (score desc, block index asc) decided in fp64 (fp32 scan with a rounding
+ * bound; candidates inside the bound are rescored in fp64), and the tail draws
+ * for sampling.  k and v are read only for the CLT base sample (may be NULL
+ * when clt_base == 0). */
+SA_API sa_status sa_select(const sa_shape* shape, const sa_select_params* params, const void* q,
+                    const sa_stats* stats, const void* k, const void* v,
+                    const sa_selection* out, float scale, void* ws, size_t ws_bytes,
+                    void* stream);
+
+/* Sparse decode: gathers I (and the draws), one fp32 online softmax over the
+ * G query heads of each unit, folds in the mode's residual, writes
+ * out [B, Hq, d] f32. */
+SA_API sa_status sa_decode(const sa_shape* shape, const sa_decode_params* dparams,
+                    const sa_select_params* sparams, const void* q, const void* k,
+                    const void* v, const sa_stats* stats, const sa_selection* sel,
+                    float* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Dense flash-decode over all L tokens (the in-build speed reference, not
+ * part of the method): out [B, Hq, d] f32 = softmax(s q K^T) V. */
+SA_API sa_status sa_dense_decode(const sa_shape* shape, const void* q, const void* k, const void* v,
+                          float* out, float scale, void* ws, size_t ws_bytes, void* stream);
+
+/* Static string for a status code. */
+SA_API const char* sa_status_string(sa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SA_DECODE_H */

@@ -1,0 +1,251 @@
+"""Python binding of libsa_b200.so: sparse single-token decode attention over
+a GQA KV cache with residual tail estimation, on NVIDIA B200 (sm_100a).
+
+Argument marshalling only: every step runs in the library's CUDA kernels.
+PyTorch provides device memory and the current stream.  There is no CPU
+fallback: if the shared library is missing, importing the ops raises.
+
+Layouts: k, v [B, Hkv, L, d]; q_ctx [B, Hq, L, d]; q [B, Hq, d]; bf16 or fp32
+(one dtype for all); outputs fp32 [B, Hq, d].
+
+    stats = prefill_stats(q_ctx, k, v)
+    sp = SelectParams(sink=64, local=128, k_blocks=8, sample_b=64, sample_cap=64, seed=1, step=t)
+    sel = select(q, stats, sp)
+    o = decode(q, k, v, stats, sel, sp, mode="resa")
+"""
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsa_b200.so")
+
+SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_CUDA = range(5)
+SA_F32, SA_BF16 = 0, 1
+MODES = {"drop": 0, "resa": 1, "proxy": 2, "sample": 3}
+OP_PREFILL, OP_SELECT, OP_DECODE, OP_DENSE = range(4)
+
+
+class SAError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (what, _lib().sa_status_string(status).decode(), status))
+
+
+class sa_shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("d", ctypes.c_int),
+                ("L", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+class sa_stats(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("mu_q", "o_est", "log_z0", "mu_k", "sum_k", "sum_v", "blk_mean", "kbar_absmax")]
+
+
+class sa_select_params(ctypes.Structure):
+    _fields_ = [("sink", ctypes.c_int), ("local", ctypes.c_int), ("k_blocks", ctypes.c_int),
+                ("sample_b", ctypes.c_int), ("clt_base", ctypes.c_int), ("sample_cap", ctypes.c_int),
+                ("eps", ctypes.c_float), ("delta", ctypes.c_float), ("seed", ctypes.c_uint64),
+                ("step", ctypes.c_int)]
+
+
+class sa_selection(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("blk_idx", "samp_idx", "samp_count", "n_rescored")]
+
+
+class sa_decode_params(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int), ("lam", ctypes.c_float), ("scale", ctypes.c_float)]
+
+
+EXPORTS = ("sa_workspace_size", "sa_prefill_stats", "sa_block_summaries", "sa_select", "sa_decode",
+           "sa_dense_decode", "sa_status_string")
+
+_LIB = None
+
+
+def _lib():
+    """Load the shared library (raises if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libsa_b200.so not built: run `python -m kv_cache_residual_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        sh, sp = ctypes.POINTER(sa_shape), ctypes.POINTER(sa_select_params)
+        st, sel, dp = ctypes.POINTER(sa_stats), ctypes.POINTER(sa_selection), ctypes.POINTER(sa_decode_params)
+        lib.sa_workspace_size.argtypes = [sh, sp, I]
+        lib.sa_workspace_size.restype = S
+        lib.sa_prefill_stats.argtypes = [sh, P, P, P, st, F, P, S, P]
+        lib.sa_block_summaries.argtypes = [sh, P, I, I, P, P, P]
+        lib.sa_select.argtypes = [sh, sp, P, st, P, P, sel, F, P, S, P]
+        lib.sa_decode.argtypes = [sh, dp, sp, P, P, P, st, sel, P, P, S, P]
+        lib.sa_dense_decode.argtypes = [sh, P, P, P, P, F, P, S, P]
+        lib.sa_status_string.argtypes = [I]
+        lib.sa_status_string.restype = ctypes.c_char_p
+        for f in ("sa_prefill_stats", "sa_block_summaries", "sa_select", "sa_decode", "sa_dense_decode"):
+            getattr(lib, f).restype = I
+        _LIB = lib
+    return _LIB
+
+
+def _check(status, what):
+    if status != SA_OK:
+        raise SAError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return SA_BF16
+    if t.dtype == torch.float32:
+        return SA_F32
+    raise TypeError("cache dtype must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def make_shape(k, Hq):
+    B, Hkv, L, d = k.shape
+    return sa_shape(B, Hq, Hkv, d, L, _dtype_code(k))
+
+
+@dataclass
+class SelectParams:
+    sink: int = 64
+    local: int = 128
+    k_blocks: int = 8
+    sample_b: int = 0
+    sample_cap: int = 0
+    clt_base: int = 0
+    eps: float = 0.05
+    delta: float = 0.05
+    seed: int = 0
+    step: int = 0
+
+    def c(self):
+        return sa_select_params(self.sink, self.local, self.k_blocks, self.sample_b, self.clt_base,
+                                max(self.sample_cap, self.sample_b), self.eps, self.delta,
+                                self.seed & ((1 << 64) - 1), self.step)
+
+
+class Stats:
+    """Prefill-end statistics (caller-owned device tensors)."""
+
+    FIELDS = ("mu_q", "o_est", "log_z0", "mu_k", "sum_k", "sum_v", "blk_mean", "kbar_absmax")
+
+    def __init__(self, B, Hq, Hkv, L, d, dtype, device):
+        f = dict(dtype=torch.float32, device=device)
+        self.mu_q = torch.empty(B, Hq, d, **f)
+        self.o_est = torch.empty(B, Hq, d, **f)
+        self.log_z0 = torch.empty(B, Hq, **f)
+        self.mu_k = torch.empty(B, Hkv, d, **f)
+        self.sum_k = torch.empty(B, Hkv, d, **f)
+        self.sum_v = torch.empty(B, Hkv, d, **f)
+        self.blk_mean = torch.empty(B, Hkv, L // 16, d, dtype=dtype, device=device)
+        self.kbar_absmax = torch.zeros(B, Hkv, **f)
+
+    def c(self):
+        return sa_stats(*[self.__dict__[n].data_ptr() for n in self.FIELDS])
+
+
+class Selection:
+    """Output of select(): chosen blocks and tail draws per unit."""
+
+    def __init__(self, B, Hkv, k_blocks, sample_cap, device):
+        i = dict(dtype=torch.int32, device=device)
+        self.blk_idx = torch.empty(B, Hkv, max(k_blocks, 1), **i)
+        self.samp_idx = torch.empty(B, Hkv, max(sample_cap, 1), **i)
+        self.samp_count = torch.zeros(B, Hkv, **i)
+        self.n_rescored = torch.zeros(B, Hkv, **i)
+
+    def c(self):
+        return sa_selection(self.blk_idx.data_ptr(), self.samp_idx.data_ptr(), self.samp_count.data_ptr(),
+                            self.n_rescored.data_ptr())
+
+
+_WS = {}
+
+
+def workspace(shape, params, op, device):
+    """Zero-filled scratch for one op, cached per (device, op, shape, params)."""
+    lib = _lib()
+    n = lib.sa_workspace_size(ctypes.byref(shape), ctypes.byref(params) if params is not None else None, op)
+    if n == 0:
+        raise SAError(SA_ERR_INVALID_ARG, "sa_workspace_size")
+    key = (str(device), op, n)
+    ws = _WS.get(key)
+    if ws is None:
+        ws = torch.zeros(n, dtype=torch.uint8, device=device)
+        _WS[key] = ws
+    return ws
+
+
+def prefill_stats(q_ctx, k, v, stats=None, scale=0.0, stream=None):
+    B, Hkv, L, d = k.shape
+    Hq = q_ctx.shape[1]
+    shape = make_shape(k, Hq)
+    if stats is None:
+        stats = Stats(B, Hq, Hkv, L, d, k.dtype, k.device)
+    ws = workspace(shape, None, OP_PREFILL, k.device)
+    st = stats.c()
+    _check(_lib().sa_prefill_stats(ctypes.byref(shape), _ptr(q_ctx), _ptr(k), _ptr(v), ctypes.byref(st),
+                                   float(scale), _ptr(ws), ws.numel(), _stream(stream)), "sa_prefill_stats")
+    return stats
+
+
+def block_summaries(k, blk_begin, blk_end, stats, Hq, stream=None):
+    shape = make_shape(k, Hq)
+    _check(_lib().sa_block_summaries(ctypes.byref(shape), _ptr(k), int(blk_begin), int(blk_end),
+                                     _ptr(stats.blk_mean), _ptr(stats.kbar_absmax), _stream(stream)),
+           "sa_block_summaries")
+
+
+def select(q, stats, params, k=None, v=None, selection=None, scale=0.0, stream=None):
+    B, Hq, d = q.shape
+    Hkv, L = stats.blk_mean.shape[1], stats.blk_mean.shape[2] * 16
+    shape = sa_shape(B, Hq, Hkv, d, L, _dtype_code(q))
+    cp = params.c()
+    if selection is None:
+        selection = Selection(B, Hkv, params.k_blocks, cp.sample_cap, q.device)
+    ws = workspace(shape, cp, OP_SELECT, q.device)
+    st = stats.c()
+    sel = selection.c()
+    _check(_lib().sa_select(ctypes.byref(shape), ctypes.byref(cp), _ptr(q), ctypes.byref(st), _ptr(k), _ptr(v),
+                            ctypes.byref(sel), float(scale), _ptr(ws), ws.numel(), _stream(stream)),
+           "sa_select")
+    return selection
+
+
+def decode(q, k, v, stats, selection, params, mode="resa", lam=1.0, scale=0.0, out=None, stream=None):
+    B, Hq, d = q.shape
+    shape = make_shape(k, Hq)
+    cp = params.c()
+    dp = sa_decode_params(MODES[mode], float(lam), float(scale))
+    if out is None:
+        out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
+    ws = workspace(shape, cp, OP_DECODE, q.device)
+    st = stats.c() if stats is not None else sa_stats()
+    sel = selection.c()
+    _check(_lib().sa_decode(ctypes.byref(shape), ctypes.byref(dp), ctypes.byref(cp), _ptr(q), _ptr(k), _ptr(v),
+                            ctypes.byref(st), ctypes.byref(sel), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+           "sa_decode")
+    return out
+
+
+def dense_decode(q, k, v, scale=0.0, out=None, stream=None):
+    B, Hq, d = q.shape
+    shape = make_shape(k, Hq)
+    if out is None:
+        out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
+    ws = workspace(shape, None, OP_DENSE, q.device)
+    _check(_lib().sa_dense_decode(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(out), float(scale),
+                                  _ptr(ws), ws.numel(), _stream(stream)), "sa_dense_decode")
+    return out

@@ -1,0 +1,176 @@
+// Host-side plans shared by the C ABI and the kernel launchers: split counts
+// and workspace offsets.  The same functions size the workspace and lay it
+// out at launch, so the two can never disagree.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/sa_decode.h"
+
+namespace sa {
+
+constexpr int kSmTarget = 148 * 4;   // CTAs to aim for: 4 per SM on B200
+
+struct Dims {
+    int B, Hq, Hkv, G, d, L;
+    int bf16;          // 1: bf16 cache and queries, 0: fp32
+    int U() const { return B * Hkv; }
+    int nb() const { return L / 16; }
+};
+
+// Exactly-read set geometry of a unit (same for all units of a shape).
+struct SetGeom {
+    int s_eff;       // sink tokens actually read: min(sink, L)
+    int w_eff;       // window tokens read, disjoint from the sink
+    int c_lo, c_hi;  // candidate blocks [c_lo, c_hi)
+    int n_cand;
+    int kk;          // blocks chosen per unit
+    int n_i;         // |I|
+    int n_t;         // L - |I|
+};
+
+inline SetGeom set_geom(const Dims& d, int sink, int local, int k_blocks) {
+    SetGeom g;
+    g.s_eff = sink < d.L ? sink : d.L;
+    int w = local < d.L ? local : d.L;
+    g.w_eff = w < d.L - g.s_eff ? w : d.L - g.s_eff;
+    g.c_lo = (sink + 15) / 16;
+    int hi = d.L - local;
+    g.c_hi = hi > 0 ? hi / 16 : 0;
+    if (g.c_hi < g.c_lo) g.c_hi = g.c_lo;
+    g.n_cand = g.c_hi - g.c_lo;
+    g.kk = k_blocks < g.n_cand ? k_blocks : g.n_cand;
+    g.n_i = g.s_eff + g.w_eff + 16 * g.kk;
+    g.n_t = d.L - g.n_i;
+    return g;
+}
+
+inline int clampi(int x, int lo, int hi) { return x < lo ? lo : (x > hi ? hi : x); }
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+struct PrefillPlan {
+    int nsq, rows_q;             // q-mean splits per (b, h), rows per split
+    int nskv, tok_kv;            // KV-pass splits per unit, tokens per split (x16)
+    size_t off_qpart, off_qcnt, off_kvpart, off_kvcnt, bytes;
+    int kv_stride;               // floats per KV-pass partial record
+};
+
+inline PrefillPlan prefill_plan(const Dims& d) {
+    PrefillPlan p;
+    const int BH = d.B * d.Hq;
+    p.nsq = clampi(cdiv(kSmTarget, BH), 1, d.L / 256 > 0 ? d.L / 256 : 1);
+    p.rows_q = cdiv(d.L, p.nsq);
+    p.nsq = cdiv(d.L, p.rows_q);
+    p.nskv = clampi(cdiv(kSmTarget, d.U()), 1, d.L / 256 > 0 ? d.L / 256 : 1);
+    p.tok_kv = cdiv(d.nb(), p.nskv) * 16;
+    p.nskv = cdiv(d.L, p.tok_kv);
+    // m[G], l[G], acc[G][d], vsum[d], absmax, pad to even, then ksum[d] as f64
+    int f = 2 * d.G + d.G * d.d + d.d + 1;
+    f = (f + 1) & ~1;
+    p.kv_stride = f + 2 * d.d;
+    size_t off = 0;
+    p.off_qpart = off; off = align256(off + sizeof(float) * (size_t)BH * p.nsq * d.d);
+    p.off_qcnt = off;  off = align256(off + sizeof(unsigned) * (size_t)BH);
+    p.off_kvpart = off; off = align256(off + sizeof(float) * (size_t)d.U() * p.nskv * p.kv_stride);
+    p.off_kvcnt = off; off = align256(off + sizeof(unsigned) * (size_t)d.U());
+    p.bytes = off;
+    return p;
+}
+
+struct SelectPlan {
+    SetGeom g;
+    int nss, rows_s;             // scan splits per unit, candidate rows per split
+    size_t off_scores, off_xkey, off_flags, off_cnt, bytes;
+};
+
+inline SelectPlan select_plan(const Dims& d, const sa_select_params& sp) {
+    SelectPlan p;
+    p.g = set_geom(d, sp.sink, sp.local, sp.k_blocks);
+    const int nc = p.g.n_cand > 0 ? p.g.n_cand : 1;
+    p.nss = clampi(cdiv(kSmTarget, d.U()), 1, cdiv(nc, 64));
+    p.rows_s = cdiv(nc, p.nss);
+    p.nss = cdiv(nc, p.rows_s);
+    size_t off = 0;
+    p.off_scores = off; off = align256(off + sizeof(float) * (size_t)d.U() * nc);
+    p.off_xkey = off;   off = align256(off + sizeof(unsigned long long) * (size_t)d.U() * nc);
+    p.off_flags = off;  off = align256(off + (size_t)d.U() * nc);
+    p.off_cnt = off;    off = align256(off + sizeof(unsigned) * (size_t)d.U());
+    p.bytes = off;
+    return p;
+}
+
+struct DecodePlan {
+    SetGeom g;
+    int n_tok_max;               // |I| + sample capacity
+    int nsd, tok_d;              // splits per unit, tokens per split
+    int rec;                     // floats per partial record
+    size_t off_part, off_cnt, bytes;
+};
+
+inline DecodePlan decode_plan(const Dims& d, const sa_select_params& sp) {
+    DecodePlan p;
+    p.g = set_geom(d, sp.sink, sp.local, sp.k_blocks);
+    p.n_tok_max = p.g.n_i + (sp.sample_cap > 0 ? sp.sample_cap : 0);
+    const int nt = p.n_tok_max > 0 ? p.n_tok_max : 1;
+    p.nsd = clampi(cdiv(kSmTarget, d.U()), 1, cdiv(nt, 32));
+    p.tok_d = cdiv(nt, p.nsd);
+    p.nsd = cdiv(nt, p.tok_d);
+    // exact (m,l,acc) + prior (m0,l0,acc0) per head, then ksum, vsum
+    p.rec = 2 * d.G * (2 + d.d) + 2 * d.d;
+    size_t off = 0;
+    p.off_part = off; off = align256(off + sizeof(float) * (size_t)d.U() * p.nsd * p.rec);
+    p.off_cnt = off;  off = align256(off + sizeof(unsigned) * (size_t)d.U());
+    p.bytes = off;
+    return p;
+}
+
+struct DensePlan {
+    int nsdn, tok;
+    int rec;
+    size_t off_part, off_cnt, bytes;
+};
+
+inline DensePlan dense_plan(const Dims& d) {
+    DensePlan p;
+    p.nsdn = clampi(cdiv(2 * kSmTarget, d.U()), 1, d.L / 256 > 0 ? d.L / 256 : 1);
+    p.tok = cdiv(d.nb(), p.nsdn) * 16;
+    p.nsdn = cdiv(d.L, p.tok);
+    p.rec = d.G * (2 + d.d);
+    size_t off = 0;
+    p.off_part = off; off = align256(off + sizeof(float) * (size_t)d.U() * p.nsdn * p.rec);
+    p.off_cnt = off;  off = align256(off + sizeof(unsigned) * (size_t)d.U());
+    p.bytes = off;
+    return p;
+}
+
+// ---- launchers (one per .cu file) -----------------------------------------
+
+struct PrefillArgs {
+    const void* q_ctx; const void* k; const void* v;
+    sa_stats st; float scale; char* ws;
+};
+cudaError_t launch_prefill(const Dims& d, const PrefillPlan& p, const PrefillArgs& a, cudaStream_t s);
+cudaError_t launch_block_summaries(const Dims& d, const void* k, int blk_begin, int blk_end,
+                                   void* blk_mean, float* kbar_absmax, cudaStream_t s);
+
+struct SelectArgs {
+    const void* q; sa_stats st; const void* k; const void* v;
+    sa_selection sel; sa_select_params sp; float scale; char* ws;
+};
+cudaError_t launch_select(const Dims& d, const SelectPlan& p, const SelectArgs& a, cudaStream_t s);
+
+struct DecodeArgs {
+    const void* q; const void* k; const void* v; sa_stats st; sa_selection sel;
+    sa_select_params sp; sa_decode_params dp; float scale; float* out; char* ws;
+};
+cudaError_t launch_decode(const Dims& d, const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
+
+struct DenseArgs {
+    const void* q; const void* k; const void* v; float scale; float* out; char* ws;
+};
+cudaError_t launch_dense(const Dims& d, const DensePlan& p, const DenseArgs& a, cudaStream_t s);
+
+}  // namespace sa

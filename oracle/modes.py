@@ -29,7 +29,11 @@ def dense(q, k, v, scale):
 
 
 def drop(q, k, v, idx, scale):
-    """Sparse attention that treats the unread tail as contributing zero."""
+    """Sparse attention that treats the unread tail as contributing zero.
+    Attention over an empty set carries no mass and returns the zero vector
+    (the pages never read nothing; this is the plain reading of an empty sum)."""
+    if len(idx) == 0:
+        return np.zeros((q.shape[0], v.shape[1]))
     return dense(q, k[idx], v[idx], scale)
 
 
@@ -52,7 +56,7 @@ def resa(q, k, v, idx, st, scale, lam=1.0):
     """
     L = k.shape[0]
     n_t = L - len(idx)
-    if n_t == 0:
+    if n_t == 0 or (lam == 0 and len(idx) == 0):    # nothing to merge: no mass at all
         return drop(q, k, v, idx, scale)
     kI, vI = k[idx], v[idx]
     c = scale * ((q - st["mu_q"]) @ st["mu_k"])                  # [G]

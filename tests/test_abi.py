@@ -1,0 +1,117 @@
+"""The C ABI loads, exports every symbol the header declares, sizes its
+workspaces, and rejects bad arguments before launching anything.
+
+Runs without a GPU: every call below fails argument validation, so nothing is
+enqueued (the pointers passed are never dereferenced)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import kv_cache_residual_b200 as sa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(sa.LIB_PATH):
+        from kv_cache_residual_b200 import build
+        build.build()
+    return sa._lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    hdr = open(os.path.join(ROOT, "include", "sa_decode.h")).read()
+    declared = set(re.findall(r"^SA_API\s+[\w\s\*]+?\b(sa_\w+)\s*\(", hdr, flags=re.M))
+    assert declared == set(sa.EXPORTS)
+    for name in declared:
+        assert hasattr(lib, name)
+
+
+def _shape(**kw):
+    base = dict(B=2, Hq=8, Hkv=2, d=128, L=4096, dtype=sa.SA_BF16)
+    base.update(kw)
+    return sa.sa_shape(base["B"], base["Hq"], base["Hkv"], base["d"], base["L"], base["dtype"])
+
+
+def test_workspace_sizes(lib):
+    sp = sa.SelectParams(sink=64, local=128, k_blocks=8, sample_b=64, sample_cap=64).c()
+    for op in range(4):
+        n = lib.sa_workspace_size(ctypes.byref(_shape()), ctypes.byref(sp), op)
+        assert n > 0 and n % 256 == 0
+    assert lib.sa_workspace_size(ctypes.byref(_shape(d=96)), ctypes.byref(sp), 0) == 0
+    assert lib.sa_workspace_size(ctypes.byref(_shape(L=100)), ctypes.byref(sp), 0) == 0
+    assert lib.sa_workspace_size(None, ctypes.byref(sp), 0) == 0
+    assert lib.sa_workspace_size(ctypes.byref(_shape()), None, sa.OP_SELECT) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=96), sa.SA_ERR_UNSUPPORTED),
+    (dict(Hq=12, Hkv=4), sa.SA_ERR_UNSUPPORTED),     # G = 3
+    (dict(Hq=9, Hkv=2), sa.SA_ERR_INVALID_ARG),
+    (dict(L=1000), sa.SA_ERR_INVALID_ARG),
+    (dict(L=0), sa.SA_ERR_INVALID_ARG),
+    (dict(B=0), sa.SA_ERR_INVALID_ARG),
+    (dict(dtype=7), sa.SA_ERR_INVALID_ARG),
+])
+def test_bad_shapes_rejected(lib, kw, status):
+    p = ctypes.c_void_p(0x10000)
+    st = sa.sa_stats(*([0x10000] * 8))
+    assert lib.sa_dense_decode(ctypes.byref(_shape(**kw)), p, p, p, p, 0.0, p, 1 << 30, None) == status
+    assert lib.sa_prefill_stats(ctypes.byref(_shape(**kw)), p, p, p, ctypes.byref(st), 0.0, p, 1 << 30, None) == status
+
+
+def test_bad_pointers_and_workspace_rejected(lib):
+    sh = _shape()
+    good = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10004)              # not 16-byte aligned
+    assert lib.sa_dense_decode(ctypes.byref(sh), None, good, good, good, 0.0, good, 1 << 30, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_dense_decode(ctypes.byref(sh), odd, good, good, good, 0.0, good, 1 << 30, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_dense_decode(ctypes.byref(sh), good, good, good, good, -1.0, good, 1 << 30, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_dense_decode(ctypes.byref(sh), good, good, good, good, 0.0, None, 1 << 30, None) == sa.SA_ERR_WORKSPACE
+    assert lib.sa_dense_decode(ctypes.byref(sh), good, good, good, good, 0.0, good, 16, None) == sa.SA_ERR_WORKSPACE
+    st_bad = sa.sa_stats(0x10000, 0x10000, 0x10000, 0x10000, 0x10000, 0x10000, 0x10008, 0x10000)
+    assert lib.sa_prefill_stats(ctypes.byref(sh), good, good, good, ctypes.byref(st_bad), 0.0, good, 1 << 30, None) == sa.SA_ERR_INVALID_ARG
+
+
+def test_select_and_decode_param_checks(lib):
+    sh = _shape()
+    p = ctypes.c_void_p(0x10000)
+    st = sa.sa_stats(*([0x10000] * 8))
+    sel = sa.sa_selection(0x10000, 0x10000, 0x10000, 0)
+    bad = [
+        sa.sa_select_params(-1, 128, 8, 0, 0, 0, 0.05, 0.05, 0, 0),     # negative sink
+        sa.sa_select_params(64, 128, -2, 0, 0, 0, 0.05, 0.05, 0, 0),    # negative k
+        sa.sa_select_params(64, 128, 8, 65, 0, 64, 0.05, 0.05, 0, 0),   # b above capacity
+    ]
+    for sp in bad:
+        assert lib.sa_select(ctypes.byref(sh), ctypes.byref(sp), p, ctypes.byref(st), None, None,
+                             ctypes.byref(sel), 0.0, p, 1 << 30, None) == sa.SA_ERR_INVALID_ARG
+    clt = sa.sa_select_params(64, 128, 8, 0, 64, 512, 0.05, 0.05, 0, 0)
+    ok_sp = sa.sa_select_params(64, 128, 8, 0, 0, 0, 0.05, 0.05, 0, 0)
+    # workspace too small
+    assert lib.sa_select(ctypes.byref(sh), ctypes.byref(ok_sp), p, ctypes.byref(st), None, None,
+                         ctypes.byref(sel), 0.0, p, 64, None) == sa.SA_ERR_WORKSPACE
+    for mode, lam in [(9, 1.0), (1, 1.5), (1, -0.1)]:
+        dp = sa.sa_decode_params(mode, lam, 0.0)
+        assert lib.sa_decode(ctypes.byref(sh), ctypes.byref(dp), ctypes.byref(ok_sp), p, p, p, ctypes.byref(st),
+                             ctypes.byref(sel), p, p, 1 << 30, None) == sa.SA_ERR_INVALID_ARG
+    # sampling without any draw capacity
+    dp = sa.sa_decode_params(sa.MODES["sample"], 1.0, 0.0)
+    assert lib.sa_decode(ctypes.byref(sh), ctypes.byref(dp), ctypes.byref(ok_sp), p, p, p, ctypes.byref(st),
+                         ctypes.byref(sel), p, p, 1 << 30, None) == sa.SA_ERR_INVALID_ARG
+    # RESA needs its statistics
+    dp = sa.sa_decode_params(sa.MODES["resa"], 1.0, 0.0)
+    assert lib.sa_decode(ctypes.byref(sh), ctypes.byref(dp), ctypes.byref(ok_sp), p, p, p, None,
+                         ctypes.byref(sel), p, p, 1 << 30, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_block_summaries(ctypes.byref(sh), p, 10, 5, p, p, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_block_summaries(ctypes.byref(sh), p, 0, 4096, p, p, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_block_summaries(ctypes.byref(sh), p, 3, 3, p, p, None) == sa.SA_OK   # empty range: no launch
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert lib.sa_status_string(s)
+    assert lib.sa_status_string(99) == b"unknown status"

@@ -1,0 +1,232 @@
+"""GPU parity: every stage of the CUDA path against the fp64 oracle on the same
+seeded inputs.
+
+Bars: block means, selected block sets and tail draws bit-exact; outputs
+within rel-L2 2e-3 (the target the method's build states); statistics within
+bounds derived from fp32 accumulation over L terms (written per check)."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+import kv_cache_residual_b200 as sa
+from parity_util import REL_L2_OUT, OracleUnit, f64, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+MODES = ("drop", "resa", "proxy", "sample")
+
+# small cases: several split tiles and a ragged tail, every dtype / d / G
+CASES = {
+    "tiny": synth.WORKLOADS["tiny"],
+    "bf16_d128_g4": synth.scaled(synth.WORKLOADS["llama"], B=2, Hq=8, Hkv=2, L=4000, n_hh=16, seed=11),
+    "bf16_d64_g8": synth.scaled(synth.WORKLOADS["llama"], B=1, Hq=16, Hkv=2, d=64, L=1072, n_hh=8, seed=12,
+                                sink=20, local=10),
+    "f32_d128_g1": synth.scaled(synth.WORKLOADS["llama"], B=2, Hq=2, Hkv=2, dtype="f32", L=2048, n_hh=8, seed=13),
+    "bf16_d128_g2": synth.scaled(synth.WORKLOADS["llama"], B=3, Hq=6, Hkv=3, L=1536, n_hh=8, seed=14, sink=16,
+                                 local=48),
+}
+
+
+def _sp(w, k_blocks=None, sample_b=64, step=0, **kw):
+    kb = w.budgets()[0][1] if k_blocks is None else k_blocks
+    if w.k_blocks is None and k_blocks is None:
+        kb = max(kb, 6)
+    return sa.SelectParams(sink=w.sink, local=w.local, k_blocks=kb, sample_b=sample_b, sample_cap=max(sample_b, 1),
+                           seed=1234 + w.seed, step=step, **kw)
+
+
+@pytest.fixture(scope="module")
+def dev():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return torch.device("cuda")
+
+
+_DATA = {}
+
+
+def _data(name, dev, steps=3):
+    if name not in _DATA:
+        w = CASES[name]
+        d = synth.make_batch(w, device="cpu", steps=steps)
+        _DATA[name] = (w, {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in d.items()})
+    return _DATA[name]
+
+
+def _units(w):
+    return [(b, g) for b in range(w.B) for g in range(w.Hkv)]
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_prefill_stats(name, dev):
+    w, data = _data(name, dev)
+    st = sa.prefill_stats(data["q_ctx"], data["k"], data["v"])
+    torch.cuda.synchronize()
+    for b, g in _units(w):
+        o = OracleUnit(data, b, g, w.G, w.dtype)
+        hs = slice(g * w.G, (g + 1) * w.G)
+        # fp32 sums of L terms: relative error ~ L * 2^-24 worst case, far less typically
+        assert rel_l2(f64(st.mu_q[b, hs]), o.st["mu_q"]) < 1e-5
+        assert rel_l2(f64(st.o_est[b, hs]), o.st["o_est"]) < 1e-4
+        np.testing.assert_allclose(f64(st.log_z0[b, hs]), o.st["log_z0"], rtol=0, atol=2e-5 * max(1, np.abs(o.st["log_z0"]).max()))
+        assert rel_l2(f64(st.mu_k[b, g]), o.st["mu_k"]) < 1e-6
+        assert rel_l2(f64(st.sum_k[b, g]), o.st["sum_k"]) < 1e-6
+        assert rel_l2(f64(st.sum_v[b, g]), o.st["sum_v"]) < 1e-4
+        # block means: one rounding of the exact mean on both sides -> identical
+        np.testing.assert_array_equal(f64(st.blk_mean[b, g]), o.st["blk_mean"])
+        assert float(st.kbar_absmax[b, g]) == o.st["kbar_absmax"]
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_select_and_decode(name, dev):
+    w, data = _data(name, dev)
+    st = sa.prefill_stats(data["q_ctx"], data["k"], data["v"])
+    oracles = {u: OracleUnit(data, u[0], u[1], w.G, w.dtype) for u in _units(w)}
+    worst = {m: 0.0 for m in MODES + ("dense",)}
+    for step in range(3):
+        sp = _sp(w, step=step)
+        q = data["q"][step]
+        sel = sa.select(q, st, sp)
+        outs = {m: sa.decode(q, data["k"], data["v"], st, sel, sp, mode=m) for m in MODES}
+        outs["dense"] = sa.dense_decode(q, data["k"], data["v"])
+        torch.cuda.synchronize()
+        for (b, g), o in oracles.items():
+            qq = o.q(q)
+            blocks, idx, tail = o.select(qq, sp)
+            kk = len(blocks)
+            got = sel.blk_idx[b, g].cpu().numpy()
+            np.testing.assert_array_equal(got[:kk], blocks)
+            assert np.all(got[kk:] == -1)
+            nb = int(sel.samp_count[b, g])
+            assert nb == (min(sp.sample_b, sp.sample_cap) if len(tail) else 0)
+            pos = o.draws(tail, sp, nb)
+            np.testing.assert_array_equal(sel.samp_idx[b, g, :nb].cpu().numpy(), pos)
+            for m in MODES + ("dense",):
+                want = o.out(m, qq, idx, pos=pos)
+                e = rel_l2(f64(outs[m][b, g * w.G:(g + 1) * w.G]), want)
+                worst[m] = max(worst[m], e)
+    for m, e in worst.items():
+        assert e < REL_L2_OUT, (m, e)
+
+
+def _edge_run(name, dev, sp, modes=MODES, lam=1.0):
+    w, data = _data(name, dev)
+    st = sa.prefill_stats(data["q_ctx"], data["k"], data["v"])
+    q = data["q"][0]
+    sel = sa.select(q, st, sp)
+    outs = {m: sa.decode(q, data["k"], data["v"], st, sel, sp, mode=m, lam=lam) for m in modes}
+    outs["dense"] = sa.dense_decode(q, data["k"], data["v"])
+    torch.cuda.synchronize()
+    return w, data, st, sel, outs
+
+
+@pytest.mark.parametrize("name", ["tiny", "bf16_d128_g4"])
+def test_full_budget_is_dense(name, dev):
+    w = CASES[name]
+    sp = _sp(w, k_blocks=10 ** 6)
+    w, data, st, sel, outs = _edge_run(name, dev, sp)
+    for b, g in _units(w):
+        o = OracleUnit(data, b, g, w.G, w.dtype)
+        want = o.out("dense", o.q(data["q"][0]), np.arange(w.L))
+        hs = slice(g * w.G, (g + 1) * w.G)
+        assert int(sel.samp_count[b, g]) == 0
+        for m in MODES:
+            assert rel_l2(f64(outs[m][b, hs]), want) < REL_L2_OUT
+            assert rel_l2(f64(outs[m][b, hs]), f64(outs["dense"][b, hs])) < 1e-5
+
+
+@pytest.mark.parametrize("sink,local,kb", [(2000, 100, 5), (0, 0, 0), (0, 0, 3), (17, 33, 4), (1024, 1024, 8)])
+def test_degenerate_sets(sink, local, kb, dev):
+    name = "tiny"
+    w = CASES[name]
+    sp = dataclasses.replace(_sp(w), sink=sink, local=local, k_blocks=kb)
+    w, data, st, sel, outs = _edge_run(name, dev, sp)
+    o = OracleUnit(data, 0, 0, w.G, w.dtype)
+    qq = o.q(data["q"][0])
+    blocks, idx, tail = o.select(qq, sp)
+    np.testing.assert_array_equal(sel.blk_idx[0, 0, :len(blocks)].cpu().numpy(), blocks)
+    nb = int(sel.samp_count[0, 0])
+    pos = o.draws(tail, sp, nb)
+    np.testing.assert_array_equal(sel.samp_idx[0, 0, :nb].cpu().numpy(), pos)
+    for m in MODES:
+        assert rel_l2(f64(outs[m][0]), o.out(m, qq, idx, pos=pos)) < REL_L2_OUT, m
+
+
+def test_ties_take_lowest_blocks_via_fp64_rescore(dev):
+    # every block of a unit has the same mean: all scores tie, the fp32 band
+    # holds every candidate, the fp64 rescore runs and ties go to low indices
+    w = synth.scaled(CASES["bf16_d128_g4"], B=1, Hkv=2, Hq=8, L=2048)
+    d = synth.make_batch(w, device="cpu", steps=1)
+    k = d["k"]
+    k[0, 0] = k[0, 0, :16].repeat(w.L // 16, 1)           # identical blocks in unit (0, 0)
+    data = {n: (t.to(dev) if torch.is_tensor(t) else t) for n, t in d.items()}
+    st = sa.prefill_stats(data["q_ctx"], data["k"], data["v"])
+    sp = sa.SelectParams(sink=64, local=128, k_blocks=7, sample_b=8, sample_cap=8, seed=3)
+    sel = sa.select(data["q"][0], st, sp)
+    torch.cuda.synchronize()
+    assert sel.blk_idx[0, 0, :7].tolist() == list(range(4, 11))
+    assert int(sel.n_rescored[0, 0]) > 7
+    o = OracleUnit(data, 0, 1, w.G, w.dtype)
+    blocks, _, _ = o.select(o.q(data["q"][0]), sp)
+    assert sel.blk_idx[0, 1, :7].tolist() == blocks.tolist()
+
+
+def test_resa_lambda_zero_is_drop(dev):
+    sp = _sp(CASES["bf16_d128_g4"])
+    w, data, st, sel, outs = _edge_run("bf16_d128_g4", dev, sp, modes=("resa", "drop"), lam=0.0)
+    assert rel_l2(f64(outs["resa"]), f64(outs["drop"])) < 1e-6
+
+
+def test_deterministic_outputs(dev):
+    sp = _sp(CASES["bf16_d128_g4"])
+    a = _edge_run("bf16_d128_g4", dev, sp)[4]
+    b = _edge_run("bf16_d128_g4", dev, sp)[4]
+    for m in a:
+        assert torch.equal(a[m], b[m]), m
+
+
+def test_block_summaries_entry_point(dev):
+    w, data = _data("bf16_d128_g4", dev)
+    st = sa.prefill_stats(data["q_ctx"], data["k"], data["v"])
+    bm = st.blk_mean.clone()
+    st.blk_mean.zero_()
+    st.kbar_absmax.zero_()
+    nb = w.L // 16
+    sa.block_summaries(data["k"], 0, nb // 3, st, w.Hq)
+    sa.block_summaries(data["k"], nb // 3, nb, st, w.Hq)
+    torch.cuda.synchronize()
+    assert torch.equal(st.blk_mean, bm)
+    assert torch.equal(st.kbar_absmax, bm.float().abs().amax(dim=(2, 3)))
+
+
+@pytest.mark.parametrize("wname,units", [("llama", [(0, 0), (0, 3), (0, 7)]),
+                                         ("batched", [(0, 0), (17, 5), (31, 7)])])
+def test_full_size_sampled_units(wname, units, dev):
+    """Full workload sizes, in the launch configuration the benchmark uses;
+    outputs of sampled units checked against the oracle one by one."""
+    w = synth.WORKLOADS[wname]
+    data = synth.make_batch(w, device=dev, steps=2)
+    st = sa.prefill_stats(data["q_ctx"], data["k"], data["v"])
+    for label, kb in w.budgets():
+        sp = sa.SelectParams(sink=w.sink, local=w.local, k_blocks=kb, sample_b=64, sample_cap=64, seed=7, step=1)
+        q = data["q"][1]
+        sel = sa.select(q, st, sp)
+        outs = {m: sa.decode(q, data["k"], data["v"], st, sel, sp, mode=m) for m in MODES}
+        outs["dense"] = sa.dense_decode(q, data["k"], data["v"])
+        torch.cuda.synchronize()
+        assert int((sel.blk_idx[..., :kb] < 0).sum()) == 0
+        for b, g in units:
+            o = OracleUnit(data, b, g, w.G, w.dtype)
+            np.testing.assert_array_equal(f64(st.blk_mean[b, g]), o.st["blk_mean"])
+            qq = o.q(q)
+            blocks, idx, tail = o.select(qq, sp)
+            np.testing.assert_array_equal(sel.blk_idx[b, g].cpu().numpy(), blocks)
+            pos = o.draws(tail, sp, 64)
+            np.testing.assert_array_equal(sel.samp_idx[b, g].cpu().numpy(), pos)
+            for m in MODES + ("dense",):
+                e = rel_l2(f64(outs[m][b, g * w.G:(g + 1) * w.G]), o.out(m, qq, idx, pos=pos))
+                assert e < REL_L2_OUT, (label, b, g, m, e)
+    del data
+    torch.cuda.empty_cache()

@@ -208,3 +208,13 @@ def test_modes_against_plain_loops(mode):
     pos = rng.sample_positions(5, 0, 0, 3, tail, 9)
     got = modes.run_mode(mode, q, k, v, idx, st, s, pos=pos)
     np.testing.assert_allclose(got, _loop_unit(mode, q, k, v, idx, st, s, pos), rtol=1e-11, atol=1e-12)
+
+
+def test_empty_exact_set():
+    q, k, v, st, s = _setup(13)
+    empty = np.zeros(0, dtype=np.int64)
+    assert np.array_equal(modes.drop(q, k, v, empty, s), np.zeros((q.shape[0], v.shape[1])))
+    assert np.array_equal(modes.resa(q, k, v, empty, st, s, 0.0), np.zeros((q.shape[0], v.shape[1])))
+    # the proxy alone is the tail-mean value (one token carries all weight)
+    np.testing.assert_allclose(modes.proxy(q, k, v, empty, st, s), np.tile(v.mean(0), (q.shape[0], 1)),
+                               rtol=1e-12, atol=1e-13)
