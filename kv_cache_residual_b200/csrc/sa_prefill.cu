@@ -161,8 +161,9 @@ k_kvpass(const T* __restrict__ k, const T* __restrict__ v, const float* __restri
             ks[e] += __shfl_xor_sync(0xffffffffu, ks[e], off);
             vs[e] += __shfl_xor_sync(0xffffffffu, vs[e], off);
         }
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     if (lane < CPR) {
 #pragma unroll
         for (int e = 0; e < EPC; ++e) {

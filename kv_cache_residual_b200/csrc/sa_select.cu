@@ -19,6 +19,8 @@
 
 namespace sa {
 
+constexpr int kSmemKeys = 4096;     // candidate keys staged in shared memory (16 KB)
+
 __device__ __forceinline__ uint32_t fkey(float y) {
     const uint32_t b = __float_as_uint(y + 0.0f);   // -0 -> +0
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
@@ -31,12 +33,17 @@ __device__ __forceinline__ unsigned long long dkey(double x) {
     return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
 }
 
-// Block-wide exclusive scan of a 0/1 flag over the CTA (index order).
-// Returns this thread's rank; *total gets the count.  Uses sw[kWarps+1].
-__device__ __forceinline__ int block_rank(bool f, int* sw, int* total) {
+// Block-wide exclusive scan of one int per thread (thread order).  Returns
+// this thread's exclusive prefix; *total gets the sum.  Uses sw[kWarps+1].
+__device__ __forceinline__ int block_exscan(int v, int* sw, int* total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const unsigned bal = __ballot_sync(0xffffffffu, f);
-    if (lane == 0) sw[warp] = __popc(bal);
+    int inc = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, inc, off);
+        if (lane >= off) inc += o;
+    }
+    if (lane == 31) sw[warp] = inc;
     __syncthreads();
     if (threadIdx.x == 0) {
         int s = 0;
@@ -44,10 +51,16 @@ __device__ __forceinline__ int block_rank(bool f, int* sw, int* total) {
         sw[kWarps] = s;
     }
     __syncthreads();
-    const int r = sw[warp] + __popc(bal & ((1u << lane) - 1u));
+    const int r = sw[warp] + inc - v;
     *total = sw[kWarps];
     __syncthreads();
     return r;
+}
+
+__device__ __forceinline__ int block_sum(int v, int* sw) {
+    int tot;
+    (void)block_exscan(v, sw, &tot);
+    return tot;
 }
 
 // Radix select (MSB first, 8 bits per pass) of the kk-th largest key among
@@ -97,21 +110,31 @@ __device__ void radix_select(KeyFn key, int n, int kk, KT* thr, int* need, unsig
     *need = rem;
 }
 
-// flags[i] = 1 for the top kk of key(), ties at the threshold to lowest index.
+// Writes, in ascending index order, c_lo + i for the top kk of key(0..n-1):
+// every key above thr, and the first `need` keys equal to thr (lowest index
+// first).  Each thread owns one contiguous chunk of indices.
 template <typename KT, typename KeyFn>
-__device__ void flag_topk(KeyFn key, int n, KT thr, int need, unsigned char* flags, int* sw) {
-    int base = 0;
-    for (int i0 = 0; i0 < n; i0 += kThreads) {
-        const int i = i0 + threadIdx.x;
-        KT kx = 0;
-        if (i < n) kx = key(i);
-        const bool eq = (i < n) && kx == thr;
-        int tot;
-        const int r = block_rank(eq, sw, &tot);
-        if (i < n) flags[i] = (kx > thr || (eq && base + r < need)) ? 1 : 0;
-        base += tot;
+__device__ void emit_topk(KeyFn key, int n, KT thr, int need, int kk, int c_lo, int32_t* out_idx, int* sw) {
+    const int C = (n + kThreads - 1) / kThreads;
+    const int i0 = min(n, (int)threadIdx.x * C), i1 = min(n, i0 + C);
+    int eqc = 0;
+    for (int i = i0; i < i1; ++i) eqc += (key(i) == thr) ? 1 : 0;
+    int tot;
+    const int eq_before = block_exscan(eqc, sw, &tot);
+    int selc = 0, r = eq_before;
+    for (int i = i0; i < i1; ++i) {
+        const KT kx = key(i);
+        if (kx > thr) ++selc;
+        else if (kx == thr) { if (r < need) ++selc; ++r; }
     }
-    __syncthreads();
+    int p = block_exscan(selc, sw, &tot);
+    r = eq_before;
+    for (int i = i0; i < i1; ++i) {
+        const KT kx = key(i);
+        bool take = kx > thr;
+        if (kx == thr) { take = r < need; ++r; }
+        if (take && p < kk) out_idx[p++] = c_lo + i;
+    }
 }
 
 template <typename T, int D, int G>
@@ -129,6 +152,7 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
     __shared__ int s_digit, s_rem, s_band;
     __shared__ double s_q64[D];
     __shared__ float s_qa[kWarps];
+    __shared__ uint32_t s_keys[kSmemKeys];
 
     const int u = blockIdx.y, split = blockIdx.x;
     const int b = u / Hkv, g = u - b * Hkv;
@@ -179,11 +203,27 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
     if (!last_cta_of_unit(cnt + u, nss)) return;
 
     // ---- top-k of the unit (last CTA) ------------------------------------------
-    unsigned char* fl = flags_ws + (size_t)u * (n > 0 ? n : 1);
     int32_t* out_idx = blk_idx + (size_t)u * kb_stride;
     int rescored = 0;
     if (kk > 0 && kk < n) {
-        auto k32 = [&](int i) -> uint32_t { return fkey(ldcg(sc + i)); };
+        // orderable keys, staged once: shared memory when they fit, else in
+        // place over the unit's scores in the workspace
+        uint32_t* keys = (n <= kSmemKeys) ? s_keys : reinterpret_cast<uint32_t*>(sc);
+        for (int i0 = 0; i0 < n; i0 += 4 * kThreads) {
+            float y[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i = i0 + j * kThreads + threadIdx.x;
+                y[j] = i < n ? ldcg(sc + i) : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i = i0 + j * kThreads + threadIdx.x;
+                if (i < n) keys[i] = fkey(y[j]);
+            }
+        }
+        __syncthreads();
+        auto k32 = [&](int i) -> uint32_t { return keys[i]; };
         uint32_t thr;
         int need;
         radix_select<uint32_t>(k32, n, kk, &thr, &need, hist, &s_digit, &s_rem);
@@ -200,17 +240,12 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
         float qsum = 0.f;
         for (int w = 0; w < kWarps; ++w) qsum += s_qa[w];
         const float E = (float)(G + D) * 0x1p-23f * qsum * kbar_absmax[u] * 1.0001f + 0x1p-100f;
-        const float lo = fkey_inv(thr) - 2.f * E;
+        const uint32_t lo_key = fkey(fkey_inv(thr) - 2.f * E);
         int band = 0;
-        for (int i = threadIdx.x; i < n; i += kThreads) band += (ldcg(sc + i) >= lo) ? 1 : 0;
-        for (int off = 16; off > 0; off >>= 1) band += __shfl_xor_sync(0xffffffffu, band, off);
-        if (threadIdx.x == 0) s_band = 0;
-        __syncthreads();
-        if (lane == 0) atomicAdd(&s_band, band);
-        __syncthreads();
-        band = s_band;
+        for (int i = threadIdx.x; i < n; i += kThreads) band += (keys[i] >= lo_key) ? 1 : 0;
+        band = block_sum(band, sw);
         if (band == kk) {
-            flag_topk<uint32_t>(k32, n, thr, need, fl, sw);
+            emit_topk<uint32_t>(k32, n, thr, need, kk, sg.c_lo, out_idx, sw);
         } else {
             // ambiguous: rescore every candidate of the band in fp64
             rescored = band;
@@ -223,7 +258,7 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
             unsigned long long* xk = xkey + (size_t)u * n;
             const T* bm = blk_mean + ((size_t)u * nb + sg.c_lo) * D;
             for (int i = warp; i < n; i += kWarps) {
-                const bool in_band = ldcg(sc + i) >= lo;       // warp-uniform
+                const bool in_band = keys[i] >= lo_key;       // warp-uniform
                 unsigned long long key = 0ull;
                 if (in_band) {
                     double x = 0.0;
@@ -239,19 +274,7 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
             unsigned long long thr64;
             int need64;
             radix_select<unsigned long long>(k64, n, kk, &thr64, &need64, hist, &s_digit, &s_rem);
-            flag_topk<unsigned long long>(k64, n, thr64, need64, fl, sw);
-        }
-        __threadfence_block();
-        __syncthreads();
-        // ascending compaction of the flags
-        int base = 0;
-        for (int i0 = 0; i0 < n; i0 += kThreads) {
-            const int i = i0 + threadIdx.x;
-            const bool f = (i < n) && fl[i];
-            int tot;
-            const int r = block_rank(f, sw, &tot);
-            if (f && base + r < kk) out_idx[base + r] = sg.c_lo + i;
-            base += tot;
+            emit_topk<unsigned long long>(k64, n, thr64, need64, kk, sg.c_lo, out_idx, sw);
         }
     } else if (kk > 0) {       // every candidate is chosen
         for (int i = threadIdx.x; i < kk; i += kThreads) out_idx[i] = sg.c_lo + i;
