@@ -49,7 +49,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--small", action="store_true", help="profiling case: B=4 (same kernels, smaller batch)")
+    ap.add_argument("--batch", type=int, default=0, help="override the batch size (profiling cases)")
     return ap.parse_args(argv)
 
 
@@ -248,8 +248,8 @@ def main(argv=None):
     args = parse_args(argv)
     import synth
     w = synth.WORKLOADS[args.workload]
-    if args.small:
-        w = synth.scaled(w, B=4)
+    if args.batch > 0:
+        w = synth.scaled(w, B=args.batch)
     kb = w.k_blocks_for(args.read) if w.k_blocks is None else w.k_blocks
     sg = set_geom(w.L, w.sink, w.local, kb)
     sp_kw = dict(sink=w.sink, local=w.local, k_blocks=kb, sample_b=args.sample_b, seed=2024)

@@ -164,11 +164,12 @@ sa_status sa_decode(const sa_shape* shape, const sa_decode_params* dparams, cons
             return SA_ERR_INVALID_ARG;
         if (m == SA_PROXY && (!aligned16(st.sum_k) || !aligned16(st.sum_v))) return SA_ERR_INVALID_ARG;
     }
-    const DecodePlan p = decode_plan(d, *sparams);
+    const DecodePlan p = decode_plan(d, *sparams, (int)m);
+    const size_t need = decode_plan(d, *sparams).bytes;
     if (p.g.kk > 0 && !aligned4(sel->blk_idx)) return SA_ERR_INVALID_ARG;
     if (m == SA_SAMPLE && (sparams->sample_cap < 1 || !aligned4(sel->samp_idx) || !aligned4(sel->samp_count)))
         return SA_ERR_INVALID_ARG;
-    if (ws == nullptr || ws_bytes < p.bytes || !aligned16(ws)) return SA_ERR_WORKSPACE;
+    if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return SA_ERR_WORKSPACE;
     DecodeArgs a{q, k, v, st, *sel, *sparams, *dparams, resolve_scale(dparams->scale, d.d), out,
                  static_cast<char*>(ws)};
     return launch_decode(d, p, a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SA_OK : SA_ERR_CUDA;

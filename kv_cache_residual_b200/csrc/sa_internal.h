@@ -71,11 +71,12 @@ inline PrefillPlan prefill_plan(const Dims& d) {
     int f = 2 * d.G + d.G * d.d + d.d + 1;
     f = (f + 1) & ~1;
     p.kv_stride = f + 2 * d.d;
+    // completion counters first: their place never depends on split counts
     size_t off = 0;
-    p.off_qpart = off; off = align256(off + sizeof(float) * (size_t)BH * p.nsq * d.d);
     p.off_qcnt = off;  off = align256(off + sizeof(unsigned) * (size_t)BH);
-    p.off_kvpart = off; off = align256(off + sizeof(float) * (size_t)d.U() * p.nskv * p.kv_stride);
     p.off_kvcnt = off; off = align256(off + sizeof(unsigned) * (size_t)d.U());
+    p.off_qpart = off; off = align256(off + sizeof(float) * (size_t)BH * p.nsq * d.d);
+    p.off_kvpart = off; off = align256(off + sizeof(float) * (size_t)d.U() * p.nskv * p.kv_stride);
     p.bytes = off;
     return p;
 }
@@ -90,14 +91,15 @@ inline SelectPlan select_plan(const Dims& d, const sa_select_params& sp) {
     SelectPlan p;
     p.g = set_geom(d, sp.sink, sp.local, sp.k_blocks);
     const int nc = p.g.n_cand > 0 ? p.g.n_cand : 1;
-    p.nss = clampi(cdiv(kSmTarget, d.U()), 1, cdiv(nc, 64));
+    // one wave: at most kSmTarget CTAs in all, at least 32 rows per CTA
+    p.nss = clampi(kSmTarget / d.U(), 1, cdiv(nc, 32));
     p.rows_s = cdiv(nc, p.nss);
     p.nss = cdiv(nc, p.rows_s);
     size_t off = 0;
+    p.off_cnt = off;    off = align256(off + sizeof(unsigned) * (size_t)d.U());
     p.off_scores = off; off = align256(off + sizeof(float) * (size_t)d.U() * nc);
     p.off_xkey = off;   off = align256(off + sizeof(unsigned long long) * (size_t)d.U() * nc);
     p.off_flags = off;  off = align256(off + (size_t)d.U() * nc);
-    p.off_cnt = off;    off = align256(off + sizeof(unsigned) * (size_t)d.U());
     p.bytes = off;
     return p;
 }
@@ -110,19 +112,29 @@ struct DecodePlan {
     size_t off_part, off_cnt, bytes;
 };
 
-inline DecodePlan decode_plan(const Dims& d, const sa_select_params& sp) {
+// mode < 0: the largest plan over all modes (workspace sizing); otherwise the
+// launch plan of that mode (only SA_SAMPLE reads the draws).  Counters sit at
+// offset 0 and records after them, so a smaller launch plan fits in the
+// workspace sized by the largest.
+inline DecodePlan decode_plan(const Dims& d, const sa_select_params& sp, int mode = -1) {
     DecodePlan p;
     p.g = set_geom(d, sp.sink, sp.local, sp.k_blocks);
-    p.n_tok_max = p.g.n_i + (sp.sample_cap > 0 ? sp.sample_cap : 0);
+    const bool draws = mode < 0 || mode == SA_SAMPLE;
+    p.n_tok_max = p.g.n_i + (draws && sp.sample_cap > 0 ? sp.sample_cap : 0);
     const int nt = p.n_tok_max > 0 ? p.n_tok_max : 1;
-    p.nsd = clampi(cdiv(kSmTarget, d.U()), 1, cdiv(nt, 32));
-    p.tok_d = cdiv(nt, p.nsd);
-    p.nsd = cdiv(nt, p.tok_d);
+    if (d.bf16) {                  // tensor-core path: one 64-token tile per CTA
+        p.tok_d = 64;
+        p.nsd = cdiv(nt, 64);
+    } else {
+        p.nsd = clampi(cdiv(kSmTarget, d.U()), 1, cdiv(nt, 32));
+        p.tok_d = cdiv(nt, p.nsd);
+        p.nsd = cdiv(nt, p.tok_d);
+    }
     // exact (m,l,acc) + prior (m0,l0,acc0) per head, then ksum, vsum
     p.rec = 2 * d.G * (2 + d.d) + 2 * d.d;
     size_t off = 0;
-    p.off_part = off; off = align256(off + sizeof(float) * (size_t)d.U() * p.nsd * p.rec);
     p.off_cnt = off;  off = align256(off + sizeof(unsigned) * (size_t)d.U());
+    p.off_part = off; off = align256(off + sizeof(float) * (size_t)d.U() * p.nsd * p.rec);
     p.bytes = off;
     return p;
 }
@@ -135,13 +147,18 @@ struct DensePlan {
 
 inline DensePlan dense_plan(const Dims& d) {
     DensePlan p;
-    p.nsdn = clampi(cdiv(2 * kSmTarget, d.U()), 1, d.L / 256 > 0 ? d.L / 256 : 1);
-    p.tok = cdiv(d.nb(), p.nsdn) * 16;
-    p.nsdn = cdiv(d.L, p.tok);
+    if (d.bf16) {                  // tensor-core path: 1024-token chunks, 3-stage pipeline
+        p.tok = d.L < 1024 ? cdiv(d.L, 64) * 64 : 1024;
+        p.nsdn = cdiv(d.L, p.tok);
+    } else {
+        p.nsdn = clampi(cdiv(2 * kSmTarget, d.U()), 1, d.L / 256 > 0 ? d.L / 256 : 1);
+        p.tok = cdiv(d.nb(), p.nsdn) * 16;
+        p.nsdn = cdiv(d.L, p.tok);
+    }
     p.rec = d.G * (2 + d.d);
     size_t off = 0;
-    p.off_part = off; off = align256(off + sizeof(float) * (size_t)d.U() * p.nsdn * p.rec);
     p.off_cnt = off;  off = align256(off + sizeof(unsigned) * (size_t)d.U());
+    p.off_part = off; off = align256(off + sizeof(float) * (size_t)d.U() * p.nsdn * p.rec);
     p.bytes = off;
     return p;
 }

@@ -20,6 +20,7 @@
 namespace sa {
 
 constexpr int kSmemKeys = 4096;     // candidate keys staged in shared memory (16 KB)
+constexpr int kBandCap = 512;       // band members ranked in shared memory
 
 __device__ __forceinline__ uint32_t fkey(float y) {
     const uint32_t b = __float_as_uint(y + 0.0f);   // -0 -> +0
@@ -75,9 +76,17 @@ __device__ void radix_select(KeyFn key, int n, int kk, KT* thr, int* need, unsig
     for (int shift = (int)sizeof(KT) * 8 - 8; shift >= 0; shift -= 8) {
         hist[threadIdx.x] = 0;   // kThreads == 256 bins
         __syncthreads();
-        for (int i = threadIdx.x; i < n; i += kThreads) {
-            const KT kx = key(i);
-            if ((kx & mask) == prefix) atomicAdd(&hist[(int)((kx >> shift) & 0xFF)], 1u);
+        // warp-aggregated: lanes with equal digits add once (scores share their
+        // top bits, so per-lane atomics would serialise on a few bins)
+        for (int i0 = 0; i0 < n; i0 += kThreads) {
+            const int i = i0 + threadIdx.x;
+            int digit = 256;                        // 256 = nothing to count
+            if (i < n) {
+                const KT kx = key(i);
+                if ((kx & mask) == prefix) digit = (int)((kx >> shift) & 0xFF);
+            }
+            const unsigned peers = __match_any_sync(0xffffffffu, digit);
+            if (digit < 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (unsigned)__popc(peers));
         }
         __syncthreads();
         if (threadIdx.x < 32) {
@@ -153,6 +162,10 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
     __shared__ double s_q64[D];
     __shared__ float s_qa[kWarps];
     __shared__ uint32_t s_keys[kSmemKeys];
+    __shared__ int s_nb;
+    __shared__ int s_bidx[kBandCap];
+    __shared__ double s_bx[kBandCap];
+    __shared__ unsigned char s_bsel[kBandCap];
 
     const int u = blockIdx.y, split = blockIdx.x;
     const int b = u / Hkv, g = u - b * Hkv;
@@ -178,26 +191,35 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
         const T* base = blk_mean + ((size_t)u * nb + sg.c_lo) * D + li * EPC;
         const int r0 = split * rows, r1 = min(n, r0 + rows);
         const int gsub = lane / CPR;
-        // warp-uniform loop: a warp step covers 4 x GPW rows (4 per lane group
-        // in flight); rows past the end load nothing and store nothing
-        for (int wr = r0 + warp * 4 * Gm::GPW; wr < r1; wr += 4 * NG) {
-            uint4 w[4];
+        // warp-uniform loop: a warp step covers 4 x GPW rows (4 per lane group);
+        // the next step's rows are loaded before this step's are reduced, so 8
+        // rows per lane group are in flight; rows past the end load nothing
+        auto load4 = [&](int wr, uint4 (&w)[4]) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int r = wr + j * Gm::GPW + gsub;
                 w[j] = (r < r1) ? ld_stream16(base + (size_t)r * D) : make_uint4(0, 0, 0, 0);
             }
+        };
+        int wr = r0 + warp * 4 * Gm::GPW;
+        uint4 cur[4];
+        load4(wr, cur);
+        for (; wr < r1; wr += 4 * NG) {
+            uint4 nxt[4];
+            load4(wr + 4 * NG, nxt);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int r = wr + j * Gm::GPW + gsub;
                 float f[EPC];
-                unpack<T>(w[j], f);
+                unpack<T>(cur[j], f);
                 float x = 0.f;
 #pragma unroll
                 for (int e = 0; e < EPC; ++e) x = fmaf(qb[e], f[e], x);
                 x = group_sum<CPR>(x);
                 if (li == 0 && r < r1) sc[r] = x;
             }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) cur[j] = nxt[j];
         }
     }
     if (!last_cta_of_unit(cnt + u, nss)) return;
@@ -247,34 +269,67 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
         if (band == kk) {
             emit_topk<uint32_t>(k32, n, thr, need, kk, sg.c_lo, out_idx, sw);
         } else {
-            // ambiguous: rescore every candidate of the band in fp64
+            // ambiguous: the exact top-k lies inside the band; rescore the band
+            // members in fp64 and take the top k among them by (x desc, index asc)
             rescored = band;
             for (int i = threadIdx.x; i < D; i += kThreads) {
                 double s = 0.0;
                 for (int h = 0; h < G; ++h) s += (double)to_f32<T>(qg[(size_t)h * D + i]);
                 s_q64[i] = s;
             }
-            __syncthreads();
-            unsigned long long* xk = xkey + (size_t)u * n;
             const T* bm = blk_mean + ((size_t)u * nb + sg.c_lo) * D;
-            for (int i = warp; i < n; i += kWarps) {
-                const bool in_band = keys[i] >= lo_key;       // warp-uniform
-                unsigned long long key = 0ull;
-                if (in_band) {
-                    double x = 0.0;
-                    for (int e = lane; e < D; e += 32) x += s_q64[e] * (double)to_f32<T>(bm[(size_t)i * D + e]);
-                    x = group_sum_f64<32>(x);
-                    key = dkey(x);
+            auto dot64 = [&](int i) -> double {      // warp-collective fp64 score of candidate i
+                double x = 0.0;
+                for (int e = lane; e < D; e += 32) x += s_q64[e] * (double)to_f32<T>(bm[(size_t)i * D + e]);
+                return group_sum_f64<32>(x) + 0.0;  // -0 -> +0
+            };
+            if (band <= kBandCap) {
+                if (threadIdx.x == 0) s_nb = 0;
+                __syncthreads();
+                for (int i = threadIdx.x; i < n; i += kThreads)
+                    if (keys[i] >= lo_key) s_bidx[atomicAdd(&s_nb, 1)] = i;
+                __syncthreads();
+                for (int j = warp; j < band; j += kWarps) {
+                    const double x = dot64(s_bidx[j]);
+                    if (lane == 0) s_bx[j] = x;
                 }
-                if (lane == 0) xk[i] = key;
+                __syncthreads();
+                for (int j = threadIdx.x; j < band; j += kThreads) {
+                    const double xj = s_bx[j];
+                    const int ij = s_bidx[j];
+                    int rank = 0;
+                    for (int m = 0; m < band; ++m) {
+                        const double xm = s_bx[m];
+                        rank += (xm > xj || (xm == xj && s_bidx[m] < ij)) ? 1 : 0;
+                    }
+                    s_bsel[j] = rank < kk ? 1 : 0;
+                }
+                __syncthreads();
+                for (int j = threadIdx.x; j < band; j += kThreads) {
+                    if (!s_bsel[j]) continue;
+                    const int ij = s_bidx[j];
+                    int pos = 0;
+                    for (int m = 0; m < band; ++m) pos += (s_bsel[m] && s_bidx[m] < ij) ? 1 : 0;
+                    if (pos < kk) out_idx[pos] = sg.c_lo + ij;
+                }
+            } else {
+                // very wide band (many near-equal scores): 64-bit keys for every
+                // candidate in the workspace (0 outside the band), radix select
+                __syncthreads();
+                unsigned long long* xk = xkey + (size_t)u * n;
+                for (int i = warp; i < n; i += kWarps) {
+                    unsigned long long key = 0ull;
+                    if (keys[i] >= lo_key) key = dkey(dot64(i));   // warp-uniform branch
+                    if (lane == 0) xk[i] = key;
+                }
+                __threadfence_block();
+                __syncthreads();
+                auto k64 = [&](int i) -> unsigned long long { return xk[i]; };
+                unsigned long long thr64;
+                int need64;
+                radix_select<unsigned long long>(k64, n, kk, &thr64, &need64, hist, &s_digit, &s_rem);
+                emit_topk<unsigned long long>(k64, n, thr64, need64, kk, sg.c_lo, out_idx, sw);
             }
-            __threadfence_block();
-            __syncthreads();
-            auto k64 = [&](int i) -> unsigned long long { return xk[i]; };
-            unsigned long long thr64;
-            int need64;
-            radix_select<unsigned long long>(k64, n, kk, &thr64, &need64, hist, &s_digit, &s_rem);
-            emit_topk<unsigned long long>(k64, n, thr64, need64, kk, sg.c_lo, out_idx, sw);
         }
     } else if (kk > 0) {       // every candidate is chosen
         for (int i = threadIdx.x; i < kk; i += kThreads) out_idx[i] = sg.c_lo + i;

@@ -154,10 +154,12 @@ def test_degenerate_sets(sink, local, kb, dev):
         assert rel_l2(f64(outs[m][0]), o.out(m, qq, idx, pos=pos)) < REL_L2_OUT, m
 
 
-def test_ties_take_lowest_blocks_via_fp64_rescore(dev):
+@pytest.mark.parametrize("L", [2048, 16384])
+def test_ties_take_lowest_blocks_via_fp64_rescore(L, dev):
     # every block of a unit has the same mean: all scores tie, the fp32 band
     # holds every candidate, the fp64 rescore runs and ties go to low indices
-    w = synth.scaled(CASES["bf16_d128_g4"], B=1, Hkv=2, Hq=8, L=2048)
+    # (L=2048: band ranked in shared memory; L=16384: band wider than that)
+    w = synth.scaled(CASES["bf16_d128_g4"], B=1, Hkv=2, Hq=8, L=L)
     d = synth.make_batch(w, device="cpu", steps=1)
     k = d["k"]
     k[0, 0] = k[0, 0, :16].repeat(w.L // 16, 1)           # identical blocks in unit (0, 0)
