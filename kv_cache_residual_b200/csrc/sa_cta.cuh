@@ -78,18 +78,26 @@ __device__ __forceinline__ float combine_splits(const float* recs, int ns, int s
 //  2. per (head, dim): acc = sum_s acc_s 2^(m_s - M), in split order, four
 //     splits' loads in flight at a time.
 // `off` selects the record (0: exact, G*(2+D): prior).  Deterministic.
-template <int G, int D>
+// Record loads: other CTAs' records through L2 (.cg), or this CTA's own
+// records in shared memory (plain generic loads).
+template <bool SH>
+__device__ __forceinline__ float ld_rec(const float* p) {
+    if constexpr (SH) return *p;
+    else return __ldcg(p);
+}
+
+template <int G, int D, bool SH = false>
 __device__ void combine_heads(const float* recs, int ns, int stride, int off, float* s_M, float* s_L) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     for (int h = warp; h < G; h += nw) {
         float M = -INFINITY;
-        for (int s = lane; s < ns; s += 32) M = fmaxf(M, ldcg(recs + (size_t)s * stride + off + h));
+        for (int s = lane; s < ns; s += 32) M = fmaxf(M, ld_rec<SH>(recs + (size_t)s * stride + off + h));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
         float Ls = 0.f;
         for (int s = lane; s < ns; s += 32) {
-            const float m = ldcg(recs + (size_t)s * stride + off + h);
-            const float l = ldcg(recs + (size_t)s * stride + off + G + h);
+            const float m = ld_rec<SH>(recs + (size_t)s * stride + off + h);
+            const float l = ld_rec<SH>(recs + (size_t)s * stride + off + G + h);
             Ls += (m == -INFINITY) ? 0.f : l * ex2(m - M);
         }
 #pragma unroll
@@ -98,7 +106,7 @@ __device__ void combine_heads(const float* recs, int ns, int stride, int off, fl
     }
 }
 
-template <int G, int D>
+template <int G, int D, bool SH = false>
 __device__ __forceinline__ float combine_acc(const float* recs, int ns, int stride, int off, int h, int e, float M) {
     float A = 0.f;
     int s = 0;
@@ -107,16 +115,16 @@ __device__ __forceinline__ float combine_acc(const float* recs, int ns, int stri
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const float* r = recs + (size_t)(s + j) * stride + off;
-            m[j] = ldcg(r + h);
-            a[j] = ldcg(r + 2 * G + h * D + e);
+            m[j] = ld_rec<SH>(r + h);
+            a[j] = ld_rec<SH>(r + 2 * G + h * D + e);
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) A = fmaf(a[j], (m[j] == -INFINITY) ? 0.f : ex2(m[j] - M), A);
     }
     for (; s < ns; ++s) {
         const float* r = recs + (size_t)s * stride + off;
-        const float m = ldcg(r + h);
-        A = fmaf(ldcg(r + 2 * G + h * D + e), (m == -INFINITY) ? 0.f : ex2(m - M), A);
+        const float m = ld_rec<SH>(r + h);
+        A = fmaf(ld_rec<SH>(r + 2 * G + h * D + e), (m == -INFINITY) ? 0.f : ex2(m - M), A);
     }
     return A;
 }

@@ -47,28 +47,29 @@ struct TokenMap {
 // out[b, h, :] for the G heads of the unit.  Record layout per split:
 // exact m[G], l[G], acc[G][D]; prior m0, l0, acc0 (same shape); ksum[D], vsum[D].
 // Shared scratch: s_acc, s_acc0 [G*D], s_ml [4G], s_t [2D], s_hs [G].
-template <typename T, int D, int G, int MODE>
+template <typename T, int D, int G, int MODE, bool SH = false>
 __device__ void decode_epilogue(const float* recs, int nsd, int rec, const T* qg, const sa_stats& st, int u,
                                 int b, int g, int Hq, int nt, float scale, float lambda, float* out,
                                 float* s_acc, float* s_acc0, float* s_ml, float* s_t, float* s_hs) {
     constexpr bool PRIOR = (MODE == SA_RESA);
     constexpr bool SUMS = (MODE == SA_PROXY);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    combine_heads<G, D>(recs, nsd, rec, 0, s_ml, s_ml + G);
-    if constexpr (PRIOR) combine_heads<G, D>(recs, nsd, rec, G * (2 + D), s_ml + 2 * G, s_ml + 3 * G);
+    combine_heads<G, D, SH>(recs, nsd, rec, 0, s_ml, s_ml + G);
+    if constexpr (PRIOR) combine_heads<G, D, SH>(recs, nsd, rec, G * (2 + D), s_ml + 2 * G, s_ml + 3 * G);
     __syncthreads();
     for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
         const int h = idx / D, e = idx - h * D;
-        s_acc[idx] = combine_acc<G, D>(recs, nsd, rec, 0, h, e, s_ml[h]);
-        if constexpr (PRIOR) s_acc0[idx] = combine_acc<G, D>(recs, nsd, rec, G * (2 + D), h, e, s_ml[2 * G + h]);
+        s_acc[idx] = combine_acc<G, D, SH>(recs, nsd, rec, 0, h, e, s_ml[h]);
+        if constexpr (PRIOR)
+            s_acc0[idx] = combine_acc<G, D, SH>(recs, nsd, rec, G * (2 + D), h, e, s_ml[2 * G + h]);
     }
     if constexpr (SUMS) {
         if (nt > 0) {
             for (int c = threadIdx.x; c < D; c += blockDim.x) {
                 float sk = 0.f, sv = 0.f;
                 for (int sp = 0; sp < nsd; ++sp) {
-                    sk += ldcg(recs + (size_t)sp * rec + 2 * G * (2 + D) + c);
-                    sv += ldcg(recs + (size_t)sp * rec + 2 * G * (2 + D) + D + c);
+                    sk += ld_rec<SH>(recs + (size_t)sp * rec + 2 * G * (2 + D) + c);
+                    sv += ld_rec<SH>(recs + (size_t)sp * rec + 2 * G * (2 + D) + D + c);
                 }
                 s_t[c] = (st.sum_k[(size_t)u * D + c] - sk) / (float)nt;       // tail-mean key
                 s_t[D + c] = (st.sum_v[(size_t)u * D + c] - sv) / (float)nt;   // tail-mean value
@@ -346,261 +347,242 @@ k_dense(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ 
 
 
 // ============================================================================
-// bf16 caches: tensor-core tiles (see sa_tc.cuh)
+// bf16 caches: one stream kernel for the sparse gather and the dense pass
 // ============================================================================
+// A CTA owns a chunk of consecutive 64-token tiles of one unit and streams
+// them through a 3-stage cp.async ring of padded shared tiles; its 4 warps
+// take 16 rows each per tile (tensor-core engine, sa_tc.cuh).  A unit that
+// fits one chunk (the usual case at batch 32: one CTA per unit, one wave)
+// finishes in the same CTA; otherwise the chunks' records are combined by
+// the unit's last CTA.
 
 constexpr int kTcTile = 64;        // tokens per shared-memory tile
-constexpr int kTcWarps = 4;        // 16 tokens per warp
+constexpr int kTcWarps = 4;        // 16 tokens per warp per tile
 constexpr int kTcThreads = 32 * kTcWarps;
+constexpr int kStages = 3;
+constexpr int kDenseMode = 4;      // MODE value of the dense pass
 
-// Copies rows pos[0..kTcTile) of K and V (16-byte cp.async; pos < 0 zero-fills)
-// into padded shared tiles.
 template <int D>
-__device__ __forceinline__ void tc_fetch_tile(const __nv_bfloat16* K, const __nv_bfloat16* V, const int* pos,
-                                              uint32_t sk, uint32_t sv) {
-    constexpr int CPR = D / 8;
-    constexpr int P = tc::Pitch<D>::kBytes;
-#pragma unroll 4
-    for (int idx = threadIdx.x; idx < 2 * kTcTile * CPR; idx += kTcThreads) {
-        const int kv = idx / (kTcTile * CPR);
-        const int rem = idx - kv * kTcTile * CPR;
-        const int row = rem / CPR, ch = rem - row * CPR;
-        const uint32_t dst = (kv ? sv : sk) + row * P + ch * 16;
-        const int p = pos[row];
-        if (p >= 0) tc::cp16(dst, (kv ? V : K) + (size_t)p * D + ch * 8);
-        else tc::st_zero16(dst);
-    }
+struct StageLayout {
+    static constexpr int kTileBytes = kTcTile * tc::Pitch<D>::kBytes;   // one of K or V
+    static constexpr int kBytes = 2 * kTileBytes + kTcTile * 8;         // K, V, pos[], lw[]
+};
+
+template <int D, int G, int MODE>
+constexpr size_t stream_smem() {
+    constexpr bool PRIOR = (MODE == SA_RESA);
+    constexpr size_t ring = (size_t)kStages * StageLayout<D>::kBytes;
+    constexpr size_t merge = (size_t)(kTcWarps * G * 4 + (PRIOR ? 2 : 1) * kTcWarps * G * D) * 4;
+    constexpr size_t tail = (size_t)(2 * G * (2 + D) + 2 * D) * 4        // own record
+                            + (size_t)(2 * G * D + 4 * G + 2 * D + G) * 4;  // epilogue scratch
+    constexpr size_t m = merge + tail;
+    return ring > m ? ring : m;
 }
 
 template <int D, int G, int MODE>
 __global__ void __launch_bounds__(kTcThreads)
-k_decode_tc(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+k_stream_tc(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
             const __nv_bfloat16* __restrict__ v, sa_stats st, const int32_t* __restrict__ blk_idx, int kb_stride,
             const int32_t* __restrict__ samp_idx, const int32_t* __restrict__ samp_count, int sample_cap, int Hq,
-            int Hkv, int L, SetGeom sg, int nsd, int rec, float qscale, float scale, float lambda,
+            int Hkv, int L, SetGeom sg, int tpc, int nchunk, int rec, float qscale, float scale, float lambda,
             float* __restrict__ part, unsigned* __restrict__ cnt, float* __restrict__ out) {
+    constexpr bool DENSE = (MODE == kDenseMode);
     constexpr bool PRIOR = (MODE == SA_RESA);
     constexpr bool SUMS = (MODE == SA_PROXY);
     constexpr bool SAMP = (MODE == SA_SAMPLE);
-    constexpr int PE = tc::Pitch<D>::kElems;
+    constexpr int P = tc::Pitch<D>::kBytes;
+    constexpr int TB = StageLayout<D>::kTileBytes;
+    constexpr int SB = StageLayout<D>::kBytes;
     extern __shared__ __align__(16) unsigned char smem[];
-    __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem);
-    __nv_bfloat16* sV = sK + kTcTile * PE;
-    int* s_pos = reinterpret_cast<int*>(sV + kTcTile * PE);
-    float* s_lw = reinterpret_cast<float*>(s_pos + kTcTile);
-    float* s_sum = s_lw + kTcTile;                       // [2D] proxy sums of this tile
-    float* fbuf = reinterpret_cast<float*>(smem);         // reused after the tiles are consumed
 
-    const int u = blockIdx.y, split = blockIdx.x;
+    const int u = blockIdx.y, chunk = blockIdx.x;
     const int b = u / Hkv, g = u - b * Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const size_t ubase = (size_t)u * L * D;
+    const __nv_bfloat16* K = k + ubase;
+    const __nv_bfloat16* V = v + ubase;
     const __nv_bfloat16* qg = q + ((size_t)b * Hq + (size_t)g * G) * D;
 
-    const int nt = sg.n_t;
+    const int nt = DENSE ? 0 : sg.n_t;
     const int bu = (SAMP && nt > 0) ? min(__ldg(samp_count + u), sample_cap) : 0;
     TokenMap tm;
     tm.s_eff = sg.s_eff; tm.kk = sg.kk; tm.n_i = sg.n_i; tm.win0 = L - sg.w_eff;
     tm.blk = blk_idx + (size_t)u * kb_stride;
     tm.samp = samp_idx + (size_t)u * (sample_cap > 0 ? sample_cap : 0);
     tm.lw_samp = bu > 0 ? log2f((float)nt / (float)bu) : 0.f;
-    const int n_tok = sg.n_i + bu;
-    const int t0 = split * kTcTile, t1 = min(n_tok, t0 + kTcTile);
+    const int n_tok = DENSE ? L : sg.n_i + bu;
+    const int n_i = DENSE ? L : sg.n_i;
+    const int ntiles = (n_tok + kTcTile - 1) / kTcTile;
+    const int tile0 = chunk * tpc, tile1 = min(ntiles, tile0 + tpc);
 
-    if (threadIdx.x < kTcTile) {
-        const int t = t0 + threadIdx.x;
-        float lw = 0.f;
-        int p = (t < t1) ? tm.pos(t, lw) : -1;
-        if ((unsigned)p >= (unsigned)L) p = -1;          // outside the cache: masked
-        s_pos[threadIdx.x] = p;
-        s_lw[threadIdx.x] = p >= 0 ? lw : -INFINITY;
-    }
-    __syncthreads();
-    tc_fetch_tile<D>(k + ubase, v + ubase, s_pos, tc::smem_u32(sK), tc::smem_u32(sV));
-    tc::cp_commit();
-
-    tc::WarpAttn<D, G, PRIOR> wa;
-    {
-        const int gh = min((lane >> 2), G - 1);
-        wa.init(qg + (size_t)gh * D, PRIOR ? st.mu_q + ((size_t)b * Hq + g * G + gh) * D : nullptr);
-    }
-    tc::cp_wait<0>();
-    __syncthreads();
-
-    if constexpr (SUMS) {            // sums of K and V over the exact rows of this tile
-        for (int c = threadIdx.x; c < 2 * D; c += kTcThreads) {
-            const __nv_bfloat16* src = (c < D ? sK : sV) + (c < D ? c : c - D);
-            float acc = 0.f;
-            for (int r = 0; r < kTcTile; ++r)
-                if (t0 + r < sg.n_i && s_pos[r] >= 0) acc += __bfloat162float(src[r * PE]);
-            s_sum[c] = acc;
-        }
-    }
-    const int r0 = warp * 16;
-    if (t0 + r0 < t1) {
-        const int tq = lane & 3;
-        const int rows[4] = {r0 + 2 * tq, r0 + 2 * tq + 1, r0 + 8 + 2 * tq, r0 + 9 + 2 * tq};
-        float xadd[4];
-        bool in_i[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            xadd[j] = s_lw[rows[j]];
-            in_i[j] = (t0 + rows[j] < sg.n_i) && s_pos[rows[j]] >= 0;
-        }
-        wa.step16(tc::smem_u32(sK), tc::smem_u32(sV), r0, xadd, in_i, qscale);
-    }
-    float sum_keep[2];
-    if constexpr (SUMS) {
-        sum_keep[0] = threadIdx.x < 2 * D ? s_sum[threadIdx.x] : 0.f;
-        sum_keep[1] = threadIdx.x + kTcThreads < 2 * D ? s_sum[threadIdx.x + kTcThreads] : 0.f;
-    }
-    __syncthreads();                   // tiles consumed: reuse the region
-    float* ml = fbuf;                                   // [W][G][4]
-    float* acc = ml + kTcWarps * G * 4;                 // [W][G][D]
-    float* acc0 = acc + kTcWarps * G * D;               // [W][G][D]
-    wa.store(ml, acc, acc0);
-    __syncthreads();
-    float* r = part + ((size_t)u * nsd + split) * rec;
-    tc::merge_warps<D, G, PRIOR>(ml, acc, acc0, kTcWarps, r);
-    if constexpr (SUMS) {
-        if (threadIdx.x < 2 * D) r[2 * G * (2 + D) + threadIdx.x] = sum_keep[0];
-        if (threadIdx.x + kTcThreads < 2 * D) r[2 * G * (2 + D) + threadIdx.x + kTcThreads] = sum_keep[1];
-    }
-    if (!last_cta_of_unit(cnt + u, nsd)) return;
-    float* s_acc = fbuf;
-    float* s_acc0 = s_acc + G * D;
-    float* s_ml = s_acc0 + G * D;
-    float* s_t = s_ml + 4 * G;
-    float* s_hs = s_t + 2 * D;
-    decode_epilogue<__nv_bfloat16, D, G, MODE>(part + (size_t)u * nsd * rec, nsd, rec, qg, st, u, b, g, Hq, nt,
-                                               scale, lambda, out, s_acc, s_acc0, s_ml, s_t, s_hs);
-    reset_counter(cnt + u);
-}
-
-constexpr int kDenseStages = 3;
-
-template <int D, int G>
-__global__ void __launch_bounds__(kTcThreads)
-k_dense_tc(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-           const __nv_bfloat16* __restrict__ v, int Hq, int Hkv, int L, int tok, int nsdn, int rec, float qscale,
-           float* __restrict__ part, unsigned* __restrict__ cnt, float* __restrict__ out) {
-    constexpr int PE = tc::Pitch<D>::kElems;
-    constexpr int STAGE = 2 * kTcTile * PE;             // bf16 elements per stage (K and V)
-    extern __shared__ __align__(16) unsigned char smem[];
-    __nv_bfloat16* tiles = reinterpret_cast<__nv_bfloat16*>(smem);
-    int* s_pos = reinterpret_cast<int*>(tiles + kDenseStages * STAGE);   // [stages][tile]
-    float* fbuf = reinterpret_cast<float*>(smem);
-
-    const int u = blockIdx.y, split = blockIdx.x;
-    const int b = u / Hkv, g = u - b * Hkv;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const size_t ubase = (size_t)u * L * D;
-    const __nv_bfloat16* qg = q + ((size_t)b * Hq + (size_t)g * G) * D;
-    const int t0 = split * tok, t1 = min(L, t0 + tok);
-    const int ntiles = (t1 - t0 + kTcTile - 1) / kTcTile;
-
+    // positions of tile i into stage arrays, then its K/V rows (cp.async)
     auto issue = [&](int i) {
-        if (i < ntiles) {
-            const int st = i % kDenseStages;
-            int* pos = s_pos + st * kTcTile;
-            // positions of the tile (the previous tile on this stage is consumed)
+        if (i < tile1) {
+            unsigned char* sb = smem + (size_t)(i % kStages) * SB;
+            int* pos = reinterpret_cast<int*>(sb + 2 * TB);
+            float* lw = reinterpret_cast<float*>(pos + kTcTile);
             if (threadIdx.x < kTcTile) {
-                const int t = t0 + i * kTcTile + threadIdx.x;
-                pos[threadIdx.x] = t < t1 ? t : -1;
+                const int t = i * kTcTile + threadIdx.x;
+                float w = 0.f;
+                int p = -1;
+                if (t < n_tok) p = DENSE ? t : tm.pos(t, w);
+                if ((unsigned)p >= (unsigned)L) p = -1;          // outside the cache: masked
+                pos[threadIdx.x] = p;
+                lw[threadIdx.x] = p >= 0 ? w : -INFINITY;
             }
             __syncthreads();
-            const uint32_t base = tc::smem_u32(tiles + st * STAGE);
-            tc_fetch_tile<D>(k + ubase, v + ubase, pos, base, base + kTcTile * tc::Pitch<D>::kBytes);
+            constexpr int CPR = D / 8;
+            const uint32_t sk = tc::smem_u32(sb), sv = sk + TB;
+#pragma unroll 4
+            for (int idx = threadIdx.x; idx < 2 * kTcTile * CPR; idx += kTcThreads) {
+                const int kv = idx / (kTcTile * CPR);
+                const int rem = idx - kv * kTcTile * CPR;
+                const int row = rem / CPR, ch = rem - row * CPR;
+                const uint32_t dst = (kv ? sv : sk) + row * P + ch * 16;
+                const int p = pos[row];
+                if (p >= 0) tc::cp16(dst, (kv ? V : K) + (size_t)p * D + ch * 8);
+                else tc::st_zero16(dst);
+            }
         }
         tc::cp_commit();
     };
 
-    tc::WarpAttn<D, G, false> wa;
-    wa.init(qg + (size_t)min(lane >> 2, G - 1) * D, nullptr);
+    tc::WarpAttn<D, G, PRIOR> wa;
+    {
+        const int gh = min(lane >> 2, G - 1);
+        wa.init(qg + (size_t)gh * D, PRIOR ? st.mu_q + ((size_t)b * Hq + g * G + gh) * D : nullptr);
+    }
+    float ks[2] = {0.f, 0.f};      // SUMS: this thread's column pair of K (c < D/2 ... ) and V
 #pragma unroll
-    for (int i = 0; i < kDenseStages - 1; ++i) issue(i);
-    for (int i = 0; i < ntiles; ++i) {
-        issue(i + kDenseStages - 1);
-        tc::cp_wait<kDenseStages - 1>();
+    for (int i = 0; i < kStages - 1; ++i) issue(tile0 + i);
+    for (int i = tile0; i < tile1; ++i) {
+        issue(i + kStages - 1);
+        tc::cp_wait<kStages - 1>();
         __syncthreads();
-        const int st = i % kDenseStages;
+        unsigned char* sb = smem + (size_t)(i % kStages) * SB;
+        const int* pos = reinterpret_cast<const int*>(sb + 2 * TB);
+        const float* lw = reinterpret_cast<const float*>(pos + kTcTile);
+        const int base = i * kTcTile;
+        if constexpr (SUMS) {
+            // column pair (2c, 2c+1) of K (c < D/2) or of V (c >= D/2) over the exact rows
+            const int c = threadIdx.x;
+            if (c < D) {
+                const unsigned char* src = sb + (c < D / 2 ? 0 : TB) + (c % (D / 2)) * 4;
+                for (int r = 0; r < kTcTile; ++r) {
+                    if (base + r < n_i && pos[r] >= 0) {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(src + r * P));
+                        ks[0] += f.x;
+                        ks[1] += f.y;
+                    }
+                }
+            }
+        }
         const int r0 = warp * 16;
-        const int rem = t1 - (t0 + i * kTcTile);
-        if (r0 < rem) {
+        if (base + r0 < n_tok) {
             const int tq = lane & 3;
             const int rows[4] = {r0 + 2 * tq, r0 + 2 * tq + 1, r0 + 8 + 2 * tq, r0 + 9 + 2 * tq};
             float xadd[4];
             bool in_i[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) { xadd[j] = rows[j] < rem ? 0.f : -INFINITY; in_i[j] = false; }
-            const uint32_t base = tc::smem_u32(tiles + st * STAGE);
-            wa.step16(base, base + kTcTile * tc::Pitch<D>::kBytes, r0, xadd, in_i, qscale);
+            for (int j = 0; j < 4; ++j) {
+                xadd[j] = lw[rows[j]];
+                in_i[j] = PRIOR && (base + rows[j] < n_i) && pos[rows[j]] >= 0;
+            }
+            const uint32_t sk = tc::smem_u32(sb);
+            wa.step16(sk, sk + TB, r0, xadd, in_i, qscale);
         }
-        __syncthreads();              // stage st is refilled by the next issue()
+        __syncthreads();              // this stage is refilled by a later issue()
     }
     tc::cp_wait<0>();
     __syncthreads();
-    float* ml = fbuf;
-    float* acc = ml + kTcWarps * G * 4;
-    wa.store(ml, acc, nullptr);
+
+    // ---- this chunk's record --------------------------------------------------------
+    float* fb = reinterpret_cast<float*>(smem);
+    float* ml = fb;                                     // [W][G][4]
+    float* acc = ml + kTcWarps * G * 4;                 // [W][G][D]
+    float* acc0 = acc + kTcWarps * G * D;               // [W][G][D] (PRIOR)
+    float* own = acc + (PRIOR ? 2 : 1) * kTcWarps * G * D;   // own record when the unit is one chunk
+    float* scratch = own + 2 * G * (2 + D) + 2 * D;
+    wa.store(ml, acc, acc0);
     __syncthreads();
-    float* r = part + ((size_t)u * nsdn + split) * rec;
-    tc::merge_warps<D, G, false>(ml, acc, nullptr, kTcWarps, r);
-    if (!last_cta_of_unit(cnt + u, nsdn)) return;
-    const float* recs = part + (size_t)u * nsdn * rec;
-    float* s_M = fbuf;
-    float* s_L = fbuf + G;
-    __syncthreads();
-    combine_heads<G, D>(recs, nsdn, rec, 0, s_M, s_L);
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < G * D; idx += kTcThreads) {
-        const int h = idx / D, e = idx - h * D;
-        out[((size_t)b * Hq + g * G + h) * D + e] = combine_acc<G, D>(recs, nsdn, rec, 0, h, e, s_M[h]) / s_L[h];
+    const bool single = (nchunk == 1);
+    float* r = single ? own : part + ((size_t)u * nchunk + chunk) * rec;
+    tc::merge_warps<D, G, PRIOR>(ml, acc, acc0, kTcWarps, r);
+    if constexpr (SUMS) {
+        if (threadIdx.x < D) {
+            const int c = threadIdx.x;
+            const int col = 2 * (c % (D / 2)) + (c < D / 2 ? 0 : D);
+            r[2 * G * (2 + D) + col] = ks[0];
+            r[2 * G * (2 + D) + col + 1] = ks[1];
+        }
     }
-    reset_counter(cnt + u);
-}
+    if (single) {
+        __syncthreads();
+    } else if (!last_cta_of_unit(cnt + u, nchunk)) {
+        return;
+    }
 
-template <int D, int G>
-size_t decode_tc_smem() {
-    constexpr int PE = tc::Pitch<D>::kElems;
-    size_t tiles = 2 * kTcTile * PE * sizeof(__nv_bfloat16) + kTcTile * 8 + 2 * D * 4;
-    size_t merge = (kTcWarps * G * 4 + 2 * kTcWarps * G * D) * sizeof(float);
-    size_t epi = (2 * G * D + 4 * G + 2 * D + G) * sizeof(float);
-    size_t m = merge > epi ? merge : epi;
-    return tiles > m ? tiles : m;
-}
-
-template <int D, int G>
-size_t dense_tc_smem() {
-    constexpr int PE = tc::Pitch<D>::kElems;
-    size_t tiles = kDenseStages * (2 * kTcTile * PE * sizeof(__nv_bfloat16) + kTcTile * 4);
-    size_t merge = (kTcWarps * G * 4 + kTcWarps * G * D) * sizeof(float);
-    return tiles > merge ? tiles : merge;
+    // ---- the unit's output --------------------------------------------------------------
+    float* s_acc = scratch;
+    float* s_acc0 = s_acc + G * D;
+    float* s_ml = s_acc0 + G * D;
+    float* s_t = s_ml + 4 * G;
+    float* s_hs = s_t + 2 * D;
+    const float* recs = single ? own : part + (size_t)u * nchunk * rec;
+    if constexpr (DENSE) {
+        if (single) combine_heads<G, D, true>(recs, 1, rec, 0, s_ml, s_ml + G);
+        else combine_heads<G, D, false>(recs, nchunk, rec, 0, s_ml, s_ml + G);
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < G * D; idx += kTcThreads) {
+            const int h = idx / D, e = idx - h * D;
+            const float A = single ? combine_acc<G, D, true>(recs, 1, rec, 0, h, e, s_ml[h])
+                                   : combine_acc<G, D, false>(recs, nchunk, rec, 0, h, e, s_ml[h]);
+            out[((size_t)b * Hq + g * G + h) * D + e] = A / s_ml[G + h];
+        }
+    } else {
+        constexpr int EM = DENSE ? SA_DROP : MODE;
+        if (single)
+            decode_epilogue<__nv_bfloat16, D, G, EM, true>(recs, 1, rec, qg, st, u, b, g, Hq, nt, scale, lambda,
+                                                           out, s_acc, s_acc0, s_ml, s_t, s_hs);
+        else
+            decode_epilogue<__nv_bfloat16, D, G, EM, false>(recs, nchunk, rec, qg, st, u, b, g, Hq, nt, scale,
+                                                            lambda, out, s_acc, s_acc0, s_ml, s_t, s_hs);
+    }
+    if (!single) reset_counter(cnt + u);
 }
 
 // ---- dispatch ----------------------------------------------------------------
 
+template <int D, int G, int MODE>
+static cudaError_t stream_launch(const Dims& d, dim3 grid, const void* q, const void* k, const void* v,
+                                 const sa_stats& st, const sa_selection& sel, const sa_select_params& sp,
+                                 const SetGeom& sg, int tpc, int nchunk, int rec, float scale, float lambda,
+                                 char* part, char* cnt, float* out, cudaStream_t s) {
+    constexpr size_t sm = stream_smem<D, G, MODE>();
+    cudaError_t e = cudaFuncSetAttribute(k_stream_tc<D, G, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    k_stream_tc<D, G, MODE><<<grid, kTcThreads, sm, s>>>(
+        reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k),
+        reinterpret_cast<const __nv_bfloat16*>(v), st, sel.blk_idx, sp.k_blocks, sel.samp_idx, sel.samp_count,
+        sp.sample_cap, d.Hq, d.Hkv, d.L, sg, tpc, nchunk, rec, scale * kLog2e, scale, lambda,
+        reinterpret_cast<float*>(part), reinterpret_cast<unsigned*>(cnt), out);
+    return cudaGetLastError();
+}
+
 template <typename T, int D, int G, int MODE>
 static cudaError_t decode_m(const Dims& d, const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
     if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-        const size_t sm = decode_tc_smem<D, G>();
-        if (sm > 48 * 1024) {
-            cudaError_t e = cudaFuncSetAttribute(k_decode_tc<D, G, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-            if (e != cudaSuccess) return e;
-        }
-        k_decode_tc<D, G, MODE><<<dim3(p.nsd, d.U()), kTcThreads, sm, s>>>(
-            reinterpret_cast<const T*>(a.q), reinterpret_cast<const T*>(a.k), reinterpret_cast<const T*>(a.v),
-            a.st, a.sel.blk_idx, a.sp.k_blocks, a.sel.samp_idx, a.sel.samp_count, a.sp.sample_cap,
-            d.Hq, d.Hkv, d.L, p.g, p.nsd, p.rec, a.scale * kLog2e, a.scale, a.dp.lambda,
-            reinterpret_cast<float*>(a.ws + p.off_part), reinterpret_cast<unsigned*>(a.ws + p.off_cnt), a.out);
+        return stream_launch<D, G, MODE>(d, dim3(p.nsd, d.U()), a.q, a.k, a.v, a.st, a.sel, a.sp, p.g, p.tok_d,
+                                         p.nsd, p.rec, a.scale, a.dp.lambda, a.ws + p.off_part, a.ws + p.off_cnt,
+                                         a.out, s);
     } else {
         k_decode<T, D, G, MODE><<<dim3(p.nsd, d.U()), kThreads, 0, s>>>(
             reinterpret_cast<const T*>(a.q), reinterpret_cast<const T*>(a.k), reinterpret_cast<const T*>(a.v),
             a.st, a.sel.blk_idx, a.sp.k_blocks, a.sel.samp_idx, a.sel.samp_count, a.sp.sample_cap,
             d.Hq, d.Hkv, d.L, p.g, p.tok_d, p.nsd, p.rec, a.scale * kLog2e, a.scale, a.dp.lambda,
             reinterpret_cast<float*>(a.ws + p.off_part), reinterpret_cast<unsigned*>(a.ws + p.off_cnt), a.out);
+        return cudaGetLastError();
     }
-    return cudaGetLastError();
 }
 
 template <typename T, int D, int G>
@@ -633,20 +615,20 @@ cudaError_t launch_decode(const Dims& d, const DecodePlan& p, const DecodeArgs& 
 template <typename T, int D, int G>
 static cudaError_t dense_t(const Dims& d, const DensePlan& p, const DenseArgs& a, cudaStream_t s) {
     if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-        const size_t sm = dense_tc_smem<D, G>();
-        cudaError_t e = cudaFuncSetAttribute(k_dense_tc<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        if (e != cudaSuccess) return e;
-        k_dense_tc<D, G><<<dim3(p.nsdn, d.U()), kTcThreads, sm, s>>>(
-            reinterpret_cast<const T*>(a.q), reinterpret_cast<const T*>(a.k), reinterpret_cast<const T*>(a.v),
-            d.Hq, d.Hkv, d.L, p.tok, p.nsdn, p.rec, a.scale * kLog2e,
-            reinterpret_cast<float*>(a.ws + p.off_part), reinterpret_cast<unsigned*>(a.ws + p.off_cnt), a.out);
+        SetGeom sg{};
+        sa_stats st{};
+        sa_selection sel{};
+        sa_select_params sp{};
+        return stream_launch<D, G, kDenseMode>(d, dim3(p.nsdn, d.U()), a.q, a.k, a.v, st, sel, sp, sg,
+                                               p.tok / kTcTile, p.nsdn, p.rec, a.scale, 1.f, a.ws + p.off_part,
+                                               a.ws + p.off_cnt, a.out, s);
     } else {
         k_dense<T, D, G><<<dim3(p.nsdn, d.U()), kThreads, 0, s>>>(
             reinterpret_cast<const T*>(a.q), reinterpret_cast<const T*>(a.k), reinterpret_cast<const T*>(a.v),
             d.Hq, d.Hkv, d.L, p.tok, p.nsdn, p.rec, a.scale * kLog2e,
             reinterpret_cast<float*>(a.ws + p.off_part), reinterpret_cast<unsigned*>(a.ws + p.off_cnt), a.out);
+        return cudaGetLastError();
     }
-    return cudaGetLastError();
 }
 
 template <typename T, int D>

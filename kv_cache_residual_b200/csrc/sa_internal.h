@@ -12,6 +12,7 @@
 namespace sa {
 
 constexpr int kSmTarget = 148 * 4;   // CTAs to aim for: 4 per SM on B200
+constexpr int kStreamSlots = 148 * 2; // resident CTAs of the bf16 stream kernel (2 per SM)
 
 struct Dims {
     int B, Hq, Hkv, G, d, L;
@@ -107,7 +108,7 @@ inline SelectPlan select_plan(const Dims& d, const sa_select_params& sp) {
 struct DecodePlan {
     SetGeom g;
     int n_tok_max;               // |I| + sample capacity
-    int nsd, tok_d;              // splits per unit, tokens per split
+    int nsd, tok_d;              // splits per unit, tokens per split (bf16: tiles per chunk)
     int rec;                     // floats per partial record
     size_t off_part, off_cnt, bytes;
 };
@@ -122,9 +123,11 @@ inline DecodePlan decode_plan(const Dims& d, const sa_select_params& sp, int mod
     const bool draws = mode < 0 || mode == SA_SAMPLE;
     p.n_tok_max = p.g.n_i + (draws && sp.sample_cap > 0 ? sp.sample_cap : 0);
     const int nt = p.n_tok_max > 0 ? p.n_tok_max : 1;
-    if (d.bf16) {                  // tensor-core path: one 64-token tile per CTA
-        p.tok_d = 64;
-        p.nsd = cdiv(nt, 64);
+    if (d.bf16) {                  // stream kernel: chunks of 64-token tiles, ~one wave
+        const int ntiles = cdiv(nt, 64);
+        p.nsd = clampi(kStreamSlots / d.U(), 1, ntiles);
+        p.tok_d = cdiv(ntiles, p.nsd);          // tiles per chunk
+        p.nsd = cdiv(ntiles, p.tok_d);
     } else {
         p.nsd = clampi(cdiv(kSmTarget, d.U()), 1, cdiv(nt, 32));
         p.tok_d = cdiv(nt, p.nsd);
@@ -147,8 +150,10 @@ struct DensePlan {
 
 inline DensePlan dense_plan(const Dims& d) {
     DensePlan p;
-    if (d.bf16) {                  // tensor-core path: 1024-token chunks, 3-stage pipeline
-        p.tok = d.L < 1024 ? cdiv(d.L, 64) * 64 : 1024;
+    if (d.bf16) {                  // stream kernel: chunks of 64-token tiles, ~one wave
+        const int ntiles = cdiv(d.L, 64);
+        p.nsdn = clampi(kStreamSlots / d.U(), 1, ntiles);
+        p.tok = cdiv(ntiles, p.nsdn) * 64;
         p.nsdn = cdiv(d.L, p.tok);
     } else {
         p.nsdn = clampi(cdiv(2 * kSmTarget, d.U()), 1, d.L / 256 > 0 ? d.L / 256 : 1);
