@@ -285,8 +285,7 @@ def main(argv=None):
 
     def step(t, mode):
         sp = sps[t % nq]
-        sa.select(Q[t % nq], stats, sp, selection=sel)
-        sa.decode(Q[t % nq], K, V, stats, sel, sp, mode=mode, out=out)
+        sa.step(Q[t % nq], K, V, stats, sp, mode=mode, selection=sel, out=out)
 
     def timed(n, fn, n_events=3):
         """Runs fn(t, ev) n times with an L2 flush before each; returns per-step
@@ -298,7 +297,19 @@ def main(argv=None):
         torch.cuda.synchronize()
         return [[evs[t][i].elapsed_time(evs[t][i + 1]) for i in range(n_events - 1)] for t in range(n)]
 
-    def sparse_step(mode):
+    def sparse_step(mode, sps_m=None, sel_m=None):
+        """One step through sa_step (selection + decode, overlapped)."""
+        sps_m = sps if sps_m is None else sps_m
+        sel_m = sel if sel_m is None else sel_m
+
+        def fn(t, ev):
+            ev[0].record(stream)
+            sa.step(Q[t % nq], K, V, stats, sps_m[t % nq], mode=mode, selection=sel_m, out=out)
+            ev[1].record(stream)
+        return fn
+
+    def split_step(mode):
+        """Selection and decode as two calls, timed separately (kernel breakdown)."""
         def fn(t, ev):
             sp = sps[t % nq]
             ev[0].record(stream)
@@ -318,14 +329,16 @@ def main(argv=None):
     barrier()
     torch.cuda.synchronize()
     clocks.start()
-    per = timed(args.steps, sparse_step(args.mode))
+    per = timed(args.steps, sparse_step(args.mode), 2)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
-    sel_ms = [p[0] for p in per]
-    dec_ms = [p[1] for p in per]
-    total_ms = sum(a + b for a, b in per)
+    total_ms = sum(p[0] for p in per)
     total_ms = reduce_max(total_ms, dev)
+    # kernel breakdown: the same step as two calls, each bracketed by events
+    brk = timed(min(args.steps, 500), split_step(args.mode))
+    sel_ms = [p[0] for p in brk]
+    dec_ms = [p[1] for p in brk]
     ms_per_step = total_ms / args.steps
     value = ws * w.B * args.steps / (total_ms / 1e3)
 
@@ -347,25 +360,16 @@ def main(argv=None):
     # other modes (same selection kernel)
     mode_vals = {}
     for m in ("drop", "resa", "proxy", "sample"):
+        sps_m, sel_m = None, None
         if m == "sample" and bdraw == 0:
             sps_m = [sa.SelectParams(sink=w.sink, local=w.local, k_blocks=kb, sample_b=args.sample_b,
                                      sample_cap=args.sample_b, seed=2024, step=t) for t in range(nq)]
             sel_m = sa.select(Q[0], stats, sps_m[0])
-
-            def fn(t, ev, sps_m=sps_m, sel_m=sel_m):
-                sp = sps_m[t % nq]
-                ev[0].record(stream)
-                sa.select(Q[t % nq], stats, sp, selection=sel_m)
-                ev[1].record(stream)
-                sa.decode(Q[t % nq], K, V, stats, sel_m, sp, mode="sample", out=out)
-                ev[2].record(stream)
-        else:
-            fn = sparse_step(m)
-        timed(3, fn)
-        pm = timed(args.mode_steps, fn)
-        ms = sum(a + b for a, b in pm) / len(pm)
-        mode_vals[m] = {"tokens_per_s": w.B / (ms * 1e-3), "ms_per_step": ms,
-                        "decode_us": 1e3 * statistics.mean(p[1] for p in pm)}
+        fn = sparse_step(m, sps_m, sel_m)
+        timed(3, fn, 2)
+        pm = timed(args.mode_steps, fn, 2)
+        ms = sum(p[0] for p in pm) / len(pm)
+        mode_vals[m] = {"tokens_per_s": w.B / (ms * 1e-3), "ms_per_step": ms}
 
     # dense flash-decode reference (in-build)
     def dense_fn(t, ev):
@@ -391,8 +395,7 @@ def main(argv=None):
             sp = sps[t % nq]
             ev[0].record(stream)
             q_dev.copy_(q_host[t % nq], non_blocking=True)
-            sa.select(q_dev, stats, sp, selection=sel)
-            sa.decode(q_dev, K, V, stats, sel, sp, mode=args.mode, out=out)
+            sa.step(q_dev, K, V, stats, sp, mode=args.mode, selection=sel, out=out)
             o_host.copy_(out, non_blocking=True)
             ev[1].record(stream)
         timed(3, e2e_fn, 2)
@@ -429,6 +432,8 @@ def main(argv=None):
             "step_roofline": {"achieved": step_gbs, "frac": step_gbs / peak, "bytes_per_step": sel_b + dec_b,
                               "decode_gbs": dec_gbs, "decode_us": 1e3 * dec_avg, "decode_bytes": dec_b},
             "dense": dense, "speedup_vs_dense": dense_ms / ms_per_step, "modes": mode_vals,
+            "kernels_us": {"k_select": 1e3 * sel_avg, "k_decode": 1e3 * dec_avg,
+                           "separate_sum": 1e3 * (sel_avg + dec_avg), "step_overlapped": 1e3 * ms_per_step},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps, "clocks": clk,
         }
         print(json.dumps(line))

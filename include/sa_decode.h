@@ -78,7 +78,8 @@ typedef enum {
     SA_OP_PREFILL = 0,   /* sa_prefill_stats */
     SA_OP_SELECT = 1,    /* sa_select        */
     SA_OP_DECODE = 2,    /* sa_decode        */
-    SA_OP_DENSE = 3      /* sa_dense_decode  */
+    SA_OP_DENSE = 3,     /* sa_dense_decode  */
+    SA_OP_STEP = 4       /* sa_step          */
 } sa_op;
 
 /* Supported: d in {64, 128}; Hq % Hkv == 0 with G = Hq/Hkv in {1,2,4,8};
@@ -193,6 +194,18 @@ SA_API sa_status sa_decode(const sa_shape* shape, const sa_decode_params* dparam
                     const sa_select_params* sparams, const void* q, const void* k,
                     const void* v, const sa_stats* stats, const sa_selection* sel,
                     float* out, void* ws, size_t ws_bytes, void* stream);
+
+/* One whole decode step: sa_select then sa_decode on the same stream, the
+ * decode launched as a programmatic dependent of the selection, so that its
+ * CTAs stream the sink and window rows (which do not depend on the selection)
+ * while the selection finishes, and wait for it (griddepcontrol.wait) before
+ * reading the chosen blocks and draws.  Same arguments, layouts and results
+ * as the two calls in sequence; scale = dparams->scale; the workspace is
+ * sa_workspace_size(..., SA_OP_STEP) bytes (selection part first). */
+SA_API sa_status sa_step(const sa_shape* shape, const sa_decode_params* dparams,
+                         const sa_select_params* sparams, const void* q, const void* k, const void* v,
+                         const sa_stats* stats, const sa_selection* sel, float* out, void* ws,
+                         size_t ws_bytes, void* stream);
 
 /* Dense flash-decode over all L tokens (the in-build speed reference, not
  * part of the method): out [B, Hq, d] f32 = softmax(s q K^T) V. */

@@ -25,7 +25,7 @@ LIB_PATH = os.path.join(_HERE, "libsa_b200.so")
 SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_CUDA = range(5)
 SA_F32, SA_BF16 = 0, 1
 MODES = {"drop": 0, "resa": 1, "proxy": 2, "sample": 3}
-OP_PREFILL, OP_SELECT, OP_DECODE, OP_DENSE = range(4)
+OP_PREFILL, OP_SELECT, OP_DECODE, OP_DENSE, OP_STEP = range(5)
 
 
 class SAError(RuntimeError):
@@ -60,7 +60,7 @@ class sa_decode_params(ctypes.Structure):
 
 
 EXPORTS = ("sa_workspace_size", "sa_prefill_stats", "sa_block_summaries", "sa_select", "sa_decode",
-           "sa_dense_decode", "sa_status_string")
+           "sa_step", "sa_dense_decode", "sa_status_string")
 
 _LIB = None
 
@@ -81,10 +81,11 @@ def _lib():
         lib.sa_block_summaries.argtypes = [sh, P, I, I, P, P, P]
         lib.sa_select.argtypes = [sh, sp, P, st, P, P, sel, F, P, S, P]
         lib.sa_decode.argtypes = [sh, dp, sp, P, P, P, st, sel, P, P, S, P]
+        lib.sa_step.argtypes = [sh, dp, sp, P, P, P, st, sel, P, P, S, P]
         lib.sa_dense_decode.argtypes = [sh, P, P, P, P, F, P, S, P]
         lib.sa_status_string.argtypes = [I]
         lib.sa_status_string.restype = ctypes.c_char_p
-        for f in ("sa_prefill_stats", "sa_block_summaries", "sa_select", "sa_decode", "sa_dense_decode"):
+        for f in ("sa_prefill_stats", "sa_block_summaries", "sa_select", "sa_decode", "sa_step", "sa_dense_decode"):
             getattr(lib, f).restype = I
         _LIB = lib
     return _LIB
@@ -238,6 +239,26 @@ def decode(q, k, v, stats, selection, params, mode="resa", lam=1.0, scale=0.0, o
                             ctypes.byref(st), ctypes.byref(sel), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
            "sa_decode")
     return out
+
+
+def step(q, k, v, stats, params, mode="resa", lam=1.0, scale=0.0, selection=None, out=None, stream=None):
+    """Selection then decode in one call (the decode overlaps the end of the
+    selection through programmatic dependent launch).  Returns (out, selection)."""
+    B, Hq, d = q.shape
+    shape = make_shape(k, Hq)
+    cp = params.c()
+    dp = sa_decode_params(MODES[mode], float(lam), float(scale))
+    if selection is None:
+        selection = Selection(B, shape.Hkv, params.k_blocks, cp.sample_cap, q.device)
+    if out is None:
+        out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
+    ws = workspace(shape, cp, OP_STEP, q.device)
+    st = stats.c()
+    sel = selection.c()
+    _check(_lib().sa_step(ctypes.byref(shape), ctypes.byref(dp), ctypes.byref(cp), _ptr(q), _ptr(k), _ptr(v),
+                          ctypes.byref(st), ctypes.byref(sel), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+           "sa_step")
+    return out, selection
 
 
 def dense_decode(q, k, v, scale=0.0, out=None, stream=None):

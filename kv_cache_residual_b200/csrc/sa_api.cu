@@ -84,6 +84,9 @@ size_t sa_workspace_size(const sa_shape* shape, const sa_select_params* params, 
         case SA_OP_DECODE:
             if (check_select_params(params) != SA_OK) return 0;
             return decode_plan(d, *params).bytes;
+        case SA_OP_STEP:
+            if (check_select_params(params) != SA_OK) return 0;
+            return select_plan(d, *params).bytes + decode_plan(d, *params).bytes;
     }
     return 0;
 }
@@ -117,34 +120,32 @@ sa_status sa_block_summaries(const sa_shape* shape, const void* k, int blk_begin
                : SA_ERR_CUDA;
 }
 
-sa_status sa_select(const sa_shape* shape, const sa_select_params* params, const void* q,
-                    const sa_stats* stats, const void* k, const void* v, const sa_selection* out,
-                    float scale, void* ws, size_t ws_bytes, void* stream) {
-    NvtxRange r("sa_select");
-    Dims d;
-    sa_status e = check_shape(shape, &d);
+}  // extern "C"
+
+namespace {
+
+sa_status prep_select(const sa_shape* shape, const sa_select_params* params, const void* q, const sa_stats* stats,
+                      const void* k, const void* v, const sa_selection* out, float scale, Dims* d,
+                      SelectPlan* p, SelectArgs* a) {
+    sa_status e = check_shape(shape, d);
     if (e != SA_OK) return e;
     e = check_select_params(params);
     if (e != SA_OK) return e;
     if (!aligned16(q) || !check_stats(stats, false) || out == nullptr || scale < 0.f) return SA_ERR_INVALID_ARG;
-    const SelectPlan p = select_plan(d, *params);
-    if (p.g.kk > 0 && !aligned4(out->blk_idx)) return SA_ERR_INVALID_ARG;
+    *p = select_plan(*d, *params);
+    if (p->g.kk > 0 && !aligned4(out->blk_idx)) return SA_ERR_INVALID_ARG;
     if (params->k_blocks > 0 && out->blk_idx == nullptr) return SA_ERR_INVALID_ARG;
     if (!aligned4(out->samp_count)) return SA_ERR_INVALID_ARG;
     if (params->sample_b > 0 && !aligned4(out->samp_idx)) return SA_ERR_INVALID_ARG;
     if (out->n_rescored != nullptr && !aligned4(out->n_rescored)) return SA_ERR_INVALID_ARG;
-    (void)k; (void)v;   // read only by the CLT budget
-    if (ws == nullptr || ws_bytes < p.bytes || !aligned16(ws)) return SA_ERR_WORKSPACE;
-    SelectArgs a{q, *stats, k, v, *out, *params, resolve_scale(scale, d.d), static_cast<char*>(ws)};
-    return launch_select(d, p, a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+    *a = SelectArgs{q, *stats, k, v, *out, *params, resolve_scale(scale, d->d), nullptr};
+    return SA_OK;
 }
 
-sa_status sa_decode(const sa_shape* shape, const sa_decode_params* dparams, const sa_select_params* sparams,
-                    const void* q, const void* k, const void* v, const sa_stats* stats,
-                    const sa_selection* sel, float* out, void* ws, size_t ws_bytes, void* stream) {
-    NvtxRange r("sa_decode");
-    Dims d;
-    sa_status e = check_shape(shape, &d);
+sa_status prep_decode(const sa_shape* shape, const sa_decode_params* dparams, const sa_select_params* sparams,
+                      const void* q, const void* k, const void* v, const sa_stats* stats, const sa_selection* sel,
+                      float* out, Dims* d, DecodePlan* p, size_t* need, DecodeArgs* a) {
+    sa_status e = check_shape(shape, d);
     if (e != SA_OK) return e;
     e = check_select_params(sparams);
     if (e != SA_OK) return e;
@@ -164,15 +165,70 @@ sa_status sa_decode(const sa_shape* shape, const sa_decode_params* dparams, cons
             return SA_ERR_INVALID_ARG;
         if (m == SA_PROXY && (!aligned16(st.sum_k) || !aligned16(st.sum_v))) return SA_ERR_INVALID_ARG;
     }
-    const DecodePlan p = decode_plan(d, *sparams, (int)m);
-    const size_t need = decode_plan(d, *sparams).bytes;
-    if (p.g.kk > 0 && !aligned4(sel->blk_idx)) return SA_ERR_INVALID_ARG;
+    *p = decode_plan(*d, *sparams, (int)m);
+    *need = decode_plan(*d, *sparams).bytes;
+    if (p->g.kk > 0 && !aligned4(sel->blk_idx)) return SA_ERR_INVALID_ARG;
     if (m == SA_SAMPLE && (sparams->sample_cap < 1 || !aligned4(sel->samp_idx) || !aligned4(sel->samp_count)))
         return SA_ERR_INVALID_ARG;
+    *a = DecodeArgs{q, k, v, st, *sel, *sparams, *dparams, resolve_scale(dparams->scale, d->d), out, nullptr, false};
+    return SA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sa_status sa_select(const sa_shape* shape, const sa_select_params* params, const void* q,
+                    const sa_stats* stats, const void* k, const void* v, const sa_selection* out,
+                    float scale, void* ws, size_t ws_bytes, void* stream) {
+    NvtxRange r("sa_select");
+    Dims d;
+    SelectPlan p;
+    SelectArgs a;
+    sa_status e = prep_select(shape, params, q, stats, k, v, out, scale, &d, &p, &a);
+    if (e != SA_OK) return e;
+    if (ws == nullptr || ws_bytes < p.bytes || !aligned16(ws)) return SA_ERR_WORKSPACE;
+    a.ws = static_cast<char*>(ws);
+    return launch_select(d, p, a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+sa_status sa_decode(const sa_shape* shape, const sa_decode_params* dparams, const sa_select_params* sparams,
+                    const void* q, const void* k, const void* v, const sa_stats* stats,
+                    const sa_selection* sel, float* out, void* ws, size_t ws_bytes, void* stream) {
+    NvtxRange r("sa_decode");
+    Dims d;
+    DecodePlan p;
+    size_t need;
+    DecodeArgs a;
+    sa_status e = prep_decode(shape, dparams, sparams, q, k, v, stats, sel, out, &d, &p, &need, &a);
+    if (e != SA_OK) return e;
     if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return SA_ERR_WORKSPACE;
-    DecodeArgs a{q, k, v, st, *sel, *sparams, *dparams, resolve_scale(dparams->scale, d.d), out,
-                 static_cast<char*>(ws)};
+    a.ws = static_cast<char*>(ws);
     return launch_decode(d, p, a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+sa_status sa_step(const sa_shape* shape, const sa_decode_params* dparams, const sa_select_params* sparams,
+                  const void* q, const void* k, const void* v, const sa_stats* stats, const sa_selection* sel,
+                  float* out, void* ws, size_t ws_bytes, void* stream) {
+    NvtxRange r("sa_step");
+    Dims d;
+    SelectPlan ps;
+    SelectArgs as;
+    const float scale = dparams != nullptr ? dparams->scale : 0.f;
+    sa_status e = prep_select(shape, sparams, q, stats, k, v, sel, scale, &d, &ps, &as);
+    if (e != SA_OK) return e;
+    DecodePlan pd;
+    size_t need;
+    DecodeArgs ad;
+    e = prep_decode(shape, dparams, sparams, q, k, v, stats, sel, out, &d, &pd, &need, &ad);
+    if (e != SA_OK) return e;
+    if (ws == nullptr || ws_bytes < ps.bytes + need || !aligned16(ws)) return SA_ERR_WORKSPACE;
+    as.ws = static_cast<char*>(ws);
+    ad.ws = static_cast<char*>(ws) + ps.bytes;
+    ad.pdl = true;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (launch_select(d, ps, as, s) != cudaSuccess) return SA_ERR_CUDA;
+    return launch_decode(d, pd, ad, s) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 
 sa_status sa_dense_decode(const sa_shape* shape, const void* q, const void* k, const void* v, float* out,

@@ -109,6 +109,16 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// d = a * b + d on two fp32 lanes at once (packed FMA, round to nearest)
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 A, B, C;\n\tmov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\tmov.b64 C, {%0, %1};\n\t"
+        "fma.rn.f32x2 C, A, B, C;\n\tmov.b64 {%0, %1}, C;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+__host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
+
 template <int W>
 __device__ __forceinline__ float group_sum(float x) {
 #pragma unroll

@@ -25,20 +25,24 @@
 
 namespace sa {
 
-// Position and log2-weight of token t of a unit's list.
+// Position and log2-weight of token t of a unit's list, ordered
+//   [sink 0..s_eff) [window L-w_eff..L) [chosen blocks, ascending] [draws]
+// so that the rows that do not depend on the step's selection come first.
 struct TokenMap {
-    int s_eff, kk, n_i, win0;      // win0 = L - w_eff
-    const int32_t* blk;            // chosen blocks of the unit (ascending)
-    const int32_t* samp;           // draws of the unit
-    float lw_samp;                 // log2(n_T / b)
+    int s_eff, w_eff, kk, n_i, win0;   // win0 = L - w_eff
+    const int32_t* blk;                // chosen blocks of the unit (ascending)
+    const int32_t* samp;               // draws of the unit
+    float lw_samp;                     // log2(n_T / b)
     __device__ __forceinline__ int pos(int t, float& lw) const {
         lw = 0.f;
         if (t < s_eff) return t;
-        const int tb = t - s_eff;
-        if (tb < 16 * kk) return 16 * __ldg(blk + (tb >> 4)) + (tb & 15);
-        if (t < n_i) return win0 + (tb - 16 * kk);
+        if (t < s_eff + w_eff) return win0 + (t - s_eff);
+        if (t < n_i) {
+            const int j = t - s_eff - w_eff;
+            return 16 * __ldcg(blk + (j >> 4)) + (j & 15);
+        }
         lw = lw_samp;
-        return __ldg(samp + (t - n_i));
+        return __ldcg(samp + (t - n_i));
     }
 };
 
@@ -83,6 +87,7 @@ __device__ void decode_epilogue(const float* recs, int nsd, int rec, const T* qg
         for (int h = warp; h < G; h += nwarps) {
             const size_t qh = (size_t)b * Hq + g * G + h;
             float x = 0.f;
+#pragma unroll
             for (int e = lane; e < D; e += 32) {
                 const float qe = to_f32<T>(qg[(size_t)h * D + e]);
                 if constexpr (PRIOR) x = fmaf(qe - st.mu_q[qh * D + e], st.mu_k[(size_t)u * D + e], x);
@@ -158,7 +163,7 @@ k_decode(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__
     const int nt = sg.n_t;
     const int bu = (SAMP && nt > 0) ? min(__ldg(samp_count + u), sample_cap) : 0;
     TokenMap tm;
-    tm.s_eff = sg.s_eff; tm.kk = sg.kk; tm.n_i = sg.n_i; tm.win0 = L - sg.w_eff;
+    tm.s_eff = sg.s_eff; tm.w_eff = sg.w_eff; tm.kk = sg.kk; tm.n_i = sg.n_i; tm.win0 = L - sg.w_eff;
     tm.blk = blk_idx + (size_t)u * kb_stride;
     tm.samp = samp_idx + (size_t)u * (sample_cap > 0 ? sample_cap : 0);
     tm.lw_samp = bu > 0 ? log2f((float)nt / (float)bu) : 0.f;
@@ -365,18 +370,27 @@ constexpr int kDenseMode = 4;      // MODE value of the dense pass
 template <int D>
 struct StageLayout {
     static constexpr int kTileBytes = kTcTile * tc::Pitch<D>::kBytes;   // one of K or V
-    static constexpr int kBytes = 2 * kTileBytes + kTcTile * 8;         // K, V, pos[], lw[]
+    static constexpr int kBytes = 2 * kTileBytes + kTcTile * 4;         // K, V, row positions
 };
+
+// The unit's chosen blocks and draws are cached in shared memory (after the
+// ring) when they fit; longer lists are read from global memory.
+constexpr int kBlkCache = 1024;
+constexpr int kSampCache = 256;
 
 template <int D, int G, int MODE>
 constexpr size_t stream_smem() {
     constexpr bool PRIOR = (MODE == SA_RESA);
-    constexpr size_t ring = (size_t)kStages * StageLayout<D>::kBytes;
+    constexpr size_t ring = (size_t)kStages * StageLayout<D>::kBytes + (kBlkCache + kSampCache) * 4;
     constexpr size_t merge = (size_t)(kTcWarps * G * 4 + (PRIOR ? 2 : 1) * kTcWarps * G * D) * 4;
     constexpr size_t tail = (size_t)(2 * G * (2 + D) + 2 * D) * 4        // own record
                             + (size_t)(2 * G * D + 4 * G + 2 * D + G) * 4;  // epilogue scratch
     constexpr size_t m = merge + tail;
     return ring > m ? ring : m;
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];\n" ::"l"(p));
 }
 
 template <int D, int G, int MODE>
@@ -394,6 +408,8 @@ k_stream_tc(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict
     constexpr int TB = StageLayout<D>::kTileBytes;
     constexpr int SB = StageLayout<D>::kBytes;
     extern __shared__ __align__(16) unsigned char smem[];
+    int* s_blk = reinterpret_cast<int*>(smem + (size_t)kStages * SB);
+    int* s_samp = s_blk + kBlkCache;
 
     const int u = blockIdx.y, chunk = blockIdx.x;
     const int b = u / Hkv, g = u - b * Hkv;
@@ -402,78 +418,141 @@ k_stream_tc(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict
     const __nv_bfloat16* K = k + ubase;
     const __nv_bfloat16* V = v + ubase;
     const __nv_bfloat16* qg = q + ((size_t)b * Hq + (size_t)g * G) * D;
+    const size_t qh0 = (size_t)b * Hq + (size_t)g * G;
+
+    // the epilogue's inputs (query, prefill statistics) into L2 while streaming
+    if constexpr (!DENSE) {
+        const int t = threadIdx.x;
+        if (t * 64 < G * D * 2) prefetch_l2(reinterpret_cast<const char*>(qg) + t * 64);
+        if constexpr (PRIOR) {
+            if (t * 128 < G * D * 4) {
+                prefetch_l2(reinterpret_cast<const char*>(st.mu_q + qh0 * D) + t * 128);
+                prefetch_l2(reinterpret_cast<const char*>(st.o_est + qh0 * D) + t * 128);
+            }
+            if (t * 128 < D * 4) prefetch_l2(reinterpret_cast<const char*>(st.mu_k + (size_t)u * D) + t * 128);
+            if (t == 0) prefetch_l2(st.log_z0 + qh0);
+        }
+        if constexpr (SUMS) {
+            if (t * 128 < D * 4) {
+                prefetch_l2(reinterpret_cast<const char*>(st.sum_k + (size_t)u * D) + t * 128);
+                prefetch_l2(reinterpret_cast<const char*>(st.sum_v + (size_t)u * D) + t * 128);
+            }
+        }
+    }
 
     const int nt = DENSE ? 0 : sg.n_t;
-    const int bu = (SAMP && nt > 0) ? min(__ldg(samp_count + u), sample_cap) : 0;
-    TokenMap tm;
-    tm.s_eff = sg.s_eff; tm.kk = sg.kk; tm.n_i = sg.n_i; tm.win0 = L - sg.w_eff;
-    tm.blk = blk_idx + (size_t)u * kb_stride;
-    tm.samp = samp_idx + (size_t)u * (sample_cap > 0 ? sample_cap : 0);
-    tm.lw_samp = bu > 0 ? log2f((float)nt / (float)bu) : 0.f;
-    const int n_tok = DENSE ? L : sg.n_i + bu;
     const int n_i = DENSE ? L : sg.n_i;
-    const int ntiles = (n_tok + kTcTile - 1) / kTcTile;
+    const int win0 = L - sg.w_eff;
+    const int32_t* gblk = blk_idx + (size_t)u * kb_stride;
+    const int32_t* gsamp = samp_idx + (size_t)u * (sample_cap > 0 ? sample_cap : 0);
+    // rows [0, n_indep) do not depend on the selection; the tile range uses an
+    // upper bound on the list length (draw capacity); the exact count and the
+    // lists are read once the selection is visible
+    const int n_indep = DENSE ? L : sg.s_eff + sg.w_eff;
+    const int n_hi = DENSE ? L : sg.n_i + ((SAMP && nt > 0) ? sample_cap : 0);
+    int n_tok = n_hi;
+    float lw_samp = 0.f;
+    const bool blk_sm = sg.kk <= kBlkCache;
+    bool samp_sm = true;
+    bool sel_ready = DENSE || n_indep >= n_hi;
+    // Under programmatic dependent launch the preceding selection kernel may
+    // still be running: wait for it before the first selection-dependent read
+    // (a no-op when the kernel was launched normally).  Called at the same
+    // point by every thread.
+    auto wait_selection = [&]() {
+        if (!sel_ready) {
+            asm volatile("griddepcontrol.wait;\n" ::: "memory");
+            int bu = 0;
+            if (SAMP && nt > 0) {
+                bu = min(__ldcg(samp_count + u), sample_cap);
+                lw_samp = bu > 0 ? log2f((float)nt / (float)bu) : 0.f;
+                n_tok = sg.n_i + bu;
+            }
+            samp_sm = bu <= kSampCache;
+            if (blk_sm)
+                for (int x = threadIdx.x; x < sg.kk; x += kTcThreads) s_blk[x] = __ldcg(gblk + x);
+            if (samp_sm)
+                for (int x = threadIdx.x; x < bu; x += kTcThreads) s_samp[x] = __ldcg(gsamp + x);
+            __syncthreads();
+            sel_ready = true;
+        }
+    };
+    // token t of the unit's list -> cache row, or -1 (masked)
+    //   [sink 0..s_eff) [window L-w_eff..L) [chosen blocks] [draws]
+    auto pos_of = [&](int t) -> int {
+        int p;
+        if (DENSE) p = t < L ? t : -1;
+        else if (t >= n_tok) p = -1;
+        else if (t < sg.s_eff) p = t;
+        else if (t < n_indep) p = win0 + (t - sg.s_eff);
+        else if (t < n_i) {
+            const int j = t - n_indep;
+            p = 16 * (blk_sm ? s_blk[j >> 4] : __ldcg(gblk + (j >> 4))) + (j & 15);
+        } else {
+            const int j = t - n_i;
+            p = samp_sm ? s_samp[j] : __ldcg(gsamp + j);
+        }
+        return (unsigned)p < (unsigned)L ? p : -1;         // outside the cache: masked
+    };
+    const int ntiles = (n_hi + kTcTile - 1) / kTcTile;
     const int tile0 = chunk * tpc, tile1 = min(ntiles, tile0 + tpc);
 
-    // positions of tile i into stage arrays, then its K/V rows (cp.async)
+    // K/V rows of tile i into its stage (cp.async; masked rows zero-filled).
+    // The tile's row positions go to the stage first (one barrier), so the
+    // copy loop reads one shared word per 16-byte chunk.
     auto issue = [&](int i) {
         if (i < tile1) {
+            if ((i + 1) * kTcTile > n_indep) wait_selection();
             unsigned char* sb = smem + (size_t)(i % kStages) * SB;
             int* pos = reinterpret_cast<int*>(sb + 2 * TB);
-            float* lw = reinterpret_cast<float*>(pos + kTcTile);
-            if (threadIdx.x < kTcTile) {
-                const int t = i * kTcTile + threadIdx.x;
-                float w = 0.f;
-                int p = -1;
-                if (t < n_tok) p = DENSE ? t : tm.pos(t, w);
-                if ((unsigned)p >= (unsigned)L) p = -1;          // outside the cache: masked
-                pos[threadIdx.x] = p;
-                lw[threadIdx.x] = p >= 0 ? w : -INFINITY;
-            }
+            if (threadIdx.x < kTcTile) pos[threadIdx.x] = pos_of(i * kTcTile + threadIdx.x);
             __syncthreads();
             constexpr int CPR = D / 8;
             const uint32_t sk = tc::smem_u32(sb), sv = sk + TB;
 #pragma unroll 4
-            for (int idx = threadIdx.x; idx < 2 * kTcTile * CPR; idx += kTcThreads) {
-                const int kv = idx / (kTcTile * CPR);
-                const int rem = idx - kv * kTcTile * CPR;
-                const int row = rem / CPR, ch = rem - row * CPR;
-                const uint32_t dst = (kv ? sv : sk) + row * P + ch * 16;
+            for (int idx = threadIdx.x; idx < kTcTile * CPR; idx += kTcThreads) {
+                const int row = idx / CPR, ch = idx - row * CPR;
                 const int p = pos[row];
-                if (p >= 0) tc::cp16(dst, (kv ? V : K) + (size_t)p * D + ch * 8);
-                else tc::st_zero16(dst);
+                const uint32_t o = row * P + ch * 16;
+                if (p >= 0) {
+                    tc::cp16(sk + o, K + (size_t)p * D + ch * 8);
+                    tc::cp16(sv + o, V + (size_t)p * D + ch * 8);
+                } else {
+                    tc::st_zero16(sk + o);
+                    tc::st_zero16(sv + o);
+                }
             }
         }
         tc::cp_commit();
     };
 
+    // first tiles in flight before the query / prior fragments are loaded
+#pragma unroll
+    for (int i = 0; i < kStages - 1; ++i) issue(tile0 + i);
     tc::WarpAttn<D, G, PRIOR> wa;
     {
         const int gh = min(lane >> 2, G - 1);
-        wa.init(qg + (size_t)gh * D, PRIOR ? st.mu_q + ((size_t)b * Hq + g * G + gh) * D : nullptr);
+        wa.init(qg + (size_t)gh * D, PRIOR ? st.mu_q + (qh0 + gh) * D : nullptr);
     }
-    float ks[2] = {0.f, 0.f};      // SUMS: this thread's column pair of K (c < D/2 ... ) and V
-#pragma unroll
-    for (int i = 0; i < kStages - 1; ++i) issue(tile0 + i);
+    float ks[2] = {0.f, 0.f};      // SUMS: this thread's column pair of K (c < D/2) or V (c >= D/2)
     for (int i = tile0; i < tile1; ++i) {
         issue(i + kStages - 1);
         tc::cp_wait<kStages - 1>();
         __syncthreads();
         unsigned char* sb = smem + (size_t)(i % kStages) * SB;
-        const int* pos = reinterpret_cast<const int*>(sb + 2 * TB);
-        const float* lw = reinterpret_cast<const float*>(pos + kTcTile);
         const int base = i * kTcTile;
         if constexpr (SUMS) {
-            // column pair (2c, 2c+1) of K (c < D/2) or of V (c >= D/2) over the exact rows
+            // column pair (2c, 2c+1) of K (c < D/2) or of V (c >= D/2) over the
+            // exact rows of the tile, which form the prefix [0, nr)
             const int c = threadIdx.x;
+            const int nr = max(0, min(kTcTile, n_i - base));
             if (c < D) {
                 const unsigned char* src = sb + (c < D / 2 ? 0 : TB) + (c % (D / 2)) * 4;
-                for (int r = 0; r < kTcTile; ++r) {
-                    if (base + r < n_i && pos[r] >= 0) {
-                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(src + r * P));
-                        ks[0] += f.x;
-                        ks[1] += f.y;
-                    }
+#pragma unroll 8
+                for (int r = 0; r < nr; ++r) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(src + r * P));
+                    ks[0] += f.x;
+                    ks[1] += f.y;
                 }
             }
         }
@@ -483,10 +562,13 @@ k_stream_tc(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict
             const int rows[4] = {r0 + 2 * tq, r0 + 2 * tq + 1, r0 + 8 + 2 * tq, r0 + 9 + 2 * tq};
             float xadd[4];
             bool in_i[4];
+            const int* pos = reinterpret_cast<const int*>(sb + 2 * TB);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                xadd[j] = lw[rows[j]];
-                in_i[j] = PRIOR && (base + rows[j] < n_i) && pos[rows[j]] >= 0;
+                const int t = base + rows[j];
+                const bool ok = pos[rows[j]] >= 0;
+                xadd[j] = !ok ? -INFINITY : (t >= n_i ? lw_samp : 0.f);
+                in_i[j] = PRIOR && ok && t < n_i;
             }
             const uint32_t sk = tc::smem_u32(sb);
             wa.step16(sk, sk + TB, r0, xadd, in_i, qscale);
@@ -557,16 +639,26 @@ template <int D, int G, int MODE>
 static cudaError_t stream_launch(const Dims& d, dim3 grid, const void* q, const void* k, const void* v,
                                  const sa_stats& st, const sa_selection& sel, const sa_select_params& sp,
                                  const SetGeom& sg, int tpc, int nchunk, int rec, float scale, float lambda,
-                                 char* part, char* cnt, float* out, cudaStream_t s) {
+                                 char* part, char* cnt, float* out, bool pdl, cudaStream_t s) {
     constexpr size_t sm = stream_smem<D, G, MODE>();
     cudaError_t e = cudaFuncSetAttribute(k_stream_tc<D, G, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
-    k_stream_tc<D, G, MODE><<<grid, kTcThreads, sm, s>>>(
-        reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k),
-        reinterpret_cast<const __nv_bfloat16*>(v), st, sel.blk_idx, sp.k_blocks, sel.samp_idx, sel.samp_count,
-        sp.sample_cap, d.Hq, d.Hkv, d.L, sg, tpc, nchunk, rec, scale * kLog2e, scale, lambda,
-        reinterpret_cast<float*>(part), reinterpret_cast<unsigned*>(cnt), out);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = sm;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, k_stream_tc<D, G, MODE>, reinterpret_cast<const __nv_bfloat16*>(q),
+                              reinterpret_cast<const __nv_bfloat16*>(k), reinterpret_cast<const __nv_bfloat16*>(v),
+                              st, (const int32_t*)sel.blk_idx, (int)sp.k_blocks, (const int32_t*)sel.samp_idx,
+                              (const int32_t*)sel.samp_count, (int)sp.sample_cap, d.Hq, d.Hkv, d.L, sg, tpc, nchunk,
+                              rec, scale * kLog2e, scale, lambda, reinterpret_cast<float*>(part),
+                              reinterpret_cast<unsigned*>(cnt), out);
 }
 
 template <typename T, int D, int G, int MODE>
@@ -574,7 +666,7 @@ static cudaError_t decode_m(const Dims& d, const DecodePlan& p, const DecodeArgs
     if constexpr (std::is_same<T, __nv_bfloat16>::value) {
         return stream_launch<D, G, MODE>(d, dim3(p.nsd, d.U()), a.q, a.k, a.v, a.st, a.sel, a.sp, p.g, p.tok_d,
                                          p.nsd, p.rec, a.scale, a.dp.lambda, a.ws + p.off_part, a.ws + p.off_cnt,
-                                         a.out, s);
+                                         a.out, a.pdl, s);
     } else {
         k_decode<T, D, G, MODE><<<dim3(p.nsd, d.U()), kThreads, 0, s>>>(
             reinterpret_cast<const T*>(a.q), reinterpret_cast<const T*>(a.k), reinterpret_cast<const T*>(a.v),
@@ -621,7 +713,7 @@ static cudaError_t dense_t(const Dims& d, const DensePlan& p, const DenseArgs& a
         sa_select_params sp{};
         return stream_launch<D, G, kDenseMode>(d, dim3(p.nsdn, d.U()), a.q, a.k, a.v, st, sel, sp, sg,
                                                p.tok / kTcTile, p.nsdn, p.rec, a.scale, 1.f, a.ws + p.off_part,
-                                               a.ws + p.off_cnt, a.out, s);
+                                               a.ws + p.off_cnt, a.out, false, s);
     } else {
         k_dense<T, D, G><<<dim3(p.nsdn, d.U()), kThreads, 0, s>>>(
             reinterpret_cast<const T*>(a.q), reinterpret_cast<const T*>(a.k), reinterpret_cast<const T*>(a.v),

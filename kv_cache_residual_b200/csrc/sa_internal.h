@@ -7,7 +7,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
-#include "../../include/sa_decode.h"
+#include "sa_decode.h"
 
 namespace sa {
 
@@ -85,22 +85,22 @@ inline PrefillPlan prefill_plan(const Dims& d) {
 struct SelectPlan {
     SetGeom g;
     int nss, rows_s;             // scan splits per unit, candidate rows per split
-    size_t off_scores, off_xkey, off_flags, off_cnt, bytes;
+    size_t off_scores, off_xkey, off_cnt, bytes;
 };
 
 inline SelectPlan select_plan(const Dims& d, const sa_select_params& sp) {
     SelectPlan p;
     p.g = set_geom(d, sp.sink, sp.local, sp.k_blocks);
     const int nc = p.g.n_cand > 0 ? p.g.n_cand : 1;
-    // one wave: at most kSmTarget CTAs in all, at least 32 rows per CTA
-    p.nss = clampi(kSmTarget / d.U(), 1, cdiv(nc, 32));
+    // enough units to fill the GPU: one CTA per unit (scores stay on chip);
+    // otherwise split units so the grid is about one wave, >= 32 rows per CTA
+    p.nss = d.U() >= 148 ? 1 : clampi(kSmTarget / d.U(), 1, cdiv(nc, 32));
     p.rows_s = cdiv(nc, p.nss);
     p.nss = cdiv(nc, p.rows_s);
     size_t off = 0;
     p.off_cnt = off;    off = align256(off + sizeof(unsigned) * (size_t)d.U());
     p.off_scores = off; off = align256(off + sizeof(float) * (size_t)d.U() * nc);
     p.off_xkey = off;   off = align256(off + sizeof(unsigned long long) * (size_t)d.U() * nc);
-    p.off_flags = off;  off = align256(off + (size_t)d.U() * nc);
     p.bytes = off;
     return p;
 }
@@ -187,6 +187,7 @@ cudaError_t launch_select(const Dims& d, const SelectPlan& p, const SelectArgs& 
 struct DecodeArgs {
     const void* q; const void* k; const void* v; sa_stats st; sa_selection sel;
     sa_select_params sp; sa_decode_params dp; float scale; float* out; char* ws;
+    bool pdl;          // launched as a programmatic dependent of the selection kernel
 };
 cudaError_t launch_decode(const Dims& d, const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
 

@@ -3,24 +3,30 @@
 // block selection of Quest / ArkVale that RESA wraps).
 //
 // k_select: grid (nss, B*Hkv)
-//   scan  : every CTA scores a slice of the unit's candidate blocks in fp32,
-//           y_c = qbar . kbar_c with qbar = sum_{h in group} q_h, and stores y
-//           in the workspace (the HBM-bound part: one read of the summaries);
-//   top-k : the CTA that finishes the unit last (completion ticket, no wait)
-//           finds the k-th largest y by a 4 x 8-bit radix select, takes ties at
-//           the threshold by lowest block index, and checks the rounding bound
-//           |y_c - x_c| <= E (x_c the exact score): every candidate with
-//           y >= y_(k) - 2E may belong to the exact top-k; if more than k do,
-//           those are rescored in fp64 and the top-k is re-taken over 64-bit
-//           keys.  The decision is therefore the fp64 one.
+//   scan  : fp32 scores y_c = sum_h q_h . kbar_c of the unit's candidate blocks
+//           (computed as qbar . kbar_c, qbar = sum_h q_h), the HBM-bound part:
+//           one read of the block summaries.  With one CTA per unit (enough
+//           units to fill the GPU) the scores stay in shared memory; with
+//           several CTAs per unit they go to the workspace and the CTA that
+//           finishes the unit last (completion ticket, no wait) takes over.
+//   top-k : exact k best by (score desc, block index asc).  For k <= 32 the
+//           warps extract their local best k by argmax rounds over 64-bit
+//           (score, ~index) keys in registers and one warp merges them;
+//           otherwise a 4 x 8-bit radix select finds the k-th key.  Then the
+//           rounding bound |y_c - x_c| <= E of the fp32 scan (x_c the exact
+//           score) is applied: every candidate with y >= y_(k) - 2E may belong
+//           to the exact top k; if more than k do, those are rescored in fp64
+//           and ranked exactly.  The decision is therefore the fp64 one.
 //   draws : tail positions for the sampling estimator (SplitMix64 counters).
 #include "sa_common.cuh"
 #include "sa_internal.h"
 
 namespace sa {
 
-constexpr int kSmemKeys = 4096;     // candidate keys staged in shared memory (16 KB)
+constexpr int kSmemKeys = 4096;     // candidate keys held in shared memory (16 KB)
 constexpr int kBandCap = 512;       // band members ranked in shared memory
+constexpr int kWarpTopK = 32;       // largest k of the warp-argmax path
+constexpr int kRowsPer = 8;         // rows per lane group per scan step
 
 __device__ __forceinline__ uint32_t fkey(float y) {
     const uint32_t b = __float_as_uint(y + 0.0f);   // -0 -> +0
@@ -32,6 +38,26 @@ __device__ __forceinline__ float fkey_inv(uint32_t k) {
 __device__ __forceinline__ unsigned long long dkey(double x) {
     const unsigned long long b = (unsigned long long)__double_as_longlong(x + 0.0);
     return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+// score key and block index in one orderable word: larger = better,
+// equal scores ordered by lower index
+__device__ __forceinline__ unsigned long long comp_key(uint32_t key, int i) {
+    return ((unsigned long long)key << 32) | (unsigned long long)(~(uint32_t)i);
+}
+__device__ __forceinline__ int comp_index(unsigned long long c) { return (int)(~(uint32_t)c); }
+
+__device__ __forceinline__ unsigned long long shfl_xor_u64(unsigned long long v, int off) {
+    const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, off);
+    const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), off);
+    return ((unsigned long long)hi << 32) | lo;
+}
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const unsigned long long o = shfl_xor_u64(v, off);
+        v = o > v ? o : v;
+    }
+    return v;
 }
 
 // Block-wide exclusive scan of one int per thread (thread order).  Returns
@@ -146,91 +172,230 @@ __device__ void emit_topk(KeyFn key, int n, KT thr, int need, int kk, int c_lo, 
     }
 }
 
+// Top kk (kk <= 32, n <= kSmemKeys) of keys[0..n) by argmax rounds: every warp
+// holds a contiguous span in registers and extracts its best kk one at a time
+// (lane max, then warp max over 64-bit (key, ~index) words); warp 0 then
+// merges the per-warp lists the same way.  s_list[0..kk) gets the result in
+// rank order.  s_cand holds kWarps * kk words.
+__device__ void warp_topk(const uint32_t* keys, int n, int kk, unsigned long long* s_cand,
+                          unsigned long long* s_list) {
+    constexpr int C = kSmemKeys / kThreads;            // keys per lane (16)
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int span = (n + kWarps - 1) / kWarps;
+    const int w0 = warp * span;
+    unsigned long long c[C];
+#pragma unroll
+    for (int j = 0; j < C; ++j) {
+        const int i = w0 + j * 32 + lane;
+        c[j] = (j * 32 + lane < span && i < n) ? comp_key(keys[i], i) : 0ull;
+    }
+    for (int r = 0; r < kk; ++r) {
+        unsigned long long m = 0ull;
+#pragma unroll
+        for (int j = 0; j < C; ++j) m = c[j] > m ? c[j] : m;
+        const unsigned long long best = warp_max_u64(m);
+#pragma unroll
+        for (int j = 0; j < C; ++j) if (c[j] == best) c[j] = 0ull;     // keys are unique
+        if (lane == 0) s_cand[warp * kk + r] = best;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        constexpr int CM = kWarps * kWarpTopK / 32;     // candidates per lane (8)
+        unsigned long long d[CM];
+#pragma unroll
+        for (int j = 0; j < CM; ++j) {
+            const int i = j * 32 + lane;
+            d[j] = i < kWarps * kk ? s_cand[i] : 0ull;
+        }
+        for (int r = 0; r < kk; ++r) {
+            unsigned long long m = 0ull;
+#pragma unroll
+            for (int j = 0; j < CM; ++j) m = d[j] > m ? d[j] : m;
+            const unsigned long long best = warp_max_u64(m);
+#pragma unroll
+            for (int j = 0; j < CM; ++j) if (d[j] == best) d[j] = 0ull;
+            if (lane == 0) s_list[r] = best;
+        }
+    }
+    __syncthreads();
+}
+
+// Sorts s_list[0..kk) (kk <= 32) by block index and writes c_lo + index in
+// ascending order (one warp, bitonic network over the 32 lanes).
+__device__ void emit_sorted_list(const unsigned long long* s_list, int kk, int c_lo, int32_t* out_idx) {
+    if (threadIdx.x >= 32) return;
+    const int lane = threadIdx.x;
+    int v = lane < kk ? comp_index(s_list[lane]) : 0x7fffffff;
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const int o = __shfl_xor_sync(0xffffffffu, v, stride);
+            const bool up = ((lane & size) == 0);
+            const bool lower = ((lane & stride) == 0);
+            v = (lower == up) ? min(v, o) : max(v, o);
+        }
+    }
+    if (lane < kk) out_idx[lane] = c_lo + v;
+}
+
+// fp64 scores of the band members s_bidx[0..nb) into s_bx (a warp per member,
+// four members' rows in flight per warp).
+template <typename T, int D>
+__device__ void rescore_members(const T* bm, const int* s_bidx, int nb, const double* s_q64, double* s_bx) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int j0 = warp * 4; j0 < nb; j0 += kWarps * 4) {
+        float v[4][D / 32];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int j = j0 + m;
+#pragma unroll
+            for (int e = 0; e < D / 32; ++e)
+                v[m][e] = j < nb ? to_f32<T>(bm[(size_t)s_bidx[j] * D + lane + 32 * e]) : 0.f;
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            double x = 0.0;
+#pragma unroll
+            for (int e = 0; e < D / 32; ++e) x += s_q64[lane + 32 * e] * (double)v[m][e];
+            x = group_sum_f64<32>(x) + 0.0;        // -0 -> +0
+            if (lane == 0 && j0 + m < nb) s_bx[j0 + m] = x;
+        }
+    }
+}
+
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads)
 k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* __restrict__ kbar_absmax,
          int Hq, int Hkv, int L, SetGeom sg, int rows, int nss,
-         float* __restrict__ scores, unsigned long long* __restrict__ xkey, unsigned char* __restrict__ flags_ws,
+         float* __restrict__ scores, unsigned long long* __restrict__ xkey,
          unsigned* __restrict__ cnt, int kb_stride, int32_t* __restrict__ blk_idx,
          int32_t* __restrict__ samp_idx, int32_t* __restrict__ samp_count, int32_t* __restrict__ n_rescored,
          int sample_b, int sample_cap, unsigned long long seed, int step) {
     using Gm = Geom<T, D>;
     constexpr int EPC = Gm::EPC, CPR = Gm::CPR, NG = Gm::NG;
+    constexpr int R = kRowsPer;
+    static_assert(CPR >= R, "transposed reduction needs at least one lane per row");
     __shared__ unsigned hist[kThreads];
     __shared__ int sw[kWarps + 1];
-    __shared__ int s_digit, s_rem, s_band;
+    __shared__ int s_digit, s_rem, s_nb;
     __shared__ double s_q64[D];
-    __shared__ float s_qa[kWarps];
+    __shared__ float s_qsum;
     __shared__ uint32_t s_keys[kSmemKeys];
-    __shared__ int s_nb;
     __shared__ int s_bidx[kBandCap];
     __shared__ double s_bx[kBandCap];
     __shared__ unsigned char s_bsel[kBandCap];
+    __shared__ unsigned long long s_cand[kWarps * kWarpTopK];
+    __shared__ unsigned long long s_list[kWarpTopK];
 
+    // a decode kernel launched as a programmatic dependent may start as soon as
+    // every CTA of this grid has begun; it waits for this grid's completion
+    // before reading the selection
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
     const int u = blockIdx.y, split = blockIdx.x;
     const int b = u / Hkv, g = u - b * Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int gi = warp * Gm::GPW + lane / CPR, li = lane % CPR;
+    const int li = lane % CPR;
     const int nb = L / 16;
     const int n = sg.n_cand, kk = sg.kk;
     const T* qg = q + ((size_t)b * Hq + (size_t)g * G) * D;
     float* sc = scores + (size_t)u * (n > 0 ? n : 1);
+    // one CTA per unit: the scores never leave shared memory
+    const bool local = (nss == 1) && n <= kSmemKeys;
 
     // ---- scan: fp32 scores of this CTA's slice -------------------------------
     {
         float qb[EPC];
+        double q64[EPC];
+        float qa = 0.f;
 #pragma unroll
-        for (int e = 0; e < EPC; ++e) qb[e] = 0.f;
+        for (int e = 0; e < EPC; ++e) { qb[e] = 0.f; q64[e] = 0.0; }
 #pragma unroll
         for (int h = 0; h < G; ++h) {
             float f[EPC];
             unpack<T>(ld_nc16(qg + (size_t)h * D + li * EPC), f);
 #pragma unroll
-            for (int e = 0; e < EPC; ++e) qb[e] += f[e];
+            for (int e = 0; e < EPC; ++e) {
+                qb[e] += f[e];
+                q64[e] += (double)f[e];
+                qa += fabsf(f[e]);
+            }
+        }
+        // for the top-k (whichever CTA ends up doing it): the fp64 group query
+        // and sum_i sum_h |q_hi| for the rounding bound, from lane group 0
+        qa = group_sum<CPR>(qa);
+        if (lane < CPR && warp == 0) {
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) s_q64[li * EPC + e] = q64[e];
+            if (lane == 0) s_qsum = qa;
         }
         const T* base = blk_mean + ((size_t)u * nb + sg.c_lo) * D + li * EPC;
         const int r0 = split * rows, r1 = min(n, r0 + rows);
         const int gsub = lane / CPR;
-        // warp-uniform loop: a warp step covers 4 x GPW rows (4 per lane group);
-        // the next step's rows are loaded before this step's are reduced, so 8
-        // rows per lane group are in flight; rows past the end load nothing
-        auto load4 = [&](int wr, uint4 (&w)[4]) {
+        // warp-uniform loop: a warp step covers R x GPW rows (R per lane group);
+        // the next step's rows are loaded before this step's are reduced, so
+        // 2R rows per lane group are in flight; rows past the end load nothing
+        auto loadR = [&](int wr, uint4 (&w)[R]) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < R; ++j) {
                 const int r = wr + j * Gm::GPW + gsub;
                 w[j] = (r < r1) ? ld_stream16(base + (size_t)r * D) : make_uint4(0, 0, 0, 0);
             }
         };
-        int wr = r0 + warp * 4 * Gm::GPW;
-        uint4 cur[4];
-        load4(wr, cur);
-        for (; wr < r1; wr += 4 * NG) {
-            uint4 nxt[4];
-            load4(wr + 4 * NG, nxt);
+        int wr = r0 + warp * R * Gm::GPW;
+        uint4 cur[R];
+        loadR(wr, cur);
+        for (; wr < r1; wr += R * NG) {
+            uint4 nxt[R];
+            loadR(wr + R * NG, nxt);
+            // lane partial dot of each row: packed FMAs over element pairs,
+            // then the two halves added
+            float x[R];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int r = wr + j * Gm::GPW + gsub;
+            for (int j = 0; j < R; ++j) {
                 float f[EPC];
                 unpack<T>(cur[j], f);
-                float x = 0.f;
+                float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-                for (int e = 0; e < EPC; ++e) x = fmaf(qb[e], f[e], x);
-                x = group_sum<CPR>(x);
-                if (li == 0 && r < r1) sc[r] = x;
+                for (int e = 0; e < EPC; e += 2) ffma2(a0, a1, qb[e], qb[e + 1], f[e], f[e + 1]);
+                x[j] = a0 + a1;
+            }
+            // transposed reduction over the CPR lanes of the group: each of the
+            // first log2(R) levels keeps half of the remaining rows, so the lane
+            // bits select one row; the remaining levels add across lanes
+            int row = 0;
+#pragma unroll
+            for (int half = R / 2, off = CPR / 2; half > 0; half >>= 1, off >>= 1) {
+                const int bit = (li & off) ? 1 : 0;
+#pragma unroll
+                for (int j = 0; j < half; ++j) {
+                    const float send = bit ? x[j] : x[j + half];
+                    const float keep = bit ? x[j + half] : x[j];
+                    x[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                }
+                row = 2 * row + bit;
             }
 #pragma unroll
-            for (int j = 0; j < 4; ++j) cur[j] = nxt[j];
+            for (int off = CPR / (2 * R); off > 0; off >>= 1) x[0] += __shfl_xor_sync(0xffffffffu, x[0], off);
+            const int r = wr + row * Gm::GPW + gsub;
+            if ((li & (CPR / R - 1)) == 0 && r < r1) {
+                if (local) s_keys[r] = fkey(x[0]);
+                else sc[r] = x[0];
+            }
+#pragma unroll
+            for (int j = 0; j < R; ++j) cur[j] = nxt[j];
         }
     }
-    if (!last_cta_of_unit(cnt + u, nss)) return;
 
-    // ---- top-k of the unit (last CTA) ------------------------------------------
-    int32_t* out_idx = blk_idx + (size_t)u * kb_stride;
-    int rescored = 0;
-    if (kk > 0 && kk < n) {
+    // ---- gather the unit's scores ------------------------------------------------
+    uint32_t* keys = s_keys;
+    if (local) {
+        __syncthreads();
+    } else {
+        if (!last_cta_of_unit(cnt + u, nss)) return;
         // orderable keys, staged once: shared memory when they fit, else in
         // place over the unit's scores in the workspace
-        uint32_t* keys = (n <= kSmemKeys) ? s_keys : reinterpret_cast<uint32_t*>(sc);
+        if (n > kSmemKeys) keys = reinterpret_cast<uint32_t*>(sc);
         for (int i0 = 0; i0 < n; i0 += 4 * kThreads) {
             float y[4];
 #pragma unroll
@@ -245,54 +410,50 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
             }
         }
         __syncthreads();
+    }
+
+    // ---- top-k of the unit ------------------------------------------------------------
+    int32_t* out_idx = blk_idx + (size_t)u * kb_stride;
+    int rescored = 0;
+    if (kk > 0 && kk < n) {
         auto k32 = [&](int i) -> uint32_t { return keys[i]; };
+        const bool fast = kk <= kWarpTopK && n <= kSmemKeys;
         uint32_t thr;
-        int need;
-        radix_select<uint32_t>(k32, n, kk, &thr, &need, hist, &s_digit, &s_rem);
-        // rounding bound of the fp32 scan: |y - x| <= (G + D) 2^-23 sum_i qa_i * max|kbar|
-        float qa = 0.f;
-        for (int i = threadIdx.x; i < D; i += kThreads) {
-            float s = 0.f;
-            for (int h = 0; h < G; ++h) s += fabsf(to_f32<T>(qg[(size_t)h * D + i]));
-            qa += s;
+        int need = 0;
+        if (fast) {
+            warp_topk(keys, n, kk, s_cand, s_list);
+            thr = (uint32_t)(s_list[kk - 1] >> 32);
+        } else {
+            radix_select<uint32_t>(k32, n, kk, &thr, &need, hist, &s_digit, &s_rem);
         }
-        for (int off = 16; off > 0; off >>= 1) qa += __shfl_xor_sync(0xffffffffu, qa, off);
-        if (lane == 0) s_qa[warp] = qa;
-        __syncthreads();
-        float qsum = 0.f;
-        for (int w = 0; w < kWarps; ++w) qsum += s_qa[w];
-        const float E = (float)(G + D) * 0x1p-23f * qsum * kbar_absmax[u] * 1.0001f + 0x1p-100f;
+        // rounding bound of the fp32 scan.  qbar_i is a sum of G terms (G-1
+        // roundings) and each score is EPC/2 fused multiply-adds on each of two
+        // accumulators per lane, their sum, then a log2(CPR)-level shuffle tree
+        // (depth h = EPC/2 + 1 + log2(CPR)), so with u = 2^-24
+        //   |y - x| <= (gamma_{G-1} + gamma_h (1 + gamma_{G-1})) sum_i qa_i |kbar_ci|
+        //           <= (G + h + 2) 2^-24 sum_i qa_i * max|kbar|,
+        // taken twice over for margin.
+        constexpr int kDepth = EPC / 2 + 1 + ilog2(CPR);
+        const float E = (float)(G + kDepth + 2) * 0x1p-23f * s_qsum * kbar_absmax[u] * 1.0001f + 0x1p-100f;
         const uint32_t lo_key = fkey(fkey_inv(thr) - 2.f * E);
         int band = 0;
         for (int i = threadIdx.x; i < n; i += kThreads) band += (keys[i] >= lo_key) ? 1 : 0;
         band = block_sum(band, sw);
         if (band == kk) {
-            emit_topk<uint32_t>(k32, n, thr, need, kk, sg.c_lo, out_idx, sw);
+            if (fast) emit_sorted_list(s_list, kk, sg.c_lo, out_idx);
+            else emit_topk<uint32_t>(k32, n, thr, need, kk, sg.c_lo, out_idx, sw);
         } else {
             // ambiguous: the exact top-k lies inside the band; rescore the band
             // members in fp64 and take the top k among them by (x desc, index asc)
             rescored = band;
-            for (int i = threadIdx.x; i < D; i += kThreads) {
-                double s = 0.0;
-                for (int h = 0; h < G; ++h) s += (double)to_f32<T>(qg[(size_t)h * D + i]);
-                s_q64[i] = s;
-            }
             const T* bm = blk_mean + ((size_t)u * nb + sg.c_lo) * D;
-            auto dot64 = [&](int i) -> double {      // warp-collective fp64 score of candidate i
-                double x = 0.0;
-                for (int e = lane; e < D; e += 32) x += s_q64[e] * (double)to_f32<T>(bm[(size_t)i * D + e]);
-                return group_sum_f64<32>(x) + 0.0;  // -0 -> +0
-            };
             if (band <= kBandCap) {
                 if (threadIdx.x == 0) s_nb = 0;
                 __syncthreads();
                 for (int i = threadIdx.x; i < n; i += kThreads)
                     if (keys[i] >= lo_key) s_bidx[atomicAdd(&s_nb, 1)] = i;
                 __syncthreads();
-                for (int j = warp; j < band; j += kWarps) {
-                    const double x = dot64(s_bidx[j]);
-                    if (lane == 0) s_bx[j] = x;
-                }
+                rescore_members<T, D>(bm, s_bidx, band, s_q64, s_bx);
                 __syncthreads();
                 for (int j = threadIdx.x; j < band; j += kThreads) {
                     const double xj = s_bx[j];
@@ -319,7 +480,11 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
                 unsigned long long* xk = xkey + (size_t)u * n;
                 for (int i = warp; i < n; i += kWarps) {
                     unsigned long long key = 0ull;
-                    if (keys[i] >= lo_key) key = dkey(dot64(i));   // warp-uniform branch
+                    if (keys[i] >= lo_key) {                        // warp-uniform branch
+                        double x = 0.0;
+                        for (int e = lane; e < D; e += 32) x += s_q64[e] * (double)to_f32<T>(bm[(size_t)i * D + e]);
+                        key = dkey(group_sum_f64<32>(x));
+                    }
                     if (lane == 0) xk[i] = key;
                 }
                 __threadfence_block();
@@ -359,7 +524,7 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
             out_s[i] = sg.s_eff + r + 16 * lo_j;
         }
     }
-    reset_counter(cnt + u);
+    if (!local) reset_counter(cnt + u);
 }
 
 template <typename T, int D, int G>
@@ -369,9 +534,9 @@ static cudaError_t select_t(const Dims& d, const SelectPlan& p, const SelectArgs
         reinterpret_cast<const T*>(a.q), reinterpret_cast<const T*>(a.st.blk_mean), a.st.kbar_absmax,
         d.Hq, d.Hkv, d.L, p.g, p.rows_s, p.nss,
         reinterpret_cast<float*>(ws + p.off_scores), reinterpret_cast<unsigned long long*>(ws + p.off_xkey),
-        reinterpret_cast<unsigned char*>(ws + p.off_flags), reinterpret_cast<unsigned*>(ws + p.off_cnt),
-        a.sp.k_blocks, a.sel.blk_idx, a.sel.samp_idx, a.sel.samp_count, a.sel.n_rescored,
-        a.sp.sample_b, a.sp.sample_cap, (unsigned long long)a.sp.seed, a.sp.step);
+        reinterpret_cast<unsigned*>(ws + p.off_cnt), a.sp.k_blocks, a.sel.blk_idx, a.sel.samp_idx,
+        a.sel.samp_count, a.sel.n_rescored, a.sp.sample_b, a.sp.sample_cap, (unsigned long long)a.sp.seed,
+        a.sp.step);
     return cudaGetLastError();
 }
 

@@ -232,3 +232,20 @@ def test_full_size_sampled_units(wname, units, dev):
                 assert e < REL_L2_OUT, (label, b, g, m, e)
     del data
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", ["bf16_d128_g4", "tiny", "bf16_d64_g8"])
+def test_step_equals_select_then_decode(name, dev):
+    """sa_step (decode overlapped with the selection) gives exactly the
+    results of the two calls in sequence."""
+    w, data = _data(name, dev)
+    st = sa.prefill_stats(data["q_ctx"], data["k"], data["v"])
+    q = data["q"][1]
+    for m in MODES:
+        sp = _sp(w, step=1)
+        sel = sa.select(q, st, sp)
+        want = sa.decode(q, data["k"], data["v"], st, sel, sp, mode=m)
+        got, sel2 = sa.step(q, data["k"], data["v"], st, sp, mode=m)
+        torch.cuda.synchronize()
+        assert torch.equal(sel.blk_idx, sel2.blk_idx) and torch.equal(sel.samp_idx, sel2.samp_idx)
+        assert torch.equal(got, want), m
