@@ -36,7 +36,7 @@ FLUSH_BYTES = 256 << 20
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="batched")
@@ -84,6 +84,37 @@ def set_geom(L, sink, local, k_blocks):
     return {"n_cand": n_cand, "kk": kk, "n_i": n_i, "n_t": L - n_i}
 
 
+def sources_sha1():
+    """sha1 over the CUDA sources (name + bytes), to tell whether an ncu
+    capture still describes the kernels being run."""
+    import glob
+    import hashlib
+    h = hashlib.sha1()
+    d = os.path.join(ROOT, "kv_cache_residual_b200", "csrc")
+    for f in sorted(glob.glob(os.path.join(d, "*.cu")) + glob.glob(os.path.join(d, "*.cuh")) +
+                    glob.glob(os.path.join(d, "*.h"))):
+        h.update(os.path.basename(f).encode())
+        h.update(open(f, "rb").read())
+    return h.hexdigest()
+
+
+def select_traffic(workload, read, units):
+    """DRAM bytes per k_select launch from profiles/traffic.txt, scaled to
+    `units`; None when absent or captured from different kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    sha = sources_sha1()
+    for line in open(path):
+        if line.startswith("#") or "=" not in line:
+            continue
+        kv = dict(tok.split("=", 1) for tok in line.split())
+        if (kv.get("kernel") == "k_select" and kv.get("workload") == workload
+                and abs(float(kv.get("read", "-1")) - read) < 1e-9 and kv.get("sources_sha1") == sha):
+            return int(kv["bytes_per_unit"]) * units
+    return None
+
+
 # ---------------------------------------------------------------------------
 # clocks during the timed region (nvidia-smi, read-only)
 
@@ -103,7 +134,7 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY, "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
 
@@ -412,13 +443,7 @@ def main(argv=None):
                "sample": "%d units (one KV head of sequence 0 at one decode step each), %.0f s, mode %s, fp64 numpy"
                          % (units, args.cpu_seconds, args.mode)}
 
-    traffic = None
-    tp = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tp):
-        tr = json.load(open(tp))
-        key = "%s:%s:%s" % (args.workload, args.read, "k_select")
-        if key in tr:
-            traffic = tr[key]
+    traffic = select_traffic(args.workload, args.read, w.B * w.Hkv)
 
     if rank == 0:
         line = {
