@@ -187,6 +187,22 @@ SA_API sa_status sa_select(const sa_shape* shape, const sa_select_params* params
                     const sa_selection* out, float scale, void* ws, size_t ws_bytes,
                     void* stream);
 
+/* sa_select without a workspace, for callers that cannot allocate device
+ * memory (for example code that runs inside an allocator's hooks or in a
+ * plug-in restricted to the buffers it is given).  The paper has no
+ * counterpart: this is a deployment convenience.  Same inputs, outputs and
+ * results as sa_select; the scratch is a fixed 8 MiB array inside the
+ * library (present on every device that loads it), so shapes whose
+ * selection workspace exceeds 8 MiB return SA_ERR_WORKSPACE.  The array is
+ * shared by all calls on a device: the call clears its completion counters
+ * with cudaMemsetAsync on `stream` first, and calls that overlap on the GPU
+ * race and must not be issued.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture.  Allocates nothing. */
+SA_API sa_status sa_select_noalloc(const sa_shape* shape, const sa_select_params* params, const void* q,
+                                   const sa_stats* stats, const void* k, const void* v,
+                                   const sa_selection* out, float scale, void* stream);
+
 /* Sparse decode: gathers I (and the draws), one fp32 online softmax over the
  * G query heads of each unit, folds in the mode's residual, writes
  * out [B, Hq, d] f32. */

@@ -59,8 +59,8 @@ class sa_decode_params(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int), ("lam", ctypes.c_float), ("scale", ctypes.c_float)]
 
 
-EXPORTS = ("sa_workspace_size", "sa_prefill_stats", "sa_block_summaries", "sa_select", "sa_decode",
-           "sa_step", "sa_dense_decode", "sa_status_string")
+EXPORTS = ("sa_workspace_size", "sa_prefill_stats", "sa_block_summaries", "sa_select", "sa_select_noalloc",
+           "sa_decode", "sa_step", "sa_dense_decode", "sa_status_string")
 
 _LIB = None
 
@@ -80,12 +80,14 @@ def _lib():
         lib.sa_prefill_stats.argtypes = [sh, P, P, P, st, F, P, S, P]
         lib.sa_block_summaries.argtypes = [sh, P, I, I, P, P, P]
         lib.sa_select.argtypes = [sh, sp, P, st, P, P, sel, F, P, S, P]
+        lib.sa_select_noalloc.argtypes = [sh, sp, P, st, P, P, sel, F, P]
         lib.sa_decode.argtypes = [sh, dp, sp, P, P, P, st, sel, P, P, S, P]
         lib.sa_step.argtypes = [sh, dp, sp, P, P, P, st, sel, P, P, S, P]
         lib.sa_dense_decode.argtypes = [sh, P, P, P, P, F, P, S, P]
         lib.sa_status_string.argtypes = [I]
         lib.sa_status_string.restype = ctypes.c_char_p
-        for f in ("sa_prefill_stats", "sa_block_summaries", "sa_select", "sa_decode", "sa_step", "sa_dense_decode"):
+        for f in ("sa_prefill_stats", "sa_block_summaries", "sa_select", "sa_select_noalloc", "sa_decode", "sa_step",
+                  "sa_dense_decode"):
             getattr(lib, f).restype = I
         _LIB = lib
     return _LIB
