@@ -12,12 +12,19 @@ Readings where the pages are silent:
   * score_c = sum_{h in group} q_h . kbar_c (the 1/sqrt(d) factor is positive
     and common, so it does not change the ranking and is left out);
   * ties go to the lower block index: rank by (score desc, index asc);
-  * the decision is taken in fp64.
+  * the decision is taken in fp64 on the exact score rounded once: the real
+    number sum_h sum_e q_he kbar_ce (q and kbar are bf16 / fp32 values, so
+    each product is exact in fp64) correctly rounded by fsum.  Equal real
+    scores therefore compare equal whatever the order of the terms, and two
+    blocks with identical summaries always tie.
 
 Parity pins (tests/test_oracle_select.py): brute force over all subsets on
 tiny inputs, sorting with Python's own sort, all-equal scores, planted blocks
-whose rank is known.
+whose rank is known, scores against exact rational arithmetic, ties between
+identical and permuted summaries.
 """
+import math
+
 import numpy as np
 
 BLOCK = 16
@@ -31,9 +38,15 @@ def candidate_blocks(L, sink, local):
 
 
 def block_scores(q, blk_mean, cand):
-    """q [G, d], blk_mean [nb, d] -> score of each candidate block (fp64)."""
-    per_head = q @ blk_mean[cand].T            # [G, n_cand]
-    return per_head.sum(axis=0)
+    """q [G, d], blk_mean [nb, d] (bf16 / fp32 values) -> score of each
+    candidate block: sum over heads and dims of q_he * kbar_ce, every product
+    exact in fp64, summed exactly and rounded once (math.fsum)."""
+    q = np.asarray(q, dtype=np.float64)
+    blk_mean = np.asarray(blk_mean, dtype=np.float64)
+    out = np.empty(len(cand), dtype=np.float64)
+    for i, c in enumerate(cand):
+        out[i] = math.fsum((q * blk_mean[c]).ravel())
+    return out
 
 
 def top_blocks(scores, cand, k):

@@ -1,5 +1,7 @@
-"""Pins for oracle.select: brute-force ranking, ties, known block order."""
+"""Pins for oracle.select: brute-force ranking, ties, known block order,
+exact scores."""
 import itertools
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -71,3 +73,53 @@ def test_candidate_ranges_and_index_sets():
     idx2 = S.index_set(64, 20, 10, [2])
     assert S.tail_set(64, idx2).tolist() == [20, 21, 22, 23, 24, 25, 26, 27, 28, 29, 30, 31,
                                               48, 49, 50, 51, 52, 53]
+
+
+def _f32(a):
+    return np.asarray(a, dtype=np.float32).astype(np.float64)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_scores_are_the_exact_value_rounded_once(seed):
+    # rational arithmetic is exact; float(Fraction) rounds once to nearest
+    rng = np.random.default_rng(100 + seed)
+    G, d, nb = 3, 24, 9
+    q = _f32(rng.standard_normal((G, d)) * 2.0 ** rng.integers(-20, 20, (G, d)))
+    blk = _f32(rng.standard_normal((nb, d)) * 2.0 ** rng.integers(-20, 20, (nb, d)))
+    cand = np.arange(nb)
+    got = S.block_scores(q, blk, cand)
+    for i in range(nb):
+        exact = sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(q.ravel(), np.tile(blk[i], G)))
+        assert got[i] == float(exact)
+
+
+def test_identical_summaries_tie_anywhere():
+    # the same summary row at many positions: equal scores, lowest indices win
+    # (two heads, d = 64, 182 rows: a shape where a plain fp64 matrix product
+    # rounds identical rows differently depending on their position)
+    rng = np.random.default_rng(7)
+    G, d, nb = 2, 64, 182
+    q = _f32(rng.standard_normal((G, d)))
+    rows = _f32(rng.standard_normal((5, d)))
+    pick = rng.integers(0, 5, nb)
+    blk = rows[pick]
+    cand = np.arange(nb)
+    sc = S.block_scores(q, blk, cand)
+    for r in range(5):
+        assert len(set(sc[pick == r].tolist())) == 1
+    best = max(range(5), key=lambda r: sc[pick == r][0])
+    want = np.flatnonzero(pick == best)[:3]
+    assert S.top_blocks(sc, cand, 3).tolist() == want.tolist()
+
+
+def test_permuted_summaries_tie_under_a_constant_query():
+    # q_he = const for all e: a permutation of a row leaves the exact score
+    # unchanged, so every permutation ties with the original
+    rng = np.random.default_rng(8)
+    d = 64
+    q = _f32(np.full((2, d), 0.3))
+    row = _f32(rng.standard_normal(d) * 2.0 ** rng.integers(-30, 30, d))
+    blk = np.stack([row[rng.permutation(d)] for _ in range(20)])
+    sc = S.block_scores(q, blk, np.arange(20))
+    assert len(set(sc.tolist())) == 1
+    assert S.top_blocks(sc, np.arange(20), 4).tolist() == [0, 1, 2, 3]
