@@ -8,8 +8,14 @@ One step = one decode step of the whole batch through the hot path: block
 scoring + exact top-k (sa_select, one kernel) then gather + online softmax +
 residual fold + split combine (sa_decode, one kernel).  Inputs (KV cache,
 prefill statistics, queries) are resident in HBM before timing; L2 is flushed
-(256 MB write) before every timed step and the flush is outside the timed
-events.  Prints ONE JSON line on rank 0.
+before every timed step, outside the timed events: 256 MB written, then
+another 256 MB read, so that no line of the step's inputs is cached and no
+dirty line of the flush is left to be written back during the step.  After
+the flush the GPU spins (untimed) for ~0.1 ms so that the
+step's launches are queued before its first event: the events then measure
+the device time of the step, not the host's launch latency (which the e2e
+figure, timed through the public API with host buffers, does include).
+Prints ONE JSON line on rank 0.
 
 --impl reference times the fp64 CPU oracle (the reference arm of this build)
 on a bounded sample of the same workload, on the host cores.
@@ -31,6 +37,7 @@ if ROOT not in sys.path:
 METRIC = "decode-attn tokens/sec & HBM GB/s (% of roofline) at 32K, 1% read, vs dense"
 UNIT = "tokens/s"
 FLUSH_BYTES = 256 << 20
+SETTLE_CYCLES = 200_000          # GPU spin after each flush, ~0.1 ms at 2 GHz (untimed)
 
 
 def parse_args(argv=None):
@@ -269,7 +276,7 @@ def workload_config(w, sg, args):
     return {"workload": "%s decode: B%d, %dq/%dkv heads, d%d, L%d, %s, %g%% read (sink %d + window %d + %d blocks of 16 = %d tokens)"
             % (w.name, w.B, w.Hq, w.Hkv, w.d, w.L, w.dtype, 100 * args.read, w.sink, w.local, sg["kk"], sg["n_i"]),
             "global_batch": w.B * args.gpus, "seq_len": w.L, "mode": args.mode, "k_blocks": sg["kk"],
-            "read_tokens": sg["n_i"], "l2": "flushed before every timed step (256 MB write, untimed)",
+            "read_tokens": sg["n_i"], "l2": "flushed before every timed step (256 MB write + 256 MB read, untimed)",
             "parallelism": "replicas (dp%d, no collective on the data path)" % args.gpus}
 
 
@@ -312,6 +319,11 @@ def main(argv=None):
     sel = sa.select(Q[0], stats, sps[0])
     out = torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def flush_l2():
+        flush.zero_()                       # evicts the cached inputs ...
+        torch.sum(flush_r)                  # ... and the dirty lines of the write
     stream = torch.cuda.current_stream()
 
     def step(t, mode):
@@ -323,7 +335,8 @@ def main(argv=None):
         lists of event-pair durations (ms)."""
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_events)] for _ in range(n)]
         for t in range(n):
-            flush.zero_()
+            flush_l2()
+            torch.cuda._sleep(SETTLE_CYCLES)
             fn(t, evs[t])
         torch.cuda.synchronize()
         return [[evs[t][i].elapsed_time(evs[t][i + 1]) for i in range(n_events - 1)] for t in range(n)]
@@ -352,7 +365,7 @@ def main(argv=None):
 
     # warm-up (untimed)
     for t in range(args.warmup):
-        flush.zero_()
+        flush_l2()
         step(t, args.mode)
     torch.cuda.synchronize()
 

@@ -228,6 +228,16 @@ SA_API sa_status sa_step(const sa_shape* shape, const sa_decode_params* dparams,
 SA_API sa_status sa_dense_decode(const sa_shape* shape, const void* q, const void* k, const void* v,
                           float* out, float scale, void* ws, size_t ws_bytes, void* stream);
 
+/* Bounded waits.  The selection kernel streams the block summaries into
+   shared memory with bulk copies and waits on each one for at most about two
+   seconds; a CTA whose wait runs out marks its unit's selection invalid
+   (blk_idx row all -1, samp_count 0, n_rescored -1) and returns.  *count gets
+   the number of such CTAs on the current device since the library was loaded
+   (cumulative; compare two readings).  Synchronous with respect to the device
+   (it reads a device counter).  The method has no counterpart: this is the
+   library's guard against a copy that never lands. */
+SA_API sa_status sa_wait_timeouts(unsigned* count);
+
 /* Static string for a status code. */
 SA_API const char* sa_status_string(sa_status status);
 

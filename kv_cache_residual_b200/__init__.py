@@ -60,7 +60,7 @@ class sa_decode_params(ctypes.Structure):
 
 
 EXPORTS = ("sa_workspace_size", "sa_prefill_stats", "sa_block_summaries", "sa_select", "sa_select_noalloc",
-           "sa_decode", "sa_step", "sa_dense_decode", "sa_status_string")
+           "sa_decode", "sa_step", "sa_dense_decode", "sa_wait_timeouts", "sa_status_string")
 
 _LIB = None
 
@@ -84,6 +84,8 @@ def _lib():
         lib.sa_decode.argtypes = [sh, dp, sp, P, P, P, st, sel, P, P, S, P]
         lib.sa_step.argtypes = [sh, dp, sp, P, P, P, st, sel, P, P, S, P]
         lib.sa_dense_decode.argtypes = [sh, P, P, P, P, F, P, S, P]
+        lib.sa_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+        lib.sa_wait_timeouts.restype = I
         lib.sa_status_string.argtypes = [I]
         lib.sa_status_string.restype = ctypes.c_char_p
         for f in ("sa_prefill_stats", "sa_block_summaries", "sa_select", "sa_select_noalloc", "sa_decode", "sa_step",
@@ -272,3 +274,11 @@ def dense_decode(q, k, v, scale=0.0, out=None, stream=None):
     _check(_lib().sa_dense_decode(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(out), float(scale),
                                   _ptr(ws), ws.numel(), _stream(stream)), "sa_dense_decode")
     return out
+
+
+def wait_timeouts():
+    """Selection CTAs on the current device that gave up waiting on a bulk copy
+    since the library was loaded (cumulative; see sa_wait_timeouts)."""
+    c = ctypes.c_uint(0)
+    _check(_lib().sa_wait_timeouts(ctypes.byref(c)), "sa_wait_timeouts")
+    return int(c.value)

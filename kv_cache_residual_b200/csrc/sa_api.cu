@@ -61,6 +61,11 @@ float resolve_scale(float scale, int d) { return scale > 0.f ? scale : (float)(1
 
 extern "C" {
 
+sa_status sa_wait_timeouts(unsigned* count) {
+    if (count == nullptr) return SA_ERR_INVALID_ARG;
+    return sa::select_wait_timeouts(count) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
 const char* sa_status_string(sa_status s) {
     switch (s) {
         case SA_OK: return "ok";

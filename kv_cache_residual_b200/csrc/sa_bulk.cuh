@@ -1,0 +1,80 @@
+// Bulk global -> shared copies completed on shared-memory barriers (sm_90+
+// `cp.async.bulk` with `mbarrier::complete_tx`), and a bounded wait on them.
+//
+// One thread arms a barrier with the byte count it expects and issues the
+// copy; consumers wait on the barrier's phase.  No multicast: every copy lands
+// in the issuing CTA's own shared memory.
+//
+// Every wait is bounded.  A wait that has not seen its phase complete after
+// kWaitNs of %globaltimer gives up and returns false; the CTA then bumps this
+// translation unit's timeout counter once (read from the host by the unit
+// that owns the kernel), drains the copies it has in flight (again bounded)
+// and returns with its outputs marked invalid.
+#pragma once
+
+#include <stdint.h>
+
+namespace sa {
+
+constexpr uint64_t kWaitNs = 2000000000ull;        // give up on a copy after 2 s
+constexpr uint64_t kDrainNs = 500000000ull;        // and on each in-flight copy after 0.5 s
+
+// waits abandoned in this translation unit since the host last read them
+static __device__ unsigned g_wait_timeouts;
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+// makes barrier initialisation visible to the async (bulk-copy) proxy
+__device__ __forceinline__ void mbar_init_fence() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// the calling thread's arrival, announcing `bytes` of copies to complete
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// `bytes` (multiple of 16, both addresses 16-byte aligned) from global to this
+// CTA's shared memory, completing on `bar`
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits for the phase with parity `parity` to complete; false after `limit_ns`.
+// (try_wait itself returns after a bounded, implementation-defined time.)
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns = kWaitNs) {
+    if (mbar_try(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try(bar, parity)) return true;
+        if (global_ns() - t0 > limit_ns) return false;
+    }
+}
+
+}  // namespace sa

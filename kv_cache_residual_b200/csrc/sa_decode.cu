@@ -641,7 +641,8 @@ static cudaError_t stream_launch(const Dims& d, dim3 grid, const void* q, const 
                                  const SetGeom& sg, int tpc, int nchunk, int rec, float scale, float lambda,
                                  char* part, char* cnt, float* out, bool pdl, cudaStream_t s) {
     constexpr size_t sm = stream_smem<D, G, MODE>();
-    cudaError_t e = cudaFuncSetAttribute(k_stream_tc<D, G, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    static std::atomic<unsigned long long> opted{0};
+    cudaError_t e = opt_in_smem(k_stream_tc<D, G, MODE>, sm, opted);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;

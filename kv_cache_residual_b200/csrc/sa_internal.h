@@ -9,6 +9,8 @@
 
 #include "sa_decode.h"
 
+#include <atomic>
+
 namespace sa {
 
 constexpr int kSmTarget = 148 * 4;   // CTAs to aim for: 4 per SM on B200
@@ -182,7 +184,23 @@ struct SelectArgs {
     const void* q; sa_stats st; const void* k; const void* v;
     sa_selection sel; sa_select_params sp; float scale; char* ws;
 };
+// Raises a kernel's dynamic shared-memory limit to `bytes` once per device
+// (the attribute lives in the device's context; `done` holds one bit per
+// device id < 64, larger ids set it on every call).
+template <typename K>
+inline cudaError_t opt_in_smem(K kernel, size_t bytes, std::atomic<unsigned long long>& done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = dev < 64 ? 1ull << dev : 0ull;
+    if (bit != 0ull && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
+
 cudaError_t launch_select(const Dims& d, const SelectPlan& p, const SelectArgs& a, cudaStream_t s);
+cudaError_t select_wait_timeouts(unsigned* count);    // CTAs of the selection kernel that gave up a wait
 
 struct DecodeArgs {
     const void* q; const void* k; const void* v; sa_stats st; sa_selection sel;

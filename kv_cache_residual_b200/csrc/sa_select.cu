@@ -18,6 +18,7 @@
 //           to the exact top k; if more than k do, those are rescored in fp64
 //           and ranked exactly.  The decision is therefore the fp64 one.
 //   draws : tail positions for the sampling estimator (SplitMix64 counters).
+#include "sa_bulk.cuh"
 #include "sa_common.cuh"
 #include "sa_internal.h"
 
@@ -26,7 +27,21 @@ namespace sa {
 constexpr int kSmemKeys = 4096;     // candidate keys held in shared memory (16 KB)
 constexpr int kBandCap = 512;       // band members ranked in shared memory
 constexpr int kWarpTopK = 32;       // largest k of the warp-argmax path
-constexpr int kRowsPer = 8;         // rows per lane group per scan step
+
+// The scan's shared-memory ring: kStages stages of kStageBytes, each a run of
+// SR consecutive block-summary rows of RB bytes; a warp scores R rows per
+// lane group of each stage (the stage is SR = kWarps * GPW * R rows).
+template <typename T, int D>
+struct ScanRing {
+    static constexpr int kStages = 5;
+    static constexpr int kStageBytes = 16384;
+    static constexpr int kRingBytes = kStages * kStageBytes;
+    static constexpr int RB = D * (int)sizeof(T);
+    static constexpr int SR = kStageBytes / RB;
+    static constexpr int R = SR / (kWarps * Geom<T, D>::GPW);
+    static constexpr size_t kSmem = (size_t)kRingBytes + 8 * kStages;      // ring + its barriers
+    static_assert(R >= 1 && (R & (R - 1)) == 0, "stage geometry");
+};
 
 __device__ __forceinline__ uint32_t fkey(float y) {
     const uint32_t b = __float_as_uint(y + 0.0f);   // -0 -> +0
@@ -49,6 +64,16 @@ __device__ __forceinline__ int comp_index(unsigned long long c) { return (int)(~
 __device__ __forceinline__ unsigned long long shfl_xor_u64(unsigned long long v, int off) {
     const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, off);
     const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), off);
+    return ((unsigned long long)hi << 32) | lo;
+}
+__device__ __forceinline__ unsigned long long shfl_u64(unsigned long long v, int src) {
+    const uint32_t lo = __shfl_sync(0xffffffffu, (uint32_t)v, src);
+    const uint32_t hi = __shfl_sync(0xffffffffu, (uint32_t)(v >> 32), src);
+    return ((unsigned long long)hi << 32) | lo;
+}
+__device__ __forceinline__ unsigned long long shfl_up_u64(unsigned long long v, int d) {
+    const uint32_t lo = __shfl_up_sync(0xffffffffu, (uint32_t)v, d);
+    const uint32_t hi = __shfl_up_sync(0xffffffffu, (uint32_t)(v >> 32), d);
     return ((unsigned long long)hi << 32) | lo;
 }
 __device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
@@ -220,9 +245,38 @@ __device__ void warp_topk(const uint32_t* keys, int n, int kk, unsigned long lon
     __syncthreads();
 }
 
+// Merges the warps' lists s_cand[w kk .. w kk + kk) (each sorted descending,
+// 0 = empty) into the CTA's best kk in rank order in s_list: an entry's rank is
+// its position in its own list plus the count of larger entries in the others
+// (the words are distinct, so the ranks of the best kk are exactly 0..kk-1).
+__device__ void merge_warp_lists(const unsigned long long* s_cand, int kk, unsigned long long* s_list) {
+    __syncthreads();
+    const int t = threadIdx.x;
+    if (t < kWarps * kk) {
+        const unsigned long long c = s_cand[t];
+        if (c != 0ull) {
+            const int w = t / kk;
+            int rank = t - w * kk;
+            for (int v = 0; v < kWarps; ++v) {
+                if (v == w) continue;
+                const unsigned long long* l = s_cand + v * kk;
+                int lo = 0, hi = kk;                 // first entry of list v below c
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (l[mid] > c) lo = mid + 1; else hi = mid;
+                }
+                rank += lo;
+            }
+            if (rank < kk) s_list[rank] = c;
+        }
+    }
+    __syncthreads();
+}
+
 // Sorts s_list[0..kk) (kk <= 32) by block index and writes c_lo + index in
 // ascending order (one warp, bitonic network over the 32 lanes).
-__device__ void emit_sorted_list(const unsigned long long* s_list, int kk, int c_lo, int32_t* out_idx) {
+__device__ void emit_sorted_list(const unsigned long long* s_list, int kk, int c_lo, int32_t* out_idx,
+                                 int* s_sorted) {
     if (threadIdx.x >= 32) return;
     const int lane = threadIdx.x;
     int v = lane < kk ? comp_index(s_list[lane]) : 0x7fffffff;
@@ -236,36 +290,81 @@ __device__ void emit_sorted_list(const unsigned long long* s_list, int kk, int c
             v = (lower == up) ? min(v, o) : max(v, o);
         }
     }
-    if (lane < kk) out_idx[lane] = c_lo + v;
+    if (lane < kk) {
+        out_idx[lane] = c_lo + v;
+        s_sorted[lane] = c_lo + v;
+    }
 }
 
-// fp64 scores of the band members s_bidx[0..nb) into s_bx (a warp per member,
-// four members' rows in flight per warp).
-template <typename T, int D>
-__device__ void rescore_members(const T* bm, const int* s_bidx, int nb, const double* s_q64, double* s_bx) {
+// s + p with the rounding error of the addition carried into c (error-free
+// two-sum; explicit roundings so nothing is contracted or reassociated)
+__device__ __forceinline__ void two_sum_acc(double& s, double& c, double p) {
+    const double t = __dadd_rn(s, p);
+    const double bp = __dsub_rn(t, s);
+    const double err = __dadd_rn(__dsub_rn(s, __dsub_rn(t, bp)), __dsub_rn(p, bp));
+    s = t;
+    c = __dadd_rn(c, err);
+}
+
+// Exact block score sum_h sum_e q_he kbar_ce rounded once, for M rows at a
+// time (warp-collective; lane 0 holds the results).  Each product of two bf16
+// / fp32 values is exact in fp64; the products are added in double-double
+// (two-sum, errors summed apart), lanes combined the same way, and the two
+// parts rounded together, which is the correctly rounded sum unless the exact
+// sum lies within ~n^2 2^-106 sum|terms| of a rounding boundary.  Identical
+// rows always get identical scores.
+template <typename T, int D, int G, int M>
+__device__ __forceinline__ void exact_scores(const T* const (&rows)[M], const bool (&live)[M], const float* s_qh,
+                                             double (&x)[M]) {
+    const int lane = threadIdx.x & 31;
+    float k[M][D / 32];
+#pragma unroll
+    for (int m = 0; m < M; ++m)
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) k[m][i] = live[m] ? to_f32<T>(rows[m][lane + 32 * i]) : 0.f;
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+        double s = 0.0, c = 0.0;
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) {
+            const double kv = (double)k[m][i];
+#pragma unroll
+            for (int h = 0; h < G; ++h) two_sum_acc(s, c, __dmul_rn((double)s_qh[h * D + lane + 32 * i], kv));
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const double so = __shfl_xor_sync(0xffffffffu, s, off);
+            const double co = __shfl_xor_sync(0xffffffffu, c, off);
+            two_sum_acc(s, c, so);
+            c = __dadd_rn(c, co);
+        }
+        x[m] = __dadd_rn(s, c) + 0.0;          // -0 -> +0
+    }
+}
+
+// exact scores of the band members s_bidx[0..nb) into s_bx (a warp per
+// member, four members' rows in flight per warp)
+template <typename T, int D, int G>
+__device__ void rescore_members(const T* bm, const int* s_bidx, int nb, const float* s_qh, double* s_bx) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int j0 = warp * 4; j0 < nb; j0 += kWarps * 4) {
-        float v[4][D / 32];
+        const T* rows[4];
+        bool live[4];
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-            const int j = j0 + m;
-#pragma unroll
-            for (int e = 0; e < D / 32; ++e)
-                v[m][e] = j < nb ? to_f32<T>(bm[(size_t)s_bidx[j] * D + lane + 32 * e]) : 0.f;
+            live[m] = j0 + m < nb;
+            rows[m] = bm + (size_t)(live[m] ? s_bidx[j0 + m] : 0) * D;
         }
+        double x[4];
+        exact_scores<T, D, G, 4>(rows, live, s_qh, x);
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            double x = 0.0;
-#pragma unroll
-            for (int e = 0; e < D / 32; ++e) x += s_q64[lane + 32 * e] * (double)v[m][e];
-            x = group_sum_f64<32>(x) + 0.0;        // -0 -> +0
-            if (lane == 0 && j0 + m < nb) s_bx[j0 + m] = x;
-        }
+        for (int m = 0; m < 4; ++m)
+            if (lane == 0 && live[m]) s_bx[j0 + m] = x[m];
     }
 }
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* __restrict__ kbar_absmax,
          int Hq, int Hkv, int L, SetGeom sg, int rows, int nss,
          float* __restrict__ scores, unsigned long long* __restrict__ xkey,
@@ -273,20 +372,25 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
          int32_t* __restrict__ samp_idx, int32_t* __restrict__ samp_count, int32_t* __restrict__ n_rescored,
          int sample_b, int sample_cap, unsigned long long seed, int step) {
     using Gm = Geom<T, D>;
-    constexpr int EPC = Gm::EPC, CPR = Gm::CPR, NG = Gm::NG;
-    constexpr int R = kRowsPer;
+    constexpr int EPC = Gm::EPC, CPR = Gm::CPR;
+    using Ring = ScanRing<T, D>;
+    constexpr int R = Ring::R;
     static_assert(CPR >= R, "transposed reduction needs at least one lane per row");
     __shared__ unsigned hist[kThreads];
     __shared__ int sw[kWarps + 1];
     __shared__ int s_digit, s_rem, s_nb;
-    __shared__ double s_q64[D];
+    __shared__ float s_qh[G * D];          // the group's queries (exact), for fp64 rescoring
     __shared__ float s_qsum;
     __shared__ uint32_t s_keys[kSmemKeys];
-    __shared__ int s_bidx[kBandCap];
-    __shared__ double s_bx[kBandCap];
-    __shared__ unsigned char s_bsel[kBandCap];
-    __shared__ unsigned long long s_cand[kWarps * kWarpTopK];
-    __shared__ unsigned long long s_list[kWarpTopK];
+    __shared__ int s_sorted[kWarpTopK];
+    // the scan's copy ring; reused for the top-k / band arrays once the scan is done
+    extern __shared__ __align__(128) unsigned char s_ring[];
+    uint64_t* s_bar = reinterpret_cast<uint64_t*>(s_ring + Ring::kRingBytes);
+    unsigned long long* s_cand = reinterpret_cast<unsigned long long*>(s_ring);          // kWarps * kWarpTopK
+    unsigned long long* s_list = s_cand + kWarps * kWarpTopK;                            // kWarpTopK
+    double* s_bx = reinterpret_cast<double*>(s_list + kWarpTopK);                        // kBandCap
+    int* s_bidx = reinterpret_cast<int*>(s_bx + kBandCap);                               // kBandCap
+    unsigned char* s_bsel = reinterpret_cast<unsigned char*>(s_bidx + kBandCap);         // kBandCap
 
     // a decode kernel launched as a programmatic dependent may start as soon as
     // every CTA of this grid has begun; it waits for this grid's completion
@@ -302,14 +406,43 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
     float* sc = scores + (size_t)u * (n > 0 ? n : 1);
     // one CTA per unit: the scores never leave shared memory
     const bool local = (nss == 1) && n <= kSmemKeys;
+    // k <= 32 with one CTA per unit: each warp keeps its best k while scanning
+    const bool run_topk = local && kk > 0 && kk < n && kk <= kWarpTopK;
+    const float amax = kbar_absmax[u];
 
     // ---- scan: fp32 scores of this CTA's slice -------------------------------
+    // The slice's block summaries are contiguous: thread 0 streams them through
+    // a ring of kStages shared-memory stages with bulk copies, kStages stages
+    // in flight; all warps score each stage as it lands.
+    const int r0 = split * rows, r1 = min(n, r0 + rows);
+    const int nrows = max(0, r1 - r0);
+    const int nst = (nrows + Ring::SR - 1) / Ring::SR;
+    const char* src0 = reinterpret_cast<const char*>(blk_mean + ((size_t)u * nb + sg.c_lo + r0) * D);
+    const uint32_t ring = smem_addr(s_ring), bar0 = smem_addr(s_bar);
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int j = 0; j < Ring::kStages; ++j) mbar_init(bar0 + 8 * j, 1);
+        mbar_init_fence();
+    }
+    __syncthreads();
+    auto issue = [&](int j) {                      // thread 0
+        if (j < nst) {
+            const uint32_t bytes = (uint32_t)min(Ring::SR, nrows - j * Ring::SR) * Ring::RB;
+            const uint32_t bar = bar0 + 8 * (j % Ring::kStages);
+            mbar_arrive_expect_tx(bar, bytes);
+            bulk_g2s(ring + (j % Ring::kStages) * Ring::kStageBytes, src0 + (size_t)j * Ring::kStageBytes, bytes, bar);
+        }
+    };
+    if (threadIdx.x == 0)
+        for (int j = 0; j < Ring::kStages; ++j) issue(j);
+    __syncwarp();
+
+    bool failed = false;
     {
         float qb[EPC];
-        double q64[EPC];
         float qa = 0.f;
 #pragma unroll
-        for (int e = 0; e < EPC; ++e) { qb[e] = 0.f; q64[e] = 0.0; }
+        for (int e = 0; e < EPC; ++e) qb[e] = 0.f;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
             float f[EPC];
@@ -317,48 +450,42 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
 #pragma unroll
             for (int e = 0; e < EPC; ++e) {
                 qb[e] += f[e];
-                q64[e] += (double)f[e];
                 qa += fabsf(f[e]);
             }
-        }
-        // for the top-k (whichever CTA ends up doing it): the fp64 group query
-        // and sum_i sum_h |q_hi| for the rounding bound, from lane group 0
-        qa = group_sum<CPR>(qa);
-        if (lane < CPR && warp == 0) {
+            // for the top-k (whichever CTA ends up doing it): the group's
+            // queries and sum_i sum_h |q_hi| for the rounding bound
+            if (warp == 0 && lane < CPR) {
 #pragma unroll
-            for (int e = 0; e < EPC; ++e) s_q64[li * EPC + e] = q64[e];
-            if (lane == 0) s_qsum = qa;
-        }
-        const T* base = blk_mean + ((size_t)u * nb + sg.c_lo) * D + li * EPC;
-        const int r0 = split * rows, r1 = min(n, r0 + rows);
-        const int gsub = lane / CPR;
-        // warp-uniform loop: a warp step covers R x GPW rows (R per lane group);
-        // the next step's rows are loaded before this step's are reduced, so
-        // 2R rows per lane group are in flight; rows past the end load nothing
-        auto loadR = [&](int wr, uint4 (&w)[R]) {
-#pragma unroll
-            for (int j = 0; j < R; ++j) {
-                const int r = wr + j * Gm::GPW + gsub;
-                w[j] = (r < r1) ? ld_stream16(base + (size_t)r * D) : make_uint4(0, 0, 0, 0);
+                for (int e = 0; e < EPC; ++e) s_qh[h * D + li * EPC + e] = f[e];
             }
-        };
-        int wr = r0 + warp * R * Gm::GPW;
-        uint4 cur[R];
-        loadR(wr, cur);
-        for (; wr < r1; wr += R * NG) {
-            uint4 nxt[R];
-            loadR(wr + R * NG, nxt);
+        }
+        qa = group_sum<CPR>(qa);
+        if (warp == 0 && lane == 0) s_qsum = qa;
+        const int gsub = lane / CPR;
+        // this warp's rows of a stage: warp * R * GPW + j * GPW + gsub, j < R
+        const int wrow = warp * R * Gm::GPW + gsub;
+        // running best kk of the rows this warp scored: lane i < kk holds the
+        // i-th best (score key, ~index) word, 0 when empty; thr = the kk-th
+        unsigned long long best = 0ull, thr = 0ull;
+        int j = 0;
+        for (; j < nst; ++j) {
+            const bool ok = mbar_wait(bar0 + 8 * (j % Ring::kStages), (uint32_t)(j / Ring::kStages) & 1u);
+            const unsigned char* sb = s_ring + (size_t)(j % Ring::kStages) * Ring::kStageBytes;
+            const int rows_j = min(Ring::SR, nrows - j * Ring::SR);
             // lane partial dot of each row: packed FMAs over element pairs,
             // then the two halves added
             float x[R];
 #pragma unroll
-            for (int j = 0; j < R; ++j) {
+            for (int jj = 0; jj < R; ++jj) {
+                const int rr = wrow + jj * Gm::GPW;
+                const uint4 w = (rr < rows_j) ? *reinterpret_cast<const uint4*>(sb + (size_t)rr * Ring::RB + li * 16)
+                                              : make_uint4(0, 0, 0, 0);
                 float f[EPC];
-                unpack<T>(cur[j], f);
+                unpack<T>(w, f);
                 float a0 = 0.f, a1 = 0.f;
 #pragma unroll
                 for (int e = 0; e < EPC; e += 2) ffma2(a0, a1, qb[e], qb[e + 1], f[e], f[e + 1]);
-                x[j] = a0 + a1;
+                x[jj] = a0 + a1;
             }
             // transposed reduction over the CPR lanes of the group: each of the
             // first log2(R) levels keeps half of the remaining rows, so the lane
@@ -368,23 +495,71 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
             for (int half = R / 2, off = CPR / 2; half > 0; half >>= 1, off >>= 1) {
                 const int bit = (li & off) ? 1 : 0;
 #pragma unroll
-                for (int j = 0; j < half; ++j) {
-                    const float send = bit ? x[j] : x[j + half];
-                    const float keep = bit ? x[j + half] : x[j];
-                    x[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                for (int jj = 0; jj < half; ++jj) {
+                    const float send = bit ? x[jj] : x[jj + half];
+                    const float keep = bit ? x[jj + half] : x[jj];
+                    x[jj] = keep + __shfl_xor_sync(0xffffffffu, send, off);
                 }
                 row = 2 * row + bit;
             }
 #pragma unroll
             for (int off = CPR / (2 * R); off > 0; off >>= 1) x[0] += __shfl_xor_sync(0xffffffffu, x[0], off);
-            const int r = wr + row * Gm::GPW + gsub;
-            if ((li & (CPR / R - 1)) == 0 && r < r1) {
-                if (local) s_keys[r] = fkey(x[0]);
+            const int rr = wrow + row * Gm::GPW;
+            const int r = r0 + j * Ring::SR + rr;
+            const bool owner = (li & (CPR / R - 1)) == 0 && rr < rows_j;
+            const uint32_t key = fkey(x[0]);
+            if (owner) {
+                if (local) s_keys[r] = key;
                 else sc[r] = x[0];
             }
-#pragma unroll
-            for (int j = 0; j < R; ++j) cur[j] = nxt[j];
+            // compiler barrier: without it the shared-memory traffic around the
+            // list update is scheduled so badly that the scan runs ~2.5x slower
+            // (measured); it emits no instruction
+            asm volatile("" ::: "memory");
+            if (run_topk) {
+                // rows that beat the warp's current kk-th best enter its list
+                const unsigned long long c = owner ? comp_key(key, r) : 0ull;
+                unsigned m = __ballot_sync(0xffffffffu, c > thr);
+                while (m) {
+                    const int src = __ffs(m) - 1;
+                    m &= m - 1;
+                    const unsigned long long cv = shfl_u64(c, src);
+                    const int pos = __popc(__ballot_sync(0xffffffffu, lane < kk && best > cv));
+                    const unsigned long long up = shfl_up_u64(best, 1);
+                    if (lane < kk && lane >= pos) best = (lane == pos) ? cv : up;
+                }
+                thr = shfl_u64(best, kk - 1);
+            }
+            // the stage is free once every warp has scored it
+            if (__syncthreads_or(!ok)) { failed = true; break; }
+            if (threadIdx.x == 0) issue(j + Ring::kStages);
+            // warp 0 reconverges here: its other lanes must not spin on the
+            // next stage's barrier while lane 0 still has the copy to issue
+            __syncwarp();
         }
+        if (failed) {
+            // give the copies still in flight a bounded time to land, then
+            // return with the unit's outputs marked invalid
+            if (threadIdx.x == 0) {
+                atomicAdd(&g_wait_timeouts, 1u);
+                for (int jj = j; jj < min(nst, j + Ring::kStages); ++jj)
+                    mbar_wait(bar0 + 8 * (jj % Ring::kStages), (uint32_t)(jj / Ring::kStages) & 1u, kDrainNs);
+            }
+        } else if (run_topk) {
+            // every thread is past the last stage's barrier: the ring is free
+            if (lane < kk) s_cand[warp * kk + lane] = best;
+        }
+    }
+    if (failed) {
+        int32_t* out_idx = blk_idx + (size_t)u * kb_stride;
+        for (int i = threadIdx.x; i < kb_stride; i += kThreads) out_idx[i] = -1;
+        if (threadIdx.x == 0) {
+            samp_count[u] = 0;
+            if (n_rescored != nullptr) n_rescored[u] = -1;
+        }
+        // keep the unit's completion count consistent for the next call
+        if (!local && last_cta_of_unit(cnt + u, nss)) reset_counter(cnt + u);
+        return;
     }
 
     // ---- gather the unit's scores ------------------------------------------------
@@ -415,12 +590,16 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
     // ---- top-k of the unit ------------------------------------------------------------
     int32_t* out_idx = blk_idx + (size_t)u * kb_stride;
     int rescored = 0;
+    bool sorted_smem = false;          // the chosen indices are also in s_sorted
     if (kk > 0 && kk < n) {
         auto k32 = [&](int i) -> uint32_t { return keys[i]; };
         const bool fast = kk <= kWarpTopK && n <= kSmemKeys;
         uint32_t thr;
         int need = 0;
-        if (fast) {
+        if (run_topk) {
+            merge_warp_lists(s_cand, kk, s_list);
+            thr = (uint32_t)(s_list[kk - 1] >> 32);
+        } else if (fast) {
             warp_topk(keys, n, kk, s_cand, s_list);
             thr = (uint32_t)(s_list[kk - 1] >> 32);
         } else {
@@ -434,13 +613,16 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
         //           <= (G + h + 2) 2^-24 sum_i qa_i * max|kbar|,
         // taken twice over for margin.
         constexpr int kDepth = EPC / 2 + 1 + ilog2(CPR);
-        const float E = (float)(G + kDepth + 2) * 0x1p-23f * s_qsum * kbar_absmax[u] * 1.0001f + 0x1p-100f;
+        const float E = (float)(G + kDepth + 2) * 0x1p-23f * s_qsum * amax * 1.0001f + 0x1p-100f;
         const uint32_t lo_key = fkey(fkey_inv(thr) - 2.f * E);
         int band = 0;
         for (int i = threadIdx.x; i < n; i += kThreads) band += (keys[i] >= lo_key) ? 1 : 0;
         band = block_sum(band, sw);
         if (band == kk) {
-            if (fast) emit_sorted_list(s_list, kk, sg.c_lo, out_idx);
+            if (fast) {
+                emit_sorted_list(s_list, kk, sg.c_lo, out_idx, s_sorted);
+                sorted_smem = true;
+            }
             else emit_topk<uint32_t>(k32, n, thr, need, kk, sg.c_lo, out_idx, sw);
         } else {
             // ambiguous: the exact top-k lies inside the band; rescore the band
@@ -453,7 +635,7 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
                 for (int i = threadIdx.x; i < n; i += kThreads)
                     if (keys[i] >= lo_key) s_bidx[atomicAdd(&s_nb, 1)] = i;
                 __syncthreads();
-                rescore_members<T, D>(bm, s_bidx, band, s_q64, s_bx);
+                rescore_members<T, D, G>(bm, s_bidx, band, s_qh, s_bx);
                 __syncthreads();
                 for (int j = threadIdx.x; j < band; j += kThreads) {
                     const double xj = s_bx[j];
@@ -481,9 +663,11 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
                 for (int i = warp; i < n; i += kWarps) {
                     unsigned long long key = 0ull;
                     if (keys[i] >= lo_key) {                        // warp-uniform branch
-                        double x = 0.0;
-                        for (int e = lane; e < D; e += 32) x += s_q64[e] * (double)to_f32<T>(bm[(size_t)i * D + e]);
-                        key = dkey(group_sum_f64<32>(x));
+                        const T* rows[1] = {bm + (size_t)i * D};
+                        const bool live[1] = {true};
+                        double x[1];
+                        exact_scores<T, D, G, 1>(rows, live, s_qh, x);
+                        key = dkey(x[0]);
                     }
                     if (lane == 0) xk[i] = key;
                 }
@@ -518,7 +702,7 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
             int lo_j = 0, hi_j = kk;             // count of j with g_j <= r
             while (lo_j < hi_j) {
                 const int mid = (lo_j + hi_j) >> 1;
-                const int gj = 16 * out_idx[mid] - sg.s_eff - 16 * mid;
+                const int gj = 16 * (sorted_smem ? s_sorted[mid] : out_idx[mid]) - sg.s_eff - 16 * mid;
                 if (gj <= r) lo_j = mid + 1; else hi_j = mid;
             }
             out_s[i] = sg.s_eff + r + 16 * lo_j;
@@ -530,7 +714,11 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
 template <typename T, int D, int G>
 static cudaError_t select_t(const Dims& d, const SelectPlan& p, const SelectArgs& a, cudaStream_t s) {
     char* ws = a.ws;
-    k_select<T, D, G><<<dim3(p.nss, d.U()), kThreads, 0, s>>>(
+    constexpr size_t smem = ScanRing<T, D>::kSmem;
+    static std::atomic<unsigned long long> opted{0};
+    cudaError_t e = opt_in_smem(k_select<T, D, G>, smem, opted);
+    if (e != cudaSuccess) return e;
+    k_select<T, D, G><<<dim3(p.nss, d.U()), kThreads, smem, s>>>(
         reinterpret_cast<const T*>(a.q), reinterpret_cast<const T*>(a.st.blk_mean), a.st.kbar_absmax,
         d.Hq, d.Hkv, d.L, p.g, p.rows_s, p.nss,
         reinterpret_cast<float*>(ws + p.off_scores), reinterpret_cast<unsigned long long*>(ws + p.off_xkey),
@@ -549,6 +737,10 @@ static cudaError_t select_g(const Dims& d, const SelectPlan& p, const SelectArgs
         case 8: return select_t<T, D, 8>(d, p, a, s);
     }
     return cudaErrorInvalidValue;
+}
+
+cudaError_t select_wait_timeouts(unsigned* count) {
+    return cudaMemcpyFromSymbol(count, g_wait_timeouts, sizeof(unsigned));
 }
 
 cudaError_t launch_select(const Dims& d, const SelectPlan& p, const SelectArgs& a, cudaStream_t s) {
