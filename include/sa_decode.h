@@ -100,8 +100,21 @@ typedef struct {
  *   sum_v       [B, Hkv, d]  f32  sum of the L cached values
  *   blk_mean    [B, Hkv, L/16, d] in dtype: 16-token block means, summed in
  *               fp64 and rounded once (nearest, ties to even)
- *   kbar_absmax [B, Hkv]     f32  max |blk_mean| (bounds the fp32 scoring
- *               error in sa_select)                                          */
+ *   kbar_absmax [B, Hkv]     f32  max |blk_mean| (reported; not needed by
+ *               sa_select)
+ *   blk_code    [B, Hkv, L/16, d] int8 and
+ *   blk_meta    [B, Hkv, L/16, 4] f32: the scan sketch of blk_mean relative
+ *               to mu_k, written with it.  Per block row kbar, t = kbar - mu_k
+ *               (fp64), s = fl32(max_e |t_e| / 127), code_e = clamp(rint(t_e /
+ *               s), -127, 127) (0 when s = 0), meta = {s, rn, kn, 0} with
+ *               rn >= ||t - s code||_2 and kn >= ||s code||_2 (f32 upper
+ *               bounds).  Centring shifts every block's score by one constant,
+ *               so the ranking is unchanged.  sa_select ranks the blocks on the
+ *               sketch with these bounds and certifies the top-k exactly from
+ *               blk_mean, so the selection equals the one on blk_mean alone; a
+ *               sketch not built from this blk_mean and mu_k (rebuild it with
+ *               sa_block_sketch when either changes) makes it wrong.  The
+ *               selector's own data structure: the pages have no counterpart. */
 typedef struct {
     float* mu_q;
     float* o_est;
@@ -111,6 +124,8 @@ typedef struct {
     float* sum_v;
     void* blk_mean;
     float* kbar_absmax;
+    int8_t* blk_code;
+    float* blk_meta;
 } sa_stats;
 
 /* Which tokens one step reads exactly, and how the tail is sampled.
@@ -141,9 +156,9 @@ typedef struct {
  *               min(k_blocks, n_cand) valid entries per unit, rest = -1
  *   samp_idx    [B, Hkv, sample_cap] int32: drawn token positions (draw order)
  *   samp_count  [B, Hkv] int32: draws per unit (0 unless sampling)
- *   n_rescored  [B, Hkv] int32 or NULL: candidates whose fp32 score fell
- *               within the rounding bound of the k-th and were rescored in
- *               fp64 (diagnostic)                                            */
+ *   n_rescored  [B, Hkv] int32 or NULL: candidates whose sketch interval
+ *               reached the k-th best lower bound and were rescored exactly
+ *               (0 when the sketch alone decided; diagnostic)                */
 typedef struct {
     int32_t* blk_idx;
     int32_t* samp_idx;
@@ -172,15 +187,28 @@ SA_API sa_status sa_prefill_stats(const sa_shape* shape, const void* q_ctx, cons
                            void* ws, size_t ws_bytes, void* stream);
 
 /* Block means of blocks [blk_begin, blk_end) of every unit into blk_mean
- * ([B, Hkv, L/16, d], dtype) and raises kbar_absmax [B, Hkv] to cover them
- * (for a cache that grew by whole blocks).  No workspace. */
+ * ([B, Hkv, L/16, d], dtype), their sketch relative to mu_k ([B, Hkv, d] f32,
+ * read only) into blk_code / blk_meta (layouts of sa_stats), and raises
+ * kbar_absmax [B, Hkv] to cover them (for a cache that grew by whole blocks;
+ * keep mu_k as it was when the other rows were sketched).  No workspace. */
 SA_API sa_status sa_block_summaries(const sa_shape* shape, const void* k, int blk_begin, int blk_end,
-                             void* blk_mean, float* kbar_absmax, void* stream);
+                                    void* blk_mean, float* kbar_absmax, const float* mu_k, int8_t* blk_code,
+                                    float* blk_meta, void* stream);
+
+/* Rebuilds the sketch (blk_code, blk_meta) of blocks [blk_begin, blk_end) of
+ * every unit from blk_mean relative to mu_k, for callers that write blk_mean
+ * or mu_k themselves (sa_prefill_stats and sa_block_summaries already write
+ * the sketch).  No workspace.  The pages have no counterpart (see blk_code in
+ * sa_stats). */
+SA_API sa_status sa_block_sketch(const sa_shape* shape, const void* blk_mean, const float* mu_k, int blk_begin,
+                                 int blk_end, int8_t* blk_code, float* blk_meta, void* stream);
 
 /* Selection of one decode step for every unit: block scores, exact top-k by
- * (score desc, block index asc) decided in fp64 (fp32 scan with a rounding
- * bound; candidates inside the bound are rescored in fp64), and the tail draws
- * for sampling.  k and v are read only for the CLT base sample (may be NULL
+ * (score desc, block index asc) on the exact score rounded once to fp64, and
+ * the tail draws for sampling.  The scan reads the int8 sketch (integer dot
+ * products with an int8 copy of the group query) and bounds each score's
+ * error; every candidate whose interval reaches the k-th best lower bound is
+ * rescored exactly from blk_mean.  k and v are read only for the CLT base sample (may be NULL
  * when clt_base == 0). */
 SA_API sa_status sa_select(const sa_shape* shape, const sa_select_params* params, const void* q,
                     const sa_stats* stats, const void* k, const void* v,

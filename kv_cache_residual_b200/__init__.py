@@ -41,7 +41,8 @@ class sa_shape(ctypes.Structure):
 
 class sa_stats(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("mu_q", "o_est", "log_z0", "mu_k", "sum_k", "sum_v", "blk_mean", "kbar_absmax")]
+                ("mu_q", "o_est", "log_z0", "mu_k", "sum_k", "sum_v", "blk_mean", "kbar_absmax", "blk_code",
+                 "blk_meta")]
 
 
 class sa_select_params(ctypes.Structure):
@@ -59,7 +60,8 @@ class sa_decode_params(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int), ("lam", ctypes.c_float), ("scale", ctypes.c_float)]
 
 
-EXPORTS = ("sa_workspace_size", "sa_prefill_stats", "sa_block_summaries", "sa_select", "sa_select_noalloc",
+EXPORTS = ("sa_workspace_size", "sa_prefill_stats", "sa_block_summaries", "sa_block_sketch", "sa_select",
+           "sa_select_noalloc",
            "sa_decode", "sa_step", "sa_dense_decode", "sa_wait_timeouts", "sa_status_string")
 
 _LIB = None
@@ -78,7 +80,8 @@ def _lib():
         lib.sa_workspace_size.argtypes = [sh, sp, I]
         lib.sa_workspace_size.restype = S
         lib.sa_prefill_stats.argtypes = [sh, P, P, P, st, F, P, S, P]
-        lib.sa_block_summaries.argtypes = [sh, P, I, I, P, P, P]
+        lib.sa_block_summaries.argtypes = [sh, P, I, I, P, P, P, P, P, P]
+        lib.sa_block_sketch.argtypes = [sh, P, P, I, I, P, P, P]
         lib.sa_select.argtypes = [sh, sp, P, st, P, P, sel, F, P, S, P]
         lib.sa_select_noalloc.argtypes = [sh, sp, P, st, P, P, sel, F, P]
         lib.sa_decode.argtypes = [sh, dp, sp, P, P, P, st, sel, P, P, S, P]
@@ -88,7 +91,7 @@ def _lib():
         lib.sa_wait_timeouts.restype = I
         lib.sa_status_string.argtypes = [I]
         lib.sa_status_string.restype = ctypes.c_char_p
-        for f in ("sa_prefill_stats", "sa_block_summaries", "sa_select", "sa_select_noalloc", "sa_decode", "sa_step",
+        for f in ("sa_prefill_stats", "sa_block_summaries", "sa_block_sketch", "sa_select", "sa_select_noalloc", "sa_decode", "sa_step",
                   "sa_dense_decode"):
             getattr(lib, f).restype = I
         _LIB = lib
@@ -144,7 +147,8 @@ class SelectParams:
 class Stats:
     """Prefill-end statistics (caller-owned device tensors)."""
 
-    FIELDS = ("mu_q", "o_est", "log_z0", "mu_k", "sum_k", "sum_v", "blk_mean", "kbar_absmax")
+    FIELDS = ("mu_q", "o_est", "log_z0", "mu_k", "sum_k", "sum_v", "blk_mean", "kbar_absmax", "blk_code",
+              "blk_meta")
 
     def __init__(self, B, Hq, Hkv, L, d, dtype, device):
         f = dict(dtype=torch.float32, device=device)
@@ -156,6 +160,9 @@ class Stats:
         self.sum_v = torch.empty(B, Hkv, d, **f)
         self.blk_mean = torch.empty(B, Hkv, L // 16, d, dtype=dtype, device=device)
         self.kbar_absmax = torch.zeros(B, Hkv, **f)
+        # scan sketch of blk_mean (int8 codes + {scale, residual norm, norm, 0})
+        self.blk_code = torch.empty(B, Hkv, L // 16, d, dtype=torch.int8, device=device)
+        self.blk_meta = torch.empty(B, Hkv, L // 16, 4, **f)
 
     def c(self):
         return sa_stats(*[self.__dict__[n].data_ptr() for n in self.FIELDS])
@@ -209,8 +216,22 @@ def prefill_stats(q_ctx, k, v, stats=None, scale=0.0, stream=None):
 def block_summaries(k, blk_begin, blk_end, stats, Hq, stream=None):
     shape = make_shape(k, Hq)
     _check(_lib().sa_block_summaries(ctypes.byref(shape), _ptr(k), int(blk_begin), int(blk_end),
-                                     _ptr(stats.blk_mean), _ptr(stats.kbar_absmax), _stream(stream)),
+                                     _ptr(stats.blk_mean), _ptr(stats.kbar_absmax), _ptr(stats.mu_k),
+                                     _ptr(stats.blk_code), _ptr(stats.blk_meta), _stream(stream)),
            "sa_block_summaries")
+
+
+def block_sketch(stats, Hq, blk_begin=0, blk_end=None, stream=None):
+    """Rebuilds stats.blk_code / blk_meta from stats.blk_mean relative to
+    stats.mu_k (blocks [blk_begin, blk_end) of every unit), for block means or
+    a mu_k written by hand."""
+    B, Hkv, nb, d = stats.blk_mean.shape
+    shape = sa_shape(B, Hq, Hkv, d, nb * 16, _dtype_code(stats.blk_mean))
+    blk_end = nb if blk_end is None else blk_end
+    _check(_lib().sa_block_sketch(ctypes.byref(shape), _ptr(stats.blk_mean), _ptr(stats.mu_k), int(blk_begin),
+                                  int(blk_end),
+                                  _ptr(stats.blk_code), _ptr(stats.blk_meta), _stream(stream)),
+           "sa_block_sketch")
 
 
 def select(q, stats, params, k=None, v=None, selection=None, scale=0.0, stream=None):

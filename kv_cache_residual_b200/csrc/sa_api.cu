@@ -46,7 +46,9 @@ sa_status check_select_params(const sa_select_params* p) {
 
 bool check_stats(const sa_stats* st, bool need_all) {
     if (st == nullptr) return false;
-    if (!aligned16(st->blk_mean) || !aligned4(st->kbar_absmax)) return false;
+    if (!aligned16(st->blk_mean) || !aligned4(st->kbar_absmax) || !aligned16(st->blk_code) ||
+        !aligned16(st->blk_meta))
+        return false;
     if (need_all) {
         if (!aligned16(st->mu_q) || !aligned16(st->o_est) || !aligned4(st->log_z0) ||
             !aligned16(st->mu_k) || !aligned16(st->sum_k) || !aligned16(st->sum_v))
@@ -110,17 +112,36 @@ sa_status sa_prefill_stats(const sa_shape* shape, const void* q_ctx, const void*
     return launch_prefill(d, p, a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 
-sa_status sa_block_summaries(const sa_shape* shape, const void* k, int blk_begin, int blk_end,
-                             void* blk_mean, float* kbar_absmax, void* stream) {
+sa_status sa_block_summaries(const sa_shape* shape, const void* k, int blk_begin, int blk_end, void* blk_mean,
+                             float* kbar_absmax, const float* mu_k, int8_t* blk_code, float* blk_meta,
+                             void* stream) {
     NvtxRange r("sa_block_summaries");
     Dims d;
     sa_status e = check_shape(shape, &d);
     if (e != SA_OK) return e;
-    if (!aligned16(k) || !aligned16(blk_mean) || !aligned4(kbar_absmax)) return SA_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(blk_mean) || !aligned4(kbar_absmax) || !aligned4(mu_k) ||
+        !aligned16(blk_code) || !aligned16(blk_meta))
+        return SA_ERR_INVALID_ARG;
     if (blk_begin < 0 || blk_end > d.nb() || blk_begin > blk_end) return SA_ERR_INVALID_ARG;
     if (blk_begin == blk_end) return SA_OK;
-    return launch_block_summaries(d, k, blk_begin, blk_end, blk_mean, kbar_absmax,
+    return launch_block_summaries(d, k, blk_begin, blk_end, blk_mean, kbar_absmax, mu_k, blk_code, blk_meta,
                                   static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SA_OK
+               : SA_ERR_CUDA;
+}
+
+sa_status sa_block_sketch(const sa_shape* shape, const void* blk_mean, const float* mu_k, int blk_begin,
+                          int blk_end, int8_t* blk_code, float* blk_meta, void* stream) {
+    NvtxRange r("sa_block_sketch");
+    Dims d;
+    sa_status e = check_shape(shape, &d);
+    if (e != SA_OK) return e;
+    if (!aligned16(blk_mean) || !aligned4(mu_k) || !aligned16(blk_code) || !aligned16(blk_meta))
+        return SA_ERR_INVALID_ARG;
+    if (blk_begin < 0 || blk_end > d.nb() || blk_begin > blk_end) return SA_ERR_INVALID_ARG;
+    if (blk_begin == blk_end) return SA_OK;
+    return launch_block_sketch(d, blk_mean, mu_k, blk_begin, blk_end, blk_code, blk_meta,
+                               static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? SA_OK
                : SA_ERR_CUDA;
 }

@@ -87,7 +87,7 @@ inline PrefillPlan prefill_plan(const Dims& d) {
 struct SelectPlan {
     SetGeom g;
     int nss, rows_s;             // scan splits per unit, candidate rows per split
-    size_t off_scores, off_xkey, off_cnt, bytes;
+    size_t off_scores, off_scores_up, off_xkey, off_cnt, bytes;
 };
 
 inline SelectPlan select_plan(const Dims& d, const sa_select_params& sp) {
@@ -102,6 +102,7 @@ inline SelectPlan select_plan(const Dims& d, const sa_select_params& sp) {
     size_t off = 0;
     p.off_cnt = off;    off = align256(off + sizeof(unsigned) * (size_t)d.U());
     p.off_scores = off; off = align256(off + sizeof(float) * (size_t)d.U() * nc);
+    p.off_scores_up = off; off = align256(off + sizeof(float) * (size_t)d.U() * nc);
     p.off_xkey = off;   off = align256(off + sizeof(unsigned long long) * (size_t)d.U() * nc);
     p.bytes = off;
     return p;
@@ -177,8 +178,11 @@ struct PrefillArgs {
     sa_stats st; float scale; char* ws;
 };
 cudaError_t launch_prefill(const Dims& d, const PrefillPlan& p, const PrefillArgs& a, cudaStream_t s);
-cudaError_t launch_block_summaries(const Dims& d, const void* k, int blk_begin, int blk_end,
-                                   void* blk_mean, float* kbar_absmax, cudaStream_t s);
+cudaError_t launch_block_summaries(const Dims& d, const void* k, int blk_begin, int blk_end, void* blk_mean,
+                                   float* kbar_absmax, const float* centre, int8_t* blk_code, float* blk_meta,
+                                   cudaStream_t s);
+cudaError_t launch_block_sketch(const Dims& d, const void* blk_mean, const float* centre, int blk_begin, int blk_end,
+                                int8_t* blk_code, float* blk_meta, cudaStream_t s);
 
 struct SelectArgs {
     const void* q; sa_stats st; const void* k; const void* v;

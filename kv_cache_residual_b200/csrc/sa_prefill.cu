@@ -256,6 +256,87 @@ k_blockmeans(const T* __restrict__ k, int L, int blk_begin, int blk_end, T* __re
     if (lane == 0 && amax > 0.f) atomicMax(reinterpret_cast<int*>(kbar_absmax + u), __float_as_int(amax));
 }
 
+// Scan sketch of block rows [blk_begin, blk_end) of every unit, one warp per
+// row, relative to the unit's centre m (its typical key mu_k): with
+// t = kbar - m, s = fl32(max|t| / 127), code = clamp(rint(t / s), +-127) and
+// the f32 upper bounds rn >= ||t - s code||_2, kn >= ||s code||_2.  Centring
+// shifts every block's score by the same qbar . m, which leaves the ranking
+// unchanged, and lets the 8-bit codes resolve the blocks' differences rather
+// than the key mean they share.  In fp64, t and t - s code are each rounded
+// once (|error| <= 2^-53 of the value) and the sums of squares carry at most
+// (D + 5) 2^-53 relative error: rn adds 2^-52 (||t|| + ||r||) and both bounds
+// a 2^-40 relative margin before rounding up.
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads)
+k_sketch(const T* __restrict__ bm, const float* __restrict__ centre, int nb, int blk_begin, int blk_end,
+         int8_t* __restrict__ code, float4* __restrict__ meta) {
+    constexpr int E = D / 32;                 // elements per lane
+    const int u = blockIdx.y;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    double m[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) m[e] = (double)centre[(size_t)u * D + lane * E + e];
+    for (int blk = blk_begin + blockIdx.x * kWarps + warp; blk < blk_end; blk += gridDim.x * kWarps) {
+        const size_t row = (size_t)u * nb + blk;
+        const T* src = bm + row * D + lane * E;
+        double t[E];
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            t[e] = (double)to_f32<T>(src[e]) - m[e];
+            amax = fmaxf(amax, (float)fabs(t[e]));
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        // amax may round below max|t|: the clamp keeps the codes in range
+        const float sc = amax / 127.0f;
+        int c[E];
+        double r2 = 0.0, k2 = 0.0, t2 = 0.0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            int ci = 0;
+            if (sc > 0.f) ci = max(-127, min(127, (int)rint(t[e] / (double)sc)));
+            c[e] = ci;
+            const double q = (double)sc * (double)ci;         // exact
+            const double r = t[e] - q;
+            r2 = fma(r, r, r2);
+            k2 = fma(q, q, k2);
+            t2 = fma(t[e], t[e], t2);
+        }
+        r2 = group_sum_f64<32>(r2);
+        k2 = group_sum_f64<32>(k2);
+        t2 = group_sum_f64<32>(t2);
+        uint32_t packed = 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) packed |= (uint32_t)(c[e] & 0xff) << (8 * e);
+        if constexpr (E == 4) *reinterpret_cast<uint32_t*>(code + row * D + lane * E) = packed;
+        else *reinterpret_cast<uint16_t*>(code + row * D + lane * E) = (uint16_t)packed;
+        if (lane == 0) {
+            const double mg = 1.0 + 0x1p-40;
+            const double rn = sqrt(r2) * mg + 0x1p-52 * (sqrt(t2) + sqrt(r2)) * mg;
+            meta[row] = make_float4(sc, __double2float_ru(rn), __double2float_ru(sqrt(k2) * mg), 0.f);
+        }
+    }
+}
+
+template <typename T, int D>
+static cudaError_t sketch_t(const Dims& d, const void* bm, const float* centre, int b0, int b1, int8_t* code,
+                            float* meta, cudaStream_t s) {
+    const int nblk = b1 - b0;
+    const int gx = max(1, min(cdiv(nblk, kWarps), cdiv(4 * kSmTarget, d.U())));
+    k_sketch<T, D><<<dim3(gx, d.U()), kThreads, 0, s>>>(reinterpret_cast<const T*>(bm), centre, d.L / 16, b0, b1,
+                                                        code, reinterpret_cast<float4*>(meta));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_block_sketch(const Dims& d, const void* bm, const float* centre, int b0, int b1, int8_t* code,
+                                float* meta, cudaStream_t s) {
+    if (d.bf16) return d.d == 128 ? sketch_t<__nv_bfloat16, 128>(d, bm, centre, b0, b1, code, meta, s)
+                                  : sketch_t<__nv_bfloat16, 64>(d, bm, centre, b0, b1, code, meta, s);
+    return d.d == 128 ? sketch_t<float, 128>(d, bm, centre, b0, b1, code, meta, s)
+                      : sketch_t<float, 64>(d, bm, centre, b0, b1, code, meta, s);
+}
+
 // ---- dispatch ------------------------------------------------------------
 
 template <typename T, int D, int G>
@@ -271,7 +352,9 @@ static cudaError_t prefill_t(const Dims& d, const PrefillPlan& p, const PrefillA
         reinterpret_cast<const T*>(a.k), reinterpret_cast<const T*>(a.v), a.st.mu_q, d.Hq, d.Hkv, d.L,
         p.tok_kv, p.nskv, a.scale * kLog2e, p.kv_stride, reinterpret_cast<float*>(ws + p.off_kvpart),
         reinterpret_cast<unsigned*>(ws + p.off_kvcnt), a.st);
-    return cudaGetLastError();
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_block_sketch(d, a.st.blk_mean, a.st.mu_k, 0, d.L / 16, a.st.blk_code, a.st.blk_meta, s);
 }
 
 template <typename T, int D>
@@ -291,21 +374,24 @@ cudaError_t launch_prefill(const Dims& d, const PrefillPlan& p, const PrefillArg
 }
 
 template <typename T, int D>
-static cudaError_t blockmeans_t(const Dims& d, const void* k, int b0, int b1, void* bm, float* amax, cudaStream_t s) {
+static cudaError_t blockmeans_t(const Dims& d, const void* k, int b0, int b1, void* bm, float* amax,
+                                const float* centre, int8_t* code, float* meta, cudaStream_t s) {
     using Gm = Geom<T, D>;
     const int nblk = b1 - b0;
     const int gx = max(1, min(cdiv(nblk, Gm::NG), cdiv(kSmTarget, d.U())));
     k_blockmeans<T, D><<<dim3(gx, d.U()), kThreads, 0, s>>>(
         reinterpret_cast<const T*>(k), d.L, b0, b1, reinterpret_cast<T*>(bm), amax);
-    return cudaGetLastError();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return sketch_t<T, D>(d, bm, centre, b0, b1, code, meta, s);
 }
 
 cudaError_t launch_block_summaries(const Dims& d, const void* k, int b0, int b1, void* bm, float* amax,
-                                   cudaStream_t s) {
-    if (d.bf16) return d.d == 128 ? blockmeans_t<__nv_bfloat16, 128>(d, k, b0, b1, bm, amax, s)
-                                  : blockmeans_t<__nv_bfloat16, 64>(d, k, b0, b1, bm, amax, s);
-    return d.d == 128 ? blockmeans_t<float, 128>(d, k, b0, b1, bm, amax, s)
-                      : blockmeans_t<float, 64>(d, k, b0, b1, bm, amax, s);
+                                   const float* centre, int8_t* code, float* meta, cudaStream_t s) {
+    if (d.bf16) return d.d == 128 ? blockmeans_t<__nv_bfloat16, 128>(d, k, b0, b1, bm, amax, centre, code, meta, s)
+                                  : blockmeans_t<__nv_bfloat16, 64>(d, k, b0, b1, bm, amax, centre, code, meta, s);
+    return d.d == 128 ? blockmeans_t<float, 128>(d, k, b0, b1, bm, amax, centre, code, meta, s)
+                      : blockmeans_t<float, 64>(d, k, b0, b1, bm, amax, centre, code, meta, s);
 }
 
 }  // namespace sa

@@ -3,20 +3,23 @@
 // block selection of Quest / ArkVale that RESA wraps).
 //
 // k_select: grid (nss, B*Hkv)
-//   scan  : fp32 scores y_c = sum_h q_h . kbar_c of the unit's candidate blocks
-//           (computed as qbar . kbar_c, qbar = sum_h q_h), the HBM-bound part:
-//           one read of the block summaries.  With one CTA per unit (enough
-//           units to fill the GPU) the scores stay in shared memory; with
+//   scan  : score intervals of the unit's candidate blocks from the int8
+//           sketch of the centred block summaries (0.56x their bytes at
+//           d = 128, bf16): y_c = sf s_c (Q . code_c) by integer dot products
+//           (Q a 15-bit code of qbar = sum_h q_h), and [y_c - e_c, y_c + e_c]
+//           certain to hold z_c = x_c - qbar . m, the exact score
+//           x_c = sum_h q_h . kbar_c less a constant common to all blocks.  The HBM-bound part: one read of the
+//           sketch, streamed by bulk copies.  With one CTA per unit (enough
+//           units to fill the GPU) the bounds stay in shared memory; with
 //           several CTAs per unit they go to the workspace and the CTA that
 //           finishes the unit last (completion ticket, no wait) takes over.
-//   top-k : exact k best by (score desc, block index asc).  For k <= 32 the
-//           warps extract their local best k by argmax rounds over 64-bit
-//           (score, ~index) keys in registers and one warp merges them;
-//           otherwise a 4 x 8-bit radix select finds the k-th key.  Then the
-//           rounding bound |y_c - x_c| <= E of the fp32 scan (x_c the exact
-//           score) is applied: every candidate with y >= y_(k) - 2E may belong
-//           to the exact top k; if more than k do, those are rescored in fp64
-//           and ranked exactly.  The decision is therefore the fp64 one.
+//   top-k : the k best lower bounds (per-warp running lists merged, or a
+//           radix select for k > 32); thr = the k-th.  Every candidate whose
+//           upper bound reaches thr is in the band; the exact top k by
+//           (x desc, block index asc) lies inside it.  A band of exactly k is
+//           the answer; otherwise its members are rescored exactly from the
+//           bf16 / fp32 summaries (exact products, double-double sum, one
+//           rounding) and ranked.  The decision is the exact one.
 //   draws : tail positions for the sampling estimator (SplitMix64 counters).
 #include "sa_bulk.cuh"
 #include "sa_common.cuh"
@@ -28,19 +31,25 @@ constexpr int kSmemKeys = 4096;     // candidate keys held in shared memory (16 
 constexpr int kBandCap = 512;       // band members ranked in shared memory
 constexpr int kWarpTopK = 32;       // largest k of the warp-argmax path
 
-// The scan's shared-memory ring: kStages stages of kStageBytes, each a run of
-// SR consecutive block-summary rows of RB bytes; a warp scores R rows per
-// lane group of each stage (the stage is SR = kWarps * GPW * R rows).
-template <typename T, int D>
-struct ScanRing {
-    static constexpr int kStages = 5;
-    static constexpr int kStageBytes = 16384;
+// The scan's shared-memory ring over the sketch: kStages stages, each SR = 128
+// consecutive block rows as SR x D int8 codes followed by SR x 16 bytes of
+// {s, rn, kn, 0}.  A code row is CPR 16-byte chunks (one per lane of a lane
+// group, GPW groups per warp); a warp scores R rows per lane group of each
+// stage (SR = kWarps * GPW * R).  Four stages: 72 KB at d = 128, so that two
+// CTAs (with their 36 KB of keys and query) share an SM.
+template <int D>
+struct SketchRing {
+    static constexpr int kStages = 4;
+    static constexpr int SR = 128;
+    static constexpr int kCodeBytes = SR * D;
+    static constexpr int kMetaBytes = SR * 16;
+    static constexpr int kStageBytes = kCodeBytes + kMetaBytes;
     static constexpr int kRingBytes = kStages * kStageBytes;
-    static constexpr int RB = D * (int)sizeof(T);
-    static constexpr int SR = kStageBytes / RB;
-    static constexpr int R = SR / (kWarps * Geom<T, D>::GPW);
+    static constexpr int CPR = D / 16;
+    static constexpr int GPW = 32 / CPR;
+    static constexpr int R = SR / (kWarps * GPW);
     static constexpr size_t kSmem = (size_t)kRingBytes + 8 * kStages;      // ring + its barriers
-    static_assert(R >= 1 && (R & (R - 1)) == 0, "stage geometry");
+    static_assert(R >= 1 && (R & (R - 1)) == 0 && CPR >= R, "stage geometry");
 };
 
 __device__ __forceinline__ uint32_t fkey(float y) {
@@ -365,23 +374,22 @@ __device__ void rescore_members(const T* bm, const int* s_bidx, int nb, const fl
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads, 2)
-k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* __restrict__ kbar_absmax,
-         int Hq, int Hkv, int L, SetGeom sg, int rows, int nss,
-         float* __restrict__ scores, unsigned long long* __restrict__ xkey,
+k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const int8_t* __restrict__ blk_code,
+         const float4* __restrict__ blk_meta, int Hq, int Hkv, int L, SetGeom sg, int rows, int nss,
+         float* __restrict__ sc_lo_all, float* __restrict__ sc_up_all, unsigned long long* __restrict__ xkey,
          unsigned* __restrict__ cnt, int kb_stride, int32_t* __restrict__ blk_idx,
          int32_t* __restrict__ samp_idx, int32_t* __restrict__ samp_count, int32_t* __restrict__ n_rescored,
          int sample_b, int sample_cap, unsigned long long seed, int step) {
-    using Gm = Geom<T, D>;
-    constexpr int EPC = Gm::EPC, CPR = Gm::CPR;
-    using Ring = ScanRing<T, D>;
-    constexpr int R = Ring::R;
-    static_assert(CPR >= R, "transposed reduction needs at least one lane per row");
+    using Ring = SketchRing<D>;
+    constexpr int R = Ring::R, CPR = Ring::CPR, GPW = Ring::GPW;
     __shared__ unsigned hist[kThreads];
     __shared__ int sw[kWarps + 1];
     __shared__ int s_digit, s_rem, s_nb;
-    __shared__ float s_qh[G * D];          // the group's queries (exact), for fp64 rescoring
-    __shared__ float s_qsum;
-    __shared__ uint32_t s_keys[kSmemKeys];
+    __shared__ float s_qh[G * D];                      // the group's queries (exact), for rescoring
+    __shared__ __align__(16) int8_t s_qi[2 * D];        // the group query's two int8 code halves
+    __shared__ float s_qc[3];                          // sf, qn, rq (see below)
+    __shared__ uint32_t s_ukeys[kSmemKeys];            // upper-bound keys (band membership)
+    __shared__ uint32_t s_lkeys[kSmemKeys];            // lower-bound keys (ranking without the warp lists)
     __shared__ int s_sorted[kWarpTopK];
     // the scan's copy ring; reused for the top-k / band arrays once the scan is done
     extern __shared__ __align__(128) unsigned char s_ring[];
@@ -399,25 +407,27 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
     const int u = blockIdx.y, split = blockIdx.x;
     const int b = u / Hkv, g = u - b * Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int li = lane % CPR;
+    const int li = lane % CPR, gsub = lane / CPR;
     const int nb = L / 16;
     const int n = sg.n_cand, kk = sg.kk;
     const T* qg = q + ((size_t)b * Hq + (size_t)g * G) * D;
-    float* sc = scores + (size_t)u * (n > 0 ? n : 1);
-    // one CTA per unit: the scores never leave shared memory
+    float* sc_lo = sc_lo_all + (size_t)u * (n > 0 ? n : 1);
+    float* sc_up = sc_up_all + (size_t)u * (n > 0 ? n : 1);
+    // one CTA per unit: the keys never leave shared memory
     const bool local = (nss == 1) && n <= kSmemKeys;
     // k <= 32 with one CTA per unit: each warp keeps its best k while scanning
     const bool run_topk = local && kk > 0 && kk < n && kk <= kWarpTopK;
-    const float amax = kbar_absmax[u];
 
-    // ---- scan: fp32 scores of this CTA's slice -------------------------------
-    // The slice's block summaries are contiguous: thread 0 streams them through
-    // a ring of kStages shared-memory stages with bulk copies, kStages stages
-    // in flight; all warps score each stage as it lands.
+    // ---- scan: score intervals of this CTA's slice ------------------------------
+    // The slice's sketch rows are contiguous: thread 0 streams codes and
+    // metadata through a ring of kStages shared-memory stages with bulk copies,
+    // kStages stages in flight; all warps score each stage as it lands.
     const int r0 = split * rows, r1 = min(n, r0 + rows);
     const int nrows = max(0, r1 - r0);
     const int nst = (nrows + Ring::SR - 1) / Ring::SR;
-    const char* src0 = reinterpret_cast<const char*>(blk_mean + ((size_t)u * nb + sg.c_lo + r0) * D);
+    const size_t row0 = (size_t)u * nb + sg.c_lo + r0;
+    const int8_t* code0 = blk_code + row0 * D;
+    const float4* meta0 = blk_meta + row0;
     const uint32_t ring = smem_addr(s_ring), bar0 = smem_addr(s_bar);
     if (threadIdx.x == 0) {
 #pragma unroll
@@ -427,65 +437,118 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
     __syncthreads();
     auto issue = [&](int j) {                      // thread 0
         if (j < nst) {
-            const uint32_t bytes = (uint32_t)min(Ring::SR, nrows - j * Ring::SR) * Ring::RB;
+            const int rj = min(Ring::SR, nrows - j * Ring::SR);
             const uint32_t bar = bar0 + 8 * (j % Ring::kStages);
-            mbar_arrive_expect_tx(bar, bytes);
-            bulk_g2s(ring + (j % Ring::kStages) * Ring::kStageBytes, src0 + (size_t)j * Ring::kStageBytes, bytes, bar);
+            const uint32_t dst = ring + (j % Ring::kStages) * Ring::kStageBytes;
+            mbar_arrive_expect_tx(bar, (uint32_t)rj * (D + 16));
+            bulk_g2s(dst, code0 + (size_t)j * Ring::SR * D, (uint32_t)rj * D, bar);
+            bulk_g2s(dst + Ring::kCodeBytes, meta0 + (size_t)j * Ring::SR, (uint32_t)rj * 16, bar);
         }
     };
     if (threadIdx.x == 0)
         for (int j = 0; j < Ring::kStages; ++j) issue(j);
     __syncwarp();
 
-    bool failed = false;
-    {
-        float qb[EPC];
-        float qa = 0.f;
+    // The group query, exact per head (for rescoring) and as a 15-bit code of
+    // qbar = sum_h q_h in two int8 halves: qbar64 (fp64), sq = fl32(max|qbar64|
+    // / 127), qi1 = clamp(rint(qbar64 / sq), +-127), qi2 = clamp(rint((qbar64 -
+    // sq qi1) / (sq / 128)), +-127), so qbar ~ sf Q with sf = sq / 128 and
+    // Q = 128 qi1 + qi2.  For every candidate c with sketch (s, code, rn, kn)
+    // of t_c = kbar_c - m (m the unit's centre, common to all c) and
+    // z_c = qbar . t_c = x_c - qbar . m:
+    //   z_c - sf s (Q . code) = qbar . (t_c - s code) + (qbar - sf Q) . (s code)
+    //   |z_c - sf s (Q . code)| <= qn rn + rq kn,
+    // qn >= ||qbar||_2, rq >= ||qbar - sf Q||_2 (both including the fp64
+    // rounding of qbar64, at most (G-1) 2^-53 sum_h |q_h| per element).
+    if (warp == 0) {
+        constexpr int E = D / 32;
+        double qb[E], qa[E];
+        float amax = 0.f;
 #pragma unroll
-        for (int e = 0; e < EPC; ++e) qb[e] = 0.f;
+        for (int e = 0; e < E; ++e) { qb[e] = 0.0; qa[e] = 0.0; }
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-            float f[EPC];
-            unpack<T>(ld_nc16(qg + (size_t)h * D + li * EPC), f);
 #pragma unroll
-            for (int e = 0; e < EPC; ++e) {
-                qb[e] += f[e];
-                qa += fabsf(f[e]);
-            }
-            // for the top-k (whichever CTA ends up doing it): the group's
-            // queries and sum_i sum_h |q_hi| for the rounding bound
-            if (warp == 0 && lane < CPR) {
-#pragma unroll
-                for (int e = 0; e < EPC; ++e) s_qh[h * D + li * EPC + e] = f[e];
+            for (int e = 0; e < E; ++e) {
+                const float f = to_f32<T>(qg[(size_t)h * D + lane * E + e]);
+                s_qh[h * D + lane * E + e] = f;
+                qb[e] += (double)f;
+                qa[e] += (double)fabsf(f);
             }
         }
-        qa = group_sum<CPR>(qa);
-        if (warp == 0 && lane == 0) s_qsum = qa;
-        const int gsub = lane / CPR;
-        // this warp's rows of a stage: warp * R * GPW + j * GPW + gsub, j < R
-        const int wrow = warp * R * Gm::GPW + gsub;
-        // running best kk of the rows this warp scored: lane i < kk holds the
-        // i-th best (score key, ~index) word, 0 when empty; thr = the kk-th
+#pragma unroll
+        for (int e = 0; e < E; ++e) amax = fmaxf(amax, (float)fabs(qb[e]));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        // amax may round below max|qbar64|: the clamps keep the codes in range
+        const float sq = amax / 127.0f;
+        const float sf = sq * 0x1p-7f;                 // exact
+        double r2 = 0.0, n2 = 0.0, a2 = 0.0;
+        uint32_t p1 = 0, p2 = 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            int c1 = 0, c2 = 0;
+            if (sq > 0.f) {
+                c1 = max(-127, min(127, (int)rint(qb[e] / (double)sq)));
+                c2 = max(-127, min(127, (int)rint((qb[e] - (double)sq * c1) / (double)sf)));
+            }
+            p1 |= (uint32_t)(c1 & 0xff) << (8 * e);
+            p2 |= (uint32_t)(c2 & 0xff) << (8 * e);
+            const double r = qb[e] - (double)sf * (double)(128 * c1 + c2);
+            r2 = fma(r, r, r2);
+            n2 = fma(qb[e], qb[e], n2);
+            a2 = fma(qa[e], qa[e], a2);
+        }
+        if constexpr (E == 4) {
+            *reinterpret_cast<uint32_t*>(s_qi + lane * E) = p1;
+            *reinterpret_cast<uint32_t*>(s_qi + D + lane * E) = p2;
+        } else {
+            *reinterpret_cast<uint16_t*>(s_qi + lane * E) = (uint16_t)p1;
+            *reinterpret_cast<uint16_t*>(s_qi + D + lane * E) = (uint16_t)p2;
+        }
+        r2 = group_sum_f64<32>(r2);
+        n2 = group_sum_f64<32>(n2);
+        a2 = group_sum_f64<32>(a2);
+        if (lane == 0) {
+            // r is one fp64 rounding away from exact: 2^-52 ||qbar64|| covers it
+            const double m = 1.0 + 0x1p-40;
+            const double slack = (double)(G > 1 ? G - 1 : 0) * 0x1p-52 * sqrt(a2) * m;
+            s_qc[0] = sf;
+            s_qc[1] = __double2float_ru(sqrt(n2) * m + slack);
+            s_qc[2] = __double2float_ru(sqrt(r2) * m + 0x1p-52 * sqrt(n2) * m + slack);
+        }
+    }
+    __syncthreads();
+
+    bool failed = false;
+    {
+        const uint4 qv1 = *reinterpret_cast<const uint4*>(s_qi + li * 16);
+        const uint4 qv2 = *reinterpret_cast<const uint4*>(s_qi + D + li * 16);
+        const float sf = s_qc[0], qn = s_qc[1], rq = s_qc[2];
+        // this warp's rows of a stage: warp * R * GPW + jj * GPW + gsub, jj < R
+        const int wrow = warp * R * GPW + gsub;
+        // running best kk of the rows this warp scored, by lower bound: lane
+        // i < kk holds the i-th best (key, ~index) word, 0 when empty; thr =
+        // the kk-th
         unsigned long long best = 0ull, thr = 0ull;
         int j = 0;
         for (; j < nst; ++j) {
             const bool ok = mbar_wait(bar0 + 8 * (j % Ring::kStages), (uint32_t)(j / Ring::kStages) & 1u);
             const unsigned char* sb = s_ring + (size_t)(j % Ring::kStages) * Ring::kStageBytes;
             const int rows_j = min(Ring::SR, nrows - j * Ring::SR);
-            // lane partial dot of each row: packed FMAs over element pairs,
-            // then the two halves added
-            float x[R];
+            // integer dot products Q . code of the lane's 16 codes (exact;
+            // |Q . code| < 2^14 * 127 * D < 2^31)
+            int x[R];
 #pragma unroll
             for (int jj = 0; jj < R; ++jj) {
-                const int rr = wrow + jj * Gm::GPW;
-                const uint4 w = (rr < rows_j) ? *reinterpret_cast<const uint4*>(sb + (size_t)rr * Ring::RB + li * 16)
+                const int rr = wrow + jj * GPW;
+                const uint4 w = (rr < rows_j) ? *reinterpret_cast<const uint4*>(sb + (size_t)rr * D + li * 16)
                                               : make_uint4(0, 0, 0, 0);
-                float f[EPC];
-                unpack<T>(w, f);
-                float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-                for (int e = 0; e < EPC; e += 2) ffma2(a0, a1, qb[e], qb[e + 1], f[e], f[e + 1]);
-                x[jj] = a0 + a1;
+                const int hi = __dp4a((int)w.x, (int)qv1.x, __dp4a((int)w.y, (int)qv1.y,
+                               __dp4a((int)w.z, (int)qv1.z, __dp4a((int)w.w, (int)qv1.w, 0))));
+                const int lo = __dp4a((int)w.x, (int)qv2.x, __dp4a((int)w.y, (int)qv2.y,
+                               __dp4a((int)w.z, (int)qv2.z, __dp4a((int)w.w, (int)qv2.w, 0))));
+                x[jj] = 128 * hi + lo;
             }
             // transposed reduction over the CPR lanes of the group: each of the
             // first log2(R) levels keeps half of the remaining rows, so the lane
@@ -496,29 +559,44 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
                 const int bit = (li & off) ? 1 : 0;
 #pragma unroll
                 for (int jj = 0; jj < half; ++jj) {
-                    const float send = bit ? x[jj] : x[jj + half];
-                    const float keep = bit ? x[jj + half] : x[jj];
+                    const int send = bit ? x[jj] : x[jj + half];
+                    const int keep = bit ? x[jj + half] : x[jj];
                     x[jj] = keep + __shfl_xor_sync(0xffffffffu, send, off);
                 }
                 row = 2 * row + bit;
             }
 #pragma unroll
             for (int off = CPR / (2 * R); off > 0; off >>= 1) x[0] += __shfl_xor_sync(0xffffffffu, x[0], off);
-            const int rr = wrow + row * Gm::GPW;
+            const int rr = wrow + row * GPW;
             const int r = r0 + j * Ring::SR + rr;
             const bool owner = (li & (CPR / R - 1)) == 0 && rr < rows_j;
-            const uint32_t key = fkey(x[0]);
+            // score interval: y = fl(fl(sf s) fl(y_int)) is three roundings,
+            // within 2^-21 |y| of sf s y_int; 2^-100 covers an underflow of
+            // sf s; every bound term is rounded up
+            uint32_t lkey = 0u, ukey = 0u;
             if (owner) {
-                if (local) s_keys[r] = key;
-                else sc[r] = x[0];
+                const float4 m = *reinterpret_cast<const float4*>(sb + Ring::kCodeBytes + (size_t)rr * 16);
+                const float y = __fmul_rn(__fmul_rn(sf, m.x), (float)x[0]);
+                const float e = __fadd_ru(__fmaf_ru(qn, m.y, __fmaf_ru(rq, m.z, __fmul_ru(0x1p-21f, fabsf(y)))),
+                                          0x1p-100f);
+                const float lo = __fsub_rd(y, e), up = __fadd_ru(y, e);
+                lkey = fkey(lo);
+                ukey = fkey(up);
+                if (local) {
+                    s_ukeys[r] = ukey;
+                    s_lkeys[r] = lkey;
+                } else {
+                    sc_lo[r] = lo;
+                    sc_up[r] = up;
+                }
             }
             // compiler barrier: without it the shared-memory traffic around the
             // list update is scheduled so badly that the scan runs ~2.5x slower
             // (measured); it emits no instruction
             asm volatile("" ::: "memory");
             if (run_topk) {
-                // rows that beat the warp's current kk-th best enter its list
-                const unsigned long long c = owner ? comp_key(key, r) : 0ull;
+                // rows whose lower bound beats the warp's current kk-th enter its list
+                const unsigned long long c = owner ? comp_key(lkey, r) : 0ull;
                 unsigned m = __ballot_sync(0xffffffffu, c > thr);
                 while (m) {
                     const int src = __ffs(m) - 1;
@@ -562,26 +640,35 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
         return;
     }
 
-    // ---- gather the unit's scores ------------------------------------------------
-    uint32_t* keys = s_keys;
+    // ---- gather the unit's keys --------------------------------------------------
+    uint32_t* lk = s_lkeys;            // lower-bound keys: the ranking
+    uint32_t* uk = s_ukeys;            // upper-bound keys: band membership
     if (local) {
         __syncthreads();
     } else {
         if (!last_cta_of_unit(cnt + u, nss)) return;
         // orderable keys, staged once: shared memory when they fit, else in
-        // place over the unit's scores in the workspace
-        if (n > kSmemKeys) keys = reinterpret_cast<uint32_t*>(sc);
+        // place over the unit's bounds in the workspace (each thread rewrites
+        // only the entries it read)
+        if (n > kSmemKeys) {
+            lk = reinterpret_cast<uint32_t*>(sc_lo);
+            uk = reinterpret_cast<uint32_t*>(sc_up);
+        }
         for (int i0 = 0; i0 < n; i0 += 4 * kThreads) {
-            float y[4];
+            float ylo[4], yup[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int i = i0 + j * kThreads + threadIdx.x;
-                y[j] = i < n ? ldcg(sc + i) : 0.f;
+                ylo[j] = i < n ? ldcg(sc_lo + i) : 0.f;
+                yup[j] = i < n ? ldcg(sc_up + i) : 0.f;
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int i = i0 + j * kThreads + threadIdx.x;
-                if (i < n) keys[i] = fkey(y[j]);
+                if (i < n) {
+                    lk[i] = fkey(ylo[j]);
+                    uk[i] = fkey(yup[j]);
+                }
             }
         }
         __syncthreads();
@@ -592,7 +679,7 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
     int rescored = 0;
     bool sorted_smem = false;          // the chosen indices are also in s_sorted
     if (kk > 0 && kk < n) {
-        auto k32 = [&](int i) -> uint32_t { return keys[i]; };
+        auto k32 = [&](int i) -> uint32_t { return lk[i]; };
         const bool fast = kk <= kWarpTopK && n <= kSmemKeys;
         uint32_t thr;
         int need = 0;
@@ -600,23 +687,16 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
             merge_warp_lists(s_cand, kk, s_list);
             thr = (uint32_t)(s_list[kk - 1] >> 32);
         } else if (fast) {
-            warp_topk(keys, n, kk, s_cand, s_list);
+            warp_topk(lk, n, kk, s_cand, s_list);
             thr = (uint32_t)(s_list[kk - 1] >> 32);
         } else {
             radix_select<uint32_t>(k32, n, kk, &thr, &need, hist, &s_digit, &s_rem);
         }
-        // rounding bound of the fp32 scan.  qbar_i is a sum of G terms (G-1
-        // roundings) and each score is EPC/2 fused multiply-adds on each of two
-        // accumulators per lane, their sum, then a log2(CPR)-level shuffle tree
-        // (depth h = EPC/2 + 1 + log2(CPR)), so with u = 2^-24
-        //   |y - x| <= (gamma_{G-1} + gamma_h (1 + gamma_{G-1})) sum_i qa_i |kbar_ci|
-        //           <= (G + h + 2) 2^-24 sum_i qa_i * max|kbar|,
-        // taken twice over for margin.
-        constexpr int kDepth = EPC / 2 + 1 + ilog2(CPR);
-        const float E = (float)(G + kDepth + 2) * 0x1p-23f * s_qsum * amax * 1.0001f + 0x1p-100f;
-        const uint32_t lo_key = fkey(fkey_inv(thr) - 2.f * E);
+        // thr = the kk-th largest lower bound.  A candidate whose upper bound is
+        // below it is beaten strictly by kk others, so the exact top kk lies
+        // in the band {upper >= thr}, which contains the kk best lower bounds
         int band = 0;
-        for (int i = threadIdx.x; i < n; i += kThreads) band += (keys[i] >= lo_key) ? 1 : 0;
+        for (int i = threadIdx.x; i < n; i += kThreads) band += (uk[i] >= thr) ? 1 : 0;
         band = block_sum(band, sw);
         if (band == kk) {
             if (fast) {
@@ -625,15 +705,15 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
             }
             else emit_topk<uint32_t>(k32, n, thr, need, kk, sg.c_lo, out_idx, sw);
         } else {
-            // ambiguous: the exact top-k lies inside the band; rescore the band
-            // members in fp64 and take the top k among them by (x desc, index asc)
+            // ambiguous: rescore the band members exactly and take the top k
+            // among them by (x desc, index asc)
             rescored = band;
             const T* bm = blk_mean + ((size_t)u * nb + sg.c_lo) * D;
             if (band <= kBandCap) {
                 if (threadIdx.x == 0) s_nb = 0;
                 __syncthreads();
                 for (int i = threadIdx.x; i < n; i += kThreads)
-                    if (keys[i] >= lo_key) s_bidx[atomicAdd(&s_nb, 1)] = i;
+                    if (uk[i] >= thr) s_bidx[atomicAdd(&s_nb, 1)] = i;
                 __syncthreads();
                 rescore_members<T, D, G>(bm, s_bidx, band, s_qh, s_bx);
                 __syncthreads();
@@ -662,7 +742,7 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
                 unsigned long long* xk = xkey + (size_t)u * n;
                 for (int i = warp; i < n; i += kWarps) {
                     unsigned long long key = 0ull;
-                    if (keys[i] >= lo_key) {                        // warp-uniform branch
+                    if (uk[i] >= thr) {                             // warp-uniform branch
                         const T* rows[1] = {bm + (size_t)i * D};
                         const bool live[1] = {true};
                         double x[1];
@@ -714,17 +794,17 @@ k_select(const T* __restrict__ q, const T* __restrict__ blk_mean, const float* _
 template <typename T, int D, int G>
 static cudaError_t select_t(const Dims& d, const SelectPlan& p, const SelectArgs& a, cudaStream_t s) {
     char* ws = a.ws;
-    constexpr size_t smem = ScanRing<T, D>::kSmem;
+    constexpr size_t smem = SketchRing<D>::kSmem;
     static std::atomic<unsigned long long> opted{0};
     cudaError_t e = opt_in_smem(k_select<T, D, G>, smem, opted);
     if (e != cudaSuccess) return e;
     k_select<T, D, G><<<dim3(p.nss, d.U()), kThreads, smem, s>>>(
-        reinterpret_cast<const T*>(a.q), reinterpret_cast<const T*>(a.st.blk_mean), a.st.kbar_absmax,
-        d.Hq, d.Hkv, d.L, p.g, p.rows_s, p.nss,
-        reinterpret_cast<float*>(ws + p.off_scores), reinterpret_cast<unsigned long long*>(ws + p.off_xkey),
-        reinterpret_cast<unsigned*>(ws + p.off_cnt), a.sp.k_blocks, a.sel.blk_idx, a.sel.samp_idx,
-        a.sel.samp_count, a.sel.n_rescored, a.sp.sample_b, a.sp.sample_cap, (unsigned long long)a.sp.seed,
-        a.sp.step);
+        reinterpret_cast<const T*>(a.q), reinterpret_cast<const T*>(a.st.blk_mean), a.st.blk_code,
+        reinterpret_cast<const float4*>(a.st.blk_meta), d.Hq, d.Hkv, d.L, p.g, p.rows_s, p.nss,
+        reinterpret_cast<float*>(ws + p.off_scores), reinterpret_cast<float*>(ws + p.off_scores_up),
+        reinterpret_cast<unsigned long long*>(ws + p.off_xkey), reinterpret_cast<unsigned*>(ws + p.off_cnt),
+        a.sp.k_blocks, a.sel.blk_idx, a.sel.samp_idx, a.sel.samp_count, a.sel.n_rescored, a.sp.sample_b,
+        a.sp.sample_cap, (unsigned long long)a.sp.seed, a.sp.step);
     return cudaGetLastError();
 }
 

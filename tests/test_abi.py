@@ -58,7 +58,7 @@ def test_workspace_sizes(lib):
 ])
 def test_bad_shapes_rejected(lib, kw, status):
     p = ctypes.c_void_p(0x10000)
-    st = sa.sa_stats(*([0x10000] * 8))
+    st = sa.sa_stats(*([0x10000] * 10))
     assert lib.sa_dense_decode(ctypes.byref(_shape(**kw)), p, p, p, p, 0.0, p, 1 << 30, None) == status
     assert lib.sa_prefill_stats(ctypes.byref(_shape(**kw)), p, p, p, ctypes.byref(st), 0.0, p, 1 << 30, None) == status
 
@@ -79,7 +79,7 @@ def test_bad_pointers_and_workspace_rejected(lib):
 def test_select_and_decode_param_checks(lib):
     sh = _shape()
     p = ctypes.c_void_p(0x10000)
-    st = sa.sa_stats(*([0x10000] * 8))
+    st = sa.sa_stats(*([0x10000] * 10))
     sel = sa.sa_selection(0x10000, 0x10000, 0x10000, 0)
     bad = [
         sa.sa_select_params(-1, 128, 8, 0, 0, 0, 0.05, 0.05, 0, 0),     # negative sink
@@ -106,9 +106,15 @@ def test_select_and_decode_param_checks(lib):
     dp = sa.sa_decode_params(sa.MODES["resa"], 1.0, 0.0)
     assert lib.sa_decode(ctypes.byref(sh), ctypes.byref(dp), ctypes.byref(ok_sp), p, p, p, None,
                          ctypes.byref(sel), p, p, 1 << 30, None) == sa.SA_ERR_INVALID_ARG
-    assert lib.sa_block_summaries(ctypes.byref(sh), p, 10, 5, p, p, None) == sa.SA_ERR_INVALID_ARG
-    assert lib.sa_block_summaries(ctypes.byref(sh), p, 0, 4096, p, p, None) == sa.SA_ERR_INVALID_ARG
-    assert lib.sa_block_summaries(ctypes.byref(sh), p, 3, 3, p, p, None) == sa.SA_OK   # empty range: no launch
+    assert lib.sa_block_summaries(ctypes.byref(sh), p, 10, 5, p, p, p, p, p, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_block_summaries(ctypes.byref(sh), p, 0, 4096, p, p, p, p, p, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_block_summaries(ctypes.byref(sh), p, 0, 8, p, p, p, None, p, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_block_summaries(ctypes.byref(sh), p, 0, 8, p, p, None, p, p, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_block_summaries(ctypes.byref(sh), p, 3, 3, p, p, p, p, p, None) == sa.SA_OK   # empty range: no launch
+    assert lib.sa_block_sketch(ctypes.byref(sh), p, p, 10, 5, p, p, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_block_sketch(ctypes.byref(sh), p, p, 0, 8, p, ctypes.c_void_p(0x10008), None) == sa.SA_ERR_INVALID_ARG   # misaligned
+    assert lib.sa_block_sketch(ctypes.byref(sh), p, None, 0, 8, p, p, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_block_sketch(ctypes.byref(sh), p, p, 3, 3, p, p, None) == sa.SA_OK
 
 
 def test_status_strings(lib):

@@ -192,15 +192,18 @@ def test_deterministic_outputs(dev):
 def test_block_summaries_entry_point(dev):
     w, data = _data("bf16_d128_g4", dev)
     st = sa.prefill_stats(data["q_ctx"], data["k"], data["v"])
-    bm = st.blk_mean.clone()
+    bm, code, meta = st.blk_mean.clone(), st.blk_code.clone(), st.blk_meta.clone()
     st.blk_mean.zero_()
     st.kbar_absmax.zero_()
+    st.blk_code.zero_()
+    st.blk_meta.zero_()
     nb = w.L // 16
     sa.block_summaries(data["k"], 0, nb // 3, st, w.Hq)
     sa.block_summaries(data["k"], nb // 3, nb, st, w.Hq)
     torch.cuda.synchronize()
     assert torch.equal(st.blk_mean, bm)
     assert torch.equal(st.kbar_absmax, bm.float().abs().amax(dim=(2, 3)))
+    assert torch.equal(st.blk_code, code) and torch.equal(st.blk_meta, meta)
 
 
 @pytest.mark.parametrize("wname,units", [("llama", [(0, 0), (0, 3), (0, 7)]),

@@ -36,6 +36,12 @@ def _summaries(pattern, B, Hkv, nb, d, dt, q, G, gen):
         dirn = qbar / qbar.norm(dim=-1, keepdim=True) ** 2
         ramp = torch.linspace(-4.0, 4.0, nb).view(1, 1, nb, 1)
         m = ramp * dirn.unsqueeze(2) * 16.0 + 0.01 * torch.randn(B, Hkv, nb, d, generator=gen)
+    elif pattern == "near":
+        # one common row plus a 1e-3 perturbation: every score lies within
+        # the sketch's error bound of the others, so the band is most of the
+        # candidates and the exact rescoring decides
+        base = torch.randn(B, Hkv, 1, d, generator=gen)
+        m = base + 1e-3 * torch.randn(B, Hkv, nb, d, generator=gen)
     elif pattern == "ties":
         # rows drawn from five distinct vectors: many exactly equal scores
         base = torch.randn(B, Hkv, 5, d, generator=gen)
@@ -46,7 +52,7 @@ def _summaries(pattern, B, Hkv, nb, d, dt, q, G, gen):
     return m.to(dt)
 
 
-@pytest.mark.parametrize("pattern", ["random", "ascending", "ties"])
+@pytest.mark.parametrize("pattern", ["random", "ascending", "ties", "near"])
 @pytest.mark.parametrize("name", list(SHAPES))
 def test_select_one_cta_per_unit(name, pattern):
     dtype, d, Hq, Hkv, B, L = SHAPES[name]
@@ -60,6 +66,8 @@ def test_select_one_cta_per_unit(name, pattern):
     st = sa.Stats(B, Hq, Hkv, L, d, dt, dev)
     st.blk_mean.copy_(bm.to(dev))
     st.kbar_absmax.copy_(bm.float().abs().amax(dim=(2, 3)).to(dev))
+    st.mu_k.copy_(bm.float().mean(2).to(dev))          # the sketch's centre
+    sa.block_sketch(st, Hq)
     qd = q.to(dev)
     n_cand = len(osel.candidate_blocks(L, SINK, LOCAL))
     for k in (1, 8, 32, 33, n_cand - 1):
@@ -76,6 +84,31 @@ def test_select_one_cta_per_unit(name, pattern):
                 assert (blk[b, g, len(blocks):] == -1).all()
                 pos = orng.sample_positions(77, b, g, 3, tail, 48)
                 np.testing.assert_array_equal(samp[b, g], pos, err_msg=str((name, pattern, k, b, g)))
+
+
+def test_select_wide_band_beyond_shared_memory():
+    """Near-equal scores over 1012 candidates: the band exceeds the 512
+    members ranked in shared memory and goes through the exact 64-bit keys in
+    the workspace."""
+    B, Hq, Hkv, d, L = 20, 32, 8, 128, 16384
+    G = Hq // Hkv
+    dev = torch.device("cuda")
+    gen = torch.Generator().manual_seed(4242)
+    q = torch.randn(B, Hq, d, generator=gen).to(torch.bfloat16)
+    bm = _summaries("near", B, Hkv, L // 16, d, torch.bfloat16, q.float(), G, gen)
+    st = sa.Stats(B, Hq, Hkv, L, d, torch.bfloat16, dev)
+    st.blk_mean.copy_(bm.to(dev))
+    st.mu_k.zero_()                                     # uncentred sketch
+    sa.block_sketch(st, Hq)
+    for k in (8, 40):
+        sp = sa.SelectParams(sink=SINK, local=LOCAL, k_blocks=k)
+        sel = sa.select(q.to(dev), st, sp)
+        torch.cuda.synchronize()
+        blk = sel.blk_idx.cpu().numpy()
+        assert int(sel.n_rescored.max()) > 512
+        for b, g in [(0, 0), (7, 3), (19, 7), (11, 5)]:
+            blocks, _, _ = osel.select_unit(f64(q[b, g * G:(g + 1) * G]), f64(bm[b, g]), L, SINK, LOCAL, k)
+            np.testing.assert_array_equal(blk[b, g], blocks)
 
 
 def test_no_wait_gave_up():

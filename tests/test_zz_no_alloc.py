@@ -57,7 +57,7 @@ def test_noalloc_rejects_shapes_beyond_its_array():
     cp = sa.SelectParams(k_blocks=8).c()
     assert sa._lib().sa_workspace_size(ctypes.byref(shape), ctypes.byref(cp), sa.OP_SELECT) > (8 << 20)
     p = ctypes.c_void_p(0x10000)
-    st = sa.sa_stats(*([0x10000] * 8))
+    st = sa.sa_stats(*([0x10000] * 10))
     sel = sa.sa_selection(0x10000, 0x10000, 0x10000, 0)
     status = sa._lib().sa_select_noalloc(ctypes.byref(shape), ctypes.byref(cp), p, ctypes.byref(st), None, None,
                                          ctypes.byref(sel), 0.0, None)
