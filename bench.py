@@ -64,8 +64,10 @@ def parse_args(argv=None):
 # bytes the method must move (algorithmic), per unit = (sequence, KV head)
 
 def select_bytes_per_unit(w, sg, esz, b_draws):
-    """Block summaries of every candidate + the group's queries + outputs."""
-    return sg["n_cand"] * w.d * esz + w.G * w.d * esz + 4 * sg["kk"] + 4 * b_draws + 4
+    """Sketch of every candidate (int8 codes + 16 bytes of scale and bounds)
+    + the group's queries + outputs.  The bf16 rows of the band that is
+    rescored exactly (data-dependent, typically a dozen rows) are not counted."""
+    return sg["n_cand"] * (w.d + 16) + w.G * w.d * esz + 4 * sg["kk"] + 4 * b_draws + 4
 
 
 def decode_bytes_per_unit(w, sg, esz, mode, b_draws):
@@ -464,7 +466,7 @@ def main(argv=None):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded generator, Llama-3.1-8B layer shapes)",
             "config": workload_config(w, sg, args),
-            "roofline": {"bound": "hbm", "kernel": "k_select (block scoring + top-k)", "achieved": sel_gbs,
+            "roofline": {"bound": "hbm", "kernel": "k_select (sketch scan + certified top-k)", "achieved": sel_gbs,
                          "peak": peak, "unit": "GB/s", "frac": sel_gbs / peak, "traffic": traffic,
                          "bytes_per_launch": sel_b, "us_per_launch": 1e3 * sel_avg, "peak_source": peak_src},
             "step_roofline": {"achieved": step_gbs, "frac": step_gbs / peak, "bytes_per_step": sel_b + dec_b,

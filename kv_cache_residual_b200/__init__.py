@@ -62,7 +62,7 @@ class sa_decode_params(ctypes.Structure):
 
 EXPORTS = ("sa_workspace_size", "sa_prefill_stats", "sa_block_summaries", "sa_block_sketch", "sa_select",
            "sa_select_noalloc",
-           "sa_decode", "sa_step", "sa_dense_decode", "sa_wait_timeouts", "sa_status_string")
+           "sa_decode", "sa_step", "sa_step_fused", "sa_dense_decode", "sa_wait_timeouts", "sa_status_string")
 
 _LIB = None
 
@@ -87,6 +87,8 @@ def _lib():
         lib.sa_decode.argtypes = [sh, dp, sp, P, P, P, st, sel, P, P, S, P]
         lib.sa_step.argtypes = [sh, dp, sp, P, P, P, st, sel, P, P, S, P]
         lib.sa_dense_decode.argtypes = [sh, P, P, P, P, F, P, S, P]
+        lib.sa_step_fused.argtypes = [sh, dp, sp]
+        lib.sa_step_fused.restype = I
         lib.sa_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
         lib.sa_wait_timeouts.restype = I
         lib.sa_status_string.argtypes = [I]
@@ -267,8 +269,9 @@ def decode(q, k, v, stats, selection, params, mode="resa", lam=1.0, scale=0.0, o
 
 
 def step(q, k, v, stats, params, mode="resa", lam=1.0, scale=0.0, selection=None, out=None, stream=None):
-    """Selection then decode in one call (the decode overlaps the end of the
-    selection through programmatic dependent launch).  Returns (out, selection)."""
+    """Selection then decode in one call: one fused kernel when step_fused()
+    says so, else the two kernels with the decode overlapping the end of the
+    selection (programmatic dependent launch).  Returns (out, selection)."""
     B, Hq, d = q.shape
     shape = make_shape(k, Hq)
     cp = params.c()
@@ -284,6 +287,16 @@ def step(q, k, v, stats, params, mode="resa", lam=1.0, scale=0.0, selection=None
                           ctypes.byref(st), ctypes.byref(sel), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
            "sa_step")
     return out, selection
+
+
+def step_fused(q, k, params, mode="resa"):
+    """True when step() runs as the single fused kernel for these arguments."""
+    shape = make_shape(k, q.shape[1])
+    r = _lib().sa_step_fused(ctypes.byref(shape), ctypes.byref(sa_decode_params(MODES[mode], 1.0, 0.0)),
+                             ctypes.byref(params.c()))
+    if r < 0:
+        raise SAError(SA_ERR_INVALID_ARG, "sa_step_fused")
+    return r == 1
 
 
 def dense_decode(q, k, v, scale=0.0, out=None, stream=None):

@@ -204,7 +204,12 @@ inline cudaError_t opt_in_smem(K kernel, size_t bytes, std::atomic<unsigned long
 }
 
 cudaError_t launch_select(const Dims& d, const SelectPlan& p, const SelectArgs& a, cudaStream_t s);
-cudaError_t select_wait_timeouts(unsigned* count);    // CTAs of the selection kernel that gave up a wait
+cudaError_t select_wait_timeouts(unsigned* count);
+
+// The fused step (selection + decode in one kernel, sa_fused.cu): whether it
+// applies to this step, and its launch.
+bool fused_step_ok(const Dims& d, const SelectPlan& sp, const DecodePlan& dp, const sa_select_params& prm,
+                   int mode);    // CTAs of the selection kernel that gave up a wait
 
 struct DecodeArgs {
     const void* q; const void* k; const void* v; sa_stats st; sa_selection sel;
@@ -212,6 +217,8 @@ struct DecodeArgs {
     bool pdl;          // launched as a programmatic dependent of the selection kernel
 };
 cudaError_t launch_decode(const Dims& d, const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_step_fused(const Dims& d, const SelectPlan& sp, const SelectArgs& sa_, const DecodePlan& dp,
+                              const DecodeArgs& da, cudaStream_t s);
 
 struct DenseArgs {
     const void* q; const void* k; const void* v; float scale; float* out; char* ws;

@@ -35,7 +35,7 @@ def test_byte_model_batched():
     g = bench.set_geom(w.L, w.sink, w.local, kb)
     assert kb == 8 and g["n_i"] == 320
     sel = bench.select_bytes_per_unit(w, g, 2, 0)
-    assert sel == 2036 * 128 * 2 + 4 * 128 * 2 + 4 * 8 + 4
+    assert sel == 2036 * (128 + 16) + 4 * 128 * 2 + 4 * 8 + 4
     dec = bench.decode_bytes_per_unit(w, g, 2, "resa", 0)
     assert dec == 320 * 2 * 128 * 2 + 4 * 128 * 2 + 4 * 8 + 4 * 128 * 4 + 4 * (2 * 128 + 1) * 4 + 128 * 4
 
