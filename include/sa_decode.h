@@ -252,11 +252,12 @@ SA_API sa_status sa_step(const sa_shape* shape, const sa_decode_params* dparams,
                          size_t ws_bytes, void* stream);
 
 /* 1 when sa_step runs this step as one fused kernel (selection and decode
- * by the same CTA, one CTA per unit: bf16 cache, B*Hkv large enough that each
- * unit gets a CTA of its own, k_blocks <= 32 and, for SA_SAMPLE, sample_cap
- * <= 256), 0 when it runs the selection and decode kernels as a programmatic
- * pair, -1 on invalid arguments.  Both give the same results.  Diagnostic:
- * the pages have no counterpart. */
+ * by the same CTA, one CTA per unit), 0 when it runs the selection and decode
+ * kernels as a programmatic pair, -1 on invalid arguments.  The fused kernel
+ * is opt-in (environment variable SA_FUSED_STEP=1, read at every call) and
+ * then used for a bf16 cache with B*Hkv large enough that each unit gets a
+ * CTA of its own, k_blocks <= 32 and, for SA_SAMPLE, sample_cap <= 256.  Both
+ * paths give the same results.  Diagnostic: the pages have no counterpart. */
 SA_API int sa_step_fused(const sa_shape* shape, const sa_decode_params* dparams,
                          const sa_select_params* sparams);
 

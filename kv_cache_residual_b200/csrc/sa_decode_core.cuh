@@ -43,7 +43,32 @@ __device__ void decode_epilogue(const float* recs, int nsd, int rec, const T* qg
                                 float* s_acc, float* s_acc0, float* s_ml, float* s_t, float* s_hs) {
     constexpr bool PRIOR = (MODE == SA_RESA);
     constexpr bool SUMS = (MODE == SA_PROXY);
+    constexpr int kPer = (G * D + 127) / 128;    // output elements per thread (>= 128 threads)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    // RESA: the statistics the output needs are loaded first, so that their
+    // latency overlaps the combination of the records: O_Est and ln Z0 of
+    // this thread's outputs, and the per-head bias c_h = s (q_h - mu_Q,h) . mu_K
+    float oe[kPer], lz[kPer];
+    if constexpr (PRIOR) {
+        if (nt > 0) {
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+                const int idx = threadIdx.x + k * blockDim.x;
+                const size_t qh = (size_t)b * Hq + g * G + (idx < G * D ? idx / D : 0);
+                oe[k] = idx < G * D ? st.o_est[qh * D + idx % D] : 0.f;
+                lz[k] = idx < G * D ? st.log_z0[qh] : 0.f;
+            }
+            for (int h = warp; h < G; h += nwarps) {
+                const size_t qh = (size_t)b * Hq + g * G + h;
+                float x = 0.f;
+#pragma unroll
+                for (int e = lane; e < D; e += 32)
+                    x = fmaf(to_f32<T>(qg[(size_t)h * D + e]) - st.mu_q[qh * D + e], st.mu_k[(size_t)u * D + e], x);
+                x = group_sum<32>(x);
+                if (lane == 0) s_hs[h] = x * scale * kLog2e;
+            }
+        }
+    }
     combine_heads<G, D, SH>(recs, nsd, rec, 0, s_ml, s_ml + G);
     if constexpr (PRIOR) combine_heads<G, D, SH>(recs, nsd, rec, G * (2 + D), s_ml + 2 * G, s_ml + 3 * G);
     __syncthreads();
@@ -67,24 +92,21 @@ __device__ void decode_epilogue(const float* recs, int nsd, int rec, const T* qg
         }
     }
     __syncthreads();
-    // per-head scalar, one warp per head: RESA bias c_h = s (q_h - mu_Q,h) . mu_K,
-    // PROXY logit z_h = s q_h . kbar_T + ln n_T   (both in log2 units)
-    if ((PRIOR || SUMS) && nt > 0) {
+    // PROXY logit z_h = s q_h . kbar_T + ln n_T (log2 units), one warp per head
+    if (SUMS && nt > 0) {
         for (int h = warp; h < G; h += nwarps) {
-            const size_t qh = (size_t)b * Hq + g * G + h;
             float x = 0.f;
 #pragma unroll
-            for (int e = lane; e < D; e += 32) {
-                const float qe = to_f32<T>(qg[(size_t)h * D + e]);
-                if constexpr (PRIOR) x = fmaf(qe - st.mu_q[qh * D + e], st.mu_k[(size_t)u * D + e], x);
-                else x = fmaf(qe, s_t[e], x);
-            }
+            for (int e = lane; e < D; e += 32) x = fmaf(to_f32<T>(qg[(size_t)h * D + e]), s_t[e], x);
             x = group_sum<32>(x);
-            if (lane == 0) s_hs[h] = PRIOR ? x * scale * kLog2e : x * scale * kLog2e + log2f((float)nt);
+            if (lane == 0) s_hs[h] = x * scale * kLog2e + log2f((float)nt);
         }
     }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int idx = threadIdx.x + k * blockDim.x;
+        if (idx >= G * D) break;
         const int h = idx / D, e = idx - h * D;
         const size_t qh = (size_t)b * Hq + g * G + h;
         const float M = s_ml[h], Ls = s_ml[G + h], A = s_acc[idx];
@@ -96,14 +118,14 @@ __device__ void decode_epilogue(const float* recs, int nsd, int rec, const T* qg
             //   Z (log2) = log2 A_h + c_h; prior mass at I = l0 2^(m0 + c);
             //   tail D_T = Z (1 - l0 2^(m0 - log2 A)) clamped at 0,
             //   tail N_T = Z (O_Est - acc0 2^(m0 - log2 A))
-            const float lz = st.log_z0[qh] * kLog2e;
-            const float zl = lz + s_hs[h];
+            const float lz2 = lz[k] * kLog2e;
+            const float zl = lz2 + s_hs[h];
             const float M0 = s_ml[2 * G + h], L0 = s_ml[3 * G + h];
-            const float rI = (M0 == -INFINITY) ? 0.f : ex2(M0 - lz);
+            const float rI = (M0 == -INFINITY) ? 0.f : ex2(M0 - lz2);
             const float Mx = fmaxf(M, zl);
             const float wI = (M == -INFINITY) ? 0.f : ex2(M - Mx);
             const float wT = lambda * ex2(zl - Mx);
-            const float num = A * wI + wT * (st.o_est[qh * D + e] - s_acc0[idx] * rI);
+            const float num = A * wI + wT * (oe[k] - s_acc0[idx] * rI);
             const float den = Ls * wI + wT * fmaxf(0.f, 1.f - L0 * rI);
             o = den > 0.f ? num / den : 0.f;
         } else {
@@ -309,16 +331,20 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
     const int ntiles = (n_hi + kTcTile - 1) / kTcTile;
     const int tile0 = chunk * tpc, tile1 = min(ntiles, tile0 + tpc);
 
-    // K/V rows of tile i into its stage (cp.async; masked rows zero-filled).
-    // The tile's row positions go to the stage first (one barrier), so the
-    // copy loop reads one shared word per 16-byte chunk.
-    auto issue = [&](int i) {
+    // Row positions of tile i go to its stage's pos array (every thread
+    // calls this at the same point; a barrier must follow before the copy).
+    auto put_pos = [&](int i) {
         if (i < tile1) {
             if ((i + 1) * kTcTile > n_indep) wait_selection();
-            unsigned char* sb = smem + (size_t)(i % kStages) * SB;
-            int* pos = reinterpret_cast<int*>(sb + 2 * TB);
+            int* pos = reinterpret_cast<int*>(smem + (size_t)(i % kStages) * SB + 2 * TB);
             if (threadIdx.x < kTcTile) pos[threadIdx.x] = pos_of(i * kTcTile + threadIdx.x);
-            __syncthreads();
+        }
+    };
+    // K/V rows of tile i into its stage (cp.async; masked rows zero-filled)
+    auto copy_tile = [&](int i) {
+        if (i < tile1) {
+            unsigned char* sb = smem + (size_t)(i % kStages) * SB;
+            const int* pos = reinterpret_cast<const int*>(sb + 2 * TB);
             constexpr int CPR = D / 8;
             const uint32_t sk = tc::smem_u32(sb), sv = sk + TB;
 #pragma unroll 4
@@ -338,9 +364,13 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
         tc::cp_commit();
     };
 
-    // first tiles in flight before the query / prior fragments are loaded
-#pragma unroll
-    for (int i = 0; i < kStages - 1; ++i) issue(tile0 + i);
+    // first two tiles in flight before the query / prior fragments are loaded
+    static_assert(kStages == 3, "the loop below keeps two tiles in flight");
+    put_pos(tile0);
+    put_pos(tile0 + 1);
+    __syncthreads();
+    copy_tile(tile0);
+    copy_tile(tile0 + 1);
     tc::WarpAttn<D, G, PRIOR> wa;
     {
         const int gh = min(lane >> 2, G - 1);
@@ -348,9 +378,12 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
     }
     float ks[2] = {0.f, 0.f};      // SUMS: this thread's column pair of K (c < D/2) or V (c >= D/2)
     for (int i = tile0; i < tile1; ++i) {
-        issue(i + kStages - 1);
-        tc::cp_wait<kStages - 1>();
-        __syncthreads();
+        // stage (i+2)%3 was last read by tile i-1, finished before the
+        // trailing barrier of the previous iteration
+        put_pos(i + 2);
+        tc::cp_wait<1>();           // this thread's copies of tile i have landed
+        __syncthreads();            // everyone's, and the positions of tile i+2
+        copy_tile(i + 2);
         unsigned char* sb = smem + (size_t)(i % kStages) * SB;
         const int base = i * kTcTile;
         if constexpr (SUMS) {
@@ -385,7 +418,7 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
             const uint32_t sk = tc::smem_u32(sb);
             wa.step16(sk, sk + TB, r0, xadd, in_i, qscale);
         }
-        __syncthreads();              // this stage is refilled by a later issue()
+        __syncthreads();              // stage i%3 is refilled for tile i+3
     }
     tc::cp_wait<0>();
     __syncthreads();

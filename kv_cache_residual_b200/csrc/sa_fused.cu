@@ -5,10 +5,11 @@
 // window + top-k, then attention over I_f and the sampled tail; RESA, Method:
 // the prior merge over I).
 //
-// k_step_fused: grid (B*Hkv), 128 threads, two CTAs per SM.  Used when every
-// unit gets a CTA of its own (enough units to fill the GPU), the cache is
-// bf16, k <= 32 blocks and the draws fit a shared list; otherwise sa_step runs
-// the selection and decode kernels as a programmatic pair.  The results are
+// k_step_fused: grid (B*Hkv), 128 threads, two CTAs per SM.  Used, when the
+// environment variable SA_FUSED_STEP is 1, where every unit gets a CTA of its
+// own (enough units to fill the GPU), the cache is bf16, k <= 32 blocks and
+// the draws fit a shared list; otherwise sa_step runs the selection and
+// decode kernels as a programmatic pair.  The results are
 // the ones of the two kernels: the same device code (select_unit,
 // stream_unit) runs on the same data in the same order.
 //
@@ -18,6 +19,8 @@
 // selection across (chosen blocks, draws).  The sink and window rows, which do
 // not depend on the selection, are prefetched into L2 with bulk prefetches at
 // the start, so the stream pass finds them there.
+#include <cstdlib>
+
 #include "sa_decode_core.cuh"
 #include "sa_select_core.cuh"
 
@@ -70,6 +73,19 @@ k_step_fused(SelectIo sio, StreamIo dio) {
             bulk_prefetch_l2(dio.k + w0, (uint32_t)g.w_eff * rb);
             bulk_prefetch_l2(dio.v + w0, (uint32_t)g.w_eff * rb);
         }
+        // and the decode's per-unit statistics
+        const int b = u / dio.Hkv, gg = u - b * dio.Hkv;
+        const size_t qh0 = (size_t)b * dio.Hq + (size_t)gg * G;
+        if constexpr (MODE == SA_RESA) {
+            bulk_prefetch_l2(dio.st.mu_q + qh0 * D, G * D * 4);
+            bulk_prefetch_l2(dio.st.o_est + qh0 * D, G * D * 4);
+            bulk_prefetch_l2(dio.st.mu_k + (size_t)u * D, D * 4);
+            prefetch_l2(dio.st.log_z0 + qh0);
+        }
+        if constexpr (MODE == SA_PROXY) {
+            bulk_prefetch_l2(dio.st.sum_k + (size_t)u * D, D * 4);
+            bulk_prefetch_l2(dio.st.sum_v + (size_t)u * D, D * 4);
+        }
     }
 
     const SelectSmem sm{hist, sw, misc, s_qh, s_qi, s_qc, ukeys, nullptr, s_sorted, smem, bar, s_samp,
@@ -92,6 +108,10 @@ k_step_fused(SelectIo sio, StreamIo dio) {
 // must be a single chunk per unit so that the result is the two kernels' one.
 bool fused_step_ok(const Dims& d, const SelectPlan& sp, const DecodePlan& dp, const sa_select_params& prm,
                    int mode) {
+    // opt-in: on the 32-sequence 32K workload the programmatic pair of kernels
+    // is faster (the fused CTA has 4 warps for the latency-bound decode)
+    const char* env = getenv("SA_FUSED_STEP");
+    if (env == nullptr || env[0] != '1') return false;
     if (!d.bf16 || sp.nss != 1 || sp.g.n_cand > kSmemKeys || sp.g.kk > kWarpTopK || dp.nsd != 1) return false;
     if (mode == SA_SAMPLE && prm.sample_cap > kSampCache) return false;
     return true;

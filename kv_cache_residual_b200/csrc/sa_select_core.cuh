@@ -292,13 +292,9 @@ __device__ void merge_warp_lists(const unsigned long long* s_cand, int kk, unsig
     __syncthreads();
 }
 
-// Sorts s_list[0..kk) (kk <= 32) by block index and writes c_lo + index in
-// ascending order (one warp, bitonic network over the 32 lanes).
-__device__ __forceinline__ void emit_sorted_list(const unsigned long long* s_list, int kk, int c_lo, int32_t* out_idx,
-                                 int* s_sorted) {
-    if (threadIdx.x >= 32) return;
-    const int lane = threadIdx.x;
-    int v = lane < kk ? comp_index(s_list[lane]) : 0x7fffffff;
+// Ascending sort of one int per lane across the warp (bitonic network).
+__device__ __forceinline__ int warp_sort_asc(int v) {
+    const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int size = 2; size <= 32; size <<= 1) {
 #pragma unroll
@@ -309,6 +305,16 @@ __device__ __forceinline__ void emit_sorted_list(const unsigned long long* s_lis
             v = (lower == up) ? min(v, o) : max(v, o);
         }
     }
+    return v;
+}
+
+// Sorts s_list[0..kk) (kk <= 32) by block index and writes c_lo + index in
+// ascending order (one warp).
+__device__ __forceinline__ void emit_sorted_list(const unsigned long long* s_list, int kk, int c_lo,
+                                                 int32_t* out_idx, int* s_sorted) {
+    if (threadIdx.x >= 32) return;
+    const int lane = threadIdx.x;
+    const int v = warp_sort_asc(lane < kk ? comp_index(s_list[lane]) : 0x7fffffff);
     if (lane < kk) {
         out_idx[lane] = c_lo + v;
         s_sorted[lane] = c_lo + v;
@@ -511,14 +517,16 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
         mbar_init_fence();
     }
     __syncthreads();
+    // the sketch is read once per step: evict-first in L2
+    const uint64_t pol = l2_evict_first_policy();
     auto issue = [&](int j) {                      // thread 0
         if (j < nst) {
             const int rj = min(Ring::SR, nrows - j * Ring::SR);
             const uint32_t bar = bar0 + 8 * (j % Ring::kStages);
             const uint32_t dst = ring + (j % Ring::kStages) * Ring::kStageBytes;
             mbar_arrive_expect_tx(bar, (uint32_t)rj * (D + 16));
-            bulk_g2s(dst, code0 + (size_t)j * Ring::SR * D, (uint32_t)rj * D, bar);
-            bulk_g2s(dst + Ring::kCodeBytes, meta0 + (size_t)j * Ring::SR, (uint32_t)rj * 16, bar);
+            bulk_g2s_hint(dst, code0 + (size_t)j * Ring::SR * D, (uint32_t)rj * D, bar, pol);
+            bulk_g2s_hint(dst + Ring::kCodeBytes, meta0 + (size_t)j * Ring::SR, (uint32_t)rj * 16, bar, pol);
         }
     };
     if (threadIdx.x == 0)
@@ -755,6 +763,7 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
     int rescored = 0;
     bool sorted_smem = false;          // the chosen indices are also in s_sorted
     if (kk > 0 && kk < n) {
+        if (threadIdx.x == 0) s_nb = 0;        // band counter (barriers follow on every path)
         auto k32 = [&](int i) -> uint32_t { return lk[i]; };
         const bool fast = kk <= kWarpTopK && n <= kSmemKeys;
         uint32_t thr;
@@ -770,10 +779,25 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
         }
         // thr = the kk-th largest lower bound.  A candidate whose upper bound is
         // below it is beaten strictly by kk others, so the exact top kk lies
-        // in the band {upper >= thr}, which contains the kk best lower bounds
-        int band = 0;
-        for (int i = threadIdx.x; i < n; i += NT) band += (uk[i] >= thr) ? 1 : 0;
-        band = block_sum<NT>(band, sw);
+        // in the band {upper >= thr}, which contains the kk best lower bounds.
+        // One pass counts the band and lists its members (the first kBandCap
+        // of them, in no particular order) in s_bidx.
+        for (int i0 = warp * 32; i0 < n; i0 += NT) {
+            const int i = i0 + lane;
+            const bool in = i < n && uk[i] >= thr;
+            const unsigned m = __ballot_sync(0xffffffffu, in);
+            if (m != 0u) {
+                int base = 0;
+                if (lane == 0) base = atomicAdd(&s_nb, __popc(m));
+                base = __shfl_sync(0xffffffffu, base, 0);
+                if (in) {
+                    const int pos = base + __popc(m & ((1u << lane) - 1u));
+                    if (pos < kBandCap) s_bidx[pos] = i;
+                }
+            }
+        }
+        __syncthreads();
+        const int band = s_nb;
         if (band == kk) {
             if (fast) {
                 emit_sorted_list(s_list, kk, sg.c_lo, out_idx, s_sorted);
@@ -785,12 +809,28 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
             // among them by (x desc, index asc)
             rescored = band;
             const T* bm = blk_mean + ((size_t)u * nb + sg.c_lo) * D;
-            if (band <= kBandCap) {
-                if (threadIdx.x == 0) s_nb = 0;
+            if (band <= 32) {
+                rescore_members<T, D, G, NW>(bm, s_bidx, band, s_qh, s_bx);
                 __syncthreads();
-                for (int i = threadIdx.x; i < n; i += NT)
-                    if (uk[i] >= thr) s_bidx[atomicAdd(&s_nb, 1)] = i;
-                __syncthreads();
+                // one warp: lane j ranks member j, then the chosen are sorted by index
+                if (warp == 0) {
+                    const bool live = lane < band;
+                    const double xj = live ? s_bx[lane] : -INFINITY;
+                    const int ij = live ? s_bidx[lane] : 0x7fffffff;
+                    int rank = 0;
+                    for (int m = 0; m < band; ++m) {
+                        const double xm = __shfl_sync(0xffffffffu, xj, m);
+                        const int im = __shfl_sync(0xffffffffu, ij, m);
+                        rank += (xm > xj || (xm == xj && im < ij)) ? 1 : 0;
+                    }
+                    const int v = warp_sort_asc((live && rank < kk) ? ij : 0x7fffffff);
+                    if (lane < kk) {
+                        out_idx[lane] = sg.c_lo + v;
+                        s_sorted[lane] = sg.c_lo + v;
+                    }
+                }
+                sorted_smem = true;
+            } else if (band <= kBandCap) {
                 rescore_members<T, D, G, NW>(bm, s_bidx, band, s_qh, s_bx);
                 __syncthreads();
                 for (int j = threadIdx.x; j < band; j += NT) {

@@ -2,6 +2,8 @@
 CTA): it is taken exactly where its conditions hold, its outputs and
 selections equal the two-kernel path bit for bit, and sampled units match
 the oracle."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -16,6 +18,18 @@ MODES = ("drop", "resa", "proxy", "sample")
 
 # 38 x 4 = 152 units: one CTA per unit, one decode chunk per unit
 WIDE = synth.scaled(synth.WORKLOADS["llama"], B=38, Hq=16, Hkv=4, L=2048, n_hh=8, seed=21)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def fused_on():
+    """The fused kernel is opt-in: on for this module only."""
+    old = os.environ.get("SA_FUSED_STEP")
+    os.environ["SA_FUSED_STEP"] = "1"
+    yield
+    if old is None:
+        del os.environ["SA_FUSED_STEP"]
+    else:
+        os.environ["SA_FUSED_STEP"] = old
 
 
 @pytest.fixture(scope="module")
@@ -37,6 +51,9 @@ def test_fused_taken_where_it_applies(wide):
     q, k = data["q"][0], data["k"]
     for m in MODES:
         assert sa.step_fused(q, k, _sp(), m)
+    os.environ["SA_FUSED_STEP"] = "0"
+    assert not sa.step_fused(q, k, _sp(), "resa")                       # opt-in only
+    os.environ["SA_FUSED_STEP"] = "1"
     assert not sa.step_fused(q, k, _sp(k_blocks=40), "resa")            # k above the warp lists
     assert not sa.step_fused(q, k, _sp(sample_b=300), "sample")         # draws beyond the shared list
     small = synth.scaled(synth.WORKLOADS["llama"], B=2, Hq=16, Hkv=4, L=2048, n_hh=8, seed=22)
