@@ -136,8 +136,11 @@ typedef struct {
  *   sample_b      draws per unit for SA_SAMPLE when clt_base == 0
  *   clt_base      > 0: choose b per unit by the CLT budget (vAttention, key
  *                 designs 2-3) from the first clt_base draws, target (eps,
- *                 delta) on the output, b clamped to [clt_base, min(n_T,
- *                 sample_cap)]; 0: fixed sample_b
+ *                 delta) on the output split evenly between numerator and
+ *                 denominator (Lemma 4.2), b clamped to [clt_base, min(n_T,
+ *                 sample_cap)]; requires 2 <= clt_base <= min(256,
+ *                 sample_cap), eps > 0, 0 < delta < 1 and k, v in sa_select;
+ *                 0: fixed sample_b
  *   sample_cap    capacity per unit of sa_selection.samp_idx (>= sample_b)
  *   seed, step    SplitMix64 stream of unit (b, g) at this step:
  *                 key = out(out(out(out(seed)^b)^g)^step), draw i =

@@ -40,7 +40,11 @@ sa_status check_select_params(const sa_select_params* p) {
         p->clt_base < 0)
         return SA_ERR_INVALID_ARG;
     if (p->sample_b > p->sample_cap) return SA_ERR_INVALID_ARG;
-    if (p->clt_base > 0) return SA_ERR_UNSUPPORTED;
+    if (p->clt_base > 0) {
+        if (p->clt_base < 2 || p->clt_base > p->sample_cap) return SA_ERR_INVALID_ARG;
+        if (!(p->eps > 0.f) || !(p->delta > 0.f && p->delta < 1.f)) return SA_ERR_INVALID_ARG;
+        if (p->clt_base > kCltMaxBase) return SA_ERR_UNSUPPORTED;
+    }
     return SA_OK;
 }
 
@@ -164,6 +168,8 @@ sa_status prep_select(const sa_shape* shape, const sa_select_params* params, con
     if (!aligned4(out->samp_count)) return SA_ERR_INVALID_ARG;
     if (params->sample_b > 0 && !aligned4(out->samp_idx)) return SA_ERR_INVALID_ARG;
     if (out->n_rescored != nullptr && !aligned4(out->n_rescored)) return SA_ERR_INVALID_ARG;
+    if (params->clt_base > 0 && (!aligned16(k) || !aligned16(v) || !aligned4(out->samp_idx)))
+        return SA_ERR_INVALID_ARG;                  // the CLT budget reads K and V
     *a = SelectArgs{q, *stats, k, v, *out, *params, resolve_scale(scale, d->d), nullptr};
     return SA_OK;
 }
@@ -215,7 +221,10 @@ sa_status sa_select(const sa_shape* shape, const sa_select_params* params, const
     if (e != SA_OK) return e;
     if (ws == nullptr || ws_bytes < p.bytes || !aligned16(ws)) return SA_ERR_WORKSPACE;
     a.ws = static_cast<char*>(ws);
-    return launch_select(d, p, a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+    if (launch_select(d, p, a, static_cast<cudaStream_t>(stream)) != cudaSuccess) return SA_ERR_CUDA;
+    if (params->clt_base > 0 && launch_clt(d, p, a, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return SA_ERR_CUDA;
+    return SA_OK;
 }
 
 sa_status sa_decode(const sa_shape* shape, const sa_decode_params* dparams, const sa_select_params* sparams,
@@ -256,6 +265,10 @@ sa_status sa_step(const sa_shape* shape, const sa_decode_params* dparams, const 
     if (fused_step_ok(d, ps, pd, *sparams, dparams->mode))
         return launch_step_fused(d, ps, as, pd, ad, s) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
     if (launch_select(d, ps, as, s) != cudaSuccess) return SA_ERR_CUDA;
+    if (sparams->clt_base > 0) {
+        // the budget kernel sits between: the decode waits for it as usual
+        if (launch_clt(d, ps, as, s) != cudaSuccess) return SA_ERR_CUDA;
+    }
     return launch_decode(d, pd, ad, s) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 

@@ -54,7 +54,8 @@ k_step_fused(SelectIo sio, StreamIo dio) {
     __shared__ float s_qc[3];
     __shared__ int s_sorted[kWarpTopK];
     __shared__ int s_samp[kSampCache];
-    extern __shared__ __align__(128) unsigned char smem[];
+    extern __shared__ __align__(128) unsigned char fsmem[];
+    unsigned char* smem = fsmem;
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Ring::kRingBytes);
     uint32_t* ukeys = reinterpret_cast<uint32_t*>(smem + Ring::kRingBytes + 128);
     const int u = blockIdx.x;
@@ -114,6 +115,7 @@ bool fused_step_ok(const Dims& d, const SelectPlan& sp, const DecodePlan& dp, co
     if (env == nullptr || env[0] != '1') return false;
     if (!d.bf16 || sp.nss != 1 || sp.g.n_cand > kSmemKeys || sp.g.kk > kWarpTopK || dp.nsd != 1) return false;
     if (mode == SA_SAMPLE && prm.sample_cap > kSampCache) return false;
+    if (prm.clt_base > 0) return false;             // the budget kernel runs between
     return true;
 }
 

@@ -205,6 +205,9 @@ inline cudaError_t opt_in_smem(K kernel, size_t bytes, std::atomic<unsigned long
 
 cudaError_t launch_select(const Dims& d, const SelectPlan& p, const SelectArgs& a, cudaStream_t s);
 cudaError_t select_wait_timeouts(unsigned* count);
+// The CLT sampling budget (sa_clt.cu), after the selection when clt_base > 0.
+constexpr int kCltMaxBase = 256;     // largest base sample
+cudaError_t launch_clt(const Dims& d, const SelectPlan& p, const SelectArgs& a, cudaStream_t s);
 
 // The fused step (selection + decode in one kernel, sa_fused.cu): whether it
 // applies to this step, and its launch.

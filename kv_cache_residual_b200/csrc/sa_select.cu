@@ -48,7 +48,9 @@ SelectIo select_io(const Dims& d, const SelectPlan& p, const SelectArgs& a) {
     io.samp_idx = a.sel.samp_idx;
     io.samp_count = a.sel.samp_count;
     io.n_rescored = a.sel.n_rescored;
-    io.sample_b = a.sp.sample_b; io.sample_cap = a.sp.sample_cap;
+    // with the CLT budget the selection draws the base sample only
+    io.sample_b = a.sp.clt_base > 0 ? a.sp.clt_base : a.sp.sample_b;
+    io.sample_cap = a.sp.sample_cap;
     io.seed = (unsigned long long)a.sp.seed;
     io.step = a.sp.step;
     return io;

@@ -90,6 +90,14 @@ def test_select_and_decode_param_checks(lib):
         assert lib.sa_select(ctypes.byref(sh), ctypes.byref(sp), p, ctypes.byref(st), None, None,
                              ctypes.byref(sel), 0.0, p, 1 << 30, None) == sa.SA_ERR_INVALID_ARG
     clt = sa.sa_select_params(64, 128, 8, 0, 64, 512, 0.05, 0.05, 0, 0)
+    # the CLT budget reads K and V
+    assert lib.sa_select(ctypes.byref(sh), ctypes.byref(clt), p, ctypes.byref(st), None, None,
+                         ctypes.byref(sel), 0.0, p, 1 << 30, None) == sa.SA_ERR_INVALID_ARG
+    for bad_clt, status in ((sa.sa_select_params(64, 128, 8, 0, 1, 512, 0.05, 0.05, 0, 0), sa.SA_ERR_INVALID_ARG),
+                            (sa.sa_select_params(64, 128, 8, 0, 300, 512, 0.05, 0.05, 0, 0), sa.SA_ERR_UNSUPPORTED),
+                            (sa.sa_select_params(64, 128, 8, 0, 64, 512, 0.05, 1.0, 0, 0), sa.SA_ERR_INVALID_ARG)):
+        assert lib.sa_select(ctypes.byref(sh), ctypes.byref(bad_clt), p, ctypes.byref(st), p, p,
+                             ctypes.byref(sel), 0.0, p, 1 << 30, None) == status
     ok_sp = sa.sa_select_params(64, 128, 8, 0, 0, 0, 0.05, 0.05, 0, 0)
     # workspace too small
     assert lib.sa_select(ctypes.byref(sh), ctypes.byref(ok_sp), p, ctypes.byref(st), None, None,

@@ -1,0 +1,122 @@
+"""GPU parity of the adaptive sampling budget (vAttention, Method, key
+designs 2 and 3) and of the long-context and flat workloads: per unit the
+budget b equals the oracle's (an integer decided in fp64 on both sides; a
+different summation order can only move it where the real-valued budget sits
+within rounding of an integer), the draws are the oracle's first b draws,
+and the sampled outputs are within the rel-L2 bar."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+import kv_cache_residual_b200 as sa
+from oracle import budget as obudget
+from parity_util import REL_L2_OUT, OracleUnit, f64, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_units(w, data, st, units, kb, eps, delta, b0, cap, step=1):
+    q = data["q"][step]
+    sp = sa.SelectParams(sink=w.sink, local=w.local, k_blocks=kb, sample_b=0, sample_cap=cap, clt_base=b0,
+                         eps=eps, delta=delta, seed=4321, step=step)
+    out, sel = sa.step(q, data["k"], data["v"], st, sp, mode="sample")
+    torch.cuda.synchronize()
+    counts = sel.samp_count.cpu().numpy()
+    for b, g in units:
+        o = OracleUnit(data, b, g, w.G, w.dtype)
+        qq = o.q(q)
+        blocks, idx, tail = o.select(qq, sp)
+        np.testing.assert_array_equal(sel.blk_idx[b, g].cpu().numpy()[:len(blocks)], blocks)
+        base = o.draws(tail, sp, b0)
+        want, det = obudget.clt_budget(qq, o.k, o.v, idx, base, o.scale, eps, delta, len(tail))
+        want = min(want, cap)
+        got = int(counts[b, g])
+        if got != want:
+            best = max(max(det["b_N"]), max(det["b_D"]))
+            assert math.isfinite(best) and abs(best - round(best)) <= 1e-9 * best, (b, g, got, want, best)
+        pos = o.draws(tail, sp, got)
+        np.testing.assert_array_equal(sel.samp_idx[b, g].cpu().numpy()[:got], pos)
+        e = rel_l2(f64(out[b, g * w.G:(g + 1) * w.G]), o.out("sample", qq, idx, pos=pos))
+        assert e < REL_L2_OUT, (b, g, e)
+    return counts
+
+
+@pytest.mark.parametrize("read", [0.01, 0.05])
+def test_clt_budget_small(read):
+    """Flat keys (no heavy hitters), 4K tokens: every unit checked."""
+    w = synth.scaled(synth.WORKLOADS["flat"], B=2, Hq=8, Hkv=2, L=4096, seed=31)
+    dev = torch.device("cuda")
+    data = synth.make_batch(w, device=dev, steps=2)
+    st = sa.prefill_stats(data["q_ctx"], data["k"], data["v"])
+    kb = w.k_blocks_for(read)
+    units = [(b, g) for b in range(w.B) for g in range(w.Hkv)]
+    for eps, delta in ((0.2, 0.05), (0.5, 0.2)):
+        counts = _check_units(w, data, st, units, kb, eps, delta, b0=64, cap=4096)
+        assert (counts >= 64).all()
+
+
+def test_clt_budget_capped():
+    """A tight target asks for more draws than the capacity: b = sample_cap."""
+    w = synth.scaled(synth.WORKLOADS["flat"], B=1, Hq=8, Hkv=2, L=4096, seed=32)
+    dev = torch.device("cuda")
+    data = synth.make_batch(w, device=dev, steps=2)
+    st = sa.prefill_stats(data["q_ctx"], data["k"], data["v"])
+    counts = _check_units(w, data, st, [(0, 0), (0, 1)], w.k_blocks_for(0.01), 0.01, 0.01, b0=32, cap=200)
+    assert (counts == 200).all()
+
+
+def test_clt_rejected_arguments():
+    w = synth.scaled(synth.WORKLOADS["flat"], B=1, Hq=8, Hkv=2, L=2048, seed=33)
+    dev = torch.device("cuda")
+    data = synth.make_batch(w, device=dev, steps=1)
+    st = sa.prefill_stats(data["q_ctx"], data["k"], data["v"])
+    # (the binding sizes the workspace first, which refuses them all; the
+    # statuses of sa_select itself are checked in test_abi.py)
+    for kw in (dict(clt_base=1, sample_cap=64), dict(clt_base=64, sample_cap=32),
+               dict(clt_base=300, sample_cap=400), dict(clt_base=64, sample_cap=64, eps=0.0)):
+        sp = sa.SelectParams(sink=w.sink, local=w.local, k_blocks=4, **kw)
+        with pytest.raises(sa.SAError):
+            sa.select(data["q"][0], st, sp, k=data["k"], v=data["v"])
+
+
+@pytest.mark.slow
+def test_flat_full_size_sampled_units():
+    """The flat workload at full size (32K, sigma_k = 0.25, no heavy hitters),
+    every read budget, CLT sampling; two units per budget against the oracle."""
+    w = synth.WORKLOADS["flat"]
+    dev = torch.device("cuda")
+    data = synth.make_batch(w, device=dev, steps=2)
+    st = sa.prefill_stats(data["q_ctx"], data["k"], data["v"])
+    for label, kb in w.budgets():
+        _check_units(w, data, st, [(0, 0), (5, 6)], kb, 0.1, 0.05, b0=64, cap=8192)
+
+
+@pytest.mark.slow
+def test_long_context_sampled_units():
+    """The 128K workload (B4) at both read budgets, every mode; two units per
+    budget against the oracle."""
+    w = synth.WORKLOADS["long"]
+    dev = torch.device("cuda")
+    data = synth.make_batch(w, device=dev, steps=2)
+    st = sa.prefill_stats(data["q_ctx"], data["k"], data["v"])
+    q = data["q"][1]
+    modes = ("drop", "resa", "proxy", "sample")
+    for label, kb in w.budgets():
+        sp = sa.SelectParams(sink=w.sink, local=w.local, k_blocks=kb, sample_b=64, sample_cap=64, seed=11, step=1)
+        outs = {}
+        for m in modes:
+            outs[m], sel = sa.step(q, data["k"], data["v"], st, sp, mode=m)
+        torch.cuda.synchronize()
+        for b, g in [(0, 1), (3, 7)]:
+            o = OracleUnit(data, b, g, w.G, w.dtype)
+            qq = o.q(q)
+            blocks, idx, tail = o.select(qq, sp)
+            np.testing.assert_array_equal(sel.blk_idx[b, g].cpu().numpy()[:len(blocks)], blocks)
+            pos = o.draws(tail, sp, 64)
+            np.testing.assert_array_equal(sel.samp_idx[b, g].cpu().numpy(), pos)
+            for m in modes:
+                e = rel_l2(f64(outs[m][b, g * w.G:(g + 1) * w.G]), o.out(m, qq, idx, pos=pos))
+                assert e < REL_L2_OUT, (label, b, g, m, e)
