@@ -4,6 +4,8 @@
 // sa_tc.cuh).
 #pragma once
 
+#include <type_traits>
+
 #include "sa_common.cuh"
 #include "sa_cta.cuh"
 #include "sa_internal.h"
@@ -371,8 +373,14 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
     __syncthreads();
     copy_tile(tile0);
     copy_tile(tile0 + 1);
-    tc::WarpAttn<D, G, PRIOR> wa;
-    {
+    // G <= 4: tokens on the MMA rows (no row spent on absent heads); G = 8:
+    // heads on the rows
+    constexpr bool kTokRows = (G <= 4);
+    using Engine = typename std::conditional<kTokRows, tc::WarpAttnT<D, G, PRIOR>, tc::WarpAttn<D, G, PRIOR>>::type;
+    Engine wa;
+    if constexpr (kTokRows) {
+        wa.init(qg, PRIOR ? st.mu_q + qh0 * D : nullptr);
+    } else {
         const int gh = min(lane >> 2, G - 1);
         wa.init(qg + (size_t)gh * D, PRIOR ? st.mu_q + (qh0 + gh) * D : nullptr);
     }
@@ -403,13 +411,23 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
         }
         const int r0 = warp * 16;
         if (base + r0 < n_tok) {
-            const int tq = lane & 3;
-            const int rows[4] = {r0 + 2 * tq, r0 + 2 * tq + 1, r0 + 8 + 2 * tq, r0 + 9 + 2 * tq};
-            float xadd[4];
-            bool in_i[4];
+            constexpr int NR = kTokRows ? 2 : 4;            // token rows of this lane
+            int rows[NR];
+            if constexpr (kTokRows) {
+                rows[0] = Engine::row(r0, 0);
+                rows[1] = Engine::row(r0, 1);
+            } else {
+                const int tq = lane & 3;
+                rows[0] = r0 + 2 * tq;
+                rows[1] = r0 + 2 * tq + 1;
+                rows[2] = r0 + 8 + 2 * tq;
+                rows[3] = r0 + 9 + 2 * tq;
+            }
+            float xadd[NR];
+            bool in_i[NR];
             const int* pos = reinterpret_cast<const int*>(sb + 2 * TB);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < NR; ++j) {
                 const int t = base + rows[j];
                 const bool ok = pos[rows[j]] >= 0;
                 xadd[j] = !ok ? -INFINITY : (t >= n_i ? lw_samp : 0.f);

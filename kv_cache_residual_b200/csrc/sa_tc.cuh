@@ -238,6 +238,165 @@ struct WarpAttn {
     }
 };
 
+// Tokens-on-M engine for G <= 4 (the usual GQA groups): the 16 tokens of a
+// warp are the M rows, the query columns the N dimension, so no MMA row is
+// spent on absent heads:
+//   S^T = K Q^T : A = K rows (ldmatrix), B = query columns in registers
+//                 (tile 0: q_0..q_{G-1}, then mu_Q hi of the G heads;
+//                  tile 1, RESA only: mu_Q lo at the same columns)
+//   O^T += V^T P^T : A = V rows (ldmatrix.trans), B = the weights, moved from
+//                 the S layout to the B layout with movmatrix.trans
+// Columns 0..G-1 carry the exact logits / weights and output, columns
+// G..2G-1 the RESA prior ones, so one 8-column MMA holds both.  Lane
+// (g = lane/4, t = lane%4) holds tokens g and g+8 of the step and columns
+// 2t, 2t+1; its O^T entries are dims (16 mt + g, + 8) of those columns.
+template <int D, int G, bool PRIOR>
+struct WarpAttnT {
+    static_assert(G <= 4, "the exact and prior columns share one 8-column tile");
+    static constexpr int KS = D / 16;   // k-steps over the head dim
+    static constexpr int MT = D / 16;   // 16-dim output tiles
+    static constexpr int NQ = PRIOR ? 2 : 1;
+    static constexpr int kRows = 2;     // token rows per lane per step
+    uint32_t qb[NQ][KS][2];
+    float o[MT][4];
+    float m[2], l[2];
+
+    // tile row of this lane's token j (0, 1) in the 16-token group at r0
+    __device__ static __forceinline__ int row(int r0, int j) { return r0 + ((threadIdx.x & 31) >> 2) + 8 * j; }
+
+    // qg: the G bf16 query rows of the unit; mu: the G fp32 typical queries
+    // (PRIOR only)
+    __device__ __forceinline__ void init(const __nv_bfloat16* qg, const float* mu) {
+        const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int dim = ks * 16 + 2 * t + 8 * half;
+                uint32_t v0 = 0u, v1 = 0u;
+                if (g < G) {
+                    v0 = *reinterpret_cast<const uint32_t*>(qg + (size_t)g * D + dim);
+                } else if (PRIOR && g < 2 * G) {
+                    const float2 x = *reinterpret_cast<const float2*>(mu + (size_t)(g - G) * D + dim);
+                    split_bf2(x.x, x.y, v0, v1);
+                }
+                qb[0][ks][half] = v0;
+                if constexpr (PRIOR) qb[NQ - 1][ks][half] = v1;
+            }
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) o[mt][j] = 0.f;
+        m[0] = m[1] = -INFINITY;
+        l[0] = l[1] = 0.f;
+    }
+
+    __device__ static __forceinline__ uint32_t trans8(uint32_t x) {
+        uint32_t y;
+        asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+        return y;
+    }
+
+    // 16 tokens at tile rows [r0, r0+16): xadd[j] = log2-weight added to the
+    // exact logit of token row(r0, j) (-inf masks it); in_i[j]: it belongs to I
+    __device__ __forceinline__ void step16(uint32_t k_tile, uint32_t v_tile, int r0, const float (&xadd)[2],
+                                           const bool (&in_i)[2], float qscale) {
+        constexpr int P = Pitch<D>::kBytes;
+        const int lane = threadIdx.x & 31, t = lane & 3;
+        float s[NQ][4];
+#pragma unroll
+        for (int nq = 0; nq < NQ; ++nq)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) s[nq][j] = 0.f;
+        const uint32_t ka = k_tile + (r0 + (lane & 7) + ((lane >> 3) & 1) * 8) * P + (lane >> 4) * 16;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            uint32_t a[4];
+            ldsm4(ka + ks * 32, a);
+#pragma unroll
+            for (int nq = 0; nq < NQ; ++nq) mma_bf16(s[nq], a[0], a[1], a[2], a[3], qb[nq][ks][0], qb[nq][ks][1]);
+        }
+        // logits of the lane's two tokens (j) and two columns (e)
+        float p[2][2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int c = 2 * t + e;
+            float x[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                if (c < G) x[j] = fmaf(s[0][2 * j + e], qscale, xadd[j]);
+                else if (PRIOR && c < 2 * G) x[j] = in_i[j] ? (s[0][2 * j + e] + s[NQ - 1][2 * j + e]) * qscale : -INFINITY;
+                else x[j] = -INFINITY;
+            }
+            // online softmax of column c over the 16 tokens (lanes with this t)
+            float mx = fmaxf(x[0], x[1]);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const float mn = fmaxf(m[e], mx);
+            const float sc = (m[e] == -INFINITY) ? 0.f : ex2(m[e] - mn);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) p[j][e] = (x[j] == -INFINITY) ? 0.f : ex2(x[j] - mn);
+            float ls = p[0][e] + p[1][e];
+            ls += __shfl_xor_sync(0xffffffffu, ls, 4);
+            ls += __shfl_xor_sync(0xffffffffu, ls, 8);
+            ls += __shfl_xor_sync(0xffffffffu, ls, 16);
+            if (mn != -INFINITY) {
+                l[e] = l[e] * sc + ls;
+                if (m[e] != mn) {
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) { o[mt][e] *= sc; o[mt][2 + e] *= sc; }
+                }
+                m[e] = mn;
+            }
+        }
+        // weights -> bf16 hi + lo, S layout (token, column pair) -> B layout
+        uint32_t h0, l0, h1, l1;
+        split_bf2(p[0][0], p[0][1], h0, l0);      // token g
+        split_bf2(p[1][0], p[1][1], h1, l1);      // token g + 8
+        const uint32_t bh0 = trans8(h0), bh1 = trans8(h1), bl0 = trans8(l0), bl1 = trans8(l1);
+        const uint32_t va = v_tile + (r0 + (lane & 7) + ((lane >> 4) & 1) * 8) * P + ((lane >> 3) & 1) * 16;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            uint32_t a[4];
+            ldsm4t(va + mt * 32, a);
+            mma_bf16(o[mt], a[0], a[1], a[2], a[3], bh0, bh1);
+            mma_bf16(o[mt], a[0], a[1], a[2], a[3], bl0, bl1);
+        }
+    }
+
+    // this warp's state into the arrays merge_warps reads (as WarpAttn::store)
+    __device__ __forceinline__ void store(float* ml, float* acc, float* acc0) const {
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int c = 2 * t + e;
+            const bool exact = c < G, prior = PRIOR && c >= G && c < 2 * G;
+            if (!exact && !prior) continue;
+            const int h = exact ? c : c - G;
+            float* a = (exact ? acc : acc0) + (warp * G + h) * D;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                a[mt * 16 + g] = o[mt][e];
+                a[mt * 16 + g + 8] = o[mt][2 + e];
+            }
+            if (g == 0) {
+                float* r = ml + (warp * G + h) * 4 + (exact ? 0 : 2);
+                r[0] = m[e];
+                r[1] = l[e];
+            }
+        }
+        if constexpr (!PRIOR) {
+            if (lane < G) {                      // the prior slots of a record without prior
+                float* r = ml + (warp * G + lane) * 4;
+                r[2] = -INFINITY;
+                r[3] = 0.f;
+            }
+        }
+    }
+};
+
 // Merge the stored states of `nw` warps (fixed warp order) into a split record
 // m[G], l[G], acc[G][D] (and the prior record right after it when PRIOR).
 template <int D, int G, bool PRIOR>
