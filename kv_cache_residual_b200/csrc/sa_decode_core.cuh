@@ -39,38 +39,65 @@ struct TokenMap {
 // out[b, h, :] for the G heads of the unit.  Record layout per split:
 // exact m[G], l[G], acc[G][D]; prior m0, l0, acc0 (same shape); ksum[D], vsum[D].
 // Shared scratch: s_acc, s_acc0 [G*D], s_ml [4G], s_t [2D], s_hs [G].
+// The statistics a RESA epilogue reads, loaded ahead of it: O_Est and ln Z0
+// of this thread's outputs (idx = threadIdx.x + k * blockDim.x) and the
+// per-head bias c_h = s (q_h - mu_Q,h) . mu_K (log2 units) in shared memory.
+template <int D, int G>
+struct EpiPre {
+    static constexpr int kPer = (G * D + 127) / 128;    // output elements per thread (>= 128 threads)
+    float oe[kPer], lz[kPer];
+};
+
+// Fills pre (every thread) and hs[G] (one warp per head); the caller puts a
+// barrier between this and the epilogue.
+template <typename T, int D, int G>
+__device__ __forceinline__ void epi_preload(EpiPre<D, G>& pre, float* hs, const T* qg, const sa_stats& st, int u,
+                                            int b, int g, int Hq, float scale) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+#pragma unroll
+    for (int k = 0; k < EpiPre<D, G>::kPer; ++k) {
+        const int idx = threadIdx.x + k * blockDim.x;
+        const size_t qh = (size_t)b * Hq + g * G + (idx < G * D ? idx / D : 0);
+        pre.oe[k] = idx < G * D ? st.o_est[qh * D + idx % D] : 0.f;
+        pre.lz[k] = idx < G * D ? st.log_z0[qh] : 0.f;
+    }
+    for (int h = warp; h < G; h += nwarps) {
+        const size_t qh = (size_t)b * Hq + g * G + h;
+        float x = 0.f;
+#pragma unroll
+        for (int e = lane; e < D; e += 32)
+            x = fmaf(to_f32<T>(qg[(size_t)h * D + e]) - st.mu_q[qh * D + e], st.mu_k[(size_t)u * D + e], x);
+        x = group_sum<32>(x);
+        if (lane == 0) hs[h] = x * scale * kLog2e;
+    }
+}
+
+// pre / hs_pre: RESA statistics already loaded by epi_preload (null: loaded
+// here, first, so that their latency overlaps the combination of the records)
 template <typename T, int D, int G, int MODE, bool SH = false>
-__device__ void decode_epilogue(const float* recs, int nsd, int rec, const T* qg, const sa_stats& st, int u,
-                                int b, int g, int Hq, int nt, float scale, float lambda, float* out,
-                                float* s_acc, float* s_acc0, float* s_ml, float* s_t, float* s_hs) {
+__device__ __forceinline__ void decode_epilogue(const float* recs, int nsd, int rec, const T* qg, const sa_stats& st,
+                                                int u, int b, int g, int Hq, int nt, float scale, float lambda,
+                                                float* out, float* s_acc, float* s_acc0, float* s_ml, float* s_t,
+                                                float* s_hs, const EpiPre<D, G>* pre = nullptr,
+                                                const float* hs_pre = nullptr) {
     constexpr bool PRIOR = (MODE == SA_RESA);
     constexpr bool SUMS = (MODE == SA_PROXY);
-    constexpr int kPer = (G * D + 127) / 128;    // output elements per thread (>= 128 threads)
+    constexpr int kPer = EpiPre<D, G>::kPer;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    // RESA: the statistics the output needs are loaded first, so that their
-    // latency overlaps the combination of the records: O_Est and ln Z0 of
-    // this thread's outputs, and the per-head bias c_h = s (q_h - mu_Q,h) . mu_K
-    float oe[kPer], lz[kPer];
+    EpiPre<D, G> loc;
+    const float* hsv = s_hs;
     if constexpr (PRIOR) {
         if (nt > 0) {
-#pragma unroll
-            for (int k = 0; k < kPer; ++k) {
-                const int idx = threadIdx.x + k * blockDim.x;
-                const size_t qh = (size_t)b * Hq + g * G + (idx < G * D ? idx / D : 0);
-                oe[k] = idx < G * D ? st.o_est[qh * D + idx % D] : 0.f;
-                lz[k] = idx < G * D ? st.log_z0[qh] : 0.f;
-            }
-            for (int h = warp; h < G; h += nwarps) {
-                const size_t qh = (size_t)b * Hq + g * G + h;
-                float x = 0.f;
-#pragma unroll
-                for (int e = lane; e < D; e += 32)
-                    x = fmaf(to_f32<T>(qg[(size_t)h * D + e]) - st.mu_q[qh * D + e], st.mu_k[(size_t)u * D + e], x);
-                x = group_sum<32>(x);
-                if (lane == 0) s_hs[h] = x * scale * kLog2e;
+            if (pre != nullptr) {
+                loc = *pre;
+                hsv = hs_pre;
+            } else {
+                epi_preload<T, D, G>(loc, s_hs, qg, st, u, b, g, Hq, scale);
             }
         }
     }
+    const float* oe = loc.oe;
+    const float* lz = loc.lz;
     combine_heads<G, D, SH>(recs, nsd, rec, 0, s_ml, s_ml + G);
     if constexpr (PRIOR) combine_heads<G, D, SH>(recs, nsd, rec, G * (2 + D), s_ml + 2 * G, s_ml + 3 * G);
     __syncthreads();
@@ -121,7 +148,7 @@ __device__ void decode_epilogue(const float* recs, int nsd, int rec, const T* qg
             //   tail D_T = Z (1 - l0 2^(m0 - log2 A)) clamped at 0,
             //   tail N_T = Z (O_Est - acc0 2^(m0 - log2 A))
             const float lz2 = lz[k] * kLog2e;
-            const float zl = lz2 + s_hs[h];
+            const float zl = lz2 + hsv[h];
             const float M0 = s_ml[2 * G + h], L0 = s_ml[3 * G + h];
             const float rI = (M0 == -INFINITY) ? 0.f : ex2(M0 - lz2);
             const float Mx = fmaxf(M, zl);
@@ -366,13 +393,6 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
         tc::cp_commit();
     };
 
-    // first two tiles in flight before the query / prior fragments are loaded
-    static_assert(kStages == 3, "the loop below keeps two tiles in flight");
-    put_pos(tile0);
-    put_pos(tile0 + 1);
-    __syncthreads();
-    copy_tile(tile0);
-    copy_tile(tile0 + 1);
     // G <= 4: tokens on the MMA rows (no row spent on absent heads); G = 8:
     // heads on the rows
     constexpr bool kTokRows = (G <= 4);
@@ -384,6 +404,20 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
         const int gh = min(lane >> 2, G - 1);
         wa.init(qg + (size_t)gh * D, PRIOR ? st.mu_q + (qh0 + gh) * D : nullptr);
     }
+    // RESA: the epilogue's statistics, loaded now so that their latency hides
+    // behind the tiles
+    __shared__ float s_bias[8];
+    EpiPre<D, G> pre;
+    if constexpr (PRIOR) {
+        if (nt > 0) epi_preload<__nv_bfloat16, D, G>(pre, s_bias, qg, st, u, b, g, Hq, scale);
+    }
+    // first two tiles in flight
+    static_assert(kStages == 3, "the loop below keeps two tiles in flight");
+    put_pos(tile0);
+    put_pos(tile0 + 1);
+    __syncthreads();
+    copy_tile(tile0);
+    copy_tile(tile0 + 1);
     float ks[2] = {0.f, 0.f};      // SUMS: this thread's column pair of K (c < D/2) or V (c >= D/2)
     for (int i = tile0; i < tile1; ++i) {
         // stage (i+2)%3 was last read by tile i-1, finished before the
@@ -488,10 +522,11 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
         constexpr int EM = DENSE ? SA_DROP : MODE;
         if (single)
             decode_epilogue<__nv_bfloat16, D, G, EM, true>(recs, 1, rec, qg, st, u, b, g, Hq, nt, scale, lambda,
-                                                           out, s_acc, s_acc0, s_ml, s_t, s_hs);
+                                                           out, s_acc, s_acc0, s_ml, s_t, s_hs, &pre, s_bias);
         else
             decode_epilogue<__nv_bfloat16, D, G, EM, false>(recs, nchunk, rec, qg, st, u, b, g, Hq, nt, scale,
-                                                            lambda, out, s_acc, s_acc0, s_ml, s_t, s_hs);
+                                                            lambda, out, s_acc, s_acc0, s_ml, s_t, s_hs, &pre,
+                                                            s_bias);
     }
     if (!single) reset_counter(cnt + u);
 }

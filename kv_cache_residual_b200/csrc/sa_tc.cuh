@@ -304,19 +304,28 @@ struct WarpAttnT {
                                            const bool (&in_i)[2], float qscale) {
         constexpr int P = Pitch<D>::kBytes;
         const int lane = threadIdx.x & 31, t = lane & 3;
-        float s[NQ][4];
+        // even and odd k-steps accumulate apart (two short MMA chains), summed after
+        float s2[2][NQ][4];
 #pragma unroll
-        for (int nq = 0; nq < NQ; ++nq)
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) s[nq][j] = 0.f;
+            for (int nq = 0; nq < NQ; ++nq)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) s2[c][nq][j] = 0.f;
         const uint32_t ka = k_tile + (r0 + (lane & 7) + ((lane >> 3) & 1) * 8) * P + (lane >> 4) * 16;
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
             uint32_t a[4];
             ldsm4(ka + ks * 32, a);
 #pragma unroll
-            for (int nq = 0; nq < NQ; ++nq) mma_bf16(s[nq], a[0], a[1], a[2], a[3], qb[nq][ks][0], qb[nq][ks][1]);
+            for (int nq = 0; nq < NQ; ++nq)
+                mma_bf16(s2[ks & 1][nq], a[0], a[1], a[2], a[3], qb[nq][ks][0], qb[nq][ks][1]);
         }
+        float s[NQ][4];
+#pragma unroll
+        for (int nq = 0; nq < NQ; ++nq)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) s[nq][j] = s2[0][nq][j] + s2[1][nq][j];
         // logits of the lane's two tokens (j) and two columns (e)
         float p[2][2];
 #pragma unroll
