@@ -14,7 +14,7 @@
 // stream_unit) runs on the same data in the same order.
 //
 // Shared memory: one dynamic area used first by the selection (sketch ring +
-// barriers + upper-bound keys) and then by the stream pass (tile stages, then
+// barriers + score-bound keys) and then by the stream pass (tile stages, then
 // the merge and epilogue scratch), plus small static arrays that carry the
 // selection across (chosen blocks, draws).  The sink and window rows, which do
 // not depend on the selection, are prefetched into L2 with bulk prefetches at
@@ -32,8 +32,8 @@ template <int D>
 using FusedRing = SketchRing<D, kTcWarps, kFusedStages>;
 
 template <int D>
-constexpr size_t fused_select_smem() {   // ring, its barriers (padded to 128 B), upper-bound keys
-    return (size_t)FusedRing<D>::kRingBytes + 128 + (size_t)kSmemKeys * 4;
+constexpr size_t fused_select_smem() {   // ring, its barriers (padded to 128 B), upper- and lower-bound keys
+    return (size_t)FusedRing<D>::kRingBytes + 128 + (size_t)kSmemKeys * 8;
 }
 
 template <int D, int G, int MODE>
@@ -46,7 +46,7 @@ template <int D, int G, int MODE>
 __global__ void __launch_bounds__(kTcThreads, 2)
 k_step_fused(SelectIo sio, StreamIo dio) {
     using Ring = FusedRing<D>;
-    __shared__ unsigned hist[256];
+    __shared__ __align__(16) unsigned hist[256];
     __shared__ int sw[kTcWarps + 1];
     __shared__ int misc[3];
     __shared__ float s_qh[G * D];
@@ -58,6 +58,7 @@ k_step_fused(SelectIo sio, StreamIo dio) {
     unsigned char* smem = fsmem;
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Ring::kRingBytes);
     uint32_t* ukeys = reinterpret_cast<uint32_t*>(smem + Ring::kRingBytes + 128);
+    uint32_t* lkeys = ukeys + kSmemKeys;
     const int u = blockIdx.x;
 
     // the rows every step reads whatever the selection: sink and window
@@ -89,8 +90,7 @@ k_step_fused(SelectIo sio, StreamIo dio) {
         }
     }
 
-    const SelectSmem sm{hist, sw, misc, s_qh, s_qi, s_qc, ukeys, nullptr, s_sorted, smem, bar, s_samp,
-                        kSampCache};
+    const SelectSmem sm{hist, sw, misc, s_qh, s_qi, s_qc, ukeys, lkeys, s_sorted, smem, bar, s_samp, kSampCache};
     const SelectOutcome r = select_unit<__nv_bfloat16, D, G, kTcThreads, kFusedStages>(sio, sm, u, 0);
     if (!r.done) return;                 // an abandoned wait: the unit's selection is marked invalid
     if (threadIdx.x == 0)

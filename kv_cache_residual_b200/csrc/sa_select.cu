@@ -10,7 +10,7 @@ template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads, 2)
 k_select(SelectIo io) {
     using Ring = SketchRing<D, kWarps, kSelStages>;
-    __shared__ unsigned hist[256];
+    __shared__ __align__(16) unsigned hist[256];
     __shared__ int sw[kWarps + 1];
     __shared__ int misc[3];
     __shared__ float s_qh[G * D];

@@ -263,33 +263,56 @@ __device__ void warp_topk(const uint32_t* keys, int n, int kk, unsigned long lon
     __syncthreads();
 }
 
-// Merges the warps' lists s_cand[w kk .. w kk + kk) (each sorted descending,
-// 0 = empty) into the CTA's best kk in rank order in s_list: an entry's rank is
-// its position in its own list plus the count of larger entries in the others
-// (the words are distinct, so the ranks of the best kk are exactly 0..kk-1).
-template <int NW>
-__device__ void merge_warp_lists(const unsigned long long* s_cand, int kk, unsigned long long* s_list) {
+// Top kk (kk <= 32, kk < n) of the n keys lk[] in shared memory by (key desc,
+// index asc), in rank order into s_list.  Thread t takes the maximum of its
+// contiguous chunk; in each warp the kk-th largest of its 32 chunk maxima B_w
+// has at least kk keys at or above it, and so does B = max_w B_w, so the top
+// kk are among the keys >= B, which are usually few: they are compacted into
+// s_c (up to kCandCap) and ranked exactly.  Returns false, writing nothing,
+// when more than kCandCap keys reach B.  *s_n and *s_b must be zero on entry
+// and visible to every thread (a barrier after they were set).
+constexpr int kCandCap = 256;
+template <int NT>
+__device__ bool topk_group(const uint32_t* lk, int n, int kk, unsigned long long* s_list,
+                           unsigned long long* s_c, int* s_n, unsigned* s_b) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int C = (n + NT - 1) / NT;
+    const int i0 = min(n, (int)threadIdx.x * C), i1 = min(n, i0 + C);
+    uint32_t gm = 0u;
+    for (int i = i0; i < i1; ++i) gm = max(gm, lk[i]);
+    // the kk-th largest lane value: the largest x with #(gm >= x) >= kk, bit by bit
+    uint32_t bw = 0u;
+#pragma unroll 8
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = bw | (1u << bit);
+        if (__popc(__ballot_sync(0xffffffffu, gm >= cand)) >= kk) bw = cand;
+    }
+    if (lane == 0) atomicMax(s_b, bw);
     __syncthreads();
-    const int t = threadIdx.x;
-    if (t < NW * kk) {
-        const unsigned long long c = s_cand[t];
-        if (c != 0ull) {
-            const int w = t / kk;
-            int rank = t - w * kk;
-            for (int v = 0; v < NW; ++v) {
-                if (v == w) continue;
-                const unsigned long long* l = s_cand + v * kk;
-                int lo = 0, hi = kk;                 // first entry of list v below c
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if (l[mid] > c) lo = mid + 1; else hi = mid;
-                }
-                rank += lo;
-            }
-            if (rank < kk) s_list[rank] = c;
+    const uint32_t bnd = *s_b;
+    for (int b0 = warp * 32; b0 < n; b0 += NT) {
+        const int i = b0 + lane;
+        const bool in = i < n && lk[i] >= bnd;
+        const unsigned m = __ballot_sync(0xffffffffu, in);
+        if (m != 0u) {
+            int base = 0;
+            if (lane == 0) base = atomicAdd(s_n, __popc(m));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            const int pos = base + __popc(m & ((1u << lane) - 1u));
+            if (in && pos < kCandCap) s_c[pos] = comp_key(lk[i], i);
         }
     }
     __syncthreads();
+    const int nc = *s_n;
+    if (nc > kCandCap) return false;                 // (uniform: every thread read the same count)
+    for (int j = threadIdx.x; j < nc; j += NT) {
+        const unsigned long long c = s_c[j];
+        int r = 0;
+        for (int q = 0; q < nc; ++q) r += s_c[q] > c ? 1 : 0;
+        if (r < kk) s_list[r] = c;
+    }
+    __syncthreads();
+    return true;
 }
 
 // Ascending sort of one int per lane across the warp (bitonic network).
@@ -413,9 +436,9 @@ struct SelectIo {
 };
 
 // Shared memory the selection works in (the caller lays it out):
-//   hist [256], sw [NT/32 + 1], misc [3], qh [G*D] f32, qi [2*D] (16-byte
-//   aligned), qc [3], ukeys [kSmemKeys], lkeys [kSmemKeys] or null (needed
-//   only when k > 32 or the unit is split), sorted [kWarpTopK], ring
+//   hist [256] (16-byte aligned), sw [NT/32 + 1], misc [3], qh [G*D] f32, qi
+//   [2*D] (16-byte aligned), qc [3], ukeys [kSmemKeys], lkeys [kSmemKeys],
+//   sorted [kWarpTopK], ring
 //   (SketchRing::kRingBytes, 128-byte aligned, reused for the top-k and band
 //   arrays after the scan), bar [kStages] mbarriers, samp [samp_cap] or null
 //   (a shared copy of the draws).
@@ -476,12 +499,13 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
     int8_t* s_qi = sm.qi;
     float* s_qc = sm.qc;
     uint32_t* s_ukeys = sm.ukeys;
-    uint32_t* s_lkeys = sm.lkeys;                      // may be null: only the radix path ranks from it
+    uint32_t* s_lkeys = sm.lkeys;
     int* s_sorted = sm.sorted;
     unsigned char* s_ring = sm.ring;
     uint64_t* s_bar = sm.bar;
-    unsigned long long* s_cand = reinterpret_cast<unsigned long long*>(s_ring);          // NW * kWarpTopK
-    unsigned long long* s_list = s_cand + NW * kWarpTopK;                               // kWarpTopK
+    constexpr int kCandWords = NW * kWarpTopK > kCandCap ? NW * kWarpTopK : kCandCap;
+    unsigned long long* s_cand = reinterpret_cast<unsigned long long*>(s_ring);          // kCandWords
+    unsigned long long* s_list = s_cand + kCandWords;                                    // kWarpTopK
     double* s_bx = reinterpret_cast<double*>(s_list + kWarpTopK);                        // kBandCap
     int* s_bidx = reinterpret_cast<int*>(s_bx + kBandCap);                               // kBandCap
     unsigned char* s_bsel = reinterpret_cast<unsigned char*>(s_bidx + kBandCap);         // kBandCap
@@ -496,8 +520,6 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
     float* sc_up = io.sc_up_all + (size_t)u * (n > 0 ? n : 1);
     // one CTA per unit: the keys never leave shared memory
     const bool local = (nss == 1) && n <= kSmemKeys;
-    // k <= 32 with one CTA per unit: each warp keeps its best k while scanning
-    const bool run_topk = local && kk > 0 && kk < n && kk <= kWarpTopK;
     SelectOutcome res{false, false, 0};
 
     // ---- scan: score intervals of this CTA's slice ------------------------------
@@ -611,10 +633,6 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
         const float sf = s_qc[0], qn = s_qc[1], rq = s_qc[2];
         // this warp's rows of a stage: warp * R * GPW + jj * GPW + gsub, jj < R
         const int wrow = warp * R * GPW + gsub;
-        // running best kk of the rows this warp scored, by lower bound: lane
-        // i < kk holds the i-th best (key, ~index) word, 0 when empty; thr =
-        // the kk-th
-        unsigned long long best = 0ull, thr = 0ull;
         int j = 0;
         for (; j < nst; ++j) {
             const bool ok = mbar_wait(bar0 + 8 * (j % Ring::kStages), (uint32_t)(j / Ring::kStages) & 1u);
@@ -668,29 +686,11 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
                 ukey = fkey(up);
                 if (local) {
                     s_ukeys[r] = ukey;
-                    if (s_lkeys != nullptr) s_lkeys[r] = lkey;
+                    s_lkeys[r] = lkey;
                 } else {
                     sc_lo[r] = lo;
                     sc_up[r] = up;
                 }
-            }
-            // compiler barrier: without it the shared-memory traffic around the
-            // list update is scheduled so badly that the scan runs ~2.5x slower
-            // (measured); it emits no instruction
-            asm volatile("" ::: "memory");
-            if (run_topk) {
-                // rows whose lower bound beats the warp's current kk-th enter its list
-                const unsigned long long c = owner ? comp_key(lkey, r) : 0ull;
-                unsigned m = __ballot_sync(0xffffffffu, c > thr);
-                while (m) {
-                    const int src = __ffs(m) - 1;
-                    m &= m - 1;
-                    const unsigned long long cv = shfl_u64(c, src);
-                    const int pos = __popc(__ballot_sync(0xffffffffu, lane < kk && best > cv));
-                    const unsigned long long up = shfl_up_u64(best, 1);
-                    if (lane < kk && lane >= pos) best = (lane == pos) ? cv : up;
-                }
-                thr = shfl_u64(best, kk - 1);
             }
             // the stage is free once every warp has scored it
             if (__syncthreads_or(!ok)) { failed = true; break; }
@@ -707,9 +707,6 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
                 for (int jj = j; jj < min(nst, j + Ring::kStages); ++jj)
                     mbar_wait(bar0 + 8 * (jj % Ring::kStages), (uint32_t)(jj / Ring::kStages) & 1u, kDrainNs);
             }
-        } else if (run_topk) {
-            // every thread is past the last stage's barrier: the ring is free
-            if (lane < kk) s_cand[warp * kk + lane] = best;
         }
     }
     if (failed) {
@@ -724,6 +721,11 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
         return res;
     }
 
+    // counters of the group top-k (zero before the barrier that ends the gather)
+    if (threadIdx.x == 0) {
+        s_digit = 0;
+        s_rem = 0;
+    }
     // ---- gather the unit's keys --------------------------------------------------
     uint32_t* lk = s_lkeys;            // lower-bound keys: the ranking
     uint32_t* uk = s_ukeys;            // upper-bound keys: band membership
@@ -768,11 +770,9 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
         const bool fast = kk <= kWarpTopK && n <= kSmemKeys;
         uint32_t thr;
         int need = 0;
-        if (run_topk) {
-            merge_warp_lists<NW>(s_cand, kk, s_list);
-            thr = (uint32_t)(s_list[kk - 1] >> 32);
-        } else if (fast) {
-            warp_topk<NT>(lk, n, kk, s_cand, s_list);
+        if (fast) {
+            if (!topk_group<NT>(lk, n, kk, s_list, s_cand, &s_digit, reinterpret_cast<unsigned*>(&s_rem)))
+                warp_topk<NT>(lk, n, kk, s_cand, s_list);
             thr = (uint32_t)(s_list[kk - 1] >> 32);
         } else {
             radix_select<NT, uint32_t>(k32, n, kk, &thr, &need, hist, &s_digit, &s_rem);
