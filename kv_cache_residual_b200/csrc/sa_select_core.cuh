@@ -370,44 +370,52 @@ __device__ __forceinline__ void exact_scores(const T* const (&rows)[M], const bo
     for (int m = 0; m < M; ++m)
 #pragma unroll
         for (int i = 0; i < D / 32; ++i) k[m][i] = live[m] ? to_f32<T>(rows[m][lane + 32 * i]) : 0.f;
+    // the M members' chains advance together (independent, so they overlap)
+    double s[M], c[M];
 #pragma unroll
-    for (int m = 0; m < M; ++m) {
-        double s = 0.0, c = 0.0;
+    for (int m = 0; m < M; ++m) { s[m] = 0.0; c[m] = 0.0; }
 #pragma unroll
-        for (int i = 0; i < D / 32; ++i) {
-            const double kv = (double)k[m][i];
+    for (int i = 0; i < D / 32; ++i)
 #pragma unroll
-            for (int h = 0; h < G; ++h) two_sum_acc(s, c, __dmul_rn((double)s_qh[h * D + lane + 32 * i], kv));
+        for (int h = 0; h < G; ++h) {
+            const double qv = (double)s_qh[h * D + lane + 32 * i];
+#pragma unroll
+            for (int m = 0; m < M; ++m) two_sum_acc(s[m], c[m], __dmul_rn(qv, (double)k[m][i]));
         }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const double so = __shfl_xor_sync(0xffffffffu, s, off);
-            const double co = __shfl_xor_sync(0xffffffffu, c, off);
-            two_sum_acc(s, c, so);
-            c = __dadd_rn(c, co);
+    for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            const double so = __shfl_xor_sync(0xffffffffu, s[m], off);
+            const double co = __shfl_xor_sync(0xffffffffu, c[m], off);
+            two_sum_acc(s[m], c[m], so);
+            c[m] = __dadd_rn(c[m], co);
         }
-        x[m] = __dadd_rn(s, c) + 0.0;          // -0 -> +0
-    }
+#pragma unroll
+    for (int m = 0; m < M; ++m) x[m] = __dadd_rn(s[m], c[m]) + 0.0;      // -0 -> +0
 }
 
-// exact scores of the band members s_bidx[0..nb) into s_bx (a warp per
-// member, four members' rows in flight per warp)
+// exact scores of the band members s_bidx[0..nb) into s_bx (two members
+// per warp, their rows in flight together)
 template <typename T, int D, int G, int NW>
 __device__ void rescore_members(const T* bm, const int* s_bidx, int nb, const float* s_qh, double* s_bx) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int j0 = warp * 4; j0 < nb; j0 += NW * 4) {
-        const T* rows[4];
-        bool live[4];
+    // member warp + m * NW, m < 2: a band of up to 2 NW is one round
+    for (int jb = 0; jb < nb; jb += 2 * NW) {
+        const T* rows[2];
+        bool live[2];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            live[m] = j0 + m < nb;
-            rows[m] = bm + (size_t)(live[m] ? s_bidx[j0 + m] : 0) * D;
+        for (int m = 0; m < 2; ++m) {
+            const int j = jb + warp + m * NW;
+            live[m] = j < nb;
+            rows[m] = bm + (size_t)(live[m] ? s_bidx[j] : 0) * D;
         }
-        double x[4];
-        exact_scores<T, D, G, 4>(rows, live, s_qh, x);
+        if (!live[0]) continue;                       // warp-uniform
+        double x[2];
+        exact_scores<T, D, G, 2>(rows, live, s_qh, x);
 #pragma unroll
-        for (int m = 0; m < 4; ++m)
-            if (lane == 0 && live[m]) s_bx[j0 + m] = x[m];
+        for (int m = 0; m < 2; ++m)
+            if (lane == 0 && live[m]) s_bx[jb + warp + m * NW] = x[m];
     }
 }
 
