@@ -265,8 +265,9 @@ __device__ void warp_topk(const uint32_t* keys, int n, int kk, unsigned long lon
 
 // Top kk (kk <= 32, kk < n) of the n keys lk[] in shared memory by (key desc,
 // index asc), in rank order into s_list.  Thread t takes the maximum of its
-// contiguous chunk; in each warp the kk-th largest of its 32 chunk maxima B_w
-// has at least kk keys at or above it, and so does B = max_w B_w, so the top
+// contiguous chunk; in each warp a lower bound B_w on the kk-th largest of its
+// 32 chunk maxima has at least kk keys at or above it, and so does
+// B = max_w B_w, so the top
 // kk are among the keys >= B, which are usually few: they are compacted into
 // s_c (up to kCandCap) and ranked exactly.  Returns false, writing nothing,
 // when more than kCandCap keys reach B.  *s_n and *s_b must be zero on entry
@@ -280,10 +281,12 @@ __device__ bool topk_group(const uint32_t* lk, int n, int kk, unsigned long long
     const int i0 = min(n, (int)threadIdx.x * C), i1 = min(n, i0 + C);
     uint32_t gm = 0u;
     for (int i = i0; i < i1; ++i) gm = max(gm, lk[i]);
-    // the kk-th largest lane value: the largest x with #(gm >= x) >= kk, bit by bit
+    // a lower bound on the kk-th largest lane value: the largest x with
+    // #(gm >= x) >= kk, bit by bit over the top 16 bits (the low bits left at
+    // zero only loosen the bound)
     uint32_t bw = 0u;
 #pragma unroll 8
-    for (int bit = 31; bit >= 0; --bit) {
+    for (int bit = 31; bit >= 16; --bit) {
         const uint32_t cand = bw | (1u << bit);
         if (__popc(__ballot_sync(0xffffffffu, gm >= cand)) >= kk) bw = cand;
     }
