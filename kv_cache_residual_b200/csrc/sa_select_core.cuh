@@ -263,27 +263,28 @@ __device__ void warp_topk(const uint32_t* keys, int n, int kk, unsigned long lon
     __syncthreads();
 }
 
-// Top kk (kk <= 32, kk < n) of the n keys lk[] in shared memory by (key desc,
-// index asc), in rank order into s_list.  Thread t takes the maximum of its
-// contiguous chunk; in each warp a lower bound B_w on the kk-th largest of its
-// 32 chunk maxima has at least kk keys at or above it, and so does
-// B = max_w B_w, so the top
-// kk are among the keys >= B, which are usually few: they are compacted into
-// s_c (up to kCandCap) and ranked exactly.  Returns false, writing nothing,
-// when more than kCandCap keys reach B.  *s_n and *s_b must be zero on entry
-// and visible to every thread (a barrier after they were set).
 constexpr int kCandCap = 256;
+
+// Top kk (kk <= 32, kk < n) of the n lower-bound keys lk[] in shared memory by
+// (key desc, index asc), in rank order into s_list, and the band {upper >=
+// thr} (thr = the kk-th lower key) into s_bidx / *s_band.  Thread t takes the
+// maximum of its contiguous chunk; in each warp a lower bound B_w on the kk-th
+// largest of its 32 chunk maxima has at least kk keys at or above it, and so
+// does B = max_w B_w, so thr >= B.  The candidates are the keys whose upper
+// bound reaches B: they contain the top kk by lower bound and the whole band,
+// and are usually few; they are compacted into s_c / s_u (up to kCandCap),
+// ranked exactly, and the band is read off them.  Returns false, having
+// written nothing, when more than kCandCap keys reach B.  *s_n and *s_b must
+// be zero on entry and visible to every thread (a barrier after they were set).
 template <int NT>
-__device__ bool topk_group(const uint32_t* lk, int n, int kk, unsigned long long* s_list,
-                           unsigned long long* s_c, int* s_n, unsigned* s_b) {
+__device__ bool topk_band(const uint32_t* lk, const uint32_t* uk, int n, int kk, unsigned long long* s_list,
+                          unsigned long long* s_c, uint32_t* s_u, int* s_n, unsigned* s_b, int* s_bidx,
+                          int* s_band) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int C = (n + NT - 1) / NT;
     const int i0 = min(n, (int)threadIdx.x * C), i1 = min(n, i0 + C);
     uint32_t gm = 0u;
     for (int i = i0; i < i1; ++i) gm = max(gm, lk[i]);
-    // a lower bound on the kk-th largest lane value: the largest x with
-    // #(gm >= x) >= kk, bit by bit over the top 16 bits (the low bits left at
-    // zero only loosen the bound)
     uint32_t bw = 0u;
 #pragma unroll 8
     for (int bit = 31; bit >= 16; --bit) {
@@ -295,14 +296,17 @@ __device__ bool topk_group(const uint32_t* lk, int n, int kk, unsigned long long
     const uint32_t bnd = *s_b;
     for (int b0 = warp * 32; b0 < n; b0 += NT) {
         const int i = b0 + lane;
-        const bool in = i < n && lk[i] >= bnd;
+        const bool in = i < n && uk[i] >= bnd;
         const unsigned m = __ballot_sync(0xffffffffu, in);
         if (m != 0u) {
             int base = 0;
             if (lane == 0) base = atomicAdd(s_n, __popc(m));
             base = __shfl_sync(0xffffffffu, base, 0);
             const int pos = base + __popc(m & ((1u << lane) - 1u));
-            if (in && pos < kCandCap) s_c[pos] = comp_key(lk[i], i);
+            if (in && pos < kCandCap) {
+                s_c[pos] = comp_key(lk[i], i);
+                s_u[pos] = uk[i];
+            }
         }
     }
     __syncthreads();
@@ -313,6 +317,19 @@ __device__ bool topk_group(const uint32_t* lk, int n, int kk, unsigned long long
         int r = 0;
         for (int q = 0; q < nc; ++q) r += s_c[q] > c ? 1 : 0;
         if (r < kk) s_list[r] = c;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t thr = (uint32_t)(s_list[kk - 1] >> 32);
+        int base = 0;
+        for (int j0 = 0; j0 < nc; j0 += 32) {
+            const int j = j0 + lane;
+            const bool in = j < nc && s_u[j] >= thr;
+            const unsigned m = __ballot_sync(0xffffffffu, in);
+            if (in) s_bidx[base + __popc(m & ((1u << lane) - 1u))] = comp_index(s_c[j]);
+            base += __popc(m);
+        }
+        if (lane == 0) *s_band = base;
     }
     __syncthreads();
     return true;
@@ -520,6 +537,7 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
     double* s_bx = reinterpret_cast<double*>(s_list + kWarpTopK);                        // kBandCap
     int* s_bidx = reinterpret_cast<int*>(s_bx + kBandCap);                               // kBandCap
     unsigned char* s_bsel = reinterpret_cast<unsigned char*>(s_bidx + kBandCap);         // kBandCap
+    uint32_t* s_u = reinterpret_cast<uint32_t*>(s_bsel + kBandCap);                      // kCandCap
 
     const int b = u / Hkv, g = u - b * Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -781,9 +799,11 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
         const bool fast = kk <= kWarpTopK && n <= kSmemKeys;
         uint32_t thr;
         int need = 0;
+        bool listed = false;            // band already listed (group path)
         if (fast) {
-            if (!topk_group<NT>(lk, n, kk, s_list, s_cand, &s_digit, reinterpret_cast<unsigned*>(&s_rem)))
-                warp_topk<NT>(lk, n, kk, s_cand, s_list);
+            listed = topk_band<NT>(lk, uk, n, kk, s_list, s_cand, s_u, &s_digit, reinterpret_cast<unsigned*>(&s_rem),
+                                   s_bidx, &s_nb);
+            if (!listed) warp_topk<NT>(lk, n, kk, s_cand, s_list);
             thr = (uint32_t)(s_list[kk - 1] >> 32);
         } else {
             radix_select<NT, uint32_t>(k32, n, kk, &thr, &need, hist, &s_digit, &s_rem);
@@ -791,19 +811,21 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
         // thr = the kk-th largest lower bound.  A candidate whose upper bound is
         // below it is beaten strictly by kk others, so the exact top kk lies
         // in the band {upper >= thr}, which contains the kk best lower bounds.
-        // One pass counts the band and lists its members (the first kBandCap
-        // of them, in no particular order) in s_bidx.
-        for (int i0 = warp * 32; i0 < n; i0 += NT) {
-            const int i = i0 + lane;
-            const bool in = i < n && uk[i] >= thr;
-            const unsigned m = __ballot_sync(0xffffffffu, in);
-            if (m != 0u) {
-                int base = 0;
-                if (lane == 0) base = atomicAdd(&s_nb, __popc(m));
-                base = __shfl_sync(0xffffffffu, base, 0);
-                if (in) {
-                    const int pos = base + __popc(m & ((1u << lane) - 1u));
-                    if (pos < kBandCap) s_bidx[pos] = i;
+        // Unless listed already, one pass counts the band and lists its
+        // members (the first kBandCap of them, in no particular order) in s_bidx.
+        if (!listed) {
+            for (int i0 = warp * 32; i0 < n; i0 += NT) {
+                const int i = i0 + lane;
+                const bool in = i < n && uk[i] >= thr;
+                const unsigned m = __ballot_sync(0xffffffffu, in);
+                if (m != 0u) {
+                    int base = 0;
+                    if (lane == 0) base = atomicAdd(&s_nb, __popc(m));
+                    base = __shfl_sync(0xffffffffu, base, 0);
+                    if (in) {
+                        const int pos = base + __popc(m & ((1u << lane) - 1u));
+                        if (pos < kBandCap) s_bidx[pos] = i;
+                    }
                 }
             }
         }
