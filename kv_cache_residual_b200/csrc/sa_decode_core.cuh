@@ -48,12 +48,9 @@ struct EpiPre {
     float oe[kPer], lz[kPer];
 };
 
-// Fills pre (every thread) and hs[G] (one warp per head); the caller puts a
-// barrier between this and the epilogue.
-template <typename T, int D, int G>
-__device__ __forceinline__ void epi_preload(EpiPre<D, G>& pre, float* hs, const T* qg, const sa_stats& st, int u,
-                                            int b, int g, int Hq, float scale) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+// Loads pre (every thread): O_Est and ln Z0 of this thread's outputs.
+template <int D, int G>
+__device__ __forceinline__ void epi_load(EpiPre<D, G>& pre, const sa_stats& st, int b, int g, int Hq) {
 #pragma unroll
     for (int k = 0; k < EpiPre<D, G>::kPer; ++k) {
         const int idx = threadIdx.x + k * blockDim.x;
@@ -61,6 +58,60 @@ __device__ __forceinline__ void epi_preload(EpiPre<D, G>& pre, float* hs, const 
         pre.oe[k] = idx < G * D ? st.o_est[qh * D + idx % D] : 0.f;
         pre.lz[k] = idx < G * D ? st.log_z0[qh] : 0.f;
     }
+}
+
+// The operands of the per-head bias c_h of a CTA of NW warps (warp w takes
+// heads w, w + NW, ...), loaded into registers by bias_load early and summed
+// by bias_sum late, so that their latency hides behind other work.
+template <int D, int G, int NW>
+struct BiasPre {
+    static constexpr int kHpw = (G + NW - 1) / NW;      // heads per warp
+    static constexpr int kPl = D / 32;                  // elements per lane
+    float q[kHpw][kPl], mq[kHpw][kPl], mk[kPl];
+};
+
+template <typename T, int D, int G, int NW>
+__device__ __forceinline__ void bias_load(BiasPre<D, G, NW>& bp, const T* qg, const sa_stats& st, int u, int b,
+                                          int g, int Hq) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int j = 0; j < BiasPre<D, G, NW>::kPl; ++j) bp.mk[j] = st.mu_k[(size_t)u * D + lane + 32 * j];
+#pragma unroll
+    for (int x = 0; x < BiasPre<D, G, NW>::kHpw; ++x) {
+        const int h = warp + x * NW;
+        const size_t qh = (size_t)b * Hq + g * G + (h < G ? h : 0);
+#pragma unroll
+        for (int j = 0; j < BiasPre<D, G, NW>::kPl; ++j) {
+            bp.q[x][j] = h < G ? to_f32<T>(qg[(size_t)h * D + lane + 32 * j]) : 0.f;
+            bp.mq[x][j] = h < G ? st.mu_q[qh * D + lane + 32 * j] : 0.f;
+        }
+    }
+}
+
+// hs[h] = s (q_h - mu_Q,h) . mu_K in log2 units; a barrier must follow
+// before hs is read.
+template <int D, int G, int NW>
+__device__ __forceinline__ void bias_sum(const BiasPre<D, G, NW>& bp, float* hs, float scale) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int x = 0; x < BiasPre<D, G, NW>::kHpw; ++x) {
+        const int h = warp + x * NW;
+        if (h >= G) break;
+        float y = 0.f;
+#pragma unroll
+        for (int j = 0; j < BiasPre<D, G, NW>::kPl; ++j) y = fmaf(bp.q[x][j] - bp.mq[x][j], bp.mk[j], y);
+        y = group_sum<32>(y);
+        if (lane == 0) hs[h] = y * scale * kLog2e;
+    }
+}
+
+// Fills pre (every thread) and hs[G] (one warp per head); the caller puts a
+// barrier between this and the epilogue.
+template <typename T, int D, int G>
+__device__ __forceinline__ void epi_preload(EpiPre<D, G>& pre, float* hs, const T* qg, const sa_stats& st, int u,
+                                            int b, int g, int Hq, float scale) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    epi_load<D, G>(pre, st, b, g, Hq);
     for (int h = warp; h < G; h += nwarps) {
         const size_t qh = (size_t)b * Hq + g * G + h;
         float x = 0.f;
@@ -69,6 +120,36 @@ __device__ __forceinline__ void epi_preload(EpiPre<D, G>& pre, float* hs, const 
             x = fmaf(to_f32<T>(qg[(size_t)h * D + e]) - st.mu_q[qh * D + e], st.mu_k[(size_t)u * D + e], x);
         x = group_sum<32>(x);
         if (lane == 0) hs[h] = x * scale * kLog2e;
+    }
+}
+
+// One output element of head h from the unit's combined exact state over the
+// read set (max M, mass Ls, accumulator A, log2 units) and the mode's
+// residual.  RESA (Online Aggregator, with all masses relative to one max):
+// Z (log2) = log2 A_h + c_h with log2 A_h = lz2 and c_h = hs; prior mass at
+// I = L0 2^(M0 + c); tail D_T = Z (1 - L0 2^(M0 - log2 A)) clamped at 0,
+// tail N_T = Z (O_Est - A0 2^(M0 - log2 A)), scaled by lambda.  PROXY: one
+// token of logit z (log2) and value tv.  DROP / SAMPLE (the draws are already
+// in the state), or no tail: the normalised state.
+template <int MODE>
+__device__ __forceinline__ float resid_value(int nt, float M, float Ls, float A, float M0, float L0, float A0,
+                                             float lz2, float hs, float oe, float lambda, float z, float tv) {
+    if (nt == 0 || MODE == SA_DROP || MODE == SA_SAMPLE) {
+        return Ls > 0.f ? A / Ls : 0.f;           // an empty set carries no mass
+    } else if constexpr (MODE == SA_RESA) {
+        const float zl = lz2 + hs;
+        const float rI = (M0 == -INFINITY) ? 0.f : ex2(M0 - lz2);
+        const float Mx = fmaxf(M, zl);
+        const float wI = (M == -INFINITY) ? 0.f : ex2(M - Mx);
+        const float wT = lambda * ex2(zl - Mx);
+        const float num = A * wI + wT * (oe - A0 * rI);
+        const float den = Ls * wI + wT * fmaxf(0.f, 1.f - L0 * rI);
+        return den > 0.f ? num / den : 0.f;
+    } else {
+        const float Mx = fmaxf(M, z);
+        const float wI = (M == -INFINITY) ? 0.f : ex2(M - Mx);
+        const float wP = ex2(z - Mx);
+        return (A * wI + wP * tv) / (Ls * wI + wP);
     }
 }
 
@@ -140,30 +221,14 @@ __device__ __forceinline__ void decode_epilogue(const float* recs, int nsd, int 
         const size_t qh = (size_t)b * Hq + g * G + h;
         const float M = s_ml[h], Ls = s_ml[G + h], A = s_acc[idx];
         float o;
-        if (nt == 0 || MODE == SA_DROP || MODE == SA_SAMPLE) {
-            o = Ls > 0.f ? A / Ls : 0.f;          // an empty set carries no mass
-        } else if constexpr (PRIOR) {
-            // RESA Online Aggregator with all masses relative to one max:
-            //   Z (log2) = log2 A_h + c_h; prior mass at I = l0 2^(m0 + c);
-            //   tail D_T = Z (1 - l0 2^(m0 - log2 A)) clamped at 0,
-            //   tail N_T = Z (O_Est - acc0 2^(m0 - log2 A))
-            const float lz2 = lz[k] * kLog2e;
-            const float zl = lz2 + hsv[h];
-            const float M0 = s_ml[2 * G + h], L0 = s_ml[3 * G + h];
-            const float rI = (M0 == -INFINITY) ? 0.f : ex2(M0 - lz2);
-            const float Mx = fmaxf(M, zl);
-            const float wI = (M == -INFINITY) ? 0.f : ex2(M - Mx);
-            const float wT = lambda * ex2(zl - Mx);
-            const float num = A * wI + wT * (oe[k] - s_acc0[idx] * rI);
-            const float den = Ls * wI + wT * fmaxf(0.f, 1.f - L0 * rI);
-            o = den > 0.f ? num / den : 0.f;
-        } else {
-            const float z = s_hs[h];
-            const float Mx = fmaxf(M, z);
-            const float wI = (M == -INFINITY) ? 0.f : ex2(M - Mx);
-            const float wP = ex2(z - Mx);
-            o = (A * wI + wP * s_t[D + e]) / (Ls * wI + wP);
-        }
+        if constexpr (PRIOR)
+            o = resid_value<MODE>(nt, M, Ls, A, s_ml[2 * G + h], s_ml[3 * G + h], s_acc0[idx], lz[k] * kLog2e,
+                                  nt > 0 ? hsv[h] : 0.f, oe[k], lambda, 0.f, 0.f);
+        else if constexpr (SUMS)
+            o = resid_value<MODE>(nt, M, Ls, A, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, lambda, nt > 0 ? s_hs[h] : 0.f,
+                                  nt > 0 ? s_t[D + e] : 0.f);
+        else
+            o = resid_value<MODE>(nt, M, Ls, A, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, lambda, 0.f, 0.f);
         out[qh * D + e] = o;
     }
 }
@@ -393,31 +458,36 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
         tc::cp_commit();
     };
 
+    // The query and (RESA) the epilogue's statistics are loaded into
+    // registers first and used only later, so that their latency hides
+    // behind the first two tiles, which are put in flight next.
     // G <= 4: tokens on the MMA rows (no row spent on absent heads); G = 8:
     // heads on the rows
     constexpr bool kTokRows = (G <= 4);
     using Engine = typename std::conditional<kTokRows, tc::WarpAttnT<D, G, PRIOR>, tc::WarpAttn<D, G, PRIOR>>::type;
     Engine wa;
-    if constexpr (kTokRows) {
-        wa.init(qg, PRIOR ? st.mu_q + qh0 * D : nullptr);
-    } else {
-        const int gh = min(lane >> 2, G - 1);
-        wa.init(qg + (size_t)gh * D, PRIOR ? st.mu_q + (qh0 + gh) * D : nullptr);
-    }
-    // RESA: the epilogue's statistics, loaded now so that their latency hides
-    // behind the tiles
+    if constexpr (kTokRows) wa.load(qg, PRIOR ? st.mu_q + qh0 * D : nullptr);
     __shared__ float s_bias[8];
     EpiPre<D, G> pre;
+    BiasPre<D, G, kTcWarps> bpre;
     if constexpr (PRIOR) {
-        if (nt > 0) epi_preload<__nv_bfloat16, D, G>(pre, s_bias, qg, st, u, b, g, Hq, scale);
+        if (nt > 0) {
+            epi_load<D, G>(pre, st, b, g, Hq);
+            bias_load<__nv_bfloat16, D, G, kTcWarps>(bpre, qg, st, u, b, g, Hq);
+        }
     }
-    // first two tiles in flight
     static_assert(kStages == 3, "the loop below keeps two tiles in flight");
     put_pos(tile0);
     put_pos(tile0 + 1);
     __syncthreads();
     copy_tile(tile0);
     copy_tile(tile0 + 1);
+    if constexpr (kTokRows) {
+        wa.finish();
+    } else {
+        const int gh = min(lane >> 2, G - 1);
+        wa.init(qg + (size_t)gh * D, PRIOR ? st.mu_q + (qh0 + gh) * D : nullptr);
+    }
     float ks[2] = {0.f, 0.f};      // SUMS: this thread's column pair of K (c < D/2) or V (c >= D/2)
     for (int i = tile0; i < tile1; ++i) {
         // stage (i+2)%3 was last read by tile i-1, finished before the
@@ -483,8 +553,50 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
     float* own = acc + (PRIOR ? 2 : 1) * kTcWarps * G * D;   // own record when the unit is one chunk
     float* scratch = own + 2 * G * (2 + D) + 2 * D;
     wa.store(ml, acc, acc0);
+    if constexpr (PRIOR) {
+        if (nt > 0) bias_sum<D, G, kTcWarps>(bpre, s_bias, scale);
+    }
     __syncthreads();
     const bool single = (nchunk == 1);
+    if constexpr (!DENSE && !SUMS) {
+        if (single) {
+            // the unit in one chunk: its output straight from the warps'
+            // states (the merge, in warp order, then the mode's residual)
+#pragma unroll
+            for (int k = 0; k < EpiPre<D, G>::kPer; ++k) {
+                const int idx = threadIdx.x + k * kTcThreads;
+                if (idx >= G * D) break;
+                const int h = idx / D, e = idx - h * D;
+                float st4[2][3];                      // (M, Ls, A) of the exact and prior states
+#pragma unroll
+                for (int pr = 0; pr < (PRIOR ? 2 : 1); ++pr) {
+                    float M = -INFINITY;
+#pragma unroll
+                    for (int w = 0; w < kTcWarps; ++w) M = fmaxf(M, ml[(w * G + h) * 4 + 2 * pr]);
+                    float A = 0.f, Ls = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kTcWarps; ++w) {
+                        const float mw = ml[(w * G + h) * 4 + 2 * pr];
+                        const float f = (mw == -INFINITY) ? 0.f : ex2(mw - M);
+                        A = fmaf((pr ? acc0 : acc)[(w * G + h) * D + e], f, A);
+                        Ls = fmaf(ml[(w * G + h) * 4 + 2 * pr + 1], f, Ls);
+                    }
+                    st4[pr][0] = M;
+                    st4[pr][1] = Ls;
+                    st4[pr][2] = A;
+                }
+                float o;
+                if constexpr (PRIOR)
+                    o = resid_value<MODE>(nt, st4[0][0], st4[0][1], st4[0][2], st4[1][0], st4[1][1], st4[1][2],
+                                          pre.lz[k] * kLog2e, nt > 0 ? s_bias[h] : 0.f, pre.oe[k], lambda, 0.f, 0.f);
+                else
+                    o = resid_value<MODE>(nt, st4[0][0], st4[0][1], st4[0][2], 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, lambda,
+                                          0.f, 0.f);
+                out[(qh0 + h) * D + e] = o;
+            }
+            return;
+        }
+    }
     float* r = single ? own : part + ((size_t)u * nchunk + chunk) * rec;
     tc::merge_warps<D, G, PRIOR>(ml, acc, acc0, kTcWarps, r);
     if constexpr (SUMS) {

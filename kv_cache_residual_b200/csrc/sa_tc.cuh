@@ -264,22 +264,36 @@ struct WarpAttnT {
     // tile row of this lane's token j (0, 1) in the 16-token group at r0
     __device__ static __forceinline__ int row(int r0, int j) { return r0 + ((threadIdx.x & 31) >> 2) + 8 * j; }
 
-    // qg: the G bf16 query rows of the unit; mu: the G fp32 typical queries
-    // (PRIOR only)
-    __device__ __forceinline__ void init(const __nv_bfloat16* qg, const float* mu) {
+    // init in two halves: load issues this lane's operand loads into raw
+    // (qg: the G bf16 query rows of the unit; mu: the G fp32 typical queries,
+    // PRIOR only), finish forms the B fragments and clears the state once
+    // they have landed, so other work can sit between the two.
+    float2 raw[KS][2];
+    __device__ __forceinline__ void load(const __nv_bfloat16* qg, const float* mu) {
         const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 const int dim = ks * 16 + 2 * t + 8 * half;
+                float2 x = make_float2(0.f, 0.f);
+                if (g < G)
+                    x.x = __uint_as_float(*reinterpret_cast<const uint32_t*>(qg + (size_t)g * D + dim));
+                else if (PRIOR && g < 2 * G)
+                    x = *reinterpret_cast<const float2*>(mu + (size_t)(g - G) * D + dim);
+                raw[ks][half] = x;
+            }
+        }
+    }
+    __device__ __forceinline__ void finish() {
+        const int g = (threadIdx.x & 31) >> 2;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
                 uint32_t v0 = 0u, v1 = 0u;
-                if (g < G) {
-                    v0 = *reinterpret_cast<const uint32_t*>(qg + (size_t)g * D + dim);
-                } else if (PRIOR && g < 2 * G) {
-                    const float2 x = *reinterpret_cast<const float2*>(mu + (size_t)(g - G) * D + dim);
-                    split_bf2(x.x, x.y, v0, v1);
-                }
+                if (g < G) v0 = __float_as_uint(raw[ks][half].x);
+                else if (PRIOR && g < 2 * G) split_bf2(raw[ks][half].x, raw[ks][half].y, v0, v1);
                 qb[0][ks][half] = v0;
                 if constexpr (PRIOR) qb[NQ - 1][ks][half] = v1;
             }
@@ -290,6 +304,10 @@ struct WarpAttnT {
             for (int j = 0; j < 4; ++j) o[mt][j] = 0.f;
         m[0] = m[1] = -INFINITY;
         l[0] = l[1] = 0.f;
+    }
+    __device__ __forceinline__ void init(const __nv_bfloat16* qg, const float* mu) {
+        load(qg, mu);
+        finish();
     }
 
     __device__ static __forceinline__ uint32_t trans8(uint32_t x) {
