@@ -267,24 +267,26 @@ constexpr int kCandCap = 256;
 
 // Top kk (kk <= 32, kk < n) of the n lower-bound keys lk[] in shared memory by
 // (key desc, index asc), in rank order into s_list, and the band {upper >=
-// thr} (thr = the kk-th lower key) into s_bidx / *s_band.  Thread t takes the
-// maximum of its contiguous chunk; in each warp a lower bound B_w on the kk-th
-// largest of its 32 chunk maxima has at least kk keys at or above it, and so
-// does B = max_w B_w, so thr >= B.  The candidates are the keys whose upper
-// bound reaches B: they contain the top kk by lower bound and the whole band,
-// and are usually few; they are compacted into s_c / s_u (up to kCandCap),
-// ranked exactly, and the band is read off them.  Returns false, having
-// written nothing, when more than kCandCap keys reach B.  *s_n and *s_b must
-// be zero on entry and visible to every thread (a barrier after they were set).
+// thr} (thr = the kk-th lower key) into s_bidx / *s_band.  Thread t owns the
+// keys t, t + NT, ... (n <= 32 NT) and takes their maximum; in each warp a
+// lower bound B_w on the kk-th largest of its 32 maxima has at least kk keys
+// at or above it, and so does B = max_w B_w, so thr >= B.  The candidates
+// are the keys whose upper bound reaches B: they contain the top kk by lower
+// bound and the whole band, and are usually few; they are compacted (each
+// thread's matches at its place in a block scan) into s_c / s_u (up to
+// kCandCap), ranked exactly, and the band is read off them.  Returns false,
+// having written nothing, when more than kCandCap keys reach B.  *s_b must
+// be zero on entry and visible to every thread; sw holds NT/32 ints.
 template <int NT>
 __device__ bool topk_band(const uint32_t* lk, const uint32_t* uk, int n, int kk, unsigned long long* s_list,
-                          unsigned long long* s_c, uint32_t* s_u, int* s_n, unsigned* s_b, int* s_bidx,
+                          unsigned long long* s_c, uint32_t* s_u, int* sw, unsigned* s_b, int* s_bidx,
                           int* s_band) {
+    constexpr int NW = NT / 32;
+    static_assert(kSmemKeys <= 32 * NT, "one mask bit per owned key");
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int C = (n + NT - 1) / NT;
-    const int i0 = min(n, (int)threadIdx.x * C), i1 = min(n, i0 + C);
     uint32_t gm = 0u;
-    for (int i = i0; i < i1; ++i) gm = max(gm, lk[i]);
+#pragma unroll 4
+    for (int i = threadIdx.x; i < n; i += NT) gm = max(gm, lk[i]);
     uint32_t bw = 0u;
 #pragma unroll 8
     for (int bit = 31; bit >= 16; --bit) {
@@ -294,27 +296,40 @@ __device__ bool topk_band(const uint32_t* lk, const uint32_t* uk, int n, int kk,
     if (lane == 0) atomicMax(s_b, bw);
     __syncthreads();
     const uint32_t bnd = *s_b;
-    for (int b0 = warp * 32; b0 < n; b0 += NT) {
-        const int i = b0 + lane;
-        const bool in = i < n && uk[i] >= bnd;
-        const unsigned m = __ballot_sync(0xffffffffu, in);
-        if (m != 0u) {
-            int base = 0;
-            if (lane == 0) base = atomicAdd(s_n, __popc(m));
-            base = __shfl_sync(0xffffffffu, base, 0);
-            const int pos = base + __popc(m & ((1u << lane) - 1u));
-            if (in && pos < kCandCap) {
-                s_c[pos] = comp_key(lk[i], i);
-                s_u[pos] = uk[i];
-            }
-        }
+    // this thread's keys whose upper bound reaches B, as a bit mask
+    unsigned mine = 0u;
+#pragma unroll 4
+    for (int j = 0; j * NT + (int)threadIdx.x < n; ++j) mine |= (uk[j * NT + threadIdx.x] >= bnd ? 1u : 0u) << j;
+    const int cnt = __popc(mine);
+    int inc = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += x;
+    }
+    if (lane == 31) sw[warp] = inc;
+    __syncthreads();
+    int off = inc - cnt, nc = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+        const int x = sw[w];
+        off += w < warp ? x : 0;
+        nc += x;
+    }
+    if (nc > kCandCap) return false;                 // (uniform: every thread summed the same counts)
+    while (mine != 0u) {
+        const int j = __ffs(mine) - 1;
+        mine &= mine - 1u;
+        const int i = j * NT + threadIdx.x;
+        s_c[off] = comp_key(lk[i], i);
+        s_u[off] = uk[i];
+        ++off;
     }
     __syncthreads();
-    const int nc = *s_n;
-    if (nc > kCandCap) return false;                 // (uniform: every thread read the same count)
     for (int j = threadIdx.x; j < nc; j += NT) {
         const unsigned long long c = s_c[j];
         int r = 0;
+#pragma unroll 4
         for (int q = 0; q < nc; ++q) r += s_c[q] > c ? 1 : 0;
         if (r < kk) s_list[r] = c;
     }
@@ -801,7 +816,7 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
         int need = 0;
         bool listed = false;            // band already listed (group path)
         if (fast) {
-            listed = topk_band<NT>(lk, uk, n, kk, s_list, s_cand, s_u, &s_digit, reinterpret_cast<unsigned*>(&s_rem),
+            listed = topk_band<NT>(lk, uk, n, kk, s_list, s_cand, s_u, sw, reinterpret_cast<unsigned*>(&s_rem),
                                    s_bidx, &s_nb);
             if (!listed) warp_topk<NT>(lk, n, kk, s_cand, s_list);
             thr = (uint32_t)(s_list[kk - 1] >> 32);
