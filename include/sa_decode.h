@@ -41,10 +41,13 @@
  *     atomics; partial results are combined in a fixed order.
  *
  * Layouts (dtype = shape.dtype for the cache and all queries)
- *   k, v        [B, Hkv, L, d]       KV cache
+ *   k, v        [B, Hkv, ld, d]      KV cache; tokens [0, L) are valid
  *   q_ctx       [B, Hq, L, d]        context queries (prefill only)
  *   q           [B, Hq, d]           decode queries of this step
  *   query head h belongs to KV head h / (Hq / Hkv).
+ *   ld (shape.ld, 0 = L) is the cache's capacity in tokens per unit; the
+ *   per-block arrays of sa_stats have ld / 16 rows per unit.  sa_append
+ *   grows L by one token inside that capacity.
  */
 #ifndef SA_DECODE_H
 #define SA_DECODE_H
@@ -83,10 +86,16 @@ typedef enum {
 } sa_op;
 
 /* Supported: d in {64, 128}; Hq % Hkv == 0 with G = Hq/Hkv in {1,2,4,8};
- * L a positive multiple of 16, L < 2^31 / d; B, Hkv >= 1. */
+ * L >= 16 (a multiple of 16 for sa_prefill_stats, whose statistics cover
+ * whole blocks); ld = 0 (meaning ld = L) or a multiple of 16 with
+ * L <= ld < 2^31 / d; B, Hkv >= 1.  A length L that is not a multiple of 16
+ * needs ld given.  Only the complete blocks [0, L/16) are candidates for
+ * selection, and a partial last block lies in the local window when
+ * local >= 16. */
 typedef struct {
     int B, Hq, Hkv, d, L;
     sa_dtype dtype;
+    int ld;
 } sa_shape;
 
 /* Prefill-end statistics, written by sa_prefill_stats, read by sa_select and
@@ -98,12 +107,12 @@ typedef struct {
  *   mu_k        [B, Hkv, d]  f32  typical key: mean of the L cached keys
  *   sum_k       [B, Hkv, d]  f32  sum of the L cached keys
  *   sum_v       [B, Hkv, d]  f32  sum of the L cached values
- *   blk_mean    [B, Hkv, L/16, d] in dtype: 16-token block means, summed in
+ *   blk_mean    [B, Hkv, ld/16, d] in dtype: 16-token block means, summed in
  *               fp64 and rounded once (nearest, ties to even)
  *   kbar_absmax [B, Hkv]     f32  max |blk_mean| (reported; not needed by
  *               sa_select)
- *   blk_code    [B, Hkv, L/16, d] int8 and
- *   blk_meta    [B, Hkv, L/16, 4] f32: the scan sketch of blk_mean relative
+ *   blk_code    [B, Hkv, ld/16, d] int8 and
+ *   blk_meta    [B, Hkv, ld/16, 4] f32: the scan sketch of blk_mean relative
  *               to mu_k, written with it.  Per block row kbar, t = kbar - mu_k
  *               (fp64), s = fl32(max_e |t_e| / 127), code_e = clamp(rint(t_e /
  *               s), -127, 127) (0 when s = 0), meta = {s, rn, kn, 0} with
@@ -190,13 +199,37 @@ SA_API sa_status sa_prefill_stats(const sa_shape* shape, const void* q_ctx, cons
                            void* ws, size_t ws_bytes, void* stream);
 
 /* Block means of blocks [blk_begin, blk_end) of every unit into blk_mean
- * ([B, Hkv, L/16, d], dtype), their sketch relative to mu_k ([B, Hkv, d] f32,
+ * ([B, Hkv, ld/16, d], dtype; blk_end <= L/16), their sketch relative to
+ * mu_k ([B, Hkv, d] f32,
  * read only) into blk_code / blk_meta (layouts of sa_stats), and raises
  * kbar_absmax [B, Hkv] to cover them (for a cache that grew by whole blocks;
  * keep mu_k as it was when the other rows were sketched).  No workspace. */
 SA_API sa_status sa_block_summaries(const sa_shape* shape, const void* k, int blk_begin, int blk_end,
                                     void* blk_mean, float* kbar_absmax, const float* mu_k, int8_t* blk_code,
                                     float* blk_meta, void* stream);
+
+/* Appends one token per unit at position L = shape->L of a cache with room
+ * for it (L < ld): k[b, g, L, :] = k_new[b, g, :] and v likewise (k_new,
+ * v_new [B, Hkv, d] in dtype), and refreshes the statistics so that they
+ * describe the L + 1 tokens:
+ *   sum_k += k_new, sum_v += v_new (the totals behind the tail means of
+ *   SA_PROXY, OpenAttention stage 04);
+ *   per query head h of the unit, with p = s mu_q,h . k_new (fp32):
+ *     log_z0' = ln(exp(log_z0) + exp(p)),
+ *     o_est'  = exp(log_z0 - log_z0') o_est + exp(p - log_z0') v_new,
+ *   so that O_Est and Z stay the typical query's attention over the whole
+ *   cache (RESA, key design 1), which SA_RESA's tail estimate subtracts the
+ *   read set from;
+ *   when the token completes block c = (L + 1)/16 - 1: blk_mean[c], its
+ *   sketch row and kbar_absmax, as sa_block_summaries for that block.
+ * mu_q and mu_k stay as computed at prefill end (the RESA page fixes the
+ * typical query and key there; mu_k is also the sketch's centre, which must
+ * not move while rows sketched against it remain).  After the call the
+ * cache holds L + 1 tokens: later calls pass L + 1.  scale = softmax scale
+ * (0 = 1/sqrt(d)).  No workspace; one kernel, plus the block summary
+ * kernels when a block completes. */
+SA_API sa_status sa_append(const sa_shape* shape, const void* k_new, const void* v_new, void* k, void* v,
+                           const sa_stats* stats, float scale, void* stream);
 
 /* Rebuilds the sketch (blk_code, blk_meta) of blocks [blk_begin, blk_end) of
  * every unit from blk_mean relative to mu_k, for callers that write blk_mean

@@ -36,7 +36,7 @@ class SAError(RuntimeError):
 
 class sa_shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("d", ctypes.c_int),
-                ("L", ctypes.c_int), ("dtype", ctypes.c_int)]
+                ("L", ctypes.c_int), ("dtype", ctypes.c_int), ("ld", ctypes.c_int)]
 
 
 class sa_stats(ctypes.Structure):
@@ -62,7 +62,8 @@ class sa_decode_params(ctypes.Structure):
 
 EXPORTS = ("sa_workspace_size", "sa_prefill_stats", "sa_block_summaries", "sa_block_sketch", "sa_select",
            "sa_select_noalloc",
-           "sa_decode", "sa_step", "sa_step_fused", "sa_dense_decode", "sa_wait_timeouts", "sa_status_string")
+           "sa_decode", "sa_step", "sa_step_fused", "sa_dense_decode", "sa_append", "sa_wait_timeouts",
+           "sa_status_string")
 
 _LIB = None
 
@@ -87,6 +88,7 @@ def _lib():
         lib.sa_decode.argtypes = [sh, dp, sp, P, P, P, st, sel, P, P, S, P]
         lib.sa_step.argtypes = [sh, dp, sp, P, P, P, st, sel, P, P, S, P]
         lib.sa_dense_decode.argtypes = [sh, P, P, P, P, F, P, S, P]
+        lib.sa_append.argtypes = [sh, P, P, P, P, st, F, P]
         lib.sa_step_fused.argtypes = [sh, dp, sp]
         lib.sa_step_fused.restype = I
         lib.sa_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
@@ -94,7 +96,7 @@ def _lib():
         lib.sa_status_string.argtypes = [I]
         lib.sa_status_string.restype = ctypes.c_char_p
         for f in ("sa_prefill_stats", "sa_block_summaries", "sa_block_sketch", "sa_select", "sa_select_noalloc", "sa_decode", "sa_step",
-                  "sa_dense_decode"):
+                  "sa_dense_decode", "sa_append"):
             getattr(lib, f).restype = I
         _LIB = lib
     return _LIB
@@ -122,9 +124,11 @@ def _dtype_code(t):
     raise TypeError("cache dtype must be bfloat16 or float32, got %s" % t.dtype)
 
 
-def make_shape(k, Hq):
-    B, Hkv, L, d = k.shape
-    return sa_shape(B, Hq, Hkv, d, L, _dtype_code(k))
+def make_shape(k, Hq, length=None):
+    """Shape of a cache tensor k [B, Hkv, ld, d] holding `length` valid tokens
+    per unit (default: all ld)."""
+    B, Hkv, ld, d = k.shape
+    return sa_shape(B, Hq, Hkv, d, ld if length is None else int(length), _dtype_code(k), ld)
 
 
 @dataclass
@@ -203,11 +207,13 @@ def workspace(shape, params, op, device):
 
 
 def prefill_stats(q_ctx, k, v, stats=None, scale=0.0, stream=None):
-    B, Hkv, L, d = k.shape
-    Hq = q_ctx.shape[1]
-    shape = make_shape(k, Hq)
+    """Statistics of the first L = q_ctx.shape[2] tokens of a cache k, v
+    [B, Hkv, ld, d] (ld >= L: room for appended tokens)."""
+    B, Hkv, ld, d = k.shape
+    Hq, L = q_ctx.shape[1], q_ctx.shape[2]
+    shape = make_shape(k, Hq, L)
     if stats is None:
-        stats = Stats(B, Hq, Hkv, L, d, k.dtype, k.device)
+        stats = Stats(B, Hq, Hkv, ld, d, k.dtype, k.device)
     ws = workspace(shape, None, OP_PREFILL, k.device)
     st = stats.c()
     _check(_lib().sa_prefill_stats(ctypes.byref(shape), _ptr(q_ctx), _ptr(k), _ptr(v), ctypes.byref(st),
@@ -215,8 +221,8 @@ def prefill_stats(q_ctx, k, v, stats=None, scale=0.0, stream=None):
     return stats
 
 
-def block_summaries(k, blk_begin, blk_end, stats, Hq, stream=None):
-    shape = make_shape(k, Hq)
+def block_summaries(k, blk_begin, blk_end, stats, Hq, length=None, stream=None):
+    shape = make_shape(k, Hq, length)
     _check(_lib().sa_block_summaries(ctypes.byref(shape), _ptr(k), int(blk_begin), int(blk_end),
                                      _ptr(stats.blk_mean), _ptr(stats.kbar_absmax), _ptr(stats.mu_k),
                                      _ptr(stats.blk_code), _ptr(stats.blk_meta), _stream(stream)),
@@ -236,10 +242,10 @@ def block_sketch(stats, Hq, blk_begin=0, blk_end=None, stream=None):
            "sa_block_sketch")
 
 
-def select(q, stats, params, k=None, v=None, selection=None, scale=0.0, stream=None):
+def select(q, stats, params, k=None, v=None, selection=None, scale=0.0, length=None, stream=None):
     B, Hq, d = q.shape
-    Hkv, L = stats.blk_mean.shape[1], stats.blk_mean.shape[2] * 16
-    shape = sa_shape(B, Hq, Hkv, d, L, _dtype_code(q))
+    Hkv, ld = stats.blk_mean.shape[1], stats.blk_mean.shape[2] * 16
+    shape = sa_shape(B, Hq, Hkv, d, ld if length is None else int(length), _dtype_code(q), ld)
     cp = params.c()
     if selection is None:
         selection = Selection(B, Hkv, params.k_blocks, cp.sample_cap, q.device)
@@ -252,9 +258,10 @@ def select(q, stats, params, k=None, v=None, selection=None, scale=0.0, stream=N
     return selection
 
 
-def decode(q, k, v, stats, selection, params, mode="resa", lam=1.0, scale=0.0, out=None, stream=None):
+def decode(q, k, v, stats, selection, params, mode="resa", lam=1.0, scale=0.0, out=None, length=None,
+           stream=None):
     B, Hq, d = q.shape
-    shape = make_shape(k, Hq)
+    shape = make_shape(k, Hq, length)
     cp = params.c()
     dp = sa_decode_params(MODES[mode], float(lam), float(scale))
     if out is None:
@@ -268,12 +275,13 @@ def decode(q, k, v, stats, selection, params, mode="resa", lam=1.0, scale=0.0, o
     return out
 
 
-def step(q, k, v, stats, params, mode="resa", lam=1.0, scale=0.0, selection=None, out=None, stream=None):
+def step(q, k, v, stats, params, mode="resa", lam=1.0, scale=0.0, selection=None, out=None, length=None,
+         stream=None):
     """Selection then decode in one call: one fused kernel when step_fused()
     says so, else the two kernels with the decode overlapping the end of the
     selection (programmatic dependent launch).  Returns (out, selection)."""
     B, Hq, d = q.shape
-    shape = make_shape(k, Hq)
+    shape = make_shape(k, Hq, length)
     cp = params.c()
     dp = sa_decode_params(MODES[mode], float(lam), float(scale))
     if selection is None:
@@ -289,9 +297,9 @@ def step(q, k, v, stats, params, mode="resa", lam=1.0, scale=0.0, selection=None
     return out, selection
 
 
-def step_fused(q, k, params, mode="resa"):
+def step_fused(q, k, params, mode="resa", length=None):
     """True when step() runs as the single fused kernel for these arguments."""
-    shape = make_shape(k, q.shape[1])
+    shape = make_shape(k, q.shape[1], length)
     r = _lib().sa_step_fused(ctypes.byref(shape), ctypes.byref(sa_decode_params(MODES[mode], 1.0, 0.0)),
                              ctypes.byref(params.c()))
     if r < 0:
@@ -299,15 +307,26 @@ def step_fused(q, k, params, mode="resa"):
     return r == 1
 
 
-def dense_decode(q, k, v, scale=0.0, out=None, stream=None):
+def dense_decode(q, k, v, scale=0.0, out=None, length=None, stream=None):
     B, Hq, d = q.shape
-    shape = make_shape(k, Hq)
+    shape = make_shape(k, Hq, length)
     if out is None:
         out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
     ws = workspace(shape, None, OP_DENSE, q.device)
     _check(_lib().sa_dense_decode(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(out), float(scale),
                                   _ptr(ws), ws.numel(), _stream(stream)), "sa_dense_decode")
     return out
+
+
+def append(k_new, v_new, k, v, stats, length, scale=0.0, stream=None):
+    """Writes one token per unit (k_new, v_new [B, Hkv, d]) at position
+    `length` of the cache k, v [B, Hkv, ld, d] and refreshes the statistics
+    (see sa_append).  Returns the new length."""
+    shape = make_shape(k, stats.mu_q.shape[1], length)
+    st = stats.c()
+    _check(_lib().sa_append(ctypes.byref(shape), _ptr(k_new), _ptr(v_new), _ptr(k), _ptr(v), ctypes.byref(st),
+                            float(scale), _stream(stream)), "sa_append")
+    return int(length) + 1
 
 
 def wait_timeouts():

@@ -21,15 +21,16 @@ bool aligned4(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_
 sa_status check_shape(const sa_shape* s, Dims* d) {
     if (s == nullptr) return SA_ERR_INVALID_ARG;
     if (s->B < 1 || s->Hkv < 1 || s->Hq < 1 || s->L < 16 || s->d < 1) return SA_ERR_INVALID_ARG;
-    if (s->Hq % s->Hkv != 0 || s->L % 16 != 0) return SA_ERR_INVALID_ARG;
+    const int ld = s->ld == 0 ? s->L : s->ld;
+    if (s->Hq % s->Hkv != 0 || ld % 16 != 0 || ld < s->L) return SA_ERR_INVALID_ARG;
     if (s->dtype != SA_F32 && s->dtype != SA_BF16) return SA_ERR_INVALID_ARG;
     const int G = s->Hq / s->Hkv;
     if (G != 1 && G != 2 && G != 4 && G != 8) return SA_ERR_UNSUPPORTED;
     if (s->d != 64 && s->d != 128) return SA_ERR_UNSUPPORTED;
-    if ((long long)s->L * s->d >= (1LL << 31) || (long long)s->B * s->Hq >= 65536 ||
+    if ((long long)ld * s->d >= (1LL << 31) || (long long)s->B * s->Hq >= 65536 ||
         (long long)s->B * s->Hkv >= 65536)
         return SA_ERR_UNSUPPORTED;
-    d->B = s->B; d->Hq = s->Hq; d->Hkv = s->Hkv; d->G = G; d->d = s->d; d->L = s->L;
+    d->B = s->B; d->Hq = s->Hq; d->Hkv = s->Hkv; d->G = G; d->d = s->d; d->L = s->L; d->ld = ld;
     d->bf16 = s->dtype == SA_BF16;
     return SA_OK;
 }
@@ -108,6 +109,7 @@ sa_status sa_prefill_stats(const sa_shape* shape, const void* q_ctx, const void*
     Dims d;
     sa_status e = check_shape(shape, &d);
     if (e != SA_OK) return e;
+    if (d.L % 16 != 0) return SA_ERR_INVALID_ARG;     // the statistics cover whole blocks
     if (!aligned16(q_ctx) || !aligned16(k) || !aligned16(v) || !check_stats(out, true) || scale < 0.f)
         return SA_ERR_INVALID_ARG;
     const PrefillPlan p = prefill_plan(d);
@@ -130,6 +132,22 @@ sa_status sa_block_summaries(const sa_shape* shape, const void* k, int blk_begin
     if (blk_begin == blk_end) return SA_OK;
     return launch_block_summaries(d, k, blk_begin, blk_end, blk_mean, kbar_absmax, mu_k, blk_code, blk_meta,
                                   static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SA_OK
+               : SA_ERR_CUDA;
+}
+
+sa_status sa_append(const sa_shape* shape, const void* k_new, const void* v_new, void* k, void* v,
+                    const sa_stats* stats, float scale, void* stream) {
+    NvtxRange r("sa_append");
+    Dims d;
+    sa_status e = check_shape(shape, &d);
+    if (e != SA_OK) return e;
+    if (d.L >= d.ld) return SA_ERR_INVALID_ARG;       // no room for the token
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k) || !aligned16(v) || !check_stats(stats, true) ||
+        scale < 0.f)
+        return SA_ERR_INVALID_ARG;
+    return launch_append(d, k_new, v_new, k, v, *stats, resolve_scale(scale, d.d),
+                         static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? SA_OK
                : SA_ERR_CUDA;
 }

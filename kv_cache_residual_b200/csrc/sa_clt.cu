@@ -41,7 +41,8 @@ struct CltSmem {
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads)
-k_clt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, int Hq, int Hkv, int L, SetGeom sg,
+k_clt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, int Hq, int Hkv, int L, int ld,
+      SetGeom sg,
       const int32_t* __restrict__ blk_idx, int kb_stride, int32_t* __restrict__ samp_idx,
       int32_t* __restrict__ samp_count, int sample_cap, int b0, double eps, double delta, double scale,
       unsigned long long seed, int step) {
@@ -62,8 +63,8 @@ k_clt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nt = sg.n_t;
     if (nt == 0 || b0 < 2) return;                    // the selection wrote the (empty) sample
-    const T* K = k + (size_t)u * L * D;
-    const T* V = v + (size_t)u * L * D;
+    const T* K = k + (size_t)u * ld * D;
+    const T* V = v + (size_t)u * ld * D;
     const int32_t* gblk = blk_idx + (size_t)u * kb_stride;
     const int32_t* gsamp = samp_idx + (size_t)u * sample_cap;
     const int n_indep = sg.s_eff + sg.w_eff, n_i = sg.n_i, n_tok = n_i + b0;
@@ -268,7 +269,7 @@ static cudaError_t clt_t(const Dims& d, const SelectPlan& p, const SelectArgs& a
     if (e != cudaSuccess) return e;
     k_clt<T, D, G><<<d.U(), kThreads, smem, s>>>(
         reinterpret_cast<const T*>(a.q), reinterpret_cast<const T*>(a.k), reinterpret_cast<const T*>(a.v), d.Hq,
-        d.Hkv, d.L, p.g, a.sel.blk_idx, a.sp.k_blocks, a.sel.samp_idx, a.sel.samp_count, a.sp.sample_cap,
+        d.Hkv, d.L, d.ld, p.g, a.sel.blk_idx, a.sp.k_blocks, a.sel.samp_idx, a.sel.samp_count, a.sp.sample_cap,
         a.sp.clt_base, (double)a.sp.eps, (double)a.sp.delta, (double)a.scale, (unsigned long long)a.sp.seed,
         a.sp.step);
     return cudaGetLastError();

@@ -27,7 +27,7 @@ template <typename T, int D, int G, int MODE>
 __global__ void __launch_bounds__(kThreads)
 k_decode(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, sa_stats st,
          const int32_t* __restrict__ blk_idx, int kb_stride, const int32_t* __restrict__ samp_idx,
-         const int32_t* __restrict__ samp_count, int sample_cap, int Hq, int Hkv, int L, SetGeom sg,
+         const int32_t* __restrict__ samp_count, int sample_cap, int Hq, int Hkv, int L, int ld, SetGeom sg,
          int tok, int nsd, int rec, float qscale, float scale, float lambda,
          float* __restrict__ part, unsigned* __restrict__ cnt, float* __restrict__ out) {
     constexpr bool PRIOR = (MODE == SA_RESA);
@@ -47,7 +47,7 @@ k_decode(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__
     const int b = u / Hkv, g = u - b * Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int li = lane % CPR, gsub = lane / CPR;
-    const size_t ubase = (size_t)u * L * D;
+    const size_t ubase = (size_t)u * ld * D;
     const T* K = k + ubase + li * EPC;
     const T* V = v + ubase + li * EPC;
     const T* qg = q + ((size_t)b * Hq + (size_t)g * G) * D;
@@ -179,7 +179,7 @@ k_decode(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads)
 k_dense(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, int Hq, int Hkv,
-        int L, int tok, int nsdn, int rec, float qscale, float* __restrict__ part,
+        int L, int ld, int tok, int nsdn, int rec, float qscale, float* __restrict__ part,
         unsigned* __restrict__ cnt, float* __restrict__ out) {
     using Gm = Geom<T, D>;
     constexpr int EPC = Gm::EPC, CPR = Gm::CPR, GPW = Gm::GPW, NG = Gm::NG;
@@ -188,7 +188,7 @@ k_dense(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ 
     const int b = u / Hkv, g = u - b * Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int li = lane % CPR, gsub = lane / CPR;
-    const size_t ubase = (size_t)u * L * D;
+    const size_t ubase = (size_t)u * ld * D;
     const T* K = k + ubase + li * EPC;
     const T* V = v + ubase + li * EPC;
     const T* qg = q + ((size_t)b * Hq + (size_t)g * G) * D;
@@ -264,7 +264,7 @@ static cudaError_t stream_launch(const Dims& d, dim3 grid, const void* q, const 
     io.samp_idx = sel.samp_idx;
     io.samp_count = sel.samp_count;
     io.sample_cap = sp.sample_cap;
-    io.Hq = d.Hq; io.Hkv = d.Hkv; io.L = d.L;
+    io.Hq = d.Hq; io.Hkv = d.Hkv; io.L = d.L; io.ld = d.ld;
     io.sg = sg;
     io.tpc = tpc; io.nchunk = nchunk; io.rec = rec;
     io.qscale = scale * kLog2e; io.scale = scale; io.lambda = lambda;
@@ -294,7 +294,7 @@ static cudaError_t decode_m(const Dims& d, const DecodePlan& p, const DecodeArgs
         k_decode<T, D, G, MODE><<<dim3(p.nsd, d.U()), kThreads, 0, s>>>(
             reinterpret_cast<const T*>(a.q), reinterpret_cast<const T*>(a.k), reinterpret_cast<const T*>(a.v),
             a.st, a.sel.blk_idx, a.sp.k_blocks, a.sel.samp_idx, a.sel.samp_count, a.sp.sample_cap,
-            d.Hq, d.Hkv, d.L, p.g, p.tok_d, p.nsd, p.rec, a.scale * kLog2e, a.scale, a.dp.lambda,
+            d.Hq, d.Hkv, d.L, d.ld, p.g, p.tok_d, p.nsd, p.rec, a.scale * kLog2e, a.scale, a.dp.lambda,
             reinterpret_cast<float*>(a.ws + p.off_part), reinterpret_cast<unsigned*>(a.ws + p.off_cnt), a.out);
         return cudaGetLastError();
     }
@@ -340,7 +340,7 @@ static cudaError_t dense_t(const Dims& d, const DensePlan& p, const DenseArgs& a
     } else {
         k_dense<T, D, G><<<dim3(p.nsdn, d.U()), kThreads, 0, s>>>(
             reinterpret_cast<const T*>(a.q), reinterpret_cast<const T*>(a.k), reinterpret_cast<const T*>(a.v),
-            d.Hq, d.Hkv, d.L, p.tok, p.nsdn, p.rec, a.scale * kLog2e,
+            d.Hq, d.Hkv, d.L, d.ld, p.tok, p.nsdn, p.rec, a.scale * kLog2e,
             reinterpret_cast<float*>(a.ws + p.off_part), reinterpret_cast<unsigned*>(a.ws + p.off_cnt), a.out);
         return cudaGetLastError();
     }

@@ -295,6 +295,7 @@ struct StreamIo {
     const int32_t* samp_count;
     int sample_cap;
     int Hq, Hkv, L;
+    int ld;                      // tokens per unit in the cache allocation
     SetGeom sg;
     int tpc, nchunk, rec;        // tiles per chunk, chunks per unit, floats per chunk record
     float qscale, scale, lambda;
@@ -337,7 +338,7 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
 
     const int b = u / Hkv, g = u - b * Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const size_t ubase = (size_t)u * L * D;
+    const size_t ubase = (size_t)u * io.ld * D;
     const __nv_bfloat16* K = k + ubase;
     const __nv_bfloat16* V = v + ubase;
     const __nv_bfloat16* qg = q + ((size_t)b * Hq + (size_t)g * G) * D;

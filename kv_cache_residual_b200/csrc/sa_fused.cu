@@ -64,7 +64,7 @@ k_step_fused(SelectIo sio, StreamIo dio) {
     // the rows every step reads whatever the selection: sink and window
     if (threadIdx.x == 0) {
         const SetGeom& g = dio.sg;
-        const size_t ubase = (size_t)u * dio.L * D;
+        const size_t ubase = (size_t)u * dio.ld * D;
         const uint32_t rb = D * 2;                      // bf16 row bytes
         if (g.s_eff > 0) {
             bulk_prefetch_l2(dio.k + ubase, (uint32_t)g.s_eff * rb);
@@ -164,7 +164,7 @@ cudaError_t launch_step_fused(const Dims& d, const SelectPlan& sp, const SelectA
     dio.samp_idx = da.sel.samp_idx;
     dio.samp_count = da.sel.samp_count;
     dio.sample_cap = da.sp.sample_cap;
-    dio.Hq = d.Hq; dio.Hkv = d.Hkv; dio.L = d.L;
+    dio.Hq = d.Hq; dio.Hkv = d.Hkv; dio.L = d.L; dio.ld = d.ld;
     dio.sg = dp.g;
     dio.tpc = dp.tok_d; dio.nchunk = dp.nsd; dio.rec = dp.rec;
     dio.qscale = da.scale * kLog2e; dio.scale = da.scale; dio.lambda = da.dp.lambda;

@@ -18,9 +18,11 @@ constexpr int kStreamSlots = 148 * 2; // resident CTAs of the bf16 stream kernel
 
 struct Dims {
     int B, Hq, Hkv, G, d, L;
+    int ld;            // tokens per unit in the cache allocation (>= L, multiple of 16)
     int bf16;          // 1: bf16 cache and queries, 0: fp32
     int U() const { return B * Hkv; }
-    int nb() const { return L / 16; }
+    int nb() const { return L / 16; }      // complete blocks of the current length
+    int nbl() const { return ld / 16; }    // block rows per unit in the summary arrays
 };
 
 // Exactly-read set geometry of a unit (same for all units of a shape).
@@ -183,6 +185,9 @@ cudaError_t launch_block_summaries(const Dims& d, const void* k, int blk_begin, 
                                    cudaStream_t s);
 cudaError_t launch_block_sketch(const Dims& d, const void* blk_mean, const float* centre, int blk_begin, int blk_end,
                                 int8_t* blk_code, float* blk_meta, cudaStream_t s);
+// one token per unit at position d.L (sa_append.cu)
+cudaError_t launch_append(const Dims& d, const void* k_new, const void* v_new, void* k, void* v,
+                          const sa_stats& st, float scale, cudaStream_t s);
 
 struct SelectArgs {
     const void* q; sa_stats st; const void* k; const void* v;

@@ -70,7 +70,7 @@ k_qmean(const T* __restrict__ q_ctx, int L, int rows, int nsq, float* __restrict
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads)
 k_kvpass(const T* __restrict__ k, const T* __restrict__ v, const float* __restrict__ mu_q,
-         int Hq, int Hkv, int L, int tok, int nskv, float qscale, int stride,
+         int Hq, int Hkv, int L, int ld, int tok, int nskv, float qscale, int stride,
          float* __restrict__ part, unsigned* __restrict__ cnt, sa_stats st) {
     using Gm = Geom<T, D>;
     constexpr int EPC = Gm::EPC, CPR = Gm::CPR, NG = Gm::NG;
@@ -83,10 +83,10 @@ k_kvpass(const T* __restrict__ k, const T* __restrict__ v, const float* __restri
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gi = warp * Gm::GPW + lane / CPR, li = lane % CPR;
     const int nb = L / 16;
-    const size_t ubase = (size_t)u * L * D;
+    const size_t ubase = (size_t)u * ld * D;
     const T* K = k + ubase + li * EPC;
     const T* V = v + ubase + li * EPC;
-    T* BM = reinterpret_cast<T*>(st.blk_mean) + (size_t)u * nb * D + li * EPC;
+    T* BM = reinterpret_cast<T*>(st.blk_mean) + (size_t)u * (ld / 16) * D + li * EPC;
 
     float q0[G][EPC];
 #pragma unroll
@@ -222,15 +222,15 @@ k_kvpass(const T* __restrict__ k, const T* __restrict__ v, const float* __restri
 // Block means of blocks [blk_begin, blk_end) of every unit; raises kbar_absmax.
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
-k_blockmeans(const T* __restrict__ k, int L, int blk_begin, int blk_end, T* __restrict__ blk_mean,
+k_blockmeans(const T* __restrict__ k, int ld, int blk_begin, int blk_end, T* __restrict__ blk_mean,
              float* __restrict__ kbar_absmax) {
     using Gm = Geom<T, D>;
     constexpr int EPC = Gm::EPC, CPR = Gm::CPR, NG = Gm::NG;
     const int u = blockIdx.y;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gi = warp * Gm::GPW + lane / CPR, li = lane % CPR;
-    const int nb = L / 16;
-    const T* K = k + (size_t)u * L * D + li * EPC;
+    const int nb = ld / 16;
+    const T* K = k + (size_t)u * ld * D + li * EPC;
     float amax = 0.f;
     for (int blk = blk_begin + blockIdx.x * NG + gi; blk < blk_end; blk += gridDim.x * NG) {
         double bs[EPC];
@@ -324,7 +324,7 @@ static cudaError_t sketch_t(const Dims& d, const void* bm, const float* centre, 
                             float* meta, cudaStream_t s) {
     const int nblk = b1 - b0;
     const int gx = max(1, min(cdiv(nblk, kWarps), cdiv(4 * kSmTarget, d.U())));
-    k_sketch<T, D><<<dim3(gx, d.U()), kThreads, 0, s>>>(reinterpret_cast<const T*>(bm), centre, d.L / 16, b0, b1,
+    k_sketch<T, D><<<dim3(gx, d.U()), kThreads, 0, s>>>(reinterpret_cast<const T*>(bm), centre, d.nbl(), b0, b1,
                                                         code, reinterpret_cast<float4*>(meta));
     return cudaGetLastError();
 }
@@ -349,7 +349,7 @@ static cudaError_t prefill_t(const Dims& d, const PrefillPlan& p, const PrefillA
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     k_kvpass<T, D, G><<<dim3(p.nskv, d.U()), kThreads, 0, s>>>(
-        reinterpret_cast<const T*>(a.k), reinterpret_cast<const T*>(a.v), a.st.mu_q, d.Hq, d.Hkv, d.L,
+        reinterpret_cast<const T*>(a.k), reinterpret_cast<const T*>(a.v), a.st.mu_q, d.Hq, d.Hkv, d.L, d.ld,
         p.tok_kv, p.nskv, a.scale * kLog2e, p.kv_stride, reinterpret_cast<float*>(ws + p.off_kvpart),
         reinterpret_cast<unsigned*>(ws + p.off_kvcnt), a.st);
     e = cudaGetLastError();
@@ -380,7 +380,7 @@ static cudaError_t blockmeans_t(const Dims& d, const void* k, int b0, int b1, vo
     const int nblk = b1 - b0;
     const int gx = max(1, min(cdiv(nblk, Gm::NG), cdiv(kSmTarget, d.U())));
     k_blockmeans<T, D><<<dim3(gx, d.U()), kThreads, 0, s>>>(
-        reinterpret_cast<const T*>(k), d.L, b0, b1, reinterpret_cast<T*>(bm), amax);
+        reinterpret_cast<const T*>(k), d.ld, b0, b1, reinterpret_cast<T*>(bm), amax);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return sketch_t<T, D>(d, bm, centre, b0, b1, code, meta, s);

@@ -36,7 +36,7 @@ SelectIo select_io(const Dims& d, const SelectPlan& p, const SelectArgs& a) {
     io.blk_mean = a.st.blk_mean;
     io.blk_code = a.st.blk_code;
     io.blk_meta = reinterpret_cast<const float4*>(a.st.blk_meta);
-    io.Hq = d.Hq; io.Hkv = d.Hkv; io.L = d.L;
+    io.Hq = d.Hq; io.Hkv = d.Hkv; io.L = d.L; io.ld = d.ld;
     io.sg = p.g;
     io.rows = p.rows_s; io.nss = p.nss;
     io.sc_lo_all = reinterpret_cast<float*>(ws + p.off_scores);

@@ -462,6 +462,7 @@ struct SelectIo {
     const int8_t* blk_code;
     const float4* blk_meta;
     int Hq, Hkv, L;
+    int ld;                      // tokens per unit in the cache allocation (block rows ld / 16)
     SetGeom sg;
     int rows, nss;                        // candidate rows per split, splits per unit
     float* sc_lo_all;                     // [U][n_cand] lower bounds (split units)
@@ -557,7 +558,7 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
     const int b = u / Hkv, g = u - b * Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int li = lane % CPR, gsub = lane / CPR;
-    const int nb = L / 16;
+    const int nb = io.ld / 16;         // block rows per unit
     const int n = sg.n_cand, kk = sg.kk;
     const T* qg = q + ((size_t)b * Hq + (size_t)g * G) * D;
     float* sc_lo = io.sc_lo_all + (size_t)u * (n > 0 ? n : 1);

@@ -15,10 +15,20 @@ sums are totals minus the selected part), and the 16-token block means the
 block selector ranks (Quest/ArkVale-style page summaries named on the RESA
 page's related work), rounded once to the cache dtype.
 
+Decode grows the cache after prefill end (grown_stats): the statistics then
+describe all cached tokens while the typical query and key stay the ones of
+prefill end.  Reading: the RESA page fixes mu_Q and mu_K at prefill end and
+defines O_Est and the normaliser as the typical query's attention over the
+cache, which its tail estimate removes the read set from; so O_Est, log_z0
+and the totals cover every cached token, and mu_K (also the centre the block
+sketch is built around) does not move.
+
 Parity pins (tests/test_oracle_stats.py): closed forms for constant keys /
 queries (log_z0 = ln L + s mu_Q.kappa, O_Est = mean V), O_Est against torch's
 scaled_dot_product_attention with query mu_Q, block means against torch's
-bf16 cast where the mean is an fp32 value.
+bf16 cast where the mean is an fp32 value; grown statistics against a
+token-by-token log-sum-exp recurrence from the prefill-end values and
+against constant-key closed forms at lengths that are not whole blocks.
 """
 import numpy as np
 
@@ -28,11 +38,12 @@ BLOCK = 16
 
 
 def block_means(k, kv_dtype):
-    """k [L, d] float64 -> [L/16, d]: mean of each 16-token block, computed in
-    fp64 and rounded once to the cache dtype (nearest, ties to even)."""
+    """k [L, d] float64 -> [L//16, d]: mean of each complete 16-token block,
+    computed in fp64 and rounded once to the cache dtype (nearest, ties to
+    even); a partial last block has no mean."""
     L, d = k.shape
-    assert L % BLOCK == 0
-    return round_to(k.reshape(L // BLOCK, BLOCK, d).mean(axis=1), kv_dtype)
+    nb = L // BLOCK
+    return round_to(k[: nb * BLOCK].reshape(nb, BLOCK, d).mean(axis=1), kv_dtype)
 
 
 def prefill_stats(q_ctx, k, v, scale, kv_dtype):
@@ -59,4 +70,22 @@ def prefill_stats(q_ctx, k, v, scale, kv_dtype):
         "mu_q": mu_q, "o_est": o_est, "log_z0": log_z0,
         "mu_k": mu_k, "sum_k": sum_k, "sum_v": sum_v,
         "blk_mean": bm, "kbar_absmax": float(np.abs(bm).max()),
+    }
+
+
+def grown_stats(st0, k, v, scale, kv_dtype):
+    """Statistics of a cache that holds L' = len(k) tokens after growing past
+    prefill end, with the typical query and key of prefill end (st0["mu_q"],
+    st0["mu_k"]): O_Est and log_z0 of mu_Q over all L' keys, the totals of
+    all L' keys and values, and the means of the complete blocks."""
+    mu_q = st0["mu_q"]
+    p0 = scale * (mu_q @ k.T)                  # prior logits [G, L']
+    m = p0.max(axis=1, keepdims=True)
+    w = np.exp(p0 - m)
+    a = w.sum(axis=1)
+    bm = block_means(k, kv_dtype)
+    return {
+        "mu_q": mu_q, "o_est": (w @ v) / a[:, None], "log_z0": np.log(a) + m[:, 0],
+        "mu_k": st0["mu_k"], "sum_k": k.sum(axis=0), "sum_v": v.sum(axis=0),
+        "blk_mean": bm, "kbar_absmax": float(np.abs(bm).max()) if len(bm) else 0.0,
     }

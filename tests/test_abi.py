@@ -31,9 +31,9 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def _shape(**kw):
-    base = dict(B=2, Hq=8, Hkv=2, d=128, L=4096, dtype=sa.SA_BF16)
+    base = dict(B=2, Hq=8, Hkv=2, d=128, L=4096, dtype=sa.SA_BF16, ld=0)
     base.update(kw)
-    return sa.sa_shape(base["B"], base["Hq"], base["Hkv"], base["d"], base["L"], base["dtype"])
+    return sa.sa_shape(base["B"], base["Hq"], base["Hkv"], base["d"], base["L"], base["dtype"], base["ld"])
 
 
 def test_workspace_sizes(lib):
@@ -51,7 +51,9 @@ def test_workspace_sizes(lib):
     (dict(d=96), sa.SA_ERR_UNSUPPORTED),
     (dict(Hq=12, Hkv=4), sa.SA_ERR_UNSUPPORTED),     # G = 3
     (dict(Hq=9, Hkv=2), sa.SA_ERR_INVALID_ARG),
-    (dict(L=1000), sa.SA_ERR_INVALID_ARG),
+    (dict(L=1000), sa.SA_ERR_INVALID_ARG),          # not whole blocks and no capacity given
+    (dict(L=4096, ld=4080), sa.SA_ERR_INVALID_ARG),  # capacity below the length
+    (dict(L=4096, ld=4100), sa.SA_ERR_INVALID_ARG),  # capacity not whole blocks
     (dict(L=0), sa.SA_ERR_INVALID_ARG),
     (dict(B=0), sa.SA_ERR_INVALID_ARG),
     (dict(dtype=7), sa.SA_ERR_INVALID_ARG),
@@ -123,6 +125,40 @@ def test_select_and_decode_param_checks(lib):
     assert lib.sa_block_sketch(ctypes.byref(sh), p, p, 0, 8, p, ctypes.c_void_p(0x10008), None) == sa.SA_ERR_INVALID_ARG   # misaligned
     assert lib.sa_block_sketch(ctypes.byref(sh), p, None, 0, 8, p, p, None) == sa.SA_ERR_INVALID_ARG
     assert lib.sa_block_sketch(ctypes.byref(sh), p, p, 3, 3, p, p, None) == sa.SA_OK
+
+
+def test_capacity_and_partial_lengths(lib):
+    sp = sa.SelectParams(sink=64, local=128, k_blocks=8).c()
+    # a length that is not whole blocks is valid inside a capacity that is
+    for op in (sa.OP_SELECT, sa.OP_DECODE, sa.OP_DENSE):
+        assert lib.sa_workspace_size(ctypes.byref(_shape(L=4100, ld=4112)), ctypes.byref(sp), op) > 0
+    # but the prefill statistics cover whole blocks only
+    p = ctypes.c_void_p(0x10000)
+    st = sa.sa_stats(*([0x10000] * 10))
+    assert lib.sa_prefill_stats(ctypes.byref(_shape(L=4100, ld=4112)), p, p, p, ctypes.byref(st), 0.0, p,
+                                1 << 30, None) == sa.SA_ERR_INVALID_ARG
+    # block summaries: only complete blocks of the current length
+    assert lib.sa_block_summaries(ctypes.byref(_shape(L=4100, ld=4112)), p, 256, 257, p, p, p, p, p,
+                                  None) == sa.SA_ERR_INVALID_ARG
+
+
+def test_append_checks(lib):
+    p = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)
+    st = sa.sa_stats(*([0x10000] * 10))
+    st_bad = sa.sa_stats(*([0x10000] * 9 + [0x10004]))
+    sh = _shape(L=4096, ld=4112)
+    full = _shape(L=4112, ld=4112)
+    assert lib.sa_append(ctypes.byref(full), p, p, p, p, ctypes.byref(st), 0.0, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_append(ctypes.byref(_shape()), p, p, p, p, ctypes.byref(st), 0.0, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_append(ctypes.byref(sh), None, p, p, p, ctypes.byref(st), 0.0, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_append(ctypes.byref(sh), p, odd, p, p, ctypes.byref(st), 0.0, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_append(ctypes.byref(sh), p, p, p, None, ctypes.byref(st), 0.0, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_append(ctypes.byref(sh), p, p, p, p, None, 0.0, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_append(ctypes.byref(sh), p, p, p, p, ctypes.byref(st_bad), 0.0, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_append(ctypes.byref(sh), p, p, p, p, ctypes.byref(st), -1.0, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_append(ctypes.byref(_shape(L=4096, ld=4112, d=96)), p, p, p, p, ctypes.byref(st), 0.0,
+                         None) == sa.SA_ERR_UNSUPPORTED
 
 
 def test_status_strings(lib):

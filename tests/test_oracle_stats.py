@@ -5,7 +5,7 @@ import numpy as np
 import torch
 
 from oracle.numerics import round_to_bf16
-from oracle.stats import block_means, prefill_stats
+from oracle.stats import block_means, grown_stats, prefill_stats
 
 
 def _sdpa(q, k, v, scale):
@@ -59,3 +59,54 @@ def test_block_means_against_torch_cast():
     want = torch.from_numpy(means32).to(torch.bfloat16).double().numpy()
     np.testing.assert_array_equal(block_means(k, "bf16"), want)
     np.testing.assert_array_equal(block_means(k, "f32"), means32.astype(np.float64))
+
+
+def test_grown_stats_follow_the_token_recurrence():
+    """Statistics of a cache grown past prefill end: the definition over all
+    L' tokens equals folding the appended tokens in one at a time from the
+    prefill-end values (log-sum-exp of the normaliser, mass-weighted mix of
+    O_Est, running totals), the arithmetic an incremental update performs."""
+    rng = np.random.default_rng(3)
+    G, L0, n, d = 2, 64, 37, 16
+    s = 0.25
+    q_ctx = rng.standard_normal((G, L0, d)) + rng.standard_normal((G, 1, d))
+    k = rng.standard_normal((L0 + n, d)) * 1.5
+    v = rng.standard_normal((L0 + n, d))
+    st0 = prefill_stats(q_ctx, k[:L0], v[:L0], s, "f32")
+    lz, o = st0["log_z0"].copy(), st0["o_est"].copy()
+    sk, sv = st0["sum_k"].copy(), st0["sum_v"].copy()
+    for j in range(L0, L0 + n):
+        p = s * (st0["mu_q"] @ k[j])
+        lz_new = np.logaddexp(lz, p)
+        o = np.exp(lz - lz_new)[:, None] * o + np.exp(p - lz_new)[:, None] * v[j][None, :]
+        lz = lz_new
+        sk, sv = sk + k[j], sv + v[j]
+    g = grown_stats(st0, k, v, s, "f32")
+    np.testing.assert_allclose(g["log_z0"], lz, rtol=1e-13)
+    np.testing.assert_allclose(g["o_est"], o, rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(g["sum_k"], sk, rtol=1e-13, atol=1e-12)
+    np.testing.assert_allclose(g["sum_v"], sv, rtol=1e-13, atol=1e-12)
+    # the typical query and key stay the prefill-end ones
+    assert g["mu_q"] is st0["mu_q"] and g["mu_k"] is st0["mu_k"]
+    # complete blocks only: (64 + 37) // 16 = 6 means, the first 4 as at prefill
+    assert g["blk_mean"].shape == (6, d)
+    np.testing.assert_array_equal(g["blk_mean"][:4], st0["blk_mean"])
+
+
+def test_grown_stats_constant_keys_closed_form():
+    """Constant keys kappa over a length that is not a whole number of blocks:
+    log_z0 = ln L' + s mu_Q . kappa and O_Est = the mean of all L' values."""
+    rng = np.random.default_rng(4)
+    G, L0, n, d = 3, 48, 21, 8
+    kappa = round_to_bf16(rng.standard_normal(d))
+    k = np.tile(kappa, (L0 + n, 1))
+    v = rng.standard_normal((L0 + n, d))
+    q_ctx = rng.standard_normal((G, L0, d))
+    s = 1 / math.sqrt(d)
+    st0 = prefill_stats(q_ctx, k[:L0], v[:L0], s, "bf16")
+    g = grown_stats(st0, k, v, s, "bf16")
+    Lg = L0 + n
+    np.testing.assert_allclose(g["log_z0"], math.log(Lg) + s * (st0["mu_q"] @ kappa), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(g["o_est"], np.tile(v.mean(0), (G, 1)), atol=1e-13)
+    np.testing.assert_allclose(g["sum_k"], Lg * kappa, rtol=1e-15)
+    np.testing.assert_array_equal(g["blk_mean"], np.tile(kappa, (Lg // 16, 1)))
