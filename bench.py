@@ -452,6 +452,30 @@ def main(argv=None):
                "h2d_bytes_per_step": int(Q[0].numel() * Q.element_size()),
                "d2h_bytes_per_step": int(out.numel() * 4)}
 
+    # cache append (the cache growing during decode): one token per unit
+    # through sa_append, written at the last row of the cache with that row's
+    # own values (the cache is left as it was) into a copy of the per-unit
+    # statistics; the token completes a block, so the block summary kernels
+    # run too.  Latency-bound: a few KB per unit.
+    app_st = sa.Stats.__new__(sa.Stats)
+    for f in sa.Stats.FIELDS:
+        t_ = getattr(stats, f)
+        setattr(app_st, f, t_ if f in ("blk_mean", "blk_code", "blk_meta") else t_.clone())
+    k_last = K[:, :, w.L - 1].contiguous()
+    v_last = V[:, :, w.L - 1].contiguous()
+
+    def append_fn(t, ev):
+        ev[0].record(stream)
+        sa.append(k_last, v_last, K, V, app_st, w.L - 1)
+        ev[1].record(stream)
+    timed(3, append_fn, 2)
+    pa = timed(20, append_fn, 2)
+    app_ms = statistics.mean(p[0] for p in pa)
+    app_bytes = w.B * w.Hkv * (4 * w.d * esz + 4 * w.d * 4 + w.G * (3 * w.d * 4 + 8))
+    append = {"us_per_call": 1e3 * app_ms, "algorithmic_bytes": app_bytes,
+              "note": "one token per unit, block summary included"}
+    del app_st
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
         rate, units, threads = cpu_oracle_sample(w, sp_kw, args.mode, args.cpu_seconds)
@@ -475,6 +499,7 @@ def main(argv=None):
             "dense": dense, "speedup_vs_dense": dense_ms / ms_per_step, "modes": mode_vals,
             "kernels_us": {"k_select": 1e3 * sel_avg, "k_decode": 1e3 * dec_avg,
                            "separate_sum": 1e3 * (sel_avg + dec_avg), "step_overlapped": 1e3 * ms_per_step},
+            "append": append,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps, "clocks": clk,
         }
         print(json.dumps(line))
