@@ -455,8 +455,8 @@ def main(argv=None):
     # cache append (the cache growing during decode): one token per unit
     # through sa_append, written at the last row of the cache with that row's
     # own values (the cache is left as it was) into a copy of the per-unit
-    # statistics; the token completes a block, so the block summary kernels
-    # run too.  Latency-bound: a few KB per unit.
+    # statistics; the token completes a block, so the same kernel also
+    # summarises that block.  Latency-bound: a few KB per unit.
     app_st = sa.Stats.__new__(sa.Stats)
     for f in sa.Stats.FIELDS:
         t_ = getattr(stats, f)
@@ -471,9 +471,12 @@ def main(argv=None):
     timed(3, append_fn, 2)
     pa = timed(20, append_fn, 2)
     app_ms = statistics.mean(p[0] for p in pa)
-    app_bytes = w.B * w.Hkv * (4 * w.d * esz + 4 * w.d * 4 + w.G * (3 * w.d * 4 + 8))
+    # new rows in and out, totals, mu_Q / O_Est / log_z0; the completed
+    # block's 16 rows, its mean and sketch row
+    app_bytes = w.B * w.Hkv * (4 * w.d * esz + 4 * w.d * 4 + w.G * (3 * w.d * 4 + 8)
+                               + 17 * w.d * esz + w.d + 16)
     append = {"us_per_call": 1e3 * app_ms, "algorithmic_bytes": app_bytes,
-              "note": "one token per unit, block summary included"}
+              "note": "one token per unit completing a block (one kernel: k_append)"}
     del app_st
 
     cpu = None

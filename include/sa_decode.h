@@ -226,8 +226,7 @@ SA_API sa_status sa_block_summaries(const sa_shape* shape, const void* k, int bl
  * typical query and key there; mu_k is also the sketch's centre, which must
  * not move while rows sketched against it remain).  After the call the
  * cache holds L + 1 tokens: later calls pass L + 1.  scale = softmax scale
- * (0 = 1/sqrt(d)).  No workspace; one kernel, plus the block summary
- * kernels when a block completes. */
+ * (0 = 1/sqrt(d)).  No workspace; one kernel. */
 SA_API sa_status sa_append(const sa_shape* shape, const void* k_new, const void* v_new, void* k, void* v,
                            const sa_stats* stats, float scale, void* stream);
 

@@ -8,10 +8,13 @@
 // token into the typical query's attention: log_z0 grows by ln(1 + e^(p -
 // log_z0)) and O_Est becomes the mass-weighted mix of the old O_Est and v_new
 // (RESA, key design 1: O_Est and Z are that query's softmax over the cache).
-// When the token completes a 16-token block, the host launches the block
-// summary kernels for it (sa_prefill.cu).
+// When the token completes 16-token block `blk`, warp 0 then forms that
+// block's mean (fp64 sum of its 16 rows, rounded once to the cache dtype, as
+// the prefill does), raises kbar_absmax and writes the block's sketch row
+// (sketch_row, shared with the prefill's sketch kernel).
 #include "sa_common.cuh"
 #include "sa_internal.h"
+#include "sa_sketch.cuh"
 
 namespace sa {
 
@@ -20,7 +23,7 @@ constexpr int kAppendThreads = 128;
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kAppendThreads)
 k_append(const T* __restrict__ k_new, const T* __restrict__ v_new, T* __restrict__ k, T* __restrict__ v,
-         sa_stats st, int Hq, int Hkv, int L, int ld, float scale) {
+         sa_stats st, int Hq, int Hkv, int L, int ld, float scale, int blk) {
     static_assert(D <= kAppendThreads, "one thread per column");
     constexpr int NW = kAppendThreads / 32;
     __shared__ float s_part[G][NW];
@@ -61,11 +64,40 @@ k_append(const T* __restrict__ k_new, const T* __restrict__ v_new, T* __restrict
             *o = expf(lz - lz_new[h]) * *o + expf(p - lz_new[h]) * vf;
         }
     }
-    __syncthreads();           // every thread has read log_z0
+    __syncthreads();           // every thread has read log_z0; the new row is in the cache
     if (e == 0) {
 #pragma unroll
         for (int h = 0; h < G; ++h) st.log_z0[qh0 + h] = lz_new[h];
     }
+    if (blk < 0 || warp != 0) return;
+    // the completed block: lane l owns columns [l E, l E + E)
+    constexpr int E = D / 32;
+    double sum[E];
+#pragma unroll
+    for (int c = 0; c < E; ++c) sum[c] = 0.0;
+    for (int j = 0; j < 16; ++j) {
+        const T* r = k + ((size_t)u * ld + 16 * (size_t)blk + j) * D + lane * E;
+#pragma unroll
+        for (int c = 0; c < E; ++c) sum[c] += (double)to_f32<T>(r[c]);
+    }
+    const size_t row = (size_t)u * (ld / 16) + blk;
+    T* bm = reinterpret_cast<T*>(st.blk_mean) + row * D + lane * E;
+    float kbar[E];
+    double m[E];
+    float amax = 0.f;
+#pragma unroll
+    for (int c = 0; c < E; ++c) {
+        const T mean = round_from_f64<T>(sum[c] * 0.0625);
+        bm[c] = mean;
+        kbar[c] = to_f32<T>(mean);
+        amax = fmaxf(amax, fabsf(kbar[c]));
+        m[c] = (double)st.mu_k[(size_t)u * D + lane * E + c];
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    // non-negative floats order like their bit patterns as signed ints
+    if (lane == 0 && amax > 0.f) atomicMax(reinterpret_cast<int*>(st.kbar_absmax + u), __float_as_int(amax));
+    sketch_row<D>(kbar, m, st.blk_code + row * D, reinterpret_cast<float4*>(st.blk_meta) + row);
 }
 
 template <typename T, int D, int G>
@@ -73,7 +105,7 @@ static cudaError_t append_t(const Dims& d, const void* k_new, const void* v_new,
                             const sa_stats& st, float scale, cudaStream_t s) {
     k_append<T, D, G><<<d.U(), kAppendThreads, 0, s>>>(
         reinterpret_cast<const T*>(k_new), reinterpret_cast<const T*>(v_new), reinterpret_cast<T*>(k),
-        reinterpret_cast<T*>(v), st, d.Hq, d.Hkv, d.L, d.ld, scale);
+        reinterpret_cast<T*>(v), st, d.Hq, d.Hkv, d.L, d.ld, scale, (d.L + 1) % 16 == 0 ? (d.L + 1) / 16 - 1 : -1);
     return cudaGetLastError();
 }
 
@@ -91,20 +123,11 @@ static cudaError_t append_g(const Dims& d, const void* k_new, const void* v_new,
 
 cudaError_t launch_append(const Dims& d, const void* k_new, const void* v_new, void* k, void* v,
                           const sa_stats& st, float scale, cudaStream_t s) {
-    cudaError_t e;
     if (d.bf16)
-        e = d.d == 128 ? append_g<__nv_bfloat16, 128>(d, k_new, v_new, k, v, st, scale, s)
-                       : append_g<__nv_bfloat16, 64>(d, k_new, v_new, k, v, st, scale, s);
-    else
-        e = d.d == 128 ? append_g<float, 128>(d, k_new, v_new, k, v, st, scale, s)
-                       : append_g<float, 64>(d, k_new, v_new, k, v, st, scale, s);
-    if (e != cudaSuccess || (d.L + 1) % 16 != 0) return e;
-    // the new token completes block c: its mean, sketch row and kbar_absmax
-    Dims grown = d;
-    grown.L = d.L + 1;
-    const int c = grown.L / 16 - 1;
-    return launch_block_summaries(grown, k, c, c + 1, st.blk_mean, st.kbar_absmax, st.mu_k, st.blk_code,
-                                  st.blk_meta, s);
+        return d.d == 128 ? append_g<__nv_bfloat16, 128>(d, k_new, v_new, k, v, st, scale, s)
+                          : append_g<__nv_bfloat16, 64>(d, k_new, v_new, k, v, st, scale, s);
+    return d.d == 128 ? append_g<float, 128>(d, k_new, v_new, k, v, st, scale, s)
+                      : append_g<float, 64>(d, k_new, v_new, k, v, st, scale, s);
 }
 
 }  // namespace sa

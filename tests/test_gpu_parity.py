@@ -181,6 +181,22 @@ def test_resa_lambda_zero_is_drop(dev):
     assert rel_l2(f64(outs["resa"]), f64(outs["drop"])) < 1e-6
 
 
+@pytest.mark.parametrize("lam", [0.25, 0.5, 0.75])
+def test_resa_lambda_sweep(lam, dev):
+    """Prior weights between plain sparse attention (0) and the RESA page's
+    merge (1): the tail mass scaled in numerator and denominator (reading
+    C3), against the oracle at the same lambda on every unit."""
+    name = "bf16_d128_g4"
+    sp = _sp(CASES[name])
+    w, data, st, sel, outs = _edge_run(name, dev, sp, modes=("resa",), lam=lam)
+    for b, g in _units(w):
+        o = OracleUnit(data, b, g, w.G, w.dtype)
+        qq = o.q(data["q"][0])
+        blocks, idx, tail = o.select(qq, sp)
+        want = o.out("resa", qq, idx, lam=lam)
+        assert rel_l2(f64(outs["resa"][b, g * w.G:(g + 1) * w.G]), want) < REL_L2_OUT, (lam, b, g)
+
+
 def test_deterministic_outputs(dev):
     sp = _sp(CASES["bf16_d128_g4"])
     a = _edge_run("bf16_d128_g4", dev, sp)[4]
