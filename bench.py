@@ -50,6 +50,11 @@ def parse_args(argv=None):
     ap.add_argument("--read", type=float, default=0.01, help="read budget (fraction of L)")
     ap.add_argument("--mode", default="resa", choices=["drop", "resa", "proxy", "sample"])
     ap.add_argument("--sample-b", type=int, default=64)
+    ap.add_argument("--clt-base", type=int, default=0,
+                    help="sample mode: choose b per unit by the CLT budget from this many base draws")
+    ap.add_argument("--sample-cap", type=int, default=4096, help="draw capacity per unit with --clt-base")
+    ap.add_argument("--eps", type=float, default=0.1)
+    ap.add_argument("--delta", type=float, default=0.05)
     ap.add_argument("--queries", type=int, default=64, help="distinct decode queries cycled through")
     ap.add_argument("--dense-steps", type=int, default=50)
     ap.add_argument("--mode-steps", type=int, default=200)
@@ -312,13 +317,33 @@ def main(argv=None):
     wr = synth.scaled(w, seed=w.seed + 100_000 * rank)
     data = synth.make_batch(wr, device=dev, steps=nq)
     stats = sa.prefill_stats(data["q_ctx"], data["k"], data["v"])
+    # prefill statistics (once per sequence, not part of the step): one pass
+    # over the context queries and the cache
+    pf_ms = []
+    for r in range(4):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        sa.prefill_stats(data["q_ctx"], data["k"], data["v"], stats=stats)
+        e1.record()
+        torch.cuda.synchronize()
+        if r > 0:
+            pf_ms.append(e0.elapsed_time(e1))
+    pf_bytes = (data["q_ctx"].numel() + 2 * data["k"].numel()) * data["k"].element_size()
+    prefill = {"ms": statistics.mean(pf_ms), "hbm_gbs": pf_bytes / (statistics.mean(pf_ms) * 1e-3) / 1e9,
+               "bytes": pf_bytes}
     del data["q_ctx"]
     torch.cuda.empty_cache()
     K, V, Q = data["k"], data["v"], data["q"]
-    bdraw = args.sample_b if args.mode == "sample" else 0
-    sps = [sa.SelectParams(sink=w.sink, local=w.local, k_blocks=kb, sample_b=bdraw, sample_cap=max(bdraw, 1),
-                           seed=2024, step=t) for t in range(nq)]
-    sel = sa.select(Q[0], stats, sps[0])
+    clt = args.mode == "sample" and args.clt_base > 0
+    bdraw = args.sample_b if args.mode == "sample" and not clt else 0
+    if clt:
+        sps = [sa.SelectParams(sink=w.sink, local=w.local, k_blocks=kb, sample_b=0, sample_cap=args.sample_cap,
+                               clt_base=args.clt_base, eps=args.eps, delta=args.delta, seed=2024, step=t)
+               for t in range(nq)]
+    else:
+        sps = [sa.SelectParams(sink=w.sink, local=w.local, k_blocks=kb, sample_b=bdraw, sample_cap=max(bdraw, 1),
+                               seed=2024, step=t) for t in range(nq)]
+    sel = sa.select(Q[0], stats, sps[0], k=K, v=V)
     out = torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
@@ -359,7 +384,7 @@ def main(argv=None):
         def fn(t, ev):
             sp = sps[t % nq]
             ev[0].record(stream)
-            sa.select(Q[t % nq], stats, sp, selection=sel)
+            sa.select(Q[t % nq], stats, sp, k=K, v=V, selection=sel)
             ev[1].record(stream)
             sa.decode(Q[t % nq], K, V, stats, sel, sp, mode=mode, out=out)
             ev[2].record(stream)
@@ -389,8 +414,22 @@ def main(argv=None):
     ms_per_step = total_ms / args.steps
     value = ws * w.B * args.steps / (total_ms / 1e3)
 
-    sel_b = select_bytes_per_unit(w, sg, esz, bdraw) * w.B * w.Hkv
-    dec_b = decode_bytes_per_unit(w, sg, esz, args.mode, bdraw) * w.B * w.Hkv
+    b_mean = float(bdraw)
+    clt_info = None
+    if clt:
+        # the CLT budget decides b per unit: the mean over the queries timed
+        counts = []
+        for t in range(nq):
+            s_ = sa.select(Q[t], stats, sps[t], k=K, v=V)
+            counts.append(s_.samp_count.double().mean().item())
+        b_mean = statistics.mean(counts)
+        clt_info = {"base": args.clt_base, "eps": args.eps, "delta": args.delta, "mean_b": b_mean,
+                    "cap": args.sample_cap}
+    sel_b = select_bytes_per_unit(w, sg, esz, b_mean) * w.B * w.Hkv
+    if clt:
+        # the budget kernel reads I and the base draws' K and V rows
+        sel_b += (sg["n_i"] + args.clt_base) * 2 * w.d * esz * w.B * w.Hkv
+    dec_b = decode_bytes_per_unit(w, sg, esz, args.mode, b_mean) * w.B * w.Hkv
     peaks = {}
     pk_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(pk_path):
@@ -416,7 +455,11 @@ def main(argv=None):
         timed(3, fn, 2)
         pm = timed(args.mode_steps, fn, 2)
         ms = sum(p[0] for p in pm) / len(pm)
-        mode_vals[m] = {"tokens_per_s": w.B / (ms * 1e-3), "ms_per_step": ms}
+        # output error against the in-build dense attention, for one query
+        o_m, _ = sa.step(Q[0], K, V, stats, (sps_m or sps)[0], mode=m)
+        o_d = sa.dense_decode(Q[0], K, V)
+        err = ((o_m.double() - o_d.double()).norm() / o_d.double().norm()).item()
+        mode_vals[m] = {"tokens_per_s": w.B / (ms * 1e-3), "ms_per_step": ms, "rel_l2_vs_dense": err}
 
     # dense flash-decode reference (in-build)
     def dense_fn(t, ev):
@@ -493,7 +536,7 @@ def main(argv=None):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded generator, Llama-3.1-8B layer shapes)",
-            "config": workload_config(w, sg, args),
+            "config": dict(workload_config(w, sg, args), **({"clt": clt_info} if clt_info else {})),
             "roofline": {"bound": "hbm", "kernel": "k_select (sketch scan + certified top-k)", "achieved": sel_gbs,
                          "peak": peak, "unit": "GB/s", "frac": sel_gbs / peak, "traffic": traffic,
                          "bytes_per_launch": sel_b, "us_per_launch": 1e3 * sel_avg, "peak_source": peak_src},
@@ -502,8 +545,8 @@ def main(argv=None):
             "dense": dense, "speedup_vs_dense": dense_ms / ms_per_step, "modes": mode_vals,
             "kernels_us": {"k_select": 1e3 * sel_avg, "k_decode": 1e3 * dec_avg,
                            "separate_sum": 1e3 * (sel_avg + dec_avg), "step_overlapped": 1e3 * ms_per_step},
-            "append": append,
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps, "clocks": clk,
+            "append": append, "prefill": prefill,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (3 if clt else 2) * args.steps, "clocks": clk,
         }
         print(json.dumps(line))
     barrier()

@@ -491,6 +491,10 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
     }
     float ks[2] = {0.f, 0.f};      // SUMS: this thread's column pair of K (c < D/2) or V (c >= D/2)
     for (int i = tile0; i < tile1; ++i) {
+        // the tile range was sized by the draw capacity: once the list length
+        // is known, the tiles past it hold only masked rows (the copies of
+        // the next two are drained after the loop)
+        if (sel_ready && i * kTcTile >= n_tok) break;     // uniform
         // stage (i+2)%3 was last read by tile i-1, finished before the
         // trailing barrier of the previous iteration
         put_pos(i + 2);

@@ -89,7 +89,8 @@ inline PrefillPlan prefill_plan(const Dims& d) {
 struct SelectPlan {
     SetGeom g;
     int nss, rows_s;             // scan splits per unit, candidate rows per split
-    size_t off_scores, off_scores_up, off_xkey, off_cnt, bytes;
+    int nsc, clt_chunk, clt_rec; // CLT budget: splits per unit, I tokens per split, doubles per record
+    size_t off_scores, off_scores_up, off_xkey, off_cnt, off_clt, bytes;
 };
 
 inline SelectPlan select_plan(const Dims& d, const sa_select_params& sp) {
@@ -102,10 +103,22 @@ inline SelectPlan select_plan(const Dims& d, const sa_select_params& sp) {
     p.rows_s = cdiv(nc, p.nss);
     p.nss = cdiv(nc, p.rows_s);
     size_t off = 0;
-    p.off_cnt = off;    off = align256(off + sizeof(unsigned) * (size_t)d.U());
+    // completion tickets: the selection's [0, U), the CLT budget's [U, 2U)
+    p.off_cnt = off;    off = align256(off + sizeof(unsigned) * 2 * (size_t)d.U());
     p.off_scores = off; off = align256(off + sizeof(float) * (size_t)d.U() * nc);
     p.off_scores_up = off; off = align256(off + sizeof(float) * (size_t)d.U() * nc);
     p.off_xkey = off;   off = align256(off + sizeof(unsigned long long) * (size_t)d.U() * nc);
+    // CLT budget (clt_base > 0): the read set split over about one wave of
+    // CTAs, >= 128 tokens per split; one record per split (m, S, N per head)
+    p.nsc = 0; p.clt_chunk = 0; p.clt_rec = 0; p.off_clt = off;
+    if (sp.clt_base > 0) {
+        const int ni = p.g.n_i > 0 ? p.g.n_i : 1;
+        p.nsc = clampi(kSmTarget / d.U(), 1, cdiv(ni, 128));
+        p.clt_chunk = cdiv(ni, p.nsc);
+        p.nsc = cdiv(ni, p.clt_chunk);
+        p.clt_rec = 2 * d.G + d.G * d.d;
+        off = align256(off + sizeof(double) * (size_t)d.U() * p.nsc * p.clt_rec);
+    }
     p.bytes = off;
     return p;
 }

@@ -59,9 +59,9 @@ sa_status sa_select_noalloc(const sa_shape* shape, const sa_select_params* param
     void* ws = nullptr;
     sa_status e = scratch_for_current_device(&ws);
     if (e != SA_OK) return e;
-    // the selection's completion counters (one per unit, at offset 0 of its
+    // the completion counters (two per unit: selection and CLT budget, at offset 0 of its
     // workspace) must start at zero; the array may hold a previous call's data
-    const size_t counters = sa::align256(sizeof(unsigned) * (size_t)shape->B * (size_t)shape->Hkv);
+    const size_t counters = sa::align256(sizeof(unsigned) * 2 * (size_t)shape->B * (size_t)shape->Hkv);
     if (cudaMemsetAsync(ws, 0, counters, static_cast<cudaStream_t>(stream)) != cudaSuccess) return SA_ERR_CUDA;
     return sa_select(shape, params, q, stats, k, v, out, scale, ws, kNoAllocScratchBytes, stream);
 }

@@ -1,12 +1,22 @@
-// Per-step selection kernel: one CTA of 256 threads per unit, or several
-// when there are too few units to fill the GPU (see select_unit).
+// Per-step selection: one CTA of 256 threads per unit when the unit's
+// candidate keys fit its shared memory and there are enough units to fill
+// the GPU (k_select runs the whole selection); otherwise the units are split
+// over several scanning CTAs (k_select in its scan phase, bounds into the
+// workspace) and a second kernel, k_select_finish, one 512-thread CTA per
+// unit with up to 16K keys in shared memory, gathers the bounds and runs the
+// top-k, the exact band and the draws (select_unit in its finish phase).  The
+// finish kernel is a programmatic dependent of the scan.
 #include "sa_select_core.cuh"
 
 namespace sa {
 
 constexpr int kSelStages = 4;      // 4 x 18 KB ring at d = 128: two CTAs per SM
+constexpr int kFinThreads = 512;
+constexpr int kFinishKeys = 16384; // keys of one unit in the finish kernel's shared memory
+constexpr int kFinCand = 1024;     // top-k candidates ranked in shared memory
+constexpr int kFinAlias = 24576;   // bytes for the top-k / band arrays (select_unit's ring aliases)
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, int PHASE>
 __global__ void __launch_bounds__(kThreads, 2)
 k_select(SelectIo io) {
     using Ring = SketchRing<D, kWarps, kSelStages>;
@@ -26,7 +36,33 @@ k_select(SelectIo io) {
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
     const SelectSmem sm{hist, sw, misc, s_qh, s_qi, s_qc, s_ukeys, s_lkeys, s_sorted, s_ring,
                         reinterpret_cast<uint64_t*>(s_ring + Ring::kRingBytes), nullptr, 0};
-    (void)select_unit<T, D, G, kThreads, kSelStages>(io, sm, blockIdx.y, blockIdx.x);
+    (void)select_unit<T, D, G, kThreads, kSelStages, PHASE>(io, sm, blockIdx.y, blockIdx.x);
+}
+
+// The finish of split units; dynamic shared memory: the alias area
+// (kFinAlias bytes), then upper- and lower-bound keys (n_cand each, when
+// n_cand <= kFinishKeys).
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kFinThreads, 1)
+k_select_finish(SelectIo io) {
+    constexpr int NW = kFinThreads / 32;
+    __shared__ __align__(16) unsigned hist[256];
+    __shared__ int sw[NW + 1];
+    __shared__ int misc[3];
+    __shared__ float s_qh[G * D];
+    __shared__ __align__(16) int8_t s_qi[2 * D];
+    __shared__ float s_qc[3];
+    __shared__ int s_sorted[kWarpTopK];
+    __shared__ uint64_t s_bar[kSelStages];
+    extern __shared__ __align__(128) unsigned char s_fin[];
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+    // the scan kernel's bounds are complete and visible after this
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    const int nk = io.sg.n_cand <= kFinishKeys ? io.sg.n_cand : 0;
+    uint32_t* ukeys = reinterpret_cast<uint32_t*>(s_fin + kFinAlias);
+    const SelectSmem sm{hist, sw, misc, s_qh, s_qi, s_qc, ukeys, ukeys + nk, s_sorted, s_fin, s_bar, nullptr, 0};
+    (void)select_unit<T, D, G, kFinThreads, kSelStages, kPhFinish, kFinishKeys, kFinCand, true>(io, sm,
+                                                                                                blockIdx.x, 0);
 }
 
 SelectIo select_io(const Dims& d, const SelectPlan& p, const SelectArgs& a) {
@@ -59,11 +95,35 @@ SelectIo select_io(const Dims& d, const SelectPlan& p, const SelectArgs& a) {
 template <typename T, int D, int G>
 static cudaError_t select_t(const Dims& d, const SelectPlan& p, const SelectArgs& a, cudaStream_t s) {
     constexpr size_t smem = SketchRing<D, kWarps, kSelStages>::kSmem;
-    static std::atomic<unsigned long long> opted{0};
-    cudaError_t e = opt_in_smem(k_select<T, D, G>, smem, opted);
+    const SelectIo io = select_io(d, p, a);
+    if (p.nss == 1 && p.g.n_cand <= kSmemKeys) {
+        static std::atomic<unsigned long long> opted{0};
+        cudaError_t e = opt_in_smem(k_select<T, D, G, kPhAll>, smem, opted);
+        if (e != cudaSuccess) return e;
+        k_select<T, D, G, kPhAll><<<dim3(p.nss, d.U()), kThreads, smem, s>>>(io);
+        return cudaGetLastError();
+    }
+    static std::atomic<unsigned long long> opted_scan{0}, opted_fin{0};
+    cudaError_t e = opt_in_smem(k_select<T, D, G, kPhScan>, smem, opted_scan);
     if (e != cudaSuccess) return e;
-    k_select<T, D, G><<<dim3(p.nss, d.U()), kThreads, smem, s>>>(select_io(d, p, a));
-    return cudaGetLastError();
+    k_select<T, D, G, kPhScan><<<dim3(p.nss, d.U()), kThreads, smem, s>>>(io);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    constexpr size_t fin_max = (size_t)kFinAlias + (size_t)kFinishKeys * 8;
+    e = opt_in_smem(k_select_finish<T, D, G>, fin_max, opted_fin);
+    if (e != cudaSuccess) return e;
+    const int nk = p.g.n_cand <= kFinishKeys ? p.g.n_cand : 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(d.U());
+    cfg.blockDim = dim3(kFinThreads);
+    cfg.dynamicSmemBytes = (size_t)kFinAlias + (size_t)nk * 8;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_select_finish<T, D, G>, io);
 }
 
 template <typename T, int D>

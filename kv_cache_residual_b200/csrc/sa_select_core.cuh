@@ -213,16 +213,16 @@ __device__ void emit_topk(KeyFn key, int n, KT thr, int need, int kk, int c_lo, 
     }
 }
 
-// Top kk (kk <= 32, n <= kSmemKeys) of keys[0..n) by argmax rounds: every warp
+// Top kk (kk <= 32, n <= KEYS) of keys[0..n) by argmax rounds: every warp
 // holds a contiguous span in registers and extracts its best kk one at a time
 // (lane max, then warp max over 64-bit (key, ~index) words); warp 0 then
 // merges the per-warp lists the same way.  s_list[0..kk) gets the result in
 // rank order.  s_cand holds NT/32 * kk words.
-template <int NT>
+template <int NT, int KEYS = kSmemKeys>
 __device__ void warp_topk(const uint32_t* keys, int n, int kk, unsigned long long* s_cand,
                           unsigned long long* s_list) {
     constexpr int NW = NT / 32;
-    constexpr int C = kSmemKeys / NT;                  // keys per lane
+    constexpr int C = KEYS / NT;                       // keys per lane (n <= KEYS)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int span = (n + NW - 1) / NW;
     const int w0 = warp * span;
@@ -273,29 +273,40 @@ constexpr int kCandCap = 256;
 // at or above it, and so does B = max_w B_w, so thr >= B.  The candidates
 // are the keys whose upper bound reaches B: they contain the top kk by lower
 // bound and the whole band, and are usually few; they are compacted (each
-// thread's matches at its place in a block scan) into s_c / s_u (up to
-// kCandCap), ranked exactly, and the band is read off them.  Returns false,
-// having written nothing, when more than kCandCap keys reach B.  *s_b must
-// be zero on entry and visible to every thread; sw holds NT/32 ints.
-template <int NT>
+// thread's matches at its place in a block scan) into s_c / s_u (up to CC),
+// ranked exactly, and the band is read off them (its first kBandCap members
+// listed, all counted).  Returns false, having written nothing, when more
+// than CC keys reach B.  *s_b must be zero on entry and visible to every
+// thread; sw holds NT/32 ints.  BLOCKB: B is instead the kk-th largest of all
+// NT maxima (a bitwise search with block-wide counts, 32 barriers), a tighter
+// bound when kk is large against the 32 maxima of one warp.
+template <int NT, int KEYS = kSmemKeys, int CC = kCandCap, bool BLOCKB = false>
 __device__ bool topk_band(const uint32_t* lk, const uint32_t* uk, int n, int kk, unsigned long long* s_list,
                           unsigned long long* s_c, uint32_t* s_u, int* sw, unsigned* s_b, int* s_bidx,
                           int* s_band) {
     constexpr int NW = NT / 32;
-    static_assert(kSmemKeys <= 32 * NT, "one mask bit per owned key");
+    static_assert(KEYS <= 32 * NT, "one mask bit per owned key");
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t gm = 0u;
 #pragma unroll 4
     for (int i = threadIdx.x; i < n; i += NT) gm = max(gm, lk[i]);
-    uint32_t bw = 0u;
+    uint32_t bnd = 0u;
+    if constexpr (BLOCKB) {
+        for (int bit = 31; bit >= 0; --bit) {
+            const uint32_t cand = bnd | (1u << bit);
+            if (__syncthreads_count(gm >= cand) >= kk) bnd = cand;
+        }
+    } else {
+        uint32_t bw = 0u;
 #pragma unroll 8
-    for (int bit = 31; bit >= 16; --bit) {
-        const uint32_t cand = bw | (1u << bit);
-        if (__popc(__ballot_sync(0xffffffffu, gm >= cand)) >= kk) bw = cand;
+        for (int bit = 31; bit >= 16; --bit) {
+            const uint32_t cand = bw | (1u << bit);
+            if (__popc(__ballot_sync(0xffffffffu, gm >= cand)) >= kk) bw = cand;
+        }
+        if (lane == 0) atomicMax(s_b, bw);
+        __syncthreads();
+        bnd = *s_b;
     }
-    if (lane == 0) atomicMax(s_b, bw);
-    __syncthreads();
-    const uint32_t bnd = *s_b;
     // this thread's keys whose upper bound reaches B, as a bit mask
     unsigned mine = 0u;
 #pragma unroll 4
@@ -316,7 +327,7 @@ __device__ bool topk_band(const uint32_t* lk, const uint32_t* uk, int n, int kk,
         off += w < warp ? x : 0;
         nc += x;
     }
-    if (nc > kCandCap) return false;                 // (uniform: every thread summed the same counts)
+    if (nc > CC) return false;                       // (uniform: every thread summed the same counts)
     while (mine != 0u) {
         const int j = __ffs(mine) - 1;
         mine &= mine - 1u;
@@ -341,7 +352,8 @@ __device__ bool topk_band(const uint32_t* lk, const uint32_t* uk, int n, int kk,
             const int j = j0 + lane;
             const bool in = j < nc && s_u[j] >= thr;
             const unsigned m = __ballot_sync(0xffffffffu, in);
-            if (in) s_bidx[base + __popc(m & ((1u << lane) - 1u))] = comp_index(s_c[j]);
+            const int pos = base + __popc(m & ((1u << lane) - 1u));
+            if (in && pos < kBandCap) s_bidx[pos] = comp_index(s_c[j]);
             base += __popc(m);
         }
         if (lane == 0) *s_band = base;
@@ -505,6 +517,12 @@ struct SelectSmem {
 // The kernel arguments of a selection call (workspace carved by its plan).
 SelectIo select_io(const Dims& d, const SelectPlan& p, const SelectArgs& a);
 
+// Which part of a unit's selection a call runs: everything (one CTA, or the
+// split CTAs of a unit with the last one finishing), only the scan of this
+// CTA's slice into the workspace bounds (a split unit whose finish runs in a
+// kernel of its own), or only that finish (keys gathered from the workspace).
+enum SelPhase { kPhAll = 0, kPhScan = 1, kPhFinish = 2 };
+
 // done: this CTA finished the unit (false for a split CTA that was not the
 // unit's last, or after an abandoned wait); sorted_smem: the chosen blocks
 // (ascending) are in SelectSmem::sorted as well; bdraw: draws written.
@@ -514,7 +532,10 @@ struct SelectOutcome {
     int bdraw;
 };
 
-template <typename T, int D, int G, int NT, int STAGES>
+// KEYS: capacity of SelectSmem::ukeys / lkeys (a unit's keys stay in shared
+// memory when n_cand <= KEYS, else in place in the workspace).
+template <typename T, int D, int G, int NT, int STAGES, int PHASE = kPhAll, int KEYS = kSmemKeys,
+          int CC = kCandCap, bool BLOCKB = false>
 __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const SelectSmem& sm, int u, int split) {
     constexpr int NW = NT / 32;
     using Ring = SketchRing<D, NW, STAGES>;
@@ -547,13 +568,13 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
     int* s_sorted = sm.sorted;
     unsigned char* s_ring = sm.ring;
     uint64_t* s_bar = sm.bar;
-    constexpr int kCandWords = NW * kWarpTopK > kCandCap ? NW * kWarpTopK : kCandCap;
+    constexpr int kCandWords = NW * kWarpTopK > CC ? NW * kWarpTopK : CC;
     unsigned long long* s_cand = reinterpret_cast<unsigned long long*>(s_ring);          // kCandWords
     unsigned long long* s_list = s_cand + kCandWords;                                    // kWarpTopK
     double* s_bx = reinterpret_cast<double*>(s_list + kWarpTopK);                        // kBandCap
     int* s_bidx = reinterpret_cast<int*>(s_bx + kBandCap);                               // kBandCap
     unsigned char* s_bsel = reinterpret_cast<unsigned char*>(s_bidx + kBandCap);         // kBandCap
-    uint32_t* s_u = reinterpret_cast<uint32_t*>(s_bsel + kBandCap);                      // kCandCap
+    uint32_t* s_u = reinterpret_cast<uint32_t*>(s_bsel + kBandCap);                      // CC
 
     const int b = u / Hkv, g = u - b * Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -564,7 +585,7 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
     float* sc_lo = io.sc_lo_all + (size_t)u * (n > 0 ? n : 1);
     float* sc_up = io.sc_up_all + (size_t)u * (n > 0 ? n : 1);
     // one CTA per unit: the keys never leave shared memory
-    const bool local = (nss == 1) && n <= kSmemKeys;
+    const bool local = PHASE == kPhAll && (nss == 1) && n <= KEYS;
     SelectOutcome res{false, false, 0};
 
     // ---- scan: score intervals of this CTA's slice ------------------------------
@@ -573,7 +594,7 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
     // kStages stages in flight; all warps score each stage as it lands.
     const int r0 = split * rows, r1 = min(n, r0 + rows);
     const int nrows = max(0, r1 - r0);
-    const int nst = (nrows + Ring::SR - 1) / Ring::SR;
+    const int nst = PHASE == kPhFinish ? 0 : (nrows + Ring::SR - 1) / Ring::SR;
     const size_t row0 = (size_t)u * nb + sg.c_lo + r0;
     const int8_t* code0 = blk_code + row0 * D;
     const float4* meta0 = blk_meta + row0;
@@ -754,6 +775,12 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
             }
         }
     }
+    if (PHASE == kPhScan) {
+        // the finish kernel learns of an abandoned wait from the unit's
+        // (otherwise unused) selection ticket
+        if (failed && threadIdx.x == 0) atomicAdd(cnt + u, 1u);
+        return res;
+    }
     if (failed) {
         int32_t* out_idx = blk_idx + (size_t)u * kb_stride;
         for (int i = threadIdx.x; i < kb_stride; i += NT) out_idx[i] = -1;
@@ -777,11 +804,26 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
     if (local) {
         __syncthreads();
     } else {
-        if (!last_cta_of_unit(cnt + u, nss)) return res;
+        if (PHASE == kPhAll && !last_cta_of_unit(cnt + u, nss)) return res;
+        if (PHASE == kPhFinish) {
+            __shared__ unsigned s_bad;
+            if (threadIdx.x == 0) s_bad = __ldcg(cnt + u);
+            __syncthreads();
+            if (s_bad != 0u) {               // a scan CTA of the unit gave up a wait
+                int32_t* out_idx = blk_idx + (size_t)u * kb_stride;
+                for (int i = threadIdx.x; i < kb_stride; i += NT) out_idx[i] = -1;
+                if (threadIdx.x == 0) {
+                    samp_count[u] = 0;
+                    if (n_rescored != nullptr) n_rescored[u] = -1;
+                    cnt[u] = 0u;
+                }
+                return res;
+            }
+        }
         // orderable keys, staged once: shared memory when they fit, else in
         // place over the unit's bounds in the workspace (each thread rewrites
         // only the entries it read)
-        if (n > kSmemKeys) {
+        if (n > KEYS) {
             lk = reinterpret_cast<uint32_t*>(sc_lo);
             uk = reinterpret_cast<uint32_t*>(sc_up);
         }
@@ -812,14 +854,15 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
     if (kk > 0 && kk < n) {
         if (threadIdx.x == 0) s_nb = 0;        // band counter (barriers follow on every path)
         auto k32 = [&](int i) -> uint32_t { return lk[i]; };
-        const bool fast = kk <= kWarpTopK && n <= kSmemKeys;
+        const bool fast = kk <= kWarpTopK && n <= KEYS;
         uint32_t thr;
         int need = 0;
         bool listed = false;            // band already listed (group path)
         if (fast) {
-            listed = topk_band<NT>(lk, uk, n, kk, s_list, s_cand, s_u, sw, reinterpret_cast<unsigned*>(&s_rem),
+            listed = topk_band<NT, KEYS, CC, BLOCKB>(lk, uk, n, kk, s_list, s_cand, s_u, sw,
+                                                     reinterpret_cast<unsigned*>(&s_rem),
                                    s_bidx, &s_nb);
-            if (!listed) warp_topk<NT>(lk, n, kk, s_cand, s_list);
+            if (!listed) warp_topk<NT, KEYS>(lk, n, kk, s_cand, s_list);
             thr = (uint32_t)(s_list[kk - 1] >> 32);
         } else {
             radix_select<NT, uint32_t>(k32, n, kk, &thr, &need, hist, &s_digit, &s_rem);
