@@ -98,17 +98,20 @@ def set_geom(L, sink, local, k_blocks):
     return {"n_cand": n_cand, "kk": kk, "n_i": n_i, "n_t": L - n_i}
 
 
+# the sources k_select is compiled from (its translation unit and headers)
+SELECT_SOURCES = ("kv_cache_residual_b200/csrc/sa_select.cu", "kv_cache_residual_b200/csrc/sa_select_core.cuh",
+                  "kv_cache_residual_b200/csrc/sa_bulk.cuh", "kv_cache_residual_b200/csrc/sa_common.cuh",
+                  "kv_cache_residual_b200/csrc/sa_internal.h", "include/sa_decode.h")
+
+
 def sources_sha1():
-    """sha1 over the CUDA sources (name + bytes), to tell whether an ncu
-    capture still describes the kernels being run."""
-    import glob
+    """sha1 over the sources of the selection kernel (name + bytes), to tell
+    whether an ncu capture of it still describes the kernel being run."""
     import hashlib
     h = hashlib.sha1()
-    d = os.path.join(ROOT, "kv_cache_residual_b200", "csrc")
-    for f in sorted(glob.glob(os.path.join(d, "*.cu")) + glob.glob(os.path.join(d, "*.cuh")) +
-                    glob.glob(os.path.join(d, "*.h"))):
+    for f in SELECT_SOURCES:
         h.update(os.path.basename(f).encode())
-        h.update(open(f, "rb").read())
+        h.update(open(os.path.join(ROOT, f), "rb").read())
     return h.hexdigest()
 
 
