@@ -14,7 +14,7 @@ constexpr int kSelStages = 4;      // 4 x 18 KB ring at d = 128: two CTAs per SM
 constexpr int kFinThreads = 512;
 constexpr int kFinishKeys = 16384; // keys of one unit in the finish kernel's shared memory
 constexpr int kFinCand = 1024;     // top-k candidates ranked in shared memory
-constexpr int kFinAlias = 24576;   // bytes for the top-k / band arrays (select_unit's ring aliases)
+constexpr int kFinAlias = 32768;   // bytes for the top-k / band arrays (select_unit's ring aliases)
 
 template <typename T, int D, int G, int PHASE>
 __global__ void __launch_bounds__(kThreads, 2)

@@ -265,7 +265,7 @@ __device__ void warp_topk(const uint32_t* keys, int n, int kk, unsigned long lon
 
 constexpr int kCandCap = 256;
 
-// Top kk (kk <= 32, kk < n) of the n lower-bound keys lk[] in shared memory by
+// Top kk (kk <= 32, or <= CC with BLOCKB; kk < n) of the n lower-bound keys lk[] in shared memory by
 // (key desc, index asc), in rank order into s_list, and the band {upper >=
 // thr} (thr = the kk-th lower key) into s_bidx / *s_band.  Thread t owns the
 // keys t, t + NT, ... (n <= 32 NT) and takes their maximum; in each warp a
@@ -278,8 +278,9 @@ constexpr int kCandCap = 256;
 // listed, all counted).  Returns false, having written nothing, when more
 // than CC keys reach B.  *s_b must be zero on entry and visible to every
 // thread; sw holds NT/32 ints.  BLOCKB: B is instead the kk-th largest of all
-// NT maxima (a bitwise search with block-wide counts, 32 barriers), a tighter
-// bound when kk is large against the 32 maxima of one warp.
+// NT maxima to 16 bits (a bitwise search with block-wide counts, 16
+// barriers), a tighter bound when kk is large against the 32 maxima of one
+// warp; kk may then be up to CC (s_list holds kk entries).
 template <int NT, int KEYS = kSmemKeys, int CC = kCandCap, bool BLOCKB = false>
 __device__ bool topk_band(const uint32_t* lk, const uint32_t* uk, int n, int kk, unsigned long long* s_list,
                           unsigned long long* s_c, uint32_t* s_u, int* sw, unsigned* s_b, int* s_bidx,
@@ -292,7 +293,7 @@ __device__ bool topk_band(const uint32_t* lk, const uint32_t* uk, int n, int kk,
     for (int i = threadIdx.x; i < n; i += NT) gm = max(gm, lk[i]);
     uint32_t bnd = 0u;
     if constexpr (BLOCKB) {
-        for (int bit = 31; bit >= 0; --bit) {
+        for (int bit = 31; bit >= 16; --bit) {
             const uint32_t cand = bnd | (1u << bit);
             if (__syncthreads_count(gm >= cand) >= kk) bnd = cand;
         }
@@ -570,8 +571,9 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
     uint64_t* s_bar = sm.bar;
     constexpr int kCandWords = NW * kWarpTopK > CC ? NW * kWarpTopK : CC;
     unsigned long long* s_cand = reinterpret_cast<unsigned long long*>(s_ring);          // kCandWords
-    unsigned long long* s_list = s_cand + kCandWords;                                    // kWarpTopK
-    double* s_bx = reinterpret_cast<double*>(s_list + kWarpTopK);                        // kBandCap
+    constexpr int LISTN = BLOCKB ? (CC > kWarpTopK ? CC : kWarpTopK) : kWarpTopK;
+    unsigned long long* s_list = s_cand + kCandWords;                                    // LISTN
+    double* s_bx = reinterpret_cast<double*>(s_list + LISTN);                            // kBandCap
     int* s_bidx = reinterpret_cast<int*>(s_bx + kBandCap);                               // kBandCap
     unsigned char* s_bsel = reinterpret_cast<unsigned char*>(s_bidx + kBandCap);         // kBandCap
     uint32_t* s_u = reinterpret_cast<uint32_t*>(s_bsel + kBandCap);                      // CC
@@ -854,16 +856,33 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
     if (kk > 0 && kk < n) {
         if (threadIdx.x == 0) s_nb = 0;        // band counter (barriers follow on every path)
         auto k32 = [&](int i) -> uint32_t { return lk[i]; };
-        const bool fast = kk <= kWarpTopK && n <= KEYS;
-        uint32_t thr;
+        // the ranked list s_list[0..kk) comes from the group top-k (kk up to
+        // LISTN) or, for kk <= 32 when it has too many candidates, from the
+        // per-warp lists; otherwise a radix select finds thr
+        const bool grp = kk <= LISTN && n <= KEYS;
+        uint32_t thr = 0u;
         int need = 0;
         bool listed = false;            // band already listed (group path)
-        if (fast) {
+        bool have_list = false;         // s_list[0..kk) holds the top kk in rank order
+        if (grp) {
             listed = topk_band<NT, KEYS, CC, BLOCKB>(lk, uk, n, kk, s_list, s_cand, s_u, sw,
                                                      reinterpret_cast<unsigned*>(&s_rem),
                                    s_bidx, &s_nb);
-            if (!listed) warp_topk<NT, KEYS>(lk, n, kk, s_cand, s_list);
+            have_list = listed;
+            if (!listed && kk <= kWarpTopK) {
+                warp_topk<NT, KEYS>(lk, n, kk, s_cand, s_list);
+                have_list = true;
+            }
+        }
+        if (have_list) {
             thr = (uint32_t)(s_list[kk - 1] >> 32);
+            if (kk > kWarpTopK) {
+                // the top kk's keys equal to thr are the lowest-index ones
+                // among all keys equal to thr: emit_topk takes that many
+                int c = 0;
+                for (int r = threadIdx.x; r < kk; r += NT) c += ((uint32_t)(s_list[r] >> 32) == thr) ? 1 : 0;
+                need = block_sum<NT>(c, sw);
+            }
         } else {
             radix_select<NT, uint32_t>(k32, n, kk, &thr, &need, hist, &s_digit, &s_rem);
         }
@@ -891,7 +910,7 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
         __syncthreads();
         const int band = s_nb;
         if (band == kk) {
-            if (fast) {
+            if (have_list && kk <= kWarpTopK) {
                 emit_sorted_list(s_list, kk, sg.c_lo, out_idx, s_sorted);
                 sorted_smem = true;
             }
@@ -923,6 +942,15 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
                 }
                 sorted_smem = true;
             } else if (band <= kBandCap) {
+                // several rounds of members: their rows into L2 first
+                if (band > 2 * NW) {
+                    for (int j = threadIdx.x; j < band; j += NT) {
+                        const char* r = reinterpret_cast<const char*>(bm + (size_t)s_bidx[j] * D);
+#pragma unroll
+                        for (int o = 0; o < (int)(D * sizeof(T)); o += 128)
+                            asm volatile("prefetch.global.L2 [%0];" ::"l"(r + o));
+                    }
+                }
                 rescore_members<T, D, G, NW>(bm, s_bidx, band, s_qh, s_bx);
                 __syncthreads();
                 for (int j = threadIdx.x; j < band; j += NT) {
