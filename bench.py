@@ -17,7 +17,7 @@ the device time of the step, not the host's launch latency (which the e2e
 figure, timed through the public API with host buffers, does include).
 Prints ONE JSON line on rank 0.
 
---impl reference times the fp64 CPU oracle (the reference arm of this build)
+--impl reference times the fp64 CPU oracle (the reference arm)
 on a bounded sample of the same workload, on the host cores.
 """
 import argparse

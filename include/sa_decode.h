@@ -68,7 +68,7 @@ extern "C" {
 typedef enum {
     SA_OK = 0,
     SA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer   */
-    SA_ERR_UNSUPPORTED = 2,  /* a valid request this build does not handle   */
+    SA_ERR_UNSUPPORTED = 2,  /* a valid request this library does not handle */
     SA_ERR_WORKSPACE = 3,    /* ws NULL or smaller than sa_workspace_size()  */
     SA_ERR_CUDA = 4          /* a kernel launch failed                      */
 } sa_status;
