@@ -115,3 +115,45 @@ def test_no_wait_gave_up():
     """No selection CTA in this process abandoned a bounded wait."""
     torch.cuda.synchronize()
     assert sa.wait_timeouts() == 0
+
+
+# (dtype, d, Hq, Hkv, B, L): few units, so each is split over scanning CTAs
+# and finished by the second kernel (keys of up to 16K candidates in shared
+# memory, group top-k up to 1024 blocks, radix select beyond)
+SPLIT_SHAPES = {
+    "bf16_d128_g4_64k": ("bf16", 128, 8, 2, 1, 65536),
+    "bf16_d128_g4_128k": ("bf16", 128, 8, 2, 1, 131072),
+    "f32_d64_g2_32k": ("f32", 64, 4, 2, 2, 32768),
+}
+
+
+@pytest.mark.parametrize("pattern", ["random", "ties", "near"])
+@pytest.mark.parametrize("name", list(SPLIT_SHAPES))
+def test_select_split_units(name, pattern):
+    dtype, d, Hq, Hkv, B, L = SPLIT_SHAPES[name]
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    G = Hq // Hkv
+    dev = torch.device("cuda")
+    gen = torch.Generator().manual_seed(zlib.crc32(("split/%s/%s" % (name, pattern)).encode()))
+    q = torch.randn(B, Hq, d, generator=gen).to(dt)
+    nb = L // 16
+    bm = _summaries(pattern, B, Hkv, nb, d, dt, q.float(), G, gen)
+    st = sa.Stats(B, Hq, Hkv, L, d, dt, dev)
+    st.blk_mean.copy_(bm.to(dev))
+    st.mu_k.copy_(bm.float().mean(2).to(dev))
+    sa.block_sketch(st, Hq)
+    qd = q.to(dev)
+    n_cand = len(osel.candidate_blocks(L, SINK, LOCAL))
+    for k in (8, 33, 200, 1000, n_cand - 1):
+        sp = sa.SelectParams(sink=SINK, local=LOCAL, k_blocks=k, sample_b=48, sample_cap=48, seed=78, step=2)
+        sel = sa.select(qd, st, sp)
+        torch.cuda.synchronize()
+        blk = sel.blk_idx.cpu().numpy()
+        samp = sel.samp_idx.cpu().numpy()
+        for b in range(B):
+            for g in range(Hkv):
+                qq = f64(q[b, g * G:(g + 1) * G])
+                blocks, idx, tail = osel.select_unit(qq, f64(bm[b, g]), L, SINK, LOCAL, k)
+                np.testing.assert_array_equal(blk[b, g, :len(blocks)], blocks, err_msg=str((name, pattern, k, b, g)))
+                pos = orng.sample_positions(78, b, g, 2, tail, 48)
+                np.testing.assert_array_equal(samp[b, g], pos, err_msg=str((name, pattern, k, b, g)))
