@@ -68,8 +68,10 @@ k_qmean(const T* __restrict__ q_ctx, int L, int rows, int nsq, float* __restrict
     reset_counter(cnt + bh);
 }
 
+// two CTAs per SM (registers capped at 128): one CTA of 8 warps per SM left
+// the pass latency-bound at ~0.2 of the HBM peak
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 k_kvpass(const T* __restrict__ k, const T* __restrict__ v, const float* __restrict__ mu_q,
          int Hq, int Hkv, int L, int ld, int tok, int nskv, float qscale, int stride,
          float* __restrict__ part, unsigned* __restrict__ cnt, sa_stats st) {
@@ -114,7 +116,7 @@ k_kvpass(const T* __restrict__ k, const T* __restrict__ v, const float* __restri
         double bs[EPC];
 #pragma unroll
         for (int e = 0; e < EPC; ++e) bs[e] = 0.0;
-#pragma unroll 2
+#pragma unroll 1
         for (int j0 = 0; j0 < 16; j0 += 4) {
             uint4 wk[4], wv[4];
 #pragma unroll
