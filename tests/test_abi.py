@@ -165,3 +165,21 @@ def test_status_strings(lib):
     for s in range(5):
         assert lib.sa_status_string(s)
     assert lib.sa_status_string(99) == b"unknown status"
+
+
+def test_workspace_grows_with_the_clt_budget(lib):
+    """The CLT budget's per-split records live in the selection workspace:
+    asking for it enlarges the selection and step workspaces; sizes are
+    multiples of 256 bytes and do not depend on the cache capacity beyond L."""
+    plain = sa.SelectParams(sink=64, local=128, k_blocks=8, sample_b=0, sample_cap=4096).c()
+    clt = sa.SelectParams(sink=64, local=128, k_blocks=8, sample_b=0, sample_cap=4096, clt_base=64,
+                          eps=0.05, delta=0.05).c()
+    sh = _shape(B=8, L=32768)
+    for op in (sa.OP_SELECT, sa.OP_STEP):
+        a = lib.sa_workspace_size(ctypes.byref(sh), ctypes.byref(plain), op)
+        b = lib.sa_workspace_size(ctypes.byref(sh), ctypes.byref(clt), op)
+        assert a > 0 and b > a and a % 256 == 0 and b % 256 == 0
+    grown = _shape(B=8, L=32768, ld=32768 + 4096)
+    for op in (sa.OP_SELECT, sa.OP_DECODE, sa.OP_DENSE):
+        assert (lib.sa_workspace_size(ctypes.byref(sh), ctypes.byref(plain), op) ==
+                lib.sa_workspace_size(ctypes.byref(grown), ctypes.byref(plain), op))
