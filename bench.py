@@ -230,7 +230,7 @@ def cpu_oracle_sample(w, sp_kw, mode, seconds, max_units=None, seq=0):
     from threadpoolctl import threadpool_info
 
     import synth
-    from oracle import modes, rng, select, stats
+    from oracle import budget, modes, rng, select, stats
 
     s = synth.make_sequence(w, seq, device="cpu")
     qs = synth.make_queries(w, seq, 4, s["mu_q"], device="cpu")
@@ -249,7 +249,14 @@ def cpu_oracle_sample(w, sp_kw, mode, seconds, max_units=None, seq=0):
             q = qs[step, g * w.G:(g + 1) * w.G].double().numpy()
             blocks, idx, tail = select.select_unit(q, st["blk_mean"], w.L, sp_kw["sink"], sp_kw["local"],
                                                    sp_kw["k_blocks"])
-            pos = rng.sample_positions(sp_kw["seed"], seq, g, step, tail, sp_kw["sample_b"]) if mode == "sample" else None
+            pos = None
+            if mode == "sample" and sp_kw.get("clt_base", 0) > 0 and len(tail) > 0:
+                # the CLT budget from the base draws, then that many draws
+                base = rng.sample_positions(sp_kw["seed"], seq, g, step, tail, sp_kw["clt_base"])
+                b, _ = budget.clt_budget(q, K, V, idx, base, scale, sp_kw["eps"], sp_kw["delta"], len(tail))
+                pos = rng.sample_positions(sp_kw["seed"], seq, g, step, tail, min(b, sp_kw["sample_cap"]))
+            elif mode == "sample":
+                pos = rng.sample_positions(sp_kw["seed"], seq, g, step, tail, sp_kw["sample_b"])
             modes.run_mode(mode, q, K, V, idx, st, scale, pos=pos)
             done += 1
             if max_units is not None and done >= max_units:
@@ -301,6 +308,8 @@ def main(argv=None):
     kb = w.k_blocks_for(args.read) if w.k_blocks is None else w.k_blocks
     sg = set_geom(w.L, w.sink, w.local, kb)
     sp_kw = dict(sink=w.sink, local=w.local, k_blocks=kb, sample_b=args.sample_b, seed=2024)
+    if args.mode == "sample" and args.clt_base > 0:
+        sp_kw.update(clt_base=args.clt_base, eps=args.eps, delta=args.delta, sample_cap=args.sample_cap)
     ws, rank, local = dist_setup(args.gpus)
     if args.impl == "reference":
         rc = run_reference(args, w, sg, sp_kw, rank)
