@@ -1,8 +1,11 @@
-"""GPU parity of the selection when there are enough units to give each its
-own CTA (the scores stay on chip and every warp keeps its best k while it
-scans): chosen blocks and tail draws bit-exact against the oracle, for every
-dtype / d / G, k on both sides of the in-register list limit (32), exact
-ties, and score orders that make every row enter a warp's list."""
+"""GPU parity of the selection: chosen blocks and tail draws bit-exact
+against the oracle.  With enough units each gets its own CTA (the bounds stay
+on chip): every dtype / d / G, k on both sides of the group top-k's limit
+(32), exact ties, and score orders that stress the candidate bound.  With few
+units each is split over scanning CTAs and finished by a second kernel: 64K
+and 128K-token caches, k from 8 to n_cand - 1 (group top-k up to 1024 blocks,
+radix select beyond), ties and near-equal scores whose band exceeds the 512
+members ranked in shared memory."""
 import zlib
 
 import numpy as np
