@@ -222,11 +222,12 @@ def test_block_summaries_entry_point(dev):
     assert torch.equal(st.blk_code, code) and torch.equal(st.blk_meta, meta)
 
 
-@pytest.mark.parametrize("wname,units", [("llama", [(0, 0), (0, 3), (0, 7)]),
+@pytest.mark.parametrize("wname,units", [("llama", [(0, g) for g in range(8)]),
                                          ("batched", [(0, 0), (17, 5), (31, 7)])])
 def test_full_size_sampled_units(wname, units, dev):
     """Full workload sizes, in the launch configuration the benchmark uses;
-    outputs of sampled units checked against the oracle one by one."""
+    outputs checked against the oracle unit by unit: every unit of the
+    one-sequence 32K layer, sampled units of the 32-sequence batch."""
     w = synth.WORKLOADS[wname]
     data = synth.make_batch(w, device=dev, steps=2)
     st = sa.prefill_stats(data["q_ctx"], data["k"], data["v"])
