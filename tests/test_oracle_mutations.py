@@ -1,0 +1,164 @@
+"""The oracle's pins catch plausible mistakes: each test plants one mistake in
+an oracle function (on the CPU, by replacing it for the duration of the
+test) and checks that at least one of the pins written for that function
+fails.  A pin set that passed a planted mistake would not be pinning it."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle.modes as modes
+import oracle.numerics as numerics
+import oracle.select as select
+import oracle.stats as stats
+import test_oracle_modes as pin_modes
+import test_oracle_numerics as pin_num
+import test_oracle_select as pin_sel
+import test_oracle_stats as pin_stats
+
+
+def _some_pin_fails(pins):
+    """True when at least one of the (function, kwargs) pins raises an
+    AssertionError."""
+    for fn, kw in pins:
+        try:
+            fn(**kw)
+        except AssertionError:
+            return True
+    return False
+
+
+# ---- planted mistakes ---------------------------------------------------------
+
+def _resa_without_bias(q, k, v, idx, st, scale, lam=1.0, _orig=modes.resa):
+    # the bias c = s (q - mu_Q) . mu_K dropped (mu_K enters resa only there)
+    return _orig(q, k, v, idx, dict(st, mu_k=0.0 * st["mu_k"]), scale, lam)
+
+
+def _resa_lambda_on_alpha_only(q, k, v, idx, st, scale, lam=1.0):
+    # lambda applied to alpha alone, not to the prior mass inside Z'
+    n_t = k.shape[0] - len(idx)
+    if n_t == 0 or len(idx) == 0:
+        return modes.drop(q, k, v, idx, scale) if n_t == 0 else st["o_est"].copy()
+    kI, vI = k[idx], v[idx]
+    c = scale * ((q - st["mu_q"]) @ st["mu_k"])
+    l_i = scale * (q @ kI.T)
+    p_i = scale * (st["mu_q"] @ kI.T) + c[:, None]
+    log_z = st["log_z0"] + c
+    m = np.maximum(np.maximum(log_z, l_i.max(1)), p_i.max(1))[:, None]
+    z = np.exp(log_z[:, None] - m)
+    e_p, e_l = np.exp(p_i - m), np.exp(l_i - m)
+    z_new = np.maximum(z[:, 0] - e_p.sum(1), 0.0) + e_l.sum(1)
+    alpha = lam * z[:, 0] / z_new
+    return alpha[:, None] * st["o_est"] + (e_l / z_new[:, None] - alpha[:, None] * e_p / z) @ vI
+
+
+def _proxy_without_log_n(q, k, v, idx, st, scale):
+    n_t = k.shape[0] - len(idx)
+    if n_t == 0:
+        return modes.drop(q, k, v, idx, scale)
+    kbar = (st["sum_k"] - k[idx].sum(0)) / n_t
+    vbar = (st["sum_v"] - v[idx].sum(0)) / n_t
+    z = scale * (q @ kbar)                                        # + ln n_T missing
+    logits = np.concatenate([scale * (q @ k[idx].T), z[:, None]], axis=1)
+    return modes._softmax_weighted(logits, np.concatenate([v[idx], vbar[None]], axis=0))
+
+
+def _sample_without_weight(q, k, v, idx, pos, scale):
+    n_t = k.shape[0] - len(idx)
+    if n_t == 0 or len(pos) == 0:
+        return modes.drop(q, k, v, idx, scale)
+    logits = np.concatenate([scale * (q @ k[idx].T), scale * (q @ k[pos].T)], axis=1)  # no ln(n_T / b)
+    return modes._softmax_weighted(logits, np.concatenate([v[idx], v[pos]], axis=0))
+
+
+def _sample_num_den_without_weight(q, k, v, idx, pos, scale, shift):
+    e_i = np.exp(scale * (q @ k[idx].T) - shift[:, None])
+    e_s = np.exp(scale * (q @ k[pos].T) - shift[:, None])      # the n_T / b factor missing
+    return e_i @ v[idx] + e_s @ v[pos], e_i.sum(1) + e_s.sum(1)
+
+
+def _top_blocks_high_index_first(scores, cand, k):
+    k = min(int(k), len(cand))
+    order = np.lexsort((-cand, -scores))                          # ties to the HIGHER index
+    return np.sort(cand[order[:k]])
+
+
+def _round_to_bf16_7_bits(x):
+    x = np.asarray(x, dtype=np.float64)
+    out = np.zeros_like(x)
+    nz = x != 0
+    _, e = np.frexp(x[nz])
+    sp = np.maximum(e - 7, -133)                                  # one bit short
+    out[nz] = np.ldexp(np.rint(np.ldexp(x[nz], -sp)), sp)
+    return out
+
+
+def _block_means_over_15(k, kv_dtype):
+    L, d = k.shape
+    nb = L // 16
+    return numerics.round_to(k[: nb * 16].reshape(nb, 16, d).sum(axis=1) / 15.0, kv_dtype)
+
+
+# ---- the checks -----------------------------------------------------------------
+
+MODE_PINS = [
+    (pin_modes.test_full_budget_is_dense, {"mode": m}) for m in ("drop", "resa", "proxy", "sample")
+] + [
+    (pin_modes.test_resa_delta_merge_equals_merged_logit_softmax, {"lam": lam}) for lam in (1.0, 0.5)
+] + [
+    (pin_modes.test_resa_exact_when_keys_identical, {}),
+    (pin_modes.test_resa_lambda_zero_is_drop_and_empty_set_is_prior, {}),
+    (pin_modes.test_proxy_exact_for_one_token_tail, {}),
+    (pin_modes.test_proxy_exact_for_identical_tail_keys_and_values, {}),
+    (pin_modes.test_proxy_tail_means_from_totals_equal_direct_means, {}),
+    (pin_modes.test_sample_exact_for_identical_tail_tokens, {}),
+    (pin_modes.test_sample_estimator_unbiased_over_seeds, {}),
+]
+
+
+@pytest.mark.parametrize("name,attr,mutant", [
+    ("dropped RESA bias", "resa", _resa_without_bias),
+    ("lambda on alpha only", "resa", _resa_lambda_on_alpha_only),
+    ("proxy without + ln n_T", "proxy", _proxy_without_log_n),
+    ("sample without n_T / b", "sample", _sample_without_weight),
+    ("estimator without n_T / b", "sample_num_den", _sample_num_den_without_weight),
+])
+def test_mode_mistakes_fail_a_pin(name, attr, mutant, monkeypatch):
+    monkeypatch.setattr(modes, attr, mutant)
+    assert _some_pin_fails(MODE_PINS), name
+
+
+def test_reversed_tie_break_fails_a_pin(monkeypatch):
+    monkeypatch.setattr(select, "top_blocks", _top_blocks_high_index_first)
+    pins = [(pin_sel.test_all_equal_scores_take_lowest_indices, {}),
+            (pin_sel.test_identical_summaries_tie_anywhere, {}),
+            (pin_sel.test_permuted_summaries_tie_under_a_constant_query, {})]
+    pins += [(pin_sel.test_top_blocks_brute_force, {"seed": s}) for s in range(3)]
+    assert _some_pin_fails(pins)
+
+
+def test_wrong_bf16_spacing_fails_a_pin(monkeypatch):
+    monkeypatch.setattr(numerics, "round_to_bf16", _round_to_bf16_7_bits)
+    monkeypatch.setattr(pin_num, "round_to_bf16", _round_to_bf16_7_bits)
+    pins = [(pin_num.test_bf16_matches_torch_cast_on_fp32_values, {}),
+            (pin_num.test_bf16_ties_and_single_rounding, {})]
+    assert _some_pin_fails(pins)
+
+
+def test_wrong_block_mean_divisor_fails_a_pin(monkeypatch):
+    monkeypatch.setattr(stats, "block_means", _block_means_over_15)
+    monkeypatch.setattr(pin_stats, "block_means", _block_means_over_15)
+    pins = [(pin_stats.test_block_means_against_torch_cast, {}),
+            (pin_stats.test_constant_keys_closed_form, {})]
+    assert _some_pin_fails(pins)
+
+
+def test_unmutated_oracle_passes_every_pin_used_here():
+    """The same pins pass on the oracle as written (so the checks above fail
+    because of the planted mistakes, not on their own)."""
+    pins = MODE_PINS + [(pin_sel.test_all_equal_scores_take_lowest_indices, {}),
+                        (pin_num.test_bf16_ties_and_single_rounding, {}),
+                        (pin_stats.test_block_means_against_torch_cast, {})]
+    for fn, kw in pins:
+        fn(**kw)
