@@ -162,3 +162,44 @@ def test_unmutated_oracle_passes_every_pin_used_here():
                         (pin_stats.test_block_means_against_torch_cast, {})]
     for fn, kw in pins:
         fn(**kw)
+
+
+def _mix64_wrong_shift(z, _M=(1 << 64) - 1):
+    z &= _M
+    z = ((z ^ (z >> 31)) * 0xBF58476D1CE4E5B9) & _M               # 30 -> 31
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & _M
+    return z ^ (z >> 31)
+
+
+def _z_one_sided(delta):
+    from scipy.stats import norm
+    return float(norm.ppf(1.0 - delta))                           # one-sided quantile
+
+
+def _grown_stats_prefix_prior(st0, k, v, scale, kv_dtype, _orig=stats.grown_stats):
+    # O_Est and log_z0 left at their prefill-end values (appended tokens ignored)
+    g = _orig(st0, k, v, scale, kv_dtype)
+    return dict(g, o_est=st0["o_est"], log_z0=st0["log_z0"])
+
+
+def test_rng_mixer_mistake_fails_a_pin(monkeypatch, golden_dir):
+    import oracle.rng as rng
+    import test_oracle_rng as pin_rng
+    monkeypatch.setattr(rng, "mix64", _mix64_wrong_shift)
+    assert _some_pin_fails([(pin_rng.test_splitmix64_reference_outputs, {"golden_dir": golden_dir}),
+                            (pin_rng.test_mixer_is_a_bijection_on_samples, {})])
+
+
+def test_budget_quantile_mistake_fails_a_pin(monkeypatch, golden_dir):
+    import oracle.budget as budget
+    import test_oracle_budget as pin_budget
+    monkeypatch.setattr(budget, "z_two_sided", _z_one_sided)
+    assert _some_pin_fails([(pin_budget.test_lemma_worked_example, {"golden_dir": golden_dir}),
+                            (pin_budget.test_quantile_textbook_values, {})])
+
+
+def test_grown_prior_mistake_fails_a_pin(monkeypatch):
+    monkeypatch.setattr(stats, "grown_stats", _grown_stats_prefix_prior)
+    monkeypatch.setattr(pin_stats, "grown_stats", _grown_stats_prefix_prior)
+    assert _some_pin_fails([(pin_stats.test_grown_stats_follow_the_token_recurrence, {}),
+                            (pin_stats.test_grown_stats_constant_keys_closed_form, {})])
