@@ -20,8 +20,11 @@ budget per KV head = the max over its query heads; b is clamped to
 [b0, n_T].
 
 Parity pins (tests/test_oracle_budget.py): the lemma evaluated on a worked
-example by hand (tests/golden/clt_budget.txt), monotonicity in eps / delta,
-and the bound's coverage checked by simulation.
+example by hand (tests/golden/clt_budget.txt); the whole budget of one unit
+worked by hand in exact rational arithmetic (tests/golden/clt_unit.txt: the
+n_T / b0 scale-up, the unbiased spreads, eps/4 and delta/2, both bounds of
+both heads, the max, the ceiling, the clamp); monotonicity in eps / delta;
+the bound's coverage checked by simulation.
 """
 import math
 

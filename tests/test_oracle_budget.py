@@ -66,3 +66,52 @@ def test_clt_budget_monotone_and_clamped():
     b_loose, _ = budget.clt_budget(q, k, v, idx, base, s, 0.1, 0.2, len(tail))
     b_tight, _ = budget.clt_budget(q, k, v, idx, base, s, 0.1, 0.01, len(tail))
     assert b_loose <= b_tight
+
+
+def _clt_unit(golden_dir):
+    """The hand-worked unit of tests/golden/clt_unit.txt as oracle inputs."""
+    rows, want, prm = [], {}, {}
+    with open(os.path.join(golden_dir, "clt_unit.txt")) as f:
+        for line in f:
+            t = line.split()
+            if not t or t[0].startswith("#"):
+                continue
+            if t[0] in ("I", "S"):
+                rows.append((t[0], int(t[1]), [float(x) for x in t[2:4]], [float(x) for x in t[4:6]]))
+            elif t[0] in ("bN", "bD"):
+                want[(t[0], int(t[1]) - 1)] = (int(t[2]), int(t[3]))
+            elif t[0] == "params":
+                prm = {t[i]: float(t[i + 1]) for i in range(1, len(t), 2)}
+    n_t = int(prm["n_t"])
+    idx = np.array([p for kind, p, _, _ in rows if kind == "I"])
+    base = np.array([p for kind, p, _, _ in rows if kind == "S"])
+    L = len(idx) + n_t
+    k = np.zeros((L, 2))
+    v = np.zeros((L, 2))
+    for _, p, kr, vr in rows:
+        k[p], v[p] = kr, vr
+    q = np.eye(2)
+    return q, k, v, idx, base, n_t, want, prm
+
+
+def test_clt_budget_hand_worked_unit(golden_dir):
+    # every step of the budget's composition: the n_T / b0 scale-up of the
+    # base sample in N_hat and D_hat, unbiased spreads, eps/4 and delta/2 per
+    # estimate, both bounds of both heads, the max, the ceiling and the clamp
+    q, k, v, idx, base, n_t, want, prm = _clt_unit(golden_dir)
+    b, det = budget.clt_budget(q, k, v, idx, base, math.log(2.0), prm["eps"], prm["delta"], n_t)
+    z2 = prm["z"] ** 2
+    for h in range(2):
+        for key, got in (("bN", det["b_N"][h]), ("bD", det["b_D"][h])):
+            num, den = want[(key, h)]
+            assert got == pytest.approx(z2 * num / den, rel=1e-9), (key, h)
+    assert b == int(prm["b"])
+
+
+def test_clt_budget_clamps_to_the_tail(golden_dir):
+    # the same unit with eps 50x tighter: the real budget exceeds n_T and the
+    # sample is the whole tail; 1000x looser: the base sample already suffices
+    q, k, v, idx, base, n_t, want, prm = _clt_unit(golden_dir)
+    s = math.log(2.0)
+    assert budget.clt_budget(q, k, v, idx, base, s, prm["eps"] / 50, prm["delta"], n_t)[0] == n_t
+    assert budget.clt_budget(q, k, v, idx, base, s, prm["eps"] * 1000, prm["delta"], n_t)[0] == len(base)

@@ -203,3 +203,57 @@ def test_grown_prior_mistake_fails_a_pin(monkeypatch):
     monkeypatch.setattr(pin_stats, "grown_stats", _grown_stats_prefix_prior)
     assert _some_pin_fails([(pin_stats.test_grown_stats_follow_the_token_recurrence, {}),
                             (pin_stats.test_grown_stats_constant_keys_closed_form, {})])
+
+
+def _clt_budget_variant(eps_div=4.0, delta_div=2.0, scale_up=True, ddof=1, reduce_heads=max):
+    """oracle.budget.clt_budget restated with one step changeable, to plant a
+    mistake in the budget's composition."""
+    import oracle.budget as budget
+
+    def f(q, k, v, idx, base_pos, scale, eps, delta, n_t):
+        b0 = len(base_pos)
+        if n_t == 0 or b0 < 2:
+            return 0, {}
+        e1, d1 = eps / eps_div, delta / delta_div
+        l_i, l_s = scale * (q @ k[idx].T), scale * (q @ k[base_pos].T)
+        m = np.maximum(l_i.max(axis=1), l_s.max(axis=1))
+        e_i, e_s = np.exp(l_i - m[:, None]), np.exp(l_s - m[:, None])
+        w = n_t / b0 if scale_up else 1.0
+        n_hat = e_i @ v[idx] + w * (e_s @ v[base_pos])
+        d_hat = e_i.sum(axis=1) + w * e_s.sum(axis=1)
+        det = {"b_N": [], "b_D": []}
+        per_head = []
+        for h in range(q.shape[0]):
+            r = e_s[h][:, None] * v[base_pos]
+            b_n = budget.lemma_budget(n_t, float(r.var(axis=0, ddof=ddof).sum()),
+                                      e1 * float(np.linalg.norm(n_hat[h])), d1)
+            b_d = budget.lemma_budget(n_t, float(e_s[h].var(ddof=ddof)), e1 * float(d_hat[h]), d1)
+            det["b_N"].append(b_n)
+            det["b_D"].append(b_d)
+            per_head.append(max(b_n, b_d))
+        best = reduce_heads(per_head)
+        b = int(min(max(math.ceil(best) if math.isfinite(best) else n_t, b0), n_t))
+        return b, det
+    return f
+
+
+CLT_MISTAKES = {
+    "eps split in two, not four": dict(eps_div=2.0),
+    "delta not split": dict(delta_div=1.0),
+    "no n_T / b0 scale-up of the base sample": dict(scale_up=False),
+    "biased (ddof 0) spreads": dict(ddof=0),
+    "min over the query heads": dict(reduce_heads=min),
+}
+
+
+@pytest.mark.parametrize("name", list(CLT_MISTAKES))
+def test_clt_budget_mistake_fails_a_pin(monkeypatch, golden_dir, name):
+    import oracle.budget as budget
+    import test_oracle_budget as pin_budget
+    pins = [(pin_budget.test_clt_budget_hand_worked_unit, {"golden_dir": golden_dir}),
+            (pin_budget.test_clt_budget_clamps_to_the_tail, {"golden_dir": golden_dir})]
+    monkeypatch.setattr(budget, "clt_budget", _clt_budget_variant())
+    for fn, kw in pins:                       # the restatement itself passes
+        fn(**kw)
+    monkeypatch.setattr(budget, "clt_budget", _clt_budget_variant(**CLT_MISTAKES[name]))
+    assert _some_pin_fails(pins)
