@@ -87,6 +87,35 @@ def decode_bytes_per_unit(w, sg, esz, mode, b_draws):
     return byts
 
 
+def survey_bytes_per_unit(w, sg, esz, mode, b_draws):
+    """The method's bytes per unit and step as the scope table counts them:
+    the block summaries of every candidate in the cache dtype, the group's
+    queries, the exactly read K/V rows, the mode's statistics, the output
+    and the chosen indices (written once, read once)."""
+    byts = sg["n_cand"] * w.d * esz + w.G * w.d * esz + sg["n_i"] * 2 * w.d * esz + w.G * w.d * 4 + 8 * sg["kk"]
+    if mode == "resa":
+        byts += w.G * (2 * w.d * 4 + 4) + w.d * 4
+    if mode == "proxy":
+        byts += 2 * w.d * 4
+    if mode == "sample":
+        byts += b_draws * (2 * w.d * esz + 8)
+    return byts
+
+
+def survey_select_bytes_per_unit(w, sg, esz, b_draws):
+    """The selection's share of survey_bytes_per_unit: summaries, queries,
+    the chosen indices and the draws written."""
+    return sg["n_cand"] * w.d * esz + w.G * w.d * esz + 4 * sg["kk"] + 4 * b_draws
+
+
+def launches_per_step(w, sg, clt):
+    """Kernels one sa_step launches: the selection (one kernel when every unit
+    has a CTA of its own and its keys fit shared memory, else a scan and a
+    finish kernel), the CLT budget's two kernels, the decode."""
+    one = w.B * w.Hkv >= 148 and sg["n_cand"] <= 4096
+    return (1 if one else 2) + (2 if clt else 0) + 1
+
+
 def set_geom(L, sink, local, k_blocks):
     s_eff = min(sink, L)
     w_eff = min(min(local, L), L - s_eff)
@@ -151,9 +180,17 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY, "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+        # nvidia-smi takes a moment to start: wait (bounded) for its first row
+        # so that the sampled span covers the timed region
+        t0 = time.time()
+        while time.time() - t0 < 5.0 and self.proc.poll() is None:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.05)
 
     def stop(self):
         if self.proc is None:
@@ -402,20 +439,21 @@ def main(argv=None):
             ev[2].record(stream)
         return fn
 
+    # clocks are sampled from before the warm-up until after the dense pass,
+    # so that the samples cover the timed steps whatever their number
+    clocks = ClockSampler(local)
+    clocks.start()
     # warm-up (untimed)
     for t in range(args.warmup):
         flush_l2()
         step(t, args.mode)
     torch.cuda.synchronize()
 
-    clocks = ClockSampler(local)
     barrier()
     torch.cuda.synchronize()
-    clocks.start()
     per = timed(args.steps, sparse_step(args.mode), 2)
     torch.cuda.synchronize()
     barrier()
-    clk = clocks.stop()
     total_ms = sum(p[0] for p in per)
     total_ms = reduce_max(total_ms, dev)
     # kernel breakdown: the same step as two calls, each bracketed by events
@@ -454,6 +492,12 @@ def main(argv=None):
     sel_gbs = sel_b / (sel_avg * 1e-3) / 1e9
     dec_gbs = dec_b / (dec_avg * 1e-3) / 1e9
     step_gbs = (sel_b + dec_b) / (ms_per_step * 1e-3) / 1e9
+    # the scope table's byte count (bf16 block summaries, not the int8 sketch
+    # the selection actually streams)
+    sv_sel = survey_select_bytes_per_unit(w, sg, esz, b_mean) * w.B * w.Hkv
+    sv_step = survey_bytes_per_unit(w, sg, esz, args.mode, b_mean) * w.B * w.Hkv
+    sv_sel_gbs = sv_sel / (sel_avg * 1e-3) / 1e9
+    sv_step_gbs = sv_step / (ms_per_step * 1e-3) / 1e9
 
     # other modes (same selection kernel)
     mode_vals = {}
@@ -481,6 +525,7 @@ def main(argv=None):
     timed(3, dense_fn, 2)
     pd = timed(args.dense_steps, dense_fn, 2)
     dense_ms = statistics.mean(p[0] for p in pd)
+    clk = clocks.stop()
     dense_bytes = 2 * w.B * w.Hkv * w.L * w.d * esz + w.B * w.Hq * w.d * (esz + 4)
     dense = {"tokens_per_s": w.B / (dense_ms * 1e-3), "ms_per_step": dense_ms,
              "hbm_gbs": dense_bytes / (dense_ms * 1e-3) / 1e9,
@@ -492,20 +537,28 @@ def main(argv=None):
         q_host = Q.cpu().pin_memory()
         q_dev = torch.empty_like(Q[0])
         o_host = torch.empty(w.B, w.Hq, w.d, dtype=torch.float32).pin_memory()
+        # the public API's prepared call: the step's structures built once,
+        # each call passes this step's query, output and step index
+        prep = sa.PreparedStep(K, V, stats, sps[0], mode=args.mode, selection=sel)
 
         def e2e_fn(t, ev):
-            sp = sps[t % nq]
             ev[0].record(stream)
             q_dev.copy_(q_host[t % nq], non_blocking=True)
-            sa.step(q_dev, K, V, stats, sp, mode=args.mode, selection=sel, out=out)
-            o_host.copy_(out, non_blocking=True)
             ev[1].record(stream)
-        timed(3, e2e_fn, 2)
-        pe = timed(min(args.steps, 500), e2e_fn, 2)
-        e2e_ms = reduce_max(sum(p[0] for p in pe), dev) / len(pe)
+            prep(q_dev, out, step=sps[t % nq].step)
+            ev[2].record(stream)
+            o_host.copy_(out, non_blocking=True)
+            ev[3].record(stream)
+        timed(3, e2e_fn, 4)
+        pe = timed(min(args.steps, 500), e2e_fn, 4)
+        e2e_ms = reduce_max(sum(sum(p) for p in pe), dev) / len(pe)
         e2e = {"value": ws * w.B / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": int(Q[0].numel() * Q.element_size()),
-               "d2h_bytes_per_step": int(out.numel() * 4)}
+               "d2h_bytes_per_step": int(out.numel() * 4),
+               "h2d_us": 1e3 * statistics.mean(p[0] for p in pe),
+               "step_us": 1e3 * statistics.mean(p[1] for p in pe),
+               "d2h_us": 1e3 * statistics.mean(p[2] for p in pe),
+               "api": "kv_cache_residual_b200.PreparedStep (sa_step), pinned host buffers"}
 
     # cache append (the cache growing during decode): one token per unit
     # through sa_append, written at the last row of the cache with that row's
@@ -549,16 +602,24 @@ def main(argv=None):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded generator, Llama-3.1-8B layer shapes)",
             "config": dict(workload_config(w, sg, args), **({"clt": clt_info} if clt_info else {})),
-            "roofline": {"bound": "hbm", "kernel": "k_select (sketch scan + certified top-k)", "achieved": sel_gbs,
-                         "peak": peak, "unit": "GB/s", "frac": sel_gbs / peak, "traffic": traffic,
-                         "bytes_per_launch": sel_b, "us_per_launch": 1e3 * sel_avg, "peak_source": peak_src},
-            "step_roofline": {"achieved": step_gbs, "frac": step_gbs / peak, "bytes_per_step": sel_b + dec_b,
+            "roofline": {"bound": "hbm", "kernel": "k_select (sketch scan + certified top-k)",
+                         "achieved": sv_sel_gbs, "peak": peak, "unit": "GB/s", "frac": sv_sel_gbs / peak,
+                         "traffic": traffic, "bytes_per_launch": sv_sel,
+                         "bytes_basis": "scope-table bytes: bf16 block summaries of every candidate + queries + indices",
+                         "us_per_launch": 1e3 * sel_avg, "peak_source": peak_src,
+                         "moved_bytes_per_launch": sel_b, "achieved_moved": sel_gbs, "frac_moved": sel_gbs / peak,
+                         "moved_basis": "bytes the kernel streams: int8 sketch + 16 B of bounds per candidate"},
+            "step_roofline": {"achieved": sv_step_gbs, "frac": sv_step_gbs / peak, "bytes_per_step": sv_step,
+                              "bytes_basis": "scope-table bytes of the whole step",
+                              "achieved_moved": step_gbs, "frac_moved": step_gbs / peak,
+                              "moved_bytes_per_step": sel_b + dec_b,
                               "decode_gbs": dec_gbs, "decode_us": 1e3 * dec_avg, "decode_bytes": dec_b},
             "dense": dense, "speedup_vs_dense": dense_ms / ms_per_step, "modes": mode_vals,
             "kernels_us": {"k_select": 1e3 * sel_avg, "k_decode": 1e3 * dec_avg,
                            "separate_sum": 1e3 * (sel_avg + dec_avg), "step_overlapped": 1e3 * ms_per_step},
             "append": append, "prefill": prefill,
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (3 if clt else 2) * args.steps, "clocks": clk,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step(w, sg, clt) * args.steps,
+            "clocks": clk,
         }
         print(json.dumps(line))
     barrier()

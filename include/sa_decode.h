@@ -256,10 +256,12 @@ SA_API sa_status sa_select(const sa_shape* shape, const sa_select_params* params
  * counterpart: this is a deployment convenience.  Same inputs, outputs and
  * results as sa_select; the scratch is a fixed 8 MiB array inside the
  * library (present on every device that loads it), so shapes whose
- * selection workspace exceeds 8 MiB return SA_ERR_WORKSPACE.  The array is
- * shared by all calls on a device: the call clears its completion counters
- * with cudaMemsetAsync on `stream` first, and calls that overlap on the GPU
- * race and must not be issued.  The first call on a device looks up the
+ * selection workspace exceeds 8 MiB return SA_ERR_WORKSPACE.  The arguments
+ * are checked first, exactly as sa_select checks them; a rejected call
+ * enqueues nothing.  The array is shared by all calls on a device: an
+ * accepted call clears its completion counters with cudaMemsetAsync on
+ * `stream` first, and calls that overlap on the GPU race and must not be
+ * issued.  The first call on a device looks up the
  * array's device address (cudaGetSymbolAddress) with that device current;
  * make that first call before any stream capture.  Allocates nothing. */
 SA_API sa_status sa_select_noalloc(const sa_shape* shape, const sa_select_params* params, const void* q,
@@ -285,16 +287,6 @@ SA_API sa_status sa_step(const sa_shape* shape, const sa_decode_params* dparams,
                          const sa_select_params* sparams, const void* q, const void* k, const void* v,
                          const sa_stats* stats, const sa_selection* sel, float* out, void* ws,
                          size_t ws_bytes, void* stream);
-
-/* 1 when sa_step runs this step as one fused kernel (selection and decode
- * by the same CTA, one CTA per unit), 0 when it runs the selection and decode
- * kernels as a programmatic pair, -1 on invalid arguments.  The fused kernel
- * is opt-in (environment variable SA_FUSED_STEP=1, read at every call) and
- * then used for a bf16 cache with B*Hkv large enough that each unit gets a
- * CTA of its own, k_blocks <= 32 and, for SA_SAMPLE, sample_cap <= 256.  Both
- * paths give the same results.  Diagnostic: the pages have no counterpart. */
-SA_API int sa_step_fused(const sa_shape* shape, const sa_decode_params* dparams,
-                         const sa_select_params* sparams);
 
 /* Dense flash-decode over all L tokens (the in-build speed reference, not
  * part of the method): out [B, Hq, d] f32 = softmax(s q K^T) V. */

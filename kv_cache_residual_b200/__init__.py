@@ -62,7 +62,7 @@ class sa_decode_params(ctypes.Structure):
 
 EXPORTS = ("sa_workspace_size", "sa_prefill_stats", "sa_block_summaries", "sa_block_sketch", "sa_select",
            "sa_select_noalloc",
-           "sa_decode", "sa_step", "sa_step_fused", "sa_dense_decode", "sa_append", "sa_wait_timeouts",
+           "sa_decode", "sa_step", "sa_dense_decode", "sa_append", "sa_wait_timeouts",
            "sa_status_string")
 
 _LIB = None
@@ -89,8 +89,6 @@ def _lib():
         lib.sa_step.argtypes = [sh, dp, sp, P, P, P, st, sel, P, P, S, P]
         lib.sa_dense_decode.argtypes = [sh, P, P, P, P, F, P, S, P]
         lib.sa_append.argtypes = [sh, P, P, P, P, st, F, P]
-        lib.sa_step_fused.argtypes = [sh, dp, sp]
-        lib.sa_step_fused.restype = I
         lib.sa_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
         lib.sa_wait_timeouts.restype = I
         lib.sa_status_string.argtypes = [I]
@@ -277,9 +275,9 @@ def decode(q, k, v, stats, selection, params, mode="resa", lam=1.0, scale=0.0, o
 
 def step(q, k, v, stats, params, mode="resa", lam=1.0, scale=0.0, selection=None, out=None, length=None,
          stream=None):
-    """Selection then decode in one call: one fused kernel when step_fused()
-    says so, else the two kernels with the decode overlapping the end of the
-    selection (programmatic dependent launch).  Returns (out, selection)."""
+    """Selection then decode in one call: the two kernels with the decode
+    overlapping the end of the selection (programmatic dependent launch).
+    Returns (out, selection)."""
     B, Hq, d = q.shape
     shape = make_shape(k, Hq, length)
     cp = params.c()
@@ -297,14 +295,38 @@ def step(q, k, v, stats, params, mode="resa", lam=1.0, scale=0.0, selection=None
     return out, selection
 
 
-def step_fused(q, k, params, mode="resa", length=None):
-    """True when step() runs as the single fused kernel for these arguments."""
-    shape = make_shape(k, q.shape[1], length)
-    r = _lib().sa_step_fused(ctypes.byref(shape), ctypes.byref(sa_decode_params(MODES[mode], 1.0, 0.0)),
-                             ctypes.byref(params.c()))
-    if r < 0:
-        raise SAError(SA_ERR_INVALID_ARG, "sa_step_fused")
-    return r == 1
+class PreparedStep:
+    """The arguments of sa_step built once for a fixed cache, statistics,
+    parameters and selection buffers; each call passes this step's query and
+    output (and optionally the decode step index that keys the draws) and
+    runs one sa_step.  For callers that decode many steps with the same
+    buffers: a call marshals two pointers and the stream instead of
+    rebuilding every structure."""
+
+    def __init__(self, k, v, stats, params, mode="resa", lam=1.0, scale=0.0, selection=None, length=None,
+                 Hq=None):
+        B, Hkv, ld, d = k.shape
+        Hq = stats.mu_q.shape[1] if Hq is None else Hq
+        self.k, self.v, self.stats = k, v, stats
+        self.shape = make_shape(k, Hq, length)
+        self.cp = params.c()
+        self.dp = sa_decode_params(MODES[mode], float(lam), float(scale))
+        self.selection = selection if selection is not None else Selection(B, Hkv, params.k_blocks,
+                                                                           self.cp.sample_cap, k.device)
+        self.ws = workspace(self.shape, self.cp, OP_STEP, k.device)
+        self._st = stats.c()
+        self._sel = self.selection.c()
+        self._args = (ctypes.byref(self.shape), ctypes.byref(self.dp), ctypes.byref(self.cp))
+        self._tail = (_ptr(k), _ptr(v), ctypes.byref(self._st), ctypes.byref(self._sel))
+        self._ws = (_ptr(self.ws), self.ws.numel())
+        self._fn = _lib().sa_step
+
+    def __call__(self, q, out, step=None, stream=None):
+        if step is not None:
+            self.cp.step = int(step)
+        _check(self._fn(*self._args, ctypes.c_void_p(q.data_ptr()), *self._tail, ctypes.c_void_p(out.data_ptr()),
+                        *self._ws, _stream(stream)), "sa_step")
+        return out
 
 
 def dense_decode(q, k, v, scale=0.0, out=None, length=None, stream=None):

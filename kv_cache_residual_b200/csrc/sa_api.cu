@@ -226,6 +226,15 @@ sa_status prep_decode(const sa_shape* shape, const sa_decode_params* dparams, co
 
 }  // namespace
 
+sa_status sa::check_select_call(const sa_shape* shape, const sa_select_params* params, const void* q,
+                                const sa_stats* stats, const void* k, const void* v, const sa_selection* out,
+                                float scale) {
+    Dims d;
+    SelectPlan p;
+    SelectArgs a;
+    return prep_select(shape, params, q, stats, k, v, out, scale, &d, &p, &a);
+}
+
 extern "C" {
 
 sa_status sa_select(const sa_shape* shape, const sa_select_params* params, const void* q,
@@ -280,22 +289,12 @@ sa_status sa_step(const sa_shape* shape, const sa_decode_params* dparams, const 
     ad.ws = static_cast<char*>(ws) + ps.bytes;
     ad.pdl = true;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (fused_step_ok(d, ps, pd, *sparams, dparams->mode))
-        return launch_step_fused(d, ps, as, pd, ad, s) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
     if (launch_select(d, ps, as, s) != cudaSuccess) return SA_ERR_CUDA;
     if (sparams->clt_base > 0) {
         // the budget kernel sits between: the decode waits for it as usual
         if (launch_clt(d, ps, as, s) != cudaSuccess) return SA_ERR_CUDA;
     }
     return launch_decode(d, pd, ad, s) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
-}
-
-int sa_step_fused(const sa_shape* shape, const sa_decode_params* dparams, const sa_select_params* sparams) {
-    Dims d;
-    if (dparams == nullptr || check_shape(shape, &d) != SA_OK || check_select_params(sparams) != SA_OK) return -1;
-    const SelectPlan ps = select_plan(d, *sparams);
-    const DecodePlan pd = decode_plan(d, *sparams, dparams->mode);
-    return fused_step_ok(d, ps, pd, *sparams, dparams->mode) ? 1 : 0;
 }
 
 sa_status sa_dense_decode(const sa_shape* shape, const void* q, const void* k, const void* v, float* out,

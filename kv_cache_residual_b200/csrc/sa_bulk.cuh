@@ -6,10 +6,10 @@
 // in the issuing CTA's own shared memory.
 //
 // Every wait is bounded.  A wait that has not seen its phase complete after
-// kWaitNs of %globaltimer gives up and returns false; the CTA then bumps this
-// translation unit's timeout counter once (read from the host by the unit
-// that owns the kernel), drains the copies it has in flight (again bounded)
-// and returns with its outputs marked invalid.
+// kWaitNs of %globaltimer gives up and returns false; the CTA then bumps the
+// library's timeout counter once (a single device variable whose address the
+// kernel receives in its arguments), drains the copies it has in flight
+// (again bounded) and returns with its outputs marked invalid.
 #pragma once
 
 #include <stdint.h>
@@ -18,9 +18,6 @@ namespace sa {
 
 constexpr uint64_t kWaitNs = 2000000000ull;        // give up on a copy after 2 s
 constexpr uint64_t kDrainNs = 500000000ull;        // and on each in-flight copy after 0.5 s
-
-// waits abandoned in this translation unit since the host last read them
-static __device__ unsigned g_wait_timeouts;
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -1,7 +1,6 @@
-// Device code shared by the decode kernels and the fused step kernel: the
-// residual epilogue (RESA Online Aggregator, proxy token, sampled tail) and
-// the bf16 stream pass over a unit's token list (tensor-core engine,
-// sa_tc.cuh).
+// Device code of the decode kernels: the residual epilogue (RESA Online
+// Aggregator, proxy token, sampled tail) and the bf16 stream pass over a
+// unit's token list (tensor-core engine, sa_tc.cuh).
 #pragma once
 
 #include <type_traits>
@@ -306,13 +305,11 @@ struct StreamIo {
 
 // Chunk `chunk` of unit u.  smem: the dynamic area (stream_smem<> bytes);
 // s_blk / s_samp: shared caches of the chosen blocks / draws (kBlkCache /
-// kSampCache entries).  preset_bu >= 0: the selection is already in s_blk
-// (sg.kk entries) and s_samp (preset_bu draws), visible to every thread (the
-// fused step); otherwise the lists are read from global memory once the
+// kSampCache entries); the lists are read from global memory once the
 // selection kernel (a programmatic dependency, or an earlier launch) is done.
 template <int D, int G, int MODE>
 __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* smem, int* s_blk, int* s_samp, int u,
-                                            int chunk, int preset_bu) {
+                                            int chunk) {
     const __nv_bfloat16* __restrict__ q = io.q;
     const __nv_bfloat16* __restrict__ k = io.k;
     const __nv_bfloat16* __restrict__ v = io.v;
@@ -378,12 +375,7 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
     float lw_samp = 0.f;
     const bool blk_sm = sg.kk <= kBlkCache;
     bool samp_sm = true;
-    bool sel_ready = DENSE || n_indep >= n_hi || preset_bu >= 0;
-    if (!DENSE && preset_bu >= 0 && SAMP && nt > 0) {
-        const int bu = min(preset_bu, sample_cap);
-        lw_samp = bu > 0 ? log2f((float)nt / (float)bu) : 0.f;
-        n_tok = sg.n_i + bu;
-    }
+    bool sel_ready = DENSE || n_indep >= n_hi;
     // Under programmatic dependent launch the preceding selection kernel may
     // still be running: wait for it before the first selection-dependent read
     // (a no-op when the kernel was launched normally).  Called at the same
@@ -654,7 +646,7 @@ k_stream_tc(StreamIo io) {
     constexpr int SB = StageLayout<D>::kBytes;
     extern __shared__ __align__(16) unsigned char smem[];
     int* s_blk = reinterpret_cast<int*>(smem + (size_t)kStages * SB);
-    stream_unit<D, G, MODE>(io, smem, s_blk, s_blk + kBlkCache, blockIdx.y, blockIdx.x, -1);
+    stream_unit<D, G, MODE>(io, smem, s_blk, s_blk + kBlkCache, blockIdx.y, blockIdx.x);
 }
 
 

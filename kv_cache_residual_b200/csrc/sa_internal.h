@@ -222,15 +222,17 @@ inline cudaError_t opt_in_smem(K kernel, size_t bytes, std::atomic<unsigned long
 }
 
 cudaError_t launch_select(const Dims& d, const SelectPlan& p, const SelectArgs& a, cudaStream_t s);
+// selection CTAs (on the current device) that gave up a bounded wait
 cudaError_t select_wait_timeouts(unsigned* count);
+// sa_select's argument checks alone (nothing is enqueued): SA_OK when
+// sa_select would accept these arguments with a large enough workspace
+sa_status check_select_call(const sa_shape* shape, const sa_select_params* params, const void* q,
+                            const sa_stats* stats, const void* k, const void* v, const sa_selection* out,
+                            float scale);
 // The CLT sampling budget (sa_clt.cu), after the selection when clt_base > 0.
 constexpr int kCltMaxBase = 256;     // largest base sample
 cudaError_t launch_clt(const Dims& d, const SelectPlan& p, const SelectArgs& a, cudaStream_t s);
 
-// The fused step (selection + decode in one kernel, sa_fused.cu): whether it
-// applies to this step, and its launch.
-bool fused_step_ok(const Dims& d, const SelectPlan& sp, const DecodePlan& dp, const sa_select_params& prm,
-                   int mode);    // CTAs of the selection kernel that gave up a wait
 
 struct DecodeArgs {
     const void* q; const void* k; const void* v; sa_stats st; sa_selection sel;
@@ -238,8 +240,6 @@ struct DecodeArgs {
     bool pdl;          // launched as a programmatic dependent of the selection kernel
 };
 cudaError_t launch_decode(const Dims& d, const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
-cudaError_t launch_step_fused(const Dims& d, const SelectPlan& sp, const SelectArgs& sa_, const DecodePlan& dp,
-                              const DecodeArgs& da, cudaStream_t s);
 
 struct DenseArgs {
     const void* q; const void* k; const void* v; float scale; float* out; char* ws;

@@ -53,11 +53,15 @@ extern "C" {
 sa_status sa_select_noalloc(const sa_shape* shape, const sa_select_params* params, const void* q,
                             const sa_stats* stats, const void* k, const void* v, const sa_selection* out,
                             float scale, void* stream) {
+    // every argument check first: a rejected call enqueues nothing and leaves
+    // the shared array as it was
+    sa_status e = sa::check_select_call(shape, params, q, stats, k, v, out, scale);
+    if (e != SA_OK) return e;
     const size_t need = sa_workspace_size(shape, params, SA_OP_SELECT);
     if (need == 0) return SA_ERR_INVALID_ARG;
     if (need > kNoAllocScratchBytes) return SA_ERR_WORKSPACE;     // shape too large for the fixed array
     void* ws = nullptr;
-    sa_status e = scratch_for_current_device(&ws);
+    e = scratch_for_current_device(&ws);
     if (e != SA_OK) return e;
     // the completion counters (two per unit: selection and CLT budget, at offset 0 of its
     // workspace) must start at zero; the array may hold a previous call's data

@@ -10,6 +10,29 @@
 
 namespace sa {
 
+// selection CTAs that abandoned a bounded wait, since the library was loaded
+// (the only definition: every selection kernel counts into it through
+// SelectIo::timeouts)
+__device__ unsigned g_wait_timeouts;
+
+namespace {
+std::atomic<unsigned*> g_timeouts_ptr[64];
+}
+
+// device address of this device's counter, looked up once per device
+static unsigned* wait_counter() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return nullptr;
+    if (dev < 64) {
+        unsigned* p = g_timeouts_ptr[dev].load(std::memory_order_acquire);
+        if (p != nullptr) return p;
+    }
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_wait_timeouts) != cudaSuccess) return nullptr;
+    if (dev < 64) g_timeouts_ptr[dev].store(static_cast<unsigned*>(p), std::memory_order_release);
+    return static_cast<unsigned*>(p);
+}
+
 constexpr int kSelStages = 4;      // 4 x 18 KB ring at d = 128: two CTAs per SM
 constexpr int kFinThreads = 512;
 constexpr int kFinishKeys = 16384; // keys of one unit in the finish kernel's shared memory
@@ -89,6 +112,7 @@ SelectIo select_io(const Dims& d, const SelectPlan& p, const SelectArgs& a) {
     io.sample_cap = a.sp.sample_cap;
     io.seed = (unsigned long long)a.sp.seed;
     io.step = a.sp.step;
+    io.timeouts = wait_counter();
     return io;
 }
 
@@ -96,6 +120,7 @@ template <typename T, int D, int G>
 static cudaError_t select_t(const Dims& d, const SelectPlan& p, const SelectArgs& a, cudaStream_t s) {
     constexpr size_t smem = SketchRing<D, kWarps, kSelStages>::kSmem;
     const SelectIo io = select_io(d, p, a);
+    if (io.timeouts == nullptr) return cudaErrorInvalidDevice;
     if (p.nss == 1 && p.g.n_cand <= kSmemKeys) {
         static std::atomic<unsigned long long> opted{0};
         cudaError_t e = opt_in_smem(k_select<T, D, G, kPhAll>, smem, opted);

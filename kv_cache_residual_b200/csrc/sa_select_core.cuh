@@ -2,7 +2,7 @@
 // Device code of the per-step selection (vAttention, Method, overall
 // framework: I_f = sink + local window + top-k; the top-k ranks 16-token
 // blocks by their mean key, the block selection of Quest / ArkVale that RESA
-// wraps), shared by the selection kernel and the fused step kernel.
+// wraps), used by the selection kernels.
 //
 // select_unit (one unit per CTA, or a slice of one when split):
 //   scan  : score intervals of the unit's candidate blocks from the int8
@@ -467,6 +467,40 @@ __device__ void rescore_members(const T* bm, const int* s_bidx, int nb, const fl
     }
 }
 
+// The unit's tail draws (vAttention, Method, key design 1: uniform draws
+// from the residual, with replacement): min(sample_b, sample_cap) positions
+// when the tail is not empty, written to samp_idx (and s_copy when they fit
+// s_copy_cap), their count to samp_count[u].  chosen = the unit's kk chosen
+// blocks in ascending order (shared or global memory, visible to every
+// thread).  Draw i's rank r (SplitMix64 counter stream of (seed, b, g, step))
+// maps to the r-th tail position: tail = [s_eff, L - w_eff) minus the chosen
+// blocks, and chosen block j starts after g_j = 16 c_j - s_eff - 16 j tail
+// tokens.  Returns the count.
+template <int NT>
+__device__ __forceinline__ int unit_draws(const SetGeom& sg, const int32_t* chosen, int sample_b, int sample_cap,
+                                          unsigned long long seed, int b, int g, int step, int u, int32_t* samp_idx,
+                                          int32_t* samp_count, int* s_copy, int s_copy_cap) {
+    const int nt = sg.n_t, kk = sg.kk;
+    const int bdraw = (nt > 0) ? min(sample_b, sample_cap) : 0;
+    if (threadIdx.x == 0) samp_count[u] = bdraw;
+    if (bdraw > 0) {
+        const uint64_t key = unit_key(seed, (uint64_t)b, (uint64_t)g, (uint64_t)step);
+        int32_t* out_s = samp_idx + (size_t)u * sample_cap;
+        for (int i = threadIdx.x; i < bdraw; i += NT) {
+            const int r = (int)draw_rank(key, (uint32_t)i, (uint32_t)nt);
+            int lo_j = 0, hi_j = kk;             // count of j with g_j <= r
+            while (lo_j < hi_j) {
+                const int mid = (lo_j + hi_j) >> 1;
+                const int gj = 16 * chosen[mid] - sg.s_eff - 16 * mid;
+                if (gj <= r) lo_j = mid + 1; else hi_j = mid;
+            }
+            out_s[i] = sg.s_eff + r + 16 * lo_j;
+            if (s_copy != nullptr && bdraw <= s_copy_cap) s_copy[i] = sg.s_eff + r + 16 * lo_j;
+        }
+    }
+    return bdraw;
+}
+
 // Inputs and outputs of one unit's selection (device pointers; the layouts
 // of sa_select in sa_decode.h).
 struct SelectIo {
@@ -490,6 +524,7 @@ struct SelectIo {
     int sample_b, sample_cap;
     unsigned long long seed;
     int step;
+    unsigned* timeouts;                   // the library's count of abandoned waits (one per device)
 };
 
 // Shared memory the selection works in (the caller lays it out):
@@ -771,7 +806,7 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
             // give the copies still in flight a bounded time to land, then
             // return with the unit's outputs marked invalid
             if (threadIdx.x == 0) {
-                atomicAdd(&g_wait_timeouts, 1u);
+                atomicAdd(io.timeouts, 1u);
                 for (int jj = j; jj < min(nst, j + Ring::kStages); ++jj)
                     mbar_wait(bar0 + 8 * (jj % Ring::kStages), (uint32_t)(jj / Ring::kStages) & 1u, kDrainNs);
             }
@@ -1013,26 +1048,8 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
     __syncthreads();
 
     // ---- tail draws -------------------------------------------------------------
-    const int nt = sg.n_t;
-    const int bdraw = (nt > 0) ? min(sample_b, sample_cap) : 0;
-    if (threadIdx.x == 0) samp_count[u] = bdraw;
-    if (bdraw > 0) {
-        const uint64_t key = unit_key(seed, (uint64_t)b, (uint64_t)g, (uint64_t)step);
-        int32_t* out_s = samp_idx + (size_t)u * sample_cap;
-        for (int i = threadIdx.x; i < bdraw; i += NT) {
-            const int r = (int)draw_rank(key, (uint32_t)i, (uint32_t)nt);
-            // tail = [s_eff, L - w_eff) minus the chosen blocks; chosen block j
-            // starts after g_j = 16 c_j - s_eff - 16 j tail tokens
-            int lo_j = 0, hi_j = kk;             // count of j with g_j <= r
-            while (lo_j < hi_j) {
-                const int mid = (lo_j + hi_j) >> 1;
-                const int gj = 16 * (sorted_smem ? s_sorted[mid] : out_idx[mid]) - sg.s_eff - 16 * mid;
-                if (gj <= r) lo_j = mid + 1; else hi_j = mid;
-            }
-            out_s[i] = sg.s_eff + r + 16 * lo_j;
-            if (sm.samp != nullptr && bdraw <= sm.samp_cap) sm.samp[i] = sg.s_eff + r + 16 * lo_j;
-        }
-    }
+    const int bdraw = unit_draws<NT>(sg, sorted_smem ? s_sorted : out_idx, sample_b, sample_cap, seed, b, g, step,
+                                     u, samp_idx, samp_count, sm.samp, sm.samp_cap);
     if (!local) reset_counter(cnt + u);
     res.done = true;
     res.sorted_smem = sorted_smem;

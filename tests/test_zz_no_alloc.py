@@ -15,7 +15,7 @@ import kv_cache_residual_b200 as sa
 pytestmark = pytest.mark.gpu
 
 
-def _noalloc_select(q, stats, params, scale=0.0):
+def _noalloc_select(q, stats, params, scale=0.0, k=None, v=None):
     B, Hq, d = q.shape
     Hkv, L = stats.blk_mean.shape[1], stats.blk_mean.shape[2] * 16
     shape = sa.sa_shape(B, Hq, Hkv, d, L, sa._dtype_code(q))
@@ -24,7 +24,7 @@ def _noalloc_select(q, stats, params, scale=0.0):
     st = stats.c()
     c_sel = sel.c()
     status = sa._lib().sa_select_noalloc(ctypes.byref(shape), ctypes.byref(cp), sa._ptr(q), ctypes.byref(st),
-                                         None, None, ctypes.byref(c_sel), float(scale), sa._stream())
+                                         sa._ptr(k), sa._ptr(v), ctypes.byref(c_sel), float(scale), sa._stream())
     assert status == sa.SA_OK, sa._lib().sa_status_string(status)
     return sel
 
@@ -49,6 +49,43 @@ def test_noalloc_select_matches_workspace_select_twice(wname, B):
         assert torch.equal(got.blk_idx, want.blk_idx)
         assert torch.equal(got.samp_count, want.samp_count)
         assert torch.equal(got.samp_idx, want.samp_idx)
+
+
+def test_noalloc_clt_budget_matches_workspace_select_twice():
+    """The sampling budget path through the fixed array (its completion
+    tickets and per-split fp64 records): flat keys, base sample of 64 draws,
+    two calls in a row against sa_select."""
+    w = synth.scaled(synth.WORKLOADS["flat"], B=2, L=8192)
+    dev = torch.device("cuda")
+    data = synth.make_batch(w, device=dev, steps=2)
+    st = sa.prefill_stats(data["q_ctx"], data["k"], data["v"])
+    for step in range(2):
+        sp = sa.SelectParams(sink=w.sink, local=w.local, k_blocks=w.k_blocks_for(0.05), sample_cap=2048,
+                             clt_base=64, eps=0.1, delta=0.05, seed=7, step=step)
+        q = data["q"][step]
+        want = sa.select(q, st, sp, k=data["k"], v=data["v"])
+        got = _noalloc_select(q, st, sp, k=data["k"], v=data["v"])
+        torch.cuda.synchronize()
+        assert torch.equal(got.blk_idx, want.blk_idx)
+        assert torch.equal(got.samp_count, want.samp_count)
+        assert int(want.samp_count.min()) > 64            # the budget asked for more than the base sample
+        for u in range(w.B * w.Hkv):
+            b, g = divmod(u, w.Hkv)
+            n = int(want.samp_count[b, g])
+            assert torch.equal(got.samp_idx[b, g, :n], want.samp_idx[b, g, :n])
+
+
+def test_noalloc_rejected_call_enqueues_nothing():
+    """A call whose arguments are wrong (a misaligned query) returns before
+    touching the fixed array or the stream."""
+    B, Hq, Hkv, d, L = 1, 4, 1, 64, 2048
+    shape = sa.sa_shape(B, Hq, Hkv, d, L, sa.SA_BF16)
+    cp = sa.SelectParams(k_blocks=4).c()
+    st = sa.sa_stats(*([0x10000] * 10))
+    sel = sa.sa_selection(0x10000, 0x10000, 0x10000, 0)
+    status = sa._lib().sa_select_noalloc(ctypes.byref(shape), ctypes.byref(cp), ctypes.c_void_p(0x10002),
+                                         ctypes.byref(st), None, None, ctypes.byref(sel), 0.0, None)
+    assert status == sa.SA_ERR_INVALID_ARG
 
 
 def test_noalloc_rejects_shapes_beyond_its_array():
