@@ -18,10 +18,26 @@ Readings where the pages are silent:
     scores therefore compare equal whatever the order of the terms, and two
     blocks with identical summaries always tie.
 
+Two other block scores, the alternatives the RESA page's related work (the
+page-level top-k selectors it builds on: Quest, ArkVale) and the GQA
+reading of "per-head top-k" leave open:
+  * "mean_max": score_c = max_{h in group} q_h . kbar_c, the group's
+    strongest head decides (each head's exact dot product rounded once; the
+    max of the rounded values is the rounded max, rounding being monotone);
+  * "quest": per block the elementwise minimum and maximum of its keys,
+    score_c = sum_h sum_e max(q_he min_ce, q_he max_ce), for each head an
+    upper bound of q_h . K_j over the block's tokens (Quest's criticality
+    bound), summed over the group like the default score; each term is one
+    of two exact products, summed exactly and rounded once.
+Both rank by (score desc, index asc) like the default "mean_sum".
+
 Parity pins (tests/test_oracle_select.py): brute force over all subsets on
 tiny inputs, sorting with Python's own sort, all-equal scores, planted blocks
 whose rank is known, scores against exact rational arithmetic, ties between
-identical and permuted summaries.
+identical and permuted summaries; for the two alternatives exact rational
+arithmetic on small integers, the single-head reduction to the default
+score (mean_max), the upper-bound property and its equality on constant
+blocks (quest), planted winners.
 """
 import math
 
@@ -49,6 +65,43 @@ def block_scores(q, blk_mean, cand):
     return out
 
 
+def block_scores_max_heads(q, blk_mean, cand):
+    """max over heads of the exact q_h . kbar_c (each rounded once by fsum)."""
+    q = np.asarray(q, dtype=np.float64)
+    blk_mean = np.asarray(blk_mean, dtype=np.float64)
+    out = np.empty(len(cand), dtype=np.float64)
+    for i, c in enumerate(cand):
+        out[i] = max(math.fsum(q[h] * blk_mean[c]) for h in range(q.shape[0]))
+    return out
+
+
+def block_scores_quest(q, blk_min, blk_max, cand):
+    """sum over heads and dims of max(q_he min_ce, q_he max_ce), every term an
+    exact fp64 product, summed exactly and rounded once (math.fsum)."""
+    q = np.asarray(q, dtype=np.float64)
+    blk_min = np.asarray(blk_min, dtype=np.float64)
+    blk_max = np.asarray(blk_max, dtype=np.float64)
+    out = np.empty(len(cand), dtype=np.float64)
+    for i, c in enumerate(cand):
+        out[i] = math.fsum(np.maximum(q * blk_min[c], q * blk_max[c]).ravel())
+    return out
+
+
+SCORES = ("mean_sum", "mean_max", "quest")
+
+
+def scores_for(score, q, st, cand):
+    """Block scores of the candidates by the named score; st holds blk_mean
+    (and blk_min, blk_max for "quest")."""
+    if score == "mean_sum":
+        return block_scores(q, st["blk_mean"], cand)
+    if score == "mean_max":
+        return block_scores_max_heads(q, st["blk_mean"], cand)
+    if score == "quest":
+        return block_scores_quest(q, st["blk_min"], st["blk_max"], cand)
+    raise ValueError(score)
+
+
 def top_blocks(scores, cand, k):
     """The k best candidates by (score desc, block index asc), returned in
     ascending block order."""
@@ -74,10 +127,11 @@ def tail_set(L, idx):
     return np.flatnonzero(mask)
 
 
-def select_unit(q, blk_mean, L, sink, local, k_blocks):
-    """Full selection of one unit: (chosen blocks ascending, I, T)."""
+def select_unit(q, blk_mean, L, sink, local, k_blocks, score="mean_sum", st=None):
+    """Full selection of one unit: (chosen blocks ascending, I, T).  score
+    other than "mean_sum" takes the summaries from st."""
     cand = candidate_blocks(L, sink, local)
-    sc = block_scores(q, blk_mean, cand)
+    sc = block_scores(q, blk_mean, cand) if score == "mean_sum" else scores_for(score, q, st, cand)
     blocks = top_blocks(sc, cand, k_blocks)
     idx = index_set(L, sink, local, blocks)
     return blocks, idx, tail_set(L, idx)

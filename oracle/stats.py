@@ -13,7 +13,9 @@ Follows RESA, Method, key design 1 ("Prior Estimator"):
 Also the totals the count-aware proxy needs (OpenAttention, stage 04: tail
 sums are totals minus the selected part), and the 16-token block means the
 block selector ranks (Quest/ArkVale-style page summaries named on the RESA
-page's related work), rounded once to the cache dtype.
+page's related work), rounded once to the cache dtype, and each block's
+elementwise key minimum and maximum (Quest's per-page bounds, the summaries
+of the "quest" block score).
 
 Decode grows the cache after prefill end (grown_stats): the statistics then
 describe all cached tokens while the typical query and key stay the ones of
@@ -26,7 +28,8 @@ sketch is built around) does not move.
 Parity pins (tests/test_oracle_stats.py): closed forms for constant keys /
 queries (log_z0 = ln L + s mu_Q.kappa, O_Est = mean V), O_Est against torch's
 scaled_dot_product_attention with query mu_Q, block means against torch's
-bf16 cast where the mean is an fp32 value; grown statistics against a
+bf16 cast where the mean is an fp32 value; block minima and maxima against
+Python loops and torch's amin / amax; grown statistics against a
 token-by-token log-sum-exp recurrence from the prefill-end values and
 against constant-key closed forms at lengths that are not whole blocks.
 """
@@ -44,6 +47,16 @@ def block_means(k, kv_dtype):
     L, d = k.shape
     nb = L // BLOCK
     return round_to(k[: nb * BLOCK].reshape(nb, BLOCK, d).mean(axis=1), kv_dtype)
+
+
+def block_minmax(k):
+    """k [L, d] -> (min, max) [L//16, d]: the elementwise minimum and maximum
+    of the keys of each complete 16-token block (Quest's per-page key
+    bounds); values of the cache, so no rounding."""
+    L, d = k.shape
+    nb = L // BLOCK
+    blocks = k[: nb * BLOCK].reshape(nb, BLOCK, d)
+    return blocks.min(axis=1), blocks.max(axis=1)
 
 
 def prefill_stats(q_ctx, k, v, scale, kv_dtype):
@@ -66,10 +79,12 @@ def prefill_stats(q_ctx, k, v, scale, kv_dtype):
     log_z0 = np.log(a) + m[:, 0]
     o_est = (w @ v) / a[:, None]
     bm = block_means(k, kv_dtype)
+    mn, mx = block_minmax(k)
     return {
         "mu_q": mu_q, "o_est": o_est, "log_z0": log_z0,
         "mu_k": mu_k, "sum_k": sum_k, "sum_v": sum_v,
         "blk_mean": bm, "kbar_absmax": float(np.abs(bm).max()),
+        "blk_min": mn, "blk_max": mx,
     }
 
 
@@ -84,7 +99,9 @@ def grown_stats(st0, k, v, scale, kv_dtype):
     w = np.exp(p0 - m)
     a = w.sum(axis=1)
     bm = block_means(k, kv_dtype)
+    mn, mx = block_minmax(k)
     return {
+        "blk_min": mn, "blk_max": mx,
         "mu_q": mu_q, "o_est": (w @ v) / a[:, None], "log_z0": np.log(a) + m[:, 0],
         "mu_k": st0["mu_k"], "sum_k": k.sum(axis=0), "sum_v": v.sum(axis=0),
         "blk_mean": bm, "kbar_absmax": float(np.abs(bm).max()) if len(bm) else 0.0,

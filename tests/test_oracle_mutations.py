@@ -257,3 +257,55 @@ def test_clt_budget_mistake_fails_a_pin(monkeypatch, golden_dir, name):
         fn(**kw)
     monkeypatch.setattr(budget, "clt_budget", _clt_budget_variant(**CLT_MISTAKES[name]))
     assert _some_pin_fails(pins)
+
+
+def _max_heads_as_sum(q, blk_mean, cand, _orig=select.block_scores):
+    return _orig(q, blk_mean, cand)                                  # sum over heads, not max
+
+
+def _max_heads_as_mean_query(q, blk_mean, cand, _orig=select.block_scores):
+    return _orig(np.asarray(q).max(axis=0, keepdims=True), blk_mean, cand)   # max of the query, not of the scores
+
+
+def _quest_upper_only(q, blk_min, blk_max, cand):
+    q = np.asarray(q, dtype=np.float64)
+    return np.array([math.fsum((q * np.asarray(blk_max)[c]).ravel()) for c in cand])   # min branch dropped
+
+
+def _quest_swapped(q, blk_min, blk_max, cand):
+    q = np.asarray(q, dtype=np.float64)
+    return np.array([math.fsum(np.minimum(q * np.asarray(blk_min)[c], q * np.asarray(blk_max)[c]).ravel())
+                     for c in cand])                                 # lower bound instead of the upper
+
+
+def _minmax_shifted(k):
+    L, d = k.shape
+    nb = L // 16
+    b = k[1: nb * 16 + 1] if L >= nb * 16 + 1 else k[: nb * 16]     # block boundaries off by one token
+    b = b.reshape(-1, 16, d)
+    return b.min(axis=1), b.max(axis=1)
+
+
+SELECTOR_MISTAKES = {
+    "max over heads taken as the sum": ("block_scores_max_heads", _max_heads_as_sum),
+    "max over heads of the query, not the scores": ("block_scores_max_heads", _max_heads_as_mean_query),
+    "quest without the min branch": ("block_scores_quest", _quest_upper_only),
+    "quest taking the lower bound": ("block_scores_quest", _quest_swapped),
+}
+
+
+@pytest.mark.parametrize("name", list(SELECTOR_MISTAKES))
+def test_selector_variant_mistake_fails_a_pin(monkeypatch, name):
+    attr, fn = SELECTOR_MISTAKES[name]
+    monkeypatch.setattr(select, attr, fn)
+    monkeypatch.setattr(pin_sel.S, attr, fn)
+    pins = [(pin_sel.test_max_heads_scores_exact_rational, {"seed": s}) for s in range(3)]
+    pins += [(pin_sel.test_max_heads_planted_single_head_winner, {})]
+    pins += [(pin_sel.test_quest_scores_exact_rational, {"seed": s}) for s in range(3)]
+    pins += [(pin_sel.test_quest_score_bounds_every_token_of_its_block, {})]
+    assert _some_pin_fails(pins)
+
+
+def test_block_minmax_mistake_fails_a_pin(monkeypatch):
+    monkeypatch.setattr(stats, "block_minmax", _minmax_shifted)
+    assert _some_pin_fails([(pin_stats.test_block_minmax_against_loops_and_torch, {})])

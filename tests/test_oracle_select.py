@@ -123,3 +123,118 @@ def test_permuted_summaries_tie_under_a_constant_query():
     sc = S.block_scores(q, blk, np.arange(20))
     assert len(set(sc.tolist())) == 1
     assert S.top_blocks(sc, np.arange(20), 4).tolist() == [0, 1, 2, 3]
+
+
+# ---- the two alternative block scores (max over heads; Quest min/max bounds) ----
+
+def _frac_rows(a):
+    return [[Fraction(x) for x in row] for row in np.asarray(a).tolist()]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_max_heads_scores_exact_rational(seed):
+    # dyadic small values: every score is an exact rational; the oracle's
+    # scores equal max_h sum_e q_he kbar_ce computed in Fractions, and its
+    # top-k equals brute force over those exact scores
+    rng = np.random.default_rng(100 + seed)
+    G, d, nb = 3, 8, 40
+    q = rng.integers(-6, 7, size=(G, d)) / 8.0
+    blk = rng.integers(-5, 6, size=(nb, d)) / 4.0
+    cand = np.arange(2, nb - 3, dtype=np.int64)
+    got = S.block_scores_max_heads(q, blk, cand)
+    qf, bf = _frac_rows(q), _frac_rows(blk)
+    exact = [max(sum(a * b for a, b in zip(qf[h], bf[c])) for h in range(G)) for c in cand]
+    assert [Fraction(x) for x in got] == exact
+    for k in (0, 1, 5, len(cand)):
+        assert S.top_blocks(got, cand, k).tolist() == _brute_force(exact, cand.tolist(), k)
+
+
+def test_max_heads_with_one_head_is_the_default_score():
+    rng = np.random.default_rng(7)
+    q = rng.standard_normal((1, 16)).astype(np.float32).astype(np.float64)
+    blk = rng.standard_normal((50, 16)).astype(np.float32).astype(np.float64)
+    cand = np.arange(50, dtype=np.int64)
+    assert np.array_equal(S.block_scores_max_heads(q, blk, cand), S.block_scores(q, blk, cand))
+
+
+def test_max_heads_planted_single_head_winner():
+    # block 5 matches head 0 strongly and the other heads weakly against it;
+    # block 9 matches every head moderately: the group sum prefers 9, the
+    # max over heads prefers 5
+    d = 4
+    q = np.array([[4.0, 0, 0, 0], [0, 1.0, 0, 0], [0, 0, 1.0, 0]])
+    blk = np.zeros((16, d))
+    blk[5] = [2.0, -1.0, -1.0, 0]          # head scores 8, -1, -1: sum 6, max 8
+    blk[9] = [1.0, 2.0, 2.0, 0]            # head scores 4, 2, 2: sum 8, max 4
+    cand = np.arange(16, dtype=np.int64)
+    assert S.top_blocks(S.block_scores(q, blk, cand), cand, 1).tolist() == [9]
+    assert S.top_blocks(S.block_scores_max_heads(q, blk, cand), cand, 1).tolist() == [5]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_quest_scores_exact_rational(seed):
+    rng = np.random.default_rng(200 + seed)
+    G, d, L = 2, 6, 16 * 12
+    q = rng.integers(-6, 7, size=(G, d)) / 4.0
+    k = rng.integers(-9, 10, size=(L, d)) / 8.0
+    mn, mx = _block_minmax_loops(k)
+    cand = np.arange(1, 11, dtype=np.int64)
+    got = S.block_scores_quest(q, mn, mx, cand)
+    qf, mnf, mxf = _frac_rows(q), _frac_rows(mn), _frac_rows(mx)
+    exact = [sum(max(qf[h][e] * mnf[c][e], qf[h][e] * mxf[c][e]) for h in range(G) for e in range(d))
+             for c in cand]
+    assert [Fraction(x) for x in got] == exact
+    for kk in (1, 3, len(cand)):
+        assert S.top_blocks(got, cand, kk).tolist() == _brute_force(exact, cand.tolist(), kk)
+
+
+def _block_minmax_loops(k):
+    nb = k.shape[0] // 16
+    mn = np.array([[min(k[16 * c + j, e] for j in range(16)) for e in range(k.shape[1])] for c in range(nb)])
+    mx = np.array([[max(k[16 * c + j, e] for j in range(16)) for e in range(k.shape[1])] for c in range(nb)])
+    return mn, mx
+
+
+def test_quest_score_bounds_every_token_of_its_block():
+    # per head, sum_e max(q_e min_e, q_e max_e) >= q . K_j for every token j of
+    # the block; rounding is monotone, so the rounded bound is >= the rounded
+    # largest logit (exact rational logits, rounded once by float()), with
+    # equality when the block's keys are all one row; the group score is the
+    # exact sum of the heads' exact bounds, rounded once
+    rng = np.random.default_rng(11)
+    G, d, L = 3, 8, 16 * 20
+    q = rng.standard_normal((G, d)).astype(np.float32).astype(np.float64)
+    k = rng.standard_normal((L, d)).astype(np.float32).astype(np.float64)
+    k[16 * 7: 16 * 8] = k[16 * 7]                      # block 7: sixteen copies of one key
+    mn, mx = _block_minmax_loops(k)
+    cand = np.arange(20, dtype=np.int64)
+    exact_group = [Fraction(0)] * len(cand)
+    for h in range(G):
+        bound = S.block_scores_quest(q[h:h + 1], mn, mx, cand)
+        for c in cand:
+            top = max(_exact_dot(q[h], k[16 * c + j]) for j in range(16))
+            assert bound[c] >= float(top)
+            if c == 7:
+                assert bound[c] == float(top)
+            exact_group[c] += sum(max(Fraction(a) * Fraction(lo), Fraction(a) * Fraction(hi))
+                                  for a, lo, hi in zip(q[h].tolist(), mn[c].tolist(), mx[c].tolist()))
+    assert S.block_scores_quest(q, mn, mx, cand).tolist() == [float(x) for x in exact_group]
+
+
+def _exact_dot(a, b):
+    return sum(Fraction(x) * Fraction(y) for x, y in zip(a.tolist(), b.tolist()))
+
+
+def test_select_unit_with_alternative_scores():
+    rng = np.random.default_rng(5)
+    G, d, L = 4, 16, 16 * 64
+    q = rng.standard_normal((G, d))
+    k = rng.standard_normal((L, d))
+    from oracle import stats
+    st = stats.prefill_stats(rng.standard_normal((G, L, d)), k, rng.standard_normal((L, d)), 0.25, "f32")
+    for score in S.SCORES:
+        blocks, idx, tail = S.select_unit(q, st["blk_mean"], L, 16, 32, 6, score=score, st=st)
+        cand = S.candidate_blocks(L, 16, 32)
+        want = S.top_blocks(S.scores_for(score, q, st, cand), cand, 6)
+        assert blocks.tolist() == want.tolist()
+        assert len(idx) == 16 + 32 + 6 * 16 and len(idx) + len(tail) == L

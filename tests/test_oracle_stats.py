@@ -110,3 +110,22 @@ def test_grown_stats_constant_keys_closed_form():
     np.testing.assert_allclose(g["o_est"], np.tile(v.mean(0), (G, 1)), atol=1e-13)
     np.testing.assert_allclose(g["sum_k"], Lg * kappa, rtol=1e-15)
     np.testing.assert_array_equal(g["blk_mean"], np.tile(kappa, (Lg // 16, 1)))
+
+
+def test_block_minmax_against_loops_and_torch():
+    from oracle import stats as ostats
+    # elementwise min / max over each complete 16-token block, the partial
+    # last block left out: Python loops and torch's amin / amax over the
+    # reshaped cache agree exactly (values of the cache, no rounding)
+    import torch
+    rng = np.random.default_rng(21)
+    L, d = 16 * 9 + 5, 6
+    k = rng.standard_normal((L, d)).astype(np.float32).astype(np.float64)
+    mn, mx = ostats.block_minmax(k)
+    assert mn.shape == (9, d) and mx.shape == (9, d)
+    for c in range(9):
+        for e in range(d):
+            col = [k[16 * c + j, e] for j in range(16)]
+            assert mn[c, e] == min(col) and mx[c, e] == max(col)
+    t = torch.from_numpy(k[: 16 * 9]).reshape(9, 16, d)
+    assert np.array_equal(mn, t.amin(dim=1).numpy()) and np.array_equal(mx, t.amax(dim=1).numpy())
