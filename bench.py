@@ -21,6 +21,7 @@ Prints ONE JSON line on rank 0.
 on a bounded sample of the same workload, on the host cores.
 """
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -60,6 +61,7 @@ def parse_args(argv=None):
     ap.add_argument("--mode-steps", type=int, default=200)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-selectors", action="store_true", help="skip the alternative block scores")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--batch", type=int, default=0, help="override the batch size (profiling cases)")
     return ap.parse_args(argv)
@@ -568,7 +570,7 @@ def main(argv=None):
     app_st = sa.Stats.__new__(sa.Stats)
     for f in sa.Stats.FIELDS:
         t_ = getattr(stats, f)
-        setattr(app_st, f, t_ if f in ("blk_mean", "blk_code", "blk_meta") else t_.clone())
+        setattr(app_st, f, t_ if (t_ is None or f in ("blk_mean", "blk_code", "blk_meta")) else t_.clone())
     k_last = K[:, :, w.L - 1].contiguous()
     v_last = V[:, :, w.L - 1].contiguous()
 
@@ -586,6 +588,37 @@ def main(argv=None):
     append = {"us_per_call": 1e3 * app_ms, "algorithmic_bytes": app_bytes,
               "note": "one token per unit completing a block (one kernel: k_append)"}
     del app_st
+
+    # the two alternative block scores (max over the group's heads; Quest's
+    # per-block key bounds): the same step with the selection ranking on them
+    # (one CTA per unit scanning the bf16 means, or the min and max rows)
+    selectors = None
+    if not args.no_selectors:
+        stats.blk_min = torch.empty_like(stats.blk_mean)
+        stats.blk_max = torch.empty_like(stats.blk_mean)
+        sa.block_minmax(K, 0, w.L // 16, stats, w.Hq)
+        selectors = {}
+        for score in ("mean_max", "quest"):
+            sps_s = [dataclasses.replace(sp_, score=score) for sp_ in sps]
+            fn = sparse_step(args.mode, sps_s)
+            timed(3, fn, 2)
+            ps_ = timed(args.mode_steps, fn, 2)
+            step_ms = statistics.mean(p_[0] for p_ in ps_)
+
+            def sel_fn(t, ev, sps_s=sps_s):
+                ev[0].record(stream)
+                sa.select(Q[t % nq], stats, sps_s[t % nq], k=K, v=V, selection=sel)
+                ev[1].record(stream)
+            timed(3, sel_fn, 2)
+            pss = timed(args.mode_steps, sel_fn, 2)
+            s_ms = statistics.mean(p_[0] for p_ in pss)
+            rows = 2 if score == "quest" else 1
+            s_bytes = (rows * sg["n_cand"] * w.d * esz + w.G * w.d * esz + 4 * sg["kk"] + 4 * b_mean) * w.B * w.Hkv
+            selectors[score] = {"tokens_per_s": ws * w.B / (step_ms * 1e-3), "ms_per_step": step_ms,
+                                "select_us": 1e3 * s_ms, "select_bytes": s_bytes,
+                                "select_gbs": s_bytes / (s_ms * 1e-3) / 1e9,
+                                "select_frac": s_bytes / (s_ms * 1e-3) / 1e9 / peak}
+        stats.blk_min = stats.blk_max = None
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
@@ -617,7 +650,7 @@ def main(argv=None):
             "dense": dense, "speedup_vs_dense": dense_ms / ms_per_step, "modes": mode_vals,
             "kernels_us": {"k_select": 1e3 * sel_avg, "k_decode": 1e3 * dec_avg,
                            "separate_sum": 1e3 * (sel_avg + dec_avg), "step_overlapped": 1e3 * ms_per_step},
-            "append": append, "prefill": prefill,
+            "append": append, "prefill": prefill, "selectors": selectors,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step(w, sg, clt) * args.steps,
             "clocks": clk,
         }

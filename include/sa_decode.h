@@ -77,6 +77,20 @@ typedef enum { SA_F32 = 0, SA_BF16 = 1 } sa_dtype;
 
 typedef enum { SA_DROP = 0, SA_RESA = 1, SA_PROXY = 2, SA_SAMPLE = 3 } sa_mode;
 
+/* How sa_select ranks the candidate blocks of a KV head (all three on the
+ * exact score rounded once, ties to the lower block index):
+ *   SA_SCORE_MEAN_SUM  sum_{h in group} q_h . kbar_c (the group's summed
+ *                      query against the block mean; the default)
+ *   SA_SCORE_MEAN_MAX  max_{h in group} q_h . kbar_c (the group's strongest
+ *                      head decides: the per-head alternative to one score
+ *                      per KV head)
+ *   SA_SCORE_QUEST     sum_h sum_e max(q_he min_ce, q_he max_ce) over the
+ *                      block's elementwise key minimum and maximum (the
+ *                      page-level upper-bound selector the RESA page's
+ *                      related work wraps; needs blk_min / blk_max)
+ * The two alternatives support up to 16384 candidate blocks per unit. */
+typedef enum { SA_SCORE_MEAN_SUM = 0, SA_SCORE_MEAN_MAX = 1, SA_SCORE_QUEST = 2 } sa_score;
+
 typedef enum {
     SA_OP_PREFILL = 0,   /* sa_prefill_stats */
     SA_OP_SELECT = 1,    /* sa_select        */
@@ -123,7 +137,11 @@ typedef struct {
  *               blk_mean, so the selection equals the one on blk_mean alone; a
  *               sketch not built from this blk_mean and mu_k (rebuild it with
  *               sa_block_sketch when either changes) makes it wrong.  The
- *               selector's own data structure: the pages have no counterpart. */
+ *               selector's own data structure: the pages have no counterpart.
+ *   blk_min, blk_max [B, Hkv, ld/16, d] in dtype, or both NULL: the
+ *               elementwise minimum and maximum of each block's keys (the
+ *               summaries of SA_SCORE_QUEST); written by sa_prefill_stats,
+ *               sa_block_minmax and sa_append when not NULL. */
 typedef struct {
     float* mu_q;
     float* o_est;
@@ -135,6 +153,8 @@ typedef struct {
     float* kbar_absmax;
     int8_t* blk_code;
     float* blk_meta;
+    void* blk_min;
+    void* blk_max;
 } sa_stats;
 
 /* Which tokens one step reads exactly, and how the tail is sampled.
@@ -154,13 +174,15 @@ typedef struct {
  *   seed, step    SplitMix64 stream of unit (b, g) at this step:
  *                 key = out(out(out(out(seed)^b)^g)^step), draw i =
  *                 out(key + i*0x9E3779B97F4A7C15), out(x) = SplitMix64 mixer
- *                 of x + 0x9E3779B97F4A7C15; rank = ((draw>>32)*n_T)>>32     */
+ *                 of x + 0x9E3779B97F4A7C15; rank = ((draw>>32)*n_T)>>32
+ *   score         block score, an sa_score (0 = SA_SCORE_MEAN_SUM)           */
 typedef struct {
     int sink, local, k_blocks;
     int sample_b, clt_base, sample_cap;
     float eps, delta;
     uint64_t seed;
     int step;
+    int score;
 } sa_select_params;
 
 /* Output of sa_select, input of sa_decode (caller-allocated).
@@ -221,7 +243,8 @@ SA_API sa_status sa_block_summaries(const sa_shape* shape, const void* k, int bl
  *   cache (RESA, key design 1), which SA_RESA's tail estimate subtracts the
  *   read set from;
  *   when the token completes block c = (L + 1)/16 - 1: blk_mean[c], its
- *   sketch row and kbar_absmax, as sa_block_summaries for that block.
+ *   sketch row and kbar_absmax, as sa_block_summaries for that block, and
+ *   blk_min[c] / blk_max[c] when the stats carry them.
  * mu_q and mu_k stay as computed at prefill end (the RESA page fixes the
  * typical query and key there; mu_k is also the sketch's centre, which must
  * not move while rows sketched against it remain).  After the call the
@@ -229,6 +252,15 @@ SA_API sa_status sa_block_summaries(const sa_shape* shape, const void* k, int bl
  * (0 = 1/sqrt(d)).  No workspace; one kernel. */
 SA_API sa_status sa_append(const sa_shape* shape, const void* k_new, const void* v_new, void* k, void* v,
                            const sa_stats* stats, float scale, void* stream);
+
+/* Elementwise key minimum and maximum of blocks [blk_begin, blk_end) of every
+ * unit (blk_end <= L/16) into blk_min / blk_max ([B, Hkv, ld/16, d], dtype):
+ * the per-block key bounds of SA_SCORE_QUEST (Quest's page summaries, which
+ * the RESA page's related work names).  sa_prefill_stats writes them for
+ * every block when the stats carry the two pointers; this call covers blocks
+ * written later.  No workspace. */
+SA_API sa_status sa_block_minmax(const sa_shape* shape, const void* k, int blk_begin, int blk_end, void* blk_min,
+                                 void* blk_max, void* stream);
 
 /* Rebuilds the sketch (blk_code, blk_meta) of blocks [blk_begin, blk_end) of
  * every unit from blk_mean relative to mu_k, for callers that write blk_mean
@@ -240,10 +272,12 @@ SA_API sa_status sa_block_sketch(const sa_shape* shape, const void* blk_mean, co
 
 /* Selection of one decode step for every unit: block scores, exact top-k by
  * (score desc, block index asc) on the exact score rounded once to fp64, and
- * the tail draws for sampling.  The scan reads the int8 sketch (integer dot
- * products with an int8 copy of the group query) and bounds each score's
- * error; every candidate whose interval reaches the k-th best lower bound is
- * rescored exactly from blk_mean.  k and v are read only for the CLT base sample (may be NULL
+ * the tail draws for sampling.  With SA_SCORE_MEAN_SUM the scan reads the
+ * int8 sketch (integer dot products with an int8 copy of the group query)
+ * and bounds each score's error; every candidate whose interval reaches the
+ * k-th best lower bound is rescored exactly from blk_mean.  The other scores
+ * scan blk_mean (or blk_min and blk_max) in fp32 with the same certified
+ * intervals and exact rescoring of the band.  k and v are read only for the CLT base sample (may be NULL
  * when clt_base == 0). */
 SA_API sa_status sa_select(const sa_shape* shape, const sa_select_params* params, const void* q,
                     const sa_stats* stats, const void* k, const void* v,

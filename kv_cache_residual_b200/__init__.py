@@ -25,6 +25,7 @@ LIB_PATH = os.path.join(_HERE, "libsa_b200.so")
 SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_CUDA = range(5)
 SA_F32, SA_BF16 = 0, 1
 MODES = {"drop": 0, "resa": 1, "proxy": 2, "sample": 3}
+SCORES = {"mean_sum": 0, "mean_max": 1, "quest": 2}
 OP_PREFILL, OP_SELECT, OP_DECODE, OP_DENSE, OP_STEP = range(5)
 
 
@@ -42,14 +43,14 @@ class sa_shape(ctypes.Structure):
 class sa_stats(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("mu_q", "o_est", "log_z0", "mu_k", "sum_k", "sum_v", "blk_mean", "kbar_absmax", "blk_code",
-                 "blk_meta")]
+                 "blk_meta", "blk_min", "blk_max")]
 
 
 class sa_select_params(ctypes.Structure):
     _fields_ = [("sink", ctypes.c_int), ("local", ctypes.c_int), ("k_blocks", ctypes.c_int),
                 ("sample_b", ctypes.c_int), ("clt_base", ctypes.c_int), ("sample_cap", ctypes.c_int),
                 ("eps", ctypes.c_float), ("delta", ctypes.c_float), ("seed", ctypes.c_uint64),
-                ("step", ctypes.c_int)]
+                ("step", ctypes.c_int), ("score", ctypes.c_int)]
 
 
 class sa_selection(ctypes.Structure):
@@ -60,7 +61,8 @@ class sa_decode_params(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int), ("lam", ctypes.c_float), ("scale", ctypes.c_float)]
 
 
-EXPORTS = ("sa_workspace_size", "sa_prefill_stats", "sa_block_summaries", "sa_block_sketch", "sa_select",
+EXPORTS = ("sa_workspace_size", "sa_prefill_stats", "sa_block_summaries", "sa_block_sketch", "sa_block_minmax",
+           "sa_select",
            "sa_select_noalloc",
            "sa_decode", "sa_step", "sa_dense_decode", "sa_append", "sa_wait_timeouts",
            "sa_status_string")
@@ -83,6 +85,7 @@ def _lib():
         lib.sa_prefill_stats.argtypes = [sh, P, P, P, st, F, P, S, P]
         lib.sa_block_summaries.argtypes = [sh, P, I, I, P, P, P, P, P, P]
         lib.sa_block_sketch.argtypes = [sh, P, P, I, I, P, P, P]
+        lib.sa_block_minmax.argtypes = [sh, P, I, I, P, P, P]
         lib.sa_select.argtypes = [sh, sp, P, st, P, P, sel, F, P, S, P]
         lib.sa_select_noalloc.argtypes = [sh, sp, P, st, P, P, sel, F, P]
         lib.sa_decode.argtypes = [sh, dp, sp, P, P, P, st, sel, P, P, S, P]
@@ -93,7 +96,7 @@ def _lib():
         lib.sa_wait_timeouts.restype = I
         lib.sa_status_string.argtypes = [I]
         lib.sa_status_string.restype = ctypes.c_char_p
-        for f in ("sa_prefill_stats", "sa_block_summaries", "sa_block_sketch", "sa_select", "sa_select_noalloc", "sa_decode", "sa_step",
+        for f in ("sa_prefill_stats", "sa_block_summaries", "sa_block_sketch", "sa_block_minmax", "sa_select", "sa_select_noalloc", "sa_decode", "sa_step",
                   "sa_dense_decode", "sa_append"):
             getattr(lib, f).restype = I
         _LIB = lib
@@ -141,20 +144,21 @@ class SelectParams:
     delta: float = 0.05
     seed: int = 0
     step: int = 0
+    score: str = "mean_sum"          # block score: "mean_sum", "mean_max" or "quest"
 
     def c(self):
         return sa_select_params(self.sink, self.local, self.k_blocks, self.sample_b, self.clt_base,
                                 max(self.sample_cap, self.sample_b), self.eps, self.delta,
-                                self.seed & ((1 << 64) - 1), self.step)
+                                self.seed & ((1 << 64) - 1), self.step, SCORES[self.score])
 
 
 class Stats:
     """Prefill-end statistics (caller-owned device tensors)."""
 
     FIELDS = ("mu_q", "o_est", "log_z0", "mu_k", "sum_k", "sum_v", "blk_mean", "kbar_absmax", "blk_code",
-              "blk_meta")
+              "blk_meta", "blk_min", "blk_max")
 
-    def __init__(self, B, Hq, Hkv, L, d, dtype, device):
+    def __init__(self, B, Hq, Hkv, L, d, dtype, device, minmax=False):
         f = dict(dtype=torch.float32, device=device)
         self.mu_q = torch.empty(B, Hq, d, **f)
         self.o_est = torch.empty(B, Hq, d, **f)
@@ -167,9 +171,13 @@ class Stats:
         # scan sketch of blk_mean (int8 codes + {scale, residual norm, norm, 0})
         self.blk_code = torch.empty(B, Hkv, L // 16, d, dtype=torch.int8, device=device)
         self.blk_meta = torch.empty(B, Hkv, L // 16, 4, **f)
+        # per-block key minimum and maximum (the "quest" block score), on request
+        self.blk_min = torch.empty(B, Hkv, L // 16, d, dtype=dtype, device=device) if minmax else None
+        self.blk_max = torch.empty(B, Hkv, L // 16, d, dtype=dtype, device=device) if minmax else None
 
     def c(self):
-        return sa_stats(*[self.__dict__[n].data_ptr() for n in self.FIELDS])
+        return sa_stats(*[None if self.__dict__.get(n) is None else self.__dict__[n].data_ptr()
+                          for n in self.FIELDS])
 
 
 class Selection:
@@ -204,14 +212,15 @@ def workspace(shape, params, op, device):
     return ws
 
 
-def prefill_stats(q_ctx, k, v, stats=None, scale=0.0, stream=None):
+def prefill_stats(q_ctx, k, v, stats=None, scale=0.0, stream=None, minmax=False):
     """Statistics of the first L = q_ctx.shape[2] tokens of a cache k, v
-    [B, Hkv, ld, d] (ld >= L: room for appended tokens)."""
+    [B, Hkv, ld, d] (ld >= L: room for appended tokens); minmax: also the
+    per-block key bounds the "quest" block score ranks on."""
     B, Hkv, ld, d = k.shape
     Hq, L = q_ctx.shape[1], q_ctx.shape[2]
     shape = make_shape(k, Hq, L)
     if stats is None:
-        stats = Stats(B, Hq, Hkv, ld, d, k.dtype, k.device)
+        stats = Stats(B, Hq, Hkv, ld, d, k.dtype, k.device, minmax=minmax)
     ws = workspace(shape, None, OP_PREFILL, k.device)
     st = stats.c()
     _check(_lib().sa_prefill_stats(ctypes.byref(shape), _ptr(q_ctx), _ptr(k), _ptr(v), ctypes.byref(st),
@@ -225,6 +234,14 @@ def block_summaries(k, blk_begin, blk_end, stats, Hq, length=None, stream=None):
                                      _ptr(stats.blk_mean), _ptr(stats.kbar_absmax), _ptr(stats.mu_k),
                                      _ptr(stats.blk_code), _ptr(stats.blk_meta), _stream(stream)),
            "sa_block_summaries")
+
+
+def block_minmax(k, blk_begin, blk_end, stats, Hq, length=None, stream=None):
+    """Key minimum and maximum of blocks [blk_begin, blk_end) of every unit into
+    stats.blk_min / stats.blk_max (see sa_block_minmax)."""
+    shape = make_shape(k, Hq, length)
+    _check(_lib().sa_block_minmax(ctypes.byref(shape), _ptr(k), int(blk_begin), int(blk_end), _ptr(stats.blk_min),
+                                  _ptr(stats.blk_max), _stream(stream)), "sa_block_minmax")
 
 
 def block_sketch(stats, Hq, blk_begin=0, blk_end=None, stream=None):

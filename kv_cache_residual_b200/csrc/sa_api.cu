@@ -41,6 +41,8 @@ sa_status check_select_params(const sa_select_params* p) {
         p->clt_base < 0)
         return SA_ERR_INVALID_ARG;
     if (p->sample_b > p->sample_cap) return SA_ERR_INVALID_ARG;
+    if (p->score != SA_SCORE_MEAN_SUM && p->score != SA_SCORE_MEAN_MAX && p->score != SA_SCORE_QUEST)
+        return SA_ERR_INVALID_ARG;
     if (p->clt_base > 0) {
         if (p->clt_base < 2 || p->clt_base > p->sample_cap) return SA_ERR_INVALID_ARG;
         if (!(p->eps > 0.f) || !(p->delta > 0.f && p->delta < 1.f)) return SA_ERR_INVALID_ARG;
@@ -51,6 +53,9 @@ sa_status check_select_params(const sa_select_params* p) {
 
 bool check_stats(const sa_stats* st, bool need_all) {
     if (st == nullptr) return false;
+    // the block bounds come as a pair, or not at all
+    if ((st->blk_min == nullptr) != (st->blk_max == nullptr)) return false;
+    if (st->blk_min != nullptr && (!aligned16(st->blk_min) || !aligned16(st->blk_max))) return false;
     if (!aligned16(st->blk_mean) || !aligned4(st->kbar_absmax) || !aligned16(st->blk_code) ||
         !aligned16(st->blk_meta))
         return false;
@@ -152,6 +157,21 @@ sa_status sa_append(const sa_shape* shape, const void* k_new, const void* v_new,
                : SA_ERR_CUDA;
 }
 
+sa_status sa_block_minmax(const sa_shape* shape, const void* k, int blk_begin, int blk_end, void* blk_min,
+                          void* blk_max, void* stream) {
+    NvtxRange r("sa_block_minmax");
+    Dims d;
+    sa_status e = check_shape(shape, &d);
+    if (e != SA_OK) return e;
+    if (!aligned16(k) || !aligned16(blk_min) || !aligned16(blk_max)) return SA_ERR_INVALID_ARG;
+    if (blk_begin < 0 || blk_end > d.nb() || blk_begin > blk_end) return SA_ERR_INVALID_ARG;
+    if (blk_begin == blk_end) return SA_OK;
+    return launch_block_minmax(d, k, blk_begin, blk_end, blk_min, blk_max, static_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? SA_OK
+               : SA_ERR_CUDA;
+}
+
 sa_status sa_block_sketch(const sa_shape* shape, const void* blk_mean, const float* mu_k, int blk_begin,
                           int blk_end, int8_t* blk_code, float* blk_meta, void* stream) {
     NvtxRange r("sa_block_sketch");
@@ -181,6 +201,8 @@ sa_status prep_select(const sa_shape* shape, const sa_select_params* params, con
     if (e != SA_OK) return e;
     if (!aligned16(q) || !check_stats(stats, false) || out == nullptr || scale < 0.f) return SA_ERR_INVALID_ARG;
     *p = select_plan(*d, *params);
+    if (params->score == SA_SCORE_QUEST && stats->blk_min == nullptr) return SA_ERR_INVALID_ARG;
+    if (params->score != SA_SCORE_MEAN_SUM && !select_var_ok(p->g)) return SA_ERR_UNSUPPORTED;
     if (p->g.kk > 0 && !aligned4(out->blk_idx)) return SA_ERR_INVALID_ARG;
     if (params->k_blocks > 0 && out->blk_idx == nullptr) return SA_ERR_INVALID_ARG;
     if (!aligned4(out->samp_count)) return SA_ERR_INVALID_ARG;

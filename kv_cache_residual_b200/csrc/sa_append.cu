@@ -11,7 +11,9 @@
 // When the token completes 16-token block `blk`, warp 0 then forms that
 // block's mean (fp64 sum of its 16 rows, rounded once to the cache dtype, as
 // the prefill does), raises kbar_absmax and writes the block's sketch row
-// (sketch_row, shared with the prefill's sketch kernel).
+// (sketch_row, shared with the prefill's sketch kernel).  When the statistics
+// carry per-block key bounds, a second launch forms the completed block's
+// elementwise minimum and maximum.
 #include "sa_common.cuh"
 #include "sa_internal.h"
 #include "sa_sketch.cuh"
@@ -106,7 +108,10 @@ static cudaError_t append_t(const Dims& d, const void* k_new, const void* v_new,
     k_append<T, D, G><<<d.U(), kAppendThreads, 0, s>>>(
         reinterpret_cast<const T*>(k_new), reinterpret_cast<const T*>(v_new), reinterpret_cast<T*>(k),
         reinterpret_cast<T*>(v), st, d.Hq, d.Hkv, d.L, d.ld, scale, (d.L + 1) % 16 == 0 ? (d.L + 1) / 16 - 1 : -1);
-    return cudaGetLastError();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || st.blk_min == nullptr || (d.L + 1) % 16 != 0) return e;
+    // the completed block's key bounds (after the row is written, same stream)
+    return launch_block_minmax(d, k, (d.L + 1) / 16 - 1, (d.L + 1) / 16, st.blk_min, st.blk_max, s);
 }
 
 template <typename T, int D>

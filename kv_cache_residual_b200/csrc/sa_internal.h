@@ -196,6 +196,9 @@ cudaError_t launch_prefill(const Dims& d, const PrefillPlan& p, const PrefillArg
 cudaError_t launch_block_summaries(const Dims& d, const void* k, int blk_begin, int blk_end, void* blk_mean,
                                    float* kbar_absmax, const float* centre, int8_t* blk_code, float* blk_meta,
                                    cudaStream_t s);
+// elementwise key min / max of blocks [blk_begin, blk_end) (sa_prefill.cu)
+cudaError_t launch_block_minmax(const Dims& d, const void* k, int blk_begin, int blk_end, void* blk_min,
+                                void* blk_max, cudaStream_t s);
 cudaError_t launch_block_sketch(const Dims& d, const void* blk_mean, const float* centre, int blk_begin, int blk_end,
                                 int8_t* blk_code, float* blk_meta, cudaStream_t s);
 // one token per unit at position d.L (sa_append.cu)
@@ -222,6 +225,10 @@ inline cudaError_t opt_in_smem(K kernel, size_t bytes, std::atomic<unsigned long
 }
 
 cudaError_t launch_select(const Dims& d, const SelectPlan& p, const SelectArgs& a, cudaStream_t s);
+// the alternative block scores (sa_select_var.cu): whether the shape fits
+// (candidate keys in shared memory), and the launch
+bool select_var_ok(const SetGeom& g);
+cudaError_t launch_select_var(const Dims& d, const SelectPlan& p, const SelectArgs& a, cudaStream_t s);
 // selection CTAs (on the current device) that gave up a bounded wait
 cudaError_t select_wait_timeouts(unsigned* count);
 // sa_select's argument checks alone (nothing is enqueued): SA_OK when

@@ -300,6 +300,64 @@ cudaError_t launch_block_sketch(const Dims& d, const void* bm, const float* cent
                       : sketch_t<float, 64>(d, bm, centre, b0, b1, code, meta, s);
 }
 
+// Elementwise key minimum and maximum of blocks [blk_begin, blk_end) of every
+// unit (Quest's per-block key bounds, the summaries of SA_SCORE_QUEST): one
+// thread per (block, 16-byte chunk of the row), its 16 rows read with 16-byte
+// loads.  Values of the cache, so nothing is rounded.
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads)
+k_block_minmax(const T* __restrict__ k, int ld, int blk_begin, int blk_end, T* __restrict__ bmin,
+               T* __restrict__ bmax) {
+    using Gm = Geom<T, D>;
+    constexpr int EPC = Gm::EPC, CPR = Gm::CPR;
+    const int u = blockIdx.y, nb = ld / 16;
+    const int items = (blk_end - blk_begin) * CPR;
+    for (int it = blockIdx.x * kThreads + threadIdx.x; it < items; it += gridDim.x * kThreads) {
+        const int blk = blk_begin + it / CPR, ch = it - (it / CPR) * CPR;
+        const T* src = k + ((size_t)u * ld + (size_t)blk * 16) * D + ch * EPC;
+        float mn[EPC], mx[EPC], f[EPC];
+        unpack<T>(ld_nc16(src), mn);
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) mx[e] = mn[e];
+#pragma unroll 4
+        for (int j = 1; j < 16; ++j) {
+            unpack<T>(ld_nc16(src + (size_t)j * D), f);
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) {
+                mn[e] = fminf(mn[e], f[e]);
+                mx[e] = fmaxf(mx[e], f[e]);
+            }
+        }
+        T omn[EPC], omx[EPC];
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) {
+            omn[e] = round_from_f64<T>((double)mn[e]);       // exact: a value of the cache
+            omx[e] = round_from_f64<T>((double)mx[e]);
+        }
+        const size_t o = ((size_t)u * nb + blk) * D + ch * EPC;
+        *reinterpret_cast<uint4*>(bmin + o) = pack16(omn);
+        *reinterpret_cast<uint4*>(bmax + o) = pack16(omx);
+    }
+}
+
+template <typename T, int D>
+static cudaError_t minmax_t(const Dims& d, const void* k, int b0, int b1, void* bmin, void* bmax, cudaStream_t s) {
+    using Gm = Geom<T, D>;
+    const int items = (b1 - b0) * Gm::CPR;
+    const int gx = max(1, min(cdiv(items, kThreads), cdiv(4 * kSmTarget, d.U())));
+    k_block_minmax<T, D><<<dim3(gx, d.U()), kThreads, 0, s>>>(reinterpret_cast<const T*>(k), d.ld, b0, b1,
+                                                              reinterpret_cast<T*>(bmin), reinterpret_cast<T*>(bmax));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_block_minmax(const Dims& d, const void* k, int b0, int b1, void* bmin, void* bmax,
+                                cudaStream_t s) {
+    if (d.bf16) return d.d == 128 ? minmax_t<__nv_bfloat16, 128>(d, k, b0, b1, bmin, bmax, s)
+                                  : minmax_t<__nv_bfloat16, 64>(d, k, b0, b1, bmin, bmax, s);
+    return d.d == 128 ? minmax_t<float, 128>(d, k, b0, b1, bmin, bmax, s)
+                      : minmax_t<float, 64>(d, k, b0, b1, bmin, bmax, s);
+}
+
 // ---- dispatch ------------------------------------------------------------
 
 template <typename T, int D, int G>
@@ -317,7 +375,9 @@ static cudaError_t prefill_t(const Dims& d, const PrefillPlan& p, const PrefillA
         reinterpret_cast<unsigned*>(ws + p.off_kvcnt), a.st);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    return launch_block_sketch(d, a.st.blk_mean, a.st.mu_k, 0, d.L / 16, a.st.blk_code, a.st.blk_meta, s);
+    e = launch_block_sketch(d, a.st.blk_mean, a.st.mu_k, 0, d.L / 16, a.st.blk_code, a.st.blk_meta, s);
+    if (e != cudaSuccess || a.st.blk_min == nullptr) return e;
+    return launch_block_minmax(d, a.k, 0, d.L / 16, a.st.blk_min, a.st.blk_max, s);
 }
 
 template <typename T, int D>

@@ -167,6 +167,7 @@ cudaError_t select_wait_timeouts(unsigned* count) {
 }
 
 cudaError_t launch_select(const Dims& d, const SelectPlan& p, const SelectArgs& a, cudaStream_t s) {
+    if (a.sp.score != SA_SCORE_MEAN_SUM) return launch_select_var(d, p, a, s);
     if (d.bf16) return d.d == 128 ? select_g<__nv_bfloat16, 128>(d, p, a, s) : select_g<__nv_bfloat16, 64>(d, p, a, s);
     return d.d == 128 ? select_g<float, 128>(d, p, a, s) : select_g<float, 64>(d, p, a, s);
 }

@@ -183,3 +183,33 @@ def test_workspace_grows_with_the_clt_budget(lib):
     for op in (sa.OP_SELECT, sa.OP_DECODE, sa.OP_DENSE):
         assert (lib.sa_workspace_size(ctypes.byref(sh), ctypes.byref(plain), op) ==
                 lib.sa_workspace_size(ctypes.byref(grown), ctypes.byref(plain), op))
+
+
+def test_block_score_checks(lib):
+    """An unknown score, the Quest score without the block bounds, a bound
+    pointer without its pair, and more candidates than the alternative scores
+    hold are all rejected before anything is enqueued."""
+    sh = _shape()
+    p = ctypes.c_void_p(0x10000)
+    st = sa.sa_stats(*([0x10000] * 10))                         # no blk_min / blk_max
+    st_mm = sa.sa_stats(*([0x10000] * 12))
+    st_half = sa.sa_stats(*([0x10000] * 11))                    # blk_min without blk_max
+    sel = sa.sa_selection(0x10000, 0x10000, 0x10000, 0)
+
+    def call(sp, stats, shape=sh, ws=1 << 30):
+        return lib.sa_select(ctypes.byref(shape), ctypes.byref(sp), p, ctypes.byref(stats), None, None,
+                             ctypes.byref(sel), 0.0, p, ws, None)
+
+    sp = lambda score: sa.sa_select_params(64, 128, 8, 0, 0, 0, 0.05, 0.05, 0, 0, score)
+    assert call(sp(3), st_mm) == sa.SA_ERR_INVALID_ARG
+    assert call(sp(-1), st_mm) == sa.SA_ERR_INVALID_ARG
+    assert call(sp(sa.SCORES["quest"]), st) == sa.SA_ERR_INVALID_ARG
+    assert call(sp(sa.SCORES["mean_max"]), st_half) == sa.SA_ERR_INVALID_ARG
+    big = _shape(B=1, L=16 * 20000)                              # 19988 candidates > 16384
+    assert call(sp(sa.SCORES["mean_max"]), st_mm, shape=big) == sa.SA_ERR_UNSUPPORTED
+    # accepted arguments with a workspace that is too small: the checks passed
+    assert call(sp(sa.SCORES["quest"]), st_mm, ws=64) == sa.SA_ERR_WORKSPACE
+    assert lib.sa_block_minmax(ctypes.byref(sh), p, 10, 5, p, p, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_block_minmax(ctypes.byref(sh), p, 0, 4096, p, p, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_block_minmax(ctypes.byref(sh), p, 0, 8, p, ctypes.c_void_p(0x10008), None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_block_minmax(ctypes.byref(sh), p, 3, 3, p, p, None) == sa.SA_OK
