@@ -309,3 +309,80 @@ def test_selector_variant_mistake_fails_a_pin(monkeypatch, name):
 def test_block_minmax_mistake_fails_a_pin(monkeypatch):
     monkeypatch.setattr(stats, "block_minmax", _minmax_shifted)
     assert _some_pin_fails([(pin_stats.test_block_minmax_against_loops_and_torch, {})])
+
+
+def _search_variant(eps_half=True, delta_g=1.0):
+    import oracle.budget as budget
+
+    def f_(q, k, v, idx, base_pos, scale, eps, delta, n_t):
+        b0 = len(base_pos)
+        n_hat, d_hat, e_s, r = budget._estimates(q, k, v, idx, base_pos, scale, n_t)
+        G = q.shape[0]
+        tr = [float(r[h].var(axis=0, ddof=1).sum()) for h in range(G)]
+        vd = [float(e_s[h].var(ddof=1)) for h in range(G)]
+        best = (math.inf, None, None)
+        for f in budget.GRID:
+            e1 = f * eps / 2.0 if eps_half else f * eps
+            e2 = (1.0 - f) * eps / 2.0 if eps_half else (1.0 - f) * eps
+            for g in budget.GRID:
+                d1, d2 = g * delta * delta_g, (1.0 - g) * delta * delta_g
+                b = 0.0
+                for h in range(G):
+                    b = max(b, budget.lemma_budget(n_t, tr[h], e1 * float(np.linalg.norm(n_hat[h])), d1),
+                            budget.lemma_budget(n_t, vd[h], e2 * float(d_hat[h]), d2))
+                if b < best[0]:
+                    best = (b, f, g)
+        return budget._clamp(best[0], b0, n_t), {"b_real": best[0], "f": best[1], "g": best[2]}
+    return f_
+
+
+def _hoeffding_variant(union=True, use_range=True):
+    import oracle.budget as budget
+
+    def f_(q, k, v, idx, base_pos, scale, eps, delta, n_t):
+        b0 = len(base_pos)
+        n_hat, d_hat, e_s, r = budget._estimates(q, k, v, idx, base_pos, scale, n_t)
+        G, d = q.shape[0], v.shape[1]
+        e1 = e2 = eps / 4.0
+        d1 = d2 = delta / 2.0
+        det = {"b_N": [], "b_D": []}
+        best = 0.0
+        for h in range(G):
+            if use_range:
+                rn2 = float(((r[h].max(axis=0) - r[h].min(axis=0)) ** 2).max())
+                rd2 = float((e_s[h].max() - e_s[h].min()) ** 2)
+            else:                                                   # spread by the standard deviation
+                rn2 = float(r[h].var(axis=0, ddof=1).max())
+                rd2 = float(e_s[h].var(ddof=1))
+            tn, td = e1 * float(np.linalg.norm(n_hat[h])), e2 * float(d_hat[h])
+            dd = d if union else 1
+            b_n = dd * n_t ** 2 * math.log(2.0 * dd / d1) * rn2 / (2.0 * tn ** 2)
+            b_d = n_t ** 2 * math.log(2.0 / d2) * rd2 / (2.0 * td ** 2)
+            det["b_N"].append(b_n)
+            det["b_D"].append(b_d)
+            best = max(best, b_n, b_d)
+        return budget._clamp(best, b0, n_t), det
+    return f_
+
+
+BUDGET_RULE_MISTAKES = {
+    "search: eps split not halved": ("clt_budget_search", _search_variant(eps_half=False)),
+    "search: delta halved again": ("clt_budget_search", _search_variant(delta_g=0.5)),
+    "hoeffding: no union bound over coordinates": ("hoeffding_budget", _hoeffding_variant(union=False)),
+    "hoeffding: spread instead of range": ("hoeffding_budget", _hoeffding_variant(use_range=False)),
+}
+
+
+@pytest.mark.parametrize("name", list(BUDGET_RULE_MISTAKES))
+def test_budget_rule_mistake_fails_a_pin(monkeypatch, golden_dir, name):
+    import oracle.budget as budget
+    import test_oracle_budget as pin_budget
+    pins = [(pin_budget.test_hoeffding_hand_worked_unit, {"golden_dir": golden_dir}),
+            (pin_budget.test_clt_search_against_a_continuous_optimum, {"golden_dir": golden_dir}),
+            (pin_budget.test_clt_search_corner_when_the_denominator_is_exact, {})]
+    attr, fn = BUDGET_RULE_MISTAKES[name]
+    monkeypatch.setattr(budget, attr, _search_variant() if attr == "clt_budget_search" else _hoeffding_variant())
+    for p_, kw in pins:                      # the restatements themselves pass
+        p_(**kw)
+    monkeypatch.setattr(budget, attr, fn)
+    assert _some_pin_fails(pins)
