@@ -54,6 +54,8 @@ def parse_args(argv=None):
     ap.add_argument("--clt-base", type=int, default=0,
                     help="sample mode: choose b per unit by the CLT budget from this many base draws")
     ap.add_argument("--sample-cap", type=int, default=4096, help="draw capacity per unit with --clt-base")
+    ap.add_argument("--budget", default="clt", choices=["clt", "clt_search", "hoeffding"],
+                    help="rule for b with --clt-base")
     ap.add_argument("--eps", type=float, default=0.1)
     ap.add_argument("--delta", type=float, default=0.05)
     ap.add_argument("--queries", type=int, default=64, help="distinct decode queries cycled through")
@@ -292,7 +294,9 @@ def cpu_oracle_sample(w, sp_kw, mode, seconds, max_units=None, seq=0):
             if mode == "sample" and sp_kw.get("clt_base", 0) > 0 and len(tail) > 0:
                 # the CLT budget from the base draws, then that many draws
                 base = rng.sample_positions(sp_kw["seed"], seq, g, step, tail, sp_kw["clt_base"])
-                b, _ = budget.clt_budget(q, K, V, idx, base, scale, sp_kw["eps"], sp_kw["delta"], len(tail))
+                rule = {"clt": budget.clt_budget, "clt_search": budget.clt_budget_search,
+                        "hoeffding": budget.hoeffding_budget}[sp_kw.get("budget", "clt")]
+                b, _ = rule(q, K, V, idx, base, scale, sp_kw["eps"], sp_kw["delta"], len(tail))
                 pos = rng.sample_positions(sp_kw["seed"], seq, g, step, tail, min(b, sp_kw["sample_cap"]))
             elif mode == "sample":
                 pos = rng.sample_positions(sp_kw["seed"], seq, g, step, tail, sp_kw["sample_b"])
@@ -348,7 +352,8 @@ def main(argv=None):
     sg = set_geom(w.L, w.sink, w.local, kb)
     sp_kw = dict(sink=w.sink, local=w.local, k_blocks=kb, sample_b=args.sample_b, seed=2024)
     if args.mode == "sample" and args.clt_base > 0:
-        sp_kw.update(clt_base=args.clt_base, eps=args.eps, delta=args.delta, sample_cap=args.sample_cap)
+        sp_kw.update(clt_base=args.clt_base, eps=args.eps, delta=args.delta, sample_cap=args.sample_cap,
+                     budget=args.budget)
     ws, rank, local = dist_setup(args.gpus)
     if args.impl == "reference":
         rc = run_reference(args, w, sg, sp_kw, rank)
@@ -389,7 +394,8 @@ def main(argv=None):
     bdraw = args.sample_b if args.mode == "sample" and not clt else 0
     if clt:
         sps = [sa.SelectParams(sink=w.sink, local=w.local, k_blocks=kb, sample_b=0, sample_cap=args.sample_cap,
-                               clt_base=args.clt_base, eps=args.eps, delta=args.delta, seed=2024, step=t)
+                               clt_base=args.clt_base, eps=args.eps, delta=args.delta, seed=2024, step=t,
+                               budget=args.budget)
                for t in range(nq)]
     else:
         sps = [sa.SelectParams(sink=w.sink, local=w.local, k_blocks=kb, sample_b=bdraw, sample_cap=max(bdraw, 1),
@@ -476,7 +482,7 @@ def main(argv=None):
             counts.append(s_.samp_count.double().mean().item())
         b_mean = statistics.mean(counts)
         clt_info = {"base": args.clt_base, "eps": args.eps, "delta": args.delta, "mean_b": b_mean,
-                    "cap": args.sample_cap}
+                    "cap": args.sample_cap, "rule": args.budget}
     sel_b = select_bytes_per_unit(w, sg, esz, b_mean) * w.B * w.Hkv
     if clt:
         # the budget kernel reads I and the base draws' K and V rows

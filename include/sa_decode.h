@@ -91,6 +91,26 @@ typedef enum { SA_DROP = 0, SA_RESA = 1, SA_PROXY = 2, SA_SAMPLE = 3 } sa_mode;
  * The two alternatives support up to 16384 candidate blocks per unit. */
 typedef enum { SA_SCORE_MEAN_SUM = 0, SA_SCORE_MEAN_MAX = 1, SA_SCORE_QUEST = 2 } sa_score;
 
+/* How the sampling budget b is set from the base sample when clt_base > 0
+ * ("vAttention: Verified Sparse Attention via Sampling", Method, key designs
+ * 2 and 3; the lemma b >= (Phi^-1(1 - delta_i/2) n_T sqrt(spread) / tau)^2
+ * with tau = eps1 ||N_hat|| for the numerator, eps2 D_hat for the
+ * denominator, and Lemma 4.2's 2 (eps1 + eps2) = eps, delta1 + delta2 =
+ * delta):
+ *   SA_BUDGET_CLT         even split: eps1 = eps2 = eps/4, delta1 = delta2 =
+ *                         delta/2 (the default)
+ *   SA_BUDGET_CLT_SEARCH  the split searched (Theorem 4.3's minimisation, its
+ *                         formula not printed; read as): eps1 = f eps/2,
+ *                         delta1 = g delta, f and g on {1/20, ..., 19/20}
+ *                         (eps2 < 0.5), the smallest max over heads and
+ *                         bounds, ties to the first (f, g) in order
+ *   SA_BUDGET_HOEFFDING   the conservative bound (the page's appendix
+ *                         remark), even split: b_D = n_T^2 ln(2/delta2) R_D^2
+ *                         / (2 tau_D^2), b_N = d n_T^2 ln(2d/delta1) max_e
+ *                         R_e^2 / (2 tau_N^2), R the base sample's ranges of
+ *                         the weights e and of each coordinate of e V        */
+typedef enum { SA_BUDGET_CLT = 0, SA_BUDGET_CLT_SEARCH = 1, SA_BUDGET_HOEFFDING = 2 } sa_budget;
+
 typedef enum {
     SA_OP_PREFILL = 0,   /* sa_prefill_stats */
     SA_OP_SELECT = 1,    /* sa_select        */
@@ -175,7 +195,9 @@ typedef struct {
  *                 key = out(out(out(out(seed)^b)^g)^step), draw i =
  *                 out(key + i*0x9E3779B97F4A7C15), out(x) = SplitMix64 mixer
  *                 of x + 0x9E3779B97F4A7C15; rank = ((draw>>32)*n_T)>>32
- *   score         block score, an sa_score (0 = SA_SCORE_MEAN_SUM)           */
+ *   score         block score, an sa_score (0 = SA_SCORE_MEAN_SUM)
+ *   budget        rule for b when clt_base > 0, an sa_budget (0 = the even
+ *                 CLT split)                                                  */
 typedef struct {
     int sink, local, k_blocks;
     int sample_b, clt_base, sample_cap;
@@ -183,6 +205,7 @@ typedef struct {
     uint64_t seed;
     int step;
     int score;
+    int budget;
 } sa_select_params;
 
 /* Output of sa_select, input of sa_decode (caller-allocated).

@@ -26,6 +26,7 @@ SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_CUDA = r
 SA_F32, SA_BF16 = 0, 1
 MODES = {"drop": 0, "resa": 1, "proxy": 2, "sample": 3}
 SCORES = {"mean_sum": 0, "mean_max": 1, "quest": 2}
+BUDGETS = {"clt": 0, "clt_search": 1, "hoeffding": 2}
 OP_PREFILL, OP_SELECT, OP_DECODE, OP_DENSE, OP_STEP = range(5)
 
 
@@ -50,7 +51,7 @@ class sa_select_params(ctypes.Structure):
     _fields_ = [("sink", ctypes.c_int), ("local", ctypes.c_int), ("k_blocks", ctypes.c_int),
                 ("sample_b", ctypes.c_int), ("clt_base", ctypes.c_int), ("sample_cap", ctypes.c_int),
                 ("eps", ctypes.c_float), ("delta", ctypes.c_float), ("seed", ctypes.c_uint64),
-                ("step", ctypes.c_int), ("score", ctypes.c_int)]
+                ("step", ctypes.c_int), ("score", ctypes.c_int), ("budget", ctypes.c_int)]
 
 
 class sa_selection(ctypes.Structure):
@@ -145,11 +146,13 @@ class SelectParams:
     seed: int = 0
     step: int = 0
     score: str = "mean_sum"          # block score: "mean_sum", "mean_max" or "quest"
+    budget: str = "clt"              # with clt_base > 0: "clt", "clt_search" or "hoeffding"
 
     def c(self):
         return sa_select_params(self.sink, self.local, self.k_blocks, self.sample_b, self.clt_base,
                                 max(self.sample_cap, self.sample_b), self.eps, self.delta,
-                                self.seed & ((1 << 64) - 1), self.step, SCORES[self.score])
+                                self.seed & ((1 << 64) - 1), self.step, SCORES[self.score],
+                                BUDGETS[self.budget])
 
 
 class Stats:

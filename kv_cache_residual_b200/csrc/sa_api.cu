@@ -43,6 +43,8 @@ sa_status check_select_params(const sa_select_params* p) {
     if (p->sample_b > p->sample_cap) return SA_ERR_INVALID_ARG;
     if (p->score != SA_SCORE_MEAN_SUM && p->score != SA_SCORE_MEAN_MAX && p->score != SA_SCORE_QUEST)
         return SA_ERR_INVALID_ARG;
+    if (p->budget != SA_BUDGET_CLT && p->budget != SA_BUDGET_CLT_SEARCH && p->budget != SA_BUDGET_HOEFFDING)
+        return SA_ERR_INVALID_ARG;
     if (p->clt_base > 0) {
         if (p->clt_base < 2 || p->clt_base > p->sample_cap) return SA_ERR_INVALID_ARG;
         if (!(p->eps > 0.f) || !(p->delta > 0.f && p->delta < 1.f)) return SA_ERR_INVALID_ARG;

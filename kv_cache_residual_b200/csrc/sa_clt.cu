@@ -10,11 +10,22 @@
 //   Tr Sigma = sum over dims of the unbiased variance of e V over the sample,
 //   var_D = the unbiased variance of e over the sample,
 // and applies the lemma b >= (z n_T sqrt(Tr Sigma) / tau)^2 with
-// tau = (eps/4) ||N_hat|| for the numerator and (eps/4) D_hat for the
-// denominator, z = Phi^{-1}(1 - delta/4) (eps and delta split evenly between
-// them, Lemma 4.2).  b = clamp(ceil(max over heads and both), b0,
-// min(n_T, sample_cap)); draws b0 .. b-1 of the unit's stream are appended
-// and samp_count = b.  The shift m cancels from both budgets (every term
+// tau = eps1 ||N_hat|| for the numerator and eps2 D_hat for the
+// denominator, z = Phi^{-1}(1 - delta_i/2), under one of three rules:
+//   SA_BUDGET_CLT         eps1 = eps2 = eps/4, delta1 = delta2 = delta/2 (an
+//                         even split of Lemma 4.2's 2 (eps1 + eps2) = eps);
+//   SA_BUDGET_CLT_SEARCH  the split searched (the reading of Theorem 4.3):
+//                         eps1 = f eps/2, delta1 = g delta over the grid
+//                         f, g in {1/20, ..., 19/20} (eps2 < 0.5), the
+//                         smallest max over heads and bounds, ties to the
+//                         first grid point in (f, g) order;
+//   SA_BUDGET_HOEFFDING   the conservative bound (the page's appendix
+//                         remark): b_D = n_T^2 ln(2/delta2) R_D^2 /
+//                         (2 tau_D^2), b_N = d n_T^2 ln(2d/delta1) max_e
+//                         R_e^2 / (2 tau_N^2), R the base sample's ranges of
+//                         e and of each coordinate of e V, the even split.
+// b = clamp(ceil(max over heads and both), b0, min(n_T, sample_cap)); draws
+// b0 .. b-1 of the unit's stream are appended and samp_count = b.  The shift m cancels from both budgets (every term
 // scales by e^-m), so the sums over I may be taken against any running
 // maximum and rescaled; the sample terms use m = the maximum logit over I and
 // the sample.  All of it in fp64.
@@ -39,8 +50,8 @@ constexpr int kCltBlkCache = 2048;              // chosen blocks staged for the 
 
 // Shared layout (doubles unless noted): q [G][D], per-warp token weights
 // e [W][32][G], per-warp state m, S [2][W][G], per-warp sums [W][G][D], the
-// sample weights [G][kCltMaxSamples], vectors NS, DV [2][G][D], head values
-// [8][G]; then the budget (int).
+// sample weights [G][kCltMaxSamples], vectors NS, DV, range [3][G][D], head
+// values [12][G], the grid search's per-warp minima [2][W]; then the budget.
 template <int D, int G>
 struct CltSmem {
     static constexpr size_t kQ = 0;
@@ -49,8 +60,8 @@ struct CltSmem {
     static constexpr size_t kN = kMS + (size_t)2 * kWarps * G;
     static constexpr size_t kEs = kN + (size_t)kWarps * G * D;
     static constexpr size_t kVec = kEs + (size_t)G * kCltMaxSamples;
-    static constexpr size_t kHead = kVec + (size_t)2 * G * D;
-    static constexpr size_t kDoubles = kHead + (size_t)8 * G;
+    static constexpr size_t kHead = kVec + (size_t)3 * G * D;
+    static constexpr size_t kDoubles = kHead + (size_t)12 * G + 2 * kWarps;
     static constexpr size_t kBytes = kDoubles * 8 + 16;           // + the budget (int)
 };
 
@@ -109,6 +120,7 @@ struct CltIo {
     int32_t* samp_count;
     int sample_cap, b0;
     double eps, delta, scale;
+    int rule;                     // sa_budget
     unsigned long long seed;
     int step;
     int nsc, chunk, rec;          // splits per unit, I tokens per split, doubles per split record
@@ -136,6 +148,7 @@ k_clt(CltIo io) {
     double (*s_es)[kCltMaxSamples] = reinterpret_cast<double (*)[kCltMaxSamples]>(smd + SM::kEs);
     double (*s_vec)[G][D] = reinterpret_cast<double (*)[G][D]>(smd + SM::kVec);
     double (*s_hd)[G] = reinterpret_cast<double (*)[G]>(smd + SM::kHead);
+    double* s_gmin = smd + SM::kHead + 12 * G;        // [2][kWarps]: grid minimum, its index
 
     const int u = blockIdx.y, split = blockIdx.x;
     const int b = u / io.Hkv, g = u - b * io.Hkv;
@@ -325,12 +338,16 @@ k_clt(CltIo io) {
         for (int j = 0; j < b0; ++j) a = fma(s_es[h][j], (double)to_f32<T>(s_vs[(size_t)j * D + dim]), a);
         s_vec[0][h][dim] = a;
         const double mean = a / b0;
-        double dv = 0.0;
+        double dv = 0.0, hi = -INFINITY, lo = INFINITY;
         for (int j = 0; j < b0; ++j) {
-            const double dl = s_es[h][j] * (double)to_f32<T>(s_vs[(size_t)j * D + dim]) - mean;
+            const double r = s_es[h][j] * (double)to_f32<T>(s_vs[(size_t)j * D + dim]);
+            const double dl = r - mean;
             dv = fma(dl, dl, dv);
+            hi = fmax(hi, r);
+            lo = fmin(lo, r);
         }
         s_vec[1][h][dim] = dv;
+        s_vec[2][h][dim] = hi - lo;                   // the Hoeffding range of this coordinate
     }
     // sum and unbiased variance of e over the sample (two passes), one warp per head
     for (int h = warp; h < G; h += kWarps) {
@@ -339,50 +356,112 @@ k_clt(CltIo io) {
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
         const double mean = a / b0;
-        double ss = 0.0;
+        double ss = 0.0, hi = -INFINITY, lo = INFINITY;
         for (int j = lane; j < b0; j += 32) {
             const double dl = s_es[h][j] - mean;
             ss = fma(dl, dl, ss);
+            hi = fmax(hi, s_es[h][j]);
+            lo = fmin(lo, s_es[h][j]);
         }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        for (int off = 16; off > 0; off >>= 1) {
+            ss += __shfl_xor_sync(0xffffffffu, ss, off);
+            hi = fmax(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+            lo = fmin(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+        }
         if (lane == 0) {
             s_hd[3][h] = a;
             s_hd[4][h] = ss / (b0 - 1);
+            s_hd[6][h] = hi - lo;                     // the Hoeffding range of e
         }
     }
     __syncthreads();
 
-    // the budget: one warp per head, then the maximum over heads
+    // per head: ||N_hat||, D_hat, Tr Sigma and the largest squared coordinate
+    // range (one warp per head)
     const double ratio = (double)nt / (double)b0;
-    const double tau_scale = io.eps / 4.0;
-    const double z = normcdfinv(1.0 - io.delta / 4.0);  // two-sided quantile at delta/2
     for (int h = warp; h < G; h += kWarps) {
         const double rI = exp_shift(s_hd[0][h], s_hd[2][h]);   // I's sums from their max to m
-        double nn = 0.0, tr = 0.0;
+        double nn = 0.0, tr = 0.0, rn2 = 0.0;
         for (int e = lane; e < D; e += 32) {
             const double x = s_n[0][h][e] * rI + ratio * s_vec[0][h][e];
             nn = fma(x, x, nn);
             tr += s_vec[1][h][e];
+            rn2 = fmax(rn2, s_vec[2][h][e] * s_vec[2][h][e]);
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
             nn += __shfl_xor_sync(0xffffffffu, nn, off);
             tr += __shfl_xor_sync(0xffffffffu, tr, off);
+            rn2 = fmax(rn2, __shfl_xor_sync(0xffffffffu, rn2, off));
         }
-        tr /= (b0 - 1);
         if (lane == 0) {
-            const double dh = s_hd[1][h] * rI + ratio * s_hd[3][h];
-            const double tn = tau_scale * sqrt(nn), td = tau_scale * dh;
-            const double bn = tn > 0.0 ? z * (double)nt * sqrt(fmax(tr, 0.0)) / tn : INFINITY;
-            const double bd = td > 0.0 ? z * (double)nt * sqrt(fmax(s_hd[4][h], 0.0)) / td : INFINITY;
-            s_hd[5][h] = fmax(bn * bn, bd * bd);
+            s_hd[7][h] = sqrt(nn);                                   // ||N_hat||
+            s_hd[8][h] = s_hd[1][h] * rI + ratio * s_hd[3][h];       // D_hat
+            s_hd[9][h] = tr / (b0 - 1);                              // Tr Sigma
+            s_hd[10][h] = rn2;
         }
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
+    // the lemma's b for one estimate: (z(delta_i) n_T sqrt(spread) / tau)^2
+    auto lemma = [&](double spread, double tau, double di) -> double {
+        if (!(tau > 0.0)) return INFINITY;
+        const double x = normcdfinv(1.0 - di / 2.0) * (double)nt * sqrt(fmax(spread, 0.0)) / tau;
+        return x * x;
+    };
+    __shared__ double s_best;
+    if (io.rule == SA_BUDGET_CLT_SEARCH) {
+        // one thread per grid point (f, g); the smallest budget, first point on ties
+        double bv = INFINITY;
+        int bi = 0x7fffffff;
+        for (int pnt = threadIdx.x; pnt < 19 * 19; pnt += kThreads) {
+            const double f = (double)(pnt / 19 + 1) / 20.0, gg = (double)(pnt % 19 + 1) / 20.0;
+            const double e1 = f * io.eps / 2.0, e2 = (1.0 - f) * io.eps / 2.0;
+            if (e2 >= 0.5) continue;
+            const double d1 = gg * io.delta, d2 = (1.0 - gg) * io.delta;
+            double b = 0.0;
+            for (int h = 0; h < G; ++h)
+                b = fmax(b, fmax(lemma(s_hd[9][h], e1 * s_hd[7][h], d1), lemma(s_hd[4][h], e2 * s_hd[8][h], d2)));
+            if (b < bv) { bv = b; bi = pnt; }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const double ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+            if (ov < bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+        }
+        if (lane == 0) {
+            s_gmin[warp] = bv;
+            s_gmin[kWarps + warp] = (double)bi;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            double v = INFINITY, vi = 1e30;
+            for (int w = 0; w < kWarps; ++w)
+                if (s_gmin[w] < v || (s_gmin[w] == v && s_gmin[kWarps + w] < vi)) { v = s_gmin[w]; vi = s_gmin[kWarps + w]; }
+            s_best = v;
+        }
+    } else if (threadIdx.x == 0) {
+        const double e1 = io.eps / 4.0, d1 = io.delta / 2.0;        // the even split, both estimates
         double best = 0.0;
-        for (int h = 0; h < G; ++h) best = fmax(best, s_hd[5][h]);
+        for (int h = 0; h < G; ++h) {
+            double bn, bd;
+            if (io.rule == SA_BUDGET_HOEFFDING) {
+                const double tn = e1 * s_hd[7][h], td = e1 * s_hd[8][h];
+                const double dd = (double)D, n2 = (double)nt * (double)nt;
+                bn = tn > 0.0 ? dd * n2 * log(2.0 * dd / d1) * s_hd[10][h] / (2.0 * (tn * tn)) : INFINITY;
+                bd = td > 0.0 ? n2 * log(2.0 / d1) * (s_hd[6][h] * s_hd[6][h]) / (2.0 * (td * td)) : INFINITY;
+            } else {
+                bn = lemma(s_hd[9][h], e1 * s_hd[7][h], d1);
+                bd = lemma(s_hd[4][h], e1 * s_hd[8][h], d1);
+            }
+            best = fmax(best, fmax(bn, bd));
+        }
+        s_best = best;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const double best = s_best;
         const int hi = min(nt, io.sample_cap);
         int bb;
         if (!(best < (double)hi)) bb = hi;                       // also inf / nan
@@ -442,6 +521,7 @@ static cudaError_t clt_t(const Dims& d, const SelectPlan& p, const SelectArgs& a
     io.samp_idx = a.sel.samp_idx; io.samp_count = a.sel.samp_count;
     io.sample_cap = a.sp.sample_cap; io.b0 = a.sp.clt_base;
     io.eps = (double)a.sp.eps; io.delta = (double)a.sp.delta; io.scale = (double)a.scale;
+    io.rule = a.sp.budget;
     io.seed = (unsigned long long)a.sp.seed; io.step = a.sp.step;
     io.nsc = p.nsc; io.chunk = p.clt_chunk; io.rec = p.clt_rec;
     io.part = reinterpret_cast<double*>(a.ws + p.off_clt);

@@ -213,3 +213,15 @@ def test_block_score_checks(lib):
     assert lib.sa_block_minmax(ctypes.byref(sh), p, 0, 4096, p, p, None) == sa.SA_ERR_INVALID_ARG
     assert lib.sa_block_minmax(ctypes.byref(sh), p, 0, 8, p, ctypes.c_void_p(0x10008), None) == sa.SA_ERR_INVALID_ARG
     assert lib.sa_block_minmax(ctypes.byref(sh), p, 3, 3, p, p, None) == sa.SA_OK
+
+
+def test_budget_rule_checks(lib):
+    sh = _shape()
+    p = ctypes.c_void_p(0x10000)
+    st = sa.sa_stats(*([0x10000] * 10))
+    sel = sa.sa_selection(0x10000, 0x10000, 0x10000, 0)
+    for rule, status in ((3, sa.SA_ERR_INVALID_ARG), (-1, sa.SA_ERR_INVALID_ARG),
+                         (sa.BUDGETS["hoeffding"], sa.SA_ERR_WORKSPACE), (sa.BUDGETS["clt_search"], sa.SA_ERR_WORKSPACE)):
+        sp = sa.sa_select_params(64, 128, 8, 0, 64, 512, 0.05, 0.05, 0, 0, 0, rule)
+        assert lib.sa_select(ctypes.byref(sh), ctypes.byref(sp), p, ctypes.byref(st), p, p, ctypes.byref(sel), 0.0,
+                             p, 64, None) == status

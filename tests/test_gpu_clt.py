@@ -18,10 +18,22 @@ from parity_util import REL_L2_OUT, OracleUnit, f64, rel_l2
 pytestmark = pytest.mark.gpu
 
 
-def _check_units(w, data, st, units, kb, eps, delta, b0, cap, step=1):
+ORACLE_RULE = {"clt": obudget.clt_budget, "clt_search": obudget.clt_budget_search,
+               "hoeffding": obudget.hoeffding_budget}
+
+
+def _real_budget(rule, det):
+    if rule == "clt_search":
+        return det["b_real"]
+    return max(max(det["b_N"]), max(det["b_D"]))
+
+
+def _check_units(w, data, st, units, kb, eps, delta, b0, cap, step=1, rule="clt"):
     q = data["q"][step]
     sp = sa.SelectParams(sink=w.sink, local=w.local, k_blocks=kb, sample_b=0, sample_cap=cap, clt_base=b0,
-                         eps=eps, delta=delta, seed=4321, step=step)
+                         eps=eps, delta=delta, seed=4321, step=step, budget=rule)
+    # the kernel sees eps and delta as fp32 values: the oracle gets the same
+    eps, delta = float(np.float32(eps)), float(np.float32(delta))
     out, sel = sa.step(q, data["k"], data["v"], st, sp, mode="sample")
     torch.cuda.synchronize()
     counts = sel.samp_count.cpu().numpy()
@@ -31,11 +43,11 @@ def _check_units(w, data, st, units, kb, eps, delta, b0, cap, step=1):
         blocks, idx, tail = o.select(qq, sp)
         np.testing.assert_array_equal(sel.blk_idx[b, g].cpu().numpy()[:len(blocks)], blocks)
         base = o.draws(tail, sp, b0)
-        want, det = obudget.clt_budget(qq, o.k, o.v, idx, base, o.scale, eps, delta, len(tail))
+        want, det = ORACLE_RULE[rule](qq, o.k, o.v, idx, base, o.scale, eps, delta, len(tail))
         want = min(want, cap)
         got = int(counts[b, g])
         if got != want:
-            best = max(max(det["b_N"]), max(det["b_D"]))
+            best = _real_budget(rule, det)
             assert math.isfinite(best) and abs(best - round(best)) <= 1e-9 * best, (b, g, got, want, best)
         pos = o.draws(tail, sp, got)
         np.testing.assert_array_equal(sel.samp_idx[b, g].cpu().numpy()[:got], pos)
@@ -56,6 +68,33 @@ def test_clt_budget_small(read):
     for eps, delta in ((0.2, 0.05), (0.5, 0.2)):
         counts = _check_units(w, data, st, units, kb, eps, delta, b0=64, cap=4096)
         assert (counts >= 64).all()
+
+
+@pytest.mark.parametrize("rule", ["clt_search", "hoeffding"])
+def test_budget_rules(rule):
+    """The searched split (Theorem 4.3 reading) and the Hoeffding bound:
+    every unit's b equals the oracle's, and the draws and outputs follow."""
+    w = synth.scaled(synth.WORKLOADS["flat"], B=2, Hq=8, Hkv=2, L=8192, seed=41)
+    dev = torch.device("cuda")
+    data = synth.make_batch(w, device=dev, steps=2)
+    st = sa.prefill_stats(data["q_ctx"], data["k"], data["v"])
+    units = [(b, g) for b in range(w.B) for g in range(w.Hkv)]
+    for eps, delta in ((0.3, 0.05), (0.8, 0.2)):
+        counts = _check_units(w, data, st, units, w.k_blocks_for(0.02), eps, delta, b0=64, cap=8192, rule=rule)
+        assert (counts >= 64).all()
+
+
+def test_search_never_above_the_even_split():
+    w = synth.scaled(synth.WORKLOADS["flat"], B=4, Hq=16, Hkv=4, L=8192, seed=42)
+    dev = torch.device("cuda")
+    data = synth.make_batch(w, device=dev, steps=2)
+    st = sa.prefill_stats(data["q_ctx"], data["k"], data["v"])
+    res = {}
+    for rule in ("clt", "clt_search"):
+        sp = sa.SelectParams(sink=w.sink, local=w.local, k_blocks=w.k_blocks_for(0.02), sample_cap=8192,
+                             clt_base=64, eps=1.5, delta=0.05, seed=1, step=0, budget=rule)
+        res[rule] = sa.select(data["q"][0], st, sp, k=data["k"], v=data["v"]).samp_count.cpu()
+    assert (res["clt_search"] <= res["clt"]).all() and (res["clt_search"] < res["clt"]).any()
 
 
 def test_clt_budget_capped():
