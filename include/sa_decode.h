@@ -197,7 +197,15 @@ typedef struct {
  *                 of x + 0x9E3779B97F4A7C15; rank = ((draw>>32)*n_T)>>32
  *   score         block score, an sa_score (0 = SA_SCORE_MEAN_SUM)
  *   budget        rule for b when clt_base > 0, an sa_budget (0 = the even
- *                 CLT split)                                                  */
+ *                 CLT split)
+ *   per_head      0: one draw stream and one budget per KV head, shared by
+ *                 its query heads; 1: one per query head (the vAttention
+ *                 page samples and budgets per head): query head hq of
+ *                 sequence b draws from the stream of (seed, b, hq, step),
+ *                 its budget from its own base sample, and the decode
+ *                 weights each head's draws by n_T / b_hq for that head
+ *                 alone; sa_selection's samp_idx / samp_count then have
+ *                 B * Hq rows                                                 */
 typedef struct {
     int sink, local, k_blocks;
     int sample_b, clt_base, sample_cap;
@@ -206,13 +214,16 @@ typedef struct {
     int step;
     int score;
     int budget;
+    int per_head;
 } sa_select_params;
 
 /* Output of sa_select, input of sa_decode (caller-allocated).
  *   blk_idx     [B, Hkv, k_blocks] int32: chosen block indices, ascending;
  *               min(k_blocks, n_cand) valid entries per unit, rest = -1
- *   samp_idx    [B, Hkv, sample_cap] int32: drawn token positions (draw order)
- *   samp_count  [B, Hkv] int32: draws per unit (0 unless sampling)
+ *   samp_idx    [B, Hkv, sample_cap] int32 ([B, Hq, sample_cap] with
+ *               per_head): drawn token positions (draw order)
+ *   samp_count  [B, Hkv] int32 ([B, Hq] with per_head): draws per stream
+ *               (0 unless sampling)
  *   n_rescored  [B, Hkv] int32 or NULL: candidates whose sketch interval
  *               reached the k-th best lower bound and were rescored exactly
  *               (0 when the sketch alone decided; diagnostic)                */

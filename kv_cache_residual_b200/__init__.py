@@ -51,7 +51,8 @@ class sa_select_params(ctypes.Structure):
     _fields_ = [("sink", ctypes.c_int), ("local", ctypes.c_int), ("k_blocks", ctypes.c_int),
                 ("sample_b", ctypes.c_int), ("clt_base", ctypes.c_int), ("sample_cap", ctypes.c_int),
                 ("eps", ctypes.c_float), ("delta", ctypes.c_float), ("seed", ctypes.c_uint64),
-                ("step", ctypes.c_int), ("score", ctypes.c_int), ("budget", ctypes.c_int)]
+                ("step", ctypes.c_int), ("score", ctypes.c_int), ("budget", ctypes.c_int),
+                ("per_head", ctypes.c_int)]
 
 
 class sa_selection(ctypes.Structure):
@@ -147,12 +148,13 @@ class SelectParams:
     step: int = 0
     score: str = "mean_sum"          # block score: "mean_sum", "mean_max" or "quest"
     budget: str = "clt"              # with clt_base > 0: "clt", "clt_search" or "hoeffding"
+    per_head: bool = False           # draws and budget per query head (not per KV head)
 
     def c(self):
         return sa_select_params(self.sink, self.local, self.k_blocks, self.sample_b, self.clt_base,
                                 max(self.sample_cap, self.sample_b), self.eps, self.delta,
                                 self.seed & ((1 << 64) - 1), self.step, SCORES[self.score],
-                                BUDGETS[self.budget])
+                                BUDGETS[self.budget], int(bool(self.per_head)))
 
 
 class Stats:
@@ -184,13 +186,15 @@ class Stats:
 
 
 class Selection:
-    """Output of select(): chosen blocks and tail draws per unit."""
+    """Output of select(): chosen blocks per unit and tail draws per unit (or,
+    with per-head sampling, per query head: draw_rows = Hq)."""
 
-    def __init__(self, B, Hkv, k_blocks, sample_cap, device):
+    def __init__(self, B, Hkv, k_blocks, sample_cap, device, draw_rows=None):
         i = dict(dtype=torch.int32, device=device)
+        rows = Hkv if draw_rows is None else draw_rows
         self.blk_idx = torch.empty(B, Hkv, max(k_blocks, 1), **i)
-        self.samp_idx = torch.empty(B, Hkv, max(sample_cap, 1), **i)
-        self.samp_count = torch.zeros(B, Hkv, **i)
+        self.samp_idx = torch.empty(B, rows, max(sample_cap, 1), **i)
+        self.samp_count = torch.zeros(B, rows, **i)
         self.n_rescored = torch.zeros(B, Hkv, **i)
 
     def c(self):
@@ -266,7 +270,8 @@ def select(q, stats, params, k=None, v=None, selection=None, scale=0.0, length=N
     shape = sa_shape(B, Hq, Hkv, d, ld if length is None else int(length), _dtype_code(q), ld)
     cp = params.c()
     if selection is None:
-        selection = Selection(B, Hkv, params.k_blocks, cp.sample_cap, q.device)
+        selection = Selection(B, Hkv, params.k_blocks, cp.sample_cap, q.device,
+                              draw_rows=Hq if params.per_head else None)
     ws = workspace(shape, cp, OP_SELECT, q.device)
     st = stats.c()
     sel = selection.c()
@@ -303,7 +308,8 @@ def step(q, k, v, stats, params, mode="resa", lam=1.0, scale=0.0, selection=None
     cp = params.c()
     dp = sa_decode_params(MODES[mode], float(lam), float(scale))
     if selection is None:
-        selection = Selection(B, shape.Hkv, params.k_blocks, cp.sample_cap, q.device)
+        selection = Selection(B, shape.Hkv, params.k_blocks, cp.sample_cap, q.device,
+                              draw_rows=Hq if params.per_head else None)
     if out is None:
         out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
     ws = workspace(shape, cp, OP_STEP, q.device)
@@ -331,8 +337,8 @@ class PreparedStep:
         self.shape = make_shape(k, Hq, length)
         self.cp = params.c()
         self.dp = sa_decode_params(MODES[mode], float(lam), float(scale))
-        self.selection = selection if selection is not None else Selection(B, Hkv, params.k_blocks,
-                                                                           self.cp.sample_cap, k.device)
+        self.selection = selection if selection is not None else Selection(
+            B, Hkv, params.k_blocks, self.cp.sample_cap, k.device, draw_rows=Hq if params.per_head else None)
         self.ws = workspace(self.shape, self.cp, OP_STEP, k.device)
         self._st = stats.c()
         self._sel = self.selection.c()

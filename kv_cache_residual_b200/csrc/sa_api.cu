@@ -45,6 +45,7 @@ sa_status check_select_params(const sa_select_params* p) {
         return SA_ERR_INVALID_ARG;
     if (p->budget != SA_BUDGET_CLT && p->budget != SA_BUDGET_CLT_SEARCH && p->budget != SA_BUDGET_HOEFFDING)
         return SA_ERR_INVALID_ARG;
+    if (p->per_head != 0 && p->per_head != 1) return SA_ERR_INVALID_ARG;
     if (p->clt_base > 0) {
         if (p->clt_base < 2 || p->clt_base > p->sample_cap) return SA_ERR_INVALID_ARG;
         if (!(p->eps > 0.f) || !(p->delta > 0.f && p->delta < 1.f)) return SA_ERR_INVALID_ARG;

@@ -121,6 +121,7 @@ struct CltIo {
     int sample_cap, b0;
     double eps, delta, scale;
     int rule;                     // sa_budget
+    int per_head;                 // a base sample, a budget and draws per query head
     unsigned long long seed;
     int step;
     int nsc, chunk, rec;          // splits per unit, I tokens per split, doubles per split record
@@ -296,15 +297,23 @@ k_clt(CltIo io) {
         }
         s_n[0][h][dim] = A;                           // N_I relative to M
     }
-    // the base sample's logits, one thread per draw
-    __shared__ int s_pos[kCltMaxSamples];
-    for (int i = threadIdx.x; i < b0; i += kThreads) {
+    // the base sample's logits, one thread per draw: one sample shared by the
+    // heads, or (per_head) head h's own sample, row b Hq + g G + h
+    const int ns = io.per_head ? G : 1;
+    __shared__ int s_pos[G * kCltMaxSamples];
+    for (int x = threadIdx.x; x < ns * b0; x += kThreads) {
+        const int s = x / b0, i = x - s * b0;
+        const int32_t* src = io.per_head ? io.samp_idx + ((size_t)b * io.Hq + g * G + s) * io.sample_cap : gsamp;
         double l[G];
-        const int p = __ldcg(gsamp + i);
-        s_pos[i] = p;
+        const int p = __ldcg(src + i);
+        s_pos[s * kCltMaxSamples + i] = p;
         row_logits<T, D, G>(K + (size_t)p * D, s_q, io.scale, l);
+        if (io.per_head) {
+            s_es[s][i] = l[s];
+        } else {
 #pragma unroll
-        for (int h = 0; h < G; ++h) s_es[h][i] = l[h];
+            for (int h = 0; h < G; ++h) s_es[h][i] = l[h];
+        }
     }
     __syncthreads();
     // m = the maximum logit over I and the sample (one warp per head)
@@ -321,19 +330,22 @@ k_clt(CltIo io) {
     }
     __syncthreads();
     // sample sums of e V, then the squared deviations from their mean (two
-    // passes), over the sample's value rows staged in shared memory
+    // passes), over the sample's value rows staged in shared memory (one
+    // sample at a time)
     T* s_vs = reinterpret_cast<T*>(reinterpret_cast<unsigned char*>(smd) + SM::kBytes);
+    for (int s = 0; s < ns; ++s) {
     {
         constexpr int PER = 16 / (int)sizeof(T);
         for (int x = threadIdx.x; x < b0 * (D / PER); x += kThreads) {
             const int j = x / (D / PER), c = x - j * (D / PER);
             reinterpret_cast<uint4*>(s_vs + (size_t)j * D)[c] =
-                __ldg(reinterpret_cast<const uint4*>(V + (size_t)s_pos[j] * D) + c);
+                __ldg(reinterpret_cast<const uint4*>(V + (size_t)s_pos[s * kCltMaxSamples + j] * D) + c);
         }
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < G * D; i += kThreads) {
-        const int h = i / D, dim = i - h * D;
+    const int nh = io.per_head ? 1 : G;             // heads that use this sample
+    for (int i = threadIdx.x; i < nh * D; i += kThreads) {
+        const int h = (io.per_head ? s : i / D), dim = i % D;
         double a = 0.0;
         for (int j = 0; j < b0; ++j) a = fma(s_es[h][j], (double)to_f32<T>(s_vs[(size_t)j * D + dim]), a);
         s_vec[0][h][dim] = a;
@@ -348,6 +360,8 @@ k_clt(CltIo io) {
         }
         s_vec[1][h][dim] = dv;
         s_vec[2][h][dim] = hi - lo;                   // the Hoeffding range of this coordinate
+    }
+    __syncthreads();                                  // the staged rows are rewritten by the next sample
     }
     // sum and unbiased variance of e over the sample (two passes), one warp per head
     for (int h = warp; h < G; h += kWarps) {
@@ -409,66 +423,73 @@ k_clt(CltIo io) {
         const double x = normcdfinv(1.0 - di / 2.0) * (double)nt * sqrt(fmax(spread, 0.0)) / tau;
         return x * x;
     };
-    __shared__ double s_best;
-    if (io.rule == SA_BUDGET_CLT_SEARCH) {
-        // one thread per grid point (f, g); the smallest budget, first point on ties
-        double bv = INFINITY;
-        int bi = 0x7fffffff;
-        for (int pnt = threadIdx.x; pnt < 19 * 19; pnt += kThreads) {
-            const double f = (double)(pnt / 19 + 1) / 20.0, gg = (double)(pnt % 19 + 1) / 20.0;
-            const double e1 = f * io.eps / 2.0, e2 = (1.0 - f) * io.eps / 2.0;
-            if (e2 >= 0.5) continue;
-            const double d1 = gg * io.delta, d2 = (1.0 - gg) * io.delta;
-            double b = 0.0;
-            for (int h = 0; h < G; ++h)
-                b = fmax(b, fmax(lemma(s_hd[9][h], e1 * s_hd[7][h], d1), lemma(s_hd[4][h], e2 * s_hd[8][h], d2)));
-            if (b < bv) { bv = b; bi = pnt; }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const double ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-            if (ov < bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-        }
-        if (lane == 0) {
-            s_gmin[warp] = bv;
-            s_gmin[kWarps + warp] = (double)bi;
-        }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            double v = INFINITY, vi = 1e30;
-            for (int w = 0; w < kWarps; ++w)
-                if (s_gmin[w] < v || (s_gmin[w] == v && s_gmin[kWarps + w] < vi)) { v = s_gmin[w]; vi = s_gmin[kWarps + w]; }
-            s_best = v;
-        }
-    } else if (threadIdx.x == 0) {
-        const double e1 = io.eps / 4.0, d1 = io.delta / 2.0;        // the even split, both estimates
-        double best = 0.0;
-        for (int h = 0; h < G; ++h) {
-            double bn, bd;
-            if (io.rule == SA_BUDGET_HOEFFDING) {
-                const double tn = e1 * s_hd[7][h], td = e1 * s_hd[8][h];
-                const double dd = (double)D, n2 = (double)nt * (double)nt;
-                bn = tn > 0.0 ? dd * n2 * log(2.0 * dd / d1) * s_hd[10][h] / (2.0 * (tn * tn)) : INFINITY;
-                bd = td > 0.0 ? n2 * log(2.0 / d1) * (s_hd[6][h] * s_hd[6][h]) / (2.0 * (td * td)) : INFINITY;
-            } else {
-                bn = lemma(s_hd[9][h], e1 * s_hd[7][h], d1);
-                bd = lemma(s_hd[4][h], e1 * s_hd[8][h], d1);
+    // the budget of each target: every head alone (per_head), or the group (the
+    // max over its heads)
+    __shared__ double s_best[G];
+    const int nb = io.per_head ? G : 1;
+    for (int tg = 0; tg < nb; ++tg) {
+        const int h0 = io.per_head ? tg : 0, h1 = io.per_head ? tg + 1 : G;
+        if (io.rule == SA_BUDGET_CLT_SEARCH) {
+            // one thread per grid point (f, g); the smallest budget, first point on ties
+            double bv = INFINITY;
+            int bi = 0x7fffffff;
+            for (int pnt = threadIdx.x; pnt < 19 * 19; pnt += kThreads) {
+                const double f = (double)(pnt / 19 + 1) / 20.0, gg = (double)(pnt % 19 + 1) / 20.0;
+                const double e1 = f * io.eps / 2.0, e2 = (1.0 - f) * io.eps / 2.0;
+                if (e2 >= 0.5) continue;
+                const double d1 = gg * io.delta, d2 = (1.0 - gg) * io.delta;
+                double bb = 0.0;
+                for (int h = h0; h < h1; ++h)
+                    bb = fmax(bb, fmax(lemma(s_hd[9][h], e1 * s_hd[7][h], d1), lemma(s_hd[4][h], e2 * s_hd[8][h], d2)));
+                if (bb < bv) { bv = bb; bi = pnt; }
             }
-            best = fmax(best, fmax(bn, bd));
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const double ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+                if (ov < bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+            }
+            if (lane == 0) {
+                s_gmin[warp] = bv;
+                s_gmin[kWarps + warp] = (double)bi;
+            }
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                double v = INFINITY, vi = 1e30;
+                for (int w = 0; w < kWarps; ++w)
+                    if (s_gmin[w] < v || (s_gmin[w] == v && s_gmin[kWarps + w] < vi)) { v = s_gmin[w]; vi = s_gmin[kWarps + w]; }
+                s_best[tg] = v;
+            }
+            __syncthreads();
+        } else if (threadIdx.x == 0) {
+            const double e1 = io.eps / 4.0, d1 = io.delta / 2.0;    // the even split, both estimates
+            double best = 0.0;
+            for (int h = h0; h < h1; ++h) {
+                double bn, bd;
+                if (io.rule == SA_BUDGET_HOEFFDING) {
+                    const double tn = e1 * s_hd[7][h], td = e1 * s_hd[8][h];
+                    const double dd = (double)D, n2 = (double)nt * (double)nt;
+                    bn = tn > 0.0 ? dd * n2 * log(2.0 * dd / d1) * s_hd[10][h] / (2.0 * (tn * tn)) : INFINITY;
+                    bd = td > 0.0 ? n2 * log(2.0 / d1) * (s_hd[6][h] * s_hd[6][h]) / (2.0 * (td * td)) : INFINITY;
+                } else {
+                    bn = lemma(s_hd[9][h], e1 * s_hd[7][h], d1);
+                    bd = lemma(s_hd[4][h], e1 * s_hd[8][h], d1);
+                }
+                best = fmax(best, fmax(bn, bd));
+            }
+            s_best[tg] = best;
         }
-        s_best = best;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        const double best = s_best;
+    if (threadIdx.x < nb) {
+        const double best = s_best[threadIdx.x];
         const int hi = min(nt, io.sample_cap);
         int bb;
         if (!(best < (double)hi)) bb = hi;                       // also inf / nan
         else bb = min(max((int)ceil(best), b0), hi);
-        io.samp_count[u] = bb;
-        reset_counter(io.cnt + u);
+        io.samp_count[io.per_head ? b * io.Hq + g * G + threadIdx.x : u] = bb;
     }
+    if (threadIdx.x == 0) reset_counter(io.cnt + u);
 }
 
 // Draws b0 .. b-1 of each unit's stream, b = samp_count (set by k_clt):
@@ -478,6 +499,7 @@ k_clt(CltIo io) {
 // memory when they fit).
 constexpr int kDrawsPerCta = 2048;
 
+template <int G>
 __global__ void __launch_bounds__(kThreads)
 k_clt_draws(CltIo io) {
     __shared__ int s_g[kCltBlkCache];
@@ -485,16 +507,18 @@ k_clt_draws(CltIo io) {
     const SetGeom& sg = io.sg;
     const int nt = sg.n_t, b0 = io.b0;
     if (nt == 0 || b0 < 2) return;
-    const int bb = __ldcg(io.samp_count + u);
-    const int i0 = b0 + blockIdx.x * kDrawsPerCta, i1 = min(bb, i0 + kDrawsPerCta);
-    if (i0 >= i1) return;                             // (uniform within the CTA)
     const int32_t* gblk = io.blk_idx + (size_t)u * io.kb_stride;
     const bool cached = sg.kk <= kCltBlkCache;
     if (cached)
         for (int j = threadIdx.x; j < sg.kk; j += kThreads) s_g[j] = 16 * __ldcg(gblk + j) - sg.s_eff - 16 * j;
     __syncthreads();
-    const uint64_t key = unit_key(io.seed, (uint64_t)b, (uint64_t)g, (uint64_t)io.step);
-    int32_t* out_s = io.samp_idx + (size_t)u * io.sample_cap;
+    // one stream (the unit's) or one per query head of the group
+    for (int s = 0; s < (io.per_head ? G : 1); ++s) {
+    const int row = io.per_head ? b * io.Hq + g * G + s : u;
+    const int bb = __ldcg(io.samp_count + row);
+    const int i0 = b0 + blockIdx.x * kDrawsPerCta, i1 = min(bb, i0 + kDrawsPerCta);
+    const uint64_t key = unit_key(io.seed, (uint64_t)b, (uint64_t)(io.per_head ? g * G + s : g), (uint64_t)io.step);
+    int32_t* out_s = io.samp_idx + (size_t)row * io.sample_cap;
     for (int i = i0 + threadIdx.x; i < i1; i += kThreads) {
         const int r = (int)draw_rank(key, (uint32_t)i, (uint32_t)nt);
         int lo_j = 0, hi_j = sg.kk;                           // count of chosen j with g_j <= r
@@ -504,6 +528,7 @@ k_clt_draws(CltIo io) {
             if (gj <= r) lo_j = mid + 1; else hi_j = mid;
         }
         out_s[i] = sg.s_eff + r + 16 * lo_j;
+    }
     }
 }
 
@@ -522,6 +547,7 @@ static cudaError_t clt_t(const Dims& d, const SelectPlan& p, const SelectArgs& a
     io.sample_cap = a.sp.sample_cap; io.b0 = a.sp.clt_base;
     io.eps = (double)a.sp.eps; io.delta = (double)a.sp.delta; io.scale = (double)a.scale;
     io.rule = a.sp.budget;
+    io.per_head = a.sp.per_head;
     io.seed = (unsigned long long)a.sp.seed; io.step = a.sp.step;
     io.nsc = p.nsc; io.chunk = p.clt_chunk; io.rec = p.clt_rec;
     io.part = reinterpret_cast<double*>(a.ws + p.off_clt);
@@ -530,7 +556,7 @@ static cudaError_t clt_t(const Dims& d, const SelectPlan& p, const SelectArgs& a
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int nx = io.sample_cap > io.b0 ? cdiv(io.sample_cap - io.b0, kDrawsPerCta) : 0;
-    if (nx > 0) k_clt_draws<<<dim3(nx, d.U()), kThreads, 0, s>>>(io);
+    if (nx > 0) k_clt_draws<G><<<dim3(nx, d.U()), kThreads, 0, s>>>(io);
     return cudaGetLastError();
 }
 

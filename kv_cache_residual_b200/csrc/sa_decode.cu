@@ -29,7 +29,7 @@ k_decode(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__
          const int32_t* __restrict__ blk_idx, int kb_stride, const int32_t* __restrict__ samp_idx,
          const int32_t* __restrict__ samp_count, int sample_cap, int Hq, int Hkv, int L, int ld, SetGeom sg,
          int tok, int nsd, int rec, float qscale, float scale, float lambda,
-         float* __restrict__ part, unsigned* __restrict__ cnt, float* __restrict__ out) {
+         float* __restrict__ part, unsigned* __restrict__ cnt, float* __restrict__ out, int per_head) {
     constexpr bool PRIOR = (MODE == SA_RESA);
     constexpr bool SUMS = (MODE == SA_PROXY);
     constexpr bool SAMP = (MODE == SA_SAMPLE);
@@ -53,13 +53,26 @@ k_decode(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__
     const T* qg = q + ((size_t)b * Hq + (size_t)g * G) * D;
 
     const int nt = sg.n_t;
-    const int bu = (SAMP && nt > 0) ? min(__ldg(samp_count + u), sample_cap) : 0;
+    const bool PH = SAMP && per_head != 0;
+    const int bu = (SAMP && nt > 0 && !PH) ? min(__ldg(samp_count + u), sample_cap) : 0;
     TokenMap tm;
     tm.s_eff = sg.s_eff; tm.w_eff = sg.w_eff; tm.kk = sg.kk; tm.n_i = sg.n_i; tm.win0 = L - sg.w_eff;
     tm.blk = blk_idx + (size_t)u * kb_stride;
     tm.samp = samp_idx + (size_t)u * (sample_cap > 0 ? sample_cap : 0);
     tm.lw_samp = bu > 0 ? log2f((float)nt / (float)bu) : 0.f;
-    const int n_tok = sg.n_i + bu;
+    // per-head draws: head h's list (row b Hq + g G + h) follows head h-1's,
+    // and a drawn token enters the softmax of its head alone
+    int ph_pre[G + 1];
+    float ph_lw[G];
+    ph_pre[0] = 0;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        const int bh = (PH && nt > 0) ? min(__ldg(samp_count + (size_t)b * Hq + g * G + h), sample_cap) : 0;
+        ph_pre[h + 1] = ph_pre[h] + bh;
+        ph_lw[h] = bh > 0 ? log2f((float)nt / (float)bh) : 0.f;
+    }
+    const int32_t* gsamp_ph = samp_idx + ((size_t)b * Hq + (size_t)g * G) * (sample_cap > 0 ? sample_cap : 0);
+    const int n_tok = sg.n_i + (PH ? ph_pre[G] : bu);
 
     float qv[G][EPC];
     float q0[PRIOR ? G : 1][EPC];
@@ -89,12 +102,26 @@ k_decode(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__
         uint4 wk[2], wv[2];
         float lw[2];
         bool ok[2];
+        int tag[2];
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             const int t = wt + j * GPW + gsub;
             ok[j] = t < t1;
             lw[j] = 0.f;
-            const int p = ok[j] ? tm.pos(t, lw[j]) : 0;
+            tag[j] = -1;
+            int p = 0;
+            if (ok[j] && PH && t >= sg.n_i) {
+                const int x = t - sg.n_i;
+                int h = 0;
+#pragma unroll
+                for (int y = 1; y < G; ++y) h += (x >= ph_pre[y]) ? 1 : 0;
+                tag[j] = h;
+#pragma unroll
+                for (int y = 0; y < G; ++y) lw[j] = (y == h) ? ph_lw[y] : lw[j];
+                p = __ldg(gsamp_ph + (size_t)h * sample_cap + (x - ph_pre[h]));
+            } else if (ok[j]) {
+                p = tm.pos(t, lw[j]);
+            }
             ok[j] = ok[j] && (unsigned)p < (unsigned)L;   // a position outside the cache is skipped
             if (ok[j]) {
                 const size_t off = (size_t)p * D;
@@ -117,7 +144,7 @@ k_decode(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__
 #pragma unroll
                 for (int e = 0; e < EPC; ++e) x = fmaf(qv[h][e], kf[e], x);
                 x = group_sum<CPR>(x) + lw[j];
-                if (ok[j]) os.add(h, x, vf);
+                if (ok[j] && (tag[j] < 0 || tag[j] == h)) os.add(h, x, vf);
             }
             if constexpr (PRIOR) {
                 const bool exact = ok[j] && t < sg.n_i;
@@ -271,6 +298,7 @@ static cudaError_t stream_launch(const Dims& d, dim3 grid, const void* q, const 
     io.part = reinterpret_cast<float*>(part);
     io.cnt = reinterpret_cast<unsigned*>(cnt);
     io.out = out;
+    io.per_head = sp.per_head;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(kTcThreads);
@@ -295,7 +323,8 @@ static cudaError_t decode_m(const Dims& d, const DecodePlan& p, const DecodeArgs
             reinterpret_cast<const T*>(a.q), reinterpret_cast<const T*>(a.k), reinterpret_cast<const T*>(a.v),
             a.st, a.sel.blk_idx, a.sp.k_blocks, a.sel.samp_idx, a.sel.samp_count, a.sp.sample_cap,
             d.Hq, d.Hkv, d.L, d.ld, p.g, p.tok_d, p.nsd, p.rec, a.scale * kLog2e, a.scale, a.dp.lambda,
-            reinterpret_cast<float*>(a.ws + p.off_part), reinterpret_cast<unsigned*>(a.ws + p.off_cnt), a.out);
+            reinterpret_cast<float*>(a.ws + p.off_part), reinterpret_cast<unsigned*>(a.ws + p.off_cnt), a.out,
+            a.sp.per_head);
         return cudaGetLastError();
     }
 }

@@ -251,7 +251,7 @@ constexpr int kDenseMode = 4;      // MODE value of the dense pass
 template <int D>
 struct StageLayout {
     static constexpr int kTileBytes = kTcTile * tc::Pitch<D>::kBytes;   // one of K or V
-    static constexpr int kBytes = 2 * kTileBytes + kTcTile * 4;         // K, V, row positions
+    static constexpr int kBytes = 2 * kTileBytes + kTcTile * 8;         // K, V, row positions, row heads
 };
 
 // The unit's chosen blocks and draws are cached in shared memory (after the
@@ -301,6 +301,7 @@ struct StreamIo {
     float* part;
     unsigned* cnt;
     float* out;
+    int per_head;                // draws per query head (rows b Hq + g G + h of samp_idx / samp_count)
 };
 
 // Chunk `chunk` of unit u.  smem: the dynamic area (stream_smem<> bytes);
@@ -370,7 +371,17 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
     // upper bound on the list length (draw capacity); the exact count and the
     // lists are read once the selection is visible
     const int n_indep = DENSE ? L : sg.s_eff + sg.w_eff;
-    const int n_hi = DENSE ? L : sg.n_i + ((SAMP && nt > 0) ? sample_cap : 0);
+    // per-head draws: head h's list follows head h-1's, each token tagged with
+    // its head (it enters that head's softmax alone, weighted n_T / b_h)
+    const bool PH = SAMP && io.per_head != 0;
+    const int32_t* gsamp_ph = samp_idx + ((size_t)b * Hq + (size_t)g * G) * (sample_cap > 0 ? sample_cap : 0);
+    int ph_pre[G + 1];
+    float ph_lw[G];
+#pragma unroll
+    for (int h = 0; h <= G; ++h) ph_pre[h] = 0;
+#pragma unroll
+    for (int h = 0; h < G; ++h) ph_lw[h] = 0.f;
+    const int n_hi = DENSE ? L : sg.n_i + ((SAMP && nt > 0) ? (PH ? G : 1) * sample_cap : 0);
     int n_tok = n_hi;
     float lw_samp = 0.f;
     const bool blk_sm = sg.kk <= kBlkCache;
@@ -385,11 +396,21 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
             asm volatile("griddepcontrol.wait;\n" ::: "memory");
             int bu = 0;
             if (SAMP && nt > 0) {
-                bu = min(__ldcg(samp_count + u), sample_cap);
-                lw_samp = bu > 0 ? log2f((float)nt / (float)bu) : 0.f;
-                n_tok = sg.n_i + bu;
+                if (PH) {
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const int bh = min(__ldcg(samp_count + (size_t)b * Hq + g * G + h), sample_cap);
+                        ph_pre[h + 1] = ph_pre[h] + bh;
+                        ph_lw[h] = bh > 0 ? log2f((float)nt / (float)bh) : 0.f;
+                    }
+                    n_tok = sg.n_i + ph_pre[G];
+                } else {
+                    bu = min(__ldcg(samp_count + u), sample_cap);
+                    lw_samp = bu > 0 ? log2f((float)nt / (float)bu) : 0.f;
+                    n_tok = sg.n_i + bu;
+                }
             }
-            samp_sm = bu <= kSampCache;
+            samp_sm = !PH && bu <= kSampCache;
             if (blk_sm)
                 for (int x = threadIdx.x; x < sg.kk; x += kTcThreads) s_blk[x] = __ldcg(gblk + x);
             if (samp_sm)
@@ -398,10 +419,12 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
             sel_ready = true;
         }
     };
-    // token t of the unit's list -> cache row, or -1 (masked)
+    // token t of the unit's list -> cache row, or -1 (masked), and the head
+    // it belongs to (-1: every head)
     //   [sink 0..s_eff) [window L-w_eff..L) [chosen blocks] [draws]
-    auto pos_of = [&](int t) -> int {
+    auto pos_of = [&](int t, int& tag) -> int {
         int p;
+        tag = -1;
         if (DENSE) p = t < L ? t : -1;
         else if (t >= n_tok) p = -1;
         else if (t < sg.s_eff) p = t;
@@ -409,6 +432,13 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
         else if (t < n_i) {
             const int j = t - n_indep;
             p = 16 * (blk_sm ? s_blk[j >> 4] : __ldcg(gblk + (j >> 4))) + (j & 15);
+        } else if (PH) {
+            const int j = t - n_i;
+            int h = 0;
+#pragma unroll
+            for (int x = 1; x < G; ++x) h += (j >= ph_pre[x]) ? 1 : 0;
+            tag = h;
+            p = __ldcg(gsamp_ph + (size_t)h * sample_cap + (j - ph_pre[h]));
         } else {
             const int j = t - n_i;
             p = samp_sm ? s_samp[j] : __ldcg(gsamp + j);
@@ -424,7 +454,11 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
         if (i < tile1) {
             if ((i + 1) * kTcTile > n_indep) wait_selection();
             int* pos = reinterpret_cast<int*>(smem + (size_t)(i % kStages) * SB + 2 * TB);
-            if (threadIdx.x < kTcTile) pos[threadIdx.x] = pos_of(i * kTcTile + threadIdx.x);
+            if (threadIdx.x < kTcTile) {
+                int tag;
+                pos[threadIdx.x] = pos_of(i * kTcTile + threadIdx.x, tag);
+                pos[kTcTile + threadIdx.x] = tag;
+            }
         }
     };
     // K/V rows of tile i into its stage (cp.async; masked rows zero-filled)
@@ -524,18 +558,37 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
                 rows[2] = r0 + 8 + 2 * tq;
                 rows[3] = r0 + 9 + 2 * tq;
             }
-            float xadd[NR];
             bool in_i[NR];
             const int* pos = reinterpret_cast<const int*>(sb + 2 * TB);
-#pragma unroll
-            for (int j = 0; j < NR; ++j) {
+            // log2-weight of token j for a head: 0 on I, n_T / b for a draw
+            // (per-head draws: only for the head that drew it), -inf if masked
+            auto xw = [&](int j, int head) -> float {
                 const int t = base + rows[j];
-                const bool ok = pos[rows[j]] >= 0;
-                xadd[j] = !ok ? -INFINITY : (t >= n_i ? lw_samp : 0.f);
-                in_i[j] = PRIOR && ok && t < n_i;
-            }
+                if (pos[rows[j]] < 0) return -INFINITY;
+                if (t < n_i) return 0.f;
+                if (!PH) return lw_samp;
+                const int tag = pos[kTcTile + rows[j]];
+                float lw = 0.f;
+#pragma unroll
+                for (int h = 0; h < G; ++h) lw = (h == tag) ? ph_lw[h] : lw;
+                return tag == head ? lw : -INFINITY;
+            };
+#pragma unroll
+            for (int j = 0; j < NR; ++j) in_i[j] = PRIOR && pos[rows[j]] >= 0 && base + rows[j] < n_i;
             const uint32_t sk = tc::smem_u32(sb);
-            wa.step16(sk, sk + TB, r0, xadd, in_i, qscale);
+            if constexpr (kTokRows) {
+                float xadd[2][2];
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) xadd[j][e] = xw(j, 2 * (lane & 3) + e);
+                wa.step16(sk, sk + TB, r0, xadd, in_i, qscale);
+            } else {
+                float xadd[NR];
+#pragma unroll
+                for (int j = 0; j < NR; ++j) xadd[j] = xw(j, lane >> 2);
+                wa.step16(sk, sk + TB, r0, xadd, in_i, qscale);
+            }
         }
         __syncthreads();              // stage i%3 is refilled for tile i+3
     }

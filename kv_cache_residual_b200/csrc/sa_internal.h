@@ -139,7 +139,8 @@ inline DecodePlan decode_plan(const Dims& d, const sa_select_params& sp, int mod
     DecodePlan p;
     p.g = set_geom(d, sp.sink, sp.local, sp.k_blocks);
     const bool draws = mode < 0 || mode == SA_SAMPLE;
-    p.n_tok_max = p.g.n_i + (draws && sp.sample_cap > 0 ? sp.sample_cap : 0);
+    // per-head draws: G lists of up to sample_cap each follow I
+    p.n_tok_max = p.g.n_i + (draws && sp.sample_cap > 0 ? (sp.per_head ? d.G : 1) * sp.sample_cap : 0);
     const int nt = p.n_tok_max > 0 ? p.n_tok_max : 1;
     if (d.bf16) {                  // stream kernel: chunks of 64-token tiles, ~one wave
         const int ntiles = cdiv(nt, 64);

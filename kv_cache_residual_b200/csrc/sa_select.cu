@@ -113,6 +113,7 @@ SelectIo select_io(const Dims& d, const SelectPlan& p, const SelectArgs& a) {
     io.seed = (unsigned long long)a.sp.seed;
     io.step = a.sp.step;
     io.timeouts = wait_counter();
+    io.per_head = a.sp.per_head;
     return io;
 }
 

@@ -470,23 +470,29 @@ __device__ void rescore_members(const T* bm, const int* s_bidx, int nb, const fl
 // The unit's tail draws (vAttention, Method, key design 1: uniform draws
 // from the residual, with replacement): min(sample_b, sample_cap) positions
 // when the tail is not empty, written to samp_idx (and s_copy when they fit
-// s_copy_cap), their count to samp_count[u].  chosen = the unit's kk chosen
-// blocks in ascending order (shared or global memory, visible to every
-// thread).  Draw i's rank r (SplitMix64 counter stream of (seed, b, g, step))
-// maps to the r-th tail position: tail = [s_eff, L - w_eff) minus the chosen
-// blocks, and chosen block j starts after g_j = 16 c_j - s_eff - 16 j tail
-// tokens.  Returns the count.
+// s_copy_cap), their count to samp_count.  One stream per unit (row u of
+// samp_idx / samp_count, the SplitMix64 stream of (seed, b, g, step)) or,
+// with per_head, one per query head h of the group (row b Hq + g G + h, the
+// stream of (seed, b, g G + h, step); s_copy unused).  chosen = the unit's kk
+// chosen blocks in ascending order (shared or global memory, visible to
+// every thread).  Draw i's rank r maps to the r-th tail position: tail =
+// [s_eff, L - w_eff) minus the chosen blocks, and chosen block j starts
+// after g_j = 16 c_j - s_eff - 16 j tail tokens.  Returns the count.
 template <int NT>
 __device__ __forceinline__ int unit_draws(const SetGeom& sg, const int32_t* chosen, int sample_b, int sample_cap,
                                           unsigned long long seed, int b, int g, int step, int u, int32_t* samp_idx,
-                                          int32_t* samp_count, int* s_copy, int s_copy_cap) {
+                                          int32_t* samp_count, int* s_copy, int s_copy_cap, int G = 1,
+                                          int per_head = 0, int Hq = 0) {
     const int nt = sg.n_t, kk = sg.kk;
     const int bdraw = (nt > 0) ? min(sample_b, sample_cap) : 0;
-    if (threadIdx.x == 0) samp_count[u] = bdraw;
+    const int ns = per_head ? G : 1;                         // streams
+    if (threadIdx.x < ns) samp_count[per_head ? b * Hq + g * G + threadIdx.x : u] = bdraw;
     if (bdraw > 0) {
-        const uint64_t key = unit_key(seed, (uint64_t)b, (uint64_t)g, (uint64_t)step);
-        int32_t* out_s = samp_idx + (size_t)u * sample_cap;
-        for (int i = threadIdx.x; i < bdraw; i += NT) {
+        for (int x = threadIdx.x; x < ns * bdraw; x += NT) {
+            const int s = x / bdraw, i = x - s * bdraw;
+            const int row = per_head ? b * Hq + g * G + s : u;
+            const uint64_t key = unit_key(seed, (uint64_t)b, (uint64_t)(per_head ? g * G + s : g), (uint64_t)step);
+            int32_t* out_s = samp_idx + (size_t)row * sample_cap;
             const int r = (int)draw_rank(key, (uint32_t)i, (uint32_t)nt);
             int lo_j = 0, hi_j = kk;             // count of j with g_j <= r
             while (lo_j < hi_j) {
@@ -495,7 +501,7 @@ __device__ __forceinline__ int unit_draws(const SetGeom& sg, const int32_t* chos
                 if (gj <= r) lo_j = mid + 1; else hi_j = mid;
             }
             out_s[i] = sg.s_eff + r + 16 * lo_j;
-            if (s_copy != nullptr && bdraw <= s_copy_cap) s_copy[i] = sg.s_eff + r + 16 * lo_j;
+            if (!per_head && s_copy != nullptr && bdraw <= s_copy_cap) s_copy[i] = sg.s_eff + r + 16 * lo_j;
         }
     }
     return bdraw;
@@ -525,6 +531,7 @@ struct SelectIo {
     unsigned long long seed;
     int step;
     unsigned* timeouts;                   // the library's count of abandoned waits (one per device)
+    int per_head;                         // draws per query head (rows of samp_idx: B Hq)
 };
 
 // Shared memory the selection works in (the caller lays it out):
@@ -1049,7 +1056,7 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
 
     // ---- tail draws -------------------------------------------------------------
     const int bdraw = unit_draws<NT>(sg, sorted_smem ? s_sorted : out_idx, sample_b, sample_cap, seed, b, g, step,
-                                     u, samp_idx, samp_count, sm.samp, sm.samp_cap);
+                                     u, samp_idx, samp_count, sm.samp, sm.samp_cap, G, io.per_head, Hq);
     if (!local) reset_counter(cnt + u);
     res.done = true;
     res.sorted_smem = sorted_smem;

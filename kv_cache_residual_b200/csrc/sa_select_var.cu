@@ -49,6 +49,7 @@ struct VarIo {
     int sample_b, sample_cap;
     unsigned long long seed;
     int step;
+    int per_head;
 };
 
 // Exact score of one candidate (warp-collective; every lane gets it): the
@@ -303,7 +304,7 @@ k_select_var(VarIo io) {
 
     // ---- tail draws ------------------------------------------------------------------
     (void)unit_draws<NT>(sg, sorted_smem ? s_sorted : out_idx, io.sample_b, io.sample_cap, io.seed, b, g, io.step,
-                         u, io.samp_idx, io.samp_count, nullptr, 0);
+                         u, io.samp_idx, io.samp_count, nullptr, 0, G, io.per_head, io.Hq);
 }
 
 size_t select_var_smem(int n_cand) { return (size_t)8 * (size_t)(n_cand > 0 ? n_cand : 1); }
@@ -354,6 +355,7 @@ cudaError_t launch_select_var(const Dims& d, const SelectPlan& p, const SelectAr
     io.sample_cap = a.sp.sample_cap;
     io.seed = (unsigned long long)a.sp.seed;
     io.step = a.sp.step;
+    io.per_head = a.sp.per_head;
     const int sc = a.sp.score;
     if (d.bf16) return d.d == 128 ? var_g<__nv_bfloat16, 128>(d, sc, io, s) : var_g<__nv_bfloat16, 64>(d, sc, io, s);
     return d.d == 128 ? var_g<float, 128>(d, sc, io, s) : var_g<float, 64>(d, sc, io, s);

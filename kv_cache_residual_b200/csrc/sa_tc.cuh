@@ -316,9 +316,10 @@ struct WarpAttnT {
         return y;
     }
 
-    // 16 tokens at tile rows [r0, r0+16): xadd[j] = log2-weight added to the
-    // exact logit of token row(r0, j) (-inf masks it); in_i[j]: it belongs to I
-    __device__ __forceinline__ void step16(uint32_t k_tile, uint32_t v_tile, int r0, const float (&xadd)[2],
+    // 16 tokens at tile rows [r0, r0+16): xadd[j][e] = log2-weight added to
+    // the exact logit of token row(r0, j) in this lane's column 2t + e (-inf
+    // masks it for that head); in_i[j]: the token belongs to I
+    __device__ __forceinline__ void step16(uint32_t k_tile, uint32_t v_tile, int r0, const float (&xadd)[2][2],
                                            const bool (&in_i)[2], float qscale) {
         constexpr int P = Pitch<D>::kBytes;
         const int lane = threadIdx.x & 31, t = lane & 3;
@@ -352,7 +353,7 @@ struct WarpAttnT {
             float x[2];
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                if (c < G) x[j] = fmaf(s[0][2 * j + e], qscale, xadd[j]);
+                if (c < G) x[j] = fmaf(s[0][2 * j + e], qscale, xadd[j][e]);
                 else if (PRIOR && c < 2 * G) x[j] = in_i[j] ? (s[0][2 * j + e] + s[NQ - 1][2 * j + e]) * qscale : -INFINITY;
                 else x[j] = -INFINITY;
             }

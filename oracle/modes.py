@@ -11,7 +11,9 @@ Parity pins: tests/test_oracle_modes.py (full budget = torch
 scaled_dot_product_attention; RESA delta merge = the O(L) merged-logit
 softmax; RESA exact for identical keys; lambda = 0 gives drop; proxy exact for
 a one-token tail and for identical keys; sampling estimator unbiased over
-seeds and exact for identical tail tokens).
+seeds and exact for identical tail tokens; the per-head estimator reduces
+to the group estimator when every head draws the same positions, and per
+head to the one-head estimator).
 """
 import numpy as np
 
@@ -127,6 +129,13 @@ def sample(q, k, v, idx, pos, scale):
     logits = np.concatenate([scale * (q @ k[idx].T), scale * (q @ k[pos].T) + lw], axis=1)
     values = np.concatenate([v[idx], v[pos]], axis=0)
     return _softmax_weighted(logits, values)
+
+
+def sample_per_head(q, k, v, idx, pos_per_head, scale):
+    """The sampling estimator with one sample per query head (the vAttention
+    page samples per head): head h uses its own draws pos_per_head[h] and
+    weight n_T / len(pos_per_head[h]); the exactly read set I is the group's."""
+    return np.concatenate([sample(q[h:h + 1], k, v, idx, pos_per_head[h], scale) for h in range(q.shape[0])], axis=0)
 
 
 def sample_num_den(q, k, v, idx, pos, scale, shift):

@@ -225,3 +225,19 @@ def test_budget_rule_checks(lib):
         sp = sa.sa_select_params(64, 128, 8, 0, 64, 512, 0.05, 0.05, 0, 0, 0, rule)
         assert lib.sa_select(ctypes.byref(sh), ctypes.byref(sp), p, ctypes.byref(st), p, p, ctypes.byref(sel), 0.0,
                              p, 64, None) == status
+
+
+def test_per_head_flag_checks(lib):
+    sh = _shape()
+    p = ctypes.c_void_p(0x10000)
+    st = sa.sa_stats(*([0x10000] * 10))
+    sel = sa.sa_selection(0x10000, 0x10000, 0x10000, 0)
+    for flag, status in ((2, sa.SA_ERR_INVALID_ARG), (-1, sa.SA_ERR_INVALID_ARG), (1, sa.SA_ERR_WORKSPACE)):
+        sp = sa.sa_select_params(64, 128, 8, 32, 0, 32, 0.05, 0.05, 0, 0, 0, 0, flag)
+        assert lib.sa_select(ctypes.byref(sh), ctypes.byref(sp), p, ctypes.byref(st), None, None, ctypes.byref(sel),
+                             0.0, p, 64, None) == status
+    # per-head draws need a workspace sized for G draw lists in the decode
+    one = sa.sa_select_params(64, 128, 8, 32, 0, 32, 0.05, 0.05, 0, 0, 0, 0, 0)
+    ph = sa.sa_select_params(64, 128, 8, 32, 0, 32, 0.05, 0.05, 0, 0, 0, 0, 1)
+    assert lib.sa_workspace_size(ctypes.byref(sh), ctypes.byref(ph), sa.OP_DECODE) >= \
+        lib.sa_workspace_size(ctypes.byref(sh), ctypes.byref(one), sa.OP_DECODE)

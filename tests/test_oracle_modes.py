@@ -218,3 +218,24 @@ def test_empty_exact_set():
     # the proxy alone is the tail-mean value (one token carries all weight)
     np.testing.assert_allclose(modes.proxy(q, k, v, empty, st, s), np.tile(v.mean(0), (q.shape[0], 1)),
                                rtol=1e-12, atol=1e-13)
+
+
+def test_sample_per_head_reductions():
+    # every head drawing the same positions gives the group estimator; one
+    # head alone is the one-head estimator; heads with different draws differ
+    from oracle import modes as M
+    r = np.random.default_rng(17)
+    G, d, L = 3, 8, 256
+    q = r.standard_normal((G, d))
+    k = r.standard_normal((L, d))
+    v = r.standard_normal((L, d))
+    idx = np.arange(0, 40)
+    tail = np.arange(40, L)
+    pos = r.choice(tail, 24)
+    same = M.sample_per_head(q, k, v, idx, [pos] * G, 0.3)
+    assert np.allclose(same, M.sample(q, k, v, idx, pos, 0.3), rtol=0, atol=1e-14)
+    per = [r.choice(tail, n) for n in (8, 16, 32)]
+    got = M.sample_per_head(q, k, v, idx, per, 0.3)
+    for h in range(G):
+        assert np.allclose(got[h], M.sample(q[h:h + 1], k, v, idx, per[h], 0.3)[0], rtol=0, atol=1e-14)
+    assert not np.allclose(got, M.sample(q, k, v, idx, per[0], 0.3))
