@@ -27,8 +27,10 @@ Sources (pages, by title and section):
 * OpenAttention: One Percent Is Enough with Tail Proxies
   - Abstract and method stage 04: the count-aware mean proxy, one virtual
     token with logit zbar + log n and value = the tail mean.
+  - Method overview stages 01-04 (openattn.py): query-geometry clustering,
+    ErrorGate's budget split, the QGS int8 selector and one proxy per cluster.
 
 Parity status of each function is stated in its docstring; the pins live in
 tests/test_oracle_*.py.
 """
-from . import numerics, rng, select, stats, modes, budget  # noqa: F401
+from . import numerics, rng, select, stats, modes, budget, openattn  # noqa: F401

@@ -386,3 +386,68 @@ def test_budget_rule_mistake_fails_a_pin(monkeypatch, golden_dir, name):
         p_(**kw)
     monkeypatch.setattr(budget, attr, fn)
     assert _some_pin_fails(pins)
+
+
+def _multi_proxy_without_log_n(q, k, v, read, assign, cs, scale):
+    import oracle.openattn as OA
+    cs2 = dict(cs)
+    out_logits, out_vals = [scale * (q @ k[read].T)], [v[read]]
+    for c in range(len(cs["n"])):
+        mr = read[assign[read] == c] if len(read) else read
+        n_un = int(cs["n"][c]) - len(mr)
+        if n_un <= 0:
+            continue
+        kb = (cs["sum_k"][c] - k[mr].sum(axis=0)) / n_un
+        vb = (cs["sum_v"][c] - v[mr].sum(axis=0)) / n_un
+        out_logits.append((scale * (q @ kb))[:, None])                  # + ln n' missing
+        out_vals.append(vb[None, :])
+    lg = np.concatenate(out_logits, axis=1)
+    w = np.exp(lg - lg.max(axis=1, keepdims=True))
+    return (w @ np.concatenate(out_vals, axis=0)) / w.sum(axis=1, keepdims=True)
+
+
+def _kmeans_frozen(y, n_clusters=64, rounds=10):
+    L = len(y)
+    cent = y[(np.arange(n_clusters) * L) // n_clusters].copy()          # never moved
+    d2 = ((y[:, None, :] - cent[None, :, :]) ** 2).sum(axis=2)
+    return np.argmin(d2, axis=1), cent
+
+
+def _errors_without_variance(q, cs, scale):
+    n = cs["n"].astype(np.float64)
+    live = n > 0
+    mean = np.zeros_like(cs["sum_k"])
+    mean[live] = cs["sum_k"][live] / n[live, None]
+    mu = scale * (q @ mean.T)
+    return np.where(live[None, :], n[None, :] * np.exp(mu - mu.max(axis=1, keepdims=True)), 0).sum(axis=0)
+
+
+def _scores_without_scale(qq, code, sig):
+    from oracle.numerics import round_to_f32
+    return round_to_f32((code @ qq).astype(np.float64))
+
+
+OPENATTN_MISTAKES = {
+    "proxy logit without ln n": ("multi_proxy", _multi_proxy_without_log_n),
+    "k-means centroids never updated": ("kmeans", _kmeans_frozen),
+    "weight error without the variance": ("cluster_errors", _errors_without_variance),
+    "QGS score without the token scale": ("qgs_scores", _scores_without_scale),
+}
+
+
+@pytest.mark.parametrize("name", list(OPENATTN_MISTAKES))
+def test_openattn_mistake_fails_a_pin(monkeypatch, name):
+    import oracle.openattn as OA
+    import test_oracle_openattn as pin_oa
+    attr, fn = OPENATTN_MISTAKES[name]
+    monkeypatch.setattr(OA, attr, fn)
+    pins = [(getattr(pin_oa, t), {}) for t in dir(pin_oa) if t.startswith("test_")]
+    assert _some_pin_fails(pins)
+
+
+def test_openattn_uncapped_split_fails_a_pin(monkeypatch):
+    import oracle.openattn as OA
+    import test_oracle_openattn as pin_oa
+    orig = OA.errorgate
+    monkeypatch.setattr(OA, "errorgate", lambda err, n, budget: orig(err, np.full(len(n), 10 ** 9), budget))
+    assert _some_pin_fails([(pin_oa.test_errorgate_caps_and_totals, {})])
