@@ -116,7 +116,8 @@ typedef enum {
     SA_OP_SELECT = 1,    /* sa_select        */
     SA_OP_DECODE = 2,    /* sa_decode        */
     SA_OP_DENSE = 3,     /* sa_dense_decode  */
-    SA_OP_STEP = 4       /* sa_step          */
+    SA_OP_STEP = 4,      /* sa_step          */
+    SA_OP_MULTI = 5      /* sa_multi_step    */
 } sa_op;
 
 /* Supported: d in {64, 128}; Hq % Hkv == 0 with G = Hq/Hkv in {1,2,4,8};
@@ -176,6 +177,37 @@ typedef struct {
     void* blk_min;
     void* blk_max;
 } sa_stats;
+
+/* The OpenAttention multi-proxy state of a cache ("OpenAttention: One
+ * Percent Is Enough with Tail Proxies", method overview stages 01-04), per
+ * unit (sequence b, KV head g), caller-allocated:
+ *   n_clusters  C, 1..64 (the page's C = 64)
+ *   basis       [B, Hkv, 32, d] f32: rows = the eigenvectors of the second
+ *               moment of the unit's context queries, decreasing eigenvalue
+ *               (the QGS basis, r = 32; its first 16 rows the clustering
+ *               basis); written by sa_cluster_build or by the caller
+ *   assign      [B, Hkv, ld] uint8: each token's cluster (k-means of the keys
+ *               projected on the first 16 rows); sa_cluster_build or caller
+ *   codes       [B, Hkv, ld, 32] int8 and scales [B, Hkv, ld] f32: the QGS
+ *               codes of each key, z = basis . K_j (exact sums rounded once),
+ *               sigma = fl32(max |z| / 127), code = clamp(rint(z / sigma),
+ *               +-127); written by sa_cluster_prep
+ *   count       [B, Hkv, C] int32 and sum_k, sum_v, sum_k2 [B, Hkv, C, d] f32:
+ *               per cluster the member count and the sums of keys, values and
+ *               squared keys (the cached mean and diagonal variance);
+ *               written by sa_cluster_prep
+ * Pointers 16-byte aligned. */
+typedef struct {
+    int n_clusters;
+    float* basis;
+    uint8_t* assign;
+    int8_t* codes;
+    float* scales;
+    int32_t* count;
+    float* sum_k;
+    float* sum_v;
+    float* sum_k2;
+} sa_clusters;
 
 /* Which tokens one step reads exactly, and how the tail is sampled.
  *   sink, local   >= 0: first / last tokens always read (vAttention page,
@@ -355,6 +387,37 @@ SA_API sa_status sa_step(const sa_shape* shape, const sa_decode_params* dparams,
                          const sa_select_params* sparams, const void* q, const void* k, const void* v,
                          const sa_stats* stats, const sa_selection* sel, float* out, void* ws,
                          size_t ws_bytes, void* stream);
+
+/* The per-cluster state that follows from basis and assign over tokens
+ * [0, L): the QGS codes and scales, the counts and the sums (layouts of
+ * sa_clusters).  Prefill-time; no workspace. */
+SA_API sa_status sa_cluster_prep(const sa_shape* shape, const void* k, const void* v, const sa_clusters* cl,
+                                 void* stream);
+
+/* One decode step of the multi-proxy pipeline (OpenAttention, method
+ * stages 02-04) for every unit:
+ *   ErrorGate: per cluster and query head of the group the member-logit mean
+ *   mu = s q_h . Kbar and variance s^2 sum_e q_he^2 var_e (diagonal); the
+ *   proxy's weight error n e^mu (e^(var/2) - 1) over the head's estimated
+ *   mass sum n e^(mu + var/2), summed over the heads, made integers
+ *   w = rint(2^30 err / max err); the budget E = min(budget, L) split as
+ *   q_c = min(n_c, floor(E w_c / W)) and the rest one token at a time by
+ *   largest remainder (E w_c mod W), lower cluster first, round after round;
+ *   QGS: every token's score fl32(sigma_j (qq . code_j)), qq = the group's
+ *   projected query p = basis . sum_h q_h coded to 16 bits (sq = max|p| /
+ *   32767, qq = rint(p / sq)); each cluster reads its q_c best tokens by
+ *   (score desc, position asc);
+ *   stage 04: one softmax over the read tokens' exact logits and, per cluster
+ *   with n' = n_c - q_c > 0 unread members, one proxy of logit s q . Kbar' +
+ *   ln n' and value Vbar' (means over the unread members: the cluster's sums
+ *   minus the read rows').
+ * read [B, Hkv, budget] int32 gets the read positions grouped by cluster
+ * (cluster order, ascending positions; -1 after the last), read_count
+ * [B, Hkv, C] int32 the q_c, out [B, Hq, d] f32 the output.  scale = softmax
+ * scale (0 = 1/sqrt(d)).  Workspace: sa_workspace_size(.., SA_OP_MULTI). */
+SA_API sa_status sa_multi_step(const sa_shape* shape, const void* q, const void* k, const void* v,
+                               const sa_clusters* cl, int budget, float scale, int32_t* read, int32_t* read_count,
+                               float* out, void* ws, size_t ws_bytes, void* stream);
 
 /* Dense flash-decode over all L tokens (the in-build speed reference, not
  * part of the method): out [B, Hq, d] f32 = softmax(s q K^T) V. */

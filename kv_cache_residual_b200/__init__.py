@@ -27,7 +27,7 @@ SA_F32, SA_BF16 = 0, 1
 MODES = {"drop": 0, "resa": 1, "proxy": 2, "sample": 3}
 SCORES = {"mean_sum": 0, "mean_max": 1, "quest": 2}
 BUDGETS = {"clt": 0, "clt_search": 1, "hoeffding": 2}
-OP_PREFILL, OP_SELECT, OP_DECODE, OP_DENSE, OP_STEP = range(5)
+OP_PREFILL, OP_SELECT, OP_DECODE, OP_DENSE, OP_STEP, OP_MULTI = range(6)
 
 
 class SAError(RuntimeError):
@@ -59,6 +59,12 @@ class sa_selection(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("blk_idx", "samp_idx", "samp_count", "n_rescored")]
 
 
+class sa_clusters(ctypes.Structure):
+    _fields_ = [("n_clusters", ctypes.c_int)] + [(n, ctypes.c_void_p) for n in
+                                                  ("basis", "assign", "codes", "scales", "count", "sum_k", "sum_v",
+                                                   "sum_k2")]
+
+
 class sa_decode_params(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int), ("lam", ctypes.c_float), ("scale", ctypes.c_float)]
 
@@ -66,7 +72,8 @@ class sa_decode_params(ctypes.Structure):
 EXPORTS = ("sa_workspace_size", "sa_prefill_stats", "sa_block_summaries", "sa_block_sketch", "sa_block_minmax",
            "sa_select",
            "sa_select_noalloc",
-           "sa_decode", "sa_step", "sa_dense_decode", "sa_append", "sa_wait_timeouts",
+           "sa_decode", "sa_step", "sa_dense_decode", "sa_append", "sa_wait_timeouts", "sa_cluster_prep",
+           "sa_multi_step",
            "sa_status_string")
 
 _LIB = None
@@ -94,11 +101,15 @@ def _lib():
         lib.sa_step.argtypes = [sh, dp, sp, P, P, P, st, sel, P, P, S, P]
         lib.sa_dense_decode.argtypes = [sh, P, P, P, P, F, P, S, P]
         lib.sa_append.argtypes = [sh, P, P, P, P, st, F, P]
+        cl = ctypes.POINTER(sa_clusters)
+        lib.sa_cluster_prep.argtypes = [sh, P, P, cl, P]
+        lib.sa_multi_step.argtypes = [sh, P, P, P, cl, I, F, P, P, P, P, S, P]
         lib.sa_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
         lib.sa_wait_timeouts.restype = I
         lib.sa_status_string.argtypes = [I]
         lib.sa_status_string.restype = ctypes.c_char_p
-        for f in ("sa_prefill_stats", "sa_block_summaries", "sa_block_sketch", "sa_block_minmax", "sa_select", "sa_select_noalloc", "sa_decode", "sa_step",
+        for f in ("sa_cluster_prep", "sa_multi_step",
+                  "sa_prefill_stats", "sa_block_summaries", "sa_block_sketch", "sa_block_minmax", "sa_select", "sa_select_noalloc", "sa_decode", "sa_step",
                   "sa_dense_decode", "sa_append"):
             getattr(lib, f).restype = I
         _LIB = lib
@@ -200,6 +211,59 @@ class Selection:
     def c(self):
         return sa_selection(self.blk_idx.data_ptr(), self.samp_idx.data_ptr(), self.samp_count.data_ptr(),
                             self.n_rescored.data_ptr())
+
+
+class Clusters:
+    """The multi-proxy state of a cache (caller-owned device tensors, layouts
+    of sa_clusters in sa_decode.h)."""
+
+    FIELDS = ("basis", "assign", "codes", "scales", "count", "sum_k", "sum_v", "sum_k2")
+
+    def __init__(self, B, Hkv, ld, d, n_clusters, device):
+        f = dict(dtype=torch.float32, device=device)
+        self.n_clusters = int(n_clusters)
+        self.basis = torch.zeros(B, Hkv, 32, d, **f)
+        self.assign = torch.zeros(B, Hkv, ld, dtype=torch.uint8, device=device)
+        self.codes = torch.zeros(B, Hkv, ld, 32, dtype=torch.int8, device=device)
+        self.scales = torch.zeros(B, Hkv, ld, **f)
+        self.count = torch.zeros(B, Hkv, n_clusters, dtype=torch.int32, device=device)
+        self.sum_k = torch.zeros(B, Hkv, n_clusters, d, **f)
+        self.sum_v = torch.zeros(B, Hkv, n_clusters, d, **f)
+        self.sum_k2 = torch.zeros(B, Hkv, n_clusters, d, **f)
+
+    def c(self):
+        return sa_clusters(self.n_clusters, *[getattr(self, n).data_ptr() for n in self.FIELDS])
+
+
+def cluster_prep(k, v, clusters, Hq, length=None, stream=None):
+    """Codes, scales, counts and sums of `clusters` from its basis and
+    assignment over the first `length` tokens (see sa_cluster_prep)."""
+    shape = make_shape(k, Hq, length)
+    c = clusters.c()
+    _check(_lib().sa_cluster_prep(ctypes.byref(shape), _ptr(k), _ptr(v), ctypes.byref(c), _stream(stream)),
+           "sa_cluster_prep")
+
+
+def multi_step(q, k, v, clusters, budget, scale=0.0, read=None, read_count=None, out=None, length=None,
+               stream=None):
+    """One multi-proxy decode step (see sa_multi_step).  Returns (out, read,
+    read_count)."""
+    B, Hq, d = q.shape
+    shape = make_shape(k, Hq, length)
+    Hkv = shape.Hkv
+    dev = q.device
+    if read is None:
+        read = torch.empty(B, Hkv, int(budget), dtype=torch.int32, device=dev)
+    if read_count is None:
+        read_count = torch.empty(B, Hkv, clusters.n_clusters, dtype=torch.int32, device=dev)
+    if out is None:
+        out = torch.empty(B, Hq, d, dtype=torch.float32, device=dev)
+    ws = workspace(shape, None, OP_MULTI, dev)
+    c = clusters.c()
+    _check(_lib().sa_multi_step(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(c), int(budget),
+                                float(scale), _ptr(read), _ptr(read_count), _ptr(out), _ptr(ws), ws.numel(),
+                                _stream(stream)), "sa_multi_step")
+    return out, read, read_count
 
 
 _WS = {}

@@ -107,6 +107,7 @@ size_t sa_workspace_size(const sa_shape* shape, const sa_select_params* params, 
         case SA_OP_STEP:
             if (check_select_params(params) != SA_OK) return 0;
             return select_plan(d, *params).bytes + decode_plan(d, *params).bytes;
+        case SA_OP_MULTI: return multi_workspace(d);
     }
     return 0;
 }
@@ -320,6 +321,42 @@ sa_status sa_step(const sa_shape* shape, const sa_decode_params* dparams, const 
         if (launch_clt(d, ps, as, s) != cudaSuccess) return SA_ERR_CUDA;
     }
     return launch_decode(d, pd, ad, s) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+namespace {
+bool check_clusters(const sa_clusters* cl) {
+    if (cl == nullptr || cl->n_clusters < 1 || cl->n_clusters > 64) return false;
+    return aligned16(cl->basis) && aligned16(cl->assign) && aligned16(cl->codes) && aligned16(cl->scales) &&
+           aligned16(cl->count) && aligned16(cl->sum_k) && aligned16(cl->sum_v) && aligned16(cl->sum_k2);
+}
+}  // namespace
+
+sa_status sa_cluster_prep(const sa_shape* shape, const void* k, const void* v, const sa_clusters* cl, void* stream) {
+    NvtxRange r("sa_cluster_prep");
+    Dims d;
+    sa_status e = check_shape(shape, &d);
+    if (e != SA_OK) return e;
+    if (!aligned16(k) || !aligned16(v) || !check_clusters(cl)) return SA_ERR_INVALID_ARG;
+    if (d.ld >= (1 << 24)) return SA_ERR_UNSUPPORTED;
+    return launch_cluster_prep(d, k, v, *cl, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+sa_status sa_multi_step(const sa_shape* shape, const void* q, const void* k, const void* v, const sa_clusters* cl,
+                        int budget, float scale, int32_t* read, int32_t* read_count, float* out, void* ws,
+                        size_t ws_bytes, void* stream) {
+    NvtxRange r("sa_multi_step");
+    Dims d;
+    sa_status e = check_shape(shape, &d);
+    if (e != SA_OK) return e;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !check_clusters(cl) || budget < 1 ||
+        !aligned4(read) || !aligned4(read_count) || !aligned16(out) || scale < 0.f)
+        return SA_ERR_INVALID_ARG;
+    const size_t need = multi_workspace(d);
+    if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return SA_ERR_WORKSPACE;
+    return launch_multi_step(d, q, k, v, *cl, budget, resolve_scale(scale, d.d), read, read_count, out,
+                             static_cast<char*>(ws), static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SA_OK
+               : SA_ERR_CUDA;
 }
 
 sa_status sa_dense_decode(const sa_shape* shape, const void* q, const void* k, const void* v, float* out,

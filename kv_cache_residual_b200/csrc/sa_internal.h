@@ -249,6 +249,13 @@ struct DecodeArgs {
 };
 cudaError_t launch_decode(const Dims& d, const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
 
+// The multi-proxy path (sa_multi.cu)
+cudaError_t launch_cluster_prep(const Dims& d, const void* k, const void* v, const sa_clusters& cl, cudaStream_t s);
+size_t multi_workspace(const Dims& d);
+cudaError_t launch_multi_step(const Dims& d, const void* q, const void* k, const void* v, const sa_clusters& cl,
+                              int budget, float scale, int32_t* read, int32_t* qcnt, float* out, char* ws,
+                              cudaStream_t s);
+
 struct DenseArgs {
     const void* q; const void* k; const void* v; float scale; float* out; char* ws;
 };
