@@ -117,7 +117,8 @@ typedef enum {
     SA_OP_DECODE = 2,    /* sa_decode        */
     SA_OP_DENSE = 3,     /* sa_dense_decode  */
     SA_OP_STEP = 4,      /* sa_step          */
-    SA_OP_MULTI = 5      /* sa_multi_step    */
+    SA_OP_MULTI = 5,     /* sa_multi_step    */
+    SA_OP_CLUSTER = 6    /* sa_cluster_build */
 } sa_op;
 
 /* Supported: d in {64, 128}; Hq % Hkv == 0 with G = Hq/Hkv in {1,2,4,8};
@@ -387,6 +388,20 @@ SA_API sa_status sa_step(const sa_shape* shape, const sa_decode_params* dparams,
                          const sa_select_params* sparams, const void* q, const void* k, const void* v,
                          const sa_stats* stats, const sa_selection* sel, float* out, void* ws,
                          size_t ws_bytes, void* stream);
+
+/* Query-geometry clustering of the cache at prefill end (OpenAttention,
+ * method stage 01, QGC), for every unit: unless basis_given, the second
+ * moment M = (1/(G L)) sum q q^T of the unit's context queries q_ctx
+ * [B, Hq, L, d] and its 32 leading eigenvectors into cl->basis (subspace
+ * iteration with CholeskyQR2 in fp64, ordered by Rayleigh quotient); then
+ * k-means of the keys projected on the first 16 basis rows into cl->assign
+ * (centroid c starts at the projection of token floor(c L / C); 10 rounds of
+ * nearest centroid, lowest index on ties, and member means, an empty
+ * cluster's centroid kept; a last assignment); then sa_cluster_prep.
+ * basis_given = 1 keeps the caller's basis (q_ctx unused, may be NULL).
+ * Workspace: sa_workspace_size(.., SA_OP_CLUSTER), zero-filled once. */
+SA_API sa_status sa_cluster_build(const sa_shape* shape, const void* q_ctx, const void* k, const void* v,
+                                  const sa_clusters* cl, int basis_given, void* ws, size_t ws_bytes, void* stream);
 
 /* The per-cluster state that follows from basis and assign over tokens
  * [0, L): the QGS codes and scales, the counts and the sums (layouts of

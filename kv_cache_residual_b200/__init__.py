@@ -27,7 +27,7 @@ SA_F32, SA_BF16 = 0, 1
 MODES = {"drop": 0, "resa": 1, "proxy": 2, "sample": 3}
 SCORES = {"mean_sum": 0, "mean_max": 1, "quest": 2}
 BUDGETS = {"clt": 0, "clt_search": 1, "hoeffding": 2}
-OP_PREFILL, OP_SELECT, OP_DECODE, OP_DENSE, OP_STEP, OP_MULTI = range(6)
+OP_PREFILL, OP_SELECT, OP_DECODE, OP_DENSE, OP_STEP, OP_MULTI, OP_CLUSTER = range(7)
 
 
 class SAError(RuntimeError):
@@ -72,7 +72,7 @@ class sa_decode_params(ctypes.Structure):
 EXPORTS = ("sa_workspace_size", "sa_prefill_stats", "sa_block_summaries", "sa_block_sketch", "sa_block_minmax",
            "sa_select",
            "sa_select_noalloc",
-           "sa_decode", "sa_step", "sa_dense_decode", "sa_append", "sa_wait_timeouts", "sa_cluster_prep",
+           "sa_decode", "sa_step", "sa_dense_decode", "sa_append", "sa_wait_timeouts", "sa_cluster_prep", "sa_cluster_build",
            "sa_multi_step",
            "sa_status_string")
 
@@ -103,12 +103,13 @@ def _lib():
         lib.sa_append.argtypes = [sh, P, P, P, P, st, F, P]
         cl = ctypes.POINTER(sa_clusters)
         lib.sa_cluster_prep.argtypes = [sh, P, P, cl, P]
+        lib.sa_cluster_build.argtypes = [sh, P, P, P, cl, I, P, S, P]
         lib.sa_multi_step.argtypes = [sh, P, P, P, cl, I, F, P, P, P, P, S, P]
         lib.sa_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
         lib.sa_wait_timeouts.restype = I
         lib.sa_status_string.argtypes = [I]
         lib.sa_status_string.restype = ctypes.c_char_p
-        for f in ("sa_cluster_prep", "sa_multi_step",
+        for f in ("sa_cluster_prep", "sa_cluster_build", "sa_multi_step",
                   "sa_prefill_stats", "sa_block_summaries", "sa_block_sketch", "sa_block_minmax", "sa_select", "sa_select_noalloc", "sa_decode", "sa_step",
                   "sa_dense_decode", "sa_append"):
             getattr(lib, f).restype = I
@@ -242,6 +243,25 @@ def cluster_prep(k, v, clusters, Hq, length=None, stream=None):
     c = clusters.c()
     _check(_lib().sa_cluster_prep(ctypes.byref(shape), _ptr(k), _ptr(v), ctypes.byref(c), _stream(stream)),
            "sa_cluster_prep")
+
+
+def cluster_build(q_ctx, k, v, n_clusters=64, clusters=None, basis_given=False, length=None, stream=None):
+    """Query-geometry clustering of the cache (see sa_cluster_build): basis
+    (unless given in `clusters`), assignment, codes and sums.  Returns the
+    Clusters."""
+    B, Hkv, ld, d = k.shape
+    Hq = q_ctx.shape[1] if q_ctx is not None else None
+    if Hq is None:
+        raise ValueError("q_ctx gives the number of query heads")
+    shape = make_shape(k, Hq, length if length is not None else q_ctx.shape[2])
+    if clusters is None:
+        clusters = Clusters(B, Hkv, ld, d, n_clusters, k.device)
+    ws = workspace(shape, None, OP_CLUSTER, k.device)
+    c = clusters.c()
+    _check(_lib().sa_cluster_build(ctypes.byref(shape), _ptr(q_ctx), _ptr(k), _ptr(v), ctypes.byref(c),
+                                   int(bool(basis_given)), _ptr(ws), ws.numel(), _stream(stream)),
+           "sa_cluster_build")
+    return clusters
 
 
 def multi_step(q, k, v, clusters, budget, scale=0.0, read=None, read_count=None, out=None, length=None,

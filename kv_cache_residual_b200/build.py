@@ -19,7 +19,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libsa_b200.so")
-SOURCES = ["sa_api.cu", "sa_prefill.cu", "sa_select.cu", "sa_decode.cu", "sa_clt.cu", "sa_select_var.cu", "sa_multi.cu", "sa_noalloc.cu",
+SOURCES = ["sa_api.cu", "sa_prefill.cu", "sa_select.cu", "sa_decode.cu", "sa_clt.cu", "sa_select_var.cu", "sa_multi.cu", "sa_qgc.cu", "sa_noalloc.cu",
            "sa_append.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

@@ -108,6 +108,7 @@ size_t sa_workspace_size(const sa_shape* shape, const sa_select_params* params, 
             if (check_select_params(params) != SA_OK) return 0;
             return select_plan(d, *params).bytes + decode_plan(d, *params).bytes;
         case SA_OP_MULTI: return multi_workspace(d);
+        case SA_OP_CLUSTER: return qgc_plan(d).bytes;
     }
     return 0;
 }
@@ -339,6 +340,24 @@ sa_status sa_cluster_prep(const sa_shape* shape, const void* k, const void* v, c
     if (!aligned16(k) || !aligned16(v) || !check_clusters(cl)) return SA_ERR_INVALID_ARG;
     if (d.ld >= (1 << 24)) return SA_ERR_UNSUPPORTED;
     return launch_cluster_prep(d, k, v, *cl, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+sa_status sa_cluster_build(const sa_shape* shape, const void* q_ctx, const void* k, const void* v,
+                           const sa_clusters* cl, int basis_given, void* ws, size_t ws_bytes, void* stream) {
+    NvtxRange r("sa_cluster_build");
+    Dims d;
+    sa_status e = check_shape(shape, &d);
+    if (e != SA_OK) return e;
+    if ((basis_given != 0 && basis_given != 1) || (!basis_given && !aligned16(q_ctx)) || !aligned16(k) ||
+        !aligned16(v) || !check_clusters(cl))
+        return SA_ERR_INVALID_ARG;
+    if (d.ld >= (1 << 24)) return SA_ERR_UNSUPPORTED;
+    const QgcPlan p = qgc_plan(d);
+    if (ws == nullptr || ws_bytes < p.bytes || !aligned16(ws)) return SA_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (launch_cluster_build(d, p, q_ctx, k, *cl, basis_given != 0, static_cast<char*>(ws), s) != cudaSuccess)
+        return SA_ERR_CUDA;
+    return launch_cluster_prep(d, k, v, *cl, s) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 
 sa_status sa_multi_step(const sa_shape* shape, const void* q, const void* k, const void* v, const sa_clusters* cl,

@@ -249,6 +249,15 @@ struct DecodeArgs {
 };
 cudaError_t launch_decode(const Dims& d, const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
 
+// Query-geometry clustering at prefill (sa_qgc.cu): workspace layout and launch
+struct QgcPlan {
+    int nsplit, rows_per;       // second-moment splits per unit, query rows per split
+    size_t off_cnt, off_part, off_mom, off_y, bytes;
+};
+QgcPlan qgc_plan(const Dims& d);
+cudaError_t launch_cluster_build(const Dims& d, const QgcPlan& p, const void* q_ctx, const void* k,
+                                 const sa_clusters& cl, bool basis_given, char* ws, cudaStream_t s);
+
 // The multi-proxy path (sa_multi.cu)
 cudaError_t launch_cluster_prep(const Dims& d, const void* k, const void* v, const sa_clusters& cl, cudaStream_t s);
 size_t multi_workspace(const Dims& d);

@@ -1,0 +1,118 @@
+"""GPU checks of the query-geometry clustering (OpenAttention stage 01,
+sa_cluster_build).  The kernels' basis and k-means cannot match the oracle's
+to the bit (an eigenbasis is fixed only up to rotations inside degenerate
+eigenspaces, and a nearest-centroid decision can flip on rounding), so they
+are checked by what holds of any correct result: an orthonormal basis whose
+captured second moment reaches the top eigenvalues' sum (Ky Fan) and whose
+dominant directions span the oracle's; k-means recovering planted separated
+clusters exactly, and on real keys with the oracle's basis agreeing with the
+oracle's clustering on nearly every token at a nearly equal objective."""
+import numpy as np
+import pytest
+import torch
+
+import kv_cache_residual_b200 as sa
+import synth
+from oracle import openattn as OA
+from parity_util import f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _moment(qctx):
+    x = qctx.reshape(-1, qctx.shape[-1])
+    return x.T @ x / len(x)
+
+
+@pytest.mark.parametrize("wname,L", [("llama", 4096), ("tiny", 2048)])
+def test_basis_orthonormal_and_captures_the_leading_eigenvalues(wname, L):
+    w = synth.scaled(synth.WORKLOADS[wname], B=1, L=L) if wname != "tiny" else synth.WORKLOADS["tiny"]
+    dev = torch.device("cuda")
+    data = synth.make_batch(w, device=dev, steps=1)
+    cl = sa.cluster_build(data["q_ctx"], data["k"], data["v"], n_clusters=16)
+    torch.cuda.synchronize()
+    for g in range(w.Hkv):
+        bas = f64(cl.basis[0, g])                                  # [32, d]
+        assert np.allclose(bas @ bas.T, np.eye(32), atol=2e-5)
+        m = _moment(f64(data["q_ctx"][0, g * w.G:(g + 1) * w.G]))
+        ev = np.sort(np.linalg.eigvalsh(m))[::-1]
+        # (the noise directions beyond the planted ones converge slowly: a
+        # small shortfall there is allowed)
+        for r, tol in ((16, 5e-3), (32, 1e-2)):
+            captured = np.trace(bas[:r] @ m @ bas[:r].T)
+            assert captured >= (1 - tol) * ev[:r].sum() and captured <= ev[:r].sum() * (1 + 1e-5)
+        # the G dominant directions (well separated from the rest) span the oracle's
+        u, _ = OA.query_basis(f64(data["q_ctx"][0, g * w.G:(g + 1) * w.G]), w.G)
+        assert np.allclose(bas[:w.G].T @ bas[:w.G], u @ u.T, atol=2e-3)
+        # rows ordered by captured moment, largest first
+        rq = np.einsum("id,de,ie->i", bas, m, bas)
+        assert np.all(np.diff(rq) <= 1e-5 * rq[0])
+
+
+def test_kmeans_recovers_planted_clusters():
+    """16 tight, well-separated clusters in the first 16 key coordinates, laid
+    out in position order so that the starts fall one in each; the basis is
+    given (the first 16 rows the unit vectors of those coordinates): the
+    assignment is the planted one, token for token."""
+    B, Hq, Hkv, d, L, C = 2, 4, 2, 128, 2048, 16
+    dev = torch.device("cuda")
+    gen = torch.Generator().manual_seed(5)
+    centres = 20.0 * torch.randn(B, Hkv, C, d, generator=gen)
+    labels = torch.arange(L) // (L // C)
+    k = (centres[:, :, labels] + 0.3 * torch.randn(B, Hkv, L, d, generator=gen)).to(torch.bfloat16)
+    v = torch.randn(B, Hkv, L, d, generator=gen).to(torch.bfloat16)
+    cl = sa.Clusters(B, Hkv, L, d, C, dev)
+    eye = torch.zeros(32, d)
+    eye[torch.arange(32), torch.arange(32)] = 1.0
+    cl.basis.copy_(eye.expand(B, Hkv, 32, d))
+    q_ctx = torch.zeros(B, Hq, L, d, dtype=torch.bfloat16, device=dev)
+    sa.cluster_build(q_ctx, k.to(dev), v.to(dev), clusters=cl, basis_given=True)
+    torch.cuda.synchronize()
+    for b in range(B):
+        for g in range(Hkv):
+            assert cl.assign[b, g].cpu().long().tolist() == labels.tolist()
+            assert cl.count[b, g].cpu().tolist() == [L // C] * C
+
+
+def test_kmeans_with_the_oracle_basis_agrees_with_the_oracle():
+    w = synth.scaled(synth.WORKLOADS["llama"], B=1, Hq=8, Hkv=2, L=8192, n_hh=16, seed=930)
+    dev = torch.device("cuda")
+    data = synth.make_batch(w, device=dev, steps=1)
+    C = 64
+    cl = sa.Clusters(w.B, w.Hkv, w.L, w.d, C, dev)
+    ys, oa = {}, {}
+    for g in range(w.Hkv):
+        k = f64(data["k"][0, g])
+        a, u32 = OA.qgc(f64(data["q_ctx"][0, g * w.G:(g + 1) * w.G]), k, C)
+        cl.basis[0, g] = torch.from_numpy(u32.T.copy()).float().to(dev)
+        ys[g], oa[g] = k @ u32[:, :16], a
+    sa.cluster_build(data["q_ctx"], data["k"], data["v"], clusters=cl, basis_given=True)
+    torch.cuda.synchronize()
+    for g in range(w.Hkv):
+        got = cl.assign[0, g].cpu().long().numpy()
+        assert (got == oa[g]).mean() >= 0.97, (got == oa[g]).mean()
+
+        def objective(a):
+            return sum(((ys[g][a == c] - ys[g][a == c].mean(axis=0)) ** 2).sum() for c in range(C) if (a == c).any())
+        assert objective(got) <= 1.01 * objective(oa[g])
+        # the sums and codes that follow are those of that assignment
+        cs = OA.cluster_stats(f64(data["k"][0, g]), f64(data["v"][0, g]), got, C)
+        assert cl.count[0, g].cpu().tolist() == cs["n"].tolist()
+        np.testing.assert_allclose(f64(cl.sum_k[0, g]), cs["sum_k"], rtol=1e-6, atol=1e-3)
+
+
+def test_build_then_step_reads_the_budget():
+    w = synth.scaled(synth.WORKLOADS["batched"], B=4, L=8192)
+    dev = torch.device("cuda")
+    data = synth.make_batch(w, device=dev, steps=1)
+    cl = sa.cluster_build(data["q_ctx"], data["k"], data["v"])
+    out, read, qcnt = sa.multi_step(data["q"][0], data["k"], data["v"], cl, 82)
+    torch.cuda.synchronize()
+    assert (qcnt.sum(-1) == 82).all() and (read >= 0).all()
+    assert torch.isfinite(out).all()
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            r = read[b, g].cpu().numpy()
+            a = cl.assign[b, g].cpu().long().numpy()
+            assert len(set(r.tolist())) == 82
+            assert np.bincount(a[r], minlength=64).tolist() == qcnt[b, g].cpu().tolist()
