@@ -64,6 +64,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-selectors", action="store_true", help="skip the alternative block scores")
+    ap.add_argument("--no-multi", action="store_true", help="skip the multi-proxy (clustered) path")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--batch", type=int, default=0, help="override the batch size (profiling cases)")
     return ap.parse_args(argv)
@@ -387,6 +388,17 @@ def main(argv=None):
     pf_bytes = (data["q_ctx"].numel() + 2 * data["k"].numel()) * data["k"].element_size()
     prefill = {"ms": statistics.mean(pf_ms), "hbm_gbs": pf_bytes / (statistics.mean(pf_ms) * 1e-3) / 1e9,
                "bytes": pf_bytes}
+    # the multi-proxy path's clusters (query-geometry clustering, once per
+    # sequence at prefill end): timed once, kept for the per-step timing
+    clusters, qgc_ms = None, None
+    if not args.no_multi:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        sa.cluster_build(data["q_ctx"][:1], data["k"][:1], data["v"][:1], n_clusters=64)     # warm-up (one sequence)
+        e0.record()
+        clusters = sa.cluster_build(data["q_ctx"], data["k"], data["v"], n_clusters=64)
+        e1.record()
+        torch.cuda.synchronize()
+        qgc_ms = e0.elapsed_time(e1)
     del data["q_ctx"]
     torch.cuda.empty_cache()
     K, V, Q = data["k"], data["v"], data["q"]
@@ -626,6 +638,37 @@ def main(argv=None):
                                 "select_frac": s_bytes / (s_ms * 1e-3) / 1e9 / peak}
         stats.blk_min = stats.blk_max = None
 
+    # the multi-proxy path (OpenAttention stages 02-04): ErrorGate split, the
+    # QGS selector and a proxy per cluster, with the same number of tokens
+    # read exactly as the block path
+    multi = None
+    if clusters is not None:
+        budget_m = sg["n_i"]
+        mout = torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=dev)
+        mread = torch.empty(w.B, w.Hkv, budget_m, dtype=torch.int32, device=dev)
+        mcnt = torch.empty(w.B, w.Hkv, 64, dtype=torch.int32, device=dev)
+
+        def multi_fn(t, ev):
+            ev[0].record(stream)
+            sa.multi_step(Q[t % nq], K, V, clusters, budget_m, read=mread, read_count=mcnt, out=mout)
+            ev[1].record(stream)
+        timed(3, multi_fn, 2)
+        pm_ = timed(args.mode_steps, multi_fn, 2)
+        m_ms = statistics.mean(p_[0] for p_ in pm_)
+        o_m, _, _ = sa.multi_step(Q[0], K, V, clusters, budget_m)
+        o_d = sa.dense_decode(Q[0], K, V)
+        err = ((o_m.double() - o_d.double()).norm() / o_d.double().norm()).item()
+        # per unit: codes (32 B), scale and cluster id per token; the basis and
+        # the clusters' count and key / squared-key / value sums; queries; the
+        # read rows; the read list and counts; the output
+        C_ = 64
+        m_bytes = (w.L * (32 + 4 + 1) + 32 * w.d * 4 + C_ * (4 + 3 * w.d * 4) + w.G * w.d * esz
+                   + budget_m * 2 * w.d * esz + budget_m * 4 + C_ * 4 + w.G * w.d * 4) * w.B * w.Hkv
+        multi = {"tokens_per_s": ws * w.B / (m_ms * 1e-3), "ms_per_step": m_ms, "read_tokens": budget_m,
+                 "clusters": C_, "bytes_per_step": m_bytes, "gbs": m_bytes / (m_ms * 1e-3) / 1e9,
+                 "frac": m_bytes / (m_ms * 1e-3) / 1e9 / peak, "rel_l2_vs_dense": err,
+                 "cluster_build_ms": qgc_ms}
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
         rate, units, threads = cpu_oracle_sample(w, sp_kw, args.mode, args.cpu_seconds)
@@ -656,7 +699,7 @@ def main(argv=None):
             "dense": dense, "speedup_vs_dense": dense_ms / ms_per_step, "modes": mode_vals,
             "kernels_us": {"k_select": 1e3 * sel_avg, "k_decode": 1e3 * dec_avg,
                            "separate_sum": 1e3 * (sel_avg + dec_avg), "step_overlapped": 1e3 * ms_per_step},
-            "append": append, "prefill": prefill, "selectors": selectors,
+            "append": append, "prefill": prefill, "selectors": selectors, "multi_proxy": multi,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step(w, sg, clt) * args.steps,
             "clocks": clk,
         }
