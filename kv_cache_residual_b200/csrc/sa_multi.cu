@@ -57,8 +57,16 @@ struct MultiIo {
     int32_t* read;                      // [U][budget]
     int32_t* qcnt;                      // [U][C]
     unsigned long long* keys;           // [U][ld] workspace
+    int* list;                          // [U][ld] workspace: the candidates left after two digits
     float* out;                         // [B][Hq][D]
 };
+
+// d = a . b + c over four byte lanes, a signed and b unsigned
+__device__ __forceinline__ int dp4a_su(int a, unsigned b, int c) {
+    int d;
+    asm("dp4a.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
 
 // ---- prefill: codes and cluster sums -----------------------------------------------
 
@@ -76,10 +84,19 @@ k_cluster_codes(const T* __restrict__ k, sa_clusters cl, int L, int ld) {
         const T* row = k + ((size_t)u * ld + j) * D;
         for (int e = lane; e < D; e += 32) s_row[warp][e] = to_f32<T>(row[e]);
         __syncwarp();
-        double s = 0.0, c = 0.0;
-#pragma unroll 8
-        for (int e = 0; e < D; ++e) two_sum_acc(s, c, __dmul_rn((double)basis[lane * D + e], (double)s_row[warp][e]));
-        const double z = __dadd_rn(s, c);
+        // four independent double-double chains over the dims, then combined
+        double s[4] = {0.0, 0.0, 0.0, 0.0}, c[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 4
+        for (int e = 0; e < D; e += 4)
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+                two_sum_acc(s[x], c[x], __dmul_rn((double)basis[lane * D + e + x], (double)s_row[warp][e + x]));
+#pragma unroll
+        for (int x = 1; x < 4; ++x) {
+            two_sum_acc(s[0], c[0], s[x]);
+            c[0] = __dadd_rn(c[0], c[x]);
+        }
+        const double z = __dadd_rn(s[0], c[0]);
         double amax = fabs(z);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) amax = fmax(amax, __shfl_xor_sync(0xffffffffu, amax, off));
@@ -109,14 +126,28 @@ k_cluster_stats(const T* __restrict__ k, const T* __restrict__ v, sa_clusters cl
     const T* V = v + (size_t)u * ld * D;
     const int e = threadIdx.x;
     if (e < D) {
-        for (int j = 0; j < L; ++j) {
-            const int c = a[j];
-            const double kx = (double)to_f32<T>(K[(size_t)j * D + e]);
-            const double vx = (double)to_f32<T>(V[(size_t)j * D + e]);
-            s_sum[c * D + e] += kx;
-            s_sum[(C + c) * D + e] += vx;
-            s_sum[(2 * C + c) * D + e] = fma(kx, kx, s_sum[(2 * C + c) * D + e]);
-            if (e == 0) s_cnt[c] += 1;
+        // eight tokens' loads in flight before their additions
+        constexpr int TU = 8;
+        for (int j0 = 0; j0 < L; j0 += TU) {
+            int cc[TU];
+            float kx[TU], vx[TU];
+#pragma unroll
+            for (int x = 0; x < TU; ++x) {
+                const int j = j0 + x;
+                cc[x] = j < L ? a[j] : -1;
+                kx[x] = j < L ? to_f32<T>(K[(size_t)j * D + e]) : 0.f;
+                vx[x] = j < L ? to_f32<T>(V[(size_t)j * D + e]) : 0.f;
+            }
+#pragma unroll
+            for (int x = 0; x < TU; ++x) {
+                const int c = cc[x];
+                if (c < 0) break;
+                const double kd = (double)kx[x], vd = (double)vx[x];
+                s_sum[c * D + e] += kd;
+                s_sum[(C + c) * D + e] += vd;
+                s_sum[(2 * C + c) * D + e] = fma(kd, kd, s_sum[(2 * C + c) * D + e]);
+                if (e == 0) s_cnt[c] += 1;
+            }
         }
     }
     __syncthreads();
@@ -138,6 +169,9 @@ k_multi_select(MultiIo io) {
     __shared__ float s_q[G][D];
     __shared__ double s_pp[NW][kQgsRank][2];               // partial projections (double-double)
     __shared__ int s_qq[kQgsRank];
+    __shared__ int s_qh[kQgsRank / 4];                     // qq = 256 qh + ql, packed bytes
+    __shared__ unsigned s_ql[kQgsRank / 4];
+    __shared__ int s_nlist;
     __shared__ double s_mu[G][kMaxClusters], s_sg[G][kMaxClusters];
     __shared__ double s_err[kMaxClusters];
     __shared__ long long s_w[kMaxClusters];
@@ -185,6 +219,18 @@ k_multi_select(MultiIo io) {
             qq = (int)fmax(-32767.0, fmin(32767.0, rint(p / sq)));
         }
         s_qq[lane] = qq;
+        // the 16-bit codes as a signed high byte and an unsigned low byte, packed
+        // four to a word for dp4a
+        const int qh = qq >> 8, ql = qq & 0xFF;
+        unsigned wh = (unsigned)(qh & 0xFF) << (8 * (lane & 3)), wl = (unsigned)ql << (8 * (lane & 3));
+        wh |= __shfl_xor_sync(0xffffffffu, wh, 1);
+        wl |= __shfl_xor_sync(0xffffffffu, wl, 1);
+        wh |= __shfl_xor_sync(0xffffffffu, wh, 2);
+        wl |= __shfl_xor_sync(0xffffffffu, wl, 2);
+        if ((lane & 3) == 0) {
+            s_qh[lane >> 2] = (int)wh;
+            s_ql[lane >> 2] = wl;
+        }
     }
 
     // 2. ErrorGate: member-logit mean and variance per (cluster, head)
@@ -316,33 +362,49 @@ k_multi_select(MultiIo io) {
     const int8_t* codes = io.cl.codes + (size_t)u * io.ld * kQgsRank;
     const float* sig = io.cl.scales + (size_t)u * io.ld;
     unsigned long long* keys = io.keys + (size_t)u * io.ld;
+    int* list = io.list + (size_t)u * io.ld;
+    int qh[kQgsRank / 4];
+    unsigned ql[kQgsRank / 4];
+#pragma unroll
+    for (int x = 0; x < kQgsRank / 4; ++x) { qh[x] = s_qh[x]; ql[x] = s_ql[x]; }
+    if (threadIdx.x == 0) s_nlist = 0;
     unsigned long long mask = 0ull;
     for (int shift = 56; shift >= 0; shift -= 8) {
         for (int x = threadIdx.x; x < C * 256; x += NT) s_hist[x] = 0u;
         __syncthreads();
-        for (int j = threadIdx.x; j < L; j += NT) {
-            unsigned long long key;
-            if (shift == 56) {
+        // the first two digits over every token; then over the candidates
+        // listed after them (those whose two top digits match their cluster's)
+        const bool all = shift >= 48;
+        const int n_it = all ? L : s_nlist;
+        for (int x = threadIdx.x; x < ((n_it + 31) & ~31); x += NT) {      // warp-uniform trip count
+            const bool live = x < n_it;
+            const int j = all ? x : (live ? list[x] : 0);
+            unsigned long long key = 0ull;
+            if (live && shift == 56) {
+                // the token's score: an exact integer dot with the 16-bit query
+                // code (high bytes signed, low bytes unsigned) times its scale
                 const int4* cr = reinterpret_cast<const int4*>(codes + (size_t)j * kQgsRank);
-                int dot = 0;
+                int hi = 0, lo = 0;
 #pragma unroll
                 for (int w4 = 0; w4 < kQgsRank / 16; ++w4) {
                     const int4 cw = __ldg(cr + w4);
                     const int wv[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
-                    for (int x = 0; x < 4; ++x)
-#pragma unroll
-                        for (int y = 0; y < 4; ++y) dot += s_qq[w4 * 16 + x * 4 + y] * (int)(int8_t)(wv[x] >> (8 * y));
+                    for (int y = 0; y < 4; ++y) {
+                        hi = __dp4a(wv[y], qh[w4 * 4 + y], hi);
+                        lo = dp4a_su(wv[y], ql[w4 * 4 + y], lo);
+                    }
                 }
+                const int dot = 256 * hi + lo;
                 const float sc = __double2float_rn((double)__ldg(sig + j) * (double)dot);   // exact product, one rounding
                 key = ((unsigned long long)fkey(sc) << 32) | (unsigned long long)(~(uint32_t)j);
                 keys[j] = key;
-            } else {
+            } else if (live) {
                 key = keys[j];
             }
-            const int c = __ldg(asg + j);
+            const int c = live ? __ldg(asg + j) : 0;
             int digit = 256;
-            if (s_rem[c] > 0 && (key & mask) == s_pre[c]) digit = (int)((key >> shift) & 0xFF);
+            if (live && s_rem[c] > 0 && (key & mask) == s_pre[c]) digit = (int)((key >> shift) & 0xFF);
             const unsigned bin = digit < 256 ? (unsigned)(c * 256 + digit) : 0xffffffffu;
             const unsigned peers = __match_any_sync(0xffffffffu, bin);
             if (digit < 256 && lane == __ffs(peers) - 1) atomicAdd(&s_hist[bin], (unsigned)__popc(peers));
@@ -376,6 +438,23 @@ k_multi_select(MultiIo io) {
         }
         mask |= 0xFFull << shift;
         __syncthreads();
+        if (shift == 48) {
+            // list the candidates still in play (order free: only counts follow)
+            for (int x = threadIdx.x; x < ((L + 31) & ~31); x += NT) {
+                bool in = false;
+                if (x < L) {
+                    const int c = __ldg(asg + x);
+                    in = s_rem[c] > 0 && (keys[x] & mask) == s_pre[c];
+                }
+                const unsigned m = __ballot_sync(0xffffffffu, in);
+                int base = 0;
+                if (lane == 0 && m != 0u) base = atomicAdd(&s_nlist, __popc(m));
+                base = __shfl_sync(0xffffffffu, base, 0);
+                if (in) list[base + __popc(m & ((1u << lane) - 1u))] = x;
+            }
+            __threadfence_block();
+            __syncthreads();
+        }
     }
 
     // 4. the read tokens, grouped by cluster: each thread counts its chunk's
@@ -547,7 +626,9 @@ cudaError_t launch_cluster_prep(const Dims& d, const void* k, const void* v, con
     return d.d == 128 ? prep_t<float, 128>(d, k, v, cl, C, s) : prep_t<float, 64>(d, k, v, cl, C, s);
 }
 
-size_t multi_workspace(const Dims& d) { return align256(sizeof(unsigned long long) * (size_t)d.U() * d.ld); }
+size_t multi_workspace(const Dims& d) {
+    return align256(sizeof(unsigned long long) * (size_t)d.U() * d.ld) + align256(sizeof(int) * (size_t)d.U() * d.ld);
+}
 
 template <typename T, int D, int G>
 static cudaError_t multi_t(const Dims& d, const MultiIo& io, cudaStream_t s) {
@@ -591,6 +672,7 @@ cudaError_t launch_multi_step(const Dims& d, const void* q, const void* k, const
     io.scale = scale;
     io.read = read; io.qcnt = qcnt;
     io.keys = reinterpret_cast<unsigned long long*>(ws);
+    io.list = reinterpret_cast<int*>(ws + align256(sizeof(unsigned long long) * (size_t)d.U() * d.ld));
     io.out = out;
     if (d.bf16) return d.d == 128 ? multi_g<__nv_bfloat16, 128>(d, io, s) : multi_g<__nv_bfloat16, 64>(d, io, s);
     return d.d == 128 ? multi_g<float, 128>(d, io, s) : multi_g<float, 64>(d, io, s);

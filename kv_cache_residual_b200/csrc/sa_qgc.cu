@@ -219,6 +219,10 @@ k_kmeans(const float* __restrict__ y, int L, int ld, int C, uint8_t* __restrict_
     __shared__ float s_c[64][R];
     __shared__ long long s_sum[64][R];
     __shared__ int s_n[64];
+    // each warp adds into its own copy (fewer colliding atomics), summed after
+    extern __shared__ __align__(16) long long s_wsum[];         // [kWarps][64][R]
+    int* s_wn = reinterpret_cast<int*>(s_wsum + kWarps * 64 * R);    // [kWarps][64]
+    const int warp = threadIdx.x >> 5;
     const int u = blockIdx.x;
     const float* yu = y + (size_t)u * ld * R;
     for (int x = threadIdx.x; x < C * R; x += kThreads) {
@@ -241,8 +245,8 @@ k_kmeans(const float* __restrict__ y, int L, int ld, int C, uint8_t* __restrict_
         return best;
     };
     for (int round = 0; round < kKmeansRounds; ++round) {
-        for (int x = threadIdx.x; x < C * R; x += kThreads) s_sum[x / R][x % R] = 0;
-        for (int x = threadIdx.x; x < C; x += kThreads) s_n[x] = 0;
+        for (int x = threadIdx.x; x < kWarps * 64 * R; x += kThreads) s_wsum[x] = 0;
+        for (int x = threadIdx.x; x < kWarps * 64; x += kThreads) s_wn[x] = 0;
         __syncthreads();
         for (int j = threadIdx.x; j < L; j += kThreads) {
             float v[R];
@@ -253,11 +257,22 @@ k_kmeans(const float* __restrict__ y, int L, int ld, int C, uint8_t* __restrict_
                 v[4 * i] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
             }
             const int c = nearest(v);
-            atomicAdd(&s_n[c], 1);
+            atomicAdd(&s_wn[warp * 64 + c], 1);
 #pragma unroll
             for (int i = 0; i < R; ++i)
-                atomicAdd(reinterpret_cast<unsigned long long*>(&s_sum[c][i]),
+                atomicAdd(reinterpret_cast<unsigned long long*>(&s_wsum[(warp * 64 + c) * R + i]),
                           (unsigned long long)llrint((double)v[i] * kFixScale));
+        }
+        __syncthreads();
+        for (int x = threadIdx.x; x < C * R; x += kThreads) {
+            long long t = 0;
+            for (int w = 0; w < kWarps; ++w) t += s_wsum[(w * 64 + x / R) * R + x % R];
+            s_sum[x / R][x % R] = t;
+        }
+        for (int x = threadIdx.x; x < C; x += kThreads) {
+            int t = 0;
+            for (int w = 0; w < kWarps; ++w) t += s_wn[w * 64 + x];
+            s_n[x] = t;
         }
         __syncthreads();
         for (int x = threadIdx.x; x < C * R; x += kThreads) {
@@ -319,8 +334,12 @@ static cudaError_t qgc_t(const Dims& d, const QgcPlan& p, const void* q_ctx, con
                                                        reinterpret_cast<float*>(ws + p.off_y));
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    k_kmeans<<<d.U(), kThreads, 0, s>>>(reinterpret_cast<const float*>(ws + p.off_y), d.L, d.ld, cl.n_clusters,
-                                        cl.assign);
+    constexpr size_t ksm = sizeof(long long) * kWarps * 64 * kClusterRank + sizeof(int) * kWarps * 64;
+    static std::atomic<unsigned long long> opted_k{0};
+    e = opt_in_smem(k_kmeans, ksm, opted_k);
+    if (e != cudaSuccess) return e;
+    k_kmeans<<<d.U(), kThreads, ksm, s>>>(reinterpret_cast<const float*>(ws + p.off_y), d.L, d.ld, cl.n_clusters,
+                                          cl.assign);
     return cudaGetLastError();
 }
 
