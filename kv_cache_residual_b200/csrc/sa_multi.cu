@@ -77,9 +77,12 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
 k_cluster_codes(const T* __restrict__ k, sa_clusters cl, int L, int ld) {
     __shared__ float s_row[kWarps][D];
+    __shared__ float s_b[kQgsRank][D + 1];           // the unit's basis, padded: lane i reads row i
     const int u = blockIdx.y;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const float* basis = cl.basis + (size_t)u * kQgsRank * D;
+    for (int x = threadIdx.x; x < kQgsRank * D; x += kThreads) s_b[x / D][x % D] = basis[x];
+    __syncthreads();
     for (int j = blockIdx.x * kWarps + warp; j < L; j += gridDim.x * kWarps) {
         const T* row = k + ((size_t)u * ld + j) * D;
         for (int e = lane; e < D; e += 32) s_row[warp][e] = to_f32<T>(row[e]);
@@ -90,7 +93,7 @@ k_cluster_codes(const T* __restrict__ k, sa_clusters cl, int L, int ld) {
         for (int e = 0; e < D; e += 4)
 #pragma unroll
             for (int x = 0; x < 4; ++x)
-                two_sum_acc(s[x], c[x], __dmul_rn((double)basis[lane * D + e + x], (double)s_row[warp][e + x]));
+                two_sum_acc(s[x], c[x], __dmul_rn((double)s_b[lane][e + x], (double)s_row[warp][e + x]));
 #pragma unroll
         for (int x = 1; x < 4; ++x) {
             two_sum_acc(s[0], c[0], s[x]);

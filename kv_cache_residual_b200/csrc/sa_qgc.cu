@@ -213,42 +213,64 @@ k_qproj(const T* __restrict__ k, const float* __restrict__ basis, int L, int ld,
 
 constexpr double kFixScale = 16777216.0;          // 2^24: member sums in 64-bit fixed point
 
-__global__ void __launch_bounds__(kThreads)
+constexpr int kKmThreads = 512;                   // k-means: one CTA of 16 warps per unit
+constexpr int kKmCopies = 8;                      // copies of the member sums (warp w adds to w % 8)
+
+__global__ void __launch_bounds__(kKmThreads, 1)
 k_kmeans(const float* __restrict__ y, int L, int ld, int C, uint8_t* __restrict__ assign) {
     constexpr int R = kClusterRank;
-    __shared__ float s_c[64][R];
+    __shared__ __align__(16) float s_c[64][R];
+    __shared__ float s_cn[64];                                  // |c|^2
     __shared__ long long s_sum[64][R];
     __shared__ int s_n[64];
     // each warp adds into its own copy (fewer colliding atomics), summed after
-    extern __shared__ __align__(16) long long s_wsum[];         // [kWarps][64][R]
-    int* s_wn = reinterpret_cast<int*>(s_wsum + kWarps * 64 * R);    // [kWarps][64]
-    const int warp = threadIdx.x >> 5;
+    extern __shared__ __align__(16) long long s_wsum[];         // [kKmCopies][64][R]
+    int* s_wn = reinterpret_cast<int*>(s_wsum + kKmCopies * 64 * R);    // [kKmCopies][64]
+    const int warp = (threadIdx.x >> 5) % kKmCopies;
     const int u = blockIdx.x;
     const float* yu = y + (size_t)u * ld * R;
-    for (int x = threadIdx.x; x < C * R; x += kThreads) {
+    for (int x = threadIdx.x; x < C * R; x += kKmThreads) {
         const int c = x / R;
         s_c[c][x % R] = yu[(size_t)(((long long)c * L) / C) * R + x % R];
     }
     __syncthreads();
+    auto norms = [&]() {
+        for (int c = threadIdx.x; c < C; c += kKmThreads) {
+            float t = 0.f;
+#pragma unroll
+            for (int i = 0; i < R; ++i) t = fmaf(s_c[c][i], s_c[c][i], t);
+            s_cn[c] = t;
+        }
+    };
+    // nearest centroid by |c|^2 - 2 v . c (|v - c|^2 less the common |v|^2),
+    // first minimum (lowest index) on ties
     auto nearest = [&](const float (&v)[R]) -> int {
+        float m2v[R];
+#pragma unroll
+        for (int i = 0; i < R; ++i) m2v[i] = -2.f * v[i];
         int best = 0;
         float bd = INFINITY;
         for (int c = 0; c < C; ++c) {
-            float d2 = 0.f;
+            float d2 = s_cn[c];
 #pragma unroll
-            for (int i = 0; i < R; ++i) {
-                const float t = v[i] - s_c[c][i];
-                d2 = fmaf(t, t, d2);
+            for (int i = 0; i < R; i += 4) {
+                const float4 cc = *reinterpret_cast<const float4*>(&s_c[c][i]);
+                d2 = fmaf(m2v[i], cc.x, d2);
+                d2 = fmaf(m2v[i + 1], cc.y, d2);
+                d2 = fmaf(m2v[i + 2], cc.z, d2);
+                d2 = fmaf(m2v[i + 3], cc.w, d2);
             }
-            if (d2 < bd) { bd = d2; best = c; }        // first minimum: lowest index
+            if (d2 < bd) { bd = d2; best = c; }
         }
         return best;
     };
+    norms();
+    __syncthreads();
     for (int round = 0; round < kKmeansRounds; ++round) {
-        for (int x = threadIdx.x; x < kWarps * 64 * R; x += kThreads) s_wsum[x] = 0;
-        for (int x = threadIdx.x; x < kWarps * 64; x += kThreads) s_wn[x] = 0;
+        for (int x = threadIdx.x; x < kKmCopies * 64 * R; x += kKmThreads) s_wsum[x] = 0;
+        for (int x = threadIdx.x; x < kKmCopies * 64; x += kKmThreads) s_wn[x] = 0;
         __syncthreads();
-        for (int j = threadIdx.x; j < L; j += kThreads) {
+        for (int j = threadIdx.x; j < L; j += kKmThreads) {
             float v[R];
             const float4* src = reinterpret_cast<const float4*>(yu + (size_t)j * R);
 #pragma unroll
@@ -264,24 +286,26 @@ k_kmeans(const float* __restrict__ y, int L, int ld, int C, uint8_t* __restrict_
                           (unsigned long long)llrint((double)v[i] * kFixScale));
         }
         __syncthreads();
-        for (int x = threadIdx.x; x < C * R; x += kThreads) {
+        for (int x = threadIdx.x; x < C * R; x += kKmThreads) {
             long long t = 0;
-            for (int w = 0; w < kWarps; ++w) t += s_wsum[(w * 64 + x / R) * R + x % R];
+            for (int w = 0; w < kKmCopies; ++w) t += s_wsum[(w * 64 + x / R) * R + x % R];
             s_sum[x / R][x % R] = t;
         }
-        for (int x = threadIdx.x; x < C; x += kThreads) {
+        for (int x = threadIdx.x; x < C; x += kKmThreads) {
             int t = 0;
-            for (int w = 0; w < kWarps; ++w) t += s_wn[w * 64 + x];
+            for (int w = 0; w < kKmCopies; ++w) t += s_wn[w * 64 + x];
             s_n[x] = t;
         }
         __syncthreads();
-        for (int x = threadIdx.x; x < C * R; x += kThreads) {
+        for (int x = threadIdx.x; x < C * R; x += kKmThreads) {
             const int c = x / R;
             if (s_n[c] > 0) s_c[c][x % R] = (float)((double)s_sum[c][x % R] / kFixScale / (double)s_n[c]);
         }
         __syncthreads();
+        norms();
+        __syncthreads();
     }
-    for (int j = threadIdx.x; j < L; j += kThreads) {
+    for (int j = threadIdx.x; j < L; j += kKmThreads) {
         float v[R];
         const float4* src = reinterpret_cast<const float4*>(yu + (size_t)j * R);
 #pragma unroll
@@ -334,11 +358,11 @@ static cudaError_t qgc_t(const Dims& d, const QgcPlan& p, const void* q_ctx, con
                                                        reinterpret_cast<float*>(ws + p.off_y));
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    constexpr size_t ksm = sizeof(long long) * kWarps * 64 * kClusterRank + sizeof(int) * kWarps * 64;
+    constexpr size_t ksm = sizeof(long long) * kKmCopies * 64 * kClusterRank + sizeof(int) * kKmCopies * 64;
     static std::atomic<unsigned long long> opted_k{0};
     e = opt_in_smem(k_kmeans, ksm, opted_k);
     if (e != cudaSuccess) return e;
-    k_kmeans<<<d.U(), kThreads, ksm, s>>>(reinterpret_cast<const float*>(ws + p.off_y), d.L, d.ld, cl.n_clusters,
+    k_kmeans<<<d.U(), kKmThreads, ksm, s>>>(reinterpret_cast<const float*>(ws + p.off_y), d.L, d.ld, cl.n_clusters,
                                           cl.assign);
     return cudaGetLastError();
 }
