@@ -189,15 +189,22 @@ typedef struct {
  *               basis); written by sa_cluster_build or by the caller
  *   assign      [B, Hkv, ld] uint8: each token's cluster (k-means of the keys
  *               projected on the first 16 rows); sa_cluster_build or caller
+ *   order       [B, Hkv, ld] int32: the token positions grouped by cluster
+ *               (cluster 0's members in ascending position, then cluster
+ *               1's, ...); written by sa_cluster_prep
+ *   start       [B, Hkv, C + 1] int32: cluster c's members are
+ *               order[start[c] .. start[c + 1]); written by sa_cluster_prep
  *   codes       [B, Hkv, ld, 32] int8 and scales [B, Hkv, ld] f32: the QGS
  *               codes of each key, z = basis . K_j (exact sums rounded once),
  *               sigma = fl32(max |z| / 127), code = clamp(rint(z / sigma),
- *               +-127); written by sa_cluster_prep
+ *               +-127), stored in the order of `order` (row i holds token
+ *               order[i], so that a cluster's codes are contiguous); written
+ *               by sa_cluster_prep
  *   count       [B, Hkv, C] int32 and sum_k, sum_v, sum_k2 [B, Hkv, C, d] f32:
  *               per cluster the member count and the sums of keys, values and
  *               squared keys (the cached mean and diagonal variance);
  *               written by sa_cluster_prep
- * Pointers 16-byte aligned. */
+ * Pointers non-null and 16-byte aligned. */
 typedef struct {
     int n_clusters;
     float* basis;
@@ -208,6 +215,8 @@ typedef struct {
     float* sum_k;
     float* sum_v;
     float* sum_k2;
+    int32_t* order;
+    int32_t* start;
 } sa_clusters;
 
 /* Which tokens one step reads exactly, and how the tail is sampled.
@@ -404,8 +413,8 @@ SA_API sa_status sa_cluster_build(const sa_shape* shape, const void* q_ctx, cons
                                   const sa_clusters* cl, int basis_given, void* ws, size_t ws_bytes, void* stream);
 
 /* The per-cluster state that follows from basis and assign over tokens
- * [0, L): the QGS codes and scales, the counts and the sums (layouts of
- * sa_clusters).  Prefill-time; no workspace. */
+ * [0, L): the cluster order and starts, the QGS codes and scales, the counts
+ * and the sums (layouts of sa_clusters).  Prefill-time; no workspace. */
 SA_API sa_status sa_cluster_prep(const sa_shape* shape, const void* k, const void* v, const sa_clusters* cl,
                                  void* stream);
 

@@ -62,7 +62,7 @@ class sa_selection(ctypes.Structure):
 class sa_clusters(ctypes.Structure):
     _fields_ = [("n_clusters", ctypes.c_int)] + [(n, ctypes.c_void_p) for n in
                                                   ("basis", "assign", "codes", "scales", "count", "sum_k", "sum_v",
-                                                   "sum_k2")]
+                                                   "sum_k2", "order", "start")]
 
 
 class sa_decode_params(ctypes.Structure):
@@ -218,7 +218,7 @@ class Clusters:
     """The multi-proxy state of a cache (caller-owned device tensors, layouts
     of sa_clusters in sa_decode.h)."""
 
-    FIELDS = ("basis", "assign", "codes", "scales", "count", "sum_k", "sum_v", "sum_k2")
+    FIELDS = ("basis", "assign", "codes", "scales", "count", "sum_k", "sum_v", "sum_k2", "order", "start")
 
     def __init__(self, B, Hkv, ld, d, n_clusters, device):
         f = dict(dtype=torch.float32, device=device)
@@ -231,6 +231,8 @@ class Clusters:
         self.sum_k = torch.zeros(B, Hkv, n_clusters, d, **f)
         self.sum_v = torch.zeros(B, Hkv, n_clusters, d, **f)
         self.sum_k2 = torch.zeros(B, Hkv, n_clusters, d, **f)
+        self.order = torch.zeros(B, Hkv, ld, dtype=torch.int32, device=device)
+        self.start = torch.zeros(B, Hkv, n_clusters + 1, dtype=torch.int32, device=device)
 
     def c(self):
         return sa_clusters(self.n_clusters, *[getattr(self, n).data_ptr() for n in self.FIELDS])

@@ -327,8 +327,11 @@ sa_status sa_step(const sa_shape* shape, const sa_decode_params* dparams, const 
 namespace {
 bool check_clusters(const sa_clusters* cl) {
     if (cl == nullptr || cl->n_clusters < 1 || cl->n_clusters > 64) return false;
-    return aligned16(cl->basis) && aligned16(cl->assign) && aligned16(cl->codes) && aligned16(cl->scales) &&
-           aligned16(cl->count) && aligned16(cl->sum_k) && aligned16(cl->sum_v) && aligned16(cl->sum_k2);
+    const void* p[] = {cl->basis, cl->assign, cl->codes, cl->scales, cl->count,
+                       cl->sum_k, cl->sum_v, cl->sum_k2, cl->order, cl->start};
+    for (const void* x : p)
+        if (x == nullptr || !aligned16(x)) return false;
+    return true;
 }
 }  // namespace
 

@@ -356,6 +356,35 @@ cudaError_t launch_decode(const Dims& d, const DecodePlan& p, const DecodeArgs& 
     return d.d == 128 ? decode_g<float, 128>(d, p, a, s) : decode_g<float, 64>(d, p, a, s);
 }
 
+template <int D, int G>
+static cudaError_t prefill_stream_t(const Dims& d, const PrefillPlan& p, const void* k, const void* v,
+                                    const sa_stats& st, float scale, char* part, char* cnt, cudaStream_t s) {
+    SetGeom sg{};
+    sa_selection sel{};
+    sa_select_params sp{};
+    return stream_launch<D, G, kPrefillMode>(d, dim3(p.nsp, d.U()), nullptr, k, v, st, sel, sp, sg, p.tpc, p.nsp,
+                                             p.rec_p, scale, 1.f, part, cnt, nullptr, false, s);
+}
+
+template <int D>
+static cudaError_t prefill_stream_g(const Dims& d, const PrefillPlan& p, const void* k, const void* v,
+                                    const sa_stats& st, float scale, char* part, char* cnt, cudaStream_t s) {
+    switch (d.G) {
+        case 1: return prefill_stream_t<D, 1>(d, p, k, v, st, scale, part, cnt, s);
+        case 2: return prefill_stream_t<D, 2>(d, p, k, v, st, scale, part, cnt, s);
+        case 4: return prefill_stream_t<D, 4>(d, p, k, v, st, scale, part, cnt, s);
+        case 8: return prefill_stream_t<D, 8>(d, p, k, v, st, scale, part, cnt, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_prefill_stream(const Dims& d, const PrefillPlan& p, const void* k, const void* v,
+                                  const sa_stats& st, float scale, char* part, char* cnt, cudaStream_t s) {
+    if (!d.bf16) return cudaErrorInvalidValue;
+    return d.d == 128 ? prefill_stream_g<128>(d, p, k, v, st, scale, part, cnt, s)
+                      : prefill_stream_g<64>(d, p, k, v, st, scale, part, cnt, s);
+}
+
 template <typename T, int D, int G>
 static cudaError_t dense_t(const Dims& d, const DensePlan& p, const DenseArgs& a, cudaStream_t s) {
     if constexpr (std::is_same<T, __nv_bfloat16>::value) {

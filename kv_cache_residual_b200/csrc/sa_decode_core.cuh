@@ -247,6 +247,15 @@ constexpr int kTcWarps = 4;        // 16 tokens per warp per tile
 constexpr int kTcThreads = 32 * kTcWarps;
 constexpr int kStages = 3;
 constexpr int kDenseMode = 4;      // MODE value of the dense pass
+constexpr int kPrefillMode = 5;    // MODE value of the prefill pass (RESA prior, totals, block means)
+
+// floats of a chunk record: exact (m, l, acc) and prior state per head, then
+// the key and value sums (proxy); the prefill pass keeps the key totals in
+// fp64 (2 d floats), the value totals and the largest |block mean| instead
+template <int D, int G, int MODE>
+__host__ __device__ constexpr int stream_rec() {
+    return MODE == kPrefillMode ? ((2 * G * (2 + D) + 3 * D + 1 + 3) & ~3) : 2 * G * (2 + D) + 2 * D;
+}
 
 template <int D>
 struct StageLayout {
@@ -260,18 +269,18 @@ constexpr int kBlkCache = 1024;
 constexpr int kSampCache = 256;
 
 template <int D, int G, int MODE>
-constexpr size_t stream_area_smem() {     // stages, then the merge / epilogue scratch over them
-    constexpr bool PRIOR = (MODE == SA_RESA);
+__host__ __device__ constexpr size_t stream_area_smem() {     // stages, then the merge / epilogue scratch over them
+    constexpr bool PRIOR = (MODE == SA_RESA || MODE == kPrefillMode);
     constexpr size_t ring = (size_t)kStages * StageLayout<D>::kBytes;
     constexpr size_t merge = (size_t)(kTcWarps * G * 4 + (PRIOR ? 2 : 1) * kTcWarps * G * D) * 4;
-    constexpr size_t tail = (size_t)(2 * G * (2 + D) + 2 * D) * 4        // own record
+    constexpr size_t tail = (size_t)stream_rec<D, G, MODE>() * 4       // own record
                             + (size_t)(2 * G * D + 4 * G + 2 * D + G) * 4;  // epilogue scratch
     constexpr size_t m = merge + tail;
     return ring > m ? ring : m;
 }
 
 template <int D, int G, int MODE>
-constexpr size_t stream_smem() {          // the stream kernel: area + the two list caches after the stages
+__host__ __device__ constexpr size_t stream_smem() {          // the stream kernel: area + the two list caches after the stages
     constexpr size_t lists = (size_t)kStages * StageLayout<D>::kBytes + (kBlkCache + kSampCache) * 4;
     constexpr size_t a = stream_area_smem<D, G, MODE>();
     return a > lists ? a : lists;
@@ -326,8 +335,10 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
     float* __restrict__ part = io.part;
     unsigned* __restrict__ cnt = io.cnt;
     float* __restrict__ out = io.out;
+    constexpr bool PREFILL = (MODE == kPrefillMode);   // the typical query over every token
     constexpr bool DENSE = (MODE == kDenseMode);
-    constexpr bool PRIOR = (MODE == SA_RESA);
+    constexpr bool ALL = DENSE || PREFILL;               // every token of the unit, no selection
+    constexpr bool PRIOR = (MODE == SA_RESA) || PREFILL;
     constexpr bool SUMS = (MODE == SA_PROXY);
     constexpr bool SAMP = (MODE == SA_SAMPLE);
     constexpr int P = tc::Pitch<D>::kBytes;
@@ -343,7 +354,7 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
     const size_t qh0 = (size_t)b * Hq + (size_t)g * G;
 
     // the epilogue's inputs (query, prefill statistics) into L2 while streaming
-    if constexpr (!DENSE) {
+    if constexpr (!ALL) {
         const int t = threadIdx.x;
         if (t * 64 < G * D * 2) prefetch_l2(reinterpret_cast<const char*>(qg) + t * 64);
         if constexpr (PRIOR) {
@@ -362,15 +373,15 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
         }
     }
 
-    const int nt = DENSE ? 0 : sg.n_t;
-    const int n_i = DENSE ? L : sg.n_i;
+    const int nt = ALL ? 0 : sg.n_t;
+    const int n_i = ALL ? L : sg.n_i;
     const int win0 = L - sg.w_eff;
     const int32_t* gblk = blk_idx + (size_t)u * kb_stride;
     const int32_t* gsamp = samp_idx + (size_t)u * (sample_cap > 0 ? sample_cap : 0);
     // rows [0, n_indep) do not depend on the selection; the tile range uses an
     // upper bound on the list length (draw capacity); the exact count and the
     // lists are read once the selection is visible
-    const int n_indep = DENSE ? L : sg.s_eff + sg.w_eff;
+    const int n_indep = ALL ? L : sg.s_eff + sg.w_eff;
     // per-head draws: head h's list follows head h-1's, each token tagged with
     // its head (it enters that head's softmax alone, weighted n_T / b_h)
     const bool PH = SAMP && io.per_head != 0;
@@ -381,12 +392,12 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
     for (int h = 0; h <= G; ++h) ph_pre[h] = 0;
 #pragma unroll
     for (int h = 0; h < G; ++h) ph_lw[h] = 0.f;
-    const int n_hi = DENSE ? L : sg.n_i + ((SAMP && nt > 0) ? (PH ? G : 1) * sample_cap : 0);
+    const int n_hi = ALL ? L : sg.n_i + ((SAMP && nt > 0) ? (PH ? G : 1) * sample_cap : 0);
     int n_tok = n_hi;
     float lw_samp = 0.f;
     const bool blk_sm = sg.kk <= kBlkCache;
     bool samp_sm = true;
-    bool sel_ready = DENSE || n_indep >= n_hi;
+    bool sel_ready = ALL || n_indep >= n_hi;
     // Under programmatic dependent launch the preceding selection kernel may
     // still be running: wait for it before the first selection-dependent read
     // (a no-op when the kernel was launched normally).  Called at the same
@@ -425,7 +436,7 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
     auto pos_of = [&](int t, int& tag) -> int {
         int p;
         tag = -1;
-        if (DENSE) p = t < L ? t : -1;
+        if (ALL) p = t < L ? t : -1;
         else if (t >= n_tok) p = -1;
         else if (t < sg.s_eff) p = t;
         else if (t < n_indep) p = win0 + (t - sg.s_eff);
@@ -493,7 +504,7 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
     constexpr bool kTokRows = (G <= 4);
     using Engine = typename std::conditional<kTokRows, tc::WarpAttnT<D, G, PRIOR>, tc::WarpAttn<D, G, PRIOR>>::type;
     Engine wa;
-    if constexpr (kTokRows) wa.load(qg, PRIOR ? st.mu_q + qh0 * D : nullptr);
+    if constexpr (kTokRows) wa.load(PREFILL ? nullptr : qg, PRIOR ? st.mu_q + qh0 * D : nullptr);
     __shared__ float s_bias[8];
     EpiPre<D, G> pre;
     BiasPre<D, G, kTcWarps> bpre;
@@ -513,9 +524,15 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
         wa.finish();
     } else {
         const int gh = min(lane >> 2, G - 1);
-        wa.init(qg + (size_t)gh * D, PRIOR ? st.mu_q + (qh0 + gh) * D : nullptr);
+        wa.init(PREFILL ? nullptr : qg + (size_t)gh * D, PRIOR ? st.mu_q + (qh0 + gh) * D : nullptr);
     }
     float ks[2] = {0.f, 0.f};      // SUMS: this thread's column pair of K (c < D/2) or V (c >= D/2)
+    // PREFILL: thread t takes the column pair (2c, 2c+1), c = t mod (D/2), of
+    // BPT of the tile's four 16-row blocks (group t / (D/2)): fp64 key sums,
+    // fp32 value sums, the largest |block mean|
+    constexpr int kPairs = D / 2, kGrp = kTcThreads / kPairs, kBpt = 4 / kGrp;
+    double pk[2] = {0.0, 0.0};
+    float pv[2] = {0.f, 0.f}, amax = 0.f;
     for (int i = tile0; i < tile1; ++i) {
         // the tile range was sized by the draw capacity: once the list length
         // is known, the tiles past it hold only masked rows (the copies of
@@ -541,6 +558,41 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
                     const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(src + r * P));
                     ks[0] += f.x;
                     ks[1] += f.y;
+                }
+            }
+        }
+        if constexpr (PREFILL) {
+            // block means: the fp64 sum of 16 rows times 1/16 (exact), one
+            // rounding to bf16 (L is a whole number of blocks)
+            const int c = threadIdx.x % kPairs, grp = threadIdx.x / kPairs;
+#pragma unroll
+            for (int bb = 0; bb < kBpt; ++bb) {
+                const int rb = (grp * kBpt + bb) * 16;
+                if (base + rb < L) {
+                    const unsigned char* kp = sb + rb * P + c * 4;
+                    double s0 = 0.0, s1 = 0.0;
+                    float w0 = 0.f, w1 = 0.f;
+#pragma unroll
+                    for (int r = 0; r < 16; ++r) {
+                        const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kp + r * P));
+                        const float2 vf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kp + TB + r * P));
+                        s0 += (double)kf.x;
+                        s1 += (double)kf.y;
+                        w0 += vf.x;
+                        w1 += vf.y;
+                    }
+                    __nv_bfloat162 mean;
+                    mean.x = round_from_f64<__nv_bfloat16>(s0 * 0.0625);
+                    mean.y = round_from_f64<__nv_bfloat16>(s1 * 0.0625);
+                    const size_t row = (size_t)u * (io.ld / 16) + (size_t)((base + rb) / 16);
+                    *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(st.blk_mean) + row * D + 2 * c) =
+                        mean;
+                    const float2 mf = __bfloat1622float2(mean);
+                    amax = fmaxf(amax, fmaxf(fabsf(mf.x), fabsf(mf.y)));
+                    pk[0] += s0;
+                    pk[1] += s1;
+                    pv[0] += w0;
+                    pv[1] += w1;
                 }
             }
         }
@@ -601,14 +653,14 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
     float* acc = ml + kTcWarps * G * 4;                 // [W][G][D]
     float* acc0 = acc + kTcWarps * G * D;               // [W][G][D] (PRIOR)
     float* own = acc + (PRIOR ? 2 : 1) * kTcWarps * G * D;   // own record when the unit is one chunk
-    float* scratch = own + 2 * G * (2 + D) + 2 * D;
+    float* scratch = own + stream_rec<D, G, MODE>();
     wa.store(ml, acc, acc0);
     if constexpr (PRIOR) {
         if (nt > 0) bias_sum<D, G, kTcWarps>(bpre, s_bias, scale);
     }
     __syncthreads();
     const bool single = (nchunk == 1);
-    if constexpr (!DENSE && !SUMS) {
+    if constexpr (!DENSE && !SUMS && !PREFILL) {
         if (single) {
             // the unit in one chunk: its output straight from the warps'
             // states (the merge, in warp order, then the mode's residual)
@@ -649,6 +701,38 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
     }
     float* r = single ? own : part + ((size_t)u * nchunk + chunk) * rec;
     tc::merge_warps<D, G, PRIOR>(ml, acc, acc0, kTcWarps, r);
+    if constexpr (PREFILL) {
+        // the chunk's totals (after the prior state): key sums in fp64, value
+        // sums, the largest |block mean|; thread partials meet in the
+        // list-cache area, which the prefill pass does not use
+        double* s_pk = reinterpret_cast<double*>(smem + (size_t)kStages * SB);     // [kGrp][D]
+        float* s_pv = reinterpret_cast<float*>(s_pk + kGrp * D);                  // [kGrp][D]
+        float* s_am = s_pv + kGrp * D;                                            // [warps]
+        const int c = threadIdx.x % kPairs, grp = threadIdx.x / kPairs;
+        s_pk[grp * D + 2 * c] = pk[0];
+        s_pk[grp * D + 2 * c + 1] = pk[1];
+        s_pv[grp * D + 2 * c] = pv[0];
+        s_pv[grp * D + 2 * c + 1] = pv[1];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if (lane == 0) s_am[warp] = amax;
+        __syncthreads();
+        double* rk = reinterpret_cast<double*>(r + 2 * G * (2 + D));
+        for (int e = threadIdx.x; e < D; e += kTcThreads) {
+            double a = 0.0;
+            float b2 = 0.f;
+#pragma unroll
+            for (int x = 0; x < kGrp; ++x) { a += s_pk[x * D + e]; b2 += s_pv[x * D + e]; }
+            rk[e] = a;
+            r[2 * G * (2 + D) + 2 * D + e] = b2;
+        }
+        if (threadIdx.x == 0) {
+            float a = 0.f;
+#pragma unroll
+            for (int w = 0; w < kTcWarps; ++w) a = fmaxf(a, s_am[w]);
+            r[2 * G * (2 + D) + 3 * D] = a;
+        }
+    }
     if constexpr (SUMS) {
         if (threadIdx.x < D) {
             const int c = threadIdx.x;
@@ -670,23 +754,91 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
     float* s_t = s_ml + 4 * G;
     float* s_hs = s_t + 2 * D;
     const float* recs = single ? own : part + (size_t)u * nchunk * rec;
-    if constexpr (DENSE) {
-        if (single) combine_heads<G, D, true>(recs, 1, rec, 0, s_ml, s_ml + G);
-        else combine_heads<G, D, false>(recs, nchunk, rec, 0, s_ml, s_ml + G);
+    // The other chunks' records into shared memory (after the scratch) with
+    // every load in flight at once, when they fit: combining them straight
+    // from L2 chains one round trip per few records and elements.  Dense
+    // needs only the exact state (the first G (2 + D) floats of a record).
+    int rs = rec;
+    bool sh = single;
+    if (!single) {
+        const int w = DENSE ? G * (2 + D) : rec;
+        const int o = (int)(s_hs + G - fb + 3) & ~3;                 // float index, 16-byte aligned
+        if ((w & 3) == 0 && (size_t)(o + nchunk * w) * 4 <= stream_smem<D, G, MODE>()) {
+            float4* dst = reinterpret_cast<float4*>(fb + o);
+            const int w4 = w / 4, n4 = nchunk * w4;
+            constexpr int UN = 8;
+            for (int x0 = 0; x0 < n4; x0 += UN * kTcThreads) {
+                float4 t[UN];
+#pragma unroll
+                for (int j = 0; j < UN; ++j) {
+                    const int x = x0 + j * kTcThreads + threadIdx.x;
+                    if (x < n4) {
+                        const int c = x / w4, y = x - c * w4;
+                        t[j] = __ldcg(reinterpret_cast<const float4*>(recs + (size_t)c * rec) + y);
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < UN; ++j) {
+                    const int x = x0 + j * kTcThreads + threadIdx.x;
+                    if (x < n4) dst[x] = t[j];
+                }
+            }
+            __syncthreads();
+            recs = fb + o;
+            rs = w;
+            sh = true;
+        }
+    }
+    if constexpr (PREFILL) {
+        // O_Est and log Z of the typical queries (the prior state), the key
+        // and value totals in chunk order, the largest |block mean|
+        constexpr int OP = G * (2 + D), OS = 2 * G * (2 + D);
+        if (sh) combine_heads<G, D, true>(recs, nchunk, rs, OP, s_ml, s_ml + G);
+        else combine_heads<G, D, false>(recs, nchunk, rs, OP, s_ml, s_ml + G);
         __syncthreads();
         for (int idx = threadIdx.x; idx < G * D; idx += kTcThreads) {
             const int h = idx / D, e = idx - h * D;
-            const float A = single ? combine_acc<G, D, true>(recs, 1, rec, 0, h, e, s_ml[h])
-                                   : combine_acc<G, D, false>(recs, nchunk, rec, 0, h, e, s_ml[h]);
+            const float A = sh ? combine_acc<G, D, true>(recs, nchunk, rs, OP, h, e, s_ml[h])
+                               : combine_acc<G, D, false>(recs, nchunk, rs, OP, h, e, s_ml[h]);
+            st.o_est[(qh0 + h) * D + e] = A / s_ml[G + h];
+            if (e == 0) st.log_z0[qh0 + h] = (s_ml[h] + log2f(s_ml[G + h])) * kLn2;
+        }
+        for (int e = threadIdx.x; e < D; e += kTcThreads) {
+            double a = 0.0;
+            float b2 = 0.f;
+            for (int c = 0; c < nchunk; ++c) {
+                const float* rc = recs + (size_t)c * rs;
+                a += sh ? reinterpret_cast<const double*>(rc + OS)[e] : __ldcg(reinterpret_cast<const double*>(rc + OS) + e);
+                b2 += sh ? rc[OS + 2 * D + e] : __ldcg(rc + OS + 2 * D + e);
+            }
+            st.sum_k[(size_t)u * D + e] = (float)a;
+            st.mu_k[(size_t)u * D + e] = (float)(a / (double)L);
+            st.sum_v[(size_t)u * D + e] = b2;
+        }
+        if (threadIdx.x == 0) {
+            float a = 0.f;
+            for (int c = 0; c < nchunk; ++c)
+                a = fmaxf(a, sh ? recs[(size_t)c * rs + OS + 3 * D] : __ldcg(recs + (size_t)c * rs + OS + 3 * D));
+            st.kbar_absmax[u] = a;
+        }
+    } else if constexpr (DENSE) {
+        if (sh) combine_heads<G, D, true>(recs, nchunk, rs, 0, s_ml, s_ml + G);
+        else combine_heads<G, D, false>(recs, nchunk, rs, 0, s_ml, s_ml + G);
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < G * D; idx += kTcThreads) {
+            const int h = idx / D, e = idx - h * D;
+            const float A = sh ? combine_acc<G, D, true>(recs, nchunk, rs, 0, h, e, s_ml[h])
+                               : combine_acc<G, D, false>(recs, nchunk, rs, 0, h, e, s_ml[h]);
             out[((size_t)b * Hq + g * G + h) * D + e] = A / s_ml[G + h];
         }
     } else {
         constexpr int EM = DENSE ? SA_DROP : MODE;
-        if (single)
-            decode_epilogue<__nv_bfloat16, D, G, EM, true>(recs, 1, rec, qg, st, u, b, g, Hq, nt, scale, lambda,
-                                                           out, s_acc, s_acc0, s_ml, s_t, s_hs, &pre, s_bias);
+        if (sh)
+            decode_epilogue<__nv_bfloat16, D, G, EM, true>(recs, nchunk, rs, qg, st, u, b, g, Hq, nt, scale,
+                                                           lambda, out, s_acc, s_acc0, s_ml, s_t, s_hs, &pre,
+                                                           s_bias);
         else
-            decode_epilogue<__nv_bfloat16, D, G, EM, false>(recs, nchunk, rec, qg, st, u, b, g, Hq, nt, scale,
+            decode_epilogue<__nv_bfloat16, D, G, EM, false>(recs, nchunk, rs, qg, st, u, b, g, Hq, nt, scale,
                                                             lambda, out, s_acc, s_acc0, s_ml, s_t, s_hs, &pre,
                                                             s_bias);
     }

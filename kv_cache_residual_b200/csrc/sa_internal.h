@@ -15,6 +15,7 @@ namespace sa {
 
 constexpr int kSmTarget = 148 * 4;   // CTAs to aim for: 4 per SM on B200
 constexpr int kStreamSlots = 148 * 2; // resident CTAs of the bf16 stream kernel (2 per SM)
+constexpr int kSelectSlots = 148 * 2; // resident scanning CTAs of the selection (2 per SM): one wave
 
 struct Dims {
     int B, Hq, Hkv, G, d, L;
@@ -61,6 +62,10 @@ struct PrefillPlan {
     int nskv, tok_kv;            // KV-pass splits per unit, tokens per split (x16)
     size_t off_qpart, off_qcnt, off_kvpart, off_kvcnt, bytes;
     int kv_stride;               // floats per KV-pass partial record
+    // bf16 caches: the KV pass on the tensor-core stream kernel, chunks of
+    // tpc 64-token tiles (about one wave), rec floats per chunk record (in
+    // the off_kvpart area)
+    int nsp, tpc, rec_p;
 };
 
 inline PrefillPlan prefill_plan(const Dims& d) {
@@ -81,7 +86,15 @@ inline PrefillPlan prefill_plan(const Dims& d) {
     p.off_qcnt = off;  off = align256(off + sizeof(unsigned) * (size_t)BH);
     p.off_kvcnt = off; off = align256(off + sizeof(unsigned) * (size_t)d.U());
     p.off_qpart = off; off = align256(off + sizeof(float) * (size_t)BH * p.nsq * d.d);
-    p.off_kvpart = off; off = align256(off + sizeof(float) * (size_t)d.U() * p.nskv * p.kv_stride);
+    // bf16: the stream kernel's chunks (as the dense pass) and records of
+    // the exact and prior states, fp64 key sums, value sums, absmax
+    const int ntiles = cdiv(d.L, 64);
+    p.nsp = clampi(kStreamSlots / d.U(), 1, ntiles);
+    p.tpc = cdiv(ntiles, p.nsp);
+    p.nsp = cdiv(ntiles, p.tpc);
+    p.rec_p = (2 * d.G * (2 + d.d) + 3 * d.d + 1 + 3) & ~3;
+    const size_t kv_floats = (size_t)d.U() * (size_t)(d.bf16 ? p.nsp * p.rec_p : p.nskv * p.kv_stride);
+    p.off_kvpart = off; off = align256(off + sizeof(float) * kv_floats);
     p.bytes = off;
     return p;
 }
@@ -98,8 +111,8 @@ inline SelectPlan select_plan(const Dims& d, const sa_select_params& sp) {
     p.g = set_geom(d, sp.sink, sp.local, sp.k_blocks);
     const int nc = p.g.n_cand > 0 ? p.g.n_cand : 1;
     // enough units to fill the GPU: one CTA per unit (scores stay on chip);
-    // otherwise split units so the grid is about one wave, >= 32 rows per CTA
-    p.nss = d.U() >= 148 ? 1 : clampi(kSmTarget / d.U(), 1, cdiv(nc, 32));
+    // otherwise split units so the grid is one wave, >= 32 rows per CTA
+    p.nss = d.U() >= 148 ? 1 : clampi(kSelectSlots / d.U(), 1, cdiv(nc, 32));
     p.rows_s = cdiv(nc, p.nss);
     p.nss = cdiv(nc, p.rows_s);
     size_t off = 0;
@@ -259,6 +272,11 @@ cudaError_t launch_cluster_build(const Dims& d, const QgcPlan& p, const void* q_
                                  const sa_clusters& cl, bool basis_given, char* ws, cudaStream_t s);
 
 // The multi-proxy path (sa_multi.cu)
+// The prefill KV pass of bf16 caches on the tensor-core stream kernel (prior
+// state of mu_Q, totals, block means, largest |block mean|): st.mu_q must be
+// set; part / cnt: records and tickets of the prefill plan.
+cudaError_t launch_prefill_stream(const Dims& d, const PrefillPlan& p, const void* k, const void* v,
+                                  const sa_stats& st, float scale, char* part, char* cnt, cudaStream_t s);
 cudaError_t launch_cluster_prep(const Dims& d, const void* k, const void* v, const sa_clusters& cl, cudaStream_t s);
 size_t multi_workspace(const Dims& d);
 cudaError_t launch_multi_step(const Dims& d, const void* q, const void* k, const void* v, const sa_clusters& cl,

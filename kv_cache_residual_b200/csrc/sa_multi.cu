@@ -8,15 +8,20 @@
 //   basis  [32][D] f32   the QGS basis (rows: the eigenvectors of the query
 //                        second moment, decreasing eigenvalue; the first 16
 //                        are the clustering basis)
-//   codes  [ld][32] int8 and scales [ld] f32: each key in that basis,
-//          z = basis . K_j (the exact sum rounded once), sigma = fl32(max|z| /
-//          127), code = clamp(rint(z / sigma), +-127)
 //   assign [ld] u8       the token's cluster
+//   order  [ld] i32, start [C+1] i32: the positions grouped by cluster
+//                        (ascending within a cluster), cluster c at
+//                        order[start[c] .. start[c+1])
+//   codes  [ld][32] int8 and scales [ld] f32 in that order: each key in the
+//          basis, z = basis . K_j (the exact sum rounded once), sigma =
+//          fl32(max|z| / 127), code = clamp(rint(z / sigma), +-127)
 //   count [C] i32, sum_k, sum_v, sum_k2 [C][D] f32   cluster sums
 //
-// k_cluster_codes: codes and scales from the basis (prefill).
-// k_cluster_stats: count and sums from the assignment (prefill).
-// k_multi_select (per step, one CTA of 256 threads per unit):
+// Prefill: k_cluster_order (stable counting sort of the positions by
+// cluster), k_cluster_codes (codes and scales), k_cluster_stats (counts and
+// sums).
+// Per step, two kernels (the second a programmatic dependent of the first):
+// k_multi_gate (one CTA of 256 threads per unit):
 //   1. the group's projected query p_i = basis_i . sum_h q_h (exact sums
 //      rounded once), coded to 16 bits: sq = max |p| / 32767, qq = rint(p/sq);
 //   2. ErrorGate: per cluster and head the member-logit mean mu = s q_h .
@@ -25,19 +30,22 @@
 //      sum n e^(mu + var/2), summed over the heads; the errors made integers
 //      w = rint(2^30 err / max err) and the budget E split exactly:
 //      q_c = min(n_c, floor(E w_c / W)), the rest one token at a time by
-//      largest remainder (E w_c mod W), lowest cluster first, round after round;
-//   3. QGS: every token's score fl32(sigma_j (qq . code_j)) (exact integer dot)
-//      as a 64-bit key (score, then lower position first); per cluster the
-//      q_c-th largest key by an 8-digit radix select run for all clusters at
-//      once (per-cluster histograms in shared memory, keys in the workspace);
-//   4. the read tokens written grouped by cluster (cluster order, ascending
-//      positions), and q_c.
-// k_multi_decode (per step, one CTA of 256 threads per unit): each warp takes
-//   clusters c = warp, warp + 8, ...: its read rows (lane groups over rows,
-//   fp32 online softmax per head) while summing their keys and values, then
-//   the cluster's proxy for its n' = n_c - q_c unread members: key (sum_k -
-//   read keys) / n', value likewise, logit s q . key + ln n'.  Warps merge in
-//   order; out = acc / l.
+//      largest remainder (E w_c mod W), lowest cluster first, round after
+//      round; q_c, the clusters' offsets in the read list and the packed
+//      query code go to the workspace.
+// k_multi_pick (grid (C/8, U), a warp per cluster):
+//   3. QGS: each member's score fl32(sigma_j (qq . code_j)) (exact integer
+//      dot, dp4a) as an order-preserving 32-bit key; the q_c-th largest by a
+//      4-digit radix select over the cluster's keys (shared memory, or the
+//      workspace for clusters of more than kPickKeys members); the members
+//      above it and the first of those equal to it (ascending positions: the
+//      tie rule) are written to the read list in position order;
+//   4. the warp's read rows (lane groups over rows, fp32 online softmax per
+//      head) while summing their keys and values, then the cluster's proxy
+//      for its n' = n_c - q_c unread members: key (sum_k - read keys) / n',
+//      value likewise, logit s q . key + ln n'.  Warps merge in order into a
+//      CTA record; the unit's last CTA (completion ticket) combines the
+//      records in order; out = acc / l.
 #include "sa_cta.cuh"
 #include "sa_internal.h"
 #include "sa_select_core.cuh"
@@ -56,9 +64,14 @@ struct MultiIo {
     float scale;
     int32_t* read;                      // [U][budget]
     int32_t* qcnt;                      // [U][C]
-    unsigned long long* keys;           // [U][ld] workspace
-    int* list;                          // [U][ld] workspace: the candidates left after two digits
     float* out;                         // [B][Hq][D]
+    // workspace
+    int* wq;                            // [U][16]: the query code, 8 words of signed high bytes, 8 of low bytes
+    int* woff;                          // [U][kMaxClusters + 1]: cluster offsets in the read list
+    uint32_t* wkeys;                    // [U][ld]: score keys of clusters too large for shared memory
+    float* part;                        // [U][kPickCtas][G (2 + D)]: CTA records
+    unsigned* cnt;                      // [U]: completion tickets
+    int npick;                          // pick CTAs per unit
 };
 
 // d = a . b + c over four byte lanes, a signed and b unsigned
@@ -70,9 +83,65 @@ __device__ __forceinline__ int dp4a_su(int a, unsigned b, int c) {
 
 // ---- prefill: codes and cluster sums -----------------------------------------------
 
-// One warp per token: lane i forms z_i = basis_i . K_j in double-double (the
-// products of fp32 and bf16 / fp32 values are exact in fp64), the scale and
-// the codes follow.
+// One CTA per unit: a stable counting sort of the positions by cluster.  The
+// counts give start[]; then 256 positions at a time (one per thread, in
+// position order) each token's slot = its cluster's running offset + the
+// members of its cluster before it in this chunk (earlier warps, then lower
+// lanes of its own warp).
+__global__ void __launch_bounds__(kThreads)
+k_cluster_order(sa_clusters cl, int L, int ld, int C) {
+    __shared__ int s_cnt[kMaxClusters];
+    __shared__ int s_run[kMaxClusters];
+    __shared__ int s_wc[kWarps][kMaxClusters];
+    const int u = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint8_t* a = cl.assign + (size_t)u * ld;
+    for (int c = threadIdx.x; c < kMaxClusters; c += kThreads) s_cnt[c] = 0;
+    __syncthreads();
+    for (int j = threadIdx.x; j < L; j += kThreads) {
+        const int c = __ldg(a + j);
+        if (c < C) atomicAdd(&s_cnt[c], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int off = 0;
+        for (int c = 0; c < C; ++c) {
+            cl.start[(size_t)u * (C + 1) + c] = off;
+            s_run[c] = off;
+            off += s_cnt[c];
+        }
+        cl.start[(size_t)u * (C + 1) + C] = off;
+    }
+    const unsigned lt = (1u << lane) - 1u;
+    for (int j0 = 0; j0 < L; j0 += kThreads) {
+        for (int x = threadIdx.x; x < kWarps * kMaxClusters; x += kThreads) (&s_wc[0][0])[x] = 0;
+        __syncthreads();
+        const int j = j0 + threadIdx.x;
+        int c = j < L ? __ldg(a + j) : 255;
+        if (c >= C) c = 255;                                     // outside the clusters: not placed
+        const unsigned peers = __match_any_sync(0xffffffffu, c);
+        const int rank = __popc(peers & lt);
+        if (c != 255 && rank == 0) s_wc[warp][c] = __popc(peers);
+        __syncthreads();
+        int slot = 0;
+        if (c != 255) {
+            slot = s_run[c] + rank;
+            for (int w = 0; w < warp; ++w) slot += s_wc[w][c];
+        }
+        __syncthreads();                                         // every slot read s_run before it moves
+        if (c != 255) cl.order[(size_t)u * ld + slot] = j;
+        for (int x = threadIdx.x; x < C; x += kThreads) {
+            int t = 0;
+            for (int w = 0; w < kWarps; ++w) t += s_wc[w][x];
+            s_run[x] += t;
+        }
+        __syncthreads();
+    }
+}
+
+// One warp per slot i (token j = order[i]): lane r forms z_r = basis_r . K_j
+// in double-double (the products of fp32 and bf16 / fp32 values are exact in
+// fp64), the scale and the codes follow, stored at slot i.
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
 k_cluster_codes(const T* __restrict__ k, sa_clusters cl, int L, int ld) {
@@ -83,7 +152,8 @@ k_cluster_codes(const T* __restrict__ k, sa_clusters cl, int L, int ld) {
     const float* basis = cl.basis + (size_t)u * kQgsRank * D;
     for (int x = threadIdx.x; x < kQgsRank * D; x += kThreads) s_b[x / D][x % D] = basis[x];
     __syncthreads();
-    for (int j = blockIdx.x * kWarps + warp; j < L; j += gridDim.x * kWarps) {
+    for (int i = blockIdx.x * kWarps + warp; i < L; i += gridDim.x * kWarps) {
+        const int j = __ldg(cl.order + (size_t)u * ld + i);           // slot i holds token j
         const T* row = k + ((size_t)u * ld + j) * D;
         for (int e = lane; e < D; e += 32) s_row[warp][e] = to_f32<T>(row[e]);
         __syncwarp();
@@ -106,8 +176,8 @@ k_cluster_codes(const T* __restrict__ k, sa_clusters cl, int L, int ld) {
         const float sig = __double2float_rn(amax / 127.0);
         int code = 0;
         if (sig > 0.f) code = max(-127, min(127, (int)rint(z / (double)sig)));
-        cl.codes[((size_t)u * ld + j) * kQgsRank + lane] = (int8_t)code;
-        if (lane == 0) cl.scales[(size_t)u * ld + j] = sig;
+        cl.codes[((size_t)u * ld + i) * kQgsRank + lane] = (int8_t)code;
+        if (lane == 0) cl.scales[(size_t)u * ld + i] = sig;
         __syncwarp();
     }
 }
@@ -163,29 +233,28 @@ k_cluster_stats(const T* __restrict__ k, const T* __restrict__ v, sa_clusters cl
     for (int x = threadIdx.x; x < C; x += kThreads) cl.count[(size_t)u * C + x] = s_cnt[x];
 }
 
-// ---- per step: the selection -----------------------------------------------------------
+// ---- per step: ErrorGate and the query code ----------------------------------------
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads)
-k_multi_select(MultiIo io) {
+k_multi_gate(MultiIo io) {
     constexpr int NT = kThreads, NW = kWarps;
     __shared__ float s_q[G][D];
     __shared__ double s_pp[NW][kQgsRank][2];               // partial projections (double-double)
     __shared__ int s_qq[kQgsRank];
     __shared__ int s_qh[kQgsRank / 4];                     // qq = 256 qh + ql, packed bytes
     __shared__ unsigned s_ql[kQgsRank / 4];
-    __shared__ int s_nlist;
     __shared__ double s_mu[G][kMaxClusters], s_sg[G][kMaxClusters];
     __shared__ double s_err[kMaxClusters];
     __shared__ long long s_w[kMaxClusters];
     __shared__ int s_qc[kMaxClusters], s_off[kMaxClusters + 1], s_rem[kMaxClusters];
-    __shared__ unsigned long long s_pre[kMaxClusters];
-    extern __shared__ __align__(16) unsigned s_hist[];      // [C][256] (also [C][NT] counts at the end)
+    // the pick kernel may start now: it waits for this grid before reading
+    // what this kernel writes
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 
     const int u = blockIdx.x, b = u / io.Hkv, g = u - b * io.Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int C = io.C, L = io.L;
+    const int C = io.C;
     const T* qg = static_cast<const T*>(io.q) + ((size_t)b * io.Hq + (size_t)g * G) * D;
     for (int i = threadIdx.x; i < G * D; i += NT) s_q[i / D][i % D] = to_f32<T>(qg[i]);
     __syncthreads();
@@ -195,12 +264,21 @@ k_multi_select(MultiIo io) {
     {
         const float* basis = io.cl.basis + (size_t)u * kQgsRank * D;
         constexpr int EW = D / NW;
+        // the lane's EW basis entries, every load in flight at once
+        float bv[EW];
+#pragma unroll
+        for (int j = 0; j < EW; j += 4) {
+            const float4 f = __ldg(reinterpret_cast<const float4*>(basis + (size_t)lane * D + warp * EW + j));
+            bv[j] = f.x; bv[j + 1] = f.y; bv[j + 2] = f.z; bv[j + 3] = f.w;
+        }
         double s = 0.0, c = 0.0;
-        for (int e = warp * EW; e < (warp + 1) * EW; ++e) {
+#pragma unroll
+        for (int j = 0; j < EW; ++j) {
+            const int e = warp * EW + j;
             double qb = 0.0;
 #pragma unroll
             for (int h = 0; h < G; ++h) qb += (double)s_q[h][e];          // exact: G bf16 / fp32 values
-            two_sum_acc(s, c, __dmul_rn(qb, (double)basis[lane * D + e]));
+            two_sum_acc(s, c, __dmul_rn(qb, (double)bv[j]));
         }
         s_pp[warp][lane][0] = s;
         s_pp[warp][lane][1] = c;
@@ -239,16 +317,34 @@ k_multi_select(MultiIo io) {
     // 2. ErrorGate: member-logit mean and variance per (cluster, head)
     const double scale = (double)io.scale;
     const int32_t* cnt = io.cl.count + (size_t)u * C;
-    for (int c = warp; c < C; c += NW) {
-        const int n = __ldg(cnt + c);
-        const float* sk = io.cl.sum_k + ((size_t)u * C + c) * D;
-        const float* sk2 = io.cl.sum_k2 + ((size_t)u * C + c) * D;
+    // the warp's clusters c = warp, warp + 8, ...: their counts and sums
+    // loaded first, all in flight together
+    constexpr int CPW = kMaxClusters / NW;
+    int rn[CPW];
+    float rk[CPW][D / 32], rk2[CPW][D / 32];
+#pragma unroll
+    for (int y = 0; y < CPW; ++y) {
+        const int c = warp + y * NW;
+        const bool ok = c < C;
+        rn[y] = ok ? __ldg(cnt + c) : 0;
+        const float* sk = io.cl.sum_k + ((size_t)u * C + (ok ? c : 0)) * D;
+        const float* sk2 = io.cl.sum_k2 + ((size_t)u * C + (ok ? c : 0)) * D;
+#pragma unroll
+        for (int x = 0; x < D / 32; ++x) {
+            rk[y][x] = ok ? __ldg(sk + lane + 32 * x) : 0.f;
+            rk2[y][x] = ok ? __ldg(sk2 + lane + 32 * x) : 0.f;
+        }
+    }
+#pragma unroll
+    for (int y = 0; y < CPW; ++y) {
+        const int c = warp + y * NW;
+        if (c >= C) break;                                 // uniform in the warp
+        const int n = rn[y];
         double mean[D / 32], var[D / 32];
 #pragma unroll
         for (int x = 0; x < D / 32; ++x) {
-            const int e = lane + 32 * x;
-            mean[x] = n > 0 ? (double)sk[e] / (double)n : 0.0;
-            var[x] = n > 0 ? fmax((double)sk2[e] / (double)n - mean[x] * mean[x], 0.0) : 0.0;
+            mean[x] = n > 0 ? (double)rk[y][x] / (double)n : 0.0;
+            var[x] = n > 0 ? fmax((double)rk2[y][x] / (double)n - mean[x] * mean[x], 0.0) : 0.0;
         }
 #pragma unroll
         for (int h = 0; h < G; ++h) {
@@ -298,27 +394,51 @@ k_multi_select(MultiIo io) {
         for (int x = 0; x < kMaxClusters / 32; ++x)
             if (lane + 32 * x < C) s_err[lane + 32 * x] = err[x];
         __syncwarp();
-        // the clusters' weights as integers, and their order for the tokens
-        // left after the floors: remainder desc, lowest cluster on ties
-        // (lanes rank two clusters each against all)
+        // the clusters' weights as integers, their floors and remainders (the
+        // lane of each cluster), then their order for the tokens left after
+        // the floors: remainder desc, lowest cluster on ties (lanes rank two
+        // clusters each against all, from shared memory)
         double top = 0.0;
-        for (int c = 0; c < C; ++c) top = fmax(top, s_err[c]);
-        long long W = 0;
-        for (int c = 0; c < C; ++c) W += top > 0.0 ? (long long)rint(s_err[c] / top * 1073741824.0) : 0;
-        long long total = 0;
-        for (int c = 0; c < C; ++c) total += __ldg(cnt + c);
+        for (int c = lane; c < C; c += 32) top = fmax(top, s_err[c]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) top = fmax(top, __shfl_xor_sync(0xffffffffu, top, o));
+        long long wl[kMaxClusters / 32], W = 0, total = 0;
+#pragma unroll
+        for (int x = 0; x < kMaxClusters / 32; ++x) {
+            const int c = lane + 32 * x;
+            wl[x] = (c < C && top > 0.0) ? (long long)rint(s_err[c] / top * 1073741824.0) : 0;
+            W += wl[x];
+            total += c < C ? __ldg(cnt + c) : 0;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            W += __shfl_xor_sync(0xffffffffu, W, o);
+            total += __shfl_xor_sync(0xffffffffu, total, o);
+        }
         const long long E = min((long long)io.budget, total);
+        long long floors = 0;
 #pragma unroll
         for (int x = 0; x < kMaxClusters / 32; ++x) {
             const int c = lane + 32 * x;
             if (c < C) {
-                const long long wc = top > 0.0 ? (long long)rint(s_err[c] / top * 1073741824.0) : 0;
-                s_w[c] = wc;
-                const long long rc = W > 0 ? (E * wc) % W : 0;
+                const long long n = __ldg(cnt + c);
+                const long long qc = W > 0 ? min(n, E * wl[x] / W) : 0;
+                s_qc[c] = (int)qc;
+                s_w[c] = W > 0 ? (E * wl[x]) % W : 0;       // (the remainder)
+                floors += qc;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) floors += __shfl_xor_sync(0xffffffffu, floors, o);
+        __syncwarp();
+#pragma unroll
+        for (int x = 0; x < kMaxClusters / 32; ++x) {
+            const int c = lane + 32 * x;
+            if (c < C) {
+                const long long rc = s_w[c];
                 int rank = 0;
                 for (int o = 0; o < C; ++o) {
-                    const long long wo = top > 0.0 ? (long long)rint(s_err[o] / top * 1073741824.0) : 0;
-                    const long long ro = W > 0 ? (E * wo) % W : 0;
+                    const long long ro = s_w[o];
                     rank += (ro > rc || (ro == rc && o < c)) ? 1 : 0;
                 }
                 s_rem[rank] = c;                      // (reused: the order)
@@ -326,15 +446,7 @@ k_multi_select(MultiIo io) {
         }
         __syncwarp();
         if (lane == 0) {
-            // integer split of the budget (exact)
-            for (int c = 0; c < C; ++c) top = fmax(top, s_err[c]);
-            long long left = E;
-            for (int c = 0; c < C; ++c) {
-                const long long n = __ldg(cnt + c);
-                const long long qc = W > 0 ? min(n, E * s_w[c] / W) : 0;
-                s_qc[c] = (int)qc;
-                left -= qc;
-            }
+            long long left = E - floors;
             // one token at a time in that order, round after round
             while (left > 0) {
                 bool gave = false;
@@ -352,186 +464,59 @@ k_multi_select(MultiIo io) {
             for (int c = 0; c < C; ++c) {
                 s_off[c] = off;
                 off += s_qc[c];
-                s_rem[c] = s_qc[c];
-                s_pre[c] = 0ull;
             }
             s_off[C] = off;
         }
     }
     __syncthreads();
-
-    // 3. scores as keys (score desc, position asc), and the per-cluster radix select
-    const uint8_t* asg = io.cl.assign + (size_t)u * io.ld;
-    const int8_t* codes = io.cl.codes + (size_t)u * io.ld * kQgsRank;
-    const float* sig = io.cl.scales + (size_t)u * io.ld;
-    unsigned long long* keys = io.keys + (size_t)u * io.ld;
-    int* list = io.list + (size_t)u * io.ld;
-    int qh[kQgsRank / 4];
-    unsigned ql[kQgsRank / 4];
-#pragma unroll
-    for (int x = 0; x < kQgsRank / 4; ++x) { qh[x] = s_qh[x]; ql[x] = s_ql[x]; }
-    if (threadIdx.x == 0) s_nlist = 0;
-    unsigned long long mask = 0ull;
-    for (int shift = 56; shift >= 0; shift -= 8) {
-        for (int x = threadIdx.x; x < C * 256; x += NT) s_hist[x] = 0u;
-        __syncthreads();
-        // the first two digits over every token; then over the candidates
-        // listed after them (those whose two top digits match their cluster's)
-        const bool all = shift >= 48;
-        const int n_it = all ? L : s_nlist;
-        for (int x = threadIdx.x; x < ((n_it + 31) & ~31); x += NT) {      // warp-uniform trip count
-            const bool live = x < n_it;
-            const int j = all ? x : (live ? list[x] : 0);
-            unsigned long long key = 0ull;
-            if (live && shift == 56) {
-                // the token's score: an exact integer dot with the 16-bit query
-                // code (high bytes signed, low bytes unsigned) times its scale
-                const int4* cr = reinterpret_cast<const int4*>(codes + (size_t)j * kQgsRank);
-                int hi = 0, lo = 0;
-#pragma unroll
-                for (int w4 = 0; w4 < kQgsRank / 16; ++w4) {
-                    const int4 cw = __ldg(cr + w4);
-                    const int wv[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-                    for (int y = 0; y < 4; ++y) {
-                        hi = __dp4a(wv[y], qh[w4 * 4 + y], hi);
-                        lo = dp4a_su(wv[y], ql[w4 * 4 + y], lo);
-                    }
-                }
-                const int dot = 256 * hi + lo;
-                const float sc = __double2float_rn((double)__ldg(sig + j) * (double)dot);   // exact product, one rounding
-                key = ((unsigned long long)fkey(sc) << 32) | (unsigned long long)(~(uint32_t)j);
-                keys[j] = key;
-            } else if (live) {
-                key = keys[j];
-            }
-            const int c = live ? __ldg(asg + j) : 0;
-            int digit = 256;
-            if (live && s_rem[c] > 0 && (key & mask) == s_pre[c]) digit = (int)((key >> shift) & 0xFF);
-            const unsigned bin = digit < 256 ? (unsigned)(c * 256 + digit) : 0xffffffffu;
-            const unsigned peers = __match_any_sync(0xffffffffu, bin);
-            if (digit < 256 && lane == __ffs(peers) - 1) atomicAdd(&s_hist[bin], (unsigned)__popc(peers));
-        }
-        __syncthreads();
-        // per cluster: the digit at which the count from the top reaches rem
-        for (int c = warp; c < C; c += NW) {
-            const int rem = s_rem[c];
-            if (rem <= 0) continue;
-            unsigned cc[8], loc = 0;
-#pragma unroll
-            for (int y = 0; y < 8; ++y) { cc[y] = s_hist[c * 256 + 255 - 8 * lane - y]; loc += cc[y]; }
-            unsigned inc = loc;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const unsigned o = __shfl_up_sync(0xffffffffu, inc, off);
-                if (lane >= off) inc += o;
-            }
-            unsigned ex = inc - loc;
-            if (ex < (unsigned)rem && inc >= (unsigned)rem) {
-#pragma unroll
-                for (int y = 0; y < 8; ++y) {
-                    if (ex + cc[y] >= (unsigned)rem) {
-                        s_pre[c] |= (unsigned long long)(255 - 8 * lane - y) << shift;
-                        s_rem[c] = rem - (int)ex;
-                        break;
-                    }
-                    ex += cc[y];
-                }
-            }
-        }
-        mask |= 0xFFull << shift;
-        __syncthreads();
-        if (shift == 48) {
-            // list the candidates still in play (order free: only counts follow)
-            for (int x = threadIdx.x; x < ((L + 31) & ~31); x += NT) {
-                bool in = false;
-                if (x < L) {
-                    const int c = __ldg(asg + x);
-                    in = s_rem[c] > 0 && (keys[x] & mask) == s_pre[c];
-                }
-                const unsigned m = __ballot_sync(0xffffffffu, in);
-                int base = 0;
-                if (lane == 0 && m != 0u) base = atomicAdd(&s_nlist, __popc(m));
-                base = __shfl_sync(0xffffffffu, base, 0);
-                if (in) list[base + __popc(m & ((1u << lane) - 1u))] = x;
-            }
-            __threadfence_block();
-            __syncthreads();
-        }
-    }
-
-    // 4. the read tokens, grouped by cluster: each thread counts its chunk's
-    // selected tokens per cluster, a scan per cluster gives the places
-    const int chunk = (L + NT - 1) / NT;
-    const int j0 = min(L, (int)threadIdx.x * chunk), j1 = min(L, j0 + chunk);
-    unsigned* s_cnt = s_hist;                                 // [C][NT]
-    for (int x = threadIdx.x; x < C * NT; x += NT) s_cnt[x] = 0u;
-    __syncthreads();
-    for (int j = j0; j < j1; ++j) {
-        const int c = __ldg(asg + j);
-        if (s_qc[c] > 0 && keys[j] >= s_pre[c]) s_cnt[c * NT + threadIdx.x] += 1u;
-    }
-    __syncthreads();
-    for (int c = warp; c < C; c += NW) {                     // exclusive scan over threads, per cluster
-        unsigned v[NT / 32], loc = 0;
-#pragma unroll
-        for (int y = 0; y < NT / 32; ++y) { v[y] = s_cnt[c * NT + lane * (NT / 32) + y]; loc += v[y]; }
-        unsigned inc = loc;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const unsigned o = __shfl_up_sync(0xffffffffu, inc, off);
-            if (lane >= off) inc += o;
-        }
-        unsigned ex = inc - loc + (unsigned)s_off[c];
-#pragma unroll
-        for (int y = 0; y < NT / 32; ++y) {
-            const unsigned t = v[y];
-            s_cnt[c * NT + lane * (NT / 32) + y] = ex;
-            ex += t;
-        }
-    }
-    __syncthreads();
-    int32_t* rd = io.read + (size_t)u * io.budget;
-    for (int j = j0; j < j1; ++j) {
-        const int c = __ldg(asg + j);
-        if (s_qc[c] > 0 && keys[j] >= s_pre[c]) {
-            const unsigned p = s_cnt[c * NT + threadIdx.x]++;
-            if (p < (unsigned)io.budget) rd[p] = j;
-        }
-    }
-    for (int p = s_off[C] + threadIdx.x; p < io.budget; p += NT) rd[p] = -1;
+    // the budgets, the offsets, the query code; -1 after the last read slot
     for (int c = threadIdx.x; c < C; c += NT) io.qcnt[(size_t)u * C + c] = s_qc[c];
+    for (int c = threadIdx.x; c <= C; c += NT) io.woff[(size_t)u * (kMaxClusters + 1) + c] = s_off[c];
+    if (threadIdx.x < kQgsRank / 4) {
+        io.wq[(size_t)u * 16 + threadIdx.x] = s_qh[threadIdx.x];
+        io.wq[(size_t)u * 16 + 8 + threadIdx.x] = (int)s_ql[threadIdx.x];
+    }
+    for (int r = s_off[C] + threadIdx.x; r < io.budget; r += NT) io.read[(size_t)u * io.budget + r] = -1;
 }
 
-// ---- per step: the decode ---------------------------------------------------------------
+// ---- per step: per-cluster top-q and the softmax with the proxies ----------------------
+
+constexpr int kPickWarps = kWarps;      // clusters per CTA
+constexpr int kPickCtas = kMaxClusters / kPickWarps;
+constexpr int kPickKeys = 1024;         // keys per warp in shared memory
+
+// dynamic shared memory of k_multi_pick: the keys and histograms (the
+// cross-warp merge area aliases them), then the CTA record
+template <int G, int D>
+struct PickSmem {
+    static constexpr size_t kPick = (size_t)kPickWarps * kPickKeys * 4 + (size_t)kPickWarps * 256 * 4;
+    static constexpr size_t kMerge = (size_t)kWarps * G * (D + 2) * 4;
+    static constexpr size_t kArea = kPick > kMerge ? kPick : kMerge;
+    static constexpr size_t kBytes = kArea + (size_t)G * (2 + D) * 4;
+};
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads)
-k_multi_decode(MultiIo io) {
+k_multi_pick(MultiIo io) {
     using Gm = Geom<T, D>;
     constexpr int EPC = Gm::EPC, CPR = Gm::CPR, GPW = Gm::GPW;
-    __shared__ float sm[kWarps * G * (D + 2)];
-    __shared__ float s_rec[G * (2 + D)];
-    __shared__ int s_qc[kMaxClusters + 1];
-    // the selection may still be running (programmatic dependent launch)
-    asm volatile("griddepcontrol.wait;\n" ::: "memory");
-    const int u = blockIdx.x, b = u / io.Hkv, g = u - b * io.Hkv;
+    extern __shared__ __align__(16) unsigned char smem[];
+    uint32_t* s_keys = reinterpret_cast<uint32_t*>(smem);                       // [warps][kPickKeys]
+    unsigned* s_hist = reinterpret_cast<unsigned*>(smem) + kPickWarps * kPickKeys;   // [warps][256]
+    float* sm = reinterpret_cast<float*>(smem);                                // merge area (aliases)
+    float* s_rec = reinterpret_cast<float*>(smem + PickSmem<G, D>::kArea);
+
+    const int u = blockIdx.y, b = u / io.Hkv, g = u - b * io.Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int li = lane % CPR, gsub = lane / CPR;
     const int C = io.C;
+    const int c = blockIdx.x * kPickWarps + warp;
+    const bool has = c < C;
     const float qscale = io.scale * kLog2e;
     const T* qg = static_cast<const T*>(io.q) + ((size_t)b * io.Hq + (size_t)g * G) * D;
     const T* K = static_cast<const T*>(io.k) + (size_t)u * io.ld * D + li * EPC;
     const T* V = static_cast<const T*>(io.v) + (size_t)u * io.ld * D + li * EPC;
-    if (threadIdx.x == 0) {
-        int off = 0;
-        for (int c = 0; c < C; ++c) {
-            s_qc[c] = off;
-            off += __ldcg(io.qcnt + (size_t)u * C + c);
-        }
-        s_qc[C] = off;
-    }
-    __syncthreads();
+    // what does not depend on the gate: the query, the cluster's extent
     float qv[G][EPC];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -540,78 +525,218 @@ k_multi_decode(MultiIo io) {
 #pragma unroll
         for (int e = 0; e < EPC; ++e) qv[h][e] = f[e] * qscale;
     }
+    const int* st = io.cl.start + (size_t)u * (C + 1);
+    const int n0 = has ? __ldg(st + c) : 0, n = has ? __ldg(st + c + 1) - n0 : 0;
+    const int nc = has ? __ldg(io.cl.count + (size_t)u * C + c) : 0;
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    const int qc = has ? __ldcg(io.qcnt + (size_t)u * C + c) : 0;
+    const int off = has ? __ldcg(io.woff + (size_t)u * (kMaxClusters + 1) + c) : 0;
+    int32_t* rd = io.read + (size_t)u * io.budget + off;
+    const int32_t* ord = io.cl.order + (size_t)u * io.ld + n0;
+    const unsigned lt = (1u << lane) - 1u;
+
+    // 3. the cluster's top qc (all of it when qc >= n)
+    if (qc >= n) {
+        for (int i = lane; i < n; i += 32) rd[i] = __ldg(ord + i);
+    } else if (qc > 0) {
+        int qh[kQgsRank / 4];
+        unsigned ql[kQgsRank / 4];
+#pragma unroll
+        for (int x = 0; x < kQgsRank / 4; ++x) {
+            qh[x] = __ldcg(io.wq + (size_t)u * 16 + x);
+            ql[x] = (unsigned)__ldcg(io.wq + (size_t)u * 16 + 8 + x);
+        }
+        uint32_t* keys = n <= kPickKeys ? s_keys + warp * kPickKeys : io.wkeys + (size_t)u * io.ld + n0;
+        const int8_t* codes = io.cl.codes + ((size_t)u * io.ld + n0) * kQgsRank;
+        const float* sig = io.cl.scales + (size_t)u * io.ld + n0;
+        for (int i = lane; i < n; i += 32) {
+            // an exact integer dot with the 16-bit query code (high bytes
+            // signed, low bytes unsigned) times the token's scale, rounded once
+            const int4* cr = reinterpret_cast<const int4*>(codes + (size_t)i * kQgsRank);
+            int hi = 0, lo = 0;
+#pragma unroll
+            for (int w4 = 0; w4 < kQgsRank / 16; ++w4) {
+                const int4 cw = __ldg(cr + w4);
+                const int wv[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+                for (int y = 0; y < 4; ++y) {
+                    hi = __dp4a(wv[y], qh[w4 * 4 + y], hi);
+                    lo = dp4a_su(wv[y], ql[w4 * 4 + y], lo);
+                }
+            }
+            const int dot = 256 * hi + lo;
+            keys[i] = fkey(__double2float_rn((double)__ldg(sig + i) * (double)dot));
+        }
+        __syncwarp();
+        // radix select of the qc-th largest key, 8 bits at a time
+        unsigned* hist = s_hist + warp * 256;
+        uint32_t pre = 0u, mask = 0u;
+        int rem = qc;
+        for (int shift = 24; shift >= 0; shift -= 8) {
+#pragma unroll
+            for (int y = 0; y < 8; ++y) hist[lane * 8 + y] = 0u;
+            __syncwarp();
+            for (int i0 = 0; i0 < n; i0 += 32) {
+                const int i = i0 + lane;
+                const uint32_t key = i < n ? keys[i] : 0u;
+                const unsigned bin = (i < n && (key & mask) == pre) ? ((key >> shift) & 0xFFu) : 256u;
+                const unsigned peers = __match_any_sync(0xffffffffu, bin);
+                if (bin < 256u && (peers & lt) == 0u) atomicAdd(&hist[bin], (unsigned)__popc(peers));
+            }
+            __syncwarp();
+            // lane l holds bins 255 - 8l - y; the digit where the count from the top reaches rem
+            unsigned cc[8], loc = 0;
+#pragma unroll
+            for (int y = 0; y < 8; ++y) { cc[y] = hist[255 - 8 * lane - y]; loc += cc[y]; }
+            unsigned inc = loc;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned t = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += t;
+            }
+            unsigned ex = inc - loc;
+            int dig = -1, nrem = 0;
+            if (ex < (unsigned)rem && inc >= (unsigned)rem) {
+#pragma unroll
+                for (int y = 0; y < 8; ++y) {
+                    if (dig < 0 && ex + cc[y] >= (unsigned)rem) {
+                        dig = 255 - 8 * lane - y;
+                        nrem = rem - (int)ex;
+                    }
+                    if (dig < 0) ex += cc[y];
+                }
+            }
+            const unsigned who = __ballot_sync(0xffffffffu, dig >= 0);
+            const int src = __ffs(who) - 1;
+            dig = __shfl_sync(0xffffffffu, dig, src);
+            rem = __shfl_sync(0xffffffffu, nrem, src);
+            pre |= (uint32_t)dig << shift;
+            mask |= 0xFFu << shift;
+            __syncwarp();
+        }
+        // the keys above pre, and the first rem equal to it, in slot order
+        int taken = 0, eqs = 0;
+        for (int i0 = 0; i0 < n; i0 += 32) {
+            const int i = i0 + lane;
+            const uint32_t key = i < n ? keys[i] : 0u;
+            const bool eq = i < n && key == pre;
+            const unsigned em = __ballot_sync(0xffffffffu, eq);
+            const bool take = (i < n && key > pre) || (eq && eqs + __popc(em & lt) < rem);
+            const unsigned tm = __ballot_sync(0xffffffffu, take);
+            if (take) rd[taken + __popc(tm & lt)] = __ldg(ord + i);
+            taken += __popc(tm);
+            eqs += __popc(em);
+        }
+    }
+    __syncwarp();                       // the warp's read list is visible to the warp
+
+    // 4. exact rows of the cluster, then its proxy
     Online<G, EPC> os;
     os.init();
-    const int32_t* rd = io.read + (size_t)u * io.budget;
-    for (int c = warp; c < C; c += kWarps) {
-        const int r0 = s_qc[c], r1 = s_qc[c + 1];
-        float ks[EPC], vs[EPC];
+    const int q_eff = qc < n ? qc : n;
+    float ks[EPC], vs[EPC];
 #pragma unroll
-        for (int e = 0; e < EPC; ++e) { ks[e] = 0.f; vs[e] = 0.f; }
-        for (int rb = r0; rb < r1; rb += GPW) {              // warp-uniform
-            const int r = rb + gsub;
-            const bool ok = r < r1;
-            const int p = ok ? __ldcg(rd + r) : 0;
-            float kf[EPC], vf[EPC];
-            unpack<T>(ok ? ld_nc16(K + (size_t)p * D) : make_uint4(0, 0, 0, 0), kf);
-            unpack<T>(ok ? ld_nc16(V + (size_t)p * D) : make_uint4(0, 0, 0, 0), vf);
+    for (int e = 0; e < EPC; ++e) { ks[e] = 0.f; vs[e] = 0.f; }
+    for (int rb = 0; rb < q_eff; rb += GPW) {              // warp-uniform
+        const int r = rb + gsub;
+        const bool ok = r < q_eff;
+        const int p = ok ? __ldcg(rd + r) : 0;
+        float kf[EPC], vf[EPC];
+        unpack<T>(ok ? ld_nc16(K + (size_t)p * D) : make_uint4(0, 0, 0, 0), kf);
+        unpack<T>(ok ? ld_nc16(V + (size_t)p * D) : make_uint4(0, 0, 0, 0), vf);
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-                float x = 0.f;
+        for (int h = 0; h < G; ++h) {
+            float x = 0.f;
 #pragma unroll
-                for (int e = 0; e < EPC; ++e) x = fmaf(qv[h][e], kf[e], x);
-                x = group_sum<CPR>(x);
-                if (ok) os.add(h, x, vf);
-            }
-#pragma unroll
-            for (int e = 0; e < EPC; ++e) { ks[e] += kf[e]; vs[e] += vf[e]; }
+            for (int e = 0; e < EPC; ++e) x = fmaf(qv[h][e], kf[e], x);
+            x = group_sum<CPR>(x);
+            if (ok) os.add(h, x, vf);
         }
-        // the cluster's read sums in every lane group, then its proxy
 #pragma unroll
-        for (int off = CPR; off < 32; off <<= 1)
+        for (int e = 0; e < EPC; ++e) { ks[e] += kf[e]; vs[e] += vf[e]; }
+    }
 #pragma unroll
-            for (int e = 0; e < EPC; ++e) {
-                ks[e] += __shfl_xor_sync(0xffffffffu, ks[e], off);
-                vs[e] += __shfl_xor_sync(0xffffffffu, vs[e], off);
-            }
-        const int n_un = __ldg(io.cl.count + (size_t)u * C + c) - (r1 - r0);
-        if (n_un > 0) {
-            const float* sk = io.cl.sum_k + ((size_t)u * C + c) * D + li * EPC;
-            const float* sv = io.cl.sum_v + ((size_t)u * C + c) * D + li * EPC;
-            const float inv = 1.f / (float)n_un;
-            float kb[EPC], vb[EPC];
+    for (int o = CPR; o < 32; o <<= 1)
 #pragma unroll
-            for (int e = 0; e < EPC; ++e) {
-                kb[e] = (__ldg(sk + e) - ks[e]) * inv;
-                vb[e] = (__ldg(sv + e) - vs[e]) * inv;
-            }
-            const float lnn = log2f((float)n_un);
+        for (int e = 0; e < EPC; ++e) {
+            ks[e] += __shfl_xor_sync(0xffffffffu, ks[e], o);
+            vs[e] += __shfl_xor_sync(0xffffffffu, vs[e], o);
+        }
+    const int n_un = nc - q_eff;
+    if (has && n_un > 0) {
+        const float* sk = io.cl.sum_k + ((size_t)u * C + c) * D + li * EPC;
+        const float* sv = io.cl.sum_v + ((size_t)u * C + c) * D + li * EPC;
+        const float inv = 1.f / (float)n_un;
+        float kb[EPC], vb[EPC];
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-                float x = 0.f;
+        for (int e = 0; e < EPC; ++e) {
+            kb[e] = (__ldg(sk + e) - ks[e]) * inv;
+            vb[e] = (__ldg(sv + e) - vs[e]) * inv;
+        }
+        const float lnn = log2f((float)n_un);
 #pragma unroll
-                for (int e = 0; e < EPC; ++e) x = fmaf(qv[h][e], kb[e], x);
-                x = group_sum<CPR>(x) + lnn;
-                if (gsub == 0) os.add(h, x, vb);
-            }
+        for (int h = 0; h < G; ++h) {
+            float x = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) x = fmaf(qv[h][e], kb[e], x);
+            x = group_sum<CPR>(x) + lnn;
+            if (gsub == 0) os.add(h, x, vb);
         }
     }
     warp_merge<G, EPC, CPR>(os);
-    cta_merge_store<G, EPC, CPR, D>(os, sm, s_rec);
+    __syncthreads();                    // the merge area aliases the keys and histograms
+    float* rec = io.npick == 1 ? s_rec : io.part + ((size_t)u * kPickCtas + blockIdx.x) * Rec<G, D>::kFloats;
+    cta_merge_store<G, EPC, CPR, D>(os, sm, rec);
+    const float* recs = s_rec;
+    if (io.npick > 1) {
+        if (!last_cta_of_unit(io.cnt + u, (unsigned)io.npick)) return;
+        // the CTAs' records into shared memory (over the merge area) with
+        // every load in flight at once, then combined in CTA order
+        constexpr int RF = Rec<G, D>::kFloats;
+        const float* src = io.part + (size_t)u * kPickCtas * RF;
+        for (int x0 = 0; x0 < io.npick * RF; x0 += 8 * kThreads) {
+            float t[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int x = x0 + j * kThreads + threadIdx.x;
+                t[j] = x < io.npick * RF ? __ldcg(src + x) : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int x = x0 + j * kThreads + threadIdx.x;
+                if (x < io.npick * RF) sm[x] = t[j];
+            }
+        }
+        __syncthreads();
+        recs = sm;
+    }
     for (int idx = threadIdx.x; idx < G * D; idx += kThreads) {
         const int h = idx / D, e = idx - h * D;
-        const float l = s_rec[G + h];
-        io.out[((size_t)b * io.Hq + g * G + h) * D + e] = l > 0.f ? s_rec[2 * G + idx] / l : 0.f;
+        constexpr int RF = Rec<G, D>::kFloats;
+        float M = -INFINITY;
+        for (int c = 0; c < io.npick; ++c) M = fmaxf(M, recs[c * RF + h]);
+        float A = 0.f, Ls = 0.f;
+        for (int c = 0; c < io.npick; ++c) {
+            const float m = recs[c * RF + h];
+            const float f = (m == -INFINITY) ? 0.f : ex2(m - M);
+            A = fmaf(recs[c * RF + 2 * G + h * D + e], f, A);
+            Ls = fmaf(recs[c * RF + G + h], f, Ls);
+        }
+        io.out[((size_t)b * io.Hq + g * G + h) * D + e] = Ls > 0.f ? A / Ls : 0.f;
     }
+    if (io.npick > 1) reset_counter(io.cnt + u);
 }
 
 // ---- launchers ---------------------------------------------------------------------------
 
 template <typename T, int D>
 static cudaError_t prep_t(const Dims& d, const void* k, const void* v, const sa_clusters& cl, int C, cudaStream_t s) {
+    k_cluster_order<<<d.U(), kThreads, 0, s>>>(cl, d.L, d.ld, C);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
     const int gx = max(1, min(cdiv(d.L, kWarps), cdiv(4 * kSmTarget, d.U())));
     k_cluster_codes<T, D><<<dim3(gx, d.U()), kThreads, 0, s>>>(static_cast<const T*>(k), cl, d.L, d.ld);
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess || v == nullptr) return e;
     const size_t smem = (size_t)3 * C * D * sizeof(double);
     static std::atomic<unsigned long long> opted{0};
@@ -629,30 +754,46 @@ cudaError_t launch_cluster_prep(const Dims& d, const void* k, const void* v, con
     return d.d == 128 ? prep_t<float, 128>(d, k, v, cl, C, s) : prep_t<float, 64>(d, k, v, cl, C, s);
 }
 
-size_t multi_workspace(const Dims& d) {
-    return align256(sizeof(unsigned long long) * (size_t)d.U() * d.ld) + align256(sizeof(int) * (size_t)d.U() * d.ld);
+// workspace: tickets, query codes, offsets, keys, CTA records (largest G = 8)
+struct MultiPlan {
+    size_t off_cnt, off_q, off_off, off_keys, off_part, bytes;
+};
+
+static MultiPlan multi_plan(const Dims& d) {
+    MultiPlan p;
+    const size_t U = (size_t)d.U();
+    size_t o = 0;
+    p.off_cnt = o;  o = align256(o + 4 * U);
+    p.off_q = o;    o = align256(o + 4 * 16 * U);
+    p.off_off = o;  o = align256(o + 4 * (size_t)(kMaxClusters + 1) * U);
+    p.off_keys = o; o = align256(o + 4 * U * d.ld);
+    p.off_part = o; o = align256(o + 4 * U * kPickCtas * (size_t)(8 * (2 + d.d)));
+    p.bytes = o;
+    return p;
 }
+
+size_t multi_workspace(const Dims& d) { return multi_plan(d).bytes; }
 
 template <typename T, int D, int G>
 static cudaError_t multi_t(const Dims& d, const MultiIo& io, cudaStream_t s) {
-    const size_t hsm = (size_t)kMaxClusters * (kThreads > 256 ? kThreads : 256) * sizeof(unsigned);
-    static std::atomic<unsigned long long> opted{0};
-    cudaError_t e = opt_in_smem(k_multi_select<T, D, G>, hsm, opted);
+    k_multi_gate<T, D, G><<<d.U(), kThreads, 0, s>>>(io);
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    k_multi_select<T, D, G><<<d.U(), kThreads, hsm, s>>>(io);
-    e = cudaGetLastError();
+    constexpr size_t smem = PickSmem<G, D>::kBytes;
+    static std::atomic<unsigned long long> opted{0};
+    e = opt_in_smem(k_multi_pick<T, D, G>, smem, opted);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(d.U());
+    cfg.gridDim = dim3(io.npick, d.U());
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_multi_decode<T, D, G>, io);
+    return cudaLaunchKernelEx(&cfg, k_multi_pick<T, D, G>, io);
 }
 
 template <typename T, int D>
@@ -669,14 +810,18 @@ static cudaError_t multi_g(const Dims& d, const MultiIo& io, cudaStream_t s) {
 cudaError_t launch_multi_step(const Dims& d, const void* q, const void* k, const void* v, const sa_clusters& cl,
                               int budget, float scale, int32_t* read, int32_t* qcnt, float* out, char* ws,
                               cudaStream_t s) {
+    const MultiPlan p = multi_plan(d);
     MultiIo io;
     io.q = q; io.k = k; io.v = v; io.cl = cl;
     io.Hq = d.Hq; io.Hkv = d.Hkv; io.L = d.L; io.ld = d.ld; io.C = cl.n_clusters; io.budget = budget;
     io.scale = scale;
-    io.read = read; io.qcnt = qcnt;
-    io.keys = reinterpret_cast<unsigned long long*>(ws);
-    io.list = reinterpret_cast<int*>(ws + align256(sizeof(unsigned long long) * (size_t)d.U() * d.ld));
-    io.out = out;
+    io.read = read; io.qcnt = qcnt; io.out = out;
+    io.cnt = reinterpret_cast<unsigned*>(ws + p.off_cnt);
+    io.wq = reinterpret_cast<int*>(ws + p.off_q);
+    io.woff = reinterpret_cast<int*>(ws + p.off_off);
+    io.wkeys = reinterpret_cast<uint32_t*>(ws + p.off_keys);
+    io.part = reinterpret_cast<float*>(ws + p.off_part);
+    io.npick = cdiv(cl.n_clusters, kPickWarps);
     if (d.bf16) return d.d == 128 ? multi_g<__nv_bfloat16, 128>(d, io, s) : multi_g<__nv_bfloat16, 64>(d, io, s);
     return d.d == 128 ? multi_g<float, 128>(d, io, s) : multi_g<float, 64>(d, io, s);
 }

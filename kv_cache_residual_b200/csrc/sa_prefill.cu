@@ -7,6 +7,12 @@
 // (summed in fp64, rounded once to the cache dtype).
 //
 //   k_qmean : grid (nsq, B*Hq)   partial column sums of Q_ctx, last CTA -> mu_q
+//   bf16 caches: the tensor-core stream kernel in its prefill mode
+//             (k_stream_tc, sa_decode_core.cuh): mu_Q (split into bf16 hi +
+//             lo) as the prior columns of the same MMAs as the decode, over
+//             every token, with the block means, key / value totals and the
+//             largest |block mean| formed from the shared-memory tiles
+//   fp32 caches:
 //   k_kvpass: grid (nskv, B*Hkv) online softmax of s*mu_q.K_j over a token range
 //                                + sums + block means; last CTA -> o_est, log_z0,
 //                                mu_k, sum_k, sum_v, kbar_absmax
@@ -14,6 +20,8 @@
 #include "sa_cta.cuh"
 #include "sa_internal.h"
 #include "sa_sketch.cuh"
+
+#include <type_traits>
 
 namespace sa {
 
@@ -369,11 +377,16 @@ static cudaError_t prefill_t(const Dims& d, const PrefillPlan& p, const PrefillA
         a.st.mu_q);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    k_kvpass<T, D, G><<<dim3(p.nskv, d.U()), kThreads, 0, s>>>(
-        reinterpret_cast<const T*>(a.k), reinterpret_cast<const T*>(a.v), a.st.mu_q, d.Hq, d.Hkv, d.L, d.ld,
-        p.tok_kv, p.nskv, a.scale * kLog2e, p.kv_stride, reinterpret_cast<float*>(ws + p.off_kvpart),
-        reinterpret_cast<unsigned*>(ws + p.off_kvcnt), a.st);
-    e = cudaGetLastError();
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        // the tensor-core stream kernel: mu_Q as the prior columns of its MMAs
+        e = launch_prefill_stream(d, p, a.k, a.v, a.st, a.scale, ws + p.off_kvpart, ws + p.off_kvcnt, s);
+    } else {
+        k_kvpass<T, D, G><<<dim3(p.nskv, d.U()), kThreads, 0, s>>>(
+            reinterpret_cast<const T*>(a.k), reinterpret_cast<const T*>(a.v), a.st.mu_q, d.Hq, d.Hkv, d.L, d.ld,
+            p.tok_kv, p.nskv, a.scale * kLog2e, p.kv_stride, reinterpret_cast<float*>(ws + p.off_kvpart),
+            reinterpret_cast<unsigned*>(ws + p.off_kvcnt), a.st);
+        e = cudaGetLastError();
+    }
     if (e != cudaSuccess) return e;
     e = launch_block_sketch(d, a.st.blk_mean, a.st.mu_k, 0, d.L / 16, a.st.blk_code, a.st.blk_meta, s);
     if (e != cudaSuccess || a.st.blk_min == nullptr) return e;

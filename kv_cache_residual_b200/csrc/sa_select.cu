@@ -79,8 +79,7 @@ k_select_finish(SelectIo io) {
     __shared__ uint64_t s_bar[kSelStages];
     extern __shared__ __align__(128) unsigned char s_fin[];
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-    // the scan kernel's bounds are complete and visible after this
-    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    // (select_unit waits for the scan kernel once the query is coded)
     const int nk = io.sg.n_cand <= kFinishKeys ? io.sg.n_cand : 0;
     uint32_t* ukeys = reinterpret_cast<uint32_t*>(s_fin + kFinAlias);
     const SelectSmem sm{hist, sw, misc, s_qh, s_qi, s_qc, ukeys, ukeys + nk, s_sorted, s_fin, s_bar, nullptr, 0};

@@ -735,6 +735,9 @@ __device__ __forceinline__ SelectOutcome select_unit(const SelectIo& io, const S
         }
     }
     __syncthreads();
+    // the finish of split units coded the query while the scan ran; the
+    // scan's bounds are complete and visible after this
+    if constexpr (PHASE == kPhFinish) asm volatile("griddepcontrol.wait;\n" ::: "memory");
 
     bool failed = false;
     {

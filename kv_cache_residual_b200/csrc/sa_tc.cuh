@@ -93,14 +93,15 @@ struct WarpAttn {
     float o[NT][4];
     float m, l, m0, l0;
 
-    // q_row: pointer to the bf16 query of head g (only read when g < G);
+    // q_row: pointer to the bf16 query of head g (only read when g < G; null
+    // for none: zero logits);
     // mu_row: fp32 typical query of head g (PRIOR only)
     __device__ __forceinline__ void init(const __nv_bfloat16* q_row, const float* mu_row) {
         const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
             uint32_t a0 = 0, a2 = 0;
-            if (g < G) {
+            if (g < G && q_row != nullptr) {
                 a0 = *reinterpret_cast<const uint32_t*>(q_row + ks * 16 + 2 * t);
                 a2 = *reinterpret_cast<const uint32_t*>(q_row + ks * 16 + 8 + 2 * t);
             }
@@ -265,8 +266,8 @@ struct WarpAttnT {
     __device__ static __forceinline__ int row(int r0, int j) { return r0 + ((threadIdx.x & 31) >> 2) + 8 * j; }
 
     // init in two halves: load issues this lane's operand loads into raw
-    // (qg: the G bf16 query rows of the unit; mu: the G fp32 typical queries,
-    // PRIOR only), finish forms the B fragments and clears the state once
+    // (qg: the G bf16 query rows of the unit, null for none (zero logits);
+    // mu: the G fp32 typical queries, PRIOR only), finish forms the B fragments and clears the state once
     // they have landed, so other work can sit between the two.
     float2 raw[KS][2];
     __device__ __forceinline__ void load(const __nv_bfloat16* qg, const float* mu) {
@@ -277,8 +278,9 @@ struct WarpAttnT {
             for (int half = 0; half < 2; ++half) {
                 const int dim = ks * 16 + 2 * t + 8 * half;
                 float2 x = make_float2(0.f, 0.f);
-                if (g < G)
-                    x.x = __uint_as_float(*reinterpret_cast<const uint32_t*>(qg + (size_t)g * D + dim));
+                if (g < G) {
+                    if (qg != nullptr) x.x = __uint_as_float(*reinterpret_cast<const uint32_t*>(qg + (size_t)g * D + dim));
+                }
                 else if (PRIOR && g < 2 * G)
                     x = *reinterpret_cast<const float2*>(mu + (size_t)(g - G) * D + dim);
                 raw[ks][half] = x;

@@ -241,3 +241,29 @@ def test_per_head_flag_checks(lib):
     ph = sa.sa_select_params(64, 128, 8, 32, 0, 32, 0.05, 0.05, 0, 0, 0, 0, 1)
     assert lib.sa_workspace_size(ctypes.byref(sh), ctypes.byref(ph), sa.OP_DECODE) >= \
         lib.sa_workspace_size(ctypes.byref(sh), ctypes.byref(one), sa.OP_DECODE)
+
+
+def test_cluster_entry_checks(lib):
+    """sa_cluster_prep / sa_cluster_build / sa_multi_step reject a missing or
+    misaligned cluster array, a cluster count outside 1..64 and an empty
+    budget before launching anything; the multi-proxy workspace is
+    positive and a multiple of 256 bytes."""
+    sh = _shape()
+    p = ctypes.c_void_p(0x10000)
+    ok = sa.sa_clusters(64, *([0x10000] * 10))
+    assert lib.sa_multi_step(ctypes.byref(sh), p, p, p, ctypes.byref(ok), 0, 0.0, p, p, p, p, 1 << 30,
+                             None) == sa.SA_ERR_INVALID_ARG                    # budget < 1
+    for bad in (sa.sa_clusters(0, *([0x10000] * 10)), sa.sa_clusters(65, *([0x10000] * 10)),
+                sa.sa_clusters(64, *([0x10000] * 9 + [0])),                   # no start array
+                sa.sa_clusters(64, *([0x10000] * 8 + [0, 0x10000])),          # no order array
+                sa.sa_clusters(64, *([0x10008] + [0x10000] * 9))):            # misaligned basis
+        assert lib.sa_cluster_prep(ctypes.byref(sh), p, p, ctypes.byref(bad), None) == sa.SA_ERR_INVALID_ARG
+        assert lib.sa_cluster_build(ctypes.byref(sh), p, p, p, ctypes.byref(bad), 0, p, 1 << 30,
+                                    None) == sa.SA_ERR_INVALID_ARG
+        assert lib.sa_multi_step(ctypes.byref(sh), p, p, p, ctypes.byref(bad), 82, 0.0, p, p, p, p, 1 << 30,
+                                 None) == sa.SA_ERR_INVALID_ARG
+    none = sa.sa_select_params(0, 0, 0, 0, 0, 0, 0.0, 0.0, 0, 0)
+    w = lib.sa_workspace_size(ctypes.byref(sh), ctypes.byref(none), sa.OP_MULTI)
+    assert w > 0 and w % 256 == 0
+    assert lib.sa_multi_step(ctypes.byref(sh), p, p, p, ctypes.byref(ok), 82, 0.0, p, p, p, p, w - 1,
+                             None) == sa.SA_ERR_WORKSPACE

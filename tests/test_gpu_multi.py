@@ -29,12 +29,23 @@ def _oracle_clusters(data, b, g, G, C, exact_codes):
     return a, u32, code, sig, cs
 
 
+def _order(a, C):
+    """The cluster-major order of the positions (ascending within a cluster)
+    and the clusters' starts."""
+    order = np.argsort(a, kind="stable")
+    start = np.concatenate([[0], np.cumsum(np.bincount(a, minlength=C))])
+    return order, start
+
+
 def _to_gpu(cl, b, g, a, u32, code, sig, cs):
     dev = cl.basis.device
+    order, start = _order(a, cl.n_clusters)
     cl.basis[b, g] = torch.from_numpy(u32.T.copy()).float().to(dev)
     cl.assign[b, g, :len(a)] = torch.from_numpy(a.astype(np.uint8)).to(dev)
-    cl.codes[b, g, :len(a)] = torch.from_numpy(code.astype(np.int8)).to(dev)
-    cl.scales[b, g, :len(a)] = torch.from_numpy(sig).float().to(dev)
+    cl.order[b, g, :len(a)] = torch.from_numpy(order.astype(np.int32)).to(dev)
+    cl.start[b, g] = torch.from_numpy(start.astype(np.int32)).to(dev)
+    cl.codes[b, g, :len(a)] = torch.from_numpy(code[order].astype(np.int8)).to(dev)
+    cl.scales[b, g, :len(a)] = torch.from_numpy(sig[order]).float().to(dev)
     cl.count[b, g] = torch.from_numpy(cs["n"].astype(np.int32)).to(dev)
     for f in ("sum_k", "sum_v", "sum_k2"):
         getattr(cl, f)[b, g] = torch.from_numpy(cs[f]).float().to(dev)
@@ -88,8 +99,11 @@ def test_prep_codes_bit_exact_and_sums():
     sa.cluster_prep(data["k"], data["v"], got, w.Hq)
     torch.cuda.synchronize()
     for (b, g), (a, u32, code, sig, cs) in orc.items():
-        assert np.array_equal(got.codes[b, g].cpu().numpy().astype(np.int64), code)
-        assert np.array_equal(got.scales[b, g].cpu().numpy().astype(np.float64), sig)
+        order, start = _order(a, 16)
+        assert np.array_equal(got.order[b, g].cpu().numpy(), order)
+        assert np.array_equal(got.start[b, g].cpu().numpy(), start)
+        assert np.array_equal(got.codes[b, g].cpu().numpy().astype(np.int64), code[order])
+        assert np.array_equal(got.scales[b, g].cpu().numpy().astype(np.float64), sig[order])
         assert got.count[b, g].cpu().tolist() == cs["n"].tolist()
         for f in ("sum_k", "sum_v", "sum_k2"):
             np.testing.assert_allclose(f64(getattr(got, f)[b, g]), cs[f], rtol=1e-6, atol=1e-4)
@@ -102,7 +116,9 @@ def test_prep_codes_bit_exact_and_sums():
     sa.cluster_prep(dt["k"], dt["v"], gt, wt.Hq)
     torch.cuda.synchronize()
     a, u32, code, sig, cs = orct[(0, 0)]
-    assert np.array_equal(gt.codes[0, 0].cpu().numpy().astype(np.int64), code)
+    order, _ = _order(a, 8)
+    assert np.array_equal(gt.order[0, 0].cpu().numpy(), order)
+    assert np.array_equal(gt.codes[0, 0].cpu().numpy().astype(np.int64), code[order])
     assert gt.count[0, 0].cpu().tolist() == cs["n"].tolist()
 
 

@@ -114,5 +114,9 @@ def test_build_then_step_reads_the_budget():
         for g in range(w.Hkv):
             r = read[b, g].cpu().numpy()
             a = cl.assign[b, g].cpu().long().numpy()
+            # the cluster-major order: a stable sort of the positions by cluster
+            assert np.array_equal(cl.order[b, g].cpu().numpy(), np.argsort(a, kind="stable"))
+            assert np.array_equal(cl.start[b, g].cpu().numpy(),
+                                  np.concatenate([[0], np.cumsum(np.bincount(a, minlength=64))]))
             assert len(set(r.tolist())) == 82
             assert np.bincount(a[r], minlength=64).tolist() == qcnt[b, g].cpu().tolist()
