@@ -658,11 +658,12 @@ def main(argv=None):
         o_m, _, _ = sa.multi_step(Q[0], K, V, clusters, budget_m)
         o_d = sa.dense_decode(Q[0], K, V)
         err = ((o_m.double() - o_d.double()).norm() / o_d.double().norm()).item()
-        # per unit: codes (32 B), scale and cluster id per token; the basis and
-        # the clusters' count and key / squared-key / value sums; queries; the
-        # read rows; the read list and counts; the output
+        # per unit: codes (32 B), scale and position per token (cluster-major
+        # order); the basis, the clusters' starts, counts and key /
+        # squared-key / value sums; queries; the read rows; the read list and
+        # counts; the output
         C_ = 64
-        m_bytes = (w.L * (32 + 4 + 1) + 32 * w.d * 4 + C_ * (4 + 3 * w.d * 4) + w.G * w.d * esz
+        m_bytes = (w.L * (32 + 4 + 4) + 32 * w.d * 4 + C_ * (4 + 4 + 3 * w.d * 4) + 4 + w.G * w.d * esz
                    + budget_m * 2 * w.d * esz + budget_m * 4 + C_ * 4 + w.G * w.d * 4) * w.B * w.Hkv
         multi = {"tokens_per_s": ws * w.B / (m_ms * 1e-3), "ms_per_step": m_ms, "read_tokens": budget_m,
                  "clusters": C_, "bytes_per_step": m_bytes, "gbs": m_bytes / (m_ms * 1e-3) / 1e9,

@@ -16,6 +16,7 @@ namespace sa {
 constexpr int kSmTarget = 148 * 4;   // CTAs to aim for: 4 per SM on B200
 constexpr int kStreamSlots = 148 * 2; // resident CTAs of the bf16 stream kernel (2 per SM)
 constexpr int kSelectSlots = 148 * 2; // resident scanning CTAs of the selection (2 per SM): one wave
+constexpr int kMinChunkTiles = 8;     // fewest 64-token tiles per CTA when a decode unit is split
 
 struct Dims {
     int B, Hq, Hkv, G, d, L;
@@ -156,8 +157,11 @@ inline DecodePlan decode_plan(const Dims& d, const sa_select_params& sp, int mod
     p.n_tok_max = p.g.n_i + (draws && sp.sample_cap > 0 ? (sp.per_head ? d.G : 1) * sp.sample_cap : 0);
     const int nt = p.n_tok_max > 0 ? p.n_tok_max : 1;
     if (d.bf16) {                  // stream kernel: chunks of 64-token tiles, ~one wave
+        // at least kMinChunkTiles tiles per chunk: a unit split over several
+        // CTAs pays a record, a ticket and the last CTA's combine (~10 us on
+        // one sequence), more than a CTA spends on that many tiles
         const int ntiles = cdiv(nt, 64);
-        p.nsd = clampi(kStreamSlots / d.U(), 1, ntiles);
+        p.nsd = clampi(kStreamSlots / d.U(), 1, cdiv(ntiles, kMinChunkTiles));
         p.tok_d = cdiv(ntiles, p.nsd);          // tiles per chunk
         p.nsd = cdiv(ntiles, p.tok_d);
     } else {

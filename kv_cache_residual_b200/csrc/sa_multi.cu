@@ -81,6 +81,26 @@ __device__ __forceinline__ int dp4a_su(int a, unsigned b, int c) {
     return d;
 }
 
+// E consecutive elements (4, 8 or 16 bytes, aligned) as floats
+template <typename T, int E>
+__device__ __forceinline__ void ld_dims(const T* __restrict__ p, float (&x)[E]) {
+    constexpr int B = (int)sizeof(T) * E;
+    static_assert(B == 4 || B == 8 || B == 16, "4, 8 or 16 bytes");
+    if constexpr (B == 16) {
+        unpack<T>(__ldg(reinterpret_cast<const uint4*>(p)), x);
+    } else if constexpr (B == 8) {
+        const uint2 w = __ldg(reinterpret_cast<const uint2*>(p));
+        const T* t = reinterpret_cast<const T*>(&w);
+#pragma unroll
+        for (int e = 0; e < E; ++e) x[e] = to_f32<T>(t[e]);
+    } else {
+        const unsigned w = __ldg(reinterpret_cast<const unsigned*>(p));
+        const T* t = reinterpret_cast<const T*>(&w);
+#pragma unroll
+        for (int e = 0; e < E; ++e) x[e] = to_f32<T>(t[e]);
+    }
+}
+
 // ---- prefill: codes and cluster sums -----------------------------------------------
 
 // One CTA per unit: a stable counting sort of the positions by cluster.  The
@@ -246,6 +266,8 @@ k_multi_gate(MultiIo io) {
     __shared__ unsigned s_ql[kQgsRank / 4];
     __shared__ double s_mu[G][kMaxClusters], s_sg[G][kMaxClusters];
     __shared__ double s_err[kMaxClusters];
+    __shared__ double s_eh[G][kMaxClusters];               // per head shares of the errors
+    __shared__ int s_n[kMaxClusters];                      // cluster sizes
     __shared__ long long s_w[kMaxClusters];
     __shared__ int s_qc[kMaxClusters], s_off[kMaxClusters + 1], s_rem[kMaxClusters];
     // the pick kernel may start now: it waits for this grid before reading
@@ -257,6 +279,7 @@ k_multi_gate(MultiIo io) {
     const int C = io.C;
     const T* qg = static_cast<const T*>(io.q) + ((size_t)b * io.Hq + (size_t)g * G) * D;
     for (int i = threadIdx.x; i < G * D; i += NT) s_q[i / D][i % D] = to_f32<T>(qg[i]);
+    for (int c = threadIdx.x; c < C; c += NT) s_n[c] = __ldg(io.cl.count + (size_t)u * C + c);
     __syncthreads();
 
     // 1. the projected group query: thread (warp w, lane i) sums dims
@@ -364,35 +387,34 @@ k_multi_gate(MultiIo io) {
         }
     }
     __syncthreads();
-    if (warp == 0) {
-        // per head: the shift m and the estimated total mass (lanes over clusters)
-        double err[kMaxClusters / 32];
+    // per head (warp h): the shift m, the estimated total mass and each
+    // cluster's share of the weight error (lanes over clusters)
+    if (warp < G) {
+        const int h = warp;
+        double m = -INFINITY;
+        for (int c = lane; c < C; c += 32) m = fmax(m, s_mu[h][c] + s_sg[h][c] / 2);
 #pragma unroll
-        for (int x = 0; x < kMaxClusters / 32; ++x) err[x] = 0.0;
-        for (int h = 0; h < G; ++h) {
-            double m = -INFINITY;
-            for (int c = lane; c < C; c += 32) m = fmax(m, s_mu[h][c] + s_sg[h][c] / 2);
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
-            double mass = 0.0;
-            for (int c = lane; c < C; c += 32) {
-                const int n = __ldg(cnt + c);
-                if (n > 0) mass += (double)n * exp(s_mu[h][c] + s_sg[h][c] / 2 - m);
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) mass += __shfl_xor_sync(0xffffffffu, mass, off);
-#pragma unroll
-            for (int x = 0; x < kMaxClusters / 32; ++x) {
-                const int c = lane + 32 * x;
-                if (c < C) {
-                    const int n = __ldg(cnt + c);
-                    if (n > 0) err[x] += (double)n * exp(s_mu[h][c] - m) * expm1(s_sg[h][c] / 2) / mass;
-                }
-            }
+        for (int off = 16; off > 0; off >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
+        double mass = 0.0;
+        for (int c = lane; c < C; c += 32) {
+            const int n = s_n[c];
+            if (n > 0) mass += (double)n * exp(s_mu[h][c] + s_sg[h][c] / 2 - m);
         }
 #pragma unroll
-        for (int x = 0; x < kMaxClusters / 32; ++x)
-            if (lane + 32 * x < C) s_err[lane + 32 * x] = err[x];
+        for (int off = 16; off > 0; off >>= 1) mass += __shfl_xor_sync(0xffffffffu, mass, off);
+        for (int c = lane; c < C; c += 32) {
+            const int n = s_n[c];
+            s_eh[h][c] = n > 0 ? (double)n * exp(s_mu[h][c] - m) * expm1(s_sg[h][c] / 2) / mass : 0.0;
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // the cluster's error: the heads' shares summed in head order
+        for (int c = lane; c < C; c += 32) {
+            double e = 0.0;
+            for (int h = 0; h < G; ++h) e += s_eh[h][c];
+            s_err[c] = e;
+        }
         __syncwarp();
         // the clusters' weights as integers, their floors and remainders (the
         // lane of each cluster), then their order for the tokens left after
@@ -408,7 +430,7 @@ k_multi_gate(MultiIo io) {
             const int c = lane + 32 * x;
             wl[x] = (c < C && top > 0.0) ? (long long)rint(s_err[c] / top * 1073741824.0) : 0;
             W += wl[x];
-            total += c < C ? __ldg(cnt + c) : 0;
+            total += c < C ? s_n[c] : 0;
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -421,7 +443,7 @@ k_multi_gate(MultiIo io) {
         for (int x = 0; x < kMaxClusters / 32; ++x) {
             const int c = lane + 32 * x;
             if (c < C) {
-                const long long n = __ldg(cnt + c);
+                const long long n = s_n[c];
                 const long long qc = W > 0 ? min(n, E * wl[x] / W) : 0;
                 s_qc[c] = (int)qc;
                 s_w[c] = W > 0 ? (E * wl[x]) % W : 0;       // (the remainder)
@@ -452,7 +474,7 @@ k_multi_gate(MultiIo io) {
                 bool gave = false;
                 for (int r = 0; r < C && left > 0; ++r) {
                     const int c = s_rem[r];
-                    if (s_qc[c] < __ldg(cnt + c)) {
+                    if (s_qc[c] < s_n[c]) {
                         s_qc[c] += 1;
                         --left;
                         gave = true;
@@ -496,10 +518,9 @@ struct PickSmem {
 };
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, G >= 8 ? 2 : 3)
 k_multi_pick(MultiIo io) {
-    using Gm = Geom<T, D>;
-    constexpr int EPC = Gm::EPC, CPR = Gm::CPR, GPW = Gm::GPW;
+    constexpr int EPC = D / 32;           // dims per lane in the softmax (lanes over the head dim)
     extern __shared__ __align__(16) unsigned char smem[];
     uint32_t* s_keys = reinterpret_cast<uint32_t*>(smem);                       // [warps][kPickKeys]
     unsigned* s_hist = reinterpret_cast<unsigned*>(smem) + kPickWarps * kPickKeys;   // [warps][256]
@@ -508,23 +529,14 @@ k_multi_pick(MultiIo io) {
 
     const int u = blockIdx.y, b = u / io.Hkv, g = u - b * io.Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int li = lane % CPR, gsub = lane / CPR;
     const int C = io.C;
     const int c = blockIdx.x * kPickWarps + warp;
     const bool has = c < C;
     const float qscale = io.scale * kLog2e;
     const T* qg = static_cast<const T*>(io.q) + ((size_t)b * io.Hq + (size_t)g * G) * D;
-    const T* K = static_cast<const T*>(io.k) + (size_t)u * io.ld * D + li * EPC;
-    const T* V = static_cast<const T*>(io.v) + (size_t)u * io.ld * D + li * EPC;
-    // what does not depend on the gate: the query, the cluster's extent
-    float qv[G][EPC];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-        float f[EPC];
-        unpack<T>(ld_nc16(qg + (size_t)h * D + li * EPC), f);
-#pragma unroll
-        for (int e = 0; e < EPC; ++e) qv[h][e] = f[e] * qscale;
-    }
+    const T* K = static_cast<const T*>(io.k) + (size_t)u * io.ld * D + lane * EPC;
+    const T* V = static_cast<const T*>(io.v) + (size_t)u * io.ld * D + lane * EPC;
+    // what does not depend on the gate: the cluster's extent
     const int* st = io.cl.start + (size_t)u * (C + 1);
     const int n0 = has ? __ldg(st + c) : 0, n = has ? __ldg(st + c + 1) - n0 : 0;
     const int nc = has ? __ldg(io.cl.count + (size_t)u * C + c) : 0;
@@ -549,23 +561,36 @@ k_multi_pick(MultiIo io) {
         uint32_t* keys = n <= kPickKeys ? s_keys + warp * kPickKeys : io.wkeys + (size_t)u * io.ld + n0;
         const int8_t* codes = io.cl.codes + ((size_t)u * io.ld + n0) * kQgsRank;
         const float* sig = io.cl.scales + (size_t)u * io.ld + n0;
-        for (int i = lane; i < n; i += 32) {
+        constexpr int UN = 4;                        // tokens per lane in flight
+        for (int i0 = lane; i0 < n; i0 += 32 * UN) {
             // an exact integer dot with the 16-bit query code (high bytes
             // signed, low bytes unsigned) times the token's scale, rounded once
-            const int4* cr = reinterpret_cast<const int4*>(codes + (size_t)i * kQgsRank);
-            int hi = 0, lo = 0;
+            int4 cw[UN][kQgsRank / 16];
+            float sg[UN];
 #pragma unroll
-            for (int w4 = 0; w4 < kQgsRank / 16; ++w4) {
-                const int4 cw = __ldg(cr + w4);
-                const int wv[4] = {cw.x, cw.y, cw.z, cw.w};
+            for (int j = 0; j < UN; ++j) {
+                const int i = i0 + 32 * j;
+                const int4* cr = reinterpret_cast<const int4*>(codes + (size_t)i * kQgsRank);
 #pragma unroll
-                for (int y = 0; y < 4; ++y) {
-                    hi = __dp4a(wv[y], qh[w4 * 4 + y], hi);
-                    lo = dp4a_su(wv[y], ql[w4 * 4 + y], lo);
-                }
+                for (int w4 = 0; w4 < kQgsRank / 16; ++w4) cw[j][w4] = i < n ? __ldg(cr + w4) : make_int4(0, 0, 0, 0);
+                sg[j] = i < n ? __ldg(sig + i) : 0.f;
             }
-            const int dot = 256 * hi + lo;
-            keys[i] = fkey(__double2float_rn((double)__ldg(sig + i) * (double)dot));
+#pragma unroll
+            for (int j = 0; j < UN; ++j) {
+                const int i = i0 + 32 * j;
+                int hi = 0, lo = 0;
+#pragma unroll
+                for (int w4 = 0; w4 < kQgsRank / 16; ++w4) {
+                    const int wv[4] = {cw[j][w4].x, cw[j][w4].y, cw[j][w4].z, cw[j][w4].w};
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) {
+                        hi = __dp4a(wv[y], qh[w4 * 4 + y], hi);
+                        lo = dp4a_su(wv[y], ql[w4 * 4 + y], lo);
+                    }
+                }
+                const int dot = 256 * hi + lo;
+                if (i < n) keys[i] = fkey(__double2float_rn((double)sg[j] * (double)dot));
+            }
         }
         __syncwarp();
         // radix select of the qc-th largest key, 8 bits at a time
@@ -616,56 +641,81 @@ k_multi_pick(MultiIo io) {
         }
         // the keys above pre, and the first rem equal to it, in slot order
         int taken = 0, eqs = 0;
-        for (int i0 = 0; i0 < n; i0 += 32) {
-            const int i = i0 + lane;
-            const uint32_t key = i < n ? keys[i] : 0u;
-            const bool eq = i < n && key == pre;
-            const unsigned em = __ballot_sync(0xffffffffu, eq);
-            const bool take = (i < n && key > pre) || (eq && eqs + __popc(em & lt) < rem);
-            const unsigned tm = __ballot_sync(0xffffffffu, take);
-            if (take) rd[taken + __popc(tm & lt)] = __ldg(ord + i);
-            taken += __popc(tm);
-            eqs += __popc(em);
+        for (int i0 = 0; i0 < n; i0 += 32 * 4) {
+            int pos[4];                               // positions loaded ahead, all in flight
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i = i0 + 32 * j + lane;
+                pos[j] = i < n ? __ldg(ord + i) : -1;
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i = i0 + 32 * j + lane;
+                const uint32_t key = i < n ? keys[i] : 0u;
+                const bool eq = i < n && key == pre;
+                const unsigned em = __ballot_sync(0xffffffffu, eq);
+                const bool take = (i < n && key > pre) || (eq && eqs + __popc(em & lt) < rem);
+                const unsigned tm = __ballot_sync(0xffffffffu, take);
+                if (take) rd[taken + __popc(tm & lt)] = pos[j];
+                taken += __popc(tm);
+                eqs += __popc(em);
+            }
         }
     }
     __syncwarp();                       // the warp's read list is visible to the warp
 
-    // 4. exact rows of the cluster, then its proxy
+    // 4. exact rows of the cluster (two at a time, both rows' loads in
+    // flight), then its proxy; each lane holds EPC dims of every head
+    float qv[G][EPC];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        float f[EPC];
+        ld_dims<T, EPC>(qg + (size_t)h * D + lane * EPC, f);
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) qv[h][e] = f[e] * qscale;
+    }
     Online<G, EPC> os;
     os.init();
     const int q_eff = qc < n ? qc : n;
     float ks[EPC], vs[EPC];
 #pragma unroll
     for (int e = 0; e < EPC; ++e) { ks[e] = 0.f; vs[e] = 0.f; }
-    for (int rb = 0; rb < q_eff; rb += GPW) {              // warp-uniform
-        const int r = rb + gsub;
-        const bool ok = r < q_eff;
-        const int p = ok ? __ldcg(rd + r) : 0;
-        float kf[EPC], vf[EPC];
-        unpack<T>(ok ? ld_nc16(K + (size_t)p * D) : make_uint4(0, 0, 0, 0), kf);
-        unpack<T>(ok ? ld_nc16(V + (size_t)p * D) : make_uint4(0, 0, 0, 0), vf);
+    for (int r0 = 0; r0 < q_eff; r0 += 32) {
+        const int nr = min(32, q_eff - r0);
+        const int pl = lane < nr ? __ldcg(rd + r0 + lane) : 0;      // 32 positions at once
+        for (int j0 = 0; j0 < nr; j0 += 2) {                         // warp-uniform
+            float kf[2][EPC], vf[2][EPC];
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            float x = 0.f;
+            for (int j = 0; j < 2; ++j) {
+                const int p = __shfl_sync(0xffffffffu, pl, (j0 + j) & 31);
+                if (j0 + j < nr) {
+                    ld_dims<T, EPC>(K + (size_t)p * D, kf[j]);
+                    ld_dims<T, EPC>(V + (size_t)p * D, vf[j]);
+                } else {
 #pragma unroll
-            for (int e = 0; e < EPC; ++e) x = fmaf(qv[h][e], kf[e], x);
-            x = group_sum<CPR>(x);
-            if (ok) os.add(h, x, vf);
+                    for (int e = 0; e < EPC; ++e) { kf[j][e] = 0.f; vf[j][e] = 0.f; }
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                if (j0 + j < nr) {
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        float x = 0.f;
+#pragma unroll
+                        for (int e = 0; e < EPC; ++e) x = fmaf(qv[h][e], kf[j][e], x);
+                        os.add(h, group_sum<32>(x), vf[j]);
+                    }
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) { ks[e] += kf[j][e]; vs[e] += vf[j][e]; }
+                }
+            }
         }
-#pragma unroll
-        for (int e = 0; e < EPC; ++e) { ks[e] += kf[e]; vs[e] += vf[e]; }
     }
-#pragma unroll
-    for (int o = CPR; o < 32; o <<= 1)
-#pragma unroll
-        for (int e = 0; e < EPC; ++e) {
-            ks[e] += __shfl_xor_sync(0xffffffffu, ks[e], o);
-            vs[e] += __shfl_xor_sync(0xffffffffu, vs[e], o);
-        }
     const int n_un = nc - q_eff;
     if (has && n_un > 0) {
-        const float* sk = io.cl.sum_k + ((size_t)u * C + c) * D + li * EPC;
-        const float* sv = io.cl.sum_v + ((size_t)u * C + c) * D + li * EPC;
+        const float* sk = io.cl.sum_k + ((size_t)u * C + c) * D + lane * EPC;
+        const float* sv = io.cl.sum_v + ((size_t)u * C + c) * D + lane * EPC;
         const float inv = 1.f / (float)n_un;
         float kb[EPC], vb[EPC];
 #pragma unroll
@@ -679,14 +729,12 @@ k_multi_pick(MultiIo io) {
             float x = 0.f;
 #pragma unroll
             for (int e = 0; e < EPC; ++e) x = fmaf(qv[h][e], kb[e], x);
-            x = group_sum<CPR>(x) + lnn;
-            if (gsub == 0) os.add(h, x, vb);
+            os.add(h, group_sum<32>(x) + lnn, vb);
         }
     }
-    warp_merge<G, EPC, CPR>(os);
     __syncthreads();                    // the merge area aliases the keys and histograms
     float* rec = io.npick == 1 ? s_rec : io.part + ((size_t)u * kPickCtas + blockIdx.x) * Rec<G, D>::kFloats;
-    cta_merge_store<G, EPC, CPR, D>(os, sm, rec);
+    cta_merge_store<G, EPC, 32, D>(os, sm, rec);
     const float* recs = s_rec;
     if (io.npick > 1) {
         if (!last_cta_of_unit(io.cnt + u, (unsigned)io.npick)) return;
