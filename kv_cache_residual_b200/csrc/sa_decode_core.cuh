@@ -251,10 +251,11 @@ constexpr int kPrefillMode = 5;    // MODE value of the prefill pass (RESA prior
 
 // floats of a chunk record: exact (m, l, acc) and prior state per head, then
 // the key and value sums (proxy); the prefill pass keeps the key totals in
-// fp64 (2 d floats), the value totals and the largest |block mean| instead
+// fp64 (2 d floats) and the largest |block mean| instead (its value totals
+// are the exact columns' accumulator: a zero query weighs every token 1)
 template <int D, int G, int MODE>
 __host__ __device__ constexpr int stream_rec() {
-    return MODE == kPrefillMode ? ((2 * G * (2 + D) + 3 * D + 1 + 3) & ~3) : 2 * G * (2 + D) + 2 * D;
+    return MODE == kPrefillMode ? ((2 * G * (2 + D) + 2 * D + 1 + 3) & ~3) : 2 * G * (2 + D) + 2 * D;
 }
 
 template <int D>
@@ -527,12 +528,12 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
         wa.init(PREFILL ? nullptr : qg + (size_t)gh * D, PRIOR ? st.mu_q + (qh0 + gh) * D : nullptr);
     }
     float ks[2] = {0.f, 0.f};      // SUMS: this thread's column pair of K (c < D/2) or V (c >= D/2)
-    // PREFILL: thread t takes the column pair (2c, 2c+1), c = t mod (D/2), of
-    // BPT of the tile's four 16-row blocks (group t / (D/2)): fp64 key sums,
-    // fp32 value sums, the largest |block mean|
-    constexpr int kPairs = D / 2, kGrp = kTcThreads / kPairs, kBpt = 4 / kGrp;
-    double pk[2] = {0.0, 0.0};
-    float pv[2] = {0.f, 0.f}, amax = 0.f;
+    // PREFILL: thread t takes the four columns 4c .. 4c+3, c = t mod (D/4), of
+    // block t / (D/4) of every tile (threads past the tile's four blocks
+    // idle at D = 64): fp64 key sums, the largest |block mean|
+    constexpr int kQuads = D / 4, kGrp = kTcThreads / kQuads;
+    double pk[4] = {0.0, 0.0, 0.0, 0.0};
+    float amax = 0.f;
     for (int i = tile0; i < tile1; ++i) {
         // the tile range was sized by the draw capacity: once the list length
         // is known, the tiles past it hold only masked rows (the copies of
@@ -564,36 +565,31 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
         if constexpr (PREFILL) {
             // block means: the fp64 sum of 16 rows times 1/16 (exact), one
             // rounding to bf16 (L is a whole number of blocks)
-            const int c = threadIdx.x % kPairs, grp = threadIdx.x / kPairs;
+            const int c = threadIdx.x % kQuads, grp = threadIdx.x / kQuads;
+            const int rb = grp * 16;
+            if (grp < 4 && base + rb < L) {
+                const unsigned char* kp = sb + rb * P + c * 8;
+                double s4[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-            for (int bb = 0; bb < kBpt; ++bb) {
-                const int rb = (grp * kBpt + bb) * 16;
-                if (base + rb < L) {
-                    const unsigned char* kp = sb + rb * P + c * 4;
-                    double s0 = 0.0, s1 = 0.0;
-                    float w0 = 0.f, w1 = 0.f;
-#pragma unroll
-                    for (int r = 0; r < 16; ++r) {
-                        const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kp + r * P));
-                        const float2 vf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kp + TB + r * P));
-                        s0 += (double)kf.x;
-                        s1 += (double)kf.y;
-                        w0 += vf.x;
-                        w1 += vf.y;
-                    }
-                    __nv_bfloat162 mean;
-                    mean.x = round_from_f64<__nv_bfloat16>(s0 * 0.0625);
-                    mean.y = round_from_f64<__nv_bfloat16>(s1 * 0.0625);
-                    const size_t row = (size_t)u * (io.ld / 16) + (size_t)((base + rb) / 16);
-                    *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(st.blk_mean) + row * D + 2 * c) =
-                        mean;
-                    const float2 mf = __bfloat1622float2(mean);
-                    amax = fmaxf(amax, fmaxf(fabsf(mf.x), fabsf(mf.y)));
-                    pk[0] += s0;
-                    pk[1] += s1;
-                    pv[0] += w0;
-                    pv[1] += w1;
+                for (int r = 0; r < 16; ++r) {
+                    const uint2 w = *reinterpret_cast<const uint2*>(kp + r * P);
+                    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
+                    const float2 b2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
+                    s4[0] += (double)a.x;
+                    s4[1] += (double)a.y;
+                    s4[2] += (double)b2.x;
+                    s4[3] += (double)b2.y;
                 }
+                __nv_bfloat16 mean[4];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    mean[x] = round_from_f64<__nv_bfloat16>(s4[x] * 0.0625);
+                    amax = fmaxf(amax, fabsf(__bfloat162float(mean[x])));
+                    pk[x] += s4[x];
+                }
+                const size_t row = (size_t)u * (io.ld / 16) + (size_t)((base + rb) / 16);
+                *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(st.blk_mean) + row * D + 4 * c) =
+                    *reinterpret_cast<const uint2*>(mean);
             }
         }
         const int r0 = warp * 16;
@@ -705,14 +701,13 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
         // the chunk's totals (after the prior state): key sums in fp64, value
         // sums, the largest |block mean|; thread partials meet in the
         // list-cache area, which the prefill pass does not use
-        double* s_pk = reinterpret_cast<double*>(smem + (size_t)kStages * SB);     // [kGrp][D]
-        float* s_pv = reinterpret_cast<float*>(s_pk + kGrp * D);                  // [kGrp][D]
-        float* s_am = s_pv + kGrp * D;                                            // [warps]
-        const int c = threadIdx.x % kPairs, grp = threadIdx.x / kPairs;
-        s_pk[grp * D + 2 * c] = pk[0];
-        s_pk[grp * D + 2 * c + 1] = pk[1];
-        s_pv[grp * D + 2 * c] = pv[0];
-        s_pv[grp * D + 2 * c + 1] = pv[1];
+        double* s_pk = reinterpret_cast<double*>(smem + (size_t)kStages * SB);     // [4][D]
+        float* s_am = reinterpret_cast<float*>(s_pk + 4 * D);                     // [warps]
+        const int c = threadIdx.x % kQuads, grp = threadIdx.x / kQuads;
+        if (grp < 4) {
+#pragma unroll
+            for (int x = 0; x < 4; ++x) s_pk[grp * D + 4 * c + x] = pk[x];
+        }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         if (lane == 0) s_am[warp] = amax;
@@ -720,17 +715,15 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
         double* rk = reinterpret_cast<double*>(r + 2 * G * (2 + D));
         for (int e = threadIdx.x; e < D; e += kTcThreads) {
             double a = 0.0;
-            float b2 = 0.f;
 #pragma unroll
-            for (int x = 0; x < kGrp; ++x) { a += s_pk[x * D + e]; b2 += s_pv[x * D + e]; }
+            for (int x = 0; x < 4; ++x) a += s_pk[x * D + e];
             rk[e] = a;
-            r[2 * G * (2 + D) + 2 * D + e] = b2;
         }
         if (threadIdx.x == 0) {
             float a = 0.f;
 #pragma unroll
             for (int w = 0; w < kTcWarps; ++w) a = fmaxf(a, s_am[w]);
-            r[2 * G * (2 + D) + 3 * D] = a;
+            r[2 * G * (2 + D) + 2 * D] = a;
         }
     }
     if constexpr (SUMS) {
@@ -790,11 +783,18 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
         }
     }
     if constexpr (PREFILL) {
-        // O_Est and log Z of the typical queries (the prior state), the key
-        // and value totals in chunk order, the largest |block mean|
+        // O_Est and log Z of the typical queries (the prior state); the value
+        // totals (head 0's exact state: every token weighted 1, so its
+        // accumulator is the sum of the value rows); the key totals in chunk
+        // order; the largest |block mean|
         constexpr int OP = G * (2 + D), OS = 2 * G * (2 + D);
-        if (sh) combine_heads<G, D, true>(recs, nchunk, rs, OP, s_ml, s_ml + G);
-        else combine_heads<G, D, false>(recs, nchunk, rs, OP, s_ml, s_ml + G);
+        if (sh) {
+            combine_heads<G, D, true>(recs, nchunk, rs, OP, s_ml, s_ml + G);
+            combine_heads<G, D, true>(recs, nchunk, rs, 0, s_ml + 2 * G, s_ml + 3 * G);
+        } else {
+            combine_heads<G, D, false>(recs, nchunk, rs, OP, s_ml, s_ml + G);
+            combine_heads<G, D, false>(recs, nchunk, rs, 0, s_ml + 2 * G, s_ml + 3 * G);
+        }
         __syncthreads();
         for (int idx = threadIdx.x; idx < G * D; idx += kTcThreads) {
             const int h = idx / D, e = idx - h * D;
@@ -804,21 +804,21 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
             if (e == 0) st.log_z0[qh0 + h] = (s_ml[h] + log2f(s_ml[G + h])) * kLn2;
         }
         for (int e = threadIdx.x; e < D; e += kTcThreads) {
+            const float sv = sh ? combine_acc<G, D, true>(recs, nchunk, rs, 0, 0, e, s_ml[2 * G])
+                                : combine_acc<G, D, false>(recs, nchunk, rs, 0, 0, e, s_ml[2 * G]);
             double a = 0.0;
-            float b2 = 0.f;
             for (int c = 0; c < nchunk; ++c) {
                 const float* rc = recs + (size_t)c * rs;
                 a += sh ? reinterpret_cast<const double*>(rc + OS)[e] : __ldcg(reinterpret_cast<const double*>(rc + OS) + e);
-                b2 += sh ? rc[OS + 2 * D + e] : __ldcg(rc + OS + 2 * D + e);
             }
             st.sum_k[(size_t)u * D + e] = (float)a;
             st.mu_k[(size_t)u * D + e] = (float)(a / (double)L);
-            st.sum_v[(size_t)u * D + e] = b2;
+            st.sum_v[(size_t)u * D + e] = sv;
         }
         if (threadIdx.x == 0) {
             float a = 0.f;
             for (int c = 0; c < nchunk; ++c)
-                a = fmaxf(a, sh ? recs[(size_t)c * rs + OS + 3 * D] : __ldcg(recs + (size_t)c * rs + OS + 3 * D));
+                a = fmaxf(a, sh ? recs[(size_t)c * rs + OS + 2 * D] : __ldcg(recs + (size_t)c * rs + OS + 2 * D));
             st.kbar_absmax[u] = a;
         }
     } else if constexpr (DENSE) {
@@ -846,7 +846,7 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
 }
 
 template <int D, int G, int MODE>
-__global__ void __launch_bounds__(kTcThreads)
+__global__ void __launch_bounds__(kTcThreads, 2)
 k_stream_tc(StreamIo io) {
     constexpr int SB = StageLayout<D>::kBytes;
     extern __shared__ __align__(16) unsigned char smem[];

@@ -88,12 +88,12 @@ inline PrefillPlan prefill_plan(const Dims& d) {
     p.off_kvcnt = off; off = align256(off + sizeof(unsigned) * (size_t)d.U());
     p.off_qpart = off; off = align256(off + sizeof(float) * (size_t)BH * p.nsq * d.d);
     // bf16: the stream kernel's chunks (as the dense pass) and records of
-    // the exact and prior states, fp64 key sums, value sums, absmax
+    // the exact and prior states, fp64 key sums, absmax
     const int ntiles = cdiv(d.L, 64);
     p.nsp = clampi(kStreamSlots / d.U(), 1, ntiles);
     p.tpc = cdiv(ntiles, p.nsp);
     p.nsp = cdiv(ntiles, p.tpc);
-    p.rec_p = (2 * d.G * (2 + d.d) + 3 * d.d + 1 + 3) & ~3;
+    p.rec_p = (2 * d.G * (2 + d.d) + 2 * d.d + 1 + 3) & ~3;
     const size_t kv_floats = (size_t)d.U() * (size_t)(d.bf16 ? p.nsp * p.rec_p : p.nskv * p.kv_stride);
     p.off_kvpart = off; off = align256(off + sizeof(float) * kv_floats);
     p.bytes = off;

@@ -27,6 +27,8 @@ CASES = {
     "f32_d128_g1": synth.scaled(synth.WORKLOADS["llama"], B=2, Hq=2, Hkv=2, dtype="f32", L=2048, n_hh=8, seed=13),
     "bf16_d128_g2": synth.scaled(synth.WORKLOADS["llama"], B=3, Hq=6, Hkv=3, L=1536, n_hh=8, seed=14, sink=16,
                                  local=48),
+    # one query head per KV head; a last 64-token tile of 16 tokens
+    "bf16_d128_g1": synth.scaled(synth.WORKLOADS["llama"], B=2, Hq=2, Hkv=2, L=2064, n_hh=8, seed=15),
 }
 
 
