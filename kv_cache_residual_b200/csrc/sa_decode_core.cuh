@@ -245,7 +245,11 @@ __device__ __forceinline__ void decode_epilogue(const float* recs, int nsd, int 
 constexpr int kTcTile = 64;        // tokens per shared-memory tile
 constexpr int kTcWarps = 4;        // 16 tokens per warp per tile
 constexpr int kTcThreads = 32 * kTcWarps;
-constexpr int kStages = 3;
+// ring stages: three for the all-token passes (dense, prefill: bandwidth);
+// two for the decode, whose units hold a few tiles (one tile in flight
+// while the previous is computed; a shorter prologue at one sequence)
+template <int MODE>
+__host__ __device__ constexpr int stream_stages() { return MODE >= 4 ? 3 : 2; }
 constexpr int kDenseMode = 4;      // MODE value of the dense pass
 constexpr int kPrefillMode = 5;    // MODE value of the prefill pass (RESA prior, totals, block means)
 
@@ -272,7 +276,7 @@ constexpr int kSampCache = 256;
 template <int D, int G, int MODE>
 __host__ __device__ constexpr size_t stream_area_smem() {     // stages, then the merge / epilogue scratch over them
     constexpr bool PRIOR = (MODE == SA_RESA || MODE == kPrefillMode);
-    constexpr size_t ring = (size_t)kStages * StageLayout<D>::kBytes;
+    constexpr size_t ring = (size_t)stream_stages<MODE>() * StageLayout<D>::kBytes;
     constexpr size_t merge = (size_t)(kTcWarps * G * 4 + (PRIOR ? 2 : 1) * kTcWarps * G * D) * 4;
     constexpr size_t tail = (size_t)stream_rec<D, G, MODE>() * 4       // own record
                             + (size_t)(2 * G * D + 4 * G + 2 * D + G) * 4;  // epilogue scratch
@@ -282,7 +286,7 @@ __host__ __device__ constexpr size_t stream_area_smem() {     // stages, then th
 
 template <int D, int G, int MODE>
 __host__ __device__ constexpr size_t stream_smem() {          // the stream kernel: area + the two list caches after the stages
-    constexpr size_t lists = (size_t)kStages * StageLayout<D>::kBytes + (kBlkCache + kSampCache) * 4;
+    constexpr size_t lists = (size_t)stream_stages<MODE>() * StageLayout<D>::kBytes + (kBlkCache + kSampCache) * 4;
     constexpr size_t a = stream_area_smem<D, G, MODE>();
     return a > lists ? a : lists;
 }
@@ -345,6 +349,7 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
     constexpr int P = tc::Pitch<D>::kBytes;
     constexpr int TB = StageLayout<D>::kTileBytes;
     constexpr int SB = StageLayout<D>::kBytes;
+    constexpr int kStages = stream_stages<MODE>();
 
     const int b = u / Hkv, g = u - b * Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -515,12 +520,12 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
             bias_load<__nv_bfloat16, D, G, kTcWarps>(bpre, qg, st, u, b, g, Hq);
         }
     }
-    static_assert(kStages == 3, "the loop below keeps two tiles in flight");
-    put_pos(tile0);
-    put_pos(tile0 + 1);
+    // kStages - 1 tiles in flight ahead of the one being computed
+#pragma unroll
+    for (int j = 0; j < kStages - 1; ++j) put_pos(tile0 + j);
     __syncthreads();
-    copy_tile(tile0);
-    copy_tile(tile0 + 1);
+#pragma unroll
+    for (int j = 0; j < kStages - 1; ++j) copy_tile(tile0 + j);
     if constexpr (kTokRows) {
         wa.finish();
     } else {
@@ -539,12 +544,12 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
         // is known, the tiles past it hold only masked rows (the copies of
         // the next two are drained after the loop)
         if (sel_ready && i * kTcTile >= n_tok) break;     // uniform
-        // stage (i+2)%3 was last read by tile i-1, finished before the
-        // trailing barrier of the previous iteration
-        put_pos(i + 2);
-        tc::cp_wait<1>();           // this thread's copies of tile i have landed
-        __syncthreads();            // everyone's, and the positions of tile i+2
-        copy_tile(i + 2);
+        // stage (i + kStages - 1) % kStages was last read by tile i-1,
+        // finished before the trailing barrier of the previous iteration
+        put_pos(i + kStages - 1);
+        tc::cp_wait<kStages - 2>();   // this thread's copies of tile i have landed
+        __syncthreads();              // everyone's, and the positions of the next tile
+        copy_tile(i + kStages - 1);
         unsigned char* sb = smem + (size_t)(i % kStages) * SB;
         const int base = i * kTcTile;
         if constexpr (SUMS) {
@@ -850,7 +855,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 k_stream_tc(StreamIo io) {
     constexpr int SB = StageLayout<D>::kBytes;
     extern __shared__ __align__(16) unsigned char smem[];
-    int* s_blk = reinterpret_cast<int*>(smem + (size_t)kStages * SB);
+    int* s_blk = reinterpret_cast<int*>(smem + (size_t)stream_stages<MODE>() * SB);
     stream_unit<D, G, MODE>(io, smem, s_blk, s_blk + kBlkCache, blockIdx.y, blockIdx.x);
 }
 
