@@ -256,7 +256,7 @@ k_cluster_stats(const T* __restrict__ k, const T* __restrict__ v, sa_clusters cl
 // ---- per step: ErrorGate and the query code ----------------------------------------
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 k_multi_gate(MultiIo io) {
     constexpr int NT = kThreads, NW = kWarps;
     __shared__ float s_q[G][D];
@@ -593,72 +593,103 @@ k_multi_pick(MultiIo io) {
             }
         }
         __syncwarp();
-        // radix select of the qc-th largest key, 8 bits at a time
-        unsigned* hist = s_hist + warp * 256;
-        uint32_t pre = 0u, mask = 0u;
-        int rem = qc;
-        for (int shift = 24; shift >= 0; shift -= 8) {
-#pragma unroll
-            for (int y = 0; y < 8; ++y) hist[lane * 8 + y] = 0u;
-            __syncwarp();
-            for (int i0 = 0; i0 < n; i0 += 32) {
-                const int i = i0 + lane;
-                const uint32_t key = i < n ? keys[i] : 0u;
-                const unsigned bin = (i < n && (key & mask) == pre) ? ((key >> shift) & 0xFFu) : 256u;
-                const unsigned peers = __match_any_sync(0xffffffffu, bin);
-                if (bin < 256u && (peers & lt) == 0u) atomicAdd(&hist[bin], (unsigned)__popc(peers));
-            }
-            __syncwarp();
-            // lane l holds bins 255 - 8l - y; the digit where the count from the top reaches rem
-            unsigned cc[8], loc = 0;
-#pragma unroll
-            for (int y = 0; y < 8; ++y) { cc[y] = hist[255 - 8 * lane - y]; loc += cc[y]; }
-            unsigned inc = loc;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const unsigned t = __shfl_up_sync(0xffffffffu, inc, o);
-                if (lane >= o) inc += t;
-            }
-            unsigned ex = inc - loc;
-            int dig = -1, nrem = 0;
-            if (ex < (unsigned)rem && inc >= (unsigned)rem) {
-#pragma unroll
-                for (int y = 0; y < 8; ++y) {
-                    if (dig < 0 && ex + cc[y] >= (unsigned)rem) {
-                        dig = 255 - 8 * lane - y;
-                        nrem = rem - (int)ex;
-                    }
-                    if (dig < 0) ex += cc[y];
+        if (qc <= 32 && n <= kPickKeys) {
+            // small q: q rounds of a warp argmax over (key desc, member asc);
+            // lane l owns members l, l + 32, ... and keeps its best one not
+            // yet taken (a taken key is zeroed: a finite score's key is never
+            // 0); the round's winner rescans only its own members
+            auto best_of = [&]() -> unsigned long long {
+                unsigned long long b = 0ull;
+                for (int i = lane; i < n; i += 32) {
+                    const uint32_t key = keys[i];
+                    const unsigned long long c = ((unsigned long long)key << 32) | (uint32_t)(~(uint32_t)i);
+                    if (key != 0u && c > b) b = c;
                 }
+                return b;
+            };
+            unsigned long long mine = best_of();
+            int chosen = 0x7fffffff;                 // lane r: the r-th member taken
+            for (int r = 0; r < qc; ++r) {
+                const unsigned long long w = warp_max_u64(mine);
+                const int wi = (int)(~(uint32_t)w);
+                if (lane == r) chosen = wi;
+                if ((wi & 31) == lane) {
+                    keys[wi] = 0u;
+                    mine = best_of();
+                }
+                __syncwarp();
             }
-            const unsigned who = __ballot_sync(0xffffffffu, dig >= 0);
-            const int src = __ffs(who) - 1;
-            dig = __shfl_sync(0xffffffffu, dig, src);
-            rem = __shfl_sync(0xffffffffu, nrem, src);
-            pre |= (uint32_t)dig << shift;
-            mask |= 0xFFu << shift;
-            __syncwarp();
-        }
-        // the keys above pre, and the first rem equal to it, in slot order
-        int taken = 0, eqs = 0;
-        for (int i0 = 0; i0 < n; i0 += 32 * 4) {
-            int pos[4];                               // positions loaded ahead, all in flight
+            // members ascending = positions ascending (cluster-major order)
+            chosen = warp_sort_asc(chosen);
+            if (lane < qc) rd[lane] = __ldg(ord + chosen);
+        } else {
+            // radix select of the qc-th largest key, 8 bits at a time
+            unsigned* hist = s_hist + warp * 256;
+            uint32_t pre = 0u, mask = 0u;
+            int rem = qc;
+            for (int shift = 24; shift >= 0; shift -= 8) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int i = i0 + 32 * j + lane;
-                pos[j] = i < n ? __ldg(ord + i) : -1;
+                for (int y = 0; y < 8; ++y) hist[lane * 8 + y] = 0u;
+                __syncwarp();
+                for (int i0 = 0; i0 < n; i0 += 32) {
+                    const int i = i0 + lane;
+                    const uint32_t key = i < n ? keys[i] : 0u;
+                    const unsigned bin = (i < n && (key & mask) == pre) ? ((key >> shift) & 0xFFu) : 256u;
+                    const unsigned peers = __match_any_sync(0xffffffffu, bin);
+                    if (bin < 256u && (peers & lt) == 0u) atomicAdd(&hist[bin], (unsigned)__popc(peers));
+                }
+                __syncwarp();
+                // lane l holds bins 255 - 8l - y; the digit where the count from the top reaches rem
+                unsigned cc[8], loc = 0;
+#pragma unroll
+                for (int y = 0; y < 8; ++y) { cc[y] = hist[255 - 8 * lane - y]; loc += cc[y]; }
+                unsigned inc = loc;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const unsigned t = __shfl_up_sync(0xffffffffu, inc, o);
+                    if (lane >= o) inc += t;
+                }
+                unsigned ex = inc - loc;
+                int dig = -1, nrem = 0;
+                if (ex < (unsigned)rem && inc >= (unsigned)rem) {
+#pragma unroll
+                    for (int y = 0; y < 8; ++y) {
+                        if (dig < 0 && ex + cc[y] >= (unsigned)rem) {
+                            dig = 255 - 8 * lane - y;
+                            nrem = rem - (int)ex;
+                        }
+                        if (dig < 0) ex += cc[y];
+                    }
+                }
+                const unsigned who = __ballot_sync(0xffffffffu, dig >= 0);
+                const int src = __ffs(who) - 1;
+                dig = __shfl_sync(0xffffffffu, dig, src);
+                rem = __shfl_sync(0xffffffffu, nrem, src);
+                pre |= (uint32_t)dig << shift;
+                mask |= 0xFFu << shift;
+                __syncwarp();
             }
+            // the keys above pre, and the first rem equal to it, in slot order
+            int taken = 0, eqs = 0;
+            for (int i0 = 0; i0 < n; i0 += 32 * 4) {
+                int pos[4];                               // positions loaded ahead, all in flight
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int i = i0 + 32 * j + lane;
-                const uint32_t key = i < n ? keys[i] : 0u;
-                const bool eq = i < n && key == pre;
-                const unsigned em = __ballot_sync(0xffffffffu, eq);
-                const bool take = (i < n && key > pre) || (eq && eqs + __popc(em & lt) < rem);
-                const unsigned tm = __ballot_sync(0xffffffffu, take);
-                if (take) rd[taken + __popc(tm & lt)] = pos[j];
-                taken += __popc(tm);
-                eqs += __popc(em);
+                for (int j = 0; j < 4; ++j) {
+                    const int i = i0 + 32 * j + lane;
+                    pos[j] = i < n ? __ldg(ord + i) : -1;
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int i = i0 + 32 * j + lane;
+                    const uint32_t key = i < n ? keys[i] : 0u;
+                    const bool eq = i < n && key == pre;
+                    const unsigned em = __ballot_sync(0xffffffffu, eq);
+                    const bool take = (i < n && key > pre) || (eq && eqs + __popc(em & lt) < rem);
+                    const unsigned tm = __ballot_sync(0xffffffffu, take);
+                    if (take) rd[taken + __popc(tm & lt)] = pos[j];
+                    taken += __popc(tm);
+                    eqs += __popc(em);
+                }
             }
         }
     }
