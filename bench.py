@@ -92,7 +92,7 @@ def decode_bytes_per_unit(w, sg, esz, mode, b_draws):
     return byts
 
 
-def survey_bytes_per_unit(w, sg, esz, mode, b_draws):
+def scope_bytes_per_unit(w, sg, esz, mode, b_draws):
     """The method's bytes per unit and step as the scope table counts them:
     the block summaries of every candidate in the cache dtype, the group's
     queries, the exactly read K/V rows, the mode's statistics, the output
@@ -107,8 +107,8 @@ def survey_bytes_per_unit(w, sg, esz, mode, b_draws):
     return byts
 
 
-def survey_select_bytes_per_unit(w, sg, esz, b_draws):
-    """The selection's share of survey_bytes_per_unit: summaries, queries,
+def scope_select_bytes_per_unit(w, sg, esz, b_draws):
+    """The selection's share of scope_bytes_per_unit: summaries, queries,
     the chosen indices and the draws written."""
     return sg["n_cand"] * w.d * esz + w.G * w.d * esz + 4 * sg["kk"] + 4 * b_draws
 
@@ -514,8 +514,8 @@ def main(argv=None):
     step_gbs = (sel_b + dec_b) / (ms_per_step * 1e-3) / 1e9
     # the scope table's byte count (bf16 block summaries, not the int8 sketch
     # the selection actually streams)
-    sv_sel = survey_select_bytes_per_unit(w, sg, esz, b_mean) * w.B * w.Hkv
-    sv_step = survey_bytes_per_unit(w, sg, esz, args.mode, b_mean) * w.B * w.Hkv
+    sv_sel = scope_select_bytes_per_unit(w, sg, esz, b_mean) * w.B * w.Hkv
+    sv_step = scope_bytes_per_unit(w, sg, esz, args.mode, b_mean) * w.B * w.Hkv
     sv_sel_gbs = sv_sel / (sel_avg * 1e-3) / 1e9
     sv_step_gbs = sv_step / (ms_per_step * 1e-3) / 1e9
 
