@@ -35,13 +35,16 @@
 //      query code go to the workspace.
 // k_multi_pick (grid (C/8, U), a warp per cluster):
 //   3. QGS: each member's score fl32(sigma_j (qq . code_j)) (exact integer
-//      dot, dp4a) as an order-preserving 32-bit key; the q_c-th largest by a
-//      4-digit radix select over the cluster's keys (shared memory, or the
-//      workspace for clusters of more than kPickKeys members); the members
-//      above it and the first of those equal to it (ascending positions: the
-//      tie rule) are written to the read list in position order;
-//   4. the warp's read rows (lane groups over rows, fp32 online softmax per
-//      head) while summing their keys and values, then the cluster's proxy
+//      dot, dp4a) as an order-preserving 32-bit key; for q_c <= 32 (clusters
+//      of at most kPickKeys members) q_c rounds of a warp argmax over (key
+//      desc, member asc), else the q_c-th largest key by a 4-digit radix
+//      select over the cluster's keys (shared memory, or the workspace for
+//      larger clusters) and the members above it and the first of those
+//      equal to it; either way ascending members are ascending positions,
+//      which is the tie rule, and the taken positions are written to the
+//      read list in position order;
+//   4. the warp's read rows (lanes over the head dim, fp32 online softmax
+//      per head) while summing their keys and values, then the cluster's proxy
 //      for its n' = n_c - q_c unread members: key (sum_k - read keys) / n',
 //      value likewise, logit s q . key + ln n'.  Warps merge in order into a
 //      CTA record; the unit's last CTA (completion ticket) combines the
