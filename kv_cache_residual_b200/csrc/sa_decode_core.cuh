@@ -233,14 +233,16 @@ __device__ __forceinline__ void decode_epilogue(const float* recs, int nsd, int 
 }
 
 // ============================================================================
-// bf16 caches: one stream kernel for the sparse gather and the dense pass
+// bf16 caches: one stream kernel for the sparse gather, the dense pass and
+// the prefill's KV pass
 // ============================================================================
 // A CTA owns a chunk of consecutive 64-token tiles of one unit and streams
-// them through a 3-stage cp.async ring of padded shared tiles; its 4 warps
-// take 16 rows each per tile (tensor-core engine, sa_tc.cuh).  A unit that
-// fits one chunk (the usual case at batch 32: one CTA per unit, one wave)
-// finishes in the same CTA; otherwise the chunks' records are combined by
-// the unit's last CTA.
+// them through a cp.async ring of padded shared tiles (stream_stages: two
+// stages for the decode, three for the all-token passes); its 4 warps take
+// 16 rows each per tile (tensor-core engine, sa_tc.cuh).  A unit that fits
+// one chunk (the usual case at batch 32 and at one sequence with small
+// reads: one CTA per unit) finishes in the same CTA; otherwise the chunks'
+// records are combined by the unit's last CTA.
 
 constexpr int kTcTile = 64;        // tokens per shared-memory tile
 constexpr int kTcWarps = 4;        // 16 tokens per warp per tile
