@@ -632,10 +632,12 @@ def main(argv=None):
             s_ms = statistics.mean(p_[0] for p_ in pss)
             rows = 2 if score == "quest" else 1
             s_bytes = (rows * sg["n_cand"] * w.d * esz + w.G * w.d * esz + 4 * sg["kk"] + 4 * b_mean) * w.B * w.Hkv
+            sel_s = sa.select(Q[0], stats, sps_s[0], k=K, v=V)          # the band each unit rescored exactly
             selectors[score] = {"tokens_per_s": ws * w.B / (step_ms * 1e-3), "ms_per_step": step_ms,
                                 "select_us": 1e3 * s_ms, "select_bytes": s_bytes,
                                 "select_gbs": s_bytes / (s_ms * 1e-3) / 1e9,
-                                "select_frac": s_bytes / (s_ms * 1e-3) / 1e9 / peak}
+                                "select_frac": s_bytes / (s_ms * 1e-3) / 1e9 / peak,
+                                "rescored_mean": float(sel_s.n_rescored.float().mean())}
         stats.blk_min = stats.blk_max = None
 
     # the multi-proxy path (OpenAttention stages 02-04): ErrorGate split, the
