@@ -149,7 +149,9 @@ k_select_var(VarIo io) {
     for (int h = 0; h < G; ++h)
 #pragma unroll
         for (int e = 0; e < EPC; ++e) q[h][e] = s_qh[h * D + li * EPC + e];
-    constexpr int U4 = 4;                            // rows in flight per lane group
+    // rows in flight per lane group (measured: 16 single rows, 4 min / max
+    // pairs; more pairs spill)
+    constexpr int U4 = SCORE == SA_SCORE_QUEST ? 4 : 16;
     // the loop bound is the same for every lane of a warp (its GPW * U4 rows
     // start at rw), so the lane-group shuffles below always run on the full warp
     for (int rw = warp * GPW * U4; rw < n; rw += NW * GPW * U4) {
