@@ -271,8 +271,9 @@ struct StageLayout {
 };
 
 // The unit's chosen blocks and draws are cached in shared memory (after the
-// ring) when they fit; longer lists are read from global memory.
-constexpr int kBlkCache = 1024;
+// ring) when they fit; longer lists are read from global memory.  (Sized so
+// that a decode CTA fits on an SM beside two selection CTAs.)
+constexpr int kBlkCache = 256;
 constexpr int kSampCache = 256;
 
 template <int D, int G, int MODE>
@@ -288,7 +289,10 @@ __host__ __device__ constexpr size_t stream_area_smem() {     // stages, then th
 
 template <int D, int G, int MODE>
 __host__ __device__ constexpr size_t stream_smem() {          // the stream kernel: area + the two list caches after the stages
-    constexpr size_t lists = (size_t)stream_stages<MODE>() * StageLayout<D>::kBytes + (kBlkCache + kSampCache) * 4;
+    // after the stages: the list caches, or the prefill pass's key-sum scratch
+    constexpr size_t caches = (size_t)(kBlkCache + kSampCache) * 4;
+    constexpr size_t pf = MODE == kPrefillMode ? (size_t)4 * D * 8 + 64 : 0;
+    constexpr size_t lists = (size_t)stream_stages<MODE>() * StageLayout<D>::kBytes + (caches > pf ? caches : pf);
     constexpr size_t a = stream_area_smem<D, G, MODE>();
     return a > lists ? a : lists;
 }

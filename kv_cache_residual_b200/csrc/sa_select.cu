@@ -33,33 +33,49 @@ static unsigned* wait_counter() {
     return static_cast<unsigned*>(p);
 }
 
-constexpr int kSelStages = 4;      // 4 x 18 KB ring at d = 128: two CTAs per SM
+constexpr int kSelStages = 4;      // 4 x 18 KB ring at d = 128 (split units' scan, the finish)
+// One CTA per unit: a 3-stage ring, the candidates' keys sized to the unit
+// (dynamic) and at most 80 registers, so that two selection CTAs leave room
+// on an SM for a decode CTA (a programmatic dependent), which streams its
+// selection-independent rows meanwhile
+constexpr int kSelStagesAll = 3;
+
+template <int PHASE>
+__host__ __device__ constexpr int sel_stages() { return PHASE == kPhAll ? kSelStagesAll : kSelStages; }
+
+template <int D, int PHASE>
+__host__ __device__ constexpr size_t sel_ring_smem() {      // the ring and its barriers, 16-byte aligned
+    return (SketchRing<D, kWarps, sel_stages<PHASE>()>::kSmem + 15) & ~(size_t)15;
+}
 constexpr int kFinThreads = 512;
 constexpr int kFinishKeys = 16384; // keys of one unit in the finish kernel's shared memory
 constexpr int kFinCand = 1024;     // top-k candidates ranked in shared memory
 constexpr int kFinAlias = 32768;   // bytes for the top-k / band arrays (select_unit's ring aliases)
 
 template <typename T, int D, int G, int PHASE>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, PHASE == kPhAll ? 3 : 2)
 k_select(SelectIo io) {
-    using Ring = SketchRing<D, kWarps, kSelStages>;
+    using Ring = SketchRing<D, kWarps, sel_stages<PHASE>()>;
     __shared__ __align__(16) unsigned hist[256];
     __shared__ int sw[kWarps + 1];
     __shared__ int misc[3];
     __shared__ float s_qh[G * D];
     __shared__ __align__(16) int8_t s_qi[2 * D];
     __shared__ float s_qc[3];
-    __shared__ uint32_t s_ukeys[kSmemKeys];
-    __shared__ uint32_t s_lkeys[kSmemKeys];
     __shared__ int s_sorted[kWarpTopK];
     extern __shared__ __align__(128) unsigned char s_ring[];
+    // one CTA per unit: the upper and lower keys of its candidates after the
+    // ring (a split unit's scan keeps its bounds in the workspace)
+    const int kcap = PHASE == kPhAll ? (io.sg.n_cand + 3) & ~3 : 0;
+    uint32_t* s_ukeys = reinterpret_cast<uint32_t*>(s_ring + sel_ring_smem<D, PHASE>());
+    uint32_t* s_lkeys = s_ukeys + kcap;
     // a decode kernel launched as a programmatic dependent may start as soon as
     // every CTA of this grid has begun; it waits for this grid's completion
     // before reading the selection
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
     const SelectSmem sm{hist, sw, misc, s_qh, s_qi, s_qc, s_ukeys, s_lkeys, s_sorted, s_ring,
                         reinterpret_cast<uint64_t*>(s_ring + Ring::kRingBytes), nullptr, 0};
-    (void)select_unit<T, D, G, kThreads, kSelStages, PHASE>(io, sm, blockIdx.y, blockIdx.x);
+    (void)select_unit<T, D, G, kThreads, sel_stages<PHASE>(), PHASE>(io, sm, blockIdx.y, blockIdx.x);
 }
 
 // The finish of split units; dynamic shared memory: the alias area
@@ -118,14 +134,16 @@ SelectIo select_io(const Dims& d, const SelectPlan& p, const SelectArgs& a) {
 
 template <typename T, int D, int G>
 static cudaError_t select_t(const Dims& d, const SelectPlan& p, const SelectArgs& a, cudaStream_t s) {
-    constexpr size_t smem = SketchRing<D, kWarps, kSelStages>::kSmem;
+    constexpr size_t smem = sel_ring_smem<D, kPhScan>();
     const SelectIo io = select_io(d, p, a);
     if (io.timeouts == nullptr) return cudaErrorInvalidDevice;
     if (p.nss == 1 && p.g.n_cand <= kSmemKeys) {
         static std::atomic<unsigned long long> opted{0};
-        cudaError_t e = opt_in_smem(k_select<T, D, G, kPhAll>, smem, opted);
+        constexpr size_t all_max = sel_ring_smem<D, kPhAll>() + (size_t)2 * kSmemKeys * 4;
+        cudaError_t e = opt_in_smem(k_select<T, D, G, kPhAll>, all_max, opted);
         if (e != cudaSuccess) return e;
-        k_select<T, D, G, kPhAll><<<dim3(p.nss, d.U()), kThreads, smem, s>>>(io);
+        const size_t all = sel_ring_smem<D, kPhAll>() + (size_t)2 * ((p.g.n_cand + 3) & ~3) * 4;
+        k_select<T, D, G, kPhAll><<<dim3(p.nss, d.U()), kThreads, all, s>>>(io);
         return cudaGetLastError();
     }
     static std::atomic<unsigned long long> opted_scan{0}, opted_fin{0};
