@@ -542,7 +542,7 @@ __device__ __forceinline__ void stream_unit(const StreamIo& io, unsigned char* s
     // PREFILL: thread t takes the four columns 4c .. 4c+3, c = t mod (D/4), of
     // block t / (D/4) of every tile (threads past the tile's four blocks
     // idle at D = 64): fp64 key sums, the largest |block mean|
-    constexpr int kQuads = D / 4, kGrp = kTcThreads / kQuads;
+    constexpr int kQuads = D / 4;
     double pk[4] = {0.0, 0.0, 0.0, 0.0};
     float amax = 0.f;
     for (int i = tile0; i < tile1; ++i) {
